@@ -1,0 +1,329 @@
+"""Checks that tie the oracle to what the pages and mathematics fix.
+
+Each ``pin_*`` raises AssertionError on a mismatch.  They are run as plain
+tests (test_oracle_pins.py) and, with deliberate mistakes planted in the
+oracle, as mutation tests (test_oracle_mutations.py) to show each one bites.
+None of them re-types the oracle's own formula: each compares against a
+different formulation, a library routine, hand-derived fixtures, or brute
+force.
+"""
+from __future__ import annotations
+
+import itertools
+import math
+import os
+
+import numpy as np
+import torch
+import torch.nn.functional as F
+
+import oracle
+from synthetic import make_custom, quantize_affine
+from tests.helpers import bigint_words, dims_of, oracle_run
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------- formats
+def pin_e2m1_table():
+    """e2m1 values from the bit fields (sign | 2-bit exponent, bias 1 | 1-bit mantissa)."""
+    for code in range(16):
+        s, e, m = code >> 3, (code >> 1) & 3, code & 1
+        mag = (m * 0.5) if e == 0 else (2.0 ** (e - 1)) * (1.0 + m / 2.0)
+        want = -mag if s else mag
+        got = oracle.E2M1_VALUES[code]
+        assert got == want and np.signbit(got) == bool(s), (code, got, want)
+
+
+def pin_e8m0():
+    """e8m0 byte b -> 2^(b-127), against torch's float8_e8m0fnu widening."""
+    b = torch.arange(0, 255, dtype=torch.uint8)
+    lib = b.view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    got = oracle.e8m0_value(b.numpy())
+    assert np.array_equal(got, lib), np.nonzero(got != lib)
+
+
+def pin_unpack_golden():
+    with open(os.path.join(GOLDEN, "affine_bitstream.txt")) as fh:
+        n = 0
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            bits_s, codes_s, words_s = [p.strip() for p in line.split("|")]
+            bits = int(bits_s)
+            codes = [int(c) for c in codes_s.split(",")]
+            words = np.array([int(w, 16) for w in words_s.split(",")], dtype=np.uint32)
+            got = oracle.unpack_codes(words, bits, len(codes))
+            assert got.tolist() == codes, (bits, got.tolist(), codes)
+            n += 1
+    assert n >= 8
+
+
+def pin_unpack_bigint():
+    rng = np.random.default_rng(11)
+    for bits in (2, 3, 4, 8):
+        for n in (32, 64, 96, 128):
+            codes = rng.integers(0, 1 << bits, size=n)
+            words = bigint_words(codes, bits)
+            got = oracle.unpack_codes(words, bits, n)
+            assert np.array_equal(got, codes), (bits, n)
+    # several rows at once: rows are independent streams
+    codes = rng.integers(0, 8, size=(5, 64))
+    words = np.stack([bigint_words(r, 3) for r in codes])
+    assert np.array_equal(oracle.unpack_codes(words, 3, 64), codes)
+
+
+def pin_affine_dequant():
+    """Dequantised packs reproduce the weights they were made from.
+
+    The generator's min/max quantiser bounds the reconstruction error by half
+    a quantisation step (plus bf16 rounding of scale and bias); a wrong group
+    index, a transposed row or a dropped term breaks the bound by orders of
+    magnitude.  Special codes: q = 0 gives the bias exactly, q = 2^b-1 gives
+    scale*(2^b-1)+bias.
+    """
+    g = torch.Generator().manual_seed(5)
+    for bits, group in ((2, 64), (2, 128), (3, 64), (3, 128), (4, 64), (4, 128), (8, 64), (8, 128)):
+        w = torch.randn(24, 256, generator=g) * 0.02 + torch.randn(24, 1, generator=g) * 0.01
+        q, s, b = quantize_affine(w, bits, group)
+        s32, b32 = s.float().numpy(), b.float().numpy()
+        W = oracle.dequant_affine(q.numpy().view(np.uint32), s32, b32, bits, group, 256)
+        levels = (1 << bits) - 1
+        tol = (np.repeat(s32, group, -1) * (0.5 + levels / 256.0)
+               + np.repeat(np.abs(b32), group, -1) / 256.0 + 1e-12)
+        err = np.abs(W - w.double().numpy())
+        assert (err <= tol).all(), (bits, group, float((err / tol).max()))
+    rows, n_in, group = 3, 128, 64
+    for bits in (2, 3, 4, 8):
+        nw = n_in * bits // 32
+        s = np.array([[0.25, 0.5]] * rows)
+        b = np.array([[-1.0, 2.0]] * rows)
+        W0 = oracle.dequant_affine(np.zeros((rows, nw), np.uint32), s, b, bits, group, n_in)
+        assert np.array_equal(W0, np.repeat(b, group, -1))
+        W1 = oracle.dequant_affine(np.full((rows, nw), 0xFFFFFFFF, np.uint32), s, b, bits, group, n_in)
+        assert np.array_equal(W1, np.repeat(s * ((1 << bits) - 1) + b, group, -1))
+
+
+def pin_mxfp4_dequant():
+    """mxfp4 rows decode code-by-code; every value is exact in bf16."""
+    rng = np.random.default_rng(3)
+    codes = rng.integers(0, 16, size=(4, 64))
+    scales = rng.integers(117, 124, size=(4, 2)).astype(np.uint8)
+    words = np.stack([bigint_words(r, 4) for r in codes])
+    W = oracle.dequant_mxfp4(words, scales, 64)
+    for r in range(4):
+        for i in range(64):
+            c = int(codes[r, i])
+            s, e, m = c >> 3, (c >> 1) & 3, c & 1
+            mag = (m * 0.5) if e == 0 else 2.0 ** (e - 1) * (1 + m / 2)
+            want = (-mag if s else mag) * math.ldexp(1.0, int(scales[r, i // 32]) - 127)
+            assert W[r, i] == want, (r, i, W[r, i], want)
+    # lossless in bf16 (model card conversion notes): bf16 round-trip is exact
+    t = torch.from_numpy(W)
+    assert torch.equal(t.to(torch.bfloat16).double(), t)
+    # low nibble holds the even element: a byte 0x3F is codes (15, 3)
+    W2 = oracle.dequant_mxfp4(np.array([[0x0000003F, 0, 0, 0]], np.uint32), np.array([[127]], np.uint8), 32)
+    assert W2[0, 0] == -6.0 and W2[0, 1] == 1.5
+
+
+# ---------------------------------------------------------------- routing
+def pin_sqrtsoftplus():
+    with open(os.path.join(GOLDEN, "sqrtsoftplus.txt")) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            x, v, rt = (float(p) for p in line.split("|"))
+            got = float(oracle.sqrtsoftplus(np.array([x]))[0])
+            assert math.isfinite(got)
+            assert abs(got - v) <= rt * abs(v) + (0.0 if rt else 0.0), (x, got, v)
+    from scipy.special import softplus
+    x = np.linspace(-700, 700, 20001)
+    lib = np.sqrt(softplus(x))
+    got = oracle.sqrtsoftplus(x)
+    assert np.all(np.isfinite(got))
+    rel = np.abs(got - lib) / np.maximum(lib, 1e-300)
+    assert rel.max() < 1e-12, rel.max()
+    assert np.all(np.diff(got) > 0)                 # strictly increasing
+    big = np.array([1e4, 1e6, 1e8])
+    assert np.allclose(oracle.sqrtsoftplus(big), np.sqrt(big), rtol=1e-15)
+
+
+def _rank_count_topk(keys, k):
+    """Brute force: e is selected iff fewer than k experts beat it."""
+    T, E = keys.shape
+    ids = np.zeros((T, k), np.int64)
+    for t in range(T):
+        beats = []
+        for e in range(E):
+            n = sum(1 for j in range(E) if keys[t, j] > keys[t, e] or (keys[t, j] == keys[t, e] and j < e))
+            beats.append(n)
+        for e in range(E):
+            if beats[e] < k:
+                ids[t, beats[e]] = e
+    return ids
+
+
+def pin_topk_bruteforce():
+    rng = np.random.default_rng(7)
+    for E, k in ((8, 2), (16, 4), (12, 12), (9, 1)):
+        keys = rng.normal(size=(20, E))
+        keys[:5, : E // 2] = keys[:5, [0]]          # exact ties
+        keys[5:8] = 0.25                            # all equal
+        ids, gap = oracle.topk_select(keys, k)
+        want = _rank_count_topk(keys, k)
+        assert np.array_equal(ids, want), (E, k)
+        for t in range(keys.shape[0]):
+            srt = sorted(keys[t], reverse=True)
+            g = srt[k - 1] - srt[k] if k < E else np.inf
+            assert gap[t] == g
+    # subset brute force on a small case: the chosen set has the largest key sum
+    keys = rng.normal(size=(6, 8))
+    ids, _ = oracle.topk_select(keys, 3)
+    for t in range(6):
+        best = max(itertools.combinations(range(8), 3), key=lambda c: sum(keys[t, list(c)]))
+        assert set(ids[t].tolist()) == set(best)
+
+
+def pin_route_learned():
+    """With zero bias top-k of sqrtsoftplus equals top-k of the raw logits
+    (monotone score); weights are positive and sum to one; the bias only moves
+    the selection, never the weights."""
+    rng = np.random.default_rng(9)
+    x = rng.normal(size=(33, 64))
+    wr = rng.normal(scale=0.2, size=(16, 64))
+    ids, w, gap, L = oracle.route_learned(x, wr, np.zeros(16), 4)
+    ids_raw, _ = oracle.topk_select(x @ wr.T, 4)
+    assert np.array_equal(ids, ids_raw)
+    assert np.allclose(L, x @ wr.T, rtol=1e-13, atol=1e-13)
+    assert np.allclose(w.sum(1), 1.0, atol=1e-14) and (w > 0).all()
+    from scipy.special import softplus
+    s_lib = np.sqrt(softplus(x @ wr.T))
+    assert np.allclose(w, np.take_along_axis(s_lib, ids, 1) / np.take_along_axis(s_lib, ids, 1).sum(1, keepdims=True), rtol=1e-12)
+    # a huge bias on expert 3 forces it in; its weight still comes from the score
+    b = np.zeros(16)
+    b[3] = 1e3
+    ids_b, w_b, _, _ = oracle.route_learned(x, wr, b, 4)
+    assert (ids_b[:, 0] == 3).all()
+    sel = np.take_along_axis(s_lib, ids_b, 1)
+    assert np.allclose(w_b, sel / sel.sum(1, keepdims=True), rtol=1e-12)
+
+
+def pin_route_hash():
+    """ids are exactly the table rows of each token id, independent of the
+    token's position or batch; permuting tokens permutes ids and weights."""
+    rng = np.random.default_rng(13)
+    vocab, E, k, d = 50, 16, 4, 32
+    table = np.stack([rng.permutation(E)[:k] for _ in range(vocab)]).astype(np.int32)
+    tok = rng.integers(0, vocab, size=12)
+    x = rng.normal(size=(12, d))
+    wr = rng.normal(scale=0.3, size=(E, d))
+    ids, w = oracle.route_hash(x, wr, tok, table)
+    assert np.array_equal(ids, table[tok])
+    assert np.allclose(w.sum(1), 1.0, atol=1e-14)
+    perm = rng.permutation(12)
+    ids_p, w_p = oracle.route_hash(x[perm], wr, tok[perm], table)
+    assert np.array_equal(ids_p, ids[perm]) and np.allclose(w_p, w[perm], rtol=0, atol=0)
+    ids_u, w_u = oracle.route_hash(x, None, tok, table)
+    assert np.array_equal(ids_u, ids) and np.all(w_u == 1.0 / k)
+    # weights = renormalised scores of the table's experts, via a per-pair loop
+    from scipy.special import softplus
+    for t in range(12):
+        s = np.array([math.sqrt(softplus(float(x[t] @ wr[e]))) for e in table[tok[t]]])
+        assert np.allclose(w[t], s / s.sum(), rtol=1e-12)
+
+
+def pin_permutation():
+    rng = np.random.default_rng(17)
+    for T, k, E in ((1, 8, 256), (37, 4, 16), (64, 2, 8), (5, 3, 40)):
+        ids = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+        offs, rows, inv = oracle.permute(ids, E)
+        flat = ids.reshape(-1)
+        assert offs[0] == 0 and offs[-1] == T * k and np.all(np.diff(offs) >= 0)
+        assert sorted(rows.tolist()) == list(range(T * k))
+        assert np.array_equal(inv[rows], np.arange(T * k))
+        for e in range(E):
+            seg = rows[offs[e]:offs[e + 1]]
+            assert np.all(flat[seg] == e) and np.all(np.diff(seg) > 0)
+            assert len(seg) == int((flat == e).sum())
+        # brute force: walk experts in order, scan flat indices in order
+        want = [i for e in range(E) for i in range(T * k) if flat[i] == e]
+        assert rows.tolist() == want
+
+
+# ---------------------------------------------------------------- whole layer
+def _dense_reference(inp, res):
+    """Dense mixture: every token through every expert, masked by the gate.
+
+    Uses torch fp64 linear/silu (library routines) on the oracle-dequantised
+    weights, so it shares only the (separately pinned) decode with the oracle.
+    """
+    c = inp.cfg
+    T, E, d, f = c["T"], c["E"], c["d"], c["f"]
+    x = inp.x.double()
+    G = torch.zeros(T, E, dtype=torch.float64)
+    ids = torch.from_numpy(res["ids"])
+    G.scatter_add_(1, ids, torch.from_numpy(res["w"]))
+    out = torch.zeros(T, d, dtype=torch.float64)
+    for e in range(E):
+        W = {}
+        for name, m, n_in in (("w1", inp.w1, d), ("w3", inp.w3, d), ("w2", inp.w2, f)):
+            W[name] = torch.from_numpy(oracle.dequant(m.fmt, m.bits, m.group, n_in, *m.expert_numpy(e)))
+        h = F.silu(F.linear(x, W["w1"])) * F.linear(x, W["w3"])
+        out += G[:, e:e + 1] * F.linear(h, W["w2"])
+    if inp.shared is not None:
+        s1, s3, s2 = inp.shared
+        fs = c["f_shared"]
+        Ws = [torch.from_numpy(oracle.dequant(m.fmt, m.bits, m.group, n_in, *m.expert_numpy(0)))
+              for m, n_in in ((s1, d), (s3, d), (s2, fs))]
+        out += F.linear(F.silu(F.linear(x, Ws[0])) * F.linear(x, Ws[1]), Ws[2])
+    return out.numpy()
+
+
+def pin_dense_equivalence():
+    for name, over in (("tiny", {}),
+                       ("tiny", dict(w13=("affine", 3, 64), w2=("affine", 2, 64), seed=21)),
+                       ("tiny", dict(w13=("mxfp4", 4, 32), w2=("mxfp4", 4, 32), seed=22)),
+                       ("tiny", dict(shared=("affine", 8, 64), f_shared=64, seed=23)),
+                       ("tiny", dict(routing="hash", vocab=97, seed=24, T=9))):
+        from synthetic import CONFIGS
+        cfg = dict(CONFIGS[name])
+        cfg.update(over)
+        inp = make_custom(cfg)
+        res = oracle_run(inp)
+        dense = _dense_reference(inp, res)
+        rel = np.abs(res["out"] - dense).max() / np.abs(dense).max()
+        assert rel < 1e-12, (over, rel)
+
+
+def pin_single_expert_swiglu():
+    """E=1, k=1: the layer is one plain SwiGLU FFN with routing weight 1."""
+    cfg = dict(T=7, d=64, E=1, k=1, f=96, routing="learned", vocab=0,
+               w13=("affine", 4, 32), w2=("affine", 4, 32), shared=None, f_shared=0,
+               weight_std=0.05, bias_std=0.1, seed=31)
+    inp = make_custom(cfg)
+    res = oracle_run(inp)
+    assert np.all(res["ids"] == 0) and np.all(res["w"] == 1.0)
+    W = [torch.from_numpy(oracle.dequant("affine", 4, 32, n, *m.expert_numpy(0)))
+         for m, n in ((inp.w1, 64), (inp.w3, 64), (inp.w2, 96))]
+    xd = inp.x.double()
+    want = F.linear(F.silu(F.linear(xd, W[0])) * F.linear(xd, W[1]), W[2]).numpy()
+    assert np.allclose(res["out"], want, rtol=1e-12, atol=1e-14)
+
+
+def pin_round_bf16():
+    g = torch.Generator().manual_seed(3)
+    a = torch.randn(100000, generator=g) * torch.exp(torch.randn(100000, generator=g) * 5)
+    lib = a.to(torch.bfloat16).double().numpy()           # torch: fp32 -> bf16 RNE
+    got = oracle.round_bf16(a.double().numpy())
+    assert np.array_equal(got, lib)
+    # exact halfway cases: 1 + 2^-8 (tie, even is 1), 1 + 3*2^-8 (tie, even is 1+2^-6)
+    assert oracle.round_bf16(np.array([1 + 2 ** -8]))[0] == 1.0
+    assert oracle.round_bf16(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
+
+
+ALL_PINS = [pin_e2m1_table, pin_e8m0, pin_unpack_golden, pin_unpack_bigint, pin_affine_dequant,
+            pin_mxfp4_dequant, pin_sqrtsoftplus, pin_topk_bruteforce, pin_route_learned,
+            pin_route_hash, pin_permutation, pin_dense_equivalence, pin_single_expert_swiglu,
+            pin_round_bf16]

@@ -1,0 +1,82 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin fails.
+
+Each case monkeypatches one oracle function or table with a realistic bug --
+a flipped sign, an off-by-one exponent bias, the wrong bit order, a dropped
+term, a wrong tie-break -- and asserts that at least one pin raises.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle.moe_oracle as om
+from tests import pins
+
+
+def _msb_first_unpack(words, bits, n):
+    w = np.ascontiguousarray(np.asarray(words).astype("<u4"))
+    stream = np.unpackbits(w.view(np.uint8), axis=-1, bitorder="big")
+    stream = stream[..., : n * bits].reshape(*w.shape[:-1], n, bits).astype(np.int64)
+    return (stream * (1 << np.arange(bits))).sum(-1)
+
+
+def _no_bias_dequant(words, scales, biases, bits, group, n_in):
+    q = om.unpack_codes(words, bits, n_in).astype(np.float64)
+    return np.repeat(np.asarray(scales, np.float64), group, -1) * q
+
+
+def _naive_sqrtsoftplus(L):
+    with np.errstate(over="ignore"):
+        return np.sqrt(np.log(1.0 + np.exp(np.asarray(L, np.float64))))
+
+
+def _tie_high_topk(keys, k):
+    keys = np.asarray(keys, np.float64)
+    order = np.argsort(-keys[:, ::-1], axis=1, kind="stable")
+    order = keys.shape[1] - 1 - order
+    ids = order[:, :k]
+    srt = np.take_along_axis(keys, order, 1)
+    gap = srt[:, k - 1] - srt[:, k] if keys.shape[1] > k else np.full(keys.shape[0], np.inf)
+    return ids, gap
+
+
+def _bad_silu(a):
+    return a / (1.0 + np.exp(a))
+
+
+def _unweighted_combine(y, w, y_shared=None):
+    out = np.asarray(y, np.float64).sum(1)
+    return out if y_shared is None else out + y_shared
+
+
+def _bad_e2m1():
+    t = om.E2M1_VALUES.copy()
+    t[8:] = -t[8:]          # sign bit ignored
+    return t
+
+
+def _round_trunc(a):
+    m, e = np.frexp(np.asarray(a, np.float64))
+    return np.ldexp(np.trunc(m * 256) / 256, e)
+
+
+MUTATIONS = [
+    ("E2M1_VALUES", _bad_e2m1(), [pins.pin_e2m1_table, pins.pin_mxfp4_dequant]),
+    ("e8m0_value", lambda e: np.ldexp(1.0, np.asarray(e, np.int64) - 128), [pins.pin_e8m0, pins.pin_mxfp4_dequant]),
+    ("unpack_codes", _msb_first_unpack, [pins.pin_unpack_golden, pins.pin_unpack_bigint]),
+    ("dequant_affine", _no_bias_dequant, [pins.pin_affine_dequant]),
+    ("sqrtsoftplus", _naive_sqrtsoftplus, [pins.pin_sqrtsoftplus]),
+    ("sqrtsoftplus", lambda L: np.maximum(L, 0) + np.log1p(np.exp(-np.abs(L))), [pins.pin_sqrtsoftplus, pins.pin_route_learned]),
+    ("topk_select", _tie_high_topk, [pins.pin_topk_bruteforce]),
+    ("silu", _bad_silu, [pins.pin_single_expert_swiglu, pins.pin_dense_equivalence]),
+    ("combine", _unweighted_combine, [pins.pin_dense_equivalence]),
+    ("round_bf16", _round_trunc, [pins.pin_round_bf16]),
+]
+
+
+@pytest.mark.parametrize("name,bad,catchers", MUTATIONS, ids=[f"{m[0]}-{i}" for i, m in enumerate(MUTATIONS)])
+def test_planted_mistake_is_caught(monkeypatch, name, bad, catchers):
+    monkeypatch.setattr(om, name, bad)
+    monkeypatch.setattr(oracle, name, bad, raising=False)
+    for pin in catchers:
+        with pytest.raises(AssertionError):
+            pin()
