@@ -1,0 +1,27 @@
+"""B200-native routed low-bit MoE FFN layer.
+
+The compute lives in ``libmoe_lowbit.so`` (hand-written CUDA for sm_100a,
+C ABI in ``include/moe_lowbit.h``); this package is its thin Python binding.
+"""
+from ._lib import (  # noqa: F401
+    FMT_AFFINE,
+    FMT_MXFP4,
+    LIB_PATH,
+    Dims,
+    MoEError,
+    QMatC,
+    alloc_workspace,
+    combine,
+    expert_ffn,
+    forward,
+    forward_host,
+    load_library,
+    make_dims,
+    permute,
+    qmat,
+    read_device_error,
+    route,
+    status_string,
+    workspace_size,
+)
+from .layer import MoELayer  # noqa: F401

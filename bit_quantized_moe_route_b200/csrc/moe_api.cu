@@ -1,0 +1,544 @@
+// Host side of the C ABI declared in include/moe_lowbit.h: argument
+// validation, workspace carving and kernel launches.  Nothing here computes
+// any part of the layer; every step runs in the kernels included below.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/moe_lowbit.h"
+#include "common.cuh"
+#include "ffn_gemv.cuh"
+#include "permute.cuh"
+#include "route.cuh"
+
+using namespace moe;
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+moe_status_t fail(moe_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+moe_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define MOE_CHECK_LAUNCH(what)                        \
+  do {                                                \
+    cudaError_t _e = cudaGetLastError();              \
+    if (_e != cudaSuccess) return cuda_fail(_e, what); \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+  size_t hdr, logits, ids, wts, offsets, sorted, inv, active, h, y, xstage, tokstage, outstage, total;
+};
+
+int f_max_of(const moe_dims_t& d) { return std::max(d.d_ff, d.d_ff_shared); }
+int shared_rows(const moe_dims_t& d) { return d.d_ff_shared > 0 ? d.T : 0; }
+
+WsLayout layout_of(const moe_dims_t& d) {
+  WsLayout L{};
+  size_t o = 0;
+  const size_t T = d.T, k = d.top_k, E = d.n_experts, D = d.d_model;
+  const size_t P = T * k + shared_rows(d);
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  L.hdr = take(sizeof(WsHeader));
+  L.logits = take(d.hash_mode ? 0 : T * E * sizeof(float));
+  L.ids = take(T * k * sizeof(int));
+  L.wts = take(T * k * sizeof(float));
+  L.offsets = take((E + 1) * sizeof(int));
+  L.sorted = take(T * k * sizeof(int));
+  L.inv = take(T * k * sizeof(int));
+  L.active = take((E + 1) * sizeof(int));
+  L.h = take(P * (size_t)f_max_of(d) * sizeof(float));
+  L.y = take(P * D * sizeof(float));
+  L.xstage = take(T * D * 2);
+  L.tokstage = take(T * sizeof(int));
+  L.outstage = take(T * D * 2);
+  L.total = o;
+  return L;
+}
+
+template <typename T>
+T* ws_at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<char*>(ws) + off);
+}
+
+// The GEMV path gives each thread one 32-input chunk of a row: widths are
+// multiples of 32 up to 8192 (at most 256 chunks per row).
+bool width_ok(int n) { return n >= 32 && n <= 8192 && n % 32 == 0; }
+
+moe_status_t check_dims(const moe_dims_t* d) {
+  if (!d) return fail(MOE_ERR_INVALID_ARG, "dims is NULL");
+  if (d->T < 1) return fail(MOE_ERR_INVALID_ARG, "T=%d must be >= 1", d->T);
+  if (d->n_experts < 1 || d->n_experts > 1024)
+    return fail(d->n_experts < 1 ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED, "n_experts=%d outside [1,1024]",
+                d->n_experts);
+  if (d->top_k < 1 || d->top_k > d->n_experts || d->top_k > 32)
+    return fail(MOE_ERR_INVALID_ARG, "top_k=%d must be in [1, min(n_experts, 32)]", d->top_k);
+  if (!width_ok(d->d_model)) return fail(MOE_ERR_UNSUPPORTED, "d_model=%d not supported", d->d_model);
+  if (!width_ok(d->d_ff)) return fail(MOE_ERR_UNSUPPORTED, "d_ff=%d not supported", d->d_ff);
+  if (d->d_ff_shared < 0 || (d->d_ff_shared > 0 && !width_ok(d->d_ff_shared)))
+    return fail(MOE_ERR_UNSUPPORTED, "d_ff_shared=%d not supported", d->d_ff_shared);
+  if (d->hash_mode && d->vocab < 1) return fail(MOE_ERR_INVALID_ARG, "hash mode needs vocab >= 1");
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t check_dev_ptr(const void* p, const char* name) {
+  if (!p) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+  cudaPointerAttributes a;
+  cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MOE_ERR_INVALID_ARG, "%s: cannot query pointer (%s)", name, cudaGetErrorString(e));
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(MOE_ERR_INVALID_ARG, "%s is not device memory", name);
+  return MOE_OK;
+}
+
+moe_status_t check_qmat(const moe_qmat_t* m, int n_in, const char* name, QMatDev* out, int n_out) {
+  if (!m) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+  int code;
+  if (m->fmt == MOE_FMT_AFFINE) {
+    switch (m->bits) {
+      case 2: code = F_A2; break;
+      case 3: code = F_A3; break;
+      case 4: code = F_A4; break;
+      case 8: code = F_A8; break;
+      default: return fail(MOE_ERR_UNSUPPORTED, "%s: affine bits=%d not in {2,3,4,8}", name, m->bits);
+    }
+    if (m->group != 32 && m->group != 64 && m->group != 128)
+      return fail(MOE_ERR_UNSUPPORTED, "%s: group=%d not in {32,64,128}", name, m->group);
+    if (!m->biases) return fail(MOE_ERR_INVALID_ARG, "%s: affine biases is NULL", name);
+  } else if (m->fmt == MOE_FMT_MXFP4) {
+    if (m->bits != 4 || m->group != 32)
+      return fail(MOE_ERR_UNSUPPORTED, "%s: mxfp4 needs bits=4 group=32", name);
+    code = F_MX4;
+  } else {
+    return fail(MOE_ERR_UNSUPPORTED, "%s: unknown format %d", name, m->fmt);
+  }
+  if (n_in % m->group) return fail(MOE_ERR_INVALID_ARG, "%s: in=%d not a multiple of group", name, n_in);
+  if (!m->q || !m->scales) return fail(MOE_ERR_INVALID_ARG, "%s: q/scales NULL", name);
+  if (!aligned16(m->q) || !aligned16(m->scales) || (m->biases && !aligned16(m->biases)))
+    return fail(MOE_ERR_INVALID_ARG, "%s: q/scales/biases must be 16-byte aligned", name);
+  moe_status_t st = check_dev_ptr(m->q, name);
+  if (st != MOE_OK) return st;
+  out->q = m->q;
+  out->scales = m->scales;
+  out->biases = m->biases;
+  out->fmt = code;
+  out->group = m->group;
+  out->n_in = n_in;
+  out->n_out = n_out;
+  out->wpr = n_in * m->bits / 32;
+  out->gpr = n_in / m->group;
+  return MOE_OK;
+}
+
+struct DevInfo {
+  int sms = 0;
+  int ffn1_blocks = 0, ffn2_blocks = 0;
+};
+DevInfo g_dev[64];
+std::atomic<int> g_dev_ready[64];
+
+moe_status_t dev_info(DevInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+  DevInfo& di = g_dev[dev];
+  if (g_dev_ready[dev].load(std::memory_order_acquire) != 2) {
+    int expect = 0;
+    if (g_dev_ready[dev].compare_exchange_strong(expect, 1)) {
+      cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
+      cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 34 * 1024 * 4);
+      cudaFuncSetAttribute(router_logits_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           8 * 8192 * 2);
+      int b1 = 0, b2 = 0;
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, ffn_gemv_kernel<1, 4>, kFfnThreads, 0);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, ffn_gemv_kernel<2, 8>, kFfnThreads, 0);
+      di.ffn1_blocks = std::max(1, b1);
+      di.ffn2_blocks = std::max(1, b2);
+      cudaError_t le = cudaGetLastError();
+      if (le != cudaSuccess) {
+        g_dev_ready[dev].store(0);
+        return cuda_fail(le, "device setup");
+      }
+      g_dev_ready[dev].store(2, std::memory_order_release);
+    } else {
+      while (g_dev_ready[dev].load(std::memory_order_acquire) == 1) {
+      }
+      if (g_dev_ready[dev].load(std::memory_order_acquire) != 2)
+        return fail(MOE_ERR_CUDA, "device setup failed in another thread");
+    }
+  }
+  *out = &di;
+  return MOE_OK;
+}
+
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- launches
+moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, const float* rb,
+                          const int* tok, const int* table, int* ids, float* wts, void* ws,
+                          const WsLayout& L, cudaStream_t s) {
+  int* err = &ws_at<WsHeader>(ws, L.hdr)->err;
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  if (d.hash_mode) {
+    const int blocks = ceil_div(d.T * 32, 256);
+    if (d.top_k <= 8)
+      route_hash_kernel<8><<<blocks, 256, 0, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts, d.top_k,
+                                                  d.vocab, ids, wts, err);
+    else
+      route_hash_kernel<32><<<blocks, 256, 0, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts, d.top_k,
+                                                   d.vocab, ids, wts, err);
+    MOE_CHECK_LAUNCH("route_hash_kernel");
+    return MOE_OK;
+  }
+  float* logits = ws_at<float>(ws, L.logits);
+  if (d.T <= 64) {
+    dim3 grid(ceil_div(d.n_experts, kLogitWarps), ceil_div(d.T, 8));
+    router_logits_small_kernel<8><<<grid, kLogitWarps * 32, 8 * d.d_model * 2, s>>>(xb, rw, logits, d.T,
+                                                                                      d.d_model, d.n_experts);
+    MOE_CHECK_LAUNCH("router_logits_small_kernel");
+  } else {
+    dim3 grid(ceil_div(d.n_experts, kLBN), ceil_div(d.T, kLBM));
+    router_logits_tiled_kernel<<<grid, 256, 0, s>>>(xb, rw, logits, d.T, d.d_model, d.n_experts);
+    MOE_CHECK_LAUNCH("router_logits_tiled_kernel");
+  }
+  const int blocks = ceil_div(d.T * 32, 256);
+  if (d.n_experts <= 32)
+    topk_kernel<1><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts);
+  else if (d.n_experts <= 256)
+    topk_kernel<8><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts);
+  else
+    topk_kernel<32><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts);
+  MOE_CHECK_LAUNCH("topk_kernel");
+  return MOE_OK;
+}
+
+moe_status_t launch_permute(const moe_dims_t& d, const int* ids, int* offsets, int* sorted, int* inv,
+                            void* ws, const WsLayout& L, cudaStream_t s) {
+  int* err = &ws_at<WsHeader>(ws, L.hdr)->err;
+  int* active = ws_at<int>(ws, L.active);
+  const size_t smem = (size_t)(2 + 32) * d.n_experts * sizeof(int);
+  permute_kernel<<<1, kPermThreads, smem, s>>>(ids, d.T * d.top_k, d.n_experts, offsets, sorted, inv, active,
+                                               err);
+  MOE_CHECK_LAUNCH("permute_kernel");
+  return MOE_OK;
+}
+
+// Stage 1 + stage 2 of the expert FFN (routed pairs, optional shared expert).
+moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, const int* sorted,
+                        const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh,
+                        float* y, int ld_y, void* ws, const WsLayout& L, cudaStream_t s) {
+  DevInfo* di = nullptr;
+  moe_status_t st = dev_info(&di);
+  if (st != MOE_OK) return st;
+  const int Tk = d.T * d.top_k;
+  const int max_active = std::min(d.n_experts, Tk);
+  float* h = ws_at<float>(ws, L.h);
+  const int ld_h = f_max_of(d);
+  FfnParams p{};
+  p.x = reinterpret_cast<const __nv_bfloat16*>(x);
+  p.T = d.T;
+  p.k = d.top_k;
+  p.offsets = offsets;
+  p.sorted_rows = sorted;
+  p.active = ws_at<int>(ws, L.active);
+  p.err = &ws_at<WsHeader>(ws, L.hdr)->err;
+  p.shared_pos0 = Tk;
+  p.has_shared = sh != nullptr;
+  // stage 1: h = silu(W1 x) * (W3 x)
+  {
+    FfnParams q = p;
+    q.out = h;
+    q.ld_out = ld_h;
+    q.ra = w1;
+    q.rb = w3;
+    const int rb_r = (kFfnThreads / (d.d_model / 32)) * 4;
+    q.routed_items_per_expert = ceil_div(d.d_ff, rb_r);
+    if (sh) {
+      q.sa = sh[0];
+      q.sb = sh[1];
+      q.shared_items = ceil_div(d.d_ff_shared, rb_r);
+    }
+    const int items = max_active * q.routed_items_per_expert + (sh ? q.shared_items : 0);
+    const int grid = std::max(1, std::min(items, di->sms * di->ffn1_blocks));
+    ffn_gemv_kernel<1, 4><<<grid, kFfnThreads, 0, s>>>(q);
+    MOE_CHECK_LAUNCH("ffn_gemv_kernel<1>");
+  }
+  // stage 2: y = W2 h
+  {
+    FfnParams q = p;
+    q.hin = h;
+    q.ld_in = ld_h;
+    q.out = y;
+    q.ld_out = ld_y;
+    q.ra = w2;
+    q.routed_items_per_expert = ceil_div(d.d_model, (kFfnThreads / (d.d_ff / 32)) * 8);
+    if (sh) {
+      q.sa = sh[2];
+      q.shared_items = ceil_div(d.d_model, (kFfnThreads / (d.d_ff_shared / 32)) * 8);
+    }
+    const int items = max_active * q.routed_items_per_expert + (sh ? q.shared_items : 0);
+    const int grid = std::max(1, std::min(items, di->sms * di->ffn2_blocks));
+    ffn_gemv_kernel<2, 8><<<grid, kFfnThreads, 0, s>>>(q);
+    MOE_CHECK_LAUNCH("ffn_gemv_kernel<2>");
+  }
+  return MOE_OK;
+}
+
+moe_status_t launch_combine(const moe_dims_t& d, const float* y, const int* inv, const float* w,
+                            const float* y_shared, void* out, cudaStream_t s) {
+  dim3 grid(ceil_div(d.d_model / 4, 256), d.T);
+  combine_kernel<<<grid, 256, 0, s>>>(y, inv, w, y_shared, reinterpret_cast<__nv_bfloat16*>(out), d.T,
+                                      d.top_k, d.d_model);
+  MOE_CHECK_LAUNCH("combine_kernel");
+  return MOE_OK;
+}
+
+moe_status_t check_ws(const moe_dims_t& d, void* ws, size_t ws_bytes, WsLayout* L) {
+  *L = layout_of(d);
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign) return fail(MOE_ERR_INVALID_ARG, "workspace not 256-byte aligned");
+  if (ws_bytes < L->total)
+    return fail(MOE_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, L->total);
+  return check_dev_ptr(ws, "workspace");
+}
+
+moe_status_t check_route_args(const moe_dims_t& d, const void* x, const float* rw, const int* tok,
+                              const int* table) {
+  moe_status_t st = check_dev_ptr(x, "x");
+  if (st != MOE_OK) return st;
+  if (!aligned16(x)) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  if (d.hash_mode) {
+    if ((st = check_dev_ptr(tok, "token_ids")) != MOE_OK) return st;
+    if ((st = check_dev_ptr(table, "tid2eid")) != MOE_OK) return st;
+    if (rw && !aligned16(rw)) return fail(MOE_ERR_INVALID_ARG, "router_w must be 16-byte aligned");
+  } else {
+    if ((st = check_dev_ptr(rw, "router_w")) != MOE_OK) return st;
+    if (!aligned16(rw)) return fail(MOE_ERR_INVALID_ARG, "router_w must be 16-byte aligned");
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+
+// ======================================================================= ABI
+extern "C" {
+
+size_t moe_workspace_size(const moe_dims_t* dims) {
+  if (check_dims(dims) != MOE_OK) return 0;
+  return layout_of(*dims).total;
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_INPUT: return "out-of-range routing input on device";
+  }
+  return "unknown status";
+}
+
+const char* moe_last_error_detail(void) { return g_detail; }
+
+moe_status_t moe_route(const moe_dims_t* dims, const void* x, const float* router_w, const float* router_b,
+                       const int32_t* token_ids, const int32_t* tid2eid, int32_t* topk_ids, float* topk_w,
+                       void* ws, size_t ws_bytes, void* stream) {
+  g_detail[0] = 0;
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t& d = *dims;
+  WsLayout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = check_route_args(d, x, router_w, token_ids, tid2eid)) != MOE_OK) return st;
+  if ((st = check_dev_ptr(topk_ids, "topk_ids")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(topk_w, "topk_w")) != MOE_OK) return st;
+  DevInfo* di;
+  if ((st = dev_info(&di)) != MOE_OK) return st;
+  return launch_route(d, x, router_w, router_b, token_ids, tid2eid, topk_ids, topk_w, ws, L,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_permute(const moe_dims_t* dims, const int32_t* topk_ids, int32_t* expert_offsets,
+                         int32_t* sorted_rows, int32_t* inv, void* ws, size_t ws_bytes, void* stream) {
+  g_detail[0] = 0;
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  WsLayout L;
+  if ((st = check_ws(*dims, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = check_dev_ptr(topk_ids, "topk_ids")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(expert_offsets, "expert_offsets")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(sorted_rows, "sorted_rows")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(inv, "inv")) != MOE_OK) return st;
+  DevInfo* di;
+  if ((st = dev_info(&di)) != MOE_OK) return st;
+  return launch_permute(*dims, topk_ids, expert_offsets, sorted_rows, inv, ws, L,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_expert_ffn(const moe_dims_t* dims, const void* x, const int32_t* expert_offsets,
+                            const int32_t* sorted_rows, const moe_qmat_t* w1, const moe_qmat_t* w3,
+                            const moe_qmat_t* w2, float* y, void* ws, size_t ws_bytes, void* stream) {
+  g_detail[0] = 0;
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t& d = *dims;
+  WsLayout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = check_dev_ptr(x, "x")) != MOE_OK) return st;
+  if (!aligned16(x)) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  if ((st = check_dev_ptr(expert_offsets, "expert_offsets")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(sorted_rows, "sorted_rows")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(y, "y")) != MOE_OK) return st;
+  if (!aligned16(y)) return fail(MOE_ERR_INVALID_ARG, "y must be 16-byte aligned");
+  QMatDev q1, q3, q2;
+  if ((st = check_qmat(w1, d.d_model, "w1", &q1, d.d_ff)) != MOE_OK) return st;
+  if ((st = check_qmat(w3, d.d_model, "w3", &q3, d.d_ff)) != MOE_OK) return st;
+  if ((st = check_qmat(w2, d.d_ff, "w2", &q2, d.d_model)) != MOE_OK) return st;
+  if (q1.fmt != q3.fmt || q1.group != q3.group)
+    return fail(MOE_ERR_UNSUPPORTED, "w1 and w3 must share one format");
+  DevInfo* di;
+  if ((st = dev_info(&di)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  active_from_offsets_kernel<<<1, kPermThreads, 0, s>>>(expert_offsets, d.n_experts, ws_at<int>(ws, L.active));
+  MOE_CHECK_LAUNCH("active_from_offsets_kernel");
+  moe_dims_t dn = d;
+  dn.d_ff_shared = 0;
+  return launch_ffn(dn, x, expert_offsets, sorted_rows, q1, q3, q2, nullptr, y, d.d_model, ws, L, s);
+}
+
+moe_status_t moe_combine(const moe_dims_t* dims, const float* y, const int32_t* inv, const float* topk_w,
+                         const float* y_shared, void* out, void* stream) {
+  g_detail[0] = 0;
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  if ((st = check_dev_ptr(y, "y")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(inv, "inv")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(topk_w, "topk_w")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(out, "out")) != MOE_OK) return st;
+  if (y_shared && (st = check_dev_ptr(y_shared, "y_shared")) != MOE_OK) return st;
+  if (!aligned16(y) || !aligned16(out) || (y_shared && !aligned16(y_shared)))
+    return fail(MOE_ERR_INVALID_ARG, "y, y_shared and out must be 16-byte aligned");
+  return launch_combine(*dims, y, inv, topk_w, y_shared, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* token_ids, const float* router_w,
+                         const float* router_b, const int32_t* tid2eid, const moe_qmat_t* w1,
+                         const moe_qmat_t* w3, const moe_qmat_t* w2, const moe_qmat_t* shared, void* out,
+                         int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  g_detail[0] = 0;
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t& d = *dims;
+  WsLayout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = check_route_args(d, x, router_w, token_ids, tid2eid)) != MOE_OK) return st;
+  if ((st = check_dev_ptr(out, "out")) != MOE_OK) return st;
+  if (!aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "out must be 16-byte aligned");
+  QMatDev q1, q3, q2, qs[3];
+  if ((st = check_qmat(w1, d.d_model, "w1", &q1, d.d_ff)) != MOE_OK) return st;
+  if ((st = check_qmat(w3, d.d_model, "w3", &q3, d.d_ff)) != MOE_OK) return st;
+  if ((st = check_qmat(w2, d.d_ff, "w2", &q2, d.d_model)) != MOE_OK) return st;
+  if (q1.fmt != q3.fmt || q1.group != q3.group)
+    return fail(MOE_ERR_UNSUPPORTED, "w1 and w3 must share one format");
+  if (d.d_ff_shared > 0) {
+    if (!shared) return fail(MOE_ERR_INVALID_ARG, "d_ff_shared > 0 but shared is NULL");
+    if ((st = check_qmat(&shared[0], d.d_model, "shared w1", &qs[0], d.d_ff_shared)) != MOE_OK) return st;
+    if ((st = check_qmat(&shared[1], d.d_model, "shared w3", &qs[1], d.d_ff_shared)) != MOE_OK) return st;
+    if ((st = check_qmat(&shared[2], d.d_ff_shared, "shared w2", &qs[2], d.d_model)) != MOE_OK) return st;
+    if (qs[0].fmt != qs[1].fmt || qs[0].group != qs[1].group)
+      return fail(MOE_ERR_UNSUPPORTED, "shared w1 and w3 must share one format");
+  }
+  DevInfo* di;
+  if ((st = dev_info(&di)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* ids = topk_ids_out ? topk_ids_out : ws_at<int>(ws, L.ids);
+  float* wts = topk_w_out ? topk_w_out : ws_at<float>(ws, L.wts);
+  if ((st = launch_route(d, x, router_w, router_b, token_ids, tid2eid, ids, wts, ws, L, s)) != MOE_OK) return st;
+  int* offsets = ws_at<int>(ws, L.offsets);
+  int* sorted = ws_at<int>(ws, L.sorted);
+  int* inv = ws_at<int>(ws, L.inv);
+  if ((st = launch_permute(d, ids, offsets, sorted, inv, ws, L, s)) != MOE_OK) return st;
+  float* y = ws_at<float>(ws, L.y);
+  if ((st = launch_ffn(d, x, offsets, sorted, q1, q3, q2, d.d_ff_shared > 0 ? qs : nullptr, y, d.d_model, ws, L,
+                       s)) != MOE_OK)
+    return st;
+  const float* y_sh = d.d_ff_shared > 0 ? y + (size_t)d.T * d.top_k * d.d_model : nullptr;
+  return launch_combine(d, y, inv, wts, y_sh, out, s);
+}
+
+moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const int32_t* token_ids_host,
+                              const float* router_w, const float* router_b, const int32_t* tid2eid,
+                              const moe_qmat_t* w1, const moe_qmat_t* w3, const moe_qmat_t* w2,
+                              const moe_qmat_t* shared, void* out_host, void* ws, size_t ws_bytes, void* stream) {
+  g_detail[0] = 0;
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t& d = *dims;
+  if (!x_host || !out_host) return fail(MOE_ERR_INVALID_ARG, "x_host/out_host is NULL");
+  if (d.hash_mode && !token_ids_host) return fail(MOE_ERR_INVALID_ARG, "token_ids_host is NULL");
+  WsLayout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  void* xd = ws_at<void>(ws, L.xstage);
+  int* td = ws_at<int>(ws, L.tokstage);
+  void* od = ws_at<void>(ws, L.outstage);
+  const size_t xbytes = (size_t)d.T * d.d_model * 2;
+  cudaError_t e = cudaMemcpyAsync(xd, x_host, xbytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy x to device");
+  if (d.hash_mode) {
+    e = cudaMemcpyAsync(td, token_ids_host, (size_t)d.T * sizeof(int), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy token ids to device");
+  }
+  st = moe_forward(dims, xd, d.hash_mode ? td : nullptr, router_w, router_b, tid2eid, w1, w3, w2, shared, od,
+                   nullptr, nullptr, ws, ws_bytes, stream);
+  if (st != MOE_OK) return st;
+  e = cudaMemcpyAsync(out_host, od, xbytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy out to host");
+  return MOE_OK;
+}
+
+moe_status_t moe_read_device_error(void* ws, int32_t* code_out, void* stream) {
+  g_detail[0] = 0;
+  if (!ws || !code_out) return fail(MOE_ERR_INVALID_ARG, "ws/code_out is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int v = 0;
+  e = cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  e = cudaMemset(ws, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  *code_out = v;
+  return MOE_OK;
+}
+
+}  // extern "C"

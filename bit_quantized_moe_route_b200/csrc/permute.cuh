@@ -1,0 +1,145 @@
+// Step 2 of the layer: group the T*k (token, slot) pairs by expert.
+//
+// A stable counting sort by expert id over the flat indices i = t*k + j:
+// per-expert histogram, exclusive scan -> expert_offsets, then a stable
+// scatter (ranks from warp match masks plus per-warp counts, tile by tile, so
+// no unordered atomics decide an order).  Also emits the ascending list of
+// experts that received at least one pair, used to size the FFN work lists.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kPermThreads = 1024;
+
+// Block-wide exclusive scan of one int per thread (1024 threads).
+__device__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_tot[lane];
+    int winc = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, winc, o);
+      if (lane >= o) winc += n;
+    }
+    warp_tot[lane] = winc - w;  // exclusive prefix of warp totals
+    if (lane == 31) *total = winc;
+  }
+  __syncthreads();
+  const int r = warp_tot[warp] + inc - v;
+  __syncthreads();
+  return r;
+}
+
+// One CTA of 1024 threads.  Dynamic shared memory: (2 + 32) * E ints.
+// active[0] = number of experts with pairs, active[1..] their ids ascending.
+__global__ void __launch_bounds__(kPermThreads)
+permute_kernel(const int* __restrict__ ids, int N, int E, int* __restrict__ offsets,
+               int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
+               int* err) {
+  extern __shared__ int sm[];
+  int* cnt = sm;            // [E] pairs per expert, later the running base
+  int* off = sm + E;        // [E] exclusive offsets
+  int* wc = sm + 2 * E;     // [32][E] per-warp counts of the current tile
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  __syncthreads();
+  bool bad = false;
+  for (int i = tid; i < N; i += kPermThreads) {
+    int e = ids[i];
+    if (e < 0 || e >= E) {
+      bad = true;
+      e = 0;
+    }
+    atomicAdd(&cnt[e], 1);
+  }
+  if (bad) set_error(err, kErrDeviceInput);
+  __syncthreads();
+  // exclusive scan of counts in chunks of 1024 experts
+  int carry = 0, acarry = 0;
+  for (int e0 = 0; e0 < E; e0 += kPermThreads) {
+    const int e = e0 + tid;
+    const int c = e < E ? cnt[e] : 0;
+    const int ex = block_exclusive_scan(c, warp_tot, &total);
+    const int chunk_total = total;
+    const int flag = c > 0 ? 1 : 0;
+    const int aex = block_exclusive_scan(flag, warp_tot, &total);
+    const int achunk = total;
+    if (e < E) {
+      off[e] = carry + ex;
+      offsets[e] = carry + ex;
+      if (flag) active[1 + acarry + aex] = e;
+    }
+    carry += chunk_total;
+    acarry += achunk;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    offsets[E] = carry;
+    active[0] = acarry;
+  }
+  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  __syncthreads();
+
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int t0 = 0; t0 < N; t0 += kPermThreads) {
+    for (int q = tid; q < 32 * E; q += kPermThreads) wc[q] = 0;
+    __syncthreads();
+    const int i = t0 + tid;
+    int e = -1;
+    if (i < N) {
+      e = ids[i];
+      if (e < 0 || e >= E) e = 0;
+    }
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int rank_w = __popc(peers & lt_mask);
+    if (e >= 0 && rank_w == 0) wc[warp * E + e] = __popc(peers);
+    __syncthreads();
+    if (e >= 0) {
+      int pre = 0;
+      for (int w = 0; w < warp; ++w) pre += wc[w * E + e];
+      const int p = off[e] + cnt[e] + pre + rank_w;
+      sorted_rows[p] = i;
+      inv[i] = p;
+    }
+    __syncthreads();
+    for (int x = tid; x < E; x += kPermThreads) {
+      int s = 0;
+      for (int w = 0; w < 32; ++w) s += wc[w * E + x];
+      cnt[x] += s;
+    }
+    __syncthreads();
+  }
+}
+
+// Active-expert list from caller-provided offsets (single CTA).
+__global__ void __launch_bounds__(kPermThreads)
+active_from_offsets_kernel(const int* __restrict__ offsets, int E, int* __restrict__ active) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  int acarry = 0;
+  for (int e0 = 0; e0 < E; e0 += kPermThreads) {
+    const int e = e0 + threadIdx.x;
+    const int flag = (e < E && offsets[e + 1] > offsets[e]) ? 1 : 0;
+    const int ex = block_exclusive_scan(flag, warp_tot, &total);
+    if (flag) active[1 + acarry + ex] = e;
+    acarry += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) active[0] = acarry;
+}
+
+}  // namespace moe

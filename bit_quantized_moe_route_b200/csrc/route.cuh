@@ -1,0 +1,293 @@
+// Step 1 of the layer: routing.
+//
+// learned: fp32 logits L = x . Wr^T, s = sqrt(logaddexp(L, 0)), top-k of the
+//   keys s + bias (ties to the lower expert id), w = s[ids] / sum(s[ids])
+//   [mlx-lm PR "Add DeepSeek-v4 (Flash/Pro)": gate dtype row of the
+//   cross-reference table, sqrtsoftplus stability note; model card
+//   "mlx-community / DeepSeek-V4-Flash-4bit", Architecture; model card
+//   "DeepSeek-V4-Flash-MLX-4bit", REAP-pruned builds: renormalise over the
+//   kept experts].
+// hash: ids = tid2eid[token_id] in table order; weights = renormalised
+//   sqrtsoftplus of the fp32 logits of those experts, or 1/k without a
+//   router [model card "mlx-community / DeepSeek-V4-Flash-4bit",
+//   Architecture: "Hash-routed MoE"; model card "DeepSeek-V4-Flash-MLX-4bit",
+//   "What this port implements": tid2eid keyed on token id].
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// Logits for small T: one warp per (expert, token batch).  The batch of x
+// rows sits in shared memory as bf16; each warp streams one router row with
+// 128-bit loads.
+// ---------------------------------------------------------------------------
+constexpr int kLogitWarps = 4;
+
+template <int NTB>
+__global__ void __launch_bounds__(kLogitWarps * 32)
+router_logits_small_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                           float* __restrict__ L, int T, int d, int E) {
+  extern __shared__ __align__(16) uint32_t xs_raw[];
+  const int t0 = blockIdx.y * NTB;
+  const int nt = min(NTB, T - t0);
+  const int tid = threadIdx.x;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t0 * d);
+    uint4* dst = reinterpret_cast<uint4*>(xs_raw);
+    const int n16 = nt * d / 8;
+    for (int i = tid; i < n16; i += blockDim.x) dst[i] = src[i];
+  }
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  const int e = blockIdx.x * kLogitWarps + warp;
+  if (e >= E) return;
+  float acc[NTB];
+#pragma unroll
+  for (int t = 0; t < NTB; ++t) acc[t] = 0.f;
+  const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
+  const int n4 = d >> 2;
+#pragma unroll 4
+  for (int i = lane; i < n4; i += 32) {
+    const float4 w = __ldg(wr + i);
+#pragma unroll
+    for (int t = 0; t < NTB; ++t) {
+      if (t < nt) {
+        const uint2 xv = reinterpret_cast<const uint2*>(xs_raw + (size_t)t * (d >> 1))[i];
+        acc[t] = fmaf(w.x, bf16lo(xv.x), acc[t]);
+        acc[t] = fmaf(w.y, bf16hi(xv.x), acc[t]);
+        acc[t] = fmaf(w.z, bf16lo(xv.y), acc[t]);
+        acc[t] = fmaf(w.w, bf16hi(xv.y), acc[t]);
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NTB; ++t) {
+    const float v = warp_sum(acc[t]);
+    if (lane == 0 && t < nt) L[(size_t)(t0 + t) * E + e] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Logits for large T: tiled fp32 SIMT GEMM, 128 tokens x 64 experts per CTA,
+// 8x4 outputs per thread, K in steps of 16 with register prefetch.
+// ---------------------------------------------------------------------------
+constexpr int kLBM = 128, kLBN = 64, kLBK = 16;
+
+__global__ void __launch_bounds__(256)
+router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                           float* __restrict__ L, int T, int d, int E) {
+  __shared__ __align__(16) float xs[kLBK][kLBM + 4];
+  __shared__ __align__(16) float wsm[kLBK][kLBN + 4];
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * kLBM, n0 = blockIdx.x * kLBN;
+  // loaders: x tile 128 x 16 bf16 -> each thread 8 elements (one 16-byte load)
+  const int xr = tid >> 1, xc = (tid & 1) * 8;
+  // W tile 64 x 16 fp32 -> each thread 4 elements (one float4)
+  const int wr = tid >> 2, wc = (tid & 3) * 4;
+  float acc[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+  uint4 xreg = make_uint4(0, 0, 0, 0);
+  float4 wreg = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto load = [&](int k0) {
+    const int gm = m0 + xr;
+    xreg = (gm < T) ? *reinterpret_cast<const uint4*>(x + (size_t)gm * d + k0 + xc) : make_uint4(0, 0, 0, 0);
+    const int gn = n0 + wr;
+    wreg = (gn < E) ? __ldg(reinterpret_cast<const float4*>(W + (size_t)gn * d + k0 + wc))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+  };
+  load(0);
+  for (int k0 = 0; k0 < d; k0 += kLBK) {
+    __syncthreads();
+    xs[xc + 0][xr] = bf16lo(xreg.x);
+    xs[xc + 1][xr] = bf16hi(xreg.x);
+    xs[xc + 2][xr] = bf16lo(xreg.y);
+    xs[xc + 3][xr] = bf16hi(xreg.y);
+    xs[xc + 4][xr] = bf16lo(xreg.z);
+    xs[xc + 5][xr] = bf16hi(xreg.z);
+    xs[xc + 6][xr] = bf16lo(xreg.w);
+    xs[xc + 7][xr] = bf16hi(xreg.w);
+    wsm[wc + 0][wr] = wreg.x;
+    wsm[wc + 1][wr] = wreg.y;
+    wsm[wc + 2][wr] = wreg.z;
+    wsm[wc + 3][wr] = wreg.w;
+    __syncthreads();
+    if (k0 + kLBK < d) load(k0 + kLBK);
+#pragma unroll
+    for (int kk = 0; kk < kLBK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&xs[kk][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&xs[kk][ty * 8 + 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&wsm[kk][tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int gm = m0 + ty * 8 + i;
+    if (gm >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int gn = n0 + tx * 4 + j;
+      if (gn < E) L[(size_t)gm * E + gn] = acc[i][j];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// sqrtsoftplus + biased top-k + renormalisation: one warp per token.
+// Expert e lives in lane e % 32, slot e / 32.
+// ---------------------------------------------------------------------------
+template <int MAXPER>
+__global__ void __launch_bounds__(256)
+topk_kernel(const float* __restrict__ L, const float* __restrict__ bias, int T, int E, int k,
+            int* __restrict__ ids, float* __restrict__ wts) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const int t = warp;
+  float key[MAXPER], sc[MAXPER];
+#pragma unroll
+  for (int i = 0; i < MAXPER; ++i) {
+    const int e = i * 32 + lane;
+    if (e < E) {
+      const float s = sqrt_softplus(L[(size_t)t * E + e]);
+      sc[i] = s;
+      float kv = bias ? s + bias[e] : s;
+      key[i] = (kv != kv) ? -INFINITY : kv;
+    } else {
+      sc[i] = 0.f;
+      key[i] = -INFINITY;
+    }
+  }
+  uint32_t taken = 0;  // bit i: slot i of this lane already selected
+  float my_s = 0.f;
+  int my_id = 0;
+  float ssum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    float best = -INFINITY;
+    int bidx = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < MAXPER; ++i) {
+      const int e = i * 32 + lane;
+      const bool ok = (e < E) && !((taken >> i) & 1u);
+      if (ok && (key[i] > best || (key[i] == best && e < bidx))) {
+        best = key[i];
+        bidx = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bidx, o);
+      if (ob > best || (ob == best && oi < bidx)) {
+        best = ob;
+        bidx = oi;
+      }
+    }
+    // owner lane publishes the unbiased score and marks the slot taken
+    float s_sel = 0.f;
+    const int owner = bidx & 31, slot = bidx >> 5;
+    if (lane == owner) {
+#pragma unroll
+      for (int i = 0; i < MAXPER; ++i)
+        if (i == slot) {
+          s_sel = sc[i];
+          taken |= 1u << i;
+        }
+    }
+    s_sel = __shfl_sync(0xffffffffu, s_sel, owner);
+    ssum += s_sel;
+    if (lane == j) {
+      my_s = s_sel;
+      my_id = bidx;
+    }
+  }
+  if (lane < k) {
+    ids[(size_t)t * k + lane] = my_id;
+    wts[(size_t)t * k + lane] = ssum > 0.f ? my_s / ssum : 1.f / (float)k;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Hash routing: one warp per token.  Out-of-range ids are reported through
+// the error word and routed to expert 0 with weight 0.
+// ---------------------------------------------------------------------------
+template <int KMAX>
+__global__ void __launch_bounds__(256)
+route_hash_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                  const int* __restrict__ token_ids, const int* __restrict__ table, int T, int d, int E,
+                  int k, int vocab, int* __restrict__ ids, float* __restrict__ wts, int* err) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  const int t = warp;
+  const int tok = token_ids[t];
+  const bool tok_ok = tok >= 0 && tok < vocab;
+  int eid[KMAX];
+  bool good[KMAX];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    eid[j] = 0;
+    good[j] = false;
+    if (j < k && tok_ok) {
+      const int e = table[(size_t)tok * k + j];
+      good[j] = e >= 0 && e < E;
+      eid[j] = good[j] ? e : 0;
+    }
+  }
+  bool any_bad = !tok_ok;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j)
+    if (j < k && !good[j]) any_bad = true;
+  if (any_bad && lane == 0) set_error(err, kErrDeviceInput);
+  float s[KMAX];
+  if (W != nullptr) {
+    float acc[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) acc[j] = 0.f;
+    const uint2* xr = reinterpret_cast<const uint2*>(x + (size_t)t * d);
+    for (int i = lane; i < (d >> 2); i += 32) {
+      const uint2 xv = xr[i];
+      const float x0 = bf16lo(xv.x), x1 = bf16hi(xv.x), x2 = bf16lo(xv.y), x3 = bf16hi(xv.y);
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j < k) {
+          const float4 w = __ldg(reinterpret_cast<const float4*>(W + (size_t)eid[j] * d) + i);
+          acc[j] = fmaf(w.x, x0, fmaf(w.y, x1, fmaf(w.z, x2, fmaf(w.w, x3, acc[j]))));
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      const float v = warp_sum(acc[j]);
+      s[j] = (j < k && good[j]) ? sqrt_softplus(v) : 0.f;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) s[j] = (j < k && good[j]) ? 1.f : 0.f;
+  }
+  float ssum = 0.f;
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) ssum += s[j];
+#pragma unroll
+  for (int j = 0; j < KMAX; ++j) {
+    if (j < k && lane == j) {
+      ids[(size_t)t * k + j] = eid[j];
+      float w = 0.f;
+      if (good[j]) w = ssum > 0.f ? s[j] / ssum : 0.f;
+      wts[(size_t)t * k + j] = w;
+    }
+  }
+}
+
+}  // namespace moe
