@@ -1,0 +1,421 @@
+"""Benchmark of the routed low-bit MoE layer on B200.
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one full layer forward (routing, permutation, grouped SwiGLU
+expert FFN over packed weights, combine) over one batch of synthetic input
+resident in HBM.  The default workload is the decode layer (T=1 token,
+d_model=4096, 256 routed experts, top-8, d_ff=2048, affine 4-bit group-64
+experts plus an 8-bit shared expert).  L2 is flushed (a 512 MiB write)
+between timed steps, outside the timed events.
+
+With N > 1 (launched by torchrun) every rank runs an independent replica of
+the layer on its own GPU ("replicas only": the layer has no exchange step on
+one node in this build); the value is the sum of all ranks' tokens over the
+slowest rank's device time.
+
+--impl reference times the fp64 CPU oracle (test infrastructure, run as it
+stands) on this host's cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("MoE-layer tokens/s at 1 B200; achieved HBM GB/s (decode) / tensor TFLOPS (prefill) vs peak")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default="decode")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=25.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--override", action="append", default=[],
+                    help="key=value change to the workload (profiling small cases), e.g. E=16")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), d.get("bf16_tflops", FALLBACK_BF16_TFLOPS), \
+            d.get("bf16_tflops_sustained", d.get("bf16_tflops", FALLBACK_BF16_TFLOPS)), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+def src_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "bit_quantized_moe_route_b200", "csrc", "*"))):
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def workload_desc(cfg):
+    f13, f2 = cfg["w13"], cfg["w2"]
+    fmt = lambda t: f"{t[0]}{t[1]}g{t[2]}" if t[0] == "affine" else "mxfp4g32"  # noqa: E731
+    d = {"workload": cfg["name"], "T": cfg["T"], "d_model": cfg["d"], "n_experts": cfg["E"], "top_k": cfg["k"],
+         "d_ff": cfg["f"], "routing": cfg["routing"], "w1_w3": fmt(f13), "w2": fmt(f2)}
+    if cfg.get("shared"):
+        d["shared_expert"] = f"{fmt(cfg['shared'])} d_ff={cfg['f_shared']}"
+    return d
+
+
+# ---------------------------------------------------------------- algorithmic bytes / flops
+def kernel_work(inp, ids):
+    """Algorithmic bytes (and flops) of each kernel of one forward."""
+    import numpy as np
+    c = inp.cfg
+    T, d, E, k, f = c["T"], c["d"], c["E"], c["k"], c["f"]
+    ids = np.asarray(ids)
+    active = np.unique(ids)
+    n_act = len(active)
+    b13 = inp.w1.packed_bytes_per_expert() + inp.w3.packed_bytes_per_expert()
+    b2 = inp.w2.packed_bytes_per_expert()
+    sh13 = sh2 = 0
+    P = T * k
+    if inp.shared is not None:
+        sh13 = inp.shared[0].packed_bytes_per_expert() + inp.shared[1].packed_bytes_per_expert()
+        sh2 = inp.shared[2].packed_bytes_per_expert()
+        P += T
+    fs = c.get("f_shared", 0) if inp.shared is not None else 0
+    work = {}
+    if c["routing"] == "hash":
+        rows = len(np.unique(ids))
+        work["route_hash"] = T * d * 2 + T * 4 + T * k * 4 + rows * d * 4 + T * k * 8
+    else:
+        work["router_logits"] = E * d * 4 + T * d * 2 + T * E * 4
+        work["topk"] = T * E * 4 + E * 4 + T * k * 8
+    work["permute"] = T * k * 4 * 3 + (E + 1) * 4
+    work["ffn_w13_swiglu"] = n_act * b13 + sh13 + T * d * 2 + P * max(f, fs) * 4
+    work["ffn_w2"] = n_act * b2 + sh2 + P * max(f, fs) * 4 + P * d * 4
+    work["combine"] = P * d * 4 + T * d * 2 + T * k * 8
+    flops = 2.0 * T * k * 3 * d * f + (2.0 * T * 3 * d * fs if fs else 0.0)
+    return work, flops, n_act, (n_act * (b13 + b2) + sh13 + sh2)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + ",".join(self.FIELDS), "--format=csv,noheader,nounits",
+                 "-i", self.gpu_id, "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, pw, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                pw.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(pw) if pw else None, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_sample_time(inp, budget_s: float, max_pairs=None, start_pair: int = 0):
+    """Time the oracle on a bounded sample; returns (seconds per token, sample description, pairs, blas threads).
+
+    Routing runs for every token; the expert FFN then runs for consecutive
+    (token, slot) pairs starting at ``start_pair`` until the time budget (or
+    max_pairs) is spent.  The per-token time is extrapolated from the pairs
+    done: k routed slots plus the shared expert make one token.
+    """
+    import oracle
+    c = inp.cfg
+    T, d, k = c["T"], c["d"], c["k"]
+    x = inp.x.float().cpu().numpy()
+    t0 = time.perf_counter()
+    if c["routing"] == "hash":
+        ids, w = oracle.route_hash(x, inp.router_w.cpu().numpy(), inp.token_ids.cpu().numpy(),
+                                   inp.tid2eid.cpu().numpy())
+    else:
+        ids, w, _, _ = oracle.route_learned(x, inp.router_w.cpu().numpy(), inp.router_b.cpu().numpy(), k)
+    oracle.permute(ids, c["E"])
+    t_route = time.perf_counter() - t0
+    ppt = k + (1 if inp.shared is not None else 0)
+    mats = {"w1": inp.w1, "w3": inp.w3, "w2": inp.w2}
+    shared = dict(zip(("w1", "w3", "w2"), inp.shared)) if inp.shared is not None else None
+    done, t_ffn, pair = 0, 0.0, start_pair % (T * ppt)
+    while True:
+        tok, j = divmod(pair, ppt)
+        t1 = time.perf_counter()
+        src, e = (mats, int(ids[tok, j])) if j < k else (shared, 0)
+        n_in = {"w1": d, "w3": d, "w2": src["w1"].n_out}
+        W = {n: oracle.dequant(m.fmt, m.bits, m.group, n_in[n], *m.expert_numpy(e)) for n, m in src.items()}
+        oracle.swiglu_ffn(W["w1"], W["w3"], W["w2"], x[tok:tok + 1])
+        t_ffn += time.perf_counter() - t1
+        done += 1
+        pair = (pair + 1) % (T * ppt)
+        if t_ffn >= budget_s or (max_pairs and done >= max_pairs):
+            break
+    per_token = t_ffn / done * ppt + t_route / T
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        blas = 1
+    desc = (f"routing for all {T} tokens ({t_route:.2f}s) + {done} (token, expert) FFN pairs "
+            f"({t_ffn:.1f}s); per-token time = mean pair time x {ppt} + routing time / T")
+    return per_token, desc, done, blas
+
+
+def overrides(args):
+    out = {}
+    for kv in args.override:
+        key, val = kv.split("=", 1)
+        out[key] = int(val) if val.lstrip("-").isdigit() else val
+    return out
+
+
+def reference_arm(args):
+    """The oracle, as it stands, on this host's cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np  # noqa: F401
+    import torch
+    from synthetic import make_inputs
+    dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
+    inp = make_inputs(args.config, dev, **overrides(args))
+    c = inp.cfg
+    budget_total = 150.0
+    step_budget = max(0.5, budget_total / max(1, args.steps + args.warmup))
+    times, pairs = [], 0
+    desc = ""
+    t_start = time.perf_counter()
+    n_steps = 0
+    for s in range(args.warmup + args.steps):
+        per_tok, desc, done, blas = oracle_sample_time(inp, step_budget, max_pairs=1, start_pair=s)
+        if s >= args.warmup:
+            times.append(per_tok)
+            pairs += done
+            n_steps += 1
+        if time.perf_counter() - t_start > budget_total:
+            break
+    per_tok = statistics.mean(times) if times else float("nan")
+    value = 1.0 / per_tok
+    cores = blas
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": n_steps, "warmup": args.warmup, "ms_per_step": per_tok * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_desc(c),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"per step: {desc}; steps capped at {budget_total:.0f}s of CPU work"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def ours_arm(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_moe_route_b200 as moe
+    from synthetic import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    moe.load_library()
+    inp = make_inputs(args.config, dev, **overrides(args))
+    c = inp.cfg
+    T, d, k = c["T"], c["d"], c["k"]
+    dims = moe.make_dims(T, d, c["f"], c["E"], k, c["routing"] == "hash",
+                         c.get("vocab", 0) if c["routing"] == "hash" else 0,
+                         c.get("f_shared", 0) if inp.shared is not None else 0)
+    ws = moe.alloc_workspace(dims, dev)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+    wts = torch.empty(T, k, dtype=torch.float32, device=dev)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def fwd():
+        moe.forward(dims, inp.x, inp.token_ids, inp.router_w, inp.router_b, inp.tid2eid, inp.w1, inp.w3, inp.w2,
+                    inp.shared, out, ws, topk_ids_out=ids, topk_w_out=wts)
+
+    for i in range(max(3, args.warmup)):
+        flush.fill_(i & 0xFF)
+        fwd()
+    torch.cuda.synchronize()
+    work, flops, n_act, weight_bytes = kernel_work(inp, ids.cpu().numpy())
+
+    # ---- timed region: K forwards, L2 flushed between them (outside the events)
+    n_ev = 16
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid) if getattr(props, "uuid", None) else str(local))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.2)
+    keep = []
+    for s in range(args.steps):
+        flush.fill_(s & 0xFF)
+        step_ev[s][0].record(stream)
+        keep.append(moe.set_timing_events(evs[s]))
+        fwd()
+        step_ev[s][1].record(stream)
+    torch.cuda.synchronize()
+    labels = moe.timing_labels()
+    clocks = sampler.stop()
+    if world > 1:
+        dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    total_ms = sum(step_ms)
+    per_kernel = {}
+    for s in range(args.steps):
+        for i, lab in enumerate(labels):
+            per_kernel.setdefault(lab, []).append(evs[s][i].elapsed_time(evs[s][i + 1]))
+    kern_ms = {lab: statistics.mean(v) for lab, v in per_kernel.items()}
+    ms_per_step = total_ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms_per_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_per_step = float(t.item())
+
+    # ---- end-to-end through the C ABI with host buffers (pinned), copies inside
+    x_h = inp.x.cpu().pin_memory()
+    tok_h = inp.token_ids.cpu().pin_memory() if inp.token_ids is not None else None
+    out_h = torch.empty(T, d, dtype=torch.bfloat16).pin_memory()
+    layer_args = (inp.router_w, inp.router_b, inp.tid2eid, inp.w1, inp.w3, inp.w2, inp.shared)
+    for i in range(3):
+        moe.forward_host(dims, x_h, tok_h, *layer_args, out_h, ws)
+    torch.cuda.synchronize()
+    e2e_steps = max(10, min(args.steps, 200))
+    e2e_ms = 0.0
+    for s in range(e2e_steps):
+        flush.fill_(s & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        moe.forward_host(dims, x_h, tok_h, *layer_args, out_h, ws)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms += a.elapsed_time(b)
+    e2e_ms /= e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = T * d * 2 + (T * 4 if tok_h is not None else 0)
+    d2h = T * d * 2
+    err = moe.read_device_error(ws)
+
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    dom = max(kern_ms, key=kern_ms.get)
+    dom_ms = kern_ms[dom]
+    achieved = work.get(dom, 0) / (dom_ms * 1e-3) / 1e9
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        with open(prof) as fh:
+            tj = json.load(fh)
+        ent = tj.get(c["name"], {}).get(dom)
+        if ent and ent.get("src_hash") == src_hash():
+            traffic = ent.get("dram_bytes_per_launch")
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+                "algorithmic_bytes_per_launch": work.get(dom, 0)}
+    layer_bytes = sum(work.values())
+    value = T * world / (ms_per_step * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_desc(c), l2="flushed by a 512 MiB write between timed steps (outside the events)",
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "roofline": roofline,
+        "layer": {"bytes_per_step": layer_bytes, "weight_bytes": weight_bytes, "distinct_routed_experts": n_act,
+                  "GBps_whole_step": layer_bytes / (ms_per_step * 1e-3) / 1e9,
+                  "frac_whole_step": layer_bytes / (ms_per_step * 1e-3) / 1e9 / hbm,
+                  "flops_per_step": flops, "kernel_ms": kern_ms},
+        "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": len(labels) * args.steps,
+        "clocks": clocks,
+        "device_error": err,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_tok, desc, done, blas = oracle_sample_time(inp, args.cpu_budget)
+        line["cpu_baseline"] = {"value": 1.0 / per_tok, "unit": "tokens/s", "cores": blas, "kind": "oracle",
+                                "sample": desc, "cores_available": len(os.sched_getaffinity(0))}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        reference_arm(args)
+    else:
+        ours_arm(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -59,6 +59,9 @@ _SIGS = {
     "moe_read_device_error": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int32), _VP]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_error_detail": (ctypes.c_char_p, []),
+    "moe_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
+    "moe_timing_count": (ctypes.c_int32, []),
+    "moe_timing_label": (ctypes.c_char_p, [ctypes.c_int32]),
 }
 
 
@@ -189,3 +192,26 @@ def read_device_error(ws, stream=None) -> int:
 
 def status_string(status: int) -> str:
     return load_library().moe_status_string(status).decode()
+
+
+def set_timing_events(events: Optional[Sequence["torch.cuda.Event"]]):
+    """Arm the per-kernel timing hook for the next forward on this thread.
+
+    ``events`` must be CUDA events created with timing enabled; they are
+    recorded on the forward's stream around each of its kernels.  Returns the
+    ctypes array (keep it alive until the forward has been issued).
+    """
+    lib = load_library()
+    if events is None:
+        lib.moe_set_timing_events(None, 0)
+        return None
+    arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
+    lib.moe_set_timing_events(arr, len(events))
+    return arr
+
+
+def timing_labels():
+    """Labels of the kernels timed by the last hooked forward."""
+    lib = load_library()
+    n = lib.moe_timing_count()
+    return [lib.moe_timing_label(i).decode() for i in range(max(0, n - 1))]

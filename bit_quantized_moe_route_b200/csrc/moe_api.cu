@@ -21,6 +21,38 @@ namespace {
 
 thread_local char g_detail[512] = "";
 
+// Benchmark timing hooks (see moe_set_timing_events).
+struct TimingHook {
+  void* const* events = nullptr;
+  int n = 0;
+  int used = 0;
+  const char* labels[32] = {};
+};
+thread_local TimingHook g_hook;
+thread_local int g_hook_count = 0;
+thread_local const char* g_hook_labels[32] = {};
+
+void hook_begin(cudaStream_t s) {
+  if (g_hook.events && g_hook.n > 0) {
+    cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_hook.events[0]), s);
+    g_hook.used = 1;
+  }
+}
+void hook_mark(cudaStream_t s, const char* label) {
+  if (g_hook.events && g_hook.used > 0 && g_hook.used < g_hook.n && g_hook.used <= 32) {
+    g_hook.labels[g_hook.used - 1] = label;
+    cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_hook.events[g_hook.used]), s);
+    ++g_hook.used;
+  }
+}
+void hook_end() {
+  if (g_hook.events) {
+    g_hook_count = g_hook.used;
+    for (int i = 0; i < 32; ++i) g_hook_labels[i] = g_hook.labels[i];
+    g_hook = TimingHook{};
+  }
+}
+
 moe_status_t fail(moe_status_t st, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -214,6 +246,7 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
       route_hash_kernel<32><<<blocks, 256, 0, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts, d.top_k,
                                                    d.vocab, ids, wts, err);
     MOE_CHECK_LAUNCH("route_hash_kernel");
+    hook_mark(s, "route_hash");
     return MOE_OK;
   }
   float* logits = ws_at<float>(ws, L.logits);
@@ -222,10 +255,12 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
     router_logits_small_kernel<8><<<grid, kLogitWarps * 32, 8 * d.d_model * 2, s>>>(xb, rw, logits, d.T,
                                                                                       d.d_model, d.n_experts);
     MOE_CHECK_LAUNCH("router_logits_small_kernel");
+    hook_mark(s, "router_logits");
   } else {
     dim3 grid(ceil_div(d.n_experts, kLBN), ceil_div(d.T, kLBM));
     router_logits_tiled_kernel<<<grid, 256, 0, s>>>(xb, rw, logits, d.T, d.d_model, d.n_experts);
     MOE_CHECK_LAUNCH("router_logits_tiled_kernel");
+    hook_mark(s, "router_logits");
   }
   const int blocks = ceil_div(d.T * 32, 256);
   if (d.n_experts <= 32)
@@ -235,6 +270,7 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
   else
     topk_kernel<32><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts);
   MOE_CHECK_LAUNCH("topk_kernel");
+  hook_mark(s, "topk");
   return MOE_OK;
 }
 
@@ -246,6 +282,7 @@ moe_status_t launch_permute(const moe_dims_t& d, const int* ids, int* offsets, i
   permute_kernel<<<1, kPermThreads, smem, s>>>(ids, d.T * d.top_k, d.n_experts, offsets, sorted, inv, active,
                                                err);
   MOE_CHECK_LAUNCH("permute_kernel");
+  hook_mark(s, "permute");
   return MOE_OK;
 }
 
@@ -288,6 +325,7 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
     const int grid = std::max(1, std::min(items, di->sms * di->ffn1_blocks));
     ffn_gemv_kernel<1, 4><<<grid, kFfnThreads, 0, s>>>(q);
     MOE_CHECK_LAUNCH("ffn_gemv_kernel<1>");
+    hook_mark(s, "ffn_w13_swiglu");
   }
   // stage 2: y = W2 h
   {
@@ -306,6 +344,7 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
     const int grid = std::max(1, std::min(items, di->sms * di->ffn2_blocks));
     ffn_gemv_kernel<2, 8><<<grid, kFfnThreads, 0, s>>>(q);
     MOE_CHECK_LAUNCH("ffn_gemv_kernel<2>");
+    hook_mark(s, "ffn_w2");
   }
   return MOE_OK;
 }
@@ -316,6 +355,7 @@ moe_status_t launch_combine(const moe_dims_t& d, const float* y, const int* inv,
   combine_kernel<<<grid, 256, 0, s>>>(y, inv, w, y_shared, reinterpret_cast<__nv_bfloat16*>(out), d.T,
                                       d.top_k, d.d_model);
   MOE_CHECK_LAUNCH("combine_kernel");
+  hook_mark(s, "combine");
   return MOE_OK;
 }
 
@@ -344,6 +384,11 @@ moe_status_t check_route_args(const moe_dims_t& d, const void* x, const float* r
   return MOE_OK;
 }
 
+moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t* token_ids, const float* router_w,
+                              const float* router_b, const int32_t* tid2eid, const QMatDev& q1, const QMatDev& q3,
+                              const QMatDev& q2, const QMatDev* qs, void* out, int32_t* topk_ids_out,
+                              float* topk_w_out, void* ws, const WsLayout& L, cudaStream_t s);
+
 }  // namespace
 
 // ======================================================================= ABI
@@ -368,6 +413,22 @@ const char* moe_status_string(moe_status_t s) {
 }
 
 const char* moe_last_error_detail(void) { return g_detail; }
+
+moe_status_t moe_set_timing_events(void* const* events, int32_t n_events) {
+  g_hook = TimingHook{};
+  if (events && n_events > 0) {
+    g_hook.events = events;
+    g_hook.n = std::min<int32_t>(n_events, 33);
+  }
+  return MOE_OK;
+}
+
+int32_t moe_timing_count(void) { return g_hook_count; }
+
+const char* moe_timing_label(int32_t i) {
+  if (i < 0 || i >= 32 || i + 1 >= g_hook_count || !g_hook_labels[i]) return "";
+  return g_hook_labels[i];
+}
 
 moe_status_t moe_route(const moe_dims_t* dims, const void* x, const float* router_w, const float* router_b,
                        const int32_t* token_ids, const int32_t* tid2eid, int32_t* topk_ids, float* topk_w,
@@ -480,6 +541,21 @@ moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* t
   DevInfo* di;
   if ((st = dev_info(&di)) != MOE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = forward_launches(d, x, token_ids, router_w, router_b, tid2eid, q1, q3, q2, qs, out, topk_ids_out, topk_w_out,
+                        ws, L, s);
+  hook_end();
+  return st;
+}
+
+}  // extern "C"
+
+namespace {
+moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t* token_ids, const float* router_w,
+                              const float* router_b, const int32_t* tid2eid, const QMatDev& q1, const QMatDev& q3,
+                              const QMatDev& q2, const QMatDev* qs, void* out, int32_t* topk_ids_out,
+                              float* topk_w_out, void* ws, const WsLayout& L, cudaStream_t s) {
+  moe_status_t st;
+  hook_begin(s);
   int* ids = topk_ids_out ? topk_ids_out : ws_at<int>(ws, L.ids);
   float* wts = topk_w_out ? topk_w_out : ws_at<float>(ws, L.wts);
   if ((st = launch_route(d, x, router_w, router_b, token_ids, tid2eid, ids, wts, ws, L, s)) != MOE_OK) return st;
@@ -494,6 +570,9 @@ moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* t
   const float* y_sh = d.d_ff_shared > 0 ? y + (size_t)d.T * d.top_k * d.d_model : nullptr;
   return launch_combine(d, y, inv, wts, y_sh, out, s);
 }
+}  // namespace
+
+extern "C" {
 
 moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const int32_t* token_ids_host,
                               const float* router_w, const float* router_b, const int32_t* tid2eid,

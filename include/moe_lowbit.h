@@ -222,6 +222,19 @@ moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const 
  */
 moe_status_t moe_read_device_error(void* ws, int32_t* code_out, void* stream);
 
+/*
+ * Benchmark timing hooks (calling thread only).  When `events` is non-NULL,
+ * the next moe_forward / moe_forward_host call on this thread records
+ * events[0] (a cudaEvent_t) before its first kernel and events[i+1] after its
+ * i-th kernel, for at most n_events events, on the call's stream; the hook is
+ * consumed by that call.  moe_timing_count() then returns how many events
+ * were recorded and moe_timing_label(i) names the kernel between events[i]
+ * and events[i+1].  Pass NULL to clear.
+ */
+moe_status_t moe_set_timing_events(void* const* events, int32_t n_events);
+int32_t moe_timing_count(void);
+const char* moe_timing_label(int32_t i);
+
 /* Static description of a status code. */
 const char* moe_status_string(moe_status_t status);
 
