@@ -21,7 +21,9 @@ from ._lib import (  # noqa: F401
     qmat,
     read_device_error,
     route,
+    set_timing_events,
     status_string,
+    timing_labels,
     workspace_size,
 )
 from .layer import MoELayer  # noqa: F401

@@ -205,6 +205,9 @@ def set_timing_events(events: Optional[Sequence["torch.cuda.Event"]]):
     if events is None:
         lib.moe_set_timing_events(None, 0)
         return None
+    for ev in events:                 # torch creates the CUDA event on first record
+        if not ev.cuda_event:
+            ev.record()
     arr = (ctypes.c_void_p * len(events))(*[ev.cuda_event for ev in events])
     lib.moe_set_timing_events(arr, len(events))
     return arr

@@ -32,17 +32,26 @@ thread_local TimingHook g_hook;
 thread_local int g_hook_count = 0;
 thread_local const char* g_hook_labels[32] = {};
 
+// A failed record disarms the hook and clears the CUDA error so that it
+// cannot be mistaken for a kernel launch failure.
+void hook_record(int i, cudaStream_t s) {
+  if (!g_hook.events[i] || cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_hook.events[i]), s) != cudaSuccess) {
+    cudaGetLastError();
+    g_hook.events = nullptr;
+    g_hook.used = 0;
+  }
+}
 void hook_begin(cudaStream_t s) {
   if (g_hook.events && g_hook.n > 0) {
-    cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_hook.events[0]), s);
     g_hook.used = 1;
+    hook_record(0, s);
   }
 }
 void hook_mark(cudaStream_t s, const char* label) {
   if (g_hook.events && g_hook.used > 0 && g_hook.used < g_hook.n && g_hook.used <= 32) {
     g_hook.labels[g_hook.used - 1] = label;
-    cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_hook.events[g_hook.used]), s);
     ++g_hook.used;
+    hook_record(g_hook.used - 1, s);
   }
 }
 void hook_end() {
