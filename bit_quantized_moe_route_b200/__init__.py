@@ -13,6 +13,7 @@ from ._lib import (  # noqa: F401
     alloc_workspace,
     combine,
     expert_ffn,
+    expert_ffn_noalloc,
     forward,
     forward_host,
     load_library,

@@ -49,6 +49,8 @@ _SIGS = {
     "moe_permute": (ctypes.c_int, [ctypes.POINTER(Dims), _VP, _VP, _VP, _VP, _VP, ctypes.c_size_t, _VP]),
     "moe_expert_ffn": (ctypes.c_int, [ctypes.POINTER(Dims), _VP, _VP, _VP, ctypes.POINTER(QMatC),
                                       ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP, _VP, ctypes.c_size_t, _VP]),
+    "moe_expert_ffn_noalloc": (ctypes.c_int, [ctypes.POINTER(Dims), _VP, _VP, _VP, ctypes.POINTER(QMatC),
+                                              ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP, _VP]),
     "moe_combine": (ctypes.c_int, [ctypes.POINTER(Dims), _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_forward": (ctypes.c_int, [ctypes.POINTER(Dims), _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(QMatC),
                                    ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP, _VP,
@@ -145,6 +147,17 @@ def expert_ffn(dims, x, expert_offsets, sorted_rows, w1, w3, w2, y, ws, stream=N
     _check(load_library().moe_expert_ffn(ctypes.byref(dims), _ptr(x), _ptr(expert_offsets), _ptr(sorted_rows),
                                          ctypes.byref(q1), ctypes.byref(q3), ctypes.byref(q2), _ptr(y), _ptr(ws),
                                          ws.numel(), _stream(stream)), "moe_expert_ffn")
+
+
+def expert_ffn_noalloc(dims, x, expert_offsets, sorted_rows, w1, w3, w2, y, stream=None):
+    """moe_expert_ffn_noalloc: the expert FFN for callers that cannot allocate
+    device memory; its scratch is a fixed 4 MiB static device array shared by
+    every call on the device (calls must not overlap on the GPU)."""
+    q1, q3, q2 = qmat(w1), qmat(w3), qmat(w2)
+    _check(load_library().moe_expert_ffn_noalloc(ctypes.byref(dims), _ptr(x), _ptr(expert_offsets),
+                                                 _ptr(sorted_rows), ctypes.byref(q1), ctypes.byref(q3),
+                                                 ctypes.byref(q2), _ptr(y), _stream(stream)),
+           "moe_expert_ffn_noalloc")
 
 
 def combine(dims, y, inv, topk_w, y_shared, out, stream=None):

@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/moe_lowbit.h"
 #include "common.cuh"
@@ -630,3 +631,91 @@ moe_status_t moe_read_device_error(void* ws, int32_t* code_out, void* stream) {
 }
 
 }  // extern "C"
+
+// ============================================================================
+// Allocation-free variant of moe_expert_ffn.
+//
+// Some callers cannot hand the library a workspace: a host framework that owns
+// the whole device memory pool and forbids foreign allocations, a plug-in
+// that is only ever given its input and output buffers, or code that must not
+// call cudaMalloc/cudaFree because those calls can synchronise the device.
+// For them the expert FFN's scratch (the active-expert list and the SwiGLU
+// hidden rows h) lives in one file-scope device array of fixed size instead.
+// ============================================================================
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB on every device that loads the library
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+void* g_static_addr[64] = {};
+
+// Device address of g_static_scratch on the current device.  In host code the
+// symbol is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+moe_status_t static_scratch_addr(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
+    }
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_expert_ffn_noalloc(const moe_dims_t* dims, const void* x, const int32_t* expert_offsets,
+                                               const int32_t* sorted_rows, const moe_qmat_t* w1, const moe_qmat_t* w3,
+                                               const moe_qmat_t* w2, float* y, void* stream) {
+  g_detail[0] = 0;
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t& d = *dims;
+  // scratch layout inside the static array: [error word | active list | h]
+  WsLayout Ls{};
+  Ls.hdr = 0;
+  Ls.active = align_up(sizeof(WsHeader));
+  Ls.h = align_up(Ls.active + (size_t)(d.n_experts + 1) * sizeof(int));
+  const size_t need = Ls.h + (size_t)d.T * d.top_k * d.d_ff * sizeof(float);
+  if (need > kStaticScratchBytes)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "T*top_k*d_ff = %lld hidden values need %zu bytes of scratch; the allocation-free entry point "
+                "has %zu (use moe_expert_ffn with a workspace)",
+                (long long)d.T * d.top_k * d.d_ff, need, kStaticScratchBytes);
+  if ((st = check_dev_ptr(x, "x")) != MOE_OK) return st;
+  if (!aligned16(x)) return fail(MOE_ERR_INVALID_ARG, "x must be 16-byte aligned");
+  if ((st = check_dev_ptr(expert_offsets, "expert_offsets")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(sorted_rows, "sorted_rows")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(y, "y")) != MOE_OK) return st;
+  if (!aligned16(y)) return fail(MOE_ERR_INVALID_ARG, "y must be 16-byte aligned");
+  QMatDev q1, q3, q2;
+  if ((st = check_qmat(w1, d.d_model, "w1", &q1, d.d_ff)) != MOE_OK) return st;
+  if ((st = check_qmat(w3, d.d_model, "w3", &q3, d.d_ff)) != MOE_OK) return st;
+  if ((st = check_qmat(w2, d.d_ff, "w2", &q2, d.d_model)) != MOE_OK) return st;
+  if (q1.fmt != q3.fmt || q1.group != q3.group)
+    return fail(MOE_ERR_UNSUPPORTED, "w1 and w3 must share one format");
+  DevInfo* di;
+  if ((st = dev_info(&di)) != MOE_OK) return st;
+  void* scratch = nullptr;
+  if ((st = static_scratch_addr(&scratch)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the error word starts at zero on every call; the active list and h are
+  // fully rewritten before they are read
+  cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s);
+  if (e != cudaSuccess) return cuda_fail(e, "clear static scratch header");
+  active_from_offsets_kernel<<<1, kPermThreads, 0, s>>>(expert_offsets, d.n_experts, ws_at<int>(scratch, Ls.active));
+  MOE_CHECK_LAUNCH("active_from_offsets_kernel");
+  moe_dims_t dn = d;
+  dn.d_ff_shared = 0;
+  return launch_ffn(dn, x, expert_offsets, sorted_rows, q1, q3, q2, nullptr, y, d.d_model, scratch, Ls, s);
+}

@@ -176,6 +176,30 @@ moe_status_t moe_expert_ffn(const moe_dims_t* dims, const void* x, const int32_t
                             const moe_qmat_t* w2, float* y, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_expert_ffn without a workspace (no counterpart on the pages; it exists
+ * for callers of this library that cannot allocate device memory: a host
+ * framework that owns the whole device pool and forbids foreign allocations,
+ * a plug-in that is only given its input and output buffers, or code that
+ * must not call cudaMalloc/cudaFree because those calls can synchronise the
+ * device).  Same arguments and results as moe_expert_ffn, minus ws/ws_bytes.
+ *
+ * Its scratch (error word, active-expert list, hidden rows h) is one static
+ * device array of 4 MiB that every GPU loading this library holds until the
+ * process exits.  Limit: 256 + 256-aligned 4*(n_experts+1) + 4*T*top_k*d_ff
+ * bytes must fit in 4 MiB (e.g. T*top_k <= 510 at d_ff = 2048); larger
+ * problems return MOE_ERR_UNSUPPORTED before any launch.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) and
+ * caches it, so make that first call before any stream capture.  Every call
+ * on a device shares the same array and leaves its contents behind: calls
+ * that overlap on the GPU (different streams without ordering, or several
+ * host threads) race and corrupt each other's results.  The library itself
+ * allocates nothing on this path.
+ */
+moe_status_t moe_expert_ffn_noalloc(const moe_dims_t* dims, const void* x, const int32_t* expert_offsets,
+                                    const int32_t* sorted_rows, const moe_qmat_t* w1, const moe_qmat_t* w3,
+                                    const moe_qmat_t* w2, float* y, void* stream);
+
+/*
  * Step 4 -- weighted combine:
  *   out[t] = bf16_rne( sum_{j<k} topk_w[t,j] * y[inv[t*k+j]] + y_shared[t] )
  * summed in ascending j, then the shared term.
