@@ -13,6 +13,7 @@
 #include "../../include/moe_lowbit.h"
 #include "common.cuh"
 #include "ffn_gemv.cuh"
+#include "ffn_stream.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -217,6 +218,17 @@ moe_status_t dev_info(DevInfo** out) {
       cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 34 * 1024 * 4);
       cudaFuncSetAttribute(router_logits_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            8 * 8192 * 2);
+      cudaFuncSetAttribute(route_small_fused_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(route_small_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(route_small_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(route_hash_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(route_hash_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      cudaFuncSetAttribute(ffn_stream_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+      cudaFuncSetAttribute(ffn_stream_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+      cudaFuncSetAttribute(ffn_stream_kernel<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+      cudaFuncSetAttribute(ffn_stream_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+      cudaFuncSetAttribute(ffn_stream_kernel<1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+      cudaFuncSetAttribute(ffn_stream_kernel<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
       int b1 = 0, b2 = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, ffn_gemv_kernel<1, 4>, kFfnThreads, 0);
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, ffn_gemv_kernel<2, 8>, kFfnThreads, 0);
@@ -284,6 +296,53 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
   return MOE_OK;
 }
 
+// Routing and permutation in one launch for small batches.
+bool fused_route_ok(const moe_dims_t& d) {
+  return d.T <= kFusedMaxT && d.d_model <= 4096 && d.d_model % 64 == 0 && d.top_k <= 32;
+}
+
+moe_status_t launch_route_fused(const moe_dims_t& d, const void* x, const float* rw, const float* rb, const int* tok,
+                                const int* table, int* ids, float* wts, int* offsets, int* sorted, int* inv, void* ws,
+                                const WsLayout& L, cudaStream_t s) {
+  WsHeader* hdr = ws_at<WsHeader>(ws, L.hdr);
+  int* active = ws_at<int>(ws, L.active);
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  const int nw_perm = 8;
+  const size_t perm_smem = (size_t)(2 + nw_perm) * d.n_experts * sizeof(int);
+  if (d.hash_mode) {
+    const int blocks = ceil_div(d.T * 32, 256);
+    if (d.top_k <= 8)
+      route_hash_fused_kernel<8><<<blocks, 256, perm_smem, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts,
+                                                               d.top_k, d.vocab, ids, wts, offsets, sorted, inv,
+                                                               active, &hdr->counters[1], &hdr->err);
+    else
+      route_hash_fused_kernel<32><<<blocks, 256, perm_smem, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts,
+                                                                d.top_k, d.vocab, ids, wts, offsets, sorted, inv,
+                                                                active, &hdr->counters[1], &hdr->err);
+    MOE_CHECK_LAUNCH("route_hash_fused_kernel");
+    hook_mark(s, "route_hash_permute");
+    return MOE_OK;
+  }
+  float* logits = ws_at<float>(ws, L.logits);
+  const size_t smem = std::max((size_t)kFusedTB * d.d_model * 2, perm_smem);
+  const int blocks = ceil_div(d.n_experts, 2);
+  if (d.n_experts <= 32)
+    route_small_fused_kernel<1><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
+                                                          ids, wts, offsets, sorted, inv, active, &hdr->counters[0],
+                                                          &hdr->err);
+  else if (d.n_experts <= 256)
+    route_small_fused_kernel<8><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
+                                                          ids, wts, offsets, sorted, inv, active, &hdr->counters[0],
+                                                          &hdr->err);
+  else
+    route_small_fused_kernel<32><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
+                                                           ids, wts, offsets, sorted, inv, active, &hdr->counters[0],
+                                                           &hdr->err);
+  MOE_CHECK_LAUNCH("route_small_fused_kernel");
+  hook_mark(s, "route_topk_permute");
+  return MOE_OK;
+}
+
 moe_status_t launch_permute(const moe_dims_t& d, const int* ids, int* offsets, int* sorted, int* inv,
                             void* ws, const WsLayout& L, cudaStream_t s) {
   int* err = &ws_at<WsHeader>(ws, L.hdr)->err;
@@ -294,6 +353,25 @@ moe_status_t launch_permute(const moe_dims_t& d, const int* ids, int* offsets, i
   MOE_CHECK_LAUNCH("permute_kernel");
   hook_mark(s, "permute");
   return MOE_OK;
+}
+
+// Rows per streaming tile for a matrix in stage `stage` (mirrors SF<>::RPT),
+// or 0 when the matrix does not fit the streaming kernel's constraints:
+// n_in/32 chunks in {32, 64, 128, 256}, 16-byte multiples for every copied
+// row segment, and a tile of at most 32 KiB packed + 8 KiB scales/biases.
+int stream_rows(const QMatDev& A, int stage) {
+  const int C = A.n_in / 32;
+  if (C != 32 && C != 64 && C != 128 && C != 256) return 0;
+  const int bits = A.fmt == F_A2 ? 2 : A.fmt == F_A3 ? 3 : A.fmt == F_A8 ? 8 : 4;
+  const int rpt = (A.fmt == F_A3 ? 4 : 16 / bits) * (stage == 1 ? 1 : 2);
+  const int R = (kFfnThreads / C) * rpt;
+  const int M = stage == 1 ? 2 : 1;
+  const int row_bytes = A.wpr * 4;
+  const int sb_row = A.gpr * (A.fmt == F_MX4 ? 1 : 2);
+  if (row_bytes % 16 || sb_row % 16) return 0;
+  if (R * M * row_bytes > kStageQBytes) return 0;
+  if (R * M * sb_row * (A.fmt == F_MX4 ? 1 : 2) > kStageSBBytes) return 0;
+  return R;
 }
 
 // Stage 1 + stage 2 of the expert FFN (routed pairs, optional shared expert).
@@ -317,6 +395,63 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
   p.err = &ws_at<WsHeader>(ws, L.hdr)->err;
   p.shared_pos0 = Tk;
   p.has_shared = sh != nullptr;
+  const int r1 = stream_rows(w1, 1), r2 = stream_rows(w2, 2);
+  const int s1 = sh ? stream_rows(sh[0], 1) : 1, s2 = sh ? stream_rows(sh[2], 2) : 1;
+  if (r1 && r2 && s1 && s2) {
+    StreamParams q{};
+    q.x = p.x;
+    q.T = d.T;
+    q.k = d.top_k;
+    q.offsets = offsets;
+    q.sorted_rows = sorted;
+    q.active = p.active;
+    q.err = p.err;
+    q.shared_pos0 = Tk;
+    q.has_shared = sh != nullptr;
+    q.out = h;
+    q.ld_out = ld_h;
+    q.ra = w1;
+    q.rb = w3;
+    q.r_rows = r1;
+    if (sh) {
+      q.sa = sh[0];
+      q.sb = sh[1];
+      q.s_rows = s1;
+    } else {
+      q.s_rows = 1;
+    }
+    // tokens per expert never exceed T: size the per-pass activation registers by it
+    const int ntmax = d.T >= 4 ? 4 : d.T;
+    if (ntmax == 1)
+      ffn_stream_kernel<1, 1><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
+    else if (ntmax == 2)
+      ffn_stream_kernel<1, 2><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
+    else
+      ffn_stream_kernel<1, 4><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
+    MOE_CHECK_LAUNCH("ffn_stream_kernel<1>");
+    hook_mark(s, "ffn_w13_swiglu");
+    q.hin = h;
+    q.ld_in = ld_h;
+    q.out = y;
+    q.ld_out = ld_y;
+    q.ra = w2;
+    q.rb = w2;
+    q.r_rows = r2;
+    if (sh) {
+      q.sa = sh[2];
+      q.sb = sh[2];
+      q.s_rows = s2;
+    }
+    if (ntmax == 1)
+      ffn_stream_kernel<2, 1><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
+    else if (ntmax == 2)
+      ffn_stream_kernel<2, 2><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
+    else
+      ffn_stream_kernel<2, 4><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
+    MOE_CHECK_LAUNCH("ffn_stream_kernel<2>");
+    hook_mark(s, "ffn_w2");
+    return MOE_OK;
+  }
   // stage 1: h = silu(W1 x) * (W3 x)
   {
     FfnParams q = p;
@@ -568,11 +703,17 @@ moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t*
   hook_begin(s);
   int* ids = topk_ids_out ? topk_ids_out : ws_at<int>(ws, L.ids);
   float* wts = topk_w_out ? topk_w_out : ws_at<float>(ws, L.wts);
-  if ((st = launch_route(d, x, router_w, router_b, token_ids, tid2eid, ids, wts, ws, L, s)) != MOE_OK) return st;
   int* offsets = ws_at<int>(ws, L.offsets);
   int* sorted = ws_at<int>(ws, L.sorted);
   int* inv = ws_at<int>(ws, L.inv);
-  if ((st = launch_permute(d, ids, offsets, sorted, inv, ws, L, s)) != MOE_OK) return st;
+  if (fused_route_ok(d)) {
+    if ((st = launch_route_fused(d, x, router_w, router_b, token_ids, tid2eid, ids, wts, offsets, sorted, inv, ws,
+                                 L, s)) != MOE_OK)
+      return st;
+  } else {
+    if ((st = launch_route(d, x, router_w, router_b, token_ids, tid2eid, ids, wts, ws, L, s)) != MOE_OK) return st;
+    if ((st = launch_permute(d, ids, offsets, sorted, inv, ws, L, s)) != MOE_OK) return st;
+  }
   float* y = ws_at<float>(ws, L.y);
   if ((st = launch_ffn(d, x, offsets, sorted, q1, q3, q2, d.d_ff_shared > 0 ? qs : nullptr, y, d.d_model, ws, L,
                        s)) != MOE_OK)

@@ -13,9 +13,11 @@ namespace moe {
 
 constexpr int kPermThreads = 1024;
 
-// Block-wide exclusive scan of one int per thread (1024 threads).
+// Block-wide exclusive scan of one int per thread (any multiple of 32
+// threads up to 1024).  *total receives the block sum.
 __device__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
   int inc = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -25,14 +27,14 @@ __device__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
   if (lane == 31) warp_tot[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_tot[lane];
+    const int w = lane < nwarps ? warp_tot[lane] : 0;
     int winc = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int n = __shfl_up_sync(0xffffffffu, winc, o);
       if (lane >= o) winc += n;
     }
-    warp_tot[lane] = winc - w;  // exclusive prefix of warp totals
+    if (lane < nwarps) warp_tot[lane] = winc - w;  // exclusive prefix of warp totals
     if (lane == 31) *total = winc;
   }
   __syncthreads();
@@ -41,24 +43,21 @@ __device__ int block_exclusive_scan(int v, int* warp_tot, int* total) {
   return r;
 }
 
-// One CTA of 1024 threads.  Dynamic shared memory: (2 + 32) * E ints.
-// active[0] = number of experts with pairs, active[1..] their ids ascending.
-__global__ void __launch_bounds__(kPermThreads)
-permute_kernel(const int* __restrict__ ids, int N, int E, int* __restrict__ offsets,
-               int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
-               int* err) {
-  extern __shared__ int sm[];
+// Stable counting sort of the N expert ids by expert, by one thread block of
+// any size (multiple of 32).  sm: (2 + nwarps) * E ints of shared memory.
+__device__ void permute_block(const int* __restrict__ ids, int N, int E, int* __restrict__ offsets,
+                              int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
+                              int* err, int* sm, int* warp_tot, int* total) {
+  const int nthr = blockDim.x, nwarps = nthr >> 5;
   int* cnt = sm;            // [E] pairs per expert, later the running base
   int* off = sm + E;        // [E] exclusive offsets
-  int* wc = sm + 2 * E;     // [32][E] per-warp counts of the current tile
-  __shared__ int warp_tot[32];
-  __shared__ int total;
+  int* wc = sm + 2 * E;     // [nwarps][E] per-warp counts of the current tile
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  for (int e = tid; e < E; e += nthr) cnt[e] = 0;
   __syncthreads();
   bool bad = false;
-  for (int i = tid; i < N; i += kPermThreads) {
+  for (int i = tid; i < N; i += nthr) {
     int e = ids[i];
     if (e < 0 || e >= E) {
       bad = true;
@@ -68,16 +67,15 @@ permute_kernel(const int* __restrict__ ids, int N, int E, int* __restrict__ offs
   }
   if (bad) set_error(err, kErrDeviceInput);
   __syncthreads();
-  // exclusive scan of counts in chunks of 1024 experts
   int carry = 0, acarry = 0;
-  for (int e0 = 0; e0 < E; e0 += kPermThreads) {
+  for (int e0 = 0; e0 < E; e0 += nthr) {
     const int e = e0 + tid;
     const int c = e < E ? cnt[e] : 0;
-    const int ex = block_exclusive_scan(c, warp_tot, &total);
-    const int chunk_total = total;
+    const int ex = block_exclusive_scan(c, warp_tot, total);
+    const int chunk_total = *total;
     const int flag = c > 0 ? 1 : 0;
-    const int aex = block_exclusive_scan(flag, warp_tot, &total);
-    const int achunk = total;
+    const int aex = block_exclusive_scan(flag, warp_tot, total);
+    const int achunk = *total;
     if (e < E) {
       off[e] = carry + ex;
       offsets[e] = carry + ex;
@@ -91,12 +89,12 @@ permute_kernel(const int* __restrict__ ids, int N, int E, int* __restrict__ offs
     offsets[E] = carry;
     active[0] = acarry;
   }
-  for (int e = tid; e < E; e += kPermThreads) cnt[e] = 0;
+  for (int e = tid; e < E; e += nthr) cnt[e] = 0;
   __syncthreads();
 
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int t0 = 0; t0 < N; t0 += kPermThreads) {
-    for (int q = tid; q < 32 * E; q += kPermThreads) wc[q] = 0;
+  for (int t0 = 0; t0 < N; t0 += nthr) {
+    for (int q = tid; q < nwarps * E; q += nthr) wc[q] = 0;
     __syncthreads();
     const int i = t0 + tid;
     int e = -1;
@@ -116,13 +114,25 @@ permute_kernel(const int* __restrict__ ids, int N, int E, int* __restrict__ offs
       inv[i] = p;
     }
     __syncthreads();
-    for (int x = tid; x < E; x += kPermThreads) {
+    for (int x = tid; x < E; x += nthr) {
       int s = 0;
-      for (int w = 0; w < 32; ++w) s += wc[w * E + x];
+      for (int w = 0; w < nwarps; ++w) s += wc[w * E + x];
       cnt[x] += s;
     }
     __syncthreads();
   }
+}
+
+// One CTA of 1024 threads.  Dynamic shared memory: (2 + 32) * E ints.
+// active[0] = number of experts with pairs, active[1..] their ids ascending.
+__global__ void __launch_bounds__(kPermThreads)
+permute_kernel(const int* __restrict__ ids, int N, int E, int* __restrict__ offsets,
+               int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
+               int* err) {
+  extern __shared__ int sm[];
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  permute_block(ids, N, E, offsets, sorted_rows, inv, active, err, sm, warp_tot, &total);
 }
 
 // Active-expert list from caller-provided offsets (single CTA).

@@ -15,6 +15,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "permute.cuh"
 
 namespace moe {
 
@@ -148,19 +149,15 @@ router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
 // Expert e lives in lane e % 32, slot e / 32.
 // ---------------------------------------------------------------------------
 template <int MAXPER>
-__global__ void __launch_bounds__(256)
-topk_kernel(const float* __restrict__ L, const float* __restrict__ bias, int T, int E, int k,
-            int* __restrict__ ids, float* __restrict__ wts) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+MOE_DEV void topk_token(const float* __restrict__ Lrow, const float* __restrict__ bias, int E, int k,
+                        int* __restrict__ ids_row, float* __restrict__ w_row) {
   const int lane = threadIdx.x & 31;
-  if (warp >= T) return;
-  const int t = warp;
   float key[MAXPER], sc[MAXPER];
 #pragma unroll
   for (int i = 0; i < MAXPER; ++i) {
     const int e = i * 32 + lane;
     if (e < E) {
-      const float s = sqrt_softplus(L[(size_t)t * E + e]);
+      const float s = sqrt_softplus(__ldcg(Lrow + e));
       sc[i] = s;
       float kv = bias ? s + bias[e] : s;
       key[i] = (kv != kv) ? -INFINITY : kv;
@@ -213,9 +210,18 @@ topk_kernel(const float* __restrict__ L, const float* __restrict__ bias, int T, 
     }
   }
   if (lane < k) {
-    ids[(size_t)t * k + lane] = my_id;
-    wts[(size_t)t * k + lane] = ssum > 0.f ? my_s / ssum : 1.f / (float)k;
+    ids_row[lane] = my_id;
+    w_row[lane] = ssum > 0.f ? my_s / ssum : 1.f / (float)k;
   }
+}
+
+template <int MAXPER>
+__global__ void __launch_bounds__(256)
+topk_kernel(const float* __restrict__ L, const float* __restrict__ bias, int T, int E, int k,
+            int* __restrict__ ids, float* __restrict__ wts) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= T) return;
+  topk_token<MAXPER>(L + (size_t)warp * E, bias, E, k, ids + (size_t)warp * k, wts + (size_t)warp * k);
 }
 
 // ---------------------------------------------------------------------------
@@ -223,10 +229,9 @@ topk_kernel(const float* __restrict__ L, const float* __restrict__ bias, int T, 
 // the error word and routed to expert 0 with weight 0.
 // ---------------------------------------------------------------------------
 template <int KMAX>
-__global__ void __launch_bounds__(256)
-route_hash_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
-                  const int* __restrict__ token_ids, const int* __restrict__ table, int T, int d, int E,
-                  int k, int vocab, int* __restrict__ ids, float* __restrict__ wts, int* err) {
+MOE_DEV void route_hash_warp(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                             const int* __restrict__ token_ids, const int* __restrict__ table, int T, int d, int E,
+                             int k, int vocab, int* __restrict__ ids, float* __restrict__ wts, int* err) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= T) return;
@@ -288,6 +293,133 @@ route_hash_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__
       wts[(size_t)t * k + j] = w;
     }
   }
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(256)
+route_hash_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                  const int* __restrict__ token_ids, const int* __restrict__ table, int T, int d, int E,
+                  int k, int vocab, int* __restrict__ ids, float* __restrict__ wts, int* err) {
+  route_hash_warp<KMAX>(x, W, token_ids, table, T, d, E, k, vocab, ids, wts, err);
+}
+
+// ---------------------------------------------------------------------------
+// Small-T fused routing: logits, top-k, renormalisation and the stable
+// permutation in one launch.  Every block computes the logits of two experts
+// (four warps per expert, each over a quarter of d_model) for all tokens; the
+// last block to finish (arrival counter in the workspace, reset afterwards)
+// selects the experts of every token and groups the pairs by expert.
+// ---------------------------------------------------------------------------
+constexpr int kFusedTB = 8;            // tokens per pass over the staged x rows
+constexpr int kFusedMaxT = 32;
+
+template <int MAXPER>
+__global__ void __launch_bounds__(256)
+route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                         const float* __restrict__ bias, int T, int d, int E, int k, float* __restrict__ L,
+                         int* __restrict__ ids, float* __restrict__ wts, int* __restrict__ offsets,
+                         int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
+                         int* counter, int* err) {
+  extern __shared__ __align__(16) uint32_t sm_raw[];
+  __shared__ float part[8][kFusedTB];
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ int is_last;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int e = blockIdx.x * 2 + (warp >> 2);
+  const int quarter = warp & 3;
+  const int q4 = d >> 4;  // float4 per quarter row
+  // this warp's quarter row of the router weight, kept in registers
+  float4 wv[8];
+  const bool live = e < E;
+  {
+    const float4* wr = reinterpret_cast<const float4*>(W + (size_t)min(e, E - 1) * d) + quarter * q4;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = lane + 32 * u;
+      wv[u] = (live && i < q4) ? __ldg(wr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  for (int t0 = 0; t0 < T; t0 += kFusedTB) {
+    const int nt = min(kFusedTB, T - t0);
+    __syncthreads();
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t0 * d);
+      uint4* dst = reinterpret_cast<uint4*>(sm_raw);
+      for (int i = tid; i < nt * d / 8; i += blockDim.x) dst[i] = src[i];
+    }
+    __syncthreads();
+    float acc[kFusedTB];
+#pragma unroll
+    for (int t = 0; t < kFusedTB; ++t) acc[t] = 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = lane + 32 * u;
+      if (i < q4) {
+#pragma unroll
+        for (int t = 0; t < kFusedTB; ++t) {
+          if (t < nt) {
+            const uint2 xv = reinterpret_cast<const uint2*>(sm_raw + (size_t)t * (d >> 1))[quarter * q4 + i];
+            acc[t] = fmaf(wv[u].x, bf16lo(xv.x), acc[t]);
+            acc[t] = fmaf(wv[u].y, bf16hi(xv.x), acc[t]);
+            acc[t] = fmaf(wv[u].z, bf16lo(xv.y), acc[t]);
+            acc[t] = fmaf(wv[u].w, bf16hi(xv.y), acc[t]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kFusedTB; ++t) {
+      const float v = warp_sum(acc[t]);
+      if (lane == 0) part[warp][t] = v;
+    }
+    __syncthreads();
+    if (tid < 2 * kFusedTB) {
+      const int h = tid / kFusedTB, t = tid % kFusedTB;
+      const int ee = blockIdx.x * 2 + h;
+      if (ee < E && t < nt)
+        L[(size_t)(t0 + t) * E + ee] = part[4 * h][t] + part[4 * h + 1][t] + part[4 * h + 2][t] + part[4 * h + 3][t];
+    }
+  }
+  // publish this block's logits, then count arrivals
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  for (int t = warp; t < T; t += 8)
+    topk_token<MAXPER>(L + (size_t)t * E, bias, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
+  __threadfence_block();
+  __syncthreads();
+  permute_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, reinterpret_cast<int*>(sm_raw), warp_tot,
+                &total);
+  if (tid == 0) *counter = 0;
+}
+
+// Hash routing plus permutation, one launch: one warp per token, the last
+// block groups the pairs by expert.
+template <int KMAX>
+__global__ void __launch_bounds__(256)
+route_hash_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                        const int* __restrict__ token_ids, const int* __restrict__ table, int T, int d, int E,
+                        int k, int vocab, int* __restrict__ ids, float* __restrict__ wts, int* __restrict__ offsets,
+                        int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
+                        int* counter, int* err) {
+  extern __shared__ __align__(16) uint32_t sm_raw[];
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  __shared__ int is_last;
+  route_hash_warp<KMAX>(x, W, token_ids, table, T, d, E, k, vocab, ids, wts, err);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  permute_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, reinterpret_cast<int*>(sm_raw), warp_tot,
+                &total);
+  if (threadIdx.x == 0) *counter = 0;
 }
 
 }  // namespace moe

@@ -32,6 +32,19 @@ VARIANTS = {
     "odd_chunks": dict(SMALL, d=96, f=160, T=13, w13=("affine", 4, 32), w2=("affine", 4, 32), seed=112),
     "many_tokens": dict(SMALL, T=300, E=8, k=2, d=256, f=128, seed=113),
     "k1_E1": dict(SMALL, T=5, E=1, k=1, seed=114),
+    # widths of 1024+ inputs take the bulk-copy streaming GEMV
+    "stream_a4g64_T37": dict(SMALL, d=1024, f=1024, seed=120),
+    "stream_a4g64_T5": dict(SMALL, d=1024, f=1024, T=5, seed=121),
+    "stream_T1_shared8": dict(SMALL, d=1024, f=1024, T=1, shared=("affine", 8, 64), f_shared=1024, seed=122),
+    "stream_T2_a2g128_a3g128": dict(SMALL, d=1024, f=1024, T=2, w13=("affine", 2, 128), w2=("affine", 3, 128),
+                                    seed=123),
+    "stream_a8g64_T12": dict(SMALL, d=1024, f=2048, T=12, w13=("affine", 8, 64), w2=("affine", 8, 64), seed=124),
+    "stream_hash_mxfp4": dict(SMALL, d=2048, f=1024, T=20, routing="hash", vocab=500, w13=("mxfp4", 4, 32),
+                              w2=("mxfp4", 4, 32), seed=125),
+    "stream_shared_wider": dict(SMALL, d=2048, f=1024, T=9, shared=("affine", 8, 128), f_shared=2048, seed=126),
+    "stream_a4g32": dict(SMALL, d=1024, f=1024, T=3, w13=("affine", 4, 32), w2=("affine", 4, 32), seed=127),
+    "stream_a2g64_a3g64": dict(SMALL, d=1024, f=1024, T=7, w13=("affine", 2, 64), w2=("affine", 3, 64), seed=128),
+    "stream_many_per_expert": dict(SMALL, d=1024, f=1024, T=40, E=4, k=2, seed=129),
 }
 
 
