@@ -302,8 +302,6 @@ def ours_arm(args):
     work, flops, n_act, weight_bytes = kernel_work(inp, ids.cpu().numpy())
 
     # ---- timed region: K forwards, L2 flushed between them (outside the events)
-    n_ev = 16
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     props = torch.cuda.get_device_properties(dev)
@@ -313,30 +311,40 @@ def ours_arm(args):
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.2)
-    keep = []
     for s in range(args.steps):
         flush.fill_(s & 0xFF)
         step_ev[s][0].record(stream)
-        keep.append(moe.set_timing_events(evs[s]))
         fwd()
         step_ev[s][1].record(stream)
     torch.cuda.synchronize()
-    labels = moe.timing_labels()
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    total_ms = sum(step_ms)
-    per_kernel = {}
-    for s in range(args.steps):
-        for i, lab in enumerate(labels):
-            per_kernel.setdefault(lab, []).append(evs[s][i].elapsed_time(evs[s][i + 1]))
-    kern_ms = {lab: statistics.mean(v) for lab, v in per_kernel.items()}
-    ms_per_step = total_ms / args.steps
+    ms_per_step = sum(step_ms) / args.steps
     if world > 1:
         t = torch.tensor([ms_per_step], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_per_step = float(t.item())
+
+    # ---- per-kernel durations: a second timed pass with CUDA events recorded
+    # by the library between its kernels on the same stream (the events add
+    # small gaps between kernels, so the step time above is taken without them)
+    k_steps = min(args.steps, 200)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(16)] for _ in range(k_steps)]
+    keep = []
+    torch.cuda.synchronize()
+    for s in range(k_steps):
+        flush.fill_(s & 0xFF)
+        keep.append(moe.set_timing_events(evs[s]))
+        fwd()
+    torch.cuda.synchronize()
+    labels = moe.timing_labels()
+    per_kernel = {}
+    for s in range(k_steps):
+        for i, lab in enumerate(labels):
+            per_kernel.setdefault(lab, []).append(evs[s][i].elapsed_time(evs[s][i + 1]))
+    kern_ms = {lab: statistics.mean(v) for lab, v in per_kernel.items()}
 
     # ---- end-to-end through the C ABI with host buffers (pinned), copies inside
     x_h = inp.x.cpu().pin_memory()
@@ -396,6 +404,7 @@ def ours_arm(args):
         "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": len(labels) * args.steps,
+        "kernel_timing_steps": k_steps,
         "clocks": clocks,
         "device_error": err,
     }

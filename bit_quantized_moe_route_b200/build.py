@@ -16,8 +16,8 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe_lowbit.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2",
-         "-shared", "-cudart", "static"]
+FLAGS = ["-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC,-O2"]
+OBJDIR = os.path.join(PKG, "_build")
 
 
 def nvcc() -> str:
@@ -32,8 +32,8 @@ def sources():
 
 
 def inputs():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [
-        os.path.join(ROOT, "include", "moe_lowbit.h")]
+    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + sorted(
+        glob.glob(os.path.join(CSRC, "*.inl"))) + [os.path.join(ROOT, "include", "moe_lowbit.h")]
 
 
 def up_to_date() -> bool:
@@ -43,13 +43,37 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in inputs())
 
 
+def _compile(src: str, verbose: bool) -> str:
+    obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+    cmd = [nvcc(), *ARCH, *FLAGS, "-I", os.path.join(ROOT, "include"), "-c", "-o", obj, src]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    subprocess.run(cmd, check=True)
+    return obj
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile every translation unit (in parallel) and link libmoe_lowbit.so."""
     if not force and up_to_date():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+    os.makedirs(OBJDIR, exist_ok=True)
+    srcs = sources()
+    headers = [p for p in inputs() if not p.endswith(".cu")]
+    newest_header = max(os.path.getmtime(p) for p in headers)
+    todo = []
+    for src in srcs:
+        obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
+        if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), newest_header):
+            todo.append(src)
+    workers = max(1, min(len(todo), os.cpu_count() or 1))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        list(ex.map(lambda s_: _compile(s_, verbose), todo))
+    objs = [os.path.join(OBJDIR, os.path.basename(s_) + ".o") for s_ in srcs]
     tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, *FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp, *sources()]
+    cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     if verbose:
-        print(" ".join(cmd))
+        print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
     return LIB

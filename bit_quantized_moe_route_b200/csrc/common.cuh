@@ -22,6 +22,18 @@ struct WsHeader {
   int counters[60];
 };
 
+// One stacked packed matrix as the kernels see it.
+struct QMatDev {
+  const uint32_t* q;
+  const void* scales;
+  const void* biases;
+  int fmt;    // FmtCode
+  int group;  // elements per scale group
+  int n_out, n_in;
+  int wpr;    // uint32 words per row
+  int gpr;    // scale groups per row
+};
+
 MOE_DEV void set_error(int* err, int code) { atomicCAS(err, 0, code); }
 
 MOE_DEV float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
@@ -60,5 +72,9 @@ MOE_DEV float sqrt_softplus(float x) {
 }
 
 MOE_DEV float silu(float a) { return a / (1.f + expf(-a)); }
+
+MOE_DEV float magic_u2f(uint32_t q) {  // exact for q < 2^23
+  return __uint_as_float(0x4B000000u | q) - 8388608.f;
+}
 
 }  // namespace moe

@@ -26,16 +26,7 @@
 
 namespace moe {
 
-struct QMatDev {
-  const uint32_t* q;
-  const void* scales;
-  const void* biases;
-  int fmt;    // FmtCode
-  int group;  // elements per scale group
-  int n_out, n_in;
-  int wpr;    // uint32 words per row
-  int gpr;    // scale groups per row
-};
+
 
 struct FfnParams {
   const __nv_bfloat16* x;  // stage 1 input [T, d]
@@ -59,9 +50,6 @@ constexpr int kFfnThreads = 256;
 constexpr int kFfnNT = 2;        // tokens per pass (x chunk held in registers)
 constexpr int kRed = 4096;       // floats of reduction scratch
 
-MOE_DEV float magic_u2f(uint32_t q) {  // exact for q < 2^23
-  return __uint_as_float(0x4B000000u | q) - 8388608.f;
-}
 
 // e2m1 code -> value (sign | exponent(2) | mantissa(1), exponent bias 1).
 MOE_DEV float e2m1_to_f(uint32_t c) {

@@ -1,8 +1,8 @@
 // Step 3 for small token counts, streaming version: the grouped SwiGLU expert
 // FFN as a weight-streaming GEMV whose packed rows flow HBM -> shared memory
 // through a ring of bulk asynchronous copies (cp.async.bulk + mbarrier
-// transaction counts), fed by one producer warp, while eight consumer warps
-// dequantise in registers and reduce.
+// transaction counts) issued by one producer warp, while eight consumer warps
+// dequantise in registers.
 //
 //   stage 1:  h[p] = silu(W1[e] . x[t]) * (W3[e] . x[t])
 //   stage 2:  y[p] = W2[e] . h[p]
@@ -11,26 +11,58 @@
 // gate/down/up; model card "DeepSeek-V4-Flash-0731-MLX-Serve-mixed-2-3-8bit":
 // affine packs w = scale*q + bias, mxfp4 = e2m1 codes with e8m0 group scales.]
 //
-// Arithmetic.  A thread owns one 32-input chunk of every row it touches.  Per
-// chunk and token the activations are held as a 16-bit fixed-point vector
-// xq = rint(x * 2^(141-Emax)) (Emax: largest fp32 exponent field in the
-// chunk; |xq| < 2^15), split into a signed high byte and an unsigned low byte
-// so that sum(q_i * xq_i) = 256*dp4a(q, hi) + dp4a(q, lo) is an exact int32.
-// A bf16 x within 2^6 of the chunk's largest magnitude converts exactly; the
-// error of smaller ones is below 2^-16 of the chunk maximum.  Per chunk:
+// Work split.  A persistent block per SM walks a contiguous range of tiles
+// (expert, block of R rows).  The eight consumer warps form groups of WPR
+// warps; a group owns R/G whole rows of each tile (G = 8/WPR groups) and
+// each of its lanes owns CPL 32-input chunks of every such row, so a row's
+// dot product is finished by one warp reduction (plus a small shared-memory
+// sum when WPR > 1) -- no block-wide barrier per tile.
+//
+// Arithmetic.  Per chunk and token the activations are held as a 16-bit
+// fixed-point vector xq = rint(x * 2^(141-Emax)) (Emax: largest fp32 exponent
+// field in the chunk; |xq| < 2^15), split into a signed high byte and an
+// unsigned low byte so that sum(q_i * xq_i) = 256*dp4a(q, hi) + dp4a(q, lo)
+// is an exact int32.  A bf16 x within 2^6 of the chunk's largest magnitude
+// converts exactly; the error of smaller ones is below 2^-16 of the chunk
+// maximum.  Per chunk:
 //   affine: s * 2^(Emax-141) * sum(q*xq) + b * 2^(Emax-141) * sum(xq)
 //   mxfp4 : 2^(e-128) * 2^(Emax-141) * sum(2*e2m1(c) * xq)
-// accumulated in fp32.  3-bit codes (which do not split into bytes cheaply)
-// keep fp32 activations and exact float codes instead.
+// accumulated in fp32.  3-bit codes reach byte lanes through two
+// multiply-and-mask spreads per four codes.
 #pragma once
 
-#include "common.cuh"
-#include "ffn_gemv.cuh"
+#include "stream_types.cuh"
 
 namespace moe {
 
 // ------------------------------------------------------------ async proxy
 MOE_DEV uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+MOE_DEV uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+MOE_DEV uint2 lds64(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+MOE_DEV uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+MOE_DEV uint32_t lds16(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+MOE_DEV uint32_t lds8(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
 
 MOE_DEV void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -74,7 +106,7 @@ MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
   return true;
 }
 
-MOE_DEV void consumer_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+MOE_DEV void group_bar(int id, int nthreads) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory"); }
 
 // ------------------------------------------------------------ integer dot
 MOE_DEV int dp4a_us(uint32_t a_u8, uint32_t b_s8, int c) {  // unsigned a bytes x signed b bytes
@@ -98,154 +130,169 @@ MOE_DEV int dp4a_su(uint32_t a_s8, uint32_t b_u8, int c) {
   return d;
 }
 
-// ------------------------------------------------------------ formats
-// Per format: rows per thread per tile (keeps a tile's packed words at
-// <= 32 KiB), tokens per pass, and the order in which a chunk's inputs meet
-// the dp4a byte lanes (plane word w, byte lane l -> input index).
-template <int FMT, int STAGE, int NTMAX>
+// Per format: how a chunk's 32 inputs meet the dp4a byte lanes (plane word
+// w, byte lane l -> input index), and how many tokens one pass carries.
+template <int FMT, int NTMAX>
 struct SF {
-  static constexpr int M = STAGE == 1 ? 2 : 1;
   static constexpr int bits = FMT == F_A2 ? 2 : FMT == F_A3 ? 3 : FMT == F_A8 ? 8 : 4;
-  static constexpr int RPT = (FMT == F_A3 ? 4 : 16 / bits) * (STAGE == 1 ? 1 : 2);
-  static constexpr bool kInt = FMT != F_A3;
-  static constexpr int NTc = 32 / (RPT * M);
-  static constexpr int NTi = NTc > 4 ? 4 : NTc;
-  static constexpr int NTf = kInt ? NTi : 2;
-  static constexpr int NT = NTf < NTMAX ? NTf : NTMAX;  // tokens per pass
-  static constexpr int V = RPT * M * NT;
-  // input index fed to plane word w (0..7), byte lane l (0..3)
+  static constexpr int NT = NTMAX;
+  static constexpr int kChunkBytes = bits * 4;
   static MOE_DEV constexpr int order(int w, int l) {
     if constexpr (FMT == F_A4) return 8 * (w >> 1) + 2 * l + (w & 1);  // even/odd nibbles of each word
     if constexpr (FMT == F_A2) return 16 * (w >> 2) + 4 * l + (w & 3);  // 2-bit fields by shift
-    return 4 * w + l;                                                   // bytes in natural order (A8, MX4)
+    return 4 * w + l;                                                   // natural order (A8, A3, MX4)
   }
 };
 
-constexpr int kStages = 4;
-constexpr int kStageQBytes = 32 * 1024;
-constexpr int kStageSBBytes = 8 * 1024;
-constexpr int kStageBytes = kStageQBytes + kStageSBBytes;
-constexpr int kConsumerWarps = 8;
-constexpr int kStreamThreads = kConsumerWarps * 32;
-constexpr int kRedFloats = 2 * kConsumerWarps * 32;
-constexpr size_t kStreamSmem = (size_t)kStages * kStageBytes + kRedFloats * 4 + kStages * 8 + 16;
 
-// register words holding one pass's activations
-template <int NTMAX>
-struct XWords {
-  static constexpr int n = (16 * NTMAX > 32 * (NTMAX < 2 ? NTMAX : 2)) ? 16 * NTMAX : 32 * (NTMAX < 2 ? NTMAX : 2);
-};
 
-struct StreamParams {
-  const __nv_bfloat16* x;  // stage 1 input [T, d]
-  const float* hin;        // stage 2 input rows [P, ld_in]
-  float* out;              // stage 1: h; stage 2: y
-  int ld_in, ld_out;
-  int T, k;
-  QMatDev ra, rb;          // routed (stage 1: w1, w3; stage 2: w2)
-  const int* offsets;
-  const int* sorted_rows;
-  const int* active;       // [0] = n, [1..] expert ids
-  int has_shared;
-  QMatDev sa, sb;
-  int shared_pos0;         // = T*k
-  int r_rows, s_rows;      // rows per tile: routed, shared
-  int* err;
+// Incremental walk over the block's tile range: shared-expert tiles first,
+// then the tiles of each active routed expert.  The routed expert's id and
+// position range are read from global memory once per expert, not per tile.
+struct Walker {
+  long long g, g1;
+  int n_sh, tpe, a, rb;
+  int e, pos0, npos;
+  MOE_DEV void load_seg(const StreamParams& p) {
+    if (a >= 0) {
+      e = __ldcg(p.active + 1 + a);
+      pos0 = __ldcg(p.offsets + e);
+      npos = __ldcg(p.offsets + e + 1) - pos0;
+    } else {
+      e = 0;
+      pos0 = p.shared_pos0;
+      npos = p.T;
+    }
+  }
+  MOE_DEV void start(const StreamParams& p, long long g0, long long g_end, int n_sh_, int tpe_) {
+    g = g0;
+    g1 = g_end;
+    n_sh = n_sh_;
+    tpe = tpe_;
+    if (g0 < n_sh) {
+      a = -1;
+      rb = (int)g0;
+    } else {
+      const long long h = g0 - n_sh;
+      a = (int)(h / tpe);
+      rb = (int)(h - (long long)a * tpe);
+    }
+    load_seg(p);
+  }
+  MOE_DEV void next(const StreamParams& p) {
+    ++g;
+    ++rb;
+    if (a < 0) {
+      if (rb >= n_sh) {
+        a = 0;
+        rb = 0;
+        if (g < g1) load_seg(p);
+      }
+    } else if (rb >= tpe) {
+      ++a;
+      rb = 0;
+      if (g < g1) load_seg(p);
+    }
+  }
 };
 
 struct Tile {
   const QMatDev* A;
   const QMatDev* B;
-  int e, r0, rows, R, pos0, npos, seg;  // seg: -1 shared, else active index
+  int e, r0, rows, R, wpr, pos0, npos, seg;  // seg: -1 shared, else active index
 };
 
-MOE_DEV Tile tile_at(const StreamParams& p, long long g, int n_sh, int tpe) {
+MOE_DEV Tile tile_of(const StreamParams& p, const Walker& w) {
   Tile t;
-  if (g < n_sh) {
-    t.A = &p.sa;
-    t.B = &p.sb;
-    t.e = 0;
-    t.R = p.s_rows;
-    t.r0 = (int)g * t.R;
-    t.pos0 = p.shared_pos0;
-    t.npos = p.T;
-    t.seg = -1;
-  } else {
-    const long long h = g - n_sh;
-    const int a = (int)(h / tpe);
-    t.A = &p.ra;
-    t.B = &p.rb;
-    t.e = __ldcg(p.active + 1 + a);
-    t.R = p.r_rows;
-    t.r0 = (int)(h - (long long)a * tpe) * t.R;
-    t.pos0 = __ldcg(p.offsets + t.e);
-    t.npos = __ldcg(p.offsets + t.e + 1) - t.pos0;
-    t.seg = a;
-  }
+  const bool sh = w.a < 0;
+  t.A = sh ? &p.sa : &p.ra;
+  t.B = sh ? &p.sb : &p.rb;
+  t.R = sh ? p.s_rows : p.r_rows;
+  t.wpr = sh ? p.s_wpr : p.r_wpr;
+  t.e = w.e;
+  t.pos0 = w.pos0;
+  t.npos = w.npos;
+  t.seg = w.a;
+  t.r0 = w.rb * t.R;
   t.rows = min(t.R, t.A->n_out - t.r0);
   return t;
 }
 
-// Byte offsets of a tile's regions inside a stage buffer.
+// Byte offsets of a tile's regions inside a stage buffer: packed rows of
+// each matrix, then scales (and biases) of each matrix.
 struct StageLayout {
   int q[2], s[2], b[2], total;
 };
 MOE_DEV StageLayout stage_layout(const QMatDev& A, int R, int M, int rows) {
   StageLayout L;
   const int row_bytes = A.wpr * 4;
-  const int ssz = A.fmt == F_MX4 ? 1 : 2;
-  const int sb_row = A.gpr * ssz;
+  const bool mx = A.fmt == F_MX4;
+  const int sb_row = A.gpr * (mx ? 1 : 2);
+  const int per_m = R * sb_row * (mx ? 1 : 2);
   for (int m = 0; m < 2; ++m) {
     L.q[m] = m * R * row_bytes;
-    L.s[m] = kStageQBytes + m * R * sb_row * (A.fmt == F_MX4 ? 1 : 2);
+    L.s[m] = M * R * row_bytes + m * per_m;
     L.b[m] = L.s[m] + R * sb_row;
   }
-  L.total = M * rows * (row_bytes + sb_row * (A.fmt == F_MX4 ? 1 : 2));
+  L.total = M * rows * (row_bytes + sb_row * (mx ? 1 : 2));
   return L;
 }
 
 // ------------------------------------------------------------ activations
-// Per-token chunk state: 8 high-byte and 8 low-byte plane words (integer
-// formats) or 32 fp32 values (3-bit), plus the fixed-point scale and sum.
-template <int FMT, int STAGE, int NTMAX>
-MOE_DEV void load_x(const StreamParams& p, const Tile& t, int tb, int nt, int c, uint32_t (&xw)[XWords<NTMAX>::n],
-                    float (&xs)[NTMAX], float (&xsum)[NTMAX]) {
-  using F = SF<FMT, STAGE, NTMAX>;
+// Activations of one pass for this lane's CPL chunks: 8 high-byte and 8
+// low-byte plane words per (chunk, token), plus the fixed-point scale and
+// the scaled chunk sum.
+template <int NTMAX, int CPL>
+struct XRegs {
+  static constexpr int kWords = 16 * NTMAX * CPL;
+  uint32_t w[kWords];
+  float xs[CPL][NTMAX];
+  float xsum[CPL][NTMAX];
+};
+
+template <int FMT, int STAGE, int NTMAX, int CPL>
+MOE_DEV void load_x(const StreamParams& p, const Tile& t, int tb, int nt, int cbase, XRegs<NTMAX, CPL>& X) {
+  using F = SF<FMT, NTMAX>;
+  const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int j = 0; j < F::NT; ++j) {
-    float v[32];
-    if (j < nt) {
-      if constexpr (STAGE == 1) {
-        const int tok = t.seg < 0 ? (tb + j) : (__ldcg(p.sorted_rows + t.pos0 + tb + j) / p.k);
-        const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)tok * t.A->n_in + c * 32);
+    int tok = 0;
+    if (STAGE == 1 && j < nt) tok = t.seg < 0 ? (tb + j) : (__ldcg(p.sorted_rows + t.pos0 + tb + j) / p.k);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 u = __ldcg(src + q);
-          v[8 * q + 0] = bf16lo(u.x); v[8 * q + 1] = bf16hi(u.x);
-          v[8 * q + 2] = bf16lo(u.y); v[8 * q + 3] = bf16hi(u.y);
-          v[8 * q + 4] = bf16lo(u.z); v[8 * q + 5] = bf16hi(u.z);
-          v[8 * q + 6] = bf16lo(u.w); v[8 * q + 7] = bf16hi(u.w);
+    for (int cc = 0; cc < CPL; ++cc) {
+      const int c = cbase + 32 * cc + lane;
+      float v[32];
+      if (j < nt) {
+        if constexpr (STAGE == 1) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.x + (size_t)tok * t.A->n_in + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 u = __ldcg(src + q);
+            v[8 * q + 0] = bf16lo(u.x); v[8 * q + 1] = bf16hi(u.x);
+            v[8 * q + 2] = bf16lo(u.y); v[8 * q + 3] = bf16hi(u.y);
+            v[8 * q + 4] = bf16lo(u.z); v[8 * q + 5] = bf16hi(u.z);
+            v[8 * q + 6] = bf16lo(u.w); v[8 * q + 7] = bf16hi(u.w);
+          }
+        } else {
+          const float4* src =
+              reinterpret_cast<const float4*>(p.hin + (size_t)(t.pos0 + tb + j) * p.ld_in + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 u = __ldcg(src + q);
+            v[4 * q + 0] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
+          }
         }
       } else {
-        const float4* src = reinterpret_cast<const float4*>(p.hin + (size_t)(t.pos0 + tb + j) * p.ld_in + c * 32);
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 u = __ldcg(src + q);
-          v[4 * q + 0] = u.x; v[4 * q + 1] = u.y; v[4 * q + 2] = u.z; v[4 * q + 3] = u.w;
-        }
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = 0.f;
-    }
-    if constexpr (F::kInt) {
       uint32_t emax = 0;
 #pragma unroll
       for (int i = 0; i < 32; ++i) emax = max(emax, (__float_as_uint(v[i]) >> 23) & 0xFFu);
       float scale = 0.f, inv = 0.f;
       if (emax >= 14 && emax < 255) {
-        scale = __uint_as_float((268u - emax) << 23);   // 2^(141 - emax)
-        inv = __uint_as_float((emax - 14u) << 23);      // 2^(emax - 141)
+        scale = __uint_as_float((268u - emax) << 23);  // 2^(141 - emax)
+        inv = __uint_as_float((emax - 14u) << 23);     // 2^(emax - 141)
       }
       int q[32];
       int sum = 0;
@@ -263,142 +310,127 @@ MOE_DEV void load_x(const StreamParams& p, const Tile& t, int tb, int nt, int c,
           hi |= (uint32_t)((qi >> 8) & 0xFF) << (8 * l);
           lo |= (uint32_t)(qi & 0xFF) << (8 * l);
         }
-        xw[16 * j + w] = hi;
-        xw[16 * j + 8 + w] = lo;
+        X.w[(j * CPL + cc) * 16 + w] = hi;
+        X.w[(j * CPL + cc) * 16 + 8 + w] = lo;
       }
-      xs[j] = inv;
-      xsum[j] = inv * (float)sum;
-    } else {
-      float sum = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        xw[32 * j + i] = __float_as_uint(v[i]);
-        sum += v[i];
-      }
-      xs[j] = 1.f;
-      xsum[j] = sum;
+      X.xs[cc][j] = inv;
+      X.xsum[cc][j] = inv * (float)sum;
+      // keep one chunk's raw activations live at a time (register pressure)
+      asm volatile("" ::: "memory");
     }
   }
 }
 
 // ------------------------------------------------------------ chunk dots
-// acc[j] += contribution of one chunk (row of a matrix) for tokens j < nt.
-template <int FMT, int STAGE, int NTMAX>
-MOE_DEV void chunk_dot_s(const uint8_t* qs, float sc, float bi, const uint32_t (&xw)[XWords<NTMAX>::n],
-                         const float (&xs)[NTMAX], const float (&xsum)[NTMAX], int nt, float* acc) {
-  using F = SF<FMT, STAGE, NTMAX>;
+// Packed words of one 32-input chunk (as many as the format needs).
+struct ChunkWords {
+  uint32_t w[8];
+};
+
+template <int FMT>
+MOE_DEV ChunkWords load_chunk(uint32_t a) {
+  ChunkWords c;
+  if constexpr (FMT == F_A8) {
+    const uint4 x = lds128(a), y = lds128(a + 16);
+    c.w[0] = x.x; c.w[1] = x.y; c.w[2] = x.z; c.w[3] = x.w;
+    c.w[4] = y.x; c.w[5] = y.y; c.w[6] = y.z; c.w[7] = y.w;
+  } else if constexpr (FMT == F_A2) {
+    const uint2 x = lds64(a);
+    c.w[0] = x.x; c.w[1] = x.y;
+  } else if constexpr (FMT == F_A3) {
+    c.w[0] = lds32(a); c.w[1] = lds32(a + 4); c.w[2] = lds32(a + 8);
+  } else {
+    const uint4 x = lds128(a);
+    c.w[0] = x.x; c.w[1] = x.y; c.w[2] = x.z; c.w[3] = x.w;
+  }
+  return c;
+}
+
+// acc[j] += one chunk's contribution for tokens j < nt (all NT when FULL);
+// chunk slot cc selects this lane's activation words.
+template <int FMT, int NTMAX, int CPL, bool FULL>
+MOE_DEV void chunk_dot_s(const ChunkWords& cw, float sc, float bi, const XRegs<NTMAX, CPL>& X, int cc, int nt,
+                         float (&acc)[NTMAX]) {
+  using F = SF<FMT, NTMAX>;
+  uint32_t b8[8];
   if constexpr (FMT == F_A4) {
-    const uint4 w4 = *reinterpret_cast<const uint4*>(qs);
-    const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
-    uint32_t b8[8];
+    // even nibbles masked into bytes; odd nibbles masked in place (16 * q)
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      b8[2 * k] = wd[k] & 0x0F0F0F0Fu;
-      b8[2 * k + 1] = (wd[k] >> 4) & 0x0F0F0F0Fu;
-    }
-#pragma unroll
-    for (int j = 0; j < F::NT; ++j) {
-      if (j < nt) {
-        int ph = 0, pl = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          ph = dp4a_us(b8[w], xw[16 * j + w], ph);
-          pl = dp4a_uu(b8[w], xw[16 * j + 8 + w], pl);
-        }
-        const float P = (float)(ph * 256 + pl);
-        acc[j] = fmaf(sc, P * xs[j], fmaf(bi, xsum[j], acc[j]));
-      }
+      b8[2 * k] = cw.w[k] & 0x0F0F0F0Fu;
+      b8[2 * k + 1] = cw.w[k] & 0xF0F0F0F0u;
     }
   } else if constexpr (FMT == F_A8) {
-    const uint4 a4 = *reinterpret_cast<const uint4*>(qs);
-    const uint4 c4 = *reinterpret_cast<const uint4*>(qs + 16);
-    const uint32_t b8[8] = {a4.x, a4.y, a4.z, a4.w, c4.x, c4.y, c4.z, c4.w};
 #pragma unroll
-    for (int j = 0; j < F::NT; ++j) {
-      if (j < nt) {
-        int ph = 0, pl = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          ph = dp4a_us(b8[w], xw[16 * j + w], ph);
-          pl = dp4a_uu(b8[w], xw[16 * j + 8 + w], pl);
-        }
-        const float P = (float)(ph * 256 + pl);
-        acc[j] = fmaf(sc, P * xs[j], fmaf(bi, xsum[j], acc[j]));
-      }
-    }
+    for (int k = 0; k < 8; ++k) b8[k] = cw.w[k];
   } else if constexpr (FMT == F_A2) {
-    const uint2 w2 = *reinterpret_cast<const uint2*>(qs);
-    const uint32_t wd[2] = {w2.x, w2.y};
-    uint32_t b8[8];
 #pragma unroll
     for (int k = 0; k < 2; ++k)
 #pragma unroll
-      for (int s = 0; s < 4; ++s) b8[4 * k + s] = (wd[k] >> (2 * s)) & 0x03030303u;
+      for (int s = 0; s < 4; ++s) b8[4 * k + s] = (cw.w[k] >> (2 * s)) & 0x03030303u;
+  } else if constexpr (FMT == F_A3) {
+    // 32 codes in 96 bits; plane word w holds codes 4w..4w+3 = stream bits
+    // [12w, 12w+12).  Two multiply-and-mask spreads move the four 3-bit
+    // fields to byte lanes (the shifted copies never overlap, so no carries).
+    const uint32_t w0 = cw.w[0], w1 = cw.w[1], w2 = cw.w[2];
+    const uint32_t tw[8] = {w0, w0 >> 12, __funnelshift_r(w0, w1, 24), w1 >> 4,
+                            w1 >> 16, __funnelshift_r(w1, w2, 28), w2 >> 8, w2 >> 20};
 #pragma unroll
-    for (int j = 0; j < F::NT; ++j) {
-      if (j < nt) {
-        int ph = 0, pl = 0;
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          ph = dp4a_us(b8[w], xw[16 * j + w], ph);
-          pl = dp4a_uu(b8[w], xw[16 * j + 8 + w], pl);
-        }
-        const float P = (float)(ph * 256 + pl);
-        acc[j] = fmaf(sc, P * xs[j], fmaf(bi, xsum[j], acc[j]));
-      }
+    for (int w = 0; w < 8; ++w) {
+      const uint32_t t = tw[w];
+      const uint32_t ev = ((t & 0x1C7u) * 0x401u) & 0x00070007u;   // codes 0,2 -> bytes 0,2
+      const uint32_t od = ((t & 0xE38u) * 0x8020u) & 0x07000700u;  // codes 1,3 -> bytes 1,3
+      b8[w] = ev | od;
     }
-  } else if constexpr (FMT == F_MX4) {
-    // codes -> signed bytes 2*e2m1(c) via byte-permute lookups:
-    // magnitudes {0,1,2,3,4,6,8,12}, negatives as two's complement
-    const uint4 w4 = *reinterpret_cast<const uint4*>(qs);
-    const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
-    uint32_t b8[8];
+  } else {  // F_MX4: codes -> signed bytes 2*e2m1(c) by byte-permute lookups
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const uint32_t mag = wd[k] & 0x77777777u;
-      const uint32_t sgn = (wd[k] >> 1) & 0x44444444u;
+      const uint32_t mag = cw.w[k] & 0x77777777u;
+      const uint32_t sgn = (cw.w[k] >> 1) & 0x44444444u;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const uint32_t sel = h ? (mag >> 16) : mag;
         const uint32_t ssel = h ? (sgn >> 16) : sgn;
-        const uint32_t pos = __byte_perm(0x03020100u, 0x0C080604u, sel);
-        const uint32_t neg = __byte_perm(0xFDFEFF00u, 0xF4F8FAFCu, sel);
+        const uint32_t pos = __byte_perm(0x03020100u, 0x0C080604u, sel);  // 0,1,2,3,4,6,8,12
+        const uint32_t neg = __byte_perm(0xFDFEFF00u, 0xF4F8FAFCu, sel);  // their negatives
         const uint32_t msk = __byte_perm(0x00000000u, 0xFFFFFFFFu, ssel);
         b8[2 * k + h] = (pos & ~msk) | (neg & msk);
       }
     }
+  }
 #pragma unroll
-    for (int j = 0; j < F::NT; ++j) {
-      if (j < nt) {
+  for (int j = 0; j < F::NT; ++j) {
+    if (FULL || j < nt) {
+      const uint32_t* xw = &X.w[(j * CPL + cc) * 16];
+      int P;
+      if constexpr (FMT == F_MX4) {
         int ph = 0, pl = 0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-          ph = dp4a_ss(b8[w], xw[16 * j + w], ph);
-          pl = dp4a_su(b8[w], xw[16 * j + 8 + w], pl);
+          ph = dp4a_ss(b8[w], xw[w], ph);
+          pl = dp4a_su(b8[w], xw[8 + w], pl);
         }
-        const float P = (float)(ph * 256 + pl);
-        acc[j] = fmaf(sc, P * xs[j], acc[j]);
+        P = ph * 256 + pl;
+      } else if constexpr (FMT == F_A4) {
+        int phe = 0, ple = 0, pho = 0, plo = 0;
+#pragma unroll
+        for (int w = 0; w < 8; w += 2) {
+          phe = dp4a_us(b8[w], xw[w], phe);
+          ple = dp4a_uu(b8[w], xw[8 + w], ple);
+          pho = dp4a_us(b8[w + 1], xw[w + 1], pho);
+          plo = dp4a_uu(b8[w + 1], xw[9 + w], plo);
+        }
+        P = (phe * 256 + ple) + ((pho * 256 + plo) >> 4);  // exact: the odd sum is a multiple of 16
+      } else {
+        int ph = 0, pl = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+          ph = dp4a_us(b8[w], xw[w], ph);
+          pl = dp4a_uu(b8[w], xw[8 + w], pl);
+        }
+        P = ph * 256 + pl;
       }
-    }
-  } else {  // F_A3: exact float codes, fp32 activations
-    const uint32_t* wp = reinterpret_cast<const uint32_t*>(qs);
-    const uint32_t wd[3] = {wp[0], wp[1], wp[2]};
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int pos = 3 * i, wi = pos >> 5, sh = pos & 31;
-      uint32_t c = wd[wi] >> sh;
-      if (sh > 29) c |= wd[wi + 1] << (32 - sh);
-      v[i] = magic_u2f(c & 7u);
-    }
-#pragma unroll
-    for (int j = 0; j < F::NT; ++j) {
-      if (j < nt) {
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s = fmaf(v[i], __uint_as_float(xw[32 * j + i]), s);
-        acc[j] = fmaf(sc, s, fmaf(bi, xsum[j], acc[j]));
-      }
+      acc[j] = fmaf(sc, (float)P * X.xs[cc][j], fmaf(bi, X.xsum[cc][j], acc[j]));
     }
   }
 }
@@ -430,137 +462,209 @@ MOE_DEV float warp_transpose_reduce(float (&v)[V]) {
   return v[0];
 }
 
-template <int V>
-struct Log2 {
-  static constexpr int value = V <= 1 ? 0 : 1 + Log2<V / 2>::value;
-};
-template <>
-struct Log2<1> {
-  static constexpr int value = 0;
-};
-
-struct Ring {
-  uint8_t* base;
-  uint64_t* full;
-  volatile int* abort_flag;
-};
-
-// Issue the bulk copies of tile g into stage s (one thread).
+// Write one finished (row, token) result.
 template <int STAGE>
-MOE_DEV void issue_tile(const StreamParams& p, const Ring& ring, long long g, int s, int n_sh, int tpe) {
-  const Tile t = tile_at(p, g, n_sh, tpe);
+MOE_DEV void emit(const StreamParams& p, const Tile& t, int rl, int tok_slot, float g, float u) {
+  const int prow = t.pos0 + tok_slot;
+  const int r = t.r0 + rl;
+  if constexpr (STAGE == 1)
+    p.out[(size_t)prow * p.ld_out + r] = __fdividef(g * u, 1.f + __expf(-g));  // silu(g) * u
+  else
+    p.out[(size_t)prow * p.ld_out + r] = g;
+}
+
+// The rows of one pass: each warp of a row group reduces its lanes' partial
+// sums per row and either writes the result (one warp per row) or parks it
+// for the group's first warp.
+template <int FMT, int STAGE, int NTMAX, int CPL, bool FULL>
+MOE_DEV void tile_rows(const StreamParams& p, const Tile& t, const uint32_t (&qa)[2][CPL],
+                       const uint32_t (&sa)[2][CPL], uint32_t boff, int row_bytes, int sb_row, int rpg, int grp,
+                       int wig, int tb, int nt, float* red, int buf, const XRegs<NTMAX, CPL>& X) {
+  using F = SF<FMT, NTMAX>;
   constexpr int M = STAGE == 1 ? 2 : 1;
+  constexpr int NT = F::NT;
+  constexpr int V = M * NT;
+  const int lane = threadIdx.x & 31;
+  for (int r = 0; r < rpg; ++r) {
+    const int rl = grp * rpg + r;
+    if (rl >= t.rows) break;  // group-uniform
+    const uint32_t dq = (uint32_t)(rl * row_bytes), ds = (uint32_t)(rl * sb_row);
+    float acc[M][NTMAX];
+#pragma unroll
+    for (int m = 0; m < M; ++m)
+#pragma unroll
+      for (int j = 0; j < NTMAX; ++j) acc[m][j] = 0.f;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+#pragma unroll
+      for (int cc = 0; cc < CPL; ++cc) {
+        const ChunkWords cw = load_chunk<FMT>(qa[m][cc] + dq);
+        float sc, bi = 0.f;
+        if constexpr (FMT == F_MX4) {
+          const uint32_t e8 = lds8(sa[m][cc] + ds);
+          sc = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));  // 2^(e-128)
+        } else {
+          sc = bf16_bits_to_float(lds16(sa[m][cc] + ds));
+          bi = bf16_bits_to_float(lds16(sa[m][cc] + ds + boff));
+        }
+        chunk_dot_s<FMT, NTMAX, CPL, FULL>(cw, sc, bi, X, cc, nt, acc[m]);
+      }
+    }
+    // values ordered (token j, matrix m): g and u of a token sit side by side
+    float vals[V];
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int m = 0; m < M; ++m) vals[j * M + m] = acc[m][j];
+    const float red_v = warp_transpose_reduce<V>(vals);
+    constexpr int rep = 32 / V;
+    const float other = (M == 2) ? __shfl_down_sync(0xffffffffu, red_v, rep) : 0.f;
+    const int vi = lane / rep;
+    if ((lane & (rep - 1)) == 0 && (vi % M) == 0) {
+      const int j = vi / M;
+      if (FULL || j < nt) {
+        if (t.wpr == 1) {
+          emit<STAGE>(p, t, rl, tb + j, red_v, other);
+        } else {
+          float* dst = red + (size_t)buf * kRedHalf + ((grp * t.wpr + wig) * 16 + r) * 2 * NTMAX;
+          dst[2 * j] = red_v;
+          dst[2 * j + 1] = other;
+        }
+      }
+    }
+  }
+}
+
+// Issue the bulk copies of the tile at walker position w into stage s.
+template <int STAGE>
+MOE_DEV void issue_tile(const StreamParams& p, const Walker& w, uint8_t* smem, uint64_t* full, int s) {
+  constexpr int M = STAGE == 1 ? 2 : 1;
+  const Tile t = tile_of(p, w);
   const StageLayout Lay = stage_layout(*t.A, t.R, M, t.rows);
-  uint8_t* sb = ring.base + (size_t)s * kStageBytes;
-  mbar_expect_tx(&ring.full[s], (uint32_t)Lay.total);
+  uint8_t* sb = smem + (size_t)s * kStageBytes;
+  mbar_expect_tx(&full[s], (uint32_t)Lay.total);
   const QMatDev* mats[2] = {t.A, t.B};
   const size_t row0 = (size_t)t.e * t.A->n_out + t.r0;
 #pragma unroll
   for (int m = 0; m < M; ++m) {
     const QMatDev& Q = *mats[m];
-    const uint32_t rb = Q.wpr * 4;
-    bulk_g2s(sb + Lay.q[m], reinterpret_cast<const uint8_t*>(Q.q) + row0 * rb, t.rows * rb, &ring.full[s]);
+    const uint32_t rbytes = Q.wpr * 4;
+    bulk_g2s(sb + Lay.q[m], reinterpret_cast<const uint8_t*>(Q.q) + row0 * rbytes, t.rows * rbytes, &full[s]);
     const uint32_t sr = Q.gpr * (Q.fmt == F_MX4 ? 1 : 2);
-    bulk_g2s(sb + Lay.s[m], reinterpret_cast<const uint8_t*>(Q.scales) + row0 * sr, t.rows * sr, &ring.full[s]);
+    bulk_g2s(sb + Lay.s[m], reinterpret_cast<const uint8_t*>(Q.scales) + row0 * sr, t.rows * sr, &full[s]);
     if (Q.fmt != F_MX4)
-      bulk_g2s(sb + Lay.b[m], reinterpret_cast<const uint8_t*>(Q.biases) + row0 * sr, t.rows * sr, &ring.full[s]);
+      bulk_g2s(sb + Lay.b[m], reinterpret_cast<const uint8_t*>(Q.biases) + row0 * sr, t.rows * sr, &full[s]);
   }
 }
 
-// Process one tile of format FMT held in stage `s`; after the last pass's
-// barrier (every warp is done reading the stage) thread 0 refills the stage
-// with tile `g_next` when there is one.
-template <int FMT, int STAGE, int NTMAX>
-MOE_DEV void consume_tile(const StreamParams& p, const Tile& t, const Ring& ring, int s, long long g_next,
-                          long long g1, int n_sh, int tpe, float* red, int& buf,
-                          uint32_t (&xw)[XWords<NTMAX>::n], float (&xs)[NTMAX], float (&xsum)[NTMAX],
-                          int& cached_seg, int& cached_tb) {
-  using F = SF<FMT, STAGE, NTMAX>;
-  constexpr int M = F::M, RPT = F::RPT, NT = F::NT, V = F::V;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const QMatDev& A = *t.A;
-  const int C = A.n_in >> 5;
-  const int rows_par = kFfnThreads / C;
-  const int c = tid % C, slot = tid / C;
-  const int wps = C >> 5;  // warps per slot
-  const StageLayout Lay = stage_layout(A, t.R, M, t.rows);
-  const uint8_t* sb = ring.base + (size_t)s * kStageBytes;
+// Consume a run of consecutive tiles of one segment (one expert), starting
+// at the block's tile ordinal i0: per-expert addressing is set up once, then
+// each tile is waited for, computed and released.
+template <int FMT, int STAGE, int NTMAX, int CPL>
+MOE_DEV bool consume_run(const StreamParams& p, const Walker& w0, int n_run, int i0, uint8_t* smem, uint64_t* full,
+                         uint64_t* empty, volatile int* abort_flag, float* red, int& buf, XRegs<NTMAX, CPL>& X) {
+  using F = SF<FMT, NTMAX>;
+  constexpr int M = STAGE == 1 ? 2 : 1;
+  constexpr int NT = F::NT;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Tile t = tile_of(p, w0);
+  const QMatDev A = *t.A;  // fields in registers for the whole run
+  const int wpr = t.wpr;
+  const int G = kConsumerWarps / wpr;
+  const int grp = warp / wpr, wig = warp % wpr;
+  const int rpg = t.R / G;
+  const int cbase = wig * 32 * CPL;
+  const StageLayout Lay = stage_layout(A, t.R, M, t.R);
   const int row_bytes = A.wpr * 4;
-  const int ssz = FMT == F_MX4 ? 1 : 2;
-  const int sb_row = A.gpr * ssz;
-  const int gidx = (c * 32) / A.group;
-  constexpr int kChunkBytes = F::bits * 4;
-
+  constexpr bool mx = FMT == F_MX4;
+  const int sb_row = A.gpr * (mx ? 1 : 2);
+  const int gshift = A.group == 32 ? 0 : (A.group == 64 ? 1 : 2);  // chunk -> scale group
+  uint32_t qrel[2][CPL], srel[2][CPL];
+#pragma unroll
+  for (int m = 0; m < M; ++m)
+#pragma unroll
+    for (int cc = 0; cc < CPL; ++cc) {
+      const int c = cbase + 32 * cc + lane;
+      qrel[m][cc] = Lay.q[m] + c * F::kChunkBytes;
+      srel[m][cc] = Lay.s[m] + (c >> gshift) * (mx ? 1 : 2);
+    }
+  const uint32_t boff = (uint32_t)(t.R * sb_row);  // biases follow the scales of each matrix
   const int ntb = (t.npos + NT - 1) / NT;
-  for (int b = 0; b < ntb; ++b) {
-    const int tb = b * NT;
-    const int nt = min(NT, t.npos - tb);
-    if (cached_seg != t.seg || cached_tb != tb) {
-      load_x<FMT, STAGE, NTMAX>(p, t, tb, nt, c, xw, xs, xsum);
-      cached_seg = t.seg;
-      cached_tb = tb;
+  const uint32_t smem32 = smem_u32(smem);
+
+  for (int k = 0; k < n_run; ++k) {
+    const int i = i0 + k;
+    const int s = i % kStages;
+    if (!mbar_wait(&full[s], (uint32_t)(i / kStages) & 1u, abort_flag)) {
+      set_error(p.err, kErrTimeout);
+      *abort_flag = 1;
+      return false;
     }
-    float acc[V];
+    t.r0 = (w0.rb + k) * t.R;
+    t.rows = min(t.R, A.n_out - t.r0);
+    const uint32_t sb32 = smem32 + (uint32_t)s * kStageBytes;
+    uint32_t qa[2][CPL], sa[2][CPL];
 #pragma unroll
-    for (int i = 0; i < V; ++i) acc[i] = 0.f;
+    for (int m = 0; m < M; ++m)
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-      const int rl = slot + i * rows_par;
-      if (rl < t.rows) {
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-          const uint8_t* qp = sb + Lay.q[m] + rl * row_bytes + c * kChunkBytes;
-          float sc, bi = 0.f;
-          if constexpr (FMT == F_MX4) {
-            const uint32_t e8 = sb[Lay.s[m] + rl * sb_row + gidx];
-            sc = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));  // 2^(e-128)
-          } else {
-            sc = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(sb + Lay.s[m] + rl * sb_row + gidx * 2));
-            bi = bf16_bits_to_float(*reinterpret_cast<const uint16_t*>(sb + Lay.b[m] + rl * sb_row + gidx * 2));
-          }
-          chunk_dot_s<FMT, STAGE, NTMAX>(qp, sc, bi, xw, xs, xsum, nt, &acc[(i * M + m) * NT]);
-        }
+      for (int cc = 0; cc < CPL; ++cc) {
+        qa[m][cc] = sb32 + qrel[m][cc];
+        sa[m][cc] = sb32 + srel[m][cc];
       }
-    }
-    const float r = warp_transpose_reduce<V>(acc);
-    constexpr int rep = 32 / V;
-    if ((lane & (rep - 1)) == 0) red[(buf * kConsumerWarps + warp) * 32 + (lane / rep)] = r;
-    consumer_bar();
-    if (b == ntb - 1 && tid == 0 && g_next < g1) issue_tile<STAGE>(p, ring, g_next, s, n_sh, tpe);
-    // finalise: one thread per (slot, row i, token j)
-    const int nfin = rows_par * RPT * NT;
-    if (tid < nfin) {
-      const int fs = tid / (RPT * NT), rem = tid % (RPT * NT);
-      const int i = rem / NT, j = rem % NT;
-      const int rl = fs + i * rows_par;
-      if (j < nt && rl < t.rows) {
-        float g = 0.f, u = 0.f;
-        for (int w = 0; w < wps; ++w) {
-          const float* src = red + (buf * kConsumerWarps + fs * wps + w) * 32;
-          g += src[(i * M + 0) * NT + j];
-          if constexpr (M == 2) u += src[(i * M + 1) * NT + j];
-        }
-        const int prow = t.pos0 + tb + j;
-        const int r = t.r0 + rl;
-        if constexpr (STAGE == 1)
-          p.out[(size_t)prow * p.ld_out + r] = silu(g) * u;
+    for (int b = 0; b < ntb; ++b) {
+      const int tb = b * NT;
+      const int nt = min(NT, t.npos - tb);
+      if (k == 0 || ntb > 1) load_x<FMT, STAGE, NTMAX, CPL>(p, t, tb, nt, cbase, X);
+      if constexpr (NT == 1) {
+        tile_rows<FMT, STAGE, NTMAX, CPL, true>(p, t, qa, sa, boff, row_bytes, sb_row, rpg, grp, wig, tb, nt, red,
+                                                buf, X);
+      } else {
+        if (nt == NT)
+          tile_rows<FMT, STAGE, NTMAX, CPL, true>(p, t, qa, sa, boff, row_bytes, sb_row, rpg, grp, wig, tb, nt, red,
+                                                  buf, X);
         else
-          p.out[(size_t)prow * p.ld_out + r] = g;
+          tile_rows<FMT, STAGE, NTMAX, CPL, false>(p, t, qa, sa, boff, row_bytes, sb_row, rpg, grp, wig, tb, nt,
+                                                   red, buf, X);
+      }
+      if (b == ntb - 1) {  // every read of this stage by this warp is done
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      if (wpr > 1) {
+        group_bar(1 + grp, wpr * 32);
+        // lanes of the group's first warp sum the WPR partials of each (row, token)
+        if (wig == 0) {
+          const int nval = rpg * nt;
+          for (int v = lane; v < nval; v += 32) {
+            const int r = v / nt, j = v % nt;
+            const int rl = grp * rpg + r;
+            if (rl < t.rows) {
+              float g = 0.f, u = 0.f;
+              for (int ww = 0; ww < wpr; ++ww) {
+                const float* src = red + (size_t)buf * kRedHalf + ((grp * wpr + ww) * 16 + r) * 2 * NTMAX;
+                g += src[2 * j];
+                u += src[2 * j + 1];
+              }
+              emit<STAGE>(p, t, rl, tb + j, g, u);
+            }
+          }
+        }
+        buf ^= 1;
       }
     }
-    buf ^= 1;
   }
+  return true;
 }
 
-template <int STAGE, int NTMAX>
-__global__ void __launch_bounds__(kStreamThreads, 1) ffn_stream_kernel(const __grid_constant__ StreamParams p) {
+template <int STAGE, int NTMAX, int CPL, int RFMT>
+__global__ void __launch_bounds__(kStreamThreads, 1)
+ffn_stream_kernel(const __grid_constant__ StreamParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   float* red = reinterpret_cast<float*>(smem + (size_t)kStages * kStageBytes);
-  Ring ring;
-  ring.base = smem;
-  ring.full = reinterpret_cast<uint64_t*>(red + kRedFloats);
-  ring.abort_flag = reinterpret_cast<volatile int*>(ring.full + kStages);
-  const int tid = threadIdx.x;
+  uint64_t* full = reinterpret_cast<uint64_t*>(red + kRedFloats);
+  uint64_t* empty = full + kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   const int n_active = __ldcg(p.active);
   const int n_sh = p.has_shared ? (p.sa.n_out + p.s_rows - 1) / p.s_rows : 0;
@@ -570,47 +674,65 @@ __global__ void __launch_bounds__(kStreamThreads, 1) ffn_stream_kernel(const __g
   if (g0 >= g1) return;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&ring.full[s], 1);
-    *ring.abort_flag = 0;
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
     fence_mbar_init();
-    for (int s = 0; s < kStages && g0 + s < g1; ++s) issue_tile<STAGE>(p, ring, g0 + s, s, n_sh, tpe);
   }
   __syncthreads();
 
-  uint32_t xw[XWords<NTMAX>::n];
-  float xs[NTMAX], xsum[NTMAX];
-  int cached_seg = -2, cached_tb = -1;
-  int buf = 0;
-  int i = 0;
-  long long g = g0;
-  for (; g < g1; ++g, ++i) {
-    const int s = i % kStages;
-    const uint32_t round = (uint32_t)(i / kStages);
-    if (!mbar_wait(&ring.full[s], round & 1u, ring.abort_flag)) {
-      set_error(p.err, kErrTimeout);
-      *ring.abort_flag = 1;
-      break;
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: one lane issues every copy
+    if (lane != 0) return;
+    Walker w;
+    w.start(p, g0, g1, n_sh, tpe);
+    int i = 0;
+    for (; w.g < g1; w.next(p), ++i) {
+      const int s = i % kStages;
+      const uint32_t round = (uint32_t)(i / kStages);
+      if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1u, abort_flag)) {
+        set_error(p.err, kErrTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      issue_tile<STAGE>(p, w, smem, full, s);
     }
-    const Tile t = tile_at(p, g, n_sh, tpe);
-    const long long gn = g + kStages;
-    switch (t.A->fmt) {
-      case F_A2: consume_tile<F_A2, STAGE, NTMAX>(p, t, ring, s, gn, g1, n_sh, tpe, red, buf, xw, xs, xsum, cached_seg, cached_tb); break;
-      case F_A3: consume_tile<F_A3, STAGE, NTMAX>(p, t, ring, s, gn, g1, n_sh, tpe, red, buf, xw, xs, xsum, cached_seg, cached_tb); break;
-      case F_A4: consume_tile<F_A4, STAGE, NTMAX>(p, t, ring, s, gn, g1, n_sh, tpe, red, buf, xw, xs, xsum, cached_seg, cached_tb); break;
-      case F_A8: consume_tile<F_A8, STAGE, NTMAX>(p, t, ring, s, gn, g1, n_sh, tpe, red, buf, xw, xs, xsum, cached_seg, cached_tb); break;
-      default:   consume_tile<F_MX4, STAGE, NTMAX>(p, t, ring, s, gn, g1, n_sh, tpe, red, buf, xw, xs, xsum, cached_seg, cached_tb); break;
-    }
-  }
-  // After an abort, wait (bounded) for copies still in flight before the
-  // block's shared memory goes away.
-  if (g < g1 && tid == 0) {
-    const long long issued = min(g1, g0 + (long long)i + kStages);
-    for (long long q = g0 + i; q < issued; ++q) {
-      const int s = (int)((q - g0) % kStages);
+    // drain: no copy may still be landing in shared memory when the block exits
+    for (int q = max(0, i - kStages); q < i; ++q) {
+      const int s = q % kStages;
       const long long t0 = clock64();
-      while (!mbar_try_wait(&ring.full[s], (uint32_t)((q - g0) / kStages) & 1u) && clock64() - t0 < kWaitCycles) {
+      while (!mbar_try_wait(&full[s], (uint32_t)(q / kStages) & 1u) && clock64() - t0 < kWaitCycles) {
       }
     }
+    return;
+  }
+
+  // ---------------- consumers: runs of tiles of one expert at a time
+  XRegs<NTMAX, CPL> X;
+  int buf = 0;
+  int prev_wpr = 1;
+  Walker w;
+  w.start(p, g0, g1, n_sh, tpe);
+  int i = 0;
+  while (w.g < g1) {
+    const int seg_tiles = w.a < 0 ? n_sh : tpe;
+    const int n_run = (int)min((long long)(seg_tiles - w.rb), g1 - w.g);
+    const Tile t = tile_of(p, w);
+    // when the row-group shape changes, let every old finaliser finish with
+    // the partial sums before another group may overwrite them
+    if (t.wpr != prev_wpr && prev_wpr > 1) group_bar(9, kConsumerWarps * 32);
+    prev_wpr = t.wpr;
+    bool ok;
+    // the routed format, or the 8-bit shared expert
+    if (RFMT == F_A8 || t.A->fmt == RFMT)
+      ok = consume_run<RFMT, STAGE, NTMAX, CPL>(p, w, n_run, i, smem, full, empty, abort_flag, red, buf, X);
+    else
+      ok = consume_run<F_A8, STAGE, NTMAX, CPL>(p, w, n_run, i, smem, full, empty, abort_flag, red, buf, X);
+    if (!ok) break;
+    for (int k = 0; k < n_run; ++k) w.next(p);
+    i += n_run;
   }
 }
 

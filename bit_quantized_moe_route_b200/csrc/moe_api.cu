@@ -13,7 +13,7 @@
 #include "../../include/moe_lowbit.h"
 #include "common.cuh"
 #include "ffn_gemv.cuh"
-#include "ffn_stream.cuh"
+#include "stream_types.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -198,6 +198,8 @@ moe_status_t check_qmat(const moe_qmat_t* m, int n_in, const char* name, QMatDev
   return MOE_OK;
 }
 
+extern const StreamAttrFn kStreamAttrs[10];
+
 struct DevInfo {
   int sms = 0;
   int ffn1_blocks = 0, ffn2_blocks = 0;
@@ -223,12 +225,7 @@ moe_status_t dev_info(DevInfo** out) {
       cudaFuncSetAttribute(route_small_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
       cudaFuncSetAttribute(route_hash_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
       cudaFuncSetAttribute(route_hash_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(ffn_stream_kernel<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
-      cudaFuncSetAttribute(ffn_stream_kernel<2, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
-      cudaFuncSetAttribute(ffn_stream_kernel<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
-      cudaFuncSetAttribute(ffn_stream_kernel<2, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
-      cudaFuncSetAttribute(ffn_stream_kernel<1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
-      cudaFuncSetAttribute(ffn_stream_kernel<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStreamSmem);
+      for (StreamAttrFn f : kStreamAttrs) f();
       int b1 = 0, b2 = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, ffn_gemv_kernel<1, 4>, kFfnThreads, 0);
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, ffn_gemv_kernel<2, 8>, kFfnThreads, 0);
@@ -355,23 +352,53 @@ moe_status_t launch_permute(const moe_dims_t& d, const int* ids, int* offsets, i
   return MOE_OK;
 }
 
-// Rows per streaming tile for a matrix in stage `stage` (mirrors SF<>::RPT),
-// or 0 when the matrix does not fit the streaming kernel's constraints:
-// n_in/32 chunks in {32, 64, 128, 256}, 16-byte multiples for every copied
-// row segment, and a tile of at most 32 KiB packed + 8 KiB scales/biases.
-int stream_rows(const QMatDev& A, int stage) {
+// Streaming-kernel plan for one matrix: warps per row group and rows per
+// tile, or ok = false when the matrix does not fit the kernel's constraints
+// (n_in a multiple of 32*32*cpl with at most 8 warps per row, 16-byte row
+// segments, a tile of at most one stage buffer).
+struct StreamPlan {
+  bool ok = false;
+  int wpr = 1, rows = 0;
+};
+
+StreamPlan stream_plan(const QMatDev& A, int stage, int cpl, int max_units, int sms) {
+  StreamPlan pl;
   const int C = A.n_in / 32;
-  if (C != 32 && C != 64 && C != 128 && C != 256) return 0;
-  const int bits = A.fmt == F_A2 ? 2 : A.fmt == F_A3 ? 3 : A.fmt == F_A8 ? 8 : 4;
-  const int rpt = (A.fmt == F_A3 ? 4 : 16 / bits) * (stage == 1 ? 1 : 2);
-  const int R = (kFfnThreads / C) * rpt;
+  if (C % (32 * cpl)) return pl;
+  const int wpr = C / (32 * cpl);
+  if (wpr > kConsumerWarps || kConsumerWarps % wpr) return pl;
   const int M = stage == 1 ? 2 : 1;
+  const bool mx = A.fmt == F_MX4;
   const int row_bytes = A.wpr * 4;
-  const int sb_row = A.gpr * (A.fmt == F_MX4 ? 1 : 2);
-  if (row_bytes % 16 || sb_row % 16) return 0;
-  if (R * M * row_bytes > kStageQBytes) return 0;
-  if (R * M * sb_row * (A.fmt == F_MX4 ? 1 : 2) > kStageSBBytes) return 0;
-  return R;
+  const int sb_row = A.gpr * (mx ? 1 : 2);
+  if (row_bytes % 16 || sb_row % 16) return pl;
+  const int per_row = M * (row_bytes + sb_row * (mx ? 1 : 2));
+  const int G = kConsumerWarps / wpr;
+  int rpg = std::min(16, kStageBytes / (G * per_row));
+  if (rpg < 1) return pl;
+  // keep at least ~4 tiles per block so the contiguous ranges balance
+  while (rpg > 1 && (long long)max_units * ((A.n_out + G * rpg - 1) / (G * rpg)) < 4LL * sms) rpg >>= 1;
+  pl.ok = true;
+  pl.wpr = wpr;
+  pl.rows = G * rpg;
+  return pl;
+}
+
+// Streaming launchers indexed by routed format code (F_A2..F_MX4).
+const StreamLaunchFn kStreamLaunch[2][5] = {
+    {launch_stream_s1_A2, launch_stream_s1_A3, launch_stream_s1_A4, launch_stream_s1_A8, launch_stream_s1_MX4},
+    {launch_stream_s2_A2, launch_stream_s2_A3, launch_stream_s2_A4, launch_stream_s2_A8, launch_stream_s2_MX4}};
+const StreamAttrFn kStreamAttrs[10] = {attrs_stream_s1_A2, attrs_stream_s1_A3, attrs_stream_s1_A4, attrs_stream_s1_A8,
+                                       attrs_stream_s1_MX4, attrs_stream_s2_A2, attrs_stream_s2_A3, attrs_stream_s2_A4,
+                                       attrs_stream_s2_A8, attrs_stream_s2_MX4};
+
+// chunks per lane for a stage: as many as the activation registers allow
+// (tokens per pass x chunks <= 4) and every matrix's width divides
+int stream_cpl(int ntmax, int n_in_a, int n_in_b) {
+  for (int cpl = 4 / ntmax; cpl >= 1; cpl >>= 1) {
+    if ((n_in_a / 32) % (32 * cpl) == 0 && (n_in_b / 32) % (32 * cpl) == 0) return cpl;
+  }
+  return 0;
 }
 
 // Stage 1 + stage 2 of the expert FFN (routed pairs, optional shared expert).
@@ -395,9 +422,21 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
   p.err = &ws_at<WsHeader>(ws, L.hdr)->err;
   p.shared_pos0 = Tk;
   p.has_shared = sh != nullptr;
-  const int r1 = stream_rows(w1, 1), r2 = stream_rows(w2, 2);
-  const int s1 = sh ? stream_rows(sh[0], 1) : 1, s2 = sh ? stream_rows(sh[2], 2) : 1;
-  if (r1 && r2 && s1 && s2) {
+  // tokens per pass: experts rarely see more than two tokens at decode sizes
+  const int ntmax = d.T >= 2 ? 2 : 1;
+  const int fs = sh ? d.d_ff_shared : d.d_ff;
+  const int cpl1 = stream_cpl(ntmax, d.d_model, d.d_model);
+  const int cpl2 = stream_cpl(ntmax, d.d_ff, fs);
+  StreamPlan r1, r2, s1, s2;
+  if (cpl1 && cpl2) {
+    r1 = stream_plan(w1, 1, cpl1, max_active, di->sms);
+    r2 = stream_plan(w2, 2, cpl2, max_active, di->sms);
+    s1 = sh ? stream_plan(sh[0], 1, cpl1, 1, di->sms) : r1;
+    s2 = sh ? stream_plan(sh[2], 2, cpl2, 1, di->sms) : r2;
+  }
+  // the streaming kernels compile the routed format plus the 8-bit shared path
+  const bool fmt_ok = !sh || ((sh[0].fmt == w1.fmt || sh[0].fmt == F_A8) && (sh[2].fmt == w2.fmt || sh[2].fmt == F_A8));
+  if (fmt_ok && cpl1 && cpl2 && r1.ok && r2.ok && s1.ok && s2.ok) {
     StreamParams q{};
     q.x = p.x;
     q.T = d.T;
@@ -412,22 +451,13 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
     q.ld_out = ld_h;
     q.ra = w1;
     q.rb = w3;
-    q.r_rows = r1;
-    if (sh) {
-      q.sa = sh[0];
-      q.sb = sh[1];
-      q.s_rows = s1;
-    } else {
-      q.s_rows = 1;
-    }
-    // tokens per expert never exceed T: size the per-pass activation registers by it
-    const int ntmax = d.T >= 4 ? 4 : d.T;
-    if (ntmax == 1)
-      ffn_stream_kernel<1, 1><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
-    else if (ntmax == 2)
-      ffn_stream_kernel<1, 2><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
-    else
-      ffn_stream_kernel<1, 4><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
+    q.r_rows = r1.rows;
+    q.r_wpr = r1.wpr;
+    q.sa = sh ? sh[0] : w1;
+    q.sb = sh ? sh[1] : w3;
+    q.s_rows = s1.rows;
+    q.s_wpr = s1.wpr;
+    if (!kStreamLaunch[0][w1.fmt](ntmax, cpl1, di->sms, s, q)) return fail(MOE_ERR_UNSUPPORTED, "no streaming kernel");
     MOE_CHECK_LAUNCH("ffn_stream_kernel<1>");
     hook_mark(s, "ffn_w13_swiglu");
     q.hin = h;
@@ -436,18 +466,13 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
     q.ld_out = ld_y;
     q.ra = w2;
     q.rb = w2;
-    q.r_rows = r2;
-    if (sh) {
-      q.sa = sh[2];
-      q.sb = sh[2];
-      q.s_rows = s2;
-    }
-    if (ntmax == 1)
-      ffn_stream_kernel<2, 1><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
-    else if (ntmax == 2)
-      ffn_stream_kernel<2, 2><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
-    else
-      ffn_stream_kernel<2, 4><<<di->sms, kStreamThreads, kStreamSmem, s>>>(q);
+    q.r_rows = r2.rows;
+    q.r_wpr = r2.wpr;
+    q.sa = sh ? sh[2] : w2;
+    q.sb = q.sa;
+    q.s_rows = s2.rows;
+    q.s_wpr = s2.wpr;
+    if (!kStreamLaunch[1][w2.fmt](ntmax, cpl2, di->sms, s, q)) return fail(MOE_ERR_UNSUPPORTED, "no streaming kernel");
     MOE_CHECK_LAUNCH("ffn_stream_kernel<2>");
     hook_mark(s, "ffn_w2");
     return MOE_OK;

@@ -123,6 +123,59 @@ __device__ void permute_block(const int* __restrict__ ids, int N, int E, int* __
   }
 }
 
+// The same stable grouping for N <= 32 pairs by a single warp: the sorted
+// position of pair i is the number of pairs (e_j, j) ordered before (e_i, i).
+__device__ void permute_warp(const int* __restrict__ ids, int N, int E, int* __restrict__ offsets,
+                             int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active, int* err) {
+  const int lane = threadIdx.x & 31;
+  int e = 0x7fffffff;
+  bool bad = false;
+  if (lane < N) {
+    e = ids[lane];
+    if (e < 0 || e >= E) {
+      bad = true;
+      e = 0;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, kErrDeviceInput);
+  int ev[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) ev[j] = __shfl_sync(0xffffffffu, e, j);
+  int rank = 0, first = 1, drank = 0;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j < N) {
+      rank += (ev[j] < e || (ev[j] == e && j < lane)) ? 1 : 0;
+      if (ev[j] == e && j < lane) first = 0;
+    }
+  }
+  // distinct experts below e: count first occurrences with a smaller id
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    if (j < N) {
+      bool fj = true;
+#pragma unroll
+      for (int q = 0; q < 32; ++q)
+        if (q < j && ev[q] == ev[j]) fj = false;
+      if (fj && ev[j] < e) ++drank;
+    }
+  }
+  if (lane < N) {
+    sorted_rows[rank] = lane;
+    inv[lane] = rank;
+    if (first) active[1 + drank] = e;
+  }
+  const int n_first = __popc(__ballot_sync(0xffffffffu, lane < N && first));
+  if (lane == 0) active[0] = n_first;
+  for (int x = lane; x <= E; x += 32) {
+    int c = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      if (j < N && ev[j] < x) ++c;
+    offsets[x] = c;
+  }
+}
+
 // One CTA of 1024 threads.  Dynamic shared memory: (2 + 32) * E ints.
 // active[0] = number of experts with pairs, active[1..] their ids ascending.
 __global__ void __launch_bounds__(kPermThreads)

@@ -392,8 +392,12 @@ route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __res
     topk_token<MAXPER>(L + (size_t)t * E, bias, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
   __threadfence_block();
   __syncthreads();
-  permute_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, reinterpret_cast<int*>(sm_raw), warp_tot,
-                &total);
+  if (T * k <= 32) {
+    if (warp == 0) permute_warp(ids, T * k, E, offsets, sorted_rows, inv, active, err);
+  } else {
+    permute_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, reinterpret_cast<int*>(sm_raw), warp_tot,
+                  &total);
+  }
   if (tid == 0) *counter = 0;
 }
 
@@ -417,8 +421,12 @@ route_hash_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __rest
   __syncthreads();
   if (!is_last) return;
   __threadfence();
-  permute_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, reinterpret_cast<int*>(sm_raw), warp_tot,
-                &total);
+  if (T * k <= 32) {
+    if ((threadIdx.x >> 5) == 0) permute_warp(ids, T * k, E, offsets, sorted_rows, inv, active, err);
+  } else {
+    permute_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, reinterpret_cast<int*>(sm_raw), warp_tot,
+                  &total);
+  }
   if (threadIdx.x == 0) *counter = 0;
 }
 
