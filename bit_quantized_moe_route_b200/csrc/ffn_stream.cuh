@@ -84,6 +84,17 @@ MOE_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As above, but the thread may sleep up to ~0.1 ms inside the instruction
+// until the phase completes (fewer polling iterations while waiting).
+MOE_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(100000)
+      : "memory");
+  return ok != 0;
+}
 // Bulk copy global -> shared; completion is counted on `bar` in bytes.
 // Both addresses 16-byte aligned, size a multiple of 16.
 MOE_DEV void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -99,7 +110,7 @@ constexpr long long kWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz: every wait 
 MOE_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity)) {
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitCycles) return false;
   }
@@ -473,58 +484,71 @@ MOE_DEV void emit(const StreamParams& p, const Tile& t, int rl, int tok_slot, fl
     p.out[(size_t)prow * p.ld_out + r] = g;
 }
 
-// The rows of one pass: each warp of a row group reduces its lanes' partial
-// sums per row and either writes the result (one warp per row) or parks it
-// for the group's first warp.
+// Rows reduced together: one transposed warp reduction per block of RB rows.
+template <int STAGE, int NT>
+struct RowBlock {
+  static constexpr int M = STAGE == 1 ? 2 : 1;
+  static constexpr int RB = (STAGE == 1 ? 2 : 8) / NT > 0 ? (STAGE == 1 ? 2 : 8) / NT : 1;
+  static constexpr int V = RB * M * NT;  // <= 8 values per lane
+};
+
+// The rows of one pass: a warp computes its lanes' partial sums for a block
+// of RB rows, reduces them in one transposed warp reduction, and either
+// writes the results (one warp per row) or parks them for the group's first
+// warp.
 template <int FMT, int STAGE, int NTMAX, int CPL, bool FULL>
 MOE_DEV void tile_rows(const StreamParams& p, const Tile& t, const uint32_t (&qa)[2][CPL],
                        const uint32_t (&sa)[2][CPL], uint32_t boff, int row_bytes, int sb_row, int rpg, int grp,
                        int wig, int tb, int nt, float* red, int buf, const XRegs<NTMAX, CPL>& X) {
   using F = SF<FMT, NTMAX>;
-  constexpr int M = STAGE == 1 ? 2 : 1;
-  constexpr int NT = F::NT;
-  constexpr int V = M * NT;
+  using RBk = RowBlock<STAGE, F::NT>;
+  constexpr int M = RBk::M, NT = F::NT, RB = RBk::RB, V = RBk::V;
   const int lane = threadIdx.x & 31;
-  for (int r = 0; r < rpg; ++r) {
-    const int rl = grp * rpg + r;
-    if (rl >= t.rows) break;  // group-uniform
-    const uint32_t dq = (uint32_t)(rl * row_bytes), ds = (uint32_t)(rl * sb_row);
-    float acc[M][NTMAX];
-#pragma unroll
-    for (int m = 0; m < M; ++m)
-#pragma unroll
-      for (int j = 0; j < NTMAX; ++j) acc[m][j] = 0.f;
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-#pragma unroll
-      for (int cc = 0; cc < CPL; ++cc) {
-        const ChunkWords cw = load_chunk<FMT>(qa[m][cc] + dq);
-        float sc, bi = 0.f;
-        if constexpr (FMT == F_MX4) {
-          const uint32_t e8 = lds8(sa[m][cc] + ds);
-          sc = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));  // 2^(e-128)
-        } else {
-          sc = bf16_bits_to_float(lds16(sa[m][cc] + ds));
-          bi = bf16_bits_to_float(lds16(sa[m][cc] + ds + boff));
-        }
-        chunk_dot_s<FMT, NTMAX, CPL, FULL>(cw, sc, bi, X, cc, nt, acc[m]);
-      }
-    }
-    // values ordered (token j, matrix m): g and u of a token sit side by side
+  const int rows_here = min(rpg, t.rows - grp * rpg);  // group-uniform
+  for (int r0 = 0; r0 < rows_here; r0 += RB) {
+    // values ordered (row b, token j, matrix m): g and u of a (row, token) sit side by side
     float vals[V];
 #pragma unroll
-    for (int j = 0; j < NT; ++j)
+    for (int v = 0; v < V; ++v) vals[v] = 0.f;
 #pragma unroll
-      for (int m = 0; m < M; ++m) vals[j * M + m] = acc[m][j];
+    for (int b = 0; b < RB; ++b) {
+      if (r0 + b < rows_here) {
+        const int rl = grp * rpg + r0 + b;
+        const uint32_t dq = (uint32_t)(rl * row_bytes), ds = (uint32_t)(rl * sb_row);
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          float acc[NTMAX];
+#pragma unroll
+          for (int j = 0; j < NTMAX; ++j) acc[j] = 0.f;
+#pragma unroll
+          for (int cc = 0; cc < CPL; ++cc) {
+            const ChunkWords cw = load_chunk<FMT>(qa[m][cc] + dq);
+            float sc, bi = 0.f;
+            if constexpr (FMT == F_MX4) {
+              const uint32_t e8 = lds8(sa[m][cc] + ds);
+              sc = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));  // 2^(e-128)
+            } else {
+              sc = bf16_bits_to_float(lds16(sa[m][cc] + ds));
+              bi = bf16_bits_to_float(lds16(sa[m][cc] + ds + boff));
+            }
+            chunk_dot_s<FMT, NTMAX, CPL, FULL>(cw, sc, bi, X, cc, nt, acc);
+          }
+#pragma unroll
+          for (int j = 0; j < NT; ++j) vals[(b * NT + j) * M + m] = acc[j];
+        }
+      }
+    }
     const float red_v = warp_transpose_reduce<V>(vals);
     constexpr int rep = 32 / V;
     const float other = (M == 2) ? __shfl_down_sync(0xffffffffu, red_v, rep) : 0.f;
     const int vi = lane / rep;
     if ((lane & (rep - 1)) == 0 && (vi % M) == 0) {
-      const int j = vi / M;
-      if (FULL || j < nt) {
+      const int bj = vi / M;
+      const int b = bj / NT, j = bj % NT;
+      const int r = r0 + b;
+      if (r < rows_here && (FULL || j < nt)) {
         if (t.wpr == 1) {
-          emit<STAGE>(p, t, rl, tb + j, red_v, other);
+          emit<STAGE>(p, t, grp * rpg + r, tb + j, red_v, other);
         } else {
           float* dst = red + (size_t)buf * kRedHalf + ((grp * t.wpr + wig) * 16 + r) * 2 * NTMAX;
           dst[2 * j] = red_v;

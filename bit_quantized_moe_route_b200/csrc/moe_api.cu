@@ -304,8 +304,8 @@ moe_status_t launch_route_fused(const moe_dims_t& d, const void* x, const float*
   WsHeader* hdr = ws_at<WsHeader>(ws, L.hdr);
   int* active = ws_at<int>(ws, L.active);
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-  const int nw_perm = 8;
-  const size_t perm_smem = (size_t)(2 + nw_perm) * d.n_experts * sizeof(int);
+  // tail scratch: top-k keys/scores/selected (2E + k floats), pair ids and flags (2 T*k ints)
+  const size_t perm_smem = (size_t)(2 * d.n_experts + 32 + 2 * d.T * d.top_k) * sizeof(int);
   if (d.hash_mode) {
     const int blocks = ceil_div(d.T * 32, 256);
     if (d.top_k <= 8)

@@ -138,27 +138,15 @@ __device__ void permute_warp(const int* __restrict__ ids, int N, int E, int* __r
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, kErrDeviceInput);
-  int ev[32];
-#pragma unroll
-  for (int j = 0; j < 32; ++j) ev[j] = __shfl_sync(0xffffffffu, e, j);
-  int rank = 0, first = 1, drank = 0;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    if (j < N) {
-      rank += (ev[j] < e || (ev[j] == e && j < lane)) ? 1 : 0;
-      if (ev[j] == e && j < lane) first = 0;
-    }
-  }
-  // distinct experts below e: count first occurrences with a smaller id
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    if (j < N) {
-      bool fj = true;
-#pragma unroll
-      for (int q = 0; q < 32; ++q)
-        if (q < j && ev[q] == ev[j]) fj = false;
-      if (fj && ev[j] < e) ++drank;
-    }
+  // first occurrence of each expert among the pairs (lowest lane of its peers)
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int first = (lane < N && (__ffs(peers) - 1) == lane) ? 1 : 0;
+  int rank = 0, drank = 0;
+  for (int j = 0; j < N; ++j) {
+    const int ej = __shfl_sync(0xffffffffu, e, j);
+    const int fj = __shfl_sync(0xffffffffu, first, j);
+    rank += (ej < e || (ej == e && j < lane)) ? 1 : 0;
+    drank += (fj && ej < e) ? 1 : 0;
   }
   if (lane < N) {
     sorted_rows[rank] = lane;
@@ -167,12 +155,12 @@ __device__ void permute_warp(const int* __restrict__ ids, int N, int E, int* __r
   }
   const int n_first = __popc(__ballot_sync(0xffffffffu, lane < N && first));
   if (lane == 0) active[0] = n_first;
-  for (int x = lane; x <= E; x += 32) {
+  // offsets[x] = pairs with an expert id below x
+  for (int x0 = 0; x0 <= E; x0 += 32) {
+    const int x = x0 + lane;
     int c = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (j < N && ev[j] < x) ++c;
-    offsets[x] = c;
+    for (int j = 0; j < N; ++j) c += (__shfl_sync(0xffffffffu, e, j) < x) ? 1 : 0;
+    if (x <= E) offsets[x] = c;
   }
 }
 

@@ -304,6 +304,94 @@ route_hash_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__
 }
 
 // ---------------------------------------------------------------------------
+// Block-parallel tails for the fused routing kernels (one block, <= 1024
+// threads, shared memory `sm` of at least 2*E + 2*N ints).
+// ---------------------------------------------------------------------------
+// Top-k of one token by ranks: expert e is selected at position rank(e) =
+// #{j : key_j > key_e or (key_j == key_e and j < e)} when rank(e) < k.
+__device__ void topk_token_block(const float* __restrict__ Lrow, const float* __restrict__ bias, int E, int k,
+                                 int* __restrict__ ids_row, float* __restrict__ w_row, float* keys, float* scs,
+                                 float* sel) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const float s = sqrt_softplus(__ldcg(Lrow + e));
+    const float kv = bias ? s + bias[e] : s;
+    keys[e] = (kv != kv) ? -INFINITY : kv;
+    scs[e] = s;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const float ke = keys[e];
+    int rank = 0;
+    for (int j = 0; j < E; ++j) {
+      const float kj = keys[j];
+      rank += (kj > ke || (kj == ke && j < e)) ? 1 : 0;
+    }
+    if (rank < k) {
+      ids_row[rank] = e;
+      sel[rank] = scs[e];
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < k) {
+    float ssum = 0.f;
+    for (int j = 0; j < k; ++j) ssum += sel[j];  // same order in every thread
+    w_row[threadIdx.x] = ssum > 0.f ? sel[threadIdx.x] / ssum : 1.f / (float)k;
+  }
+  __syncthreads();
+}
+
+// Stable grouping of N pairs by expert, by ranks: pair i goes to position
+// #{j : (e_j, j) < (e_i, i)}; offsets[x] = #{j : e_j < x}; the active list
+// holds each expert once, ascending.  Out-of-range ids are reported and
+// treated as expert 0.
+__device__ void permute_ranks_block(const int* __restrict__ ids, int N, int E, int* __restrict__ offsets,
+                                    int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
+                                    int* err, int* ev, int* first) {
+  bool bad = false;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    int e = ids[i];
+    if (e < 0 || e >= E) {
+      bad = true;
+      e = 0;
+    }
+    ev[i] = e;
+  }
+  if (bad) set_error(err, kErrDeviceInput);
+  __syncthreads();
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const int e = ev[i];
+    int rank = 0, f = 1;
+    for (int j = 0; j < N; ++j) {
+      const int ej = ev[j];
+      rank += (ej < e || (ej == e && j < i)) ? 1 : 0;
+      if (ej == e && j < i) f = 0;
+    }
+    sorted_rows[rank] = i;
+    inv[i] = rank;
+    first[i] = f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    if (first[i]) {
+      const int e = ev[i];
+      int dr = 0;
+      for (int j = 0; j < N; ++j) dr += (first[j] && ev[j] < e) ? 1 : 0;
+      active[1 + dr] = e;
+    }
+  }
+  for (int x = threadIdx.x; x <= E; x += blockDim.x) {
+    int c = 0;
+    for (int j = 0; j < N; ++j) c += ev[j] < x ? 1 : 0;
+    offsets[x] = c;
+  }
+  if (threadIdx.x == 0) {
+    int nf = 0;
+    for (int j = 0; j < N; ++j) nf += first[j];
+    active[0] = nf;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Small-T fused routing: logits, top-k, renormalisation and the stable
 // permutation in one launch.  Every block computes the logits of two experts
 // (four warps per expert, each over a quarter of d_model) for all tokens; the
@@ -377,28 +465,36 @@ route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __res
     if (tid < 2 * kFusedTB) {
       const int h = tid / kFusedTB, t = tid % kFusedTB;
       const int ee = blockIdx.x * 2 + h;
-      if (ee < E && t < nt)
+      if (ee < E && t < nt) {
         L[(size_t)(t0 + t) * E + ee] = part[4 * h][t] + part[4 * h + 1][t] + part[4 * h + 2][t] + part[4 * h + 3][t];
+        __threadfence();  // publish before the arrival below
+      }
     }
   }
-  // publish this block's logits, then count arrivals
-  __threadfence();
   __syncthreads();
-  if (tid == 0) is_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
+  if (tid == 0) {
+    is_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
+    if (is_last) __threadfence();
+  }
   __syncthreads();
   if (!is_last) return;
-  __threadfence();
-  for (int t = warp; t < T; t += 8)
-    topk_token<MAXPER>(L + (size_t)t * E, bias, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
+  // last block: every token's top-k, then the grouping of the T*k pairs
+  float* fsm = reinterpret_cast<float*>(sm_raw);
+  if (T <= 2) {
+    for (int t = 0; t < T; ++t)
+      topk_token_block(L + (size_t)t * E, bias, E, k, ids + (size_t)t * k, wts + (size_t)t * k, fsm, fsm + E,
+                       fsm + 2 * E);
+  } else {
+    for (int t = warp; t < T; t += 8)
+      topk_token<MAXPER>(L + (size_t)t * E, bias, E, k, ids + (size_t)t * k, wts + (size_t)t * k);
+  }
   __threadfence_block();
   __syncthreads();
-  if (T * k <= 32) {
-    if (warp == 0) permute_warp(ids, T * k, E, offsets, sorted_rows, inv, active, err);
-  } else {
-    permute_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, reinterpret_cast<int*>(sm_raw), warp_tot,
-                  &total);
-  }
+  int* ism = reinterpret_cast<int*>(sm_raw);
+  permute_ranks_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, ism, ism + T * k);
   if (tid == 0) *counter = 0;
+  (void)warp_tot;
+  (void)total;
 }
 
 // Hash routing plus permutation, one launch: one warp per token, the last
@@ -415,19 +511,19 @@ route_hash_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __rest
   __shared__ int total;
   __shared__ int is_last;
   route_hash_warp<KMAX>(x, W, token_ids, table, T, d, E, k, vocab, ids, wts, err);
-  __threadfence();
+  __threadfence();  // publish this warp's ids/weights before the arrival below
   __syncthreads();
-  if (threadIdx.x == 0) is_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
+  if (threadIdx.x == 0) {
+    is_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;
+    if (is_last) __threadfence();
+  }
   __syncthreads();
   if (!is_last) return;
-  __threadfence();
-  if (T * k <= 32) {
-    if ((threadIdx.x >> 5) == 0) permute_warp(ids, T * k, E, offsets, sorted_rows, inv, active, err);
-  } else {
-    permute_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, reinterpret_cast<int*>(sm_raw), warp_tot,
-                  &total);
-  }
+  int* ism = reinterpret_cast<int*>(sm_raw);
+  permute_ranks_block(ids, T * k, E, offsets, sorted_rows, inv, active, err, ism, ism + T * k);
   if (threadIdx.x == 0) *counter = 0;
+  (void)warp_tot;
+  (void)total;
 }
 
 }  // namespace moe
