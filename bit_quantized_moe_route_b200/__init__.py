@@ -4,6 +4,9 @@ The compute lives in ``libmoe_lowbit.so`` (hand-written CUDA for sm_100a,
 C ABI in ``include/moe_lowbit.h``); this package is its thin Python binding.
 """
 from ._lib import (  # noqa: F401
+    FFN_AUTO,
+    FFN_GEMV,
+    FFN_TENSOR_CORE,
     FMT_AFFINE,
     FMT_MXFP4,
     LIB_PATH,
@@ -22,6 +25,7 @@ from ._lib import (  # noqa: F401
     qmat,
     read_device_error,
     route,
+    set_ffn_path,
     set_timing_events,
     status_string,
     timing_labels,

@@ -64,6 +64,7 @@ _SIGS = {
     "moe_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
     "moe_timing_count": (ctypes.c_int32, []),
     "moe_timing_label": (ctypes.c_char_p, [ctypes.c_int32]),
+    "moe_set_ffn_path": (ctypes.c_int32, [ctypes.c_int32]),
 }
 
 
@@ -201,6 +202,18 @@ def read_device_error(ws, stream=None) -> int:
     _check(load_library().moe_read_device_error(_ptr(ws), ctypes.byref(code), _stream(stream)),
            "moe_read_device_error")
     return code.value
+
+
+FFN_AUTO, FFN_GEMV, FFN_TENSOR_CORE = 0, 1, 2
+
+
+def set_ffn_path(path: int) -> int:
+    """Select the expert-FFN implementation (FFN_AUTO / FFN_GEMV /
+    FFN_TENSOR_CORE) for this process; returns the previous setting."""
+    prev = load_library().moe_set_ffn_path(int(path))
+    if prev < 0:
+        raise ValueError(f"unknown FFN path {path}")
+    return prev
 
 
 def status_string(status: int) -> str:

@@ -16,6 +16,7 @@
 #include "stream_types.cuh"
 #include "permute.cuh"
 #include "route.cuh"
+#include "tc_prep.cuh"
 
 using namespace moe;
 
@@ -86,7 +87,10 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-  size_t hdr, logits, ids, wts, offsets, sorted, inv, active, h, y, xstage, tokstage, outstage, total;
+  size_t hdr, logits, ids, wts, offsets, sorted, inv, active, h, y, xstage, tokstage, outstage;
+  size_t x16, tiles, ntiles;  // tensor-core FFN: fp16 activations, token-tile plan
+  bool tc = false;            // the regions above exist
+  size_t total;
 };
 
 int f_max_of(const moe_dims_t& d) { return std::max(d.d_ff, d.d_ff_shared); }
@@ -115,6 +119,10 @@ WsLayout layout_of(const moe_dims_t& d) {
   L.xstage = take(T * D * 2);
   L.tokstage = take(T * sizeof(int));
   L.outstage = take(T * D * 2);
+  L.x16 = take(T * D * 2);
+  L.tiles = take(((T * k + kTcN - 1) / kTcN + E) * sizeof(int4));
+  L.ntiles = take(sizeof(int));
+  L.tc = true;
   L.total = o;
   return L;
 }
@@ -199,6 +207,7 @@ moe_status_t check_qmat(const moe_qmat_t* m, int n_in, const char* name, QMatDev
 }
 
 extern const StreamAttrFn kStreamAttrs[10];
+extern const TcAttrFn kTcAttrs[10];
 
 struct DevInfo {
   int sms = 0;
@@ -226,6 +235,7 @@ moe_status_t dev_info(DevInfo** out) {
       cudaFuncSetAttribute(route_hash_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
       cudaFuncSetAttribute(route_hash_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
       for (StreamAttrFn f : kStreamAttrs) f();
+      for (TcAttrFn f : kTcAttrs) f();
       int b1 = 0, b2 = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, ffn_gemv_kernel<1, 4>, kFfnThreads, 0);
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, ffn_gemv_kernel<2, 8>, kFfnThreads, 0);
@@ -401,6 +411,107 @@ int stream_cpl(int ntmax, int n_in_a, int n_in_b) {
   return 0;
 }
 
+// Tensor-core launchers indexed by format code (F_A2..F_MX4).
+const TcLaunchFn kTcLaunch[2][5] = {
+    {launch_tc_s1_A2, launch_tc_s1_A3, launch_tc_s1_A4, launch_tc_s1_A8, launch_tc_s1_MX4},
+    {launch_tc_s2_A2, launch_tc_s2_A3, launch_tc_s2_A4, launch_tc_s2_A8, launch_tc_s2_MX4}};
+const TcAttrFn kTcAttrs[10] = {attrs_tc_s1_A2, attrs_tc_s1_A3, attrs_tc_s1_A4, attrs_tc_s1_A8, attrs_tc_s1_MX4,
+                               attrs_tc_s2_A2, attrs_tc_s2_A3, attrs_tc_s2_A4, attrs_tc_s2_A8, attrs_tc_s2_MX4};
+
+std::atomic<int> g_ffn_path{MOE_FFN_AUTO};
+
+// The tensor-core kernel tiles 128 output rows x 64 inputs.
+bool tc_shape_ok(const QMatDev& A) { return A.n_out % kTcM == 0 && A.n_in % kTcK == 0; }
+
+// Tensor-core path for the expert FFN: chosen for large batches (on average
+// at least 32 tokens per active expert) or when forced, if the workspace has
+// its regions and every matrix has a supported shape.
+bool use_tc(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w2, const QMatDev* sh, const WsLayout& L) {
+  const int mode = g_ffn_path.load(std::memory_order_relaxed);
+  if (mode == MOE_FFN_GEMV || !L.tc) return false;
+  if (!tc_shape_ok(w1) || !tc_shape_ok(w2) || (sh && (!tc_shape_ok(sh[0]) || !tc_shape_ok(sh[2])))) return false;
+  if (mode == MOE_FFN_TENSOR_CORE) return true;
+  const long long Tk = (long long)d.T * d.top_k;
+  return Tk >= 32LL * std::min<long long>(d.n_experts, Tk);
+}
+
+moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offsets, const int* sorted,
+                           const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh,
+                           float* y, int ld_y, void* ws, const WsLayout& L, cudaStream_t s, const DevInfo& di) {
+  const int Tk = d.T * d.top_k;
+  int* err = &ws_at<WsHeader>(ws, L.hdr)->err;
+  __half* x16 = ws_at<__half>(ws, L.x16);
+  __half* h16 = ws_at<__half>(ws, L.h);
+  const int ld_h = f_max_of(d);
+  {
+    const size_t n8 = (size_t)d.T * d.d_model / 8;
+    const int grid = (int)std::min<size_t>((n8 + 255) / 256, (size_t)di.sms * 4);
+    tc_x_to_f16_kernel<<<std::max(grid, 1), 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(x), x16, n8, err);
+    MOE_CHECK_LAUNCH("tc_x_to_f16_kernel");
+    hook_mark(s, "x_to_f16");
+    tc_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.n_experts, ws_at<int4>(ws, L.tiles), ws_at<int>(ws, L.ntiles));
+    MOE_CHECK_LAUNCH("tc_plan_kernel");
+    hook_mark(s, "tile_plan");
+  }
+  TcParams p{};
+  p.x16 = x16;
+  p.T = d.T;
+  p.k = d.top_k;
+  p.tiles = ws_at<int4>(ws, L.tiles);
+  p.n_tiles = ws_at<int>(ws, L.ntiles);
+  p.err = err;
+  const int n_shared_tiles = (d.T + kTcN - 1) / kTcN;
+  // stage 1: H = silu(x W1^T) * (x W3^T) -> fp16 rows of the h region
+  {
+    TcParams q = p;
+    q.hout = h16;
+    q.ld_h = ld_h;
+    q.a0 = w1;
+    q.a1 = w3;
+    q.sorted_rows = sorted;
+    q.pos_base = 0;
+    if (!kTcLaunch[0][w1.fmt](q, di.sms, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
+    MOE_CHECK_LAUNCH("ffn_tc_kernel<1>");
+    hook_mark(s, "ffn_w13_swiglu");
+    if (sh) {
+      q.a0 = sh[0];
+      q.a1 = sh[1];
+      q.sorted_rows = nullptr;
+      q.pos_base = Tk;
+      const int grid = std::min(di.sms, n_shared_tiles * (sh[0].n_out / kTcM));
+      if (!kTcLaunch[0][sh[0].fmt](q, grid, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
+      MOE_CHECK_LAUNCH("ffn_tc_kernel<1> (shared)");
+      hook_mark(s, "ffn_w13_swiglu_shared");
+    }
+  }
+  // stage 2: y = H W2^T
+  {
+    TcParams q = p;
+    q.hin = h16;
+    q.ld_in = ld_h;
+    q.yout = y;
+    q.ld_y = ld_y;
+    q.a0 = w2;
+    q.a1 = w2;
+    q.sorted_rows = sorted;
+    q.pos_base = 0;
+    if (!kTcLaunch[1][w2.fmt](q, di.sms, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
+    MOE_CHECK_LAUNCH("ffn_tc_kernel<2>");
+    hook_mark(s, "ffn_w2");
+    if (sh) {
+      q.a0 = sh[2];
+      q.a1 = sh[2];
+      q.sorted_rows = nullptr;
+      q.pos_base = Tk;
+      const int grid = std::min(di.sms, n_shared_tiles * (sh[2].n_out / kTcM));
+      if (!kTcLaunch[1][sh[2].fmt](q, grid, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
+      MOE_CHECK_LAUNCH("ffn_tc_kernel<2> (shared)");
+      hook_mark(s, "ffn_w2_shared");
+    }
+  }
+  return MOE_OK;
+}
+
 // Stage 1 + stage 2 of the expert FFN (routed pairs, optional shared expert).
 moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, const int* sorted,
                         const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh,
@@ -408,6 +519,7 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
   DevInfo* di = nullptr;
   moe_status_t st = dev_info(&di);
   if (st != MOE_OK) return st;
+  if (use_tc(d, w1, w2, sh, L)) return launch_ffn_tc(d, x, offsets, sorted, w1, w3, w2, sh, y, ld_y, ws, L, s, *di);
   const int Tk = d.T * d.top_k;
   const int max_active = std::min(d.n_experts, Tk);
   float* h = ws_at<float>(ws, L.h);
@@ -583,6 +695,11 @@ const char* moe_status_string(moe_status_t s) {
 }
 
 const char* moe_last_error_detail(void) { return g_detail; }
+
+int32_t moe_set_ffn_path(int32_t path) {
+  if (path != MOE_FFN_AUTO && path != MOE_FFN_GEMV && path != MOE_FFN_TENSOR_CORE) return -1;
+  return g_ffn_path.exchange(path);
+}
 
 moe_status_t moe_set_timing_events(void* const* events, int32_t n_events) {
   g_hook = TimingHook{};

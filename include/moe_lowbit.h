@@ -47,6 +47,9 @@
  *   - Bad *data* (token id outside [0, vocab), tid2eid entry outside [0, E))
  *     never traps: the kernel records MOE_ERR_DEVICE_INPUT in the workspace
  *     error word, routes that slot to expert 0 with weight 0, and continues.
+ *     The tensor-core FFN path (step 3) records the same code when an
+ *     activation, hidden value or dequantised weight leaves the fp16 range
+ *     (|v| > 65504) that its tensor-core operands use.
  *   - A failed launch returns MOE_ERR_CUDA (the CUDA error is consumed and
  *     reported by moe_last_error_detail()).
  *   - Layouts are row-major.  Weights are stored [out, in] per expert and
@@ -69,7 +72,9 @@ typedef enum {
   MOE_ERR_WORKSPACE = 3,     /* workspace smaller than moe_workspace_size */
   MOE_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed       */
   MOE_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up         */
-  MOE_ERR_DEVICE_INPUT = 6   /* out-of-range token id / table entry seen   */
+  MOE_ERR_DEVICE_INPUT = 6   /* out-of-range token id / table entry, or a
+                                value outside fp16 range on the tensor-core
+                                FFN path                                    */
 } moe_status_t;
 
 typedef enum { MOE_FMT_AFFINE = 0, MOE_FMT_MXFP4 = 1 } moe_fmt_t;
@@ -170,6 +175,13 @@ moe_status_t moe_permute(const moe_dims_t* dims, const int32_t* topk_ids, int32_
  * with fp32 accumulation.  w1 and w3 must share one format.
  *   x : bf16 [T, d_model];  w1, w3 : [E, d_ff, d_model];  w2 : [E, d_model, d_ff]
  *   y : fp32 [T*k, d_model] (out) in sorted order.
+ * Two implementations (moe_set_ffn_path): a weight-streaming GEMV that
+ * dequantises in registers and keeps x and h in fp32, for small batches; and
+ * a tcgen05 grouped GEMM for large batches, whose operands are fp16 (x, the
+ * dequantised weights and h are each rounded once to fp16, 11-bit
+ * significand) with fp32 accumulation.  The tensor-core path needs d_ff and
+ * d_model to be multiples of 128; values beyond the fp16 range are reported
+ * as MOE_ERR_DEVICE_INPUT.
  */
 moe_status_t moe_expert_ffn(const moe_dims_t* dims, const void* x, const int32_t* expert_offsets,
                             const int32_t* sorted_rows, const moe_qmat_t* w1, const moe_qmat_t* w3,
@@ -258,6 +270,18 @@ moe_status_t moe_read_device_error(void* ws, int32_t* code_out, void* stream);
 moe_status_t moe_set_timing_events(void* const* events, int32_t n_events);
 int32_t moe_timing_count(void);
 const char* moe_timing_label(int32_t i);
+
+/*
+ * Expert-FFN implementation used by moe_expert_ffn / moe_forward /
+ * moe_forward_host (process-wide setting; not for the allocation-free entry
+ * point, which always streams).  AUTO (default) takes the tensor-core path
+ * when the batch averages at least 32 tokens per active expert
+ * (T*top_k >= 32*min(n_experts, T*top_k)) and the shapes allow it.
+ * Returns the previous setting, or -1 (setting unchanged) for an unknown
+ * value.
+ */
+typedef enum { MOE_FFN_AUTO = 0, MOE_FFN_GEMV = 1, MOE_FFN_TENSOR_CORE = 2 } moe_ffn_path_t;
+int32_t moe_set_ffn_path(int32_t path);
 
 /* Static description of a status code. */
 const char* moe_status_string(moe_status_t status);
