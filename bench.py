@@ -111,7 +111,7 @@ def kernel_work(inp, ids):
     work["combine"] = P * d * 4 + T * d * 2 + T * k * 8
     # tensor-core path: fp16 copy of x, tile plan, and fp16 H (the shared
     # expert runs as its own launches there)
-    work["x_to_f16"] = T * d * 4
+    work["gather_f16"] = T * d * 2 + P * d * 2 + T * k * 4
     work["tile_plan"] = (E + 1) * 4 + ((T * k + 127) // 128 + E) * 16
     work["ffn_w13_swiglu_shared"] = sh13 + T * d * 2 + T * fs * 2
     work["ffn_w2_shared"] = sh2 + T * fs * 2 + T * d * 4

@@ -55,14 +55,14 @@ constexpr int kTcBLook = 2;                // B copy groups in flight
 constexpr float kF16Max = 65504.f;
 
 struct TcParams {
-  const __half* x16;     // stage 1 input: token activations [T, n_in] fp16
+  const __half* x16;     // stage 1 input: token rows in position order [P, n_in] fp16
   const __half* hin;     // stage 2 input: H rows [P, ld_in] fp16
   __half* hout;          // stage 1 output: H [P, ld_h]
   float* yout;           // stage 2 output: y [P, ld_y]
   int ld_in, ld_h, ld_y;
   int T, k;
   QMatDev a0, a1;        // stage 1: w1, w3; stage 2: w2 (a1 = a0)
-  const int* sorted_rows;  // [T*k] flat indices t*k+j by expert; NULL: identity rows (shared expert)
+  const int* sorted_rows;  // routed launch: non-NULL (tiles from the plan); NULL: shared expert over T rows
   const int4* tiles;     // token tiles {expert, first position, tokens, 0} (routed)
   const int* n_tiles;    // number of routed token tiles (device)
   int pos_base;          // row offset of this launch's positions in H / y
@@ -505,19 +505,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
     const int c = q & 7, n0 = q >> 3;
     TcCursor cur;
     cur.init(p, n_items, n_mt);
-    // stage 1: token index of each of this thread's 16 rows, current and next item
-    int tok[16], tokn[16];
-    auto load_rows = [&](const int4& tl, int (&dst)[16]) {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int n = n0 + 8 * i;
-        dst[i] = (n < tl.z) ? (p.sorted_rows ? __ldcg(p.sorted_rows + tl.y + n) / p.k : tl.y + n) : 0;
-      }
-    };
-    if constexpr (STAGE == 1) {
-      load_rows(cur.tile, tok);
-      load_rows(cur.nxt, tokn);
-    }
+    const __half* rows = STAGE == 1 ? p.x16 : p.hin;
+    const int ld = STAGE == 1 ? n_in : p.ld_in;
     for (int g = 0; g < total; ++g) {
       const int s = g % S;
       const int round = g / S;
@@ -528,12 +517,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
       for (int i = 0; i < 16; ++i) {
         const int n = n0 + 8 * i;
         const bool live = n < cur.tile.z;
-        const __half* src;
-        if constexpr (STAGE == 1) {
-          src = p.x16 + (size_t)tok[i] * n_in + kofs;
-        } else {
-          src = p.hin + (size_t)(p.pos_base + cur.tile.y + (live ? n : 0)) * p.ld_in + kofs;
-        }
+        const __half* src = rows + (size_t)(p.pos_base + cur.tile.y + (live ? n : 0)) * ld + kofs;
         cp16z(bt + sw128(n, c), src, live ? 16u : 0u);
       }
       cp_commit();
@@ -542,13 +526,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) ffn_tc_kernel(const __grid_cons
         tc_fence_proxy();
         tc_bar_arrive(full_b((g - kTcBLook) % S));
       }
-      if (cur.advance(p, n_items, n_mt, n_kt)) {
-        if constexpr (STAGE == 1) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) tok[i] = tokn[i];
-          load_rows(cur.nxt, tokn);
-        }
-      }
+      cur.advance(p, n_items, n_mt, n_kt);
     }
     cp_wait<0>();
     tc_fence_proxy();

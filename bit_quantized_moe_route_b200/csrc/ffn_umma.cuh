@@ -1,0 +1,471 @@
+// Step 3 for large token counts (prefill), TMA + TMEM variant of the
+// tensor-core grouped SwiGLU expert FFN:
+//
+//   stage 1 (per expert e):  H[p, :] = silu(X[p] . W1[e]^T) * (X[p] . W3[e]^T)
+//   stage 2 (per expert e):  Y[p, :] = H[p] . W2[e]^T
+//
+// [mlx-lm PR "Add DeepSeek-v4 (Flash/Pro)": w1/w2/w3 = gate/down/up of the
+// switch MLP; model card "DeepSeek-V4-Flash-0731-MLX-Serve-mixed-2-3-8bit":
+// affine w = scale*q + bias; mxfp4 = e2m1 * 2^(e-127)].
+//
+// Data path of one block (persistent, one per SM):
+//   * packed codes and group scales/biases of the 128 weight rows of the
+//     current item arrive by TMA (2D boxes of 128 bytes x rows, 128-byte
+//     swizzle; 16-byte scale boxes) into a three-slot ring, one slot = 512
+//     inputs (256 for 8-bit codes), loaded two slots ahead;
+//   * the token rows (B operand, fp16, up to 224 per tile, gathered into
+//     expert order beforehand) arrive by TMA as 64-input K-major tiles with
+//     the 128-byte swizzle the tensor core reads directly (3-stage ring);
+//   * 8 dequant warps turn each 64-input stage of codes into fp16 weights and
+//     write them straight into tensor memory (tcgen05.st): the weights are
+//     the MMA's A operand in TMEM (two stage slots of 32 columns), so the
+//     shared memory only carries the token tiles and the packed codes;
+//   * one thread issues tcgen05.mma (A from TMEM, B from shared memory,
+//     fp32 accumulators in TMEM, double-buffered: 2 x 224 columns);
+//   * 4 epilogue warps read the accumulators (tcgen05.ld) and write H
+//     (SwiGLU, fp16) or y (fp32).
+// Stage 1 stacks 64 gate rows and the 64 up rows of the same features in
+// one 128-row tile: in every 32-lane TMEM quarter, lanes 0-15 hold W1 rows
+// and lanes 16-31 the W3 rows of the same 16 features, so the epilogue pairs
+// them with one warp shuffle.
+// Operands are fp16 (see ffn_tc.cuh for why); every wait is bounded.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "ffn_tc.cuh"
+
+namespace moe {
+
+constexpr int kUmN = 224;      // tokens per tile (MMA N <= 224, multiple of 16)
+constexpr int kUmK = 64;       // inputs per MMA stage
+constexpr int kUmThreads = 16 * 32;
+constexpr int kUmLoadWarp = 8;
+constexpr int kUmMmaWarp = 9;
+constexpr int kUmEpiWarp0 = 12;  // warps 12-15: warp % 4 = TMEM lane quarter
+constexpr int kUmBStages = 3;
+constexpr int kUmBTile = kUmN * 128;  // 224 rows x 64 fp16
+constexpr uint32_t kUmAccCol0 = 64;   // TMEM columns: A stage slots [0, 64), accumulators at 64 and 288
+constexpr uint32_t kUmAccCols = kUmN;
+constexpr uint32_t kUmTmemCols = 512;
+
+struct alignas(64) UmParams {
+  CUtensorMap b_map;     // B rows: fp16 [rows, n_in], box {64, 224}, 128B swizzle
+  CUtensorMap q_map[2];  // packed codes: uint8 [E*n_out, row bytes], box {128, R}, 128B swizzle
+  CUtensorMap s_map[2];  // scales: bf16 or e8m0 [E*n_out, groups], box {16 bytes, R}
+  CUtensorMap z_map[2];  // biases: bf16 (affine)
+  __half* hout;          // stage 1 output H [P, ld_h]
+  float* yout;           // stage 2 output y [P, ld_y]
+  int ld_h, ld_y;
+  int n_in, n_out;       // per-expert shape of each A matrix
+  int group;
+  int row_bytes, gpr;    // packed bytes and scale groups per weight row
+  int T;                 // shared expert: tokens
+  int shared;            // 1: one expert over positions 0..T-1 (no tile table)
+  const int4* tiles;     // routed token tiles {expert, first position, tokens, 0}
+  const int* n_tiles;
+  int pos_base;          // row of position 0 in the B tensor and in H / y
+  int* err;
+};
+
+template <int STAGE, int FMT>
+struct UmCfg {
+  static constexpr int bits = FMT == F_A2 ? 2 : FMT == F_A8 ? 8 : 4;
+  static constexpr bool mx = FMT == F_MX4;
+  static constexpr int M = STAGE == 1 ? 2 : 1;          // matrices stacked in one tile
+  static constexpr int R = 128 / M;                     // rows per matrix per tile
+  static constexpr int KS = bits == 8 ? 256 : 512;      // inputs per raw slot
+  static constexpr int QS = KS / kUmK;                  // MMA stages per raw slot
+  static constexpr int NPB = KS * bits / 8 / 128;       // 128-byte packed boxes per matrix per slot
+  static constexpr int PBOX = R * 128;
+  static constexpr int SBOX = R * 16;
+  static constexpr int NSB = 2;                         // scale boxes reserved per matrix per slot
+  static constexpr int packed_bytes = NPB * M * PBOX;
+  static constexpr int scale_bytes = NSB * M * SBOX;
+  static constexpr int slot_bytes = packed_bytes + 2 * scale_bytes;  // codes, scales, biases
+  static constexpr int GBOX = mx ? 16 : 8;              // groups per 16-byte scale box
+  static constexpr int ESZ = mx ? 1 : 2;                // scale element bytes
+  static constexpr int NRS = 3;                         // raw slots
+  static constexpr size_t smem = 1024 + NRS * (size_t)slot_bytes + (size_t)kUmBStages * kUmBTile + 256;
+  static_assert(FMT != F_A3, "3-bit codes take the per-thread-copy kernel");
+  static_assert(slot_bytes % 1024 == 0, "raw slots keep the 1024-byte alignment of the swizzled boxes");
+  static_assert(smem <= 227 * 1024, "TMA/TMEM FFN exceeds the per-block shared memory limit");
+};
+
+// ------------------------------------------------------------ PTX wrappers
+MOE_DEV void um_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// 2D tiled TMA load (no multicast) completing on `bar`
+MOE_DEV void um_tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+// this thread's 16 consecutive 32-bit TMEM columns of its lane
+MOE_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// D[tmem] (+)= A[tmem] . B[smem]^T, fp16 inputs, fp32 accumulation
+MOE_DEV void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+MOE_DEV uint32_t um_lds16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+MOE_DEV uint32_t um_lds8(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+
+// ------------------------------------------------------------ work items
+MOE_DEV int4 um_tile(const UmParams& p, int j) {
+  if (p.shared) {
+    const int pos0 = j * kUmN;
+    return make_int4(0, pos0, min(kUmN, p.T - pos0), 0);
+  }
+  return __ldcg(p.tiles + j);
+}
+
+// Walks this block's items (blockIdx.x, +gridDim.x, ...), each in n_sub
+// sub-steps (k-stages or raw slots), with the next item's tile loaded ahead.
+struct UmCursor {
+  int item, sub, mt;
+  int4 tile, nxt;
+  MOE_DEV void init(const UmParams& p, int n_items, int n_mt) {
+    item = blockIdx.x;
+    sub = 0;
+    mt = item % n_mt;
+    tile = item < n_items ? um_tile(p, item / n_mt) : make_int4(0, 0, 0, 0);
+    const int n2 = item + gridDim.x;
+    nxt = n2 < n_items ? um_tile(p, n2 / n_mt) : make_int4(0, 0, 0, 0);
+  }
+  MOE_DEV void next_item(const UmParams& p, int n_items, int n_mt) {
+    sub = 0;
+    item += gridDim.x;
+    mt = item % n_mt;
+    tile = nxt;
+    const int n2 = item + gridDim.x;
+    if (n2 < n_items) nxt = um_tile(p, n2 / n_mt);
+  }
+  MOE_DEV void advance(const UmParams& p, int n_items, int n_mt, int n_sub) {
+    if (++sub == n_sub) next_item(p, n_items, n_mt);
+  }
+};
+
+// ------------------------------------------------------------ the kernel
+template <int STAGE, int FMT>
+__global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_constant__ UmParams p) {
+  using C = UmCfg<STAGE, FMT>;
+  constexpr int M = C::M, QS = C::QS;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw32 = tc_smem(smem_raw);
+  const uint32_t base = (raw32 + 1023u) & ~1023u;  // swizzled boxes need 1024-byte alignment
+  constexpr int NRS = C::NRS;
+  const uint32_t slot0 = base;                      // raw slots: [codes | scales | biases] x NRS
+  const uint32_t bt0 = base + (uint32_t)(NRS * C::slot_bytes);  // B stages
+  const uint32_t bar = bt0 + (uint32_t)(kUmBStages * kUmBTile);
+  uint8_t* bar_gen = smem_raw + (bar - raw32);
+  auto raw_full = [&](int s) { return bar + 8u * s; };           // [3] TMA bytes
+  auto raw_empty = [&](int s) { return bar + 8u * (3 + s); };    // [3] 8 dequant warps
+  auto b_full = [&](int s) { return bar + 8u * (6 + s); };       // [3] TMA bytes
+  auto b_empty = [&](int s) { return bar + 8u * (9 + s); };      // [3] MMA commit
+  auto a_full = [&](int s) { return bar + 8u * (12 + s); };      // [2] 8 dequant warps
+  auto a_empty = [&](int s) { return bar + 8u * (14 + s); };     // [2] MMA commit
+  auto acc_full = [&](int s) { return bar + 8u * (16 + s); };    // [2] MMA commit
+  auto acc_empty = [&](int s) { return bar + 8u * (18 + s); };   // [2] 4 epilogue warps
+  const uint32_t drain = bar + 8u * 20;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_gen + 8 * 21);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_mt = p.n_out / (STAGE == 1 ? 64 : 128);
+  const int n_kt = p.n_in / kUmK;
+  const int n_rng = (n_kt + QS - 1) / QS;
+  const int n_tiles = p.shared ? (p.T + kUmN - 1) / kUmN : __ldcg(p.n_tiles);
+  const int n_items = n_tiles * n_mt;
+  const int my_items = (int)blockIdx.x < n_items ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int total = my_items * n_kt;
+  const int nsb = C::mx ? 1 : max(1, C::KS / p.group / 8);  // scale boxes per matrix per slot
+
+  if (tid == 0) {
+    for (int s = 0; s < NRS; ++s) {
+      tc_bar_init(raw_full(s), 1);
+      tc_bar_init(raw_empty(s), 8);
+    }
+    for (int s = 0; s < 2; ++s) {
+      tc_bar_init(a_full(s), 8);
+      tc_bar_init(a_empty(s), 1);
+      tc_bar_init(acc_full(s), 1);
+      tc_bar_init(acc_empty(s), 4);
+    }
+    for (int s = 0; s < kUmBStages; ++s) {
+      tc_bar_init(b_full(s), 1);
+      tc_bar_init(b_empty(s), 1);
+    }
+    tc_bar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kUmMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc_smem(tmem_slot)),
+                 "r"(kUmTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp < 8) {
+    // ================= dequant warps: TMEM lane quarter q, input half kh
+    const int q = warp & 3, kh = warp >> 2;
+    const int m = STAGE == 1 ? (lane >> 4) : 0;                  // matrix of this lane's row
+    const int rr = STAGE == 1 ? 16 * q + (lane & 15) : 32 * q + lane;  // row within that matrix's box
+    UmCursor cur;
+    cur.init(p, n_items, n_mt);
+    int rc = 0;  // raw slots consumed
+    bool bad = false;
+    for (int g = 0; g < total; ++g) {
+      const int kt = cur.sub, qs = kt % QS, ri = kt / QS;
+      const int rs = rc % NRS;
+      bool ok = true;
+      if (qs == 0) ok = tc_bar_wait(raw_full(rs), (uint32_t)(rc / NRS) & 1u, abort_flag);
+      const int as = g & 1;
+      if (ok && g >= 2) ok = tc_bar_wait(a_empty(as), (uint32_t)((g >> 1) - 1) & 1u, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.st below is warp-collective
+      const uint32_t slot = slot0 + (uint32_t)(rs * C::slot_bytes);
+      // this thread's 32 codes: inputs ko .. ko+31 of the slot
+      const int ko = qs * kUmK + kh * 32;
+      const int bo = ko * C::bits / 8;
+      const uint32_t prow = slot + (uint32_t)(((bo >> 7) * M + m) * C::PBOX + rr * 128);
+      const int j = (bo & 127) >> 4;
+      uint32_t w[8];
+      if constexpr (C::bits == 8) {
+        const uint4 v0 = tc_lds128(prow + (uint32_t)((j ^ (rr & 7)) << 4));
+        const uint4 v1 = tc_lds128(prow + (uint32_t)(((j + 1) ^ (rr & 7)) << 4));
+        w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+        w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+      } else if constexpr (C::bits == 4) {
+        const uint4 v0 = tc_lds128(prow + (uint32_t)((j ^ (rr & 7)) << 4));
+        w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+      } else {
+        const uint2 v0 = tc_lds64(prow + (uint32_t)((j ^ (rr & 7)) << 4) + (uint32_t)(bo & 15));
+        w[0] = v0.x; w[1] = v0.y;
+      }
+      // this thread's group scale (and bias)
+      const int g_first = ri * C::KS / p.group;
+      const int x0 = g_first / C::GBOX * C::GBOX;
+      const int gi = (ri * C::KS + ko) / p.group - x0;
+      const uint32_t saddr = slot + (uint32_t)(C::packed_bytes + ((gi / C::GBOX) * M + m) * C::SBOX + rr * 16 +
+                                               (gi % C::GBOX) * C::ESZ);
+      uint32_t out[16];
+      if constexpr (C::mx) {
+        const uint32_t e = um_lds8(saddr);
+        uint32_t f = 0;  // 2^(e-113) in fp16 (see tc_dequant32_mx)
+        if (e > 128) bad = true;
+        else if (e >= 99) f = (e - 98u) << 10;
+        tc_dequant32_mx(w, f | (f << 16), out);
+      } else {
+        const float sf = __uint_as_float(um_lds16(saddr) << 16);
+        const float bf = __uint_as_float(um_lds16(saddr + C::scale_bytes) << 16);
+        if (!(fabsf(sf) * (float)((1 << C::bits) - 1) + fabsf(bf) <= kF16Max)) bad = true;
+        const __half hs = __float2half_rn(sf), hb = __float2half_rn(bf);
+        tc_dequant32<FMT>(w, h2u(__halves2half2(hs, hs)), h2u(__halves2half2(hb, hb)), out);
+      }
+      tmem_st16(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(as * 32 + kh * 16), out);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc_bar_arrive(a_full(as));
+      if (qs == QS - 1 || kt == n_kt - 1) {  // last use of this raw slot
+        if (lane == 0) tc_bar_arrive(raw_empty(rs));
+        ++rc;
+      }
+      cur.advance(p, n_items, n_mt, n_kt);
+    }
+    if (bad) set_error(p.err, kErrDeviceInput);
+  } else if (warp == kUmLoadWarp) {
+    // ================= TMA issuer
+    if (lane == 0) {
+      UmCursor cur, rcur;  // B stages; raw slots (two ahead)
+      cur.init(p, n_items, n_mt);
+      rcur = cur;
+      int rc = 0;
+      const int m_rows = STAGE == 1 ? 64 : 128;
+      auto issue_raw = [&]() -> bool {  // slot for (rcur.item, rcur.sub = range)
+        const int rs = rc % NRS;
+        if (rc >= NRS && !tc_bar_wait(raw_empty(rs), (uint32_t)(rc / NRS - 1) & 1u, abort_flag)) return false;
+        const uint32_t slot = slot0 + (uint32_t)(rs * C::slot_bytes);
+        const int ri = rcur.sub;
+        const int row = rcur.tile.x * p.n_out + rcur.mt * m_rows;
+        const int xp = ri * C::KS * C::bits / 8;
+        const int x0 = ri * C::KS / p.group / C::GBOX * C::GBOX;
+        // boxes that start past the end of a row are not loaded (nothing reads them)
+        const int np = min(C::NPB, (p.row_bytes - xp + 127) / 128);
+        const int ns = min(nsb, (p.gpr - x0 + C::GBOX - 1) / C::GBOX);
+        um_expect_tx(raw_full(rs), (uint32_t)(M * (np * C::PBOX + ns * C::SBOX * (C::mx ? 1 : 2))));
+#pragma unroll
+        for (int mm = 0; mm < M; ++mm) {
+          for (int b = 0; b < np; ++b)
+            um_tma_2d(slot + (uint32_t)((b * M + mm) * C::PBOX), &p.q_map[mm], xp + b * 128, row, raw_full(rs));
+          for (int sb = 0; sb < ns; ++sb) {
+            const uint32_t so = slot + (uint32_t)(C::packed_bytes + (sb * M + mm) * C::SBOX);
+            um_tma_2d(so, &p.s_map[mm], x0 + sb * C::GBOX, row, raw_full(rs));
+            if constexpr (!C::mx) um_tma_2d(so + C::scale_bytes, &p.z_map[mm], x0 + sb * C::GBOX, row, raw_full(rs));
+          }
+        }
+        ++rc;
+        rcur.advance(p, n_items, n_mt, n_rng);
+        return true;
+      };
+      int raw_issued = 0;
+      const int raw_total = my_items * n_rng;
+      for (int r = 0; r < NRS - 1 && raw_issued < raw_total; ++r)
+        if (issue_raw()) ++raw_issued;
+      for (int g = 0; g < total; ++g) {
+        const int kt = cur.sub;
+        if (kt % QS == 0 && raw_issued < raw_total) {  // keep the raw ring two slots ahead
+          if (!issue_raw()) break;
+          ++raw_issued;
+        }
+        const int bs = g % kUmBStages;
+        const int round = g / kUmBStages;
+        if (round > 0 && !tc_bar_wait(b_empty(bs), (uint32_t)(round - 1) & 1u, abort_flag)) break;
+        um_expect_tx(b_full(bs), (uint32_t)kUmBTile);
+        um_tma_2d(bt0 + (uint32_t)(bs * kUmBTile), &p.b_map, kt * kUmK, p.pos_base + cur.tile.y, b_full(bs));
+        cur.advance(p, n_items, n_mt, n_kt);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kUmMmaWarp) {
+    // ================= MMA issuer
+    if (lane == 0) {
+      UmCursor cur;
+      cur.init(p, n_items, n_mt);
+      int g = 0;
+      for (int it = 0; it < my_items && !*abort_flag; ++it) {
+        const uint32_t idesc = umma_idesc_f16((cur.tile.z + 15) & ~15);
+        const int ab = it & 1;
+        if (it >= 2 && !tc_bar_wait(acc_empty(ab), (uint32_t)((it >> 1) - 1) & 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + kUmAccCol0 + (uint32_t)ab * kUmAccCols;
+        bool ok = true;
+        for (int kt = 0; kt < n_kt; ++kt, ++g) {
+          const int as = g & 1, bs = g % kUmBStages;
+          if (!tc_bar_wait(a_full(as), (uint32_t)(g >> 1) & 1u, abort_flag) ||
+              !tc_bar_wait(b_full(bs), (uint32_t)(g / kUmBStages) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t bt = bt0 + (uint32_t)(bs * kUmBTile);
+#pragma unroll
+          for (int kk = 0; kk < kUmK / 16; ++kk)  // K = 16 per MMA: 8 TMEM columns of A, 32 bytes of B
+            umma_f16_ts(d, tmem_base + (uint32_t)(as * 32 + kk * 8), umma_desc(bt + 32u * kk), idesc,
+                        (kt | kk) ? 1u : 0u);
+          umma_commit(a_empty(as));
+          umma_commit(b_empty(bs));
+        }
+        if (!ok) break;
+        umma_commit(acc_full(ab));
+        cur.next_item(p, n_items, n_mt);
+      }
+      umma_commit(drain);
+      const long long t0 = clock64();
+      while (!tc_bar_try(drain, 0) && clock64() - t0 < kTcWaitCycles) {
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kUmEpiWarp0) {
+    // ================= epilogue
+    const int q = warp & 3;
+    UmCursor cur;
+    cur.init(p, n_items, n_mt);
+    bool bad = false;
+    for (int it = 0; it < my_items; ++it) {
+      const int ab = it & 1;
+      const bool ok = tc_bar_wait(acc_full(ab), (uint32_t)(it >> 1) & 1u, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld is warp-collective
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + kUmAccCol0 + (uint32_t)ab * kUmAccCols;
+      const int ntok = cur.tile.z;
+      const int prow0 = p.pos_base + cur.tile.y;
+      for (int nb = 0; nb < ntok; nb += 16) {
+        float v[16];
+        tmem_ld16(taddr + (uint32_t)nb, v);
+        if constexpr (STAGE == 1) {
+          // lanes 0-15: gate of features f, lanes 16-31: up of the same f;
+          // the low half finishes token columns 0-7, the high half 8-15
+          const bool lo = lane < 16;
+          const int f = cur.mt * 64 + 16 * q + (lane & 15);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const float send = lo ? v[8 + jj] : v[jj];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+            const float gv = lo ? v[jj] : recv;
+            const float uv = lo ? recv : v[8 + jj];
+            const int n = nb + (lo ? jj : 8 + jj);
+            if (n < ntok) {
+              const float hv = __fdividef(gv * uv, 1.f + __expf(-gv));  // silu(g) * u
+              bad |= !(fabsf(hv) <= kF16Max);
+              p.hout[(size_t)(prow0 + n) * p.ld_h + f] = __float2half_rn(hv);
+            }
+          }
+        } else {
+          const int row = cur.mt * 128 + 32 * q + lane;
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            if (nb + jj < ntok) p.yout[(size_t)(prow0 + nb + jj) * p.ld_y + row] = v[jj];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc_bar_arrive(acc_empty(ab));
+      cur.next_item(p, n_items, n_mt);
+    }
+    if (bad) set_error(p.err, kErrDeviceInput);
+  }
+  __syncthreads();
+  if (tid == 0 && *abort_flag) set_error(p.err, kErrTimeout);
+  if (warp == kUmMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kUmTmemCols)
+                 : "memory");
+  }
+}
+
+// Launch helpers, one translation unit per (stage, format).
+using UmLaunchFn = bool (*)(const UmParams& p, int grid, cudaStream_t s);
+using UmAttrFn = void (*)();
+#define MOE_UM_DECL(ST, F)                                                 \
+  bool launch_um_s##ST##_##F(const UmParams& p, int grid, cudaStream_t s); \
+  void attrs_um_s##ST##_##F();
+MOE_UM_DECL(1, A2)
+MOE_UM_DECL(1, A4)
+MOE_UM_DECL(1, A8)
+MOE_UM_DECL(1, MX4)
+MOE_UM_DECL(2, A2)
+MOE_UM_DECL(2, A4)
+MOE_UM_DECL(2, A8)
+MOE_UM_DECL(2, MX4)
+#undef MOE_UM_DECL
+
+}  // namespace moe

@@ -17,6 +17,9 @@
 #include "permute.cuh"
 #include "route.cuh"
 #include "tc_prep.cuh"
+#include "ffn_umma.cuh"
+
+#include <cudaTypedefs.h>
 
 using namespace moe;
 
@@ -88,7 +91,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
   size_t hdr, logits, ids, wts, offsets, sorted, inv, active, h, y, xstage, tokstage, outstage;
-  size_t x16, tiles, ntiles;  // tensor-core FFN: fp16 activations, token-tile plan
+  size_t x16, tiles, tiles2, ntiles;  // tensor-core FFN: fp16 token rows by position, token-tile plans
   bool tc = false;            // the regions above exist
   size_t total;
 };
@@ -119,9 +122,10 @@ WsLayout layout_of(const moe_dims_t& d) {
   L.xstage = take(T * D * 2);
   L.tokstage = take(T * sizeof(int));
   L.outstage = take(T * D * 2);
-  L.x16 = take(T * D * 2);
+  L.x16 = take(P * D * 2);
   L.tiles = take(((T * k + kTcN - 1) / kTcN + E) * sizeof(int4));
-  L.ntiles = take(sizeof(int));
+  L.tiles2 = take(((T * k + kUmN - 1) / kUmN + E) * sizeof(int4));
+  L.ntiles = take(2 * sizeof(int));
   L.tc = true;
   L.total = o;
   return L;
@@ -208,6 +212,7 @@ moe_status_t check_qmat(const moe_qmat_t* m, int n_in, const char* name, QMatDev
 
 extern const StreamAttrFn kStreamAttrs[10];
 extern const TcAttrFn kTcAttrs[10];
+extern const UmAttrFn kUmAttrs[8];
 
 struct DevInfo {
   int sms = 0;
@@ -236,6 +241,7 @@ moe_status_t dev_info(DevInfo** out) {
       cudaFuncSetAttribute(route_hash_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
       for (StreamAttrFn f : kStreamAttrs) f();
       for (TcAttrFn f : kTcAttrs) f();
+      for (UmAttrFn f : kUmAttrs) f();
       int b1 = 0, b2 = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, ffn_gemv_kernel<1, 4>, kFfnThreads, 0);
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, ffn_gemv_kernel<2, 8>, kFfnThreads, 0);
@@ -435,80 +441,159 @@ bool use_tc(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w2, const QMa
   return Tk >= 32LL * std::min<long long>(d.n_experts, Tk);
 }
 
+// TMA/TMEM kernels indexed by format code (no 3-bit instance).
+const UmLaunchFn kUmLaunch[2][5] = {
+    {launch_um_s1_A2, nullptr, launch_um_s1_A4, launch_um_s1_A8, launch_um_s1_MX4},
+    {launch_um_s2_A2, nullptr, launch_um_s2_A4, launch_um_s2_A8, launch_um_s2_MX4}};
+const UmAttrFn kUmAttrs[8] = {attrs_um_s1_A2, attrs_um_s1_A4, attrs_um_s1_A8, attrs_um_s1_MX4,
+                              attrs_um_s2_A2, attrs_um_s2_A4, attrs_um_s2_A8, attrs_um_s2_MX4};
+
+// cuTensorMapEncodeTiled from the driver, looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    cudaGetLastError();
+  });
+  return g_encode;
+}
+
+// 2D tensor map: dim0 (contiguous) x dim1 rows, row stride in bytes, box b0 x b1.
+moe_status_t tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t dim0, uint64_t dim1,
+                     uint64_t stride, uint32_t b0, uint32_t b1, bool swizzle128) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {dim0, dim1};
+  const cuuint64_t strides[1] = {stride};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t es[2] = {1, 1};
+  const CUresult r = enc(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MOE_OK;
+}
+
+// Shapes the TMA/TMEM kernel takes: 2/4/8-bit affine or mxfp4 codes, rows of
+// a multiple of 16 bytes, scale rows of a multiple of 16 bytes (the TMA
+// stride rule), 64 (stage 1) or 128 (stage 2) output rows per tile.
+bool um_ok(const QMatDev& Q, int stage) {
+  if (Q.fmt == F_A3) return false;
+  if (Q.n_in % kUmK || Q.n_out % (stage == 1 ? 64 : 128)) return false;
+  if ((Q.wpr * 4) % 16) return false;
+  if (Q.group != 32 && Q.group != 64 && Q.group != 128) return false;
+  return Q.fmt == F_MX4 ? Q.gpr % 16 == 0 : (Q.gpr * 2) % 16 == 0;
+}
+
+// Packed-code, scale and bias maps of matrix Q (E experts) for slot m.
+moe_status_t um_weight_maps(UmParams& p, int m, const QMatDev& Q, int E, int rows_per_box) {
+  const uint64_t rows = (uint64_t)E * Q.n_out;
+  moe_status_t st = tmap_2d(&p.q_map[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.q, (uint64_t)Q.wpr * 4, rows,
+                            (uint64_t)Q.wpr * 4, 128, rows_per_box, true);
+  if (st != MOE_OK) return st;
+  if (Q.fmt == F_MX4)
+    return tmap_2d(&p.s_map[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.scales, Q.gpr, rows, Q.gpr, 16, rows_per_box, false);
+  st = tmap_2d(&p.s_map[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q.scales, Q.gpr, rows, (uint64_t)Q.gpr * 2, 8,
+               rows_per_box, false);
+  if (st != MOE_OK) return st;
+  return tmap_2d(&p.z_map[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q.biases, Q.gpr, rows, (uint64_t)Q.gpr * 2, 8,
+                 rows_per_box, false);
+}
+
 moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offsets, const int* sorted,
                            const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh,
                            float* y, int ld_y, void* ws, const WsLayout& L, cudaStream_t s, const DevInfo& di) {
   const int Tk = d.T * d.top_k;
+  const int P = Tk + (sh ? d.T : 0);
   int* err = &ws_at<WsHeader>(ws, L.hdr)->err;
-  __half* x16 = ws_at<__half>(ws, L.x16);
+  __half* xs = ws_at<__half>(ws, L.x16);
   __half* h16 = ws_at<__half>(ws, L.h);
   const int ld_h = f_max_of(d);
+  int* n_tiles = ws_at<int>(ws, L.ntiles);
   {
-    const size_t n8 = (size_t)d.T * d.d_model / 8;
-    const int grid = (int)std::min<size_t>((n8 + 255) / 256, (size_t)di.sms * 4);
-    tc_x_to_f16_kernel<<<std::max(grid, 1), 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(x), x16, n8, err);
-    MOE_CHECK_LAUNCH("tc_x_to_f16_kernel");
-    hook_mark(s, "x_to_f16");
-    tc_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.n_experts, ws_at<int4>(ws, L.tiles), ws_at<int>(ws, L.ntiles));
+    const size_t n8 = (size_t)P * d.d_model / 8;
+    const int grid = (int)std::min<size_t>((n8 + 255) / 256, (size_t)di.sms * 8);
+    tc_gather_f16_kernel<<<std::max(grid, 1), 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(x), sorted,
+                                                           d.top_k, Tk, d.T, d.d_model, sh ? 1 : 0, xs, err);
+    MOE_CHECK_LAUNCH("tc_gather_f16_kernel");
+    hook_mark(s, "gather_f16");
+    tc_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.n_experts, kTcN, ws_at<int4>(ws, L.tiles), n_tiles, kUmN,
+                                      ws_at<int4>(ws, L.tiles2), n_tiles + 1);
     MOE_CHECK_LAUNCH("tc_plan_kernel");
     hook_mark(s, "tile_plan");
   }
-  TcParams p{};
-  p.x16 = x16;
-  p.T = d.T;
-  p.k = d.top_k;
-  p.tiles = ws_at<int4>(ws, L.tiles);
-  p.n_tiles = ws_at<int>(ws, L.ntiles);
-  p.err = err;
-  const int n_shared_tiles = (d.T + kTcN - 1) / kTcN;
-  // stage 1: H = silu(x W1^T) * (x W3^T) -> fp16 rows of the h region
-  {
-    TcParams q = p;
-    q.hout = h16;
-    q.ld_h = ld_h;
-    q.a0 = w1;
-    q.a1 = w3;
-    q.sorted_rows = sorted;
-    q.pos_base = 0;
-    if (!kTcLaunch[0][w1.fmt](q, di.sms, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
-    MOE_CHECK_LAUNCH("ffn_tc_kernel<1>");
-    hook_mark(s, "ffn_w13_swiglu");
-    if (sh) {
-      q.a0 = sh[0];
-      q.a1 = sh[1];
-      q.sorted_rows = nullptr;
-      q.pos_base = Tk;
-      const int grid = std::min(di.sms, n_shared_tiles * (sh[0].n_out / kTcM));
-      if (!kTcLaunch[0][sh[0].fmt](q, grid, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
-      MOE_CHECK_LAUNCH("ffn_tc_kernel<1> (shared)");
-      hook_mark(s, "ffn_w13_swiglu_shared");
+  // One launch of stage `stage` for the routed experts (shared = nullptr) or
+  // the shared expert: the TMA/TMEM kernel when the shapes allow, else the
+  // per-thread-copy kernel.
+  auto run = [&](int stage, const QMatDev& a0, const QMatDev& a1, bool shared, const char* label) -> moe_status_t {
+    const int pos_base = shared ? Tk : 0;
+    const int E = shared ? 1 : d.n_experts;
+    if (um_ok(a0, stage) && um_ok(a1, stage)) {
+      UmParams q{};
+      moe_status_t st;
+      if (stage == 1)
+        st = tmap_2d(&q.b_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs, d.d_model, (uint64_t)P, (uint64_t)d.d_model * 2,
+                     kUmK, kUmN, true);
+      else
+        st = tmap_2d(&q.b_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h16, a0.n_in, (uint64_t)P, (uint64_t)ld_h * 2, kUmK,
+                     kUmN, true);
+      if (st != MOE_OK) return st;
+      if ((st = um_weight_maps(q, 0, a0, E, stage == 1 ? 64 : 128)) != MOE_OK) return st;
+      if (stage == 1 && (st = um_weight_maps(q, 1, a1, E, 64)) != MOE_OK) return st;
+      q.hout = h16;
+      q.yout = y;
+      q.ld_h = ld_h;
+      q.ld_y = ld_y;
+      q.n_in = a0.n_in;
+      q.n_out = a0.n_out;
+      q.group = a0.group;
+      q.row_bytes = a0.wpr * 4;
+      q.gpr = a0.gpr;
+      q.T = d.T;
+      q.shared = shared ? 1 : 0;
+      q.tiles = ws_at<int4>(ws, L.tiles2);
+      q.n_tiles = n_tiles + 1;
+      q.pos_base = pos_base;
+      q.err = err;
+      const int rows_per_item = stage == 1 ? 64 : 128;
+      const int grid = shared ? std::min(di.sms, (d.T + kUmN - 1) / kUmN * (a0.n_out / rows_per_item)) : di.sms;
+      if (!kUmLaunch[stage - 1][a0.fmt](q, grid, s)) return fail(MOE_ERR_UNSUPPORTED, "no TMA/TMEM kernel");
+    } else {
+      TcParams q{};
+      q.x16 = xs;
+      q.hin = h16;
+      q.ld_in = ld_h;
+      q.hout = h16;
+      q.ld_h = ld_h;
+      q.yout = y;
+      q.ld_y = ld_y;
+      q.T = d.T;
+      q.k = d.top_k;
+      q.a0 = a0;
+      q.a1 = a1;
+      q.sorted_rows = shared ? nullptr : sorted;
+      q.tiles = ws_at<int4>(ws, L.tiles);
+      q.n_tiles = n_tiles;
+      q.pos_base = pos_base;
+      q.err = err;
+      const int grid = shared ? std::min(di.sms, (d.T + kTcN - 1) / kTcN * (a0.n_out / kTcM)) : di.sms;
+      if (!kTcLaunch[stage - 1][a0.fmt](q, grid, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
     }
-  }
-  // stage 2: y = H W2^T
-  {
-    TcParams q = p;
-    q.hin = h16;
-    q.ld_in = ld_h;
-    q.yout = y;
-    q.ld_y = ld_y;
-    q.a0 = w2;
-    q.a1 = w2;
-    q.sorted_rows = sorted;
-    q.pos_base = 0;
-    if (!kTcLaunch[1][w2.fmt](q, di.sms, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
-    MOE_CHECK_LAUNCH("ffn_tc_kernel<2>");
-    hook_mark(s, "ffn_w2");
-    if (sh) {
-      q.a0 = sh[2];
-      q.a1 = sh[2];
-      q.sorted_rows = nullptr;
-      q.pos_base = Tk;
-      const int grid = std::min(di.sms, n_shared_tiles * (sh[2].n_out / kTcM));
-      if (!kTcLaunch[1][sh[2].fmt](q, grid, s)) return fail(MOE_ERR_UNSUPPORTED, "no tensor-core kernel");
-      MOE_CHECK_LAUNCH("ffn_tc_kernel<2> (shared)");
-      hook_mark(s, "ffn_w2_shared");
-    }
-  }
+    MOE_CHECK_LAUNCH(label);
+    hook_mark(s, label);
+    return MOE_OK;
+  };
+  moe_status_t st;
+  if ((st = run(1, w1, w3, false, "ffn_w13_swiglu")) != MOE_OK) return st;
+  if (sh && (st = run(1, sh[0], sh[1], true, "ffn_w13_swiglu_shared")) != MOE_OK) return st;
+  if ((st = run(2, w2, w2, false, "ffn_w2")) != MOE_OK) return st;
+  if (sh && (st = run(2, sh[2], sh[2], true, "ffn_w2_shared")) != MOE_OK) return st;
   return MOE_OK;
 }
 

@@ -35,6 +35,16 @@ TC_VARIANTS = {
     "skewed": dict(BASE, T=256, E=32, k=4, bias_std=2.0, seed=211),  # empty and heavy experts
     "T1": dict(BASE, T=1, seed=212),
     "wide": dict(BASE, T=160, d=1024, f=1024, seed=213),             # 16 k-tiles per stage
+    # shapes whose scale rows are whole 16-byte TMA boxes take the TMA/TMEM
+    # kernel in both stages (the ones above mix it with the per-thread-copy one)
+    "tma_a8g64": dict(BASE, T=200, d=1024, f=1024, w13=("affine", 8, 64), w2=("affine", 8, 64), seed=230),
+    "tma_a2g128": dict(BASE, T=200, d=1024, f=1024, w13=("affine", 2, 128), w2=("affine", 2, 128), seed=231),
+    "tma_mxfp4": dict(BASE, T=200, d=1024, f=1024, w13=("mxfp4", 4, 32), w2=("mxfp4", 4, 32), seed=232),
+    "tma_a4g32_partial_slot": dict(BASE, T=150, d=768, f=768, w13=("affine", 4, 32), w2=("affine", 4, 32),
+                                   seed=233),                          # 12 k-tiles: slots of 8 + 4
+    "tma_a4g128_a8g32": dict(BASE, T=200, d=1024, f=1024, w13=("affine", 4, 128), w2=("affine", 8, 32), seed=234),
+    "tma_shared8": dict(BASE, T=200, d=1024, f=512, shared=("affine", 8, 64), f_shared=512, seed=235),
+    "tma_big_experts": dict(BASE, T=600, E=4, d=512, f=512, seed=236),  # ~300 tokens per expert: 224 + rest
 }
 
 
