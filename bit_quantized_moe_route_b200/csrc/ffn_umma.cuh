@@ -11,17 +11,25 @@
 // Data path of one block (persistent, one per SM):
 //   * packed codes and group scales/biases of the 128 weight rows of the
 //     current item arrive by TMA (2D boxes of 128 bytes x rows, 128-byte
-//     swizzle; 16-byte scale boxes) into a three-slot ring, one slot = 512
-//     inputs (256 for 8-bit codes), loaded two slots ahead;
-//   * the token rows (B operand, fp16, up to 224 per tile, gathered into
-//     expert order beforehand) arrive by TMA as 64-input K-major tiles with
-//     the 128-byte swizzle the tensor core reads directly (3-stage ring);
-//   * 8 dequant warps turn each 64-input stage of codes into fp16 weights and
-//     write them straight into tensor memory (tcgen05.st): the weights are
-//     the MMA's A operand in TMEM (two stage slots of 32 columns), so the
-//     shared memory only carries the token tiles and the packed codes;
-//   * one thread issues tcgen05.mma (A from TMEM, B from shared memory,
-//     fp32 accumulators in TMEM, double-buffered: 2 x 224 columns);
+//     swizzle; 16-byte scale boxes) into a 3-slot ring, one slot = one
+//     128-byte box of codes per row (256 inputs of 4-bit codes, 128 of
+//     8-bit, 512 of 2-bit);
+//   * the token rows (B operand, fp16, up to 192 per tile, gathered into
+//     expert order beforehand) arrive by TMA as two 64-input K-major column
+//     blocks per 128-input stage, with the 128-byte swizzle the tensor core
+//     reads directly, in boxes of 64 / 128 / 192 rows as the tile needs
+//     (3-stage ring);
+//   * 8 dequant warps in two groups (even / odd stages) turn each 128-input
+//     stage of codes into fp16 weights and write them straight into tensor
+//     memory (tcgen05.st): the weights are the MMA's A operand in TMEM (two
+//     stage slots of 64 columns, one per group), so the shared memory only
+//     carries the token tiles and the packed codes;
+//   * the packed-code and token-tile TMA loads are issued by two separate
+//     threads, so neither ring waits on the other;
+//   * one thread issues 8 tcgen05.mma per stage (A from TMEM, B from shared
+//     memory, fp32 accumulators in TMEM, double-buffered: 2 x 192 columns);
+//     stages are 128 inputs deep because every barrier wait, fence and
+//     commit on the issuing thread delays the next MMA;
 //   * 4 epilogue warps read the accumulators (tcgen05.ld) and write H
 //     (SwiGLU, fp16) or y (fp32).
 // Stage 1 stacks 64 gate rows and the 64 up rows of the same features in
@@ -39,20 +47,24 @@
 
 namespace moe {
 
-constexpr int kUmN = 224;      // tokens per tile (MMA N <= 224, multiple of 16)
-constexpr int kUmK = 64;       // inputs per MMA stage
+constexpr int kUmN = 192;        // tokens per tile (MMA N <= 192, multiple of 16)
+constexpr int kUmK = 128;        // inputs per MMA stage (8 MMAs of K = 16)
+constexpr int kUmKB = 64;        // inputs per 128-byte swizzle atom of a token row
 constexpr int kUmThreads = 16 * 32;
-constexpr int kUmLoadWarp = 8;
-constexpr int kUmMmaWarp = 9;
+constexpr int kUmMmaWarp = 8;
+constexpr int kUmRawWarp = 9;    // TMA issuer of packed codes / scales / biases
+constexpr int kUmBWarp = 10;     // TMA issuer of token tiles
 constexpr int kUmEpiWarp0 = 12;  // warps 12-15: warp % 4 = TMEM lane quarter
 constexpr int kUmBStages = 3;
-constexpr int kUmBTile = kUmN * 128;  // 224 rows x 64 fp16
-constexpr uint32_t kUmAccCol0 = 64;   // TMEM columns: A stage slots [0, 64), accumulators at 64 and 288
+constexpr int kUmBBlock = kUmN * 128;       // one 64-input column block of a token tile
+constexpr int kUmBTile = 2 * kUmBBlock;     // 192 rows x 128 inputs fp16 = 48 KB
+constexpr uint32_t kUmASlotCols = kUmK / 2; // 64 TMEM columns per A stage slot
+constexpr uint32_t kUmAccCol0 = 2 * kUmASlotCols;  // accumulators at 128 and 320
 constexpr uint32_t kUmAccCols = kUmN;
 constexpr uint32_t kUmTmemCols = 512;
 
 struct alignas(64) UmParams {
-  CUtensorMap b_map;     // B rows: fp16 [rows, n_in], box {64, 224}, 128B swizzle
+  CUtensorMap b_map[3];  // B rows: fp16 [rows, n_in], boxes {64, 64 / 128 / 192 rows}, 128B swizzle
   CUtensorMap q_map[2];  // packed codes: uint8 [E*n_out, row bytes], box {128, R}, 128B swizzle
   CUtensorMap s_map[2];  // scales: bf16 or e8m0 [E*n_out, groups], box {16 bytes, R}
   CUtensorMap z_map[2];  // biases: bf16 (affine)
@@ -62,6 +74,7 @@ struct alignas(64) UmParams {
   int n_in, n_out;       // per-expert shape of each A matrix
   int group;
   int row_bytes, gpr;    // packed bytes and scale groups per weight row
+  int lg_group;          // log2(group)
   int T;                 // shared expert: tokens
   int shared;            // 1: one expert over positions 0..T-1 (no tile table)
   const int4* tiles;     // routed token tiles {expert, first position, tokens, 0}
@@ -76,18 +89,18 @@ struct UmCfg {
   static constexpr bool mx = FMT == F_MX4;
   static constexpr int M = STAGE == 1 ? 2 : 1;          // matrices stacked in one tile
   static constexpr int R = 128 / M;                     // rows per matrix per tile
-  static constexpr int KS = bits == 8 ? 256 : 512;      // inputs per raw slot
-  static constexpr int QS = KS / kUmK;                  // MMA stages per raw slot
-  static constexpr int NPB = KS * bits / 8 / 128;       // 128-byte packed boxes per matrix per slot
+  static constexpr int KS = 128 * 8 / bits;             // inputs per raw slot: one 128-byte box of codes per row
+  static constexpr int QS = KS / kUmK;                  // MMA stages per raw slot (1, 2 or 4)
   static constexpr int PBOX = R * 128;
   static constexpr int SBOX = R * 16;
-  static constexpr int NSB = 2;                         // scale boxes reserved per matrix per slot
-  static constexpr int packed_bytes = NPB * M * PBOX;
+  static constexpr int NSB = bits == 2 ? 2 : 1;         // scale boxes reserved per matrix per slot
+  static constexpr int packed_bytes = M * PBOX;
   static constexpr int scale_bytes = NSB * M * SBOX;
   static constexpr int slot_bytes = packed_bytes + 2 * scale_bytes;  // codes, scales, biases
   static constexpr int GBOX = mx ? 16 : 8;              // groups per 16-byte scale box
   static constexpr int ESZ = mx ? 1 : 2;                // scale element bytes
   static constexpr int NRS = 3;                         // raw slots
+  static constexpr int RAW_USERS = QS == 1 ? 4 : 8;     // dequant warps reading one raw slot
   static constexpr size_t smem = 1024 + NRS * (size_t)slot_bytes + (size_t)kUmBStages * kUmBTile + 256;
   static_assert(FMT != F_A3, "3-bit codes take the per-thread-copy kernel");
   static_assert(slot_bytes % 1024 == 0, "raw slots keep the 1024-byte alignment of the swizzled boxes");
@@ -106,7 +119,11 @@ MOE_DEV void um_tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint3
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
-// this thread's 16 consecutive 32-bit TMEM columns of its lane
+MOE_DEV void um_prefetch_map(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+// this thread's 16 consecutive 32-bit TMEM columns of its lane (complete
+// after tmem_st_wait)
 MOE_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
@@ -114,8 +131,8 @@ MOE_DEV void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
       "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
+MOE_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // D[tmem] (+)= A[tmem] . B[smem]^T, fp16 inputs, fp32 accumulation
 MOE_DEV void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -145,13 +162,15 @@ MOE_DEV int4 um_tile(const UmParams& p, int j) {
 }
 
 // Walks this block's items (blockIdx.x, +gridDim.x, ...), each in n_sub
-// sub-steps (k-stages or raw slots), with the next item's tile loaded ahead.
+// sub-steps (MMA stages or raw slots), with the next item's tile loaded
+// ahead; k counts this block's items.
 struct UmCursor {
-  int item, sub, mt;
+  int item, sub, mt, k;
   int4 tile, nxt;
   MOE_DEV void init(const UmParams& p, int n_items, int n_mt) {
     item = blockIdx.x;
     sub = 0;
+    k = 0;
     mt = item % n_mt;
     tile = item < n_items ? um_tile(p, item / n_mt) : make_int4(0, 0, 0, 0);
     const int n2 = item + gridDim.x;
@@ -159,6 +178,7 @@ struct UmCursor {
   }
   MOE_DEV void next_item(const UmParams& p, int n_items, int n_mt) {
     sub = 0;
+    ++k;
     item += gridDim.x;
     mt = item % n_mt;
     tile = nxt;
@@ -174,26 +194,26 @@ struct UmCursor {
 template <int STAGE, int FMT>
 __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_constant__ UmParams p) {
   using C = UmCfg<STAGE, FMT>;
-  constexpr int M = C::M, QS = C::QS;
+  constexpr int M = C::M, QS = C::QS, NRS = C::NRS, NB = kUmBStages;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw32 = tc_smem(smem_raw);
   const uint32_t base = (raw32 + 1023u) & ~1023u;  // swizzled boxes need 1024-byte alignment
-  constexpr int NRS = C::NRS;
   const uint32_t slot0 = base;                      // raw slots: [codes | scales | biases] x NRS
   const uint32_t bt0 = base + (uint32_t)(NRS * C::slot_bytes);  // B stages
-  const uint32_t bar = bt0 + (uint32_t)(kUmBStages * kUmBTile);
+  const uint32_t bar = bt0 + (uint32_t)(NB * kUmBTile);
   uint8_t* bar_gen = smem_raw + (bar - raw32);
-  auto raw_full = [&](int s) { return bar + 8u * s; };           // [3] TMA bytes
-  auto raw_empty = [&](int s) { return bar + 8u * (3 + s); };    // [3] 8 dequant warps
-  auto b_full = [&](int s) { return bar + 8u * (6 + s); };       // [3] TMA bytes
-  auto b_empty = [&](int s) { return bar + 8u * (9 + s); };      // [3] MMA commit
-  auto a_full = [&](int s) { return bar + 8u * (12 + s); };      // [2] 8 dequant warps
-  auto a_empty = [&](int s) { return bar + 8u * (14 + s); };     // [2] MMA commit
-  auto acc_full = [&](int s) { return bar + 8u * (16 + s); };    // [2] MMA commit
-  auto acc_empty = [&](int s) { return bar + 8u * (18 + s); };   // [2] 4 epilogue warps
-  const uint32_t drain = bar + 8u * 20;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_gen + 8 * 21);
+  auto raw_full = [&](int s) { return bar + 8u * s; };                      // [NRS] TMA bytes
+  auto raw_empty = [&](int s) { return bar + 8u * (NRS + s); };             // [NRS] dequant warps
+  auto b_full = [&](int s) { return bar + 8u * (2 * NRS + s); };            // [NB] TMA bytes
+  auto b_empty = [&](int s) { return bar + 8u * (2 * NRS + NB + s); };      // [NB] MMA commit
+  auto a_full = [&](int s) { return bar + 8u * (2 * NRS + 2 * NB + s); };   // [2] 4 dequant warps
+  auto a_empty = [&](int s) { return bar + 8u * (2 * NRS + 2 * NB + 2 + s); };    // [2] MMA commit
+  auto acc_full = [&](int s) { return bar + 8u * (2 * NRS + 2 * NB + 4 + s); };   // [2] MMA commit
+  auto acc_empty = [&](int s) { return bar + 8u * (2 * NRS + 2 * NB + 6 + s); };  // [2] 4 epilogue warps
+  const uint32_t drain = bar + 8u * (2 * NRS + 2 * NB + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_gen + 8 * (2 * NRS + 2 * NB + 9));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  static_assert(8 * (2 * NRS + 2 * NB + 9) + 8 <= 256, "barrier block");
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_mt = p.n_out / (STAGE == 1 ? 64 : 128);
@@ -208,17 +228,17 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
   if (tid == 0) {
     for (int s = 0; s < NRS; ++s) {
       tc_bar_init(raw_full(s), 1);
-      tc_bar_init(raw_empty(s), 8);
+      tc_bar_init(raw_empty(s), C::RAW_USERS);
+    }
+    for (int s = 0; s < NB; ++s) {
+      tc_bar_init(b_full(s), 1);
+      tc_bar_init(b_empty(s), 1);
     }
     for (int s = 0; s < 2; ++s) {
-      tc_bar_init(a_full(s), 8);
+      tc_bar_init(a_full(s), 4);
       tc_bar_init(a_empty(s), 1);
       tc_bar_init(acc_full(s), 1);
       tc_bar_init(acc_empty(s), 4);
-    }
-    for (int s = 0; s < kUmBStages; ++s) {
-      tc_bar_init(b_full(s), 1);
-      tc_bar_init(b_empty(s), 1);
     }
     tc_bar_init(drain, 1);
     *abort_flag = 0;
@@ -236,130 +256,138 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp < 8) {
-    // ================= dequant warps: TMEM lane quarter q, input half kh
-    const int q = warp & 3, kh = warp >> 2;
-    const int m = STAGE == 1 ? (lane >> 4) : 0;                  // matrix of this lane's row
+    // ================= dequant warps: group G takes the stages g = G mod 2
+    // into A slot G; warp quarter q owns TMEM lanes 32q..32q+31 (= A rows)
+    const int G = warp >> 2, q = warp & 3;
+    const int m = STAGE == 1 ? (lane >> 4) : 0;                        // matrix of this lane's row
     const int rr = STAGE == 1 ? 16 * q + (lane & 15) : 32 * q + lane;  // row within that matrix's box
     UmCursor cur;
     cur.init(p, n_items, n_mt);
-    int rc = 0;  // raw slots consumed
+    if (G == 1 && total > 1) cur.advance(p, n_items, n_mt, n_kt);
+    int held = -1;  // raw slot sequence number whose data this group is reading
     bool bad = false;
-    for (int g = 0; g < total; ++g) {
+    const uint32_t tcol = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)G * kUmASlotCols;
+    for (int g = G; g < total; g += 2) {
       const int kt = cur.sub, qs = kt % QS, ri = kt / QS;
-      const int rs = rc % NRS;
+      const int seq = cur.k * n_rng + ri;
+      const int rs = seq % NRS;
       bool ok = true;
-      if (qs == 0) ok = tc_bar_wait(raw_full(rs), (uint32_t)(rc / NRS) & 1u, abort_flag);
-      const int as = g & 1;
-      if (ok && g >= 2) ok = tc_bar_wait(a_empty(as), (uint32_t)((g >> 1) - 1) & 1u, abort_flag);
+      if (seq != held) {
+        ok = tc_bar_wait(raw_full(rs), (uint32_t)(seq / NRS) & 1u, abort_flag);
+        held = seq;
+      }
+      if (ok && g >= 2) ok = tc_bar_wait(a_empty(G), (uint32_t)((g >> 1) - 1) & 1u, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.st below is warp-collective
       const uint32_t slot = slot0 + (uint32_t)(rs * C::slot_bytes);
-      // this thread's 32 codes: inputs ko .. ko+31 of the slot
-      const int ko = qs * kUmK + kh * 32;
-      const int bo = ko * C::bits / 8;
-      const uint32_t prow = slot + (uint32_t)(((bo >> 7) * M + m) * C::PBOX + rr * 128);
-      const int j = (bo & 127) >> 4;
-      uint32_t w[8];
-      if constexpr (C::bits == 8) {
-        const uint4 v0 = tc_lds128(prow + (uint32_t)((j ^ (rr & 7)) << 4));
-        const uint4 v1 = tc_lds128(prow + (uint32_t)(((j + 1) ^ (rr & 7)) << 4));
-        w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-        w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
-      } else if constexpr (C::bits == 4) {
-        const uint4 v0 = tc_lds128(prow + (uint32_t)((j ^ (rr & 7)) << 4));
-        w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-      } else {
-        const uint2 v0 = tc_lds64(prow + (uint32_t)((j ^ (rr & 7)) << 4) + (uint32_t)(bo & 15));
-        w[0] = v0.x; w[1] = v0.y;
+      const uint32_t prow = slot + (uint32_t)(m * C::PBOX + rr * 128);
+      const int x0 = ((ri * C::KS) >> p.lg_group) & ~(C::GBOX - 1);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {  // 32 inputs per block
+        const int ko = qs * kUmK + 32 * b;        // input offset inside the slot
+        const int bo = ko * C::bits / 8;          // byte offset inside the 128-byte row
+        uint32_t w[8];
+        if constexpr (C::bits == 8) {
+          const uint4 v0 = tc_lds128(prow + (uint32_t)((((bo >> 4)) ^ (rr & 7)) << 4));
+          const uint4 v1 = tc_lds128(prow + (uint32_t)((((bo >> 4) + 1) ^ (rr & 7)) << 4));
+          w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+          w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+        } else if constexpr (C::bits == 4) {
+          const uint4 v0 = tc_lds128(prow + (uint32_t)(((bo >> 4) ^ (rr & 7)) << 4));
+          w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+        } else {
+          const uint2 v0 = tc_lds64(prow + (uint32_t)(((bo >> 4) ^ (rr & 7)) << 4) + (uint32_t)(bo & 15));
+          w[0] = v0.x; w[1] = v0.y;
+        }
+        const int gi = ((ri * C::KS + ko) >> p.lg_group) - x0;
+        const uint32_t saddr = slot + (uint32_t)(C::packed_bytes + ((gi / C::GBOX) * M + m) * C::SBOX + rr * 16 +
+                                                 (gi % C::GBOX) * C::ESZ);
+        uint32_t out[16];
+        if constexpr (C::mx) {
+          const uint32_t e = um_lds8(saddr);
+          uint32_t f = 0;  // 2^(e-113) in fp16 (see tc_dequant32_mx)
+          if (e > 128) bad = true;
+          else if (e >= 99) f = (e - 98u) << 10;
+          tc_dequant32_mx(w, f | (f << 16), out);
+        } else {
+          const float sf = __uint_as_float(um_lds16(saddr) << 16);
+          const float bf = __uint_as_float(um_lds16(saddr + C::scale_bytes) << 16);
+          if (!(fabsf(sf) * (float)((1 << C::bits) - 1) + fabsf(bf) <= kF16Max)) bad = true;
+          const __half hs = __float2half_rn(sf), hb = __float2half_rn(bf);
+          tc_dequant32<FMT>(w, h2u(__halves2half2(hs, hs)), h2u(__halves2half2(hb, hb)), out);
+        }
+        tmem_st16(tcol + 16u * b, out);
       }
-      // this thread's group scale (and bias)
-      const int g_first = ri * C::KS / p.group;
-      const int x0 = g_first / C::GBOX * C::GBOX;
-      const int gi = (ri * C::KS + ko) / p.group - x0;
-      const uint32_t saddr = slot + (uint32_t)(C::packed_bytes + ((gi / C::GBOX) * M + m) * C::SBOX + rr * 16 +
-                                               (gi % C::GBOX) * C::ESZ);
-      uint32_t out[16];
-      if constexpr (C::mx) {
-        const uint32_t e = um_lds8(saddr);
-        uint32_t f = 0;  // 2^(e-113) in fp16 (see tc_dequant32_mx)
-        if (e > 128) bad = true;
-        else if (e >= 99) f = (e - 98u) << 10;
-        tc_dequant32_mx(w, f | (f << 16), out);
-      } else {
-        const float sf = __uint_as_float(um_lds16(saddr) << 16);
-        const float bf = __uint_as_float(um_lds16(saddr + C::scale_bytes) << 16);
-        if (!(fabsf(sf) * (float)((1 << C::bits) - 1) + fabsf(bf) <= kF16Max)) bad = true;
-        const __half hs = __float2half_rn(sf), hb = __float2half_rn(bf);
-        tc_dequant32<FMT>(w, h2u(__halves2half2(hs, hs)), h2u(__halves2half2(hb, hb)), out);
-      }
-      tmem_st16(tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(as * 32 + kh * 16), out);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc_bar_arrive(a_full(as));
-      if (qs == QS - 1 || kt == n_kt - 1) {  // last use of this raw slot
-        if (lane == 0) tc_bar_arrive(raw_empty(rs));
-        ++rc;
-      }
+      if (lane == 0) tc_bar_arrive(a_full(G));
       cur.advance(p, n_items, n_mt, n_kt);
+      if (g + 1 < total) cur.advance(p, n_items, n_mt, n_kt);
+      const int next_seq = g + 2 < total ? cur.k * n_rng + cur.sub / QS : -1;
+      if (next_seq != seq && lane == 0) tc_bar_arrive(raw_empty(rs));  // this group's last use of the slot
     }
     if (bad) set_error(p.err, kErrDeviceInput);
-  } else if (warp == kUmLoadWarp) {
-    // ================= TMA issuer
+  } else if (warp == kUmRawWarp) {
+    // ================= TMA issuer: packed codes, scales, biases (up to NRS slots ahead)
     if (lane == 0) {
-      UmCursor cur, rcur;  // B stages; raw slots (two ahead)
-      cur.init(p, n_items, n_mt);
-      rcur = cur;
-      int rc = 0;
+      for (int mm = 0; mm < M; ++mm) {
+        um_prefetch_map(&p.q_map[mm]);
+        um_prefetch_map(&p.s_map[mm]);
+        if constexpr (!C::mx) um_prefetch_map(&p.z_map[mm]);
+      }
+      UmCursor rcur;
+      rcur.init(p, n_items, n_mt);
       const int m_rows = STAGE == 1 ? 64 : 128;
-      auto issue_raw = [&]() -> bool {  // slot for (rcur.item, rcur.sub = range)
-        const int rs = rc % NRS;
-        if (rc >= NRS && !tc_bar_wait(raw_empty(rs), (uint32_t)(rc / NRS - 1) & 1u, abort_flag)) return false;
+      const int raw_total = my_items * n_rng;
+      for (int seq = 0; seq < raw_total; ++seq) {
+        const int rs = seq % NRS;
+        if (seq >= NRS && !tc_bar_wait(raw_empty(rs), (uint32_t)(seq / NRS - 1) & 1u, abort_flag)) break;
         const uint32_t slot = slot0 + (uint32_t)(rs * C::slot_bytes);
         const int ri = rcur.sub;
         const int row = rcur.tile.x * p.n_out + rcur.mt * m_rows;
-        const int xp = ri * C::KS * C::bits / 8;
-        const int x0 = ri * C::KS / p.group / C::GBOX * C::GBOX;
-        // boxes that start past the end of a row are not loaded (nothing reads them)
-        const int np = min(C::NPB, (p.row_bytes - xp + 127) / 128);
-        const int ns = min(nsb, (p.gpr - x0 + C::GBOX - 1) / C::GBOX);
-        um_expect_tx(raw_full(rs), (uint32_t)(M * (np * C::PBOX + ns * C::SBOX * (C::mx ? 1 : 2))));
+        const int xp = ri * 128;
+        const int x0 = ((ri * C::KS) >> p.lg_group) & ~(C::GBOX - 1);
+        const int ns = min(nsb, (p.gpr - x0 + C::GBOX - 1) / C::GBOX);  // boxes past the row end are skipped
+        um_expect_tx(raw_full(rs), (uint32_t)(M * (C::PBOX + ns * C::SBOX * (C::mx ? 1 : 2))));
 #pragma unroll
         for (int mm = 0; mm < M; ++mm) {
-          for (int b = 0; b < np; ++b)
-            um_tma_2d(slot + (uint32_t)((b * M + mm) * C::PBOX), &p.q_map[mm], xp + b * 128, row, raw_full(rs));
+          um_tma_2d(slot + (uint32_t)(mm * C::PBOX), &p.q_map[mm], xp, row, raw_full(rs));
           for (int sb = 0; sb < ns; ++sb) {
             const uint32_t so = slot + (uint32_t)(C::packed_bytes + (sb * M + mm) * C::SBOX);
             um_tma_2d(so, &p.s_map[mm], x0 + sb * C::GBOX, row, raw_full(rs));
             if constexpr (!C::mx) um_tma_2d(so + C::scale_bytes, &p.z_map[mm], x0 + sb * C::GBOX, row, raw_full(rs));
           }
         }
-        ++rc;
         rcur.advance(p, n_items, n_mt, n_rng);
-        return true;
-      };
-      int raw_issued = 0;
-      const int raw_total = my_items * n_rng;
-      for (int r = 0; r < NRS - 1 && raw_issued < raw_total; ++r)
-        if (issue_raw()) ++raw_issued;
+      }
+    }
+    __syncwarp();
+  } else if (warp == kUmBWarp) {
+    // ================= TMA issuer: token tiles, two 64-input column blocks per
+    // stage, box height 64 / 128 / 192 rows as the tile needs
+    if (lane == 0) {
+      for (int h = 0; h < 3; ++h) um_prefetch_map(&p.b_map[h]);
+      UmCursor cur;
+      cur.init(p, n_items, n_mt);
       for (int g = 0; g < total; ++g) {
-        const int kt = cur.sub;
-        if (kt % QS == 0 && raw_issued < raw_total) {  // keep the raw ring two slots ahead
-          if (!issue_raw()) break;
-          ++raw_issued;
-        }
-        const int bs = g % kUmBStages;
-        const int round = g / kUmBStages;
-        if (round > 0 && !tc_bar_wait(b_empty(bs), (uint32_t)(round - 1) & 1u, abort_flag)) break;
-        um_expect_tx(b_full(bs), (uint32_t)kUmBTile);
-        um_tma_2d(bt0 + (uint32_t)(bs * kUmBTile), &p.b_map, kt * kUmK, p.pos_base + cur.tile.y, b_full(bs));
+        const int bs = g % NB;
+        if (g >= NB && !tc_bar_wait(b_empty(bs), (uint32_t)(g / NB - 1) & 1u, abort_flag)) break;
+        const int h = cur.tile.z <= 64 ? 0 : cur.tile.z <= 128 ? 1 : 2;
+        um_expect_tx(b_full(bs), (uint32_t)(2 * 64 * (h + 1) * 128));
+        const uint32_t dst = bt0 + (uint32_t)(bs * kUmBTile);
+        const int y = p.pos_base + cur.tile.y;
+        um_tma_2d(dst, &p.b_map[h], cur.sub * kUmK, y, b_full(bs));
+        um_tma_2d(dst + kUmBBlock, &p.b_map[h], cur.sub * kUmK + kUmKB, y, b_full(bs));
         cur.advance(p, n_items, n_mt, n_kt);
       }
     }
     __syncwarp();
   } else if (warp == kUmMmaWarp) {
-    // ================= MMA issuer
+    // ================= MMA issuer: 8 MMAs (K = 16 each) per stage
     if (lane == 0) {
       UmCursor cur;
       cur.init(p, n_items, n_mt);
+      const uint64_t db_base = umma_desc(bt0);
       int g = 0;
       for (int it = 0; it < my_items && !*abort_flag; ++it) {
         const uint32_t idesc = umma_idesc_f16((cur.tile.z + 15) & ~15);
@@ -369,17 +397,20 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
         const uint32_t d = tmem_base + kUmAccCol0 + (uint32_t)ab * kUmAccCols;
         bool ok = true;
         for (int kt = 0; kt < n_kt; ++kt, ++g) {
-          const int as = g & 1, bs = g % kUmBStages;
+          const int as = g & 1, bs = g % NB;
           if (!tc_bar_wait(a_full(as), (uint32_t)(g >> 1) & 1u, abort_flag) ||
-              !tc_bar_wait(b_full(bs), (uint32_t)(g / kUmBStages) & 1u, abort_flag)) {
+              !tc_bar_wait(b_full(bs), (uint32_t)(g / NB) & 1u, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t bt = bt0 + (uint32_t)(bs * kUmBTile);
+          const uint32_t a0 = tmem_base + (uint32_t)as * kUmASlotCols;
+          // B descriptor start advances 32 bytes per K = 16 inside a column
+          // block, and one column block (24 KB) after four MMAs
+          const uint64_t db0 = db_base + (uint64_t)((bs * kUmBTile) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kUmK / 16; ++kk)  // K = 16 per MMA: 8 TMEM columns of A, 32 bytes of B
-            umma_f16_ts(d, tmem_base + (uint32_t)(as * 32 + kk * 8), umma_desc(bt + 32u * kk), idesc,
+          for (int kk = 0; kk < 8; ++kk)
+            umma_f16_ts(d, a0 + 8u * kk, db0 + (uint64_t)(((kk >> 2) * kUmBBlock + (kk & 3) * 32) >> 4), idesc,
                         (kt | kk) ? 1u : 0u);
           umma_commit(a_empty(as));
           umma_commit(b_empty(bs));

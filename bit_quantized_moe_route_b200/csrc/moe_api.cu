@@ -482,10 +482,11 @@ moe_status_t tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, ui
 
 // Shapes the TMA/TMEM kernel takes: 2/4/8-bit affine or mxfp4 codes, rows of
 // a multiple of 16 bytes, scale rows of a multiple of 16 bytes (the TMA
-// stride rule), 64 (stage 1) or 128 (stage 2) output rows per tile.
+// stride rule), 64 (stage 1) or 128 (stage 2) output rows per tile, an even
+// number of 128-input stages (the two dequant groups split them).
 bool um_ok(const QMatDev& Q, int stage) {
   if (Q.fmt == F_A3) return false;
-  if (Q.n_in % kUmK || Q.n_out % (stage == 1 ? 64 : 128)) return false;
+  if (Q.n_in % (2 * kUmK) || Q.n_out % (stage == 1 ? 64 : 128)) return false;
   if ((Q.wpr * 4) % 16) return false;
   if (Q.group != 32 && Q.group != 64 && Q.group != 128) return false;
   return Q.fmt == F_MX4 ? Q.gpr % 16 == 0 : (Q.gpr * 2) % 16 == 0;
@@ -536,13 +537,15 @@ moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offset
     const int E = shared ? 1 : d.n_experts;
     if (um_ok(a0, stage) && um_ok(a1, stage)) {
       UmParams q{};
-      moe_status_t st;
-      if (stage == 1)
-        st = tmap_2d(&q.b_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs, d.d_model, (uint64_t)P, (uint64_t)d.d_model * 2,
-                     kUmK, kUmN, true);
-      else
-        st = tmap_2d(&q.b_map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h16, a0.n_in, (uint64_t)P, (uint64_t)ld_h * 2, kUmK,
-                     kUmN, true);
+      moe_status_t st = MOE_OK;
+      for (int h = 0; h < 3 && st == MOE_OK; ++h) {  // token boxes of 64, 128, 192 rows
+        if (stage == 1)
+          st = tmap_2d(&q.b_map[h], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs, d.d_model, (uint64_t)P,
+                       (uint64_t)d.d_model * 2, kUmKB, 64 * (h + 1), true);
+        else
+          st = tmap_2d(&q.b_map[h], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h16, a0.n_in, (uint64_t)P, (uint64_t)ld_h * 2,
+                       kUmKB, 64 * (h + 1), true);
+      }
       if (st != MOE_OK) return st;
       if ((st = um_weight_maps(q, 0, a0, E, stage == 1 ? 64 : 128)) != MOE_OK) return st;
       if (stage == 1 && (st = um_weight_maps(q, 1, a1, E, 64)) != MOE_OK) return st;
@@ -555,6 +558,7 @@ moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offset
       q.group = a0.group;
       q.row_bytes = a0.wpr * 4;
       q.gpr = a0.gpr;
+      q.lg_group = a0.group == 32 ? 5 : a0.group == 64 ? 6 : 7;
       q.T = d.T;
       q.shared = shared ? 1 : 0;
       q.tiles = ws_at<int4>(ws, L.tiles2);
