@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--config", default="decode")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ffn-path", default="auto", choices=["auto", "gemv", "tc"],
+                    help="expert-FFN implementation: library default, weight-streaming GEMV, tensor-core GEMM")
     ap.add_argument("--cpu-budget", type=float, default=25.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--override", action="append", default=[],
                     help="key=value change to the workload (profiling small cases), e.g. E=16")
@@ -286,6 +288,7 @@ def ours_arm(args):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     moe.load_library()
+    moe.set_ffn_path({"auto": moe.FFN_AUTO, "gemv": moe.FFN_GEMV, "tc": moe.FFN_TENSOR_CORE}[args.ffn_path])
     inp = make_inputs(args.config, dev, **overrides(args))
     c = inp.cfg
     T, d, k = c["T"], c["d"], c["k"]
@@ -415,7 +418,8 @@ def ours_arm(args):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16" if tensor_path else "f32", "data": "synthetic",
-        "config": dict(workload_desc(c), l2="flushed by a 512 MiB write between timed steps (outside the events)",
+        "config": dict(workload_desc(c), ffn_path=args.ffn_path,
+                       l2="flushed by a 512 MiB write between timed steps (outside the events)",
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "roofline": roofline,
         "layer": {"bytes_per_step": layer_bytes, "weight_bytes": weight_bytes, "distinct_routed_experts": n_act,

@@ -36,6 +36,14 @@ struct QMatDev {
 
 MOE_DEV void set_error(int* err, int code) { atomicCAS(err, 0, code); }
 
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream serialization attribute may start before its predecessor in the
+// stream has finished; pdl_wait() blocks until that predecessor has completed
+// and its memory is visible (a no-op without the attribute), pdl_trigger()
+// lets this kernel's own dependent start launching.
+MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+MOE_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 MOE_DEV float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
 MOE_DEV float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }

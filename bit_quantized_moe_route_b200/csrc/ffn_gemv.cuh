@@ -322,6 +322,7 @@ ffn_gemv_kernel(const FfnParams p) {
 __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ y, const int* __restrict__ inv, const float* __restrict__ w,
                const float* __restrict__ y_shared, __nv_bfloat16* __restrict__ out, int T, int k, int d) {
+  pdl_wait();  // y comes from the kernel before (possibly launched programmatically)
   const int t = blockIdx.y;
   const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
   if (c4 * 4 >= d) return;

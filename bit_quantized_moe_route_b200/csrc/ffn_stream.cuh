@@ -690,6 +690,13 @@ ffn_stream_kernel(const __grid_constant__ StreamParams p) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kStages);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
+  // Programmatic launch: stage 1 waits for the routing (it reads the active
+  // list right away) and then releases stage 2; stage 2 releases the combine
+  // at once and its copy warp starts streaming weights before stage 1 has
+  // finished -- weights and routing were complete when stage 1 released it
+  // -- while its consumers wait for stage 1 before reading h.
+  if constexpr (STAGE == 1) pdl_wait();
+  pdl_trigger();
   const int n_active = __ldcg(p.active);
   const int n_sh = p.has_shared ? (p.sa.n_out + p.s_rows - 1) / p.s_rows : 0;
   const int tpe = (p.ra.n_out + p.r_rows - 1) / p.r_rows;
@@ -734,6 +741,7 @@ ffn_stream_kernel(const __grid_constant__ StreamParams p) {
   }
 
   // ---------------- consumers: runs of tiles of one expert at a time
+  if constexpr (STAGE == 2) pdl_wait();  // h is written by stage 1
   XRegs<NTMAX, CPL> X;
   int buf = 0;
   int prev_wpr = 1;

@@ -17,7 +17,7 @@
 //   * the token rows (B operand, fp16, up to 192 per tile, gathered into
 //     expert order beforehand) arrive by TMA as two 64-input K-major column
 //     blocks per 128-input stage, with the 128-byte swizzle the tensor core
-//     reads directly, in boxes of 64 / 128 / 192 rows as the tile needs
+//     reads directly, in boxes of 16 / 64 / 128 / 192 rows as the tile needs
 //     (3-stage ring);
 //   * 8 dequant warps in two groups (even / odd stages) turn each 128-input
 //     stage of codes into fp16 weights and write them straight into tensor
@@ -64,7 +64,7 @@ constexpr uint32_t kUmAccCols = kUmN;
 constexpr uint32_t kUmTmemCols = 512;
 
 struct alignas(64) UmParams {
-  CUtensorMap b_map[3];  // B rows: fp16 [rows, n_in], boxes {64, 64 / 128 / 192 rows}, 128B swizzle
+  CUtensorMap b_map[4];  // B rows: fp16 [rows, n_in], boxes {64, 16 / 64 / 128 / 192 rows}, 128B swizzle
   CUtensorMap q_map[2];  // packed codes: uint8 [E*n_out, row bytes], box {128, R}, 128B swizzle
   CUtensorMap s_map[2];  // scales: bf16 or e8m0 [E*n_out, groups], box {16 bytes, R}
   CUtensorMap z_map[2];  // biases: bf16 (affine)
@@ -364,16 +364,17 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
     __syncwarp();
   } else if (warp == kUmBWarp) {
     // ================= TMA issuer: token tiles, two 64-input column blocks per
-    // stage, box height 64 / 128 / 192 rows as the tile needs
+    // stage, box height 16 / 64 / 128 / 192 rows as the tile needs
     if (lane == 0) {
-      for (int h = 0; h < 3; ++h) um_prefetch_map(&p.b_map[h]);
+      for (int h = 0; h < 4; ++h) um_prefetch_map(&p.b_map[h]);
       UmCursor cur;
       cur.init(p, n_items, n_mt);
       for (int g = 0; g < total; ++g) {
         const int bs = g % NB;
         if (g >= NB && !tc_bar_wait(b_empty(bs), (uint32_t)(g / NB - 1) & 1u, abort_flag)) break;
-        const int h = cur.tile.z <= 64 ? 0 : cur.tile.z <= 128 ? 1 : 2;
-        um_expect_tx(b_full(bs), (uint32_t)(2 * 64 * (h + 1) * 128));
+        const int h = cur.tile.z <= 16 ? 0 : cur.tile.z <= 64 ? 1 : cur.tile.z <= 128 ? 2 : 3;
+        const int box_rows = h == 0 ? 16 : 64 * h;
+        um_expect_tx(b_full(bs), (uint32_t)(2 * box_rows * 128));
         const uint32_t dst = bt0 + (uint32_t)(bs * kUmBTile);
         const int y = p.pos_base + cur.tile.y;
         um_tma_2d(dst, &p.b_map[h], cur.sub * kUmK, y, b_full(bs));

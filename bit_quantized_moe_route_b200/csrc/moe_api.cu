@@ -323,7 +323,7 @@ moe_status_t launch_route_fused(const moe_dims_t& d, const void* x, const float*
   // tail scratch: top-k keys/scores/selected (2E + k floats), pair ids and flags (2 T*k ints)
   const size_t perm_smem = (size_t)(2 * d.n_experts + 32 + 2 * d.T * d.top_k) * sizeof(int);
   if (d.hash_mode) {
-    const int blocks = ceil_div(d.T * 32, 256);
+    const int blocks = d.T;  // one block (8 warps) per token
     if (d.top_k <= 8)
       route_hash_fused_kernel<8><<<blocks, 256, perm_smem, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts,
                                                                d.top_k, d.vocab, ids, wts, offsets, sorted, inv,
@@ -429,16 +429,17 @@ std::atomic<int> g_ffn_path{MOE_FFN_AUTO};
 // The tensor-core kernel tiles 128 output rows x 64 inputs.
 bool tc_shape_ok(const QMatDev& A) { return A.n_out % kTcM == 0 && A.n_in % kTcK == 0; }
 
-// Tensor-core path for the expert FFN: chosen for large batches (on average
-// at least 32 tokens per active expert) or when forced, if the workspace has
-// its regions and every matrix has a supported shape.
+// Tensor-core path for the expert FFN: chosen from 4 tokens up (measured on
+// B200: the weight-streaming GEMV wins at T = 1, the tensor-core kernels at
+// T = 8 and 32 even with ~1-2 tokens per expert, since their dequantisation
+// keeps pace with HBM) or when forced, if the workspace has its regions and
+// every matrix has a supported shape.
 bool use_tc(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w2, const QMatDev* sh, const WsLayout& L) {
   const int mode = g_ffn_path.load(std::memory_order_relaxed);
   if (mode == MOE_FFN_GEMV || !L.tc) return false;
   if (!tc_shape_ok(w1) || !tc_shape_ok(w2) || (sh && (!tc_shape_ok(sh[0]) || !tc_shape_ok(sh[2])))) return false;
   if (mode == MOE_FFN_TENSOR_CORE) return true;
-  const long long Tk = (long long)d.T * d.top_k;
-  return Tk >= 32LL * std::min<long long>(d.n_experts, Tk);
+  return d.T >= 4;
 }
 
 // TMA/TMEM kernels indexed by format code (no 3-bit instance).
@@ -538,13 +539,14 @@ moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offset
     if (um_ok(a0, stage) && um_ok(a1, stage)) {
       UmParams q{};
       moe_status_t st = MOE_OK;
-      for (int h = 0; h < 3 && st == MOE_OK; ++h) {  // token boxes of 64, 128, 192 rows
+      for (int h = 0; h < 4 && st == MOE_OK; ++h) {  // token boxes of 16, 64, 128, 192 rows
+        const uint32_t box_rows = h == 0 ? 16u : 64u * h;
         if (stage == 1)
           st = tmap_2d(&q.b_map[h], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs, d.d_model, (uint64_t)P,
-                       (uint64_t)d.d_model * 2, kUmKB, 64 * (h + 1), true);
+                       (uint64_t)d.d_model * 2, kUmKB, box_rows, true);
         else
           st = tmap_2d(&q.b_map[h], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, h16, a0.n_in, (uint64_t)P, (uint64_t)ld_h * 2,
-                       kUmKB, 64 * (h + 1), true);
+                       kUmKB, box_rows, true);
       }
       if (st != MOE_OK) return st;
       if ((st = um_weight_maps(q, 0, a0, E, stage == 1 ? 64 : 128)) != MOE_OK) return st;
@@ -722,9 +724,21 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
 
 moe_status_t launch_combine(const moe_dims_t& d, const float* y, const int* inv, const float* w,
                             const float* y_shared, void* out, cudaStream_t s) {
-  dim3 grid(ceil_div(d.d_model / 4, 256), d.T);
-  combine_kernel<<<grid, 256, 0, s>>>(y, inv, w, y_shared, reinterpret_cast<__nv_bfloat16*>(out), d.T,
-                                      d.top_k, d.d_model);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // combine_kernel waits for y itself
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ceil_div(d.d_model / 4, 256), d.T);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaLaunchKernelEx(&cfg, combine_kernel, y, inv, w, y_shared,
+                                      reinterpret_cast<__nv_bfloat16*>(out), d.T, d.top_k, d.d_model);
+  if (le != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(le, "combine_kernel");
+  }
   MOE_CHECK_LAUNCH("combine_kernel");
   hook_mark(s, "combine");
   return MOE_OK;

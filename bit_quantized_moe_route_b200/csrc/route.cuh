@@ -413,6 +413,7 @@ route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __res
   __shared__ int warp_tot[32];
   __shared__ int total;
   __shared__ int is_last;
+  pdl_trigger();  // the expert FFN may start its launch (it waits for this grid before reading)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int e = blockIdx.x * 2 + (warp >> 2);
   const int quarter = warp & 3;
@@ -497,7 +498,83 @@ route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __res
   (void)total;
 }
 
-// Hash routing plus permutation, one launch: one warp per token, the last
+// Hash routing of token t = blockIdx.x by the whole block: warp 0 gathers
+// the token's table row, every warp dots x[t] with the k router rows over its
+// slice of d (partials in `part`), warp 0 finishes the weights.  Same rules as
+// route_hash_warp (bad ids: expert 0, weight 0, error word).
+template <int KMAX>
+MOE_DEV void route_hash_block(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+                              const int* __restrict__ token_ids, const int* __restrict__ table, int d, int E, int k,
+                              int vocab, int* __restrict__ ids, float* __restrict__ wts, int* err,
+                              float (*part)[KMAX], int* s_eid, int* s_good) {
+  const int t = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (warp == 0) {
+    const int tok = token_ids[t];
+    const bool tok_ok = tok >= 0 && tok < vocab;
+    int e = 0;
+    bool good = false;
+    if (lane < k && tok_ok) {
+      e = table[(size_t)tok * k + lane];
+      good = e >= 0 && e < E;
+      if (!good) e = 0;
+    }
+    const bool bad = !tok_ok || (lane < k && !good);
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_error(err, kErrDeviceInput);
+    if (lane < KMAX) {
+      s_eid[lane] = e;
+      s_good[lane] = good ? 1 : 0;
+    }
+  }
+  __syncthreads();
+  if (W != nullptr) {
+    float acc[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) acc[j] = 0.f;
+    const int n4 = d >> 2;
+    const int lo = n4 * warp / nw, hi = n4 * (warp + 1) / nw;
+    const uint2* xr = reinterpret_cast<const uint2*>(x + (size_t)t * d);
+    const float4* wr[KMAX];
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) wr[j] = reinterpret_cast<const float4*>(W + (size_t)(j < k ? s_eid[j] : 0) * d);
+    for (int i = lo + lane; i < hi; i += 32) {
+      const uint2 xv = xr[i];
+      const float x0 = bf16lo(xv.x), x1 = bf16hi(xv.x), x2 = bf16lo(xv.y), x3 = bf16hi(xv.y);
+#pragma unroll
+      for (int j = 0; j < KMAX; ++j) {
+        if (j < k) {
+          const float4 w = __ldg(wr[j] + i);
+          acc[j] = fmaf(w.x, x0, fmaf(w.y, x1, fmaf(w.z, x2, fmaf(w.w, x3, acc[j]))));
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < KMAX; ++j) {
+      const float v = warp_sum(acc[j]);
+      if (lane == 0 && j < k) part[warp][j] = v;
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float sj = 0.f;
+    const bool gj = lane < k && s_good[lane] != 0;
+    if (gj) {
+      if (W != nullptr) {
+        float l = 0.f;
+        for (int w = 0; w < nw; ++w) l += part[w][lane];
+        sj = sqrt_softplus(l);
+      } else {
+        sj = 1.f;
+      }
+    }
+    const float ssum = warp_sum(sj);
+    if (lane < k) {
+      ids[(size_t)t * k + lane] = s_eid[lane];
+      wts[(size_t)t * k + lane] = gj && ssum > 0.f ? sj / ssum : 0.f;
+    }
+  }
+}
+
+// Hash routing plus permutation, one launch: one block per token, the last
 // block groups the pairs by expert.
 template <int KMAX>
 __global__ void __launch_bounds__(256)
@@ -510,8 +587,11 @@ route_hash_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __rest
   __shared__ int warp_tot[32];
   __shared__ int total;
   __shared__ int is_last;
-  route_hash_warp<KMAX>(x, W, token_ids, table, T, d, E, k, vocab, ids, wts, err);
-  __threadfence();  // publish this warp's ids/weights before the arrival below
+  __shared__ float part[8][KMAX];
+  __shared__ int s_eid[KMAX], s_good[KMAX];
+  pdl_trigger();  // the expert FFN may start its launch (it waits for this grid before reading)
+  route_hash_block<KMAX>(x, W, token_ids, table, d, E, k, vocab, ids, wts, err, part, s_eid, s_good);
+  __threadfence();  // publish this token's ids/weights before the arrival below
   __syncthreads();
   if (threadIdx.x == 0) {
     is_last = atomicAdd(counter, 1) == (int)gridDim.x - 1;

@@ -9,9 +9,21 @@ namespace moe {
 
 bool MOE_NAME(launch_stream_s, MOE_ST, MOE_RF)(int ntmax, int cpl, int grid, cudaStream_t s,
                                                 const StreamParams& q) {
+  // programmatic stream serialization: the kernel waits (griddepcontrol)
+  // for its predecessor's results where it needs them
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kStreamThreads);
+  cfg.dynamicSmemBytes = kStreamSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
 #define MOE_CASE(NT, CP)                                                                          \
   if (ntmax == NT && cpl == CP) {                                                                 \
-    ffn_stream_kernel<MOE_ST, NT, CP, MOE_RF_CODE><<<grid, kStreamThreads, kStreamSmem, s>>>(q); \
+    cudaLaunchKernelEx(&cfg, ffn_stream_kernel<MOE_ST, NT, CP, MOE_RF_CODE>, q); /* errors: caller checks */ \
     return true;                                                                                  \
   }
   MOE_CASE(1, 4)

@@ -275,8 +275,8 @@ const char* moe_timing_label(int32_t i);
  * Expert-FFN implementation used by moe_expert_ffn / moe_forward /
  * moe_forward_host (process-wide setting; not for the allocation-free entry
  * point, which always streams).  AUTO (default) takes the tensor-core path
- * when the batch averages at least 32 tokens per active expert
- * (T*top_k >= 32*min(n_experts, T*top_k)) and the shapes allow it.
+ * from T >= 4 tokens when the shapes allow it (d_ff, d_model multiples of
+ * 128), and the weight-streaming GEMV below that.
  * Returns the previous setting, or -1 (setting unchanged) for an unknown
  * value.
  */

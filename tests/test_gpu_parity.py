@@ -50,8 +50,12 @@ VARIANTS = {
 
 @pytest.fixture(scope="module")
 def device(cuda_device):
+    """These cases cover the weight-streaming GEMV path (the tensor-core path
+    has its own file), so the module forces it."""
     moe.load_library()
-    return cuda_device
+    prev = moe.set_ffn_path(moe.FFN_GEMV)
+    yield cuda_device
+    moe.set_ffn_path(prev)
 
 
 @pytest.mark.parametrize("name", list(VARIANTS))

@@ -115,11 +115,11 @@ def test_tc_flags_fp16_overflow(device):
     assert moe.read_device_error(ws) == 6  # MOE_ERR_DEVICE_INPUT
 
 
-def test_auto_picks_tc_for_large_batches(device):
-    """AUTO uses the tensor-core kernels once experts average >= 32 tokens (timing labels show which ran)."""
+def test_auto_picks_tc_from_four_tokens(device):
+    """AUTO uses the tensor-core kernels from T = 4 up (timing labels show which ran)."""
     moe.set_ffn_path(moe.FFN_AUTO)
     try:
-        for T, want in ((8, False), (512, True)):
+        for T, want in ((1, False), (3, False), (4, True), (512, True)):
             inp = make_custom(dict(BASE, T=T, seed=220), device)
             evs = [torch.cuda.Event(enable_timing=True) for _ in range(16)]
             keep = moe.set_timing_events(evs)
