@@ -5,7 +5,9 @@ static device array.  This file is collected last so that a run stopping at
 the first failure has already run every other test.  Each case compares the
 new entry point with moe_expert_ffn (which uses a caller workspace) on the
 same inputs, twice in a row, so the second call also checks that leftover
-contents of the shared static array do not leak into results.
+contents of the shared static array do not leak into results.  The
+allocation-free entry point always runs the weight-streaming GEMV, so
+moe_expert_ffn is run with that path selected for the bitwise comparison.
 """
 import numpy as np
 import pytest
@@ -45,7 +47,11 @@ def test_noalloc_matches_workspace_entry_point(cuda_device, name):
     ws = moe.alloc_workspace(dims, cuda_device)
     n = c["T"] * c["k"]
     y_ws = torch.empty(n, c["d"], dtype=torch.float32, device=cuda_device)
-    moe.expert_ffn(dims, inp.x, offs, rows, inp.w1, inp.w3, inp.w2, y_ws, ws)
+    prev = moe.set_ffn_path(moe.FFN_GEMV)
+    try:
+        moe.expert_ffn(dims, inp.x, offs, rows, inp.w1, inp.w3, inp.w2, y_ws, ws)
+    finally:
+        moe.set_ffn_path(prev)
     y_ref = res["y_slots"].reshape(n, c["d"])[res["sorted_rows"]]
     for call in range(2):
         y_na = torch.full((n, c["d"]), float("nan"), dtype=torch.float32, device=cuda_device)
