@@ -64,9 +64,13 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
-def src_hash():
+def src_hash(files=None):
+    """Hash of the kernel sources (the listed csrc files, else all of them):
+    a stored ncu traffic figure only applies while its kernel is unchanged."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "bit_quantized_moe_route_b200", "csrc", "*"))):
+    csrc = os.path.join(ROOT, "bit_quantized_moe_route_b200", "csrc")
+    paths = [os.path.join(csrc, f) for f in files] if files else glob.glob(os.path.join(csrc, "*"))
+    for p in sorted(paths):
         with open(p, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -394,7 +398,7 @@ def ours_arm(args):
         with open(prof) as fh:
             tj = json.load(fh)
         ent = tj.get(c["name"], {}).get(dom)
-        if ent and ent.get("src_hash") == src_hash():
+        if ent and ent.get("src_hash") == src_hash(ent.get("files")):
             traffic = ent.get("dram_bytes_per_launch")
     tensor_path = "tile_plan" in labels
     if tensor_path and dom in kflops:
