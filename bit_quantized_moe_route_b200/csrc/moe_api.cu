@@ -110,7 +110,7 @@ WsLayout layout_of(const moe_dims_t& d) {
     return at;
   };
   L.hdr = take(sizeof(WsHeader));
-  L.logits = take(d.hash_mode ? 0 : T * E * sizeof(float));
+  L.logits = take(d.hash_mode ? 0 : 2 * T * E * sizeof(float));  // two K-half partials at large T
   L.ids = take(T * k * sizeof(int));
   L.wts = take(T * k * sizeof(float));
   L.offsets = take((E + 1) * sizeof(int));
@@ -285,6 +285,7 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
     return MOE_OK;
   }
   float* logits = ws_at<float>(ws, L.logits);
+  int split = 1;  // K halves of the logits GEMM (partials summed by the top-k)
   if (d.T <= 64) {
     dim3 grid(ceil_div(d.n_experts, kLogitWarps), ceil_div(d.T, 8));
     router_logits_small_kernel<8><<<grid, kLogitWarps * 32, 8 * d.d_model * 2, s>>>(xb, rw, logits, d.T,
@@ -292,18 +293,21 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
     MOE_CHECK_LAUNCH("router_logits_small_kernel");
     hook_mark(s, "router_logits");
   } else {
-    dim3 grid(ceil_div(d.n_experts, kLBN), ceil_div(d.T, kLBM));
+    // two K halves (more CTAs than SMs) when there is enough work
+    split = d.T >= 256 && d.d_model % (2 * kLBK) == 0 ? 2 : 1;
+    dim3 grid(ceil_div(d.n_experts, kLBN), ceil_div(d.T, kLBM), split);
     router_logits_tiled_kernel<<<grid, 256, 0, s>>>(xb, rw, logits, d.T, d.d_model, d.n_experts);
     MOE_CHECK_LAUNCH("router_logits_tiled_kernel");
     hook_mark(s, "router_logits");
   }
   const int blocks = ceil_div(d.T * 32, 256);
+  const float* L2 = split == 2 ? logits + (size_t)d.T * d.n_experts : nullptr;
   if (d.n_experts <= 32)
-    topk_kernel<1><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts);
+    topk_kernel<1><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts, L2);
   else if (d.n_experts <= 256)
-    topk_kernel<8><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts);
+    topk_kernel<8><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts, L2);
   else
-    topk_kernel<32><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts);
+    topk_kernel<32><<<blocks, 256, 0, s>>>(logits, rb, d.T, d.n_experts, d.top_k, ids, wts, L2);
   MOE_CHECK_LAUNCH("topk_kernel");
   hook_mark(s, "topk");
   return MOE_OK;

@@ -72,7 +72,9 @@ router_logits_small_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
 
 // ---------------------------------------------------------------------------
 // Logits for large T: tiled fp32 SIMT GEMM, 128 tokens x 64 experts per CTA,
-// 8x4 outputs per thread, K in steps of 16 with register prefetch.
+// 8x4 outputs per thread, K in steps of 16 with register prefetch.  With
+// gridDim.z = 2 each CTA sums one half of K into its own partial array
+// (L + z*T*E); the top-k adds the two partials in a fixed order.
 // ---------------------------------------------------------------------------
 constexpr int kLBM = 128, kLBN = 64, kLBK = 16;
 
@@ -84,6 +86,8 @@ router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
   const int tid = threadIdx.x;
   const int tx = tid & 15, ty = tid >> 4;
   const int m0 = blockIdx.y * kLBM, n0 = blockIdx.x * kLBN;
+  const int kspan = d / gridDim.z, kbeg = blockIdx.z * kspan, kend = kbeg + kspan;
+  L += (size_t)blockIdx.z * T * E;
   // loaders: x tile 128 x 16 bf16 -> each thread 8 elements (one 16-byte load)
   const int xr = tid >> 1, xc = (tid & 1) * 8;
   // W tile 64 x 16 fp32 -> each thread 4 elements (one float4)
@@ -102,8 +106,8 @@ router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
     wreg = (gn < E) ? __ldg(reinterpret_cast<const float4*>(W + (size_t)gn * d + k0 + wc))
                     : make_float4(0.f, 0.f, 0.f, 0.f);
   };
-  load(0);
-  for (int k0 = 0; k0 < d; k0 += kLBK) {
+  load(kbeg);
+  for (int k0 = kbeg; k0 < kend; k0 += kLBK) {
     __syncthreads();
     xs[xc + 0][xr] = bf16lo(xreg.x);
     xs[xc + 1][xr] = bf16hi(xreg.x);
@@ -118,7 +122,7 @@ router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
     wsm[wc + 2][wr] = wreg.z;
     wsm[wc + 3][wr] = wreg.w;
     __syncthreads();
-    if (k0 + kLBK < d) load(k0 + kLBK);
+    if (k0 + kLBK < kend) load(k0 + kLBK);
 #pragma unroll
     for (int kk = 0; kk < kLBK; ++kk) {
       const float4 a0 = *reinterpret_cast<const float4*>(&xs[kk][ty * 8]);
@@ -150,14 +154,15 @@ router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
 // ---------------------------------------------------------------------------
 template <int MAXPER>
 MOE_DEV void topk_token(const float* __restrict__ Lrow, const float* __restrict__ bias, int E, int k,
-                        int* __restrict__ ids_row, float* __restrict__ w_row) {
+                        int* __restrict__ ids_row, float* __restrict__ w_row,
+                        const float* __restrict__ Lrow2 = nullptr) {
   const int lane = threadIdx.x & 31;
   float key[MAXPER], sc[MAXPER];
 #pragma unroll
   for (int i = 0; i < MAXPER; ++i) {
     const int e = i * 32 + lane;
     if (e < E) {
-      const float s = sqrt_softplus(__ldcg(Lrow + e));
+      const float s = sqrt_softplus(Lrow2 ? __ldcg(Lrow + e) + __ldcg(Lrow2 + e) : __ldcg(Lrow + e));
       sc[i] = s;
       float kv = bias ? s + bias[e] : s;
       key[i] = (kv != kv) ? -INFINITY : kv;
@@ -218,10 +223,11 @@ MOE_DEV void topk_token(const float* __restrict__ Lrow, const float* __restrict_
 template <int MAXPER>
 __global__ void __launch_bounds__(256)
 topk_kernel(const float* __restrict__ L, const float* __restrict__ bias, int T, int E, int k,
-            int* __restrict__ ids, float* __restrict__ wts) {
+            int* __restrict__ ids, float* __restrict__ wts, const float* __restrict__ L2) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (warp >= T) return;
-  topk_token<MAXPER>(L + (size_t)warp * E, bias, E, k, ids + (size_t)warp * k, wts + (size_t)warp * k);
+  topk_token<MAXPER>(L + (size_t)warp * E, bias, E, k, ids + (size_t)warp * k, wts + (size_t)warp * k,
+                     L2 ? L2 + (size_t)warp * E : nullptr);
 }
 
 // ---------------------------------------------------------------------------
