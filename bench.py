@@ -401,7 +401,17 @@ def ours_arm(args):
         if ent and ent.get("src_hash") == src_hash(ent.get("files")):
             traffic = ent.get("dram_bytes_per_launch")
     tensor_path = "tile_plan" in labels
-    if tensor_path and dom in kflops:
+    if tensor_path:  # H is fp16 on the tensor-core path
+        fs_ = c.get("f_shared", 0) if inp.shared is not None else 0
+        P_ = T * k + (T if inp.shared is not None else 0)
+        for lab in ("ffn_w13_swiglu", "ffn_w2"):
+            work[lab] -= P_ * max(c["f"], fs_) * 2
+    # the binding roofline of the dominant kernel: tensor FLOPs or HBM bytes,
+    # whichever it is closer to (small batches on the tensor-core path stream
+    # weights far below the machine balance point)
+    tflops_dom = kflops.get(dom, 0.0) / (dom_ms * 1e-3) / 1e12 if tensor_path else 0.0
+    gbs_dom = work.get(dom, 0) / (dom_ms * 1e-3) / 1e9
+    if tensor_path and dom in kflops and tflops_dom / bf16_sus >= gbs_dom / hbm:
         # fp16 x fp16 -> fp32 tcgen05 MMAs: the nominal fp16 and bf16 dense rates are equal,
         # so the measured bf16 cuBLAS rate is the denominator (sustained: the kernel runs
         # inside a long back-to-back step loop under the power cap)
