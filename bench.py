@@ -391,7 +391,6 @@ def ours_arm(args):
     hbm, bf16, bf16_sus, peak_kind = peaks()
     dom = max(kern_ms, key=kern_ms.get)
     dom_ms = kern_ms[dom]
-    achieved = work.get(dom, 0) / (dom_ms * 1e-3) / 1e9
     traffic = None
     prof = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(prof):
@@ -423,9 +422,11 @@ def ours_arm(args):
                     "algorithmic_bytes_per_launch": work.get(dom, 0),
                     "hbm_frac": work.get(dom, 0) / (dom_ms * 1e-3) / 1e9 / hbm}
     else:
-        roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                    "frac": achieved / hbm, "traffic": traffic, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+        roofline = {"bound": "hbm", "kernel": dom, "achieved": gbs_dom, "peak": hbm, "unit": "GB/s",
+                    "frac": gbs_dom / hbm, "traffic": traffic, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
                     "algorithmic_bytes_per_launch": work.get(dom, 0)}
+        if tensor_path and dom in kflops:
+            roofline["tensor_frac"] = tflops_dom / bf16_sus
     layer_bytes = sum(work.values())
     value = T * world / (ms_per_step * 1e-3)
     line = {
