@@ -92,6 +92,7 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 struct WsLayout {
   size_t hdr, logits, ids, wts, offsets, sorted, inv, active, h, y, xstage, tokstage, outstage;
   size_t x16, tiles, tiles2, ntiles;  // tensor-core FFN: fp16 token rows by position, token-tile plans
+  size_t pchunks;                     // multi-CTA permutation: per-chunk expert counts / bases
   bool tc = false;            // the regions above exist
   size_t total;
 };
@@ -126,6 +127,7 @@ WsLayout layout_of(const moe_dims_t& d) {
   L.tiles = take(((T * k + kTcN - 1) / kTcN + E) * sizeof(int4));
   L.tiles2 = take(((T * k + kUmN - 1) / kUmN + E) * sizeof(int4));
   L.ntiles = take(2 * sizeof(int));
+  L.pchunks = take(((T * k + kPermThreads - 1) / kPermThreads) * E * sizeof(int));
   L.tc = true;
   L.total = o;
   return L;
@@ -232,6 +234,7 @@ moe_status_t dev_info(DevInfo** out) {
     if (g_dev_ready[dev].compare_exchange_strong(expect, 1)) {
       cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
       cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 34 * 1024 * 4);
+      cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024 * 4);
       cudaFuncSetAttribute(router_logits_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            8 * 8192 * 2);
       cudaFuncSetAttribute(route_small_fused_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
@@ -364,9 +367,25 @@ moe_status_t launch_permute(const moe_dims_t& d, const int* ids, int* offsets, i
                             void* ws, const WsLayout& L, cudaStream_t s) {
   int* err = &ws_at<WsHeader>(ws, L.hdr)->err;
   int* active = ws_at<int>(ws, L.active);
+  const int N = d.T * d.top_k;
+  if (N > 4 * kPermThreads && L.pchunks) {
+    // chunks of 1024 pairs on separate CTAs: counts, one scan, placement
+    const int nb = ceil_div(N, kPermThreads);
+    int* cnt = ws_at<int>(ws, L.pchunks);
+    permute_count_kernel<<<nb, kPermThreads, d.n_experts * sizeof(int), s>>>(ids, N, d.n_experts, cnt, err);
+    MOE_CHECK_LAUNCH("permute_count_kernel");
+    hook_mark(s, "permute_count");
+    permute_scan_kernel<<<1, kPermThreads, 0, s>>>(cnt, nb, d.n_experts, offsets, active);
+    MOE_CHECK_LAUNCH("permute_scan_kernel");
+    hook_mark(s, "permute_scan");
+    permute_scatter_kernel<<<nb, kPermThreads, (size_t)32 * d.n_experts * sizeof(int), s>>>(
+        ids, N, d.n_experts, cnt, sorted, inv);
+    MOE_CHECK_LAUNCH("permute_scatter_kernel");
+    hook_mark(s, "permute");
+    return MOE_OK;
+  }
   const size_t smem = (size_t)(2 + 32) * d.n_experts * sizeof(int);
-  permute_kernel<<<1, kPermThreads, smem, s>>>(ids, d.T * d.top_k, d.n_experts, offsets, sorted, inv, active,
-                                               err);
+  permute_kernel<<<1, kPermThreads, smem, s>>>(ids, N, d.n_experts, offsets, sorted, inv, active, err);
   MOE_CHECK_LAUNCH("permute_kernel");
   hook_mark(s, "permute");
   return MOE_OK;

@@ -176,6 +176,99 @@ permute_kernel(const int* __restrict__ ids, int N, int E, int* __restrict__ offs
   permute_block(ids, N, E, offsets, sorted_rows, inv, active, err, sm, warp_tot, &total);
 }
 
+// ---------------------------------------------------------------------------
+// The same stable grouping for large N in three launches: CTA b owns pairs
+// [b*1024, (b+1)*1024).  The sorted position of pair i (expert e) is
+// offsets[e] + #{pairs before i's chunk with expert e} + #{pairs of i's chunk
+// before i with expert e}; the middle term comes from per-chunk counts.
+// ---------------------------------------------------------------------------
+// 1: per-chunk expert counts -> cnt[b * E + e]
+__global__ void __launch_bounds__(kPermThreads)
+permute_count_kernel(const int* __restrict__ ids, int N, int E, int* __restrict__ cnt, int* err) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < E; e += kPermThreads) hist[e] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * kPermThreads + threadIdx.x;
+  bool bad = false;
+  if (i < N) {
+    int e = ids[i];
+    if (e < 0 || e >= E) {
+      bad = true;
+      e = 0;
+    }
+    atomicAdd(&hist[e], 1);
+  }
+  if (bad) set_error(err, kErrDeviceInput);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kPermThreads) cnt[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// 2: one CTA: offsets[e], the active list, and cnt[b * E + e] turned into the
+// first sorted position of expert e's pairs in chunk b
+__global__ void __launch_bounds__(kPermThreads)
+permute_scan_kernel(int* __restrict__ cnt, int n_chunks, int E, int* __restrict__ offsets,
+                    int* __restrict__ active) {
+  __shared__ int warp_tot[32];
+  __shared__ int total;
+  int carry = 0, acarry = 0;
+  for (int e0 = 0; e0 < E; e0 += kPermThreads) {
+    const int e = e0 + threadIdx.x;
+    int c = 0;
+    if (e < E)
+      for (int b = 0; b < n_chunks; ++b) c += cnt[(size_t)b * E + e];
+    const int ex = block_exclusive_scan(c, warp_tot, &total);
+    const int chunk_total = total;
+    const int flag = c > 0 ? 1 : 0;
+    const int aex = block_exclusive_scan(flag, warp_tot, &total);
+    const int achunk = total;
+    if (e < E) {
+      offsets[e] = carry + ex;
+      if (flag) active[1 + acarry + aex] = e;
+      int run = carry + ex;
+      for (int b = 0; b < n_chunks; ++b) {
+        const int v = cnt[(size_t)b * E + e];
+        cnt[(size_t)b * E + e] = run;
+        run += v;
+      }
+    }
+    carry += chunk_total;
+    acarry += achunk;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = carry;
+    active[0] = acarry;
+  }
+}
+
+// 3: each CTA places its chunk: warp-level ranks (match_any) plus the counts
+// of the warps before it.  Dynamic shared memory: 32 * E ints.
+__global__ void __launch_bounds__(kPermThreads)
+permute_scatter_kernel(const int* __restrict__ ids, int N, int E, const int* __restrict__ base,
+                       int* __restrict__ sorted_rows, int* __restrict__ inv) {
+  extern __shared__ int wc[];  // [32 warps][E] counts of this chunk
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  for (int q = tid; q < 32 * E; q += kPermThreads) wc[q] = 0;
+  __syncthreads();
+  const int i = blockIdx.x * kPermThreads + tid;
+  int e = -1;
+  if (i < N) {
+    e = ids[i];
+    if (e < 0 || e >= E) e = 0;
+  }
+  const unsigned peers = __match_any_sync(0xffffffffu, e);
+  const int rank_w = __popc(peers & ((1u << lane) - 1u));
+  if (e >= 0 && rank_w == 0) wc[warp * E + e] = __popc(peers);
+  __syncthreads();
+  if (e >= 0) {
+    int pre = 0;
+    for (int w = 0; w < warp; ++w) pre += wc[w * E + e];
+    const int p = base[(size_t)blockIdx.x * E + e] + pre + rank_w;
+    sorted_rows[p] = i;
+    inv[i] = p;
+  }
+}
+
 // Active-expert list from caller-provided offsets (single CTA).
 __global__ void __launch_bounds__(kPermThreads)
 active_from_offsets_kernel(const int* __restrict__ offsets, int E, int* __restrict__ active) {
