@@ -85,13 +85,16 @@ struct alignas(64) UmParams {
 
 template <int STAGE, int FMT>
 struct UmCfg {
-  static constexpr int bits = FMT == F_A2 ? 2 : FMT == F_A8 ? 8 : 4;
+  static constexpr int bits = FMT == F_A2 ? 2 : FMT == F_A3 ? 3 : FMT == F_A8 ? 8 : 4;
   static constexpr bool mx = FMT == F_MX4;
   static constexpr int M = STAGE == 1 ? 2 : 1;          // matrices stacked in one tile
   static constexpr int R = 128 / M;                     // rows per matrix per tile
-  static constexpr int KS = 128 * 8 / bits;             // inputs per raw slot: one 128-byte box of codes per row
+  // inputs per raw slot: one 128-byte box of codes per row (128B-swizzled),
+  // for 3-bit codes a 96-byte box (256 inputs, no swizzle)
+  static constexpr int KS = bits == 3 ? 256 : 128 * 8 / bits;
+  static constexpr int BOXB = KS * bits / 8;            // packed bytes per row per slot
   static constexpr int QS = KS / kUmK;                  // MMA stages per raw slot (1, 2 or 4)
-  static constexpr int PBOX = R * 128;
+  static constexpr int PBOX = R * BOXB;
   static constexpr int SBOX = R * 16;
   static constexpr int NSB = bits == 2 ? 2 : 1;         // scale boxes reserved per matrix per slot
   static constexpr int packed_bytes = M * PBOX;
@@ -102,7 +105,6 @@ struct UmCfg {
   static constexpr int NRS = 3;                         // raw slots
   static constexpr int RAW_USERS = QS == 1 ? 4 : 8;     // dequant warps reading one raw slot
   static constexpr size_t smem = 1024 + NRS * (size_t)slot_bytes + (size_t)kUmBStages * kUmBTile + 256;
-  static_assert(FMT != F_A3, "3-bit codes take the per-thread-copy kernel");
   static_assert(slot_bytes % 1024 == 0, "raw slots keep the 1024-byte alignment of the swizzled boxes");
   static_assert(smem <= 227 * 1024, "TMA/TMEM FFN exceeds the per-block shared memory limit");
 };
@@ -279,8 +281,16 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
       if (ok && g >= 2) ok = tc_bar_wait(a_empty(G), (uint32_t)((g >> 1) - 1) & 1u, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.st below is warp-collective
       const uint32_t slot = slot0 + (uint32_t)(rs * C::slot_bytes);
-      const uint32_t prow = slot + (uint32_t)(m * C::PBOX + rr * 128);
+      const uint32_t prow = slot + (uint32_t)(m * C::PBOX + rr * C::BOXB);
       const int x0 = ((ri * C::KS) >> p.lg_group) & ~(C::GBOX - 1);
+      uint32_t w3[12];  // 3-bit codes: the stage's 48 bytes of this row (unswizzled box)
+      if constexpr (C::bits == 3) {
+#pragma unroll
+        for (int c = 0; c < 3; ++c) {
+          const uint4 v = tc_lds128(prow + (uint32_t)(qs * 48 + 16 * c));
+          w3[4 * c] = v.x; w3[4 * c + 1] = v.y; w3[4 * c + 2] = v.z; w3[4 * c + 3] = v.w;
+        }
+      }
 #pragma unroll
       for (int b = 0; b < 4; ++b) {  // 32 inputs per block
         const int ko = qs * kUmK + 32 * b;        // input offset inside the slot
@@ -294,6 +304,8 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
         } else if constexpr (C::bits == 4) {
           const uint4 v0 = tc_lds128(prow + (uint32_t)(((bo >> 4) ^ (rr & 7)) << 4));
           w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+        } else if constexpr (C::bits == 3) {
+          w[0] = w3[3 * b]; w[1] = w3[3 * b + 1]; w[2] = w3[3 * b + 2];
         } else {
           const uint2 v0 = tc_lds64(prow + (uint32_t)(((bo >> 4) ^ (rr & 7)) << 4) + (uint32_t)(bo & 15));
           w[0] = v0.x; w[1] = v0.y;
@@ -345,7 +357,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
         const uint32_t slot = slot0 + (uint32_t)(rs * C::slot_bytes);
         const int ri = rcur.sub;
         const int row = rcur.tile.x * p.n_out + rcur.mt * m_rows;
-        const int xp = ri * 128;
+        const int xp = ri * C::BOXB;
         const int x0 = ((ri * C::KS) >> p.lg_group) & ~(C::GBOX - 1);
         const int ns = min(nsb, (p.gpr - x0 + C::GBOX - 1) / C::GBOX);  // boxes past the row end are skipped
         um_expect_tx(raw_full(rs), (uint32_t)(M * (C::PBOX + ns * C::SBOX * (C::mx ? 1 : 2))));
@@ -491,10 +503,12 @@ using UmAttrFn = void (*)();
   bool launch_um_s##ST##_##F(const UmParams& p, int grid, cudaStream_t s); \
   void attrs_um_s##ST##_##F();
 MOE_UM_DECL(1, A2)
+MOE_UM_DECL(1, A3)
 MOE_UM_DECL(1, A4)
 MOE_UM_DECL(1, A8)
 MOE_UM_DECL(1, MX4)
 MOE_UM_DECL(2, A2)
+MOE_UM_DECL(2, A3)
 MOE_UM_DECL(2, A4)
 MOE_UM_DECL(2, A8)
 MOE_UM_DECL(2, MX4)

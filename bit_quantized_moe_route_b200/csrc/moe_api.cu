@@ -214,7 +214,7 @@ moe_status_t check_qmat(const moe_qmat_t* m, int n_in, const char* name, QMatDev
 
 extern const StreamAttrFn kStreamAttrs[10];
 extern const TcAttrFn kTcAttrs[10];
-extern const UmAttrFn kUmAttrs[8];
+extern const UmAttrFn kUmAttrs[10];
 
 struct DevInfo {
   int sms = 0;
@@ -467,10 +467,10 @@ bool use_tc(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w2, const QMa
 
 // TMA/TMEM kernels indexed by format code (no 3-bit instance).
 const UmLaunchFn kUmLaunch[2][5] = {
-    {launch_um_s1_A2, nullptr, launch_um_s1_A4, launch_um_s1_A8, launch_um_s1_MX4},
-    {launch_um_s2_A2, nullptr, launch_um_s2_A4, launch_um_s2_A8, launch_um_s2_MX4}};
-const UmAttrFn kUmAttrs[8] = {attrs_um_s1_A2, attrs_um_s1_A4, attrs_um_s1_A8, attrs_um_s1_MX4,
-                              attrs_um_s2_A2, attrs_um_s2_A4, attrs_um_s2_A8, attrs_um_s2_MX4};
+    {launch_um_s1_A2, launch_um_s1_A3, launch_um_s1_A4, launch_um_s1_A8, launch_um_s1_MX4},
+    {launch_um_s2_A2, launch_um_s2_A3, launch_um_s2_A4, launch_um_s2_A8, launch_um_s2_MX4}};
+const UmAttrFn kUmAttrs[10] = {attrs_um_s1_A2, attrs_um_s1_A3, attrs_um_s1_A4, attrs_um_s1_A8, attrs_um_s1_MX4,
+                               attrs_um_s2_A2, attrs_um_s2_A3, attrs_um_s2_A4, attrs_um_s2_A8, attrs_um_s2_MX4};
 
 // cuTensorMapEncodeTiled from the driver, looked up once.
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -504,12 +504,11 @@ moe_status_t tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, ui
   return MOE_OK;
 }
 
-// Shapes the TMA/TMEM kernel takes: 2/4/8-bit affine or mxfp4 codes, rows of
-// a multiple of 16 bytes, scale rows of a multiple of 16 bytes (the TMA
-// stride rule), 64 (stage 1) or 128 (stage 2) output rows per tile, an even
-// number of 128-input stages (the two dequant groups split them).
+// Shapes the TMA/TMEM kernel takes: any packed format, rows of a multiple of
+// 16 bytes, scale rows of a multiple of 16 bytes (the TMA stride rule), 64
+// (stage 1) or 128 (stage 2) output rows per tile, an even number of
+// 128-input stages (the two dequant groups split them).
 bool um_ok(const QMatDev& Q, int stage) {
-  if (Q.fmt == F_A3) return false;
   if (Q.n_in % (2 * kUmK) || Q.n_out % (stage == 1 ? 64 : 128)) return false;
   if ((Q.wpr * 4) % 16) return false;
   if (Q.group != 32 && Q.group != 64 && Q.group != 128) return false;
@@ -519,8 +518,10 @@ bool um_ok(const QMatDev& Q, int stage) {
 // Packed-code, scale and bias maps of matrix Q (E experts) for slot m.
 moe_status_t um_weight_maps(UmParams& p, int m, const QMatDev& Q, int E, int rows_per_box) {
   const uint64_t rows = (uint64_t)E * Q.n_out;
+  // 3-bit codes: 96-byte boxes (256 inputs) without swizzle; else 128-byte swizzled boxes
+  const bool b3 = Q.fmt == F_A3;
   moe_status_t st = tmap_2d(&p.q_map[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.q, (uint64_t)Q.wpr * 4, rows,
-                            (uint64_t)Q.wpr * 4, 128, rows_per_box, true);
+                            (uint64_t)Q.wpr * 4, b3 ? 96 : 128, rows_per_box, !b3);
   if (st != MOE_OK) return st;
   if (Q.fmt == F_MX4)
     return tmap_2d(&p.s_map[m], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.scales, Q.gpr, rows, Q.gpr, 16, rows_per_box, false);
