@@ -236,6 +236,22 @@ def overrides(args):
     return out
 
 
+def max_over_ranks(v, device):
+    """The largest of every rank's v (the slowest rank's time); v itself on one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank, world, ms):
+    """Tokens per second of the whole job: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (ms * 1e-3)
+
+
 def reference_arm(args):
     """The oracle, as it stands, on this host's cores (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -336,11 +352,7 @@ def ours_arm(args):
     if world > 1:
         dist.barrier()
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    ms_per_step = sum(step_ms) / args.steps
-    if world > 1:
-        t = torch.tensor([ms_per_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step = float(t.item())
+    ms_per_step = max_over_ranks(sum(step_ms) / args.steps, dev)
 
     # ---- per-kernel durations: a second timed pass with CUDA events recorded
     # by the library between its kernels on the same stream (the events add
@@ -379,11 +391,7 @@ def ours_arm(args):
         b.record(stream)
         b.synchronize()
         e2e_ms += a.elapsed_time(b)
-    e2e_ms /= e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms / e2e_steps, dev)
     h2d = T * d * 2 + (T * 4 if tok_h is not None else 0)
     d2h = T * d * 2
     err = moe.read_device_error(ws)
@@ -428,7 +436,7 @@ def ours_arm(args):
         if tensor_path and dom in kflops:
             roofline["tensor_frac"] = tflops_dom / bf16_sus
     layer_bytes = sum(work.values())
-    value = T * world / (ms_per_step * 1e-3)
+    value = whole_job_rate(T, world, ms_per_step)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -442,7 +450,7 @@ def ours_arm(args):
                   "frac_whole_step": layer_bytes / (ms_per_step * 1e-3) / 1e9 / hbm,
                   "flops_per_step": flops, "TFLOPs_whole_step": flops / (ms_per_step * 1e-3) / 1e12,
                   "kernel_ms": kern_ms},
-        "e2e": {"value": T * world / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": len(labels) * args.steps,
         "kernel_timing_steps": k_steps,
