@@ -1,0 +1,96 @@
+"""The roofline numerators bench.py reports (algorithmic bytes and flops per
+kernel), checked on CPU against closed forms of the packed formats.
+
+A packed matrix of n weights with b-bit codes and bf16 scale + bias per
+group of g inputs holds n·(b/8 + 4/g) bytes; mxfp4 holds n·(1/2 + 1/32)
+(one e8m0 byte per 32 codes).  The per-expert figures of the five layer
+configurations follow from these; tensors are built on the meta device, so
+nothing of the full-size packs is allocated."""
+import os
+import sys
+import types
+
+import numpy as np
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from synthetic.moe_inputs import QMat  # noqa: E402
+
+
+def qmat(fmt, bits, group, E, n_out, n_in):
+    q = torch.empty(E, n_out, n_in * bits // 32, dtype=torch.int32, device="meta")
+    if fmt == "mxfp4":
+        return QMat(fmt, 4, 32, n_out, n_in, q, torch.empty(E, n_out, n_in // 32, dtype=torch.uint8, device="meta"),
+                    None)
+    s = torch.empty(E, n_out, n_in // group, dtype=torch.bfloat16, device="meta")
+    return QMat(fmt, bits, group, n_out, n_in, q, s, torch.empty_like(s))
+
+
+def layer(T, d, E, k, f, w13, w2, shared=None, f_shared=0, routing="learned"):
+    cfg = dict(T=T, d=d, E=E, k=k, f=f, routing=routing, f_shared=f_shared)
+    sh = None
+    if shared:
+        sh = (qmat(*shared, 1, f_shared, d), qmat(*shared, 1, f_shared, d), qmat(*shared, 1, d, f_shared))
+    return types.SimpleNamespace(cfg=cfg, w1=qmat(*w13, E, f, d), w3=qmat(*w13, E, f, d), w2=qmat(*w2, E, d, f),
+                                 shared=sh)
+
+
+def closed_form(n, fmt, bits, group):
+    if fmt == "mxfp4":
+        return n * (0.5 + 1 / 32)
+    return n * (bits / 8 + 4 / group)
+
+
+@pytest.mark.parametrize("w13,w2,want", [
+    (("affine", 4, 64), ("affine", 4, 64), 14_155_776),
+    (("mxfp4", 4, 32), ("mxfp4", 4, 32), 13_369_344),
+    (("affine", 2, 128), ("affine", 3, 128), 8_126_464),
+])
+def test_per_expert_bytes(w13, w2, want):
+    d, f = 4096, 2048
+    inp = layer(1, d, 256, 8, f, w13, w2)
+    per = (inp.w1.packed_bytes_per_expert() + inp.w3.packed_bytes_per_expert()
+           + inp.w2.packed_bytes_per_expert())
+    assert per == want
+    assert per == closed_form(2 * d * f, *w13) + closed_form(d * f, *w2)
+
+
+def test_decode_weight_bytes_count_distinct_experts_and_shared():
+    d, f, k = 4096, 2048, 8
+    inp = layer(1, d, 256, k, f, ("affine", 4, 64), ("affine", 4, 64), shared=("affine", 8, 64), f_shared=2048)
+    ids = np.array([[3, 17, 17, 40, 41, 99, 200, 255]])  # 7 distinct experts (17 twice)
+    work, flops, n_act, weight_bytes, kflops = bench.kernel_work(inp, ids)
+    assert n_act == 7
+    shared = 26_738_688
+    assert shared == closed_form(3 * d * 2048, "affine", 8, 64)
+    assert weight_bytes == 7 * 14_155_776 + shared
+    # stage 1 reads W1 and W3 of each active expert and of the shared expert
+    w13_routed = 7 * 2 * closed_form(d * f, "affine", 4, 64)
+    w13_shared = 2 * closed_form(d * 2048, "affine", 8, 64)
+    P = 1 * k + 1
+    assert work["ffn_w13_swiglu"] == w13_routed + w13_shared + d * 2 + P * f * 4
+    assert work["ffn_w2"] == 7 * closed_form(d * f, "affine", 4, 64) + closed_form(d * 2048, "affine", 8, 64) \
+        + P * f * 4 + P * d * 4
+    # the fp32 router matrix is read once
+    assert work["router_logits"] == 256 * d * 4 + d * 2 + 256 * 4
+
+
+def test_prefill_flops():
+    T, d, E, k, f = 4096, 4096, 256, 8, 2048
+    inp = layer(T, d, E, k, f, ("affine", 4, 64), ("affine", 4, 64))
+    ids = np.arange(T * k).reshape(T, k) % E
+    work, flops, n_act, weight_bytes, kflops = bench.kernel_work(inp, ids)
+    assert flops == 2 * T * k * 3 * d * f
+    assert abs(flops - 1.649e12) < 1e9
+    assert kflops["ffn_w13_swiglu"] + kflops["ffn_w2"] == flops
+    assert kflops["ffn_w13_swiglu"] == 2 * kflops["ffn_w2"]
+    assert n_act == E and weight_bytes == E * 14_155_776
+
+
+def test_whole_job_rate_is_tokens_over_slowest_time():
+    assert bench.whole_job_rate(1, 1, 0.094) == pytest.approx(1 / 94e-6)
+    assert bench.whole_job_rate(4096, 8, 2.5) == pytest.approx(8 * 4096 / 2.5e-3)
