@@ -115,6 +115,8 @@ def make_dims(T: int, d_model: int, d_ff: int, n_experts: int, top_k: int, hash_
 def qmat(m) -> QMatC:
     """Describe a packed matrix: any object with fmt ('affine'|'mxfp4'), bits,
     group and CUDA tensors q, scales, biases (None for mxfp4)."""
+    if m.fmt not in ("affine", "mxfp4"):
+        raise ValueError(f"packed format {m.fmt!r} is not supported by the library (affine, mxfp4)")
     fmt = FMT_AFFINE if m.fmt == "affine" else FMT_MXFP4
     return QMatC(fmt, m.bits, m.group, 0, _ptr(m.q), _ptr(m.scales),
                  None if m.biases is None else _ptr(m.biases))

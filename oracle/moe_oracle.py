@@ -26,6 +26,15 @@ and section:
 [PR1190]  mlx-lm pull request "Add DeepSeek-V4 model and safetensors/tokenizer
           fallback handling" -- description: E8M0 scales are unsigned
           exponents, 2^(b-127).
+[PR1192-FP8]  the same pull request's review thread on re-quantising from the
+          FP8 source: e4m3 weight bytes with e8m0 block scales decode through
+          MLX's mxfp8 mode with group_size=32 (four weight bytes per uint32
+          word, eight words per scale); the checkpoint's 128x128 block
+          scales are repeated four times along the input axis and 128 times
+          along the output axis to reach that grouping.
+[CARD-MLX4-SRC]  model card "DeepSeek-V4-Flash-MLX-4bit", the note after
+          "What this port implements": the source checkpoint stores most
+          matmuls as FP8 e4m3 with e8m0 128x128 block scales.
 [CARD-MIXED]  model card "DeepSeek-V4-Flash-0731-MLX-Serve-mixed-2-3-8bit",
           precision table (w1/w3 affine 2-bit g128, w2 affine 3-bit g128,
           shared experts 8-bit g64) and conversion notes (fp4 e2m1 with e8m0
@@ -50,7 +59,8 @@ from typing import Callable, Dict, Optional, Sequence, Tuple
 import numpy as np
 
 __all__ = [
-    "E2M1_VALUES", "unpack_codes", "e8m0_value", "dequant_affine", "dequant_mxfp4",
+    "E2M1_VALUES", "E4M3_VALUES", "unpack_codes", "e8m0_value", "dequant_affine", "dequant_mxfp4",
+    "dequant_mxfp8", "block128_scales_to_group32",
     "dequant", "router_logits", "sqrtsoftplus", "topk_select", "renormalize",
     "route_learned", "route_hash", "permute", "silu", "swiglu_ffn", "combine",
     "round_bf16", "forward", "parity_stats",
@@ -63,6 +73,28 @@ __all__ = [
 # subnormal (0 or 0.5).  Code 8 is negative zero.
 E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0,
                         -0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0], dtype=np.float64)
+
+
+
+def _e4m3_table() -> np.ndarray:
+    """e4m3 (the "fn" variant: no infinities): sign bit 7, exponent bits 6..3
+    with bias 7, mantissa bits 2..0; exponent 0 is subnormal (m/8 * 2^-6);
+    exponent 15 with mantissa 7 is NaN, so the largest finite value is 448."""
+    out = np.empty(256, dtype=np.float64)
+    for code in range(256):
+        sign = -1.0 if code & 0x80 else 1.0
+        exp = (code >> 3) & 0xF
+        man = code & 0x7
+        if exp == 0xF and man == 0x7:
+            out[code] = np.nan
+        elif exp == 0:
+            out[code] = sign * (man / 8.0) * 2.0 ** -6
+        else:
+            out[code] = sign * (1.0 + man / 8.0) * 2.0 ** (exp - 7)
+    return out
+
+
+E4M3_VALUES = _e4m3_table()
 
 
 def unpack_codes(words: np.ndarray, bits: int, n: int) -> np.ndarray:
@@ -99,11 +131,30 @@ def dequant_mxfp4(words, scales_u8, n_in: int) -> np.ndarray:
     return E2M1_VALUES[c] * np.repeat(e8m0_value(scales_u8), 32, axis=-1)
 
 
+def dequant_mxfp8(words, scales_u8, n_in: int) -> np.ndarray:
+    """W[o, i] = e4m3(byte i of row o) * 2^(e[o, i//32] - 127), in fp64
+    [PR1192-FP8].  Bytes are the same LSB-first stream with 8-bit codes:
+    byte i of a row is element i."""
+    c = unpack_codes(words, 8, n_in)
+    return E4M3_VALUES[c] * np.repeat(e8m0_value(scales_u8), 32, axis=-1)
+
+
+def block128_scales_to_group32(block_scales, n_out: int, n_in: int) -> np.ndarray:
+    """Per-(row, 32-input group) e8m0 bytes from 128x128 block scales
+    [CARD-MLX4-SRC; PR1192-FP8]: row o, group g takes block (o // 128, g // 4)."""
+    bs = np.asarray(block_scales)
+    rows = np.arange(n_out) // 128
+    groups = np.arange(n_in // 32) // 4
+    return bs[rows[:, None], groups[None, :]]
+
+
 def dequant(fmt: str, bits: int, group: int, n_in: int, words, scales, biases) -> np.ndarray:
     if fmt == "affine":
         return dequant_affine(words, scales, biases, bits, group, n_in)
     if fmt == "mxfp4":
         return dequant_mxfp4(words, scales, n_in)
+    if fmt == "mxfp8":
+        return dequant_mxfp8(words, scales, n_in)
     raise ValueError(fmt)
 
 

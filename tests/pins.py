@@ -127,6 +127,58 @@ def pin_mxfp4_dequant():
     assert W2[0, 0] == -6.0 and W2[0, 1] == 1.5
 
 
+def pin_e4m3_table():
+    """e4m3 decode for all 256 bytes against torch's float8_e4m3fn widening,
+    plus hand-derived values (1.0, the largest finite 448, the smallest
+    subnormal 2^-9 and normal 2^-6, -1.0, -0.0, NaN)."""
+    b = torch.arange(0, 256, dtype=torch.int32).to(torch.uint8)
+    lib = b.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = oracle.E4M3_VALUES
+    assert np.array_equal(np.isnan(got), np.isnan(lib))
+    ok = ~np.isnan(lib)
+    assert np.array_equal(got[ok], lib[ok]) and np.array_equal(np.signbit(got[ok]), np.signbit(lib[ok]))
+    hand = {0x38: 1.0, 0x7E: 448.0, 0x01: 2.0 ** -9, 0x08: 2.0 ** -6, 0xB8: -1.0, 0x3F: 1.875, 0x07: 7 * 2.0 ** -9}
+    for code, want in hand.items():
+        assert got[code] == want, (hex(code), got[code], want)
+    assert got[0x80] == 0.0 and np.signbit(got[0x80])
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF])
+    assert np.nanmax(got) == 448.0
+
+
+def pin_mxfp8_dequant():
+    """mxfp8 rows decode byte-by-byte (torch e4m3 widening times the e8m0
+    power of two); byte i of a row is element i; every value is exact in bf16."""
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 256, size=(3, 96))
+    codes[(codes & 0x7F) == 0x7F] = 0x38           # no NaN codes in weights
+    scales = rng.integers(118, 132, size=(3, 3)).astype(np.uint8)
+    words = np.stack([bigint_words(r, 8) for r in codes])
+    W = oracle.dequant_mxfp8(words, scales, 96)
+    f8 = torch.from_numpy(codes.astype(np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for r in range(3):
+        for i in range(96):
+            want = f8[r, i] * math.ldexp(1.0, int(scales[r, i // 32]) - 127)
+            assert W[r, i] == want, (r, i, W[r, i], want)
+    t = torch.from_numpy(W)
+    assert torch.equal(t.to(torch.bfloat16).double(), t)
+    # little-endian bytes: the word 0x003F00B8 holds elements (-1.0, 0, 1.875, 0)
+    W2 = oracle.dequant_mxfp8(np.array([[0x003F00B8] + [0] * 7], np.uint32), np.array([[127]], np.uint8), 32)
+    assert W2[0, :4].tolist() == [-1.0, 0.0, 1.875, 0.0]
+
+
+def pin_block128_scales():
+    """128x128 block scales spread to (row, 32-input group): element (o, i)
+    takes block (o // 128, i // 128), checked element by element."""
+    rng = np.random.default_rng(6)
+    n_out, n_in = 300, 512
+    bs = rng.integers(100, 140, size=((n_out + 127) // 128, n_in // 128)).astype(np.uint8)
+    g = oracle.block128_scales_to_group32(bs, n_out, n_in)
+    assert g.shape == (n_out, n_in // 32)
+    for o in range(n_out):
+        for i in range(0, n_in, 7):
+            assert g[o, i // 32] == bs[o // 128, i // 128], (o, i)
+
+
 # ---------------------------------------------------------------- routing
 def pin_sqrtsoftplus():
     with open(os.path.join(GOLDEN, "sqrtsoftplus.txt")) as fh:
@@ -326,4 +378,4 @@ def pin_round_bf16():
 ALL_PINS = [pin_e2m1_table, pin_e8m0, pin_unpack_golden, pin_unpack_bigint, pin_affine_dequant,
             pin_mxfp4_dequant, pin_sqrtsoftplus, pin_topk_bruteforce, pin_route_learned,
             pin_route_hash, pin_permutation, pin_dense_equivalence, pin_single_expert_swiglu,
-            pin_round_bf16]
+            pin_round_bf16, pin_e4m3_table, pin_mxfp8_dequant, pin_block128_scales]

@@ -86,3 +86,11 @@ def test_binding_fails_loudly_without_library(tmp_path):
     from bit_quantized_moe_route_b200 import _lib
     with pytest.raises(ImportError):
         _lib.load_library(str(tmp_path / "missing.so"))
+
+
+def test_binding_rejects_unknown_pack_format():
+    import types
+    from bit_quantized_moe_route_b200 import _lib
+    m = types.SimpleNamespace(fmt="mxfp8", bits=8, group=32, q=None, scales=None, biases=None)
+    with pytest.raises(ValueError):
+        _lib.qmat(m)

@@ -54,6 +54,18 @@ def _bad_e2m1():
     return t
 
 
+def _bad_e4m3():
+    t = om.E4M3_VALUES.copy()
+    return t * 0.5          # exponent bias 8 instead of 7
+
+
+def _block_scales_wrong_group(bs, n_out, n_in):
+    # eight 32-input groups per block (the word count per scale) instead of four
+    bs = np.asarray(bs)
+    g = np.minimum(np.arange(n_in // 32) // 8, bs.shape[1] - 1)
+    return bs[(np.arange(n_out) // 128)[:, None], g[None, :]]
+
+
 def _round_trunc(a):
     m, e = np.frexp(np.asarray(a, np.float64))
     return np.ldexp(np.trunc(m * 256) / 256, e)
@@ -70,6 +82,8 @@ MUTATIONS = [
     ("silu", _bad_silu, [pins.pin_single_expert_swiglu, pins.pin_dense_equivalence]),
     ("combine", _unweighted_combine, [pins.pin_dense_equivalence]),
     ("round_bf16", _round_trunc, [pins.pin_round_bf16]),
+    ("E4M3_VALUES", _bad_e4m3(), [pins.pin_e4m3_table, pins.pin_mxfp8_dequant]),
+    ("block128_scales_to_group32", _block_scales_wrong_group, [pins.pin_block128_scales]),
 ]
 
 
