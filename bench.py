@@ -64,6 +64,39 @@ def peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
 
 
+NOMINAL_HBM_GBS = 8000.0       # B200 HBM3e, the figure the layer's bandwidth target is set against
+NOMINAL_F16_TFLOPS = 2250.0    # B200 dense fp16/bf16 tensor rate
+
+
+def roofline_entry(dom, dom_ms, work, kflops, tensor_path, peak, traffic):
+    """The binding roofline of the dominant kernel `dom` (mean launch time
+    `dom_ms`): tensor FLOPs or HBM bytes, whichever it is closer to (small
+    batches on the tensor-core path stream weights far below the machine
+    balance point).  `peak` = (hbm GB/s, bf16 burst TFLOP/s, bf16 sustained
+    TFLOP/s, "measured"|"fallback")."""
+    hbm, bf16, bf16_sus, peak_kind = peak
+    sec = dom_ms * 1e-3
+    tflops_dom = kflops.get(dom, 0.0) / sec / 1e12 if tensor_path else 0.0
+    gbs_dom = work.get(dom, 0) / sec / 1e9
+    if tensor_path and dom in kflops and tflops_dom / bf16_sus >= gbs_dom / hbm:
+        # fp16 x fp16 -> fp32 tcgen05 MMAs: the nominal fp16 and bf16 dense rates are equal,
+        # so the measured bf16 cuBLAS rate is the denominator (sustained: the kernel runs
+        # inside a long back-to-back step loop under the power cap)
+        return {"bound": "tensor", "kernel": dom, "achieved": tflops_dom, "peak": bf16_sus, "unit": "TFLOP/s",
+                "frac": tflops_dom / bf16_sus, "traffic": traffic,
+                "peak_kind": f"{peak_kind} bf16_tflops_sustained (cuBLAS; fp16 nominal = bf16 nominal)",
+                "frac_of_burst_peak": tflops_dom / bf16, "frac_of_nominal": tflops_dom / NOMINAL_F16_TFLOPS,
+                "nominal_peak": NOMINAL_F16_TFLOPS, "algorithmic_flops_per_launch": kflops[dom],
+                "algorithmic_bytes_per_launch": work.get(dom, 0), "hbm_frac": gbs_dom / hbm}
+    out = {"bound": "hbm", "kernel": dom, "achieved": gbs_dom, "peak": hbm, "unit": "GB/s",
+           "frac": gbs_dom / hbm, "traffic": traffic, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
+           "frac_of_nominal": gbs_dom / NOMINAL_HBM_GBS, "nominal_peak": NOMINAL_HBM_GBS,
+           "algorithmic_bytes_per_launch": work.get(dom, 0)}
+    if tensor_path and dom in kflops:
+        out["tensor_frac"] = tflops_dom / bf16_sus
+    return out
+
+
 def src_hash(files=None):
     """Hash of the kernel sources (the listed csrc files, else all of them):
     a stored ncu traffic figure only applies while its kernel is unchanged."""
@@ -413,28 +446,7 @@ def ours_arm(args):
         P_ = T * k + (T if inp.shared is not None else 0)
         for lab in ("ffn_w13_swiglu", "ffn_w2"):
             work[lab] -= P_ * max(c["f"], fs_) * 2
-    # the binding roofline of the dominant kernel: tensor FLOPs or HBM bytes,
-    # whichever it is closer to (small batches on the tensor-core path stream
-    # weights far below the machine balance point)
-    tflops_dom = kflops.get(dom, 0.0) / (dom_ms * 1e-3) / 1e12 if tensor_path else 0.0
-    gbs_dom = work.get(dom, 0) / (dom_ms * 1e-3) / 1e9
-    if tensor_path and dom in kflops and tflops_dom / bf16_sus >= gbs_dom / hbm:
-        # fp16 x fp16 -> fp32 tcgen05 MMAs: the nominal fp16 and bf16 dense rates are equal,
-        # so the measured bf16 cuBLAS rate is the denominator (sustained: the kernel runs
-        # inside a long back-to-back step loop under the power cap)
-        tflops = kflops[dom] / (dom_ms * 1e-3) / 1e12
-        roofline = {"bound": "tensor", "kernel": dom, "achieved": tflops, "peak": bf16_sus, "unit": "TFLOP/s",
-                    "frac": tflops / bf16_sus, "traffic": traffic,
-                    "peak_kind": f"{peak_kind} bf16_tflops_sustained (cuBLAS; fp16 nominal = bf16 nominal)",
-                    "frac_of_burst_peak": tflops / bf16, "algorithmic_flops_per_launch": kflops[dom],
-                    "algorithmic_bytes_per_launch": work.get(dom, 0),
-                    "hbm_frac": work.get(dom, 0) / (dom_ms * 1e-3) / 1e9 / hbm}
-    else:
-        roofline = {"bound": "hbm", "kernel": dom, "achieved": gbs_dom, "peak": hbm, "unit": "GB/s",
-                    "frac": gbs_dom / hbm, "traffic": traffic, "peak_kind": f"{peak_kind} hbm_gbs (copy)",
-                    "algorithmic_bytes_per_launch": work.get(dom, 0)}
-        if tensor_path and dom in kflops:
-            roofline["tensor_frac"] = tflops_dom / bf16_sus
+    roofline = roofline_entry(dom, dom_ms, work, kflops, tensor_path, (hbm, bf16, bf16_sus, peak_kind), traffic)
     layer_bytes = sum(work.values())
     value = whole_job_rate(T, world, ms_per_step)
     line = {

@@ -94,3 +94,37 @@ def test_prefill_flops():
 def test_whole_job_rate_is_tokens_over_slowest_time():
     assert bench.whole_job_rate(1, 1, 0.094) == pytest.approx(1 / 94e-6)
     assert bench.whole_job_rate(4096, 8, 2.5) == pytest.approx(8 * 4096 / 2.5e-3)
+
+
+PEAK = (6539.5, 1624.7, 1376.7, "measured")
+
+
+def test_roofline_decode_is_hbm_bound():
+    work = {"ffn_w13_swiglu": 93_405_184, "ffn_w2": 46_882_816}
+    r = bench.roofline_entry("ffn_w13_swiglu", 0.042, work, {}, False, PEAK, 93_613_824)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == 6539.5
+    assert r["achieved"] == pytest.approx(93_405_184 / 42e-6 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6539.5)
+    assert r["frac_of_nominal"] == pytest.approx(r["achieved"] / 8000.0)
+    assert r["traffic"] == 93_613_824 and "tensor_frac" not in r
+
+
+def test_roofline_prefill_is_tensor_bound():
+    flops = 2.0 * 4096 * 8 * 2 * 4096 * 2048
+    r = bench.roofline_entry("ffn_w13_swiglu", 1.40, {"ffn_w13_swiglu": 3.0e9}, {"ffn_w13_swiglu": flops}, True,
+                             PEAK, None)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == 1376.7
+    assert r["achieved"] == pytest.approx(flops / 1.40e-3 / 1e12)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1376.7)
+    assert r["frac_of_burst_peak"] == pytest.approx(r["achieved"] / 1624.7)
+    assert r["frac_of_nominal"] == pytest.approx(r["achieved"] / 2250.0)
+
+
+def test_roofline_small_batch_tensor_path_stays_hbm_bound():
+    # 32 tokens over ~160 experts: few flops per weight byte
+    flops = 2.0 * 32 * 8 * 2 * 4096 * 2048
+    r = bench.roofline_entry("ffn_w13_swiglu", 0.758, {"ffn_w13_swiglu": 1.49e9}, {"ffn_w13_swiglu": flops}, True,
+                             PEAK, None)
+    assert r["bound"] == "hbm"
+    assert r["tensor_frac"] == pytest.approx(flops / 0.758e-3 / 1e12 / 1376.7)
+    assert r["tensor_frac"] < r["frac"]
