@@ -94,3 +94,20 @@ def test_binding_rejects_unknown_pack_format():
     m = types.SimpleNamespace(fmt="mxfp8", bits=8, group=32, q=None, scales=None, biases=None)
     with pytest.raises(ValueError):
         _lib.qmat(m)
+
+
+def test_plain_c_caller(lib, tmp_path):
+    """The header compiles as strict C99 and a C program links and calls the library."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    libdir = os.path.join(ROOT, "bit_quantized_moe_route_b200")
+    exe = str(tmp_path / "abi_from_c")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "abi_from_c.c"), "-L", libdir, "-lmoe_lowbit",
+                    f"-Wl,-rpath,{libdir}", "-o", exe], check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.startswith("ok ")
