@@ -114,6 +114,9 @@ typedef struct {
  * hash_mode != 0 selects tid2eid routing (top_k = table width).  vocab is
  * the number of tid2eid rows (hash mode only).  d_ff_shared > 0 declares
  * one always-on shared expert of that hidden width (0: none).
+ * n_experts is the layer's own routed expert count: a REAP-pruned layer
+ * [CARD-MLX4 "REAP-pruned builds"] passes the number of experts it kept and
+ * the survivors' router rows and packs, so routing renormalises over them.
  * Limits: 1 <= T, 32 <= d_model, d_ff, d_ff_shared <= 8192 and multiples of
  * 32 and of every group size used; 1 <= top_k <= min(n_experts, 32);
  * n_experts <= 1024.
