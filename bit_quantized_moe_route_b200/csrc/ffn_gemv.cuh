@@ -323,29 +323,31 @@ __global__ void __launch_bounds__(256)
 combine_kernel(const float* __restrict__ y, const int* __restrict__ inv, const float* __restrict__ w,
                const float* __restrict__ y_shared, __nv_bfloat16* __restrict__ out, int T, int k, int d) {
   pdl_wait();  // y comes from the kernel before (possibly launched programmatically)
-  const int t = blockIdx.y;
   const int c4 = blockIdx.x * blockDim.x + threadIdx.x;
   if (c4 * 4 >= d) return;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < k; ++j) {
-    const int pidx = inv[(size_t)t * k + j];
-    const float wt = w[(size_t)t * k + j];
-    const float4 v = reinterpret_cast<const float4*>(y + (size_t)pidx * d)[c4];
-    acc.x = fmaf(wt, v.x, acc.x);
-    acc.y = fmaf(wt, v.y, acc.y);
-    acc.z = fmaf(wt, v.z, acc.z);
-    acc.w = fmaf(wt, v.w, acc.w);
+  // tokens stride over gridDim.y (at most 65535 rows of blocks per launch)
+  for (int t = blockIdx.y; t < T; t += gridDim.y) {
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const int pidx = inv[(size_t)t * k + j];
+      const float wt = w[(size_t)t * k + j];
+      const float4 v = reinterpret_cast<const float4*>(y + (size_t)pidx * d)[c4];
+      acc.x = fmaf(wt, v.x, acc.x);
+      acc.y = fmaf(wt, v.y, acc.y);
+      acc.z = fmaf(wt, v.z, acc.z);
+      acc.w = fmaf(wt, v.w, acc.w);
+    }
+    if (y_shared) {
+      const float4 v = reinterpret_cast<const float4*>(y_shared + (size_t)t * d)[c4];
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(out + (size_t)t * d)[c4] = pk;
   }
-  if (y_shared) {
-    const float4 v = reinterpret_cast<const float4*>(y_shared + (size_t)t * d)[c4];
-    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-  }
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-  uint2 pk;
-  pk.x = *reinterpret_cast<uint32_t*>(&lo);
-  pk.y = *reinterpret_cast<uint32_t*>(&hi);
-  reinterpret_cast<uint2*>(out + (size_t)t * d)[c4] = pk;
 }
 
 }  // namespace moe

@@ -752,7 +752,7 @@ moe_status_t launch_combine(const moe_dims_t& d, const float* y, const int* inv,
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // combine_kernel waits for y itself
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(ceil_div(d.d_model / 4, 256), d.T);
+  cfg.gridDim = dim3(ceil_div(d.d_model / 4, 256), std::min(d.T, 65535));
   cfg.blockDim = dim3(256);
   cfg.stream = s;
   cfg.attrs = attr;
