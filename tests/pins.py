@@ -153,6 +153,8 @@ def pin_mxfp8_dequant():
     codes[(codes & 0x7F) == 0x7F] = 0x38           # no NaN codes in weights
     scales = rng.integers(118, 132, size=(3, 3)).astype(np.uint8)
     words = np.stack([bigint_words(r, 8) for r in codes])
+    # the review thread's count: group_size 32 at 8 bits is 8 uint32 words per scale
+    assert words.shape[1] // scales.shape[1] == 8
     W = oracle.dequant_mxfp8(words, scales, 96)
     f8 = torch.from_numpy(codes.astype(np.uint8)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
     for r in range(3):
