@@ -128,3 +128,21 @@ def test_roofline_small_batch_tensor_path_stays_hbm_bound():
     assert r["bound"] == "hbm"
     assert r["tensor_frac"] == pytest.approx(flops / 0.758e-3 / 1e12 / 1376.7)
     assert r["tensor_frac"] < r["frac"]
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "hash", "mixed", "prefill"])
+def test_every_workload_accounts_and_describes(name):
+    """kernel_work and workload_desc run for each layer configuration the
+    benchmark knows, with a routing that touches min(E, T*k) experts."""
+    from synthetic import CONFIGS
+    c = dict(CONFIGS[name], name=name)
+    inp = layer(c["T"], c["d"], c["E"], c["k"], c["f"], c["w13"], c["w2"], shared=c["shared"],
+                f_shared=c["f_shared"], routing=c["routing"])
+    ids = (np.arange(c["T"] * c["k"]) % c["E"]).reshape(c["T"], c["k"])
+    work, flops, n_act, weight_bytes, kflops = bench.kernel_work(inp, ids)
+    assert n_act == min(c["E"], c["T"] * c["k"])
+    assert all(v > 0 for v in work.values() if v is not None)
+    assert flops == 2 * c["T"] * c["k"] * 3 * c["d"] * c["f"] + 2 * c["T"] * 3 * c["d"] * c["f_shared"]
+    assert ("route_hash" in work) == (c["routing"] == "hash")
+    desc = bench.workload_desc(c)
+    assert desc["workload"] == name and desc["T"] == c["T"] and desc["n_experts"] == c["E"]
