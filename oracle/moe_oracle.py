@@ -62,7 +62,7 @@ __all__ = [
     "E2M1_VALUES", "E4M3_VALUES", "unpack_codes", "e8m0_value", "dequant_affine", "dequant_mxfp4",
     "dequant_mxfp8", "block128_scales_to_group32",
     "dequant", "router_logits", "sqrtsoftplus", "topk_select", "renormalize",
-    "route_learned", "route_hash", "permute", "silu", "swiglu_ffn", "combine",
+    "route_learned", "route_hash", "route_forced", "permute", "silu", "swiglu_ffn", "combine",
     "round_bf16", "forward", "parity_stats",
 ]
 
@@ -290,26 +290,50 @@ def round_bf16(a: np.ndarray) -> np.ndarray:
 ExpertFetch = Callable[[str, int], Tuple[np.ndarray, np.ndarray, Optional[np.ndarray]]]
 
 
+def route_forced(x, w_router, forced_ids):
+    """Forced routing: the experts are given (e.g. the ids another
+    implementation selected for a token whose k-th and (k+1)-th keys nearly
+    tie); the weights are computed for them exactly as in learned routing,
+    w = s[ids] / sum(s[ids]) with the unbiased scores, in the given slot order.
+    """
+    ids = np.asarray(forced_ids, np.int64)
+    L = router_logits(x, w_router)
+    s = sqrtsoftplus(L)
+    return ids, renormalize(np.take_along_axis(s, ids, axis=1)), L
+
+
 def forward(dims: Dict, x: np.ndarray, *, router_w=None, router_b=None, token_ids=None,
             tid2eid=None, fetch: ExpertFetch, fmts: Dict[str, Tuple[str, int, int]],
             shared_fetch: Optional[ExpertFetch] = None, shared_fmts=None,
-            tokens: Optional[Sequence[int]] = None) -> Dict[str, np.ndarray]:
+            tokens: Optional[Sequence[int]] = None,
+            forced_ids: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
     """Run the layer for all tokens' routing and the requested tokens' outputs.
 
     dims: T, d, E, k, f, f_shared, routing ("learned"|"hash").
     fetch(name, e) -> packs of expert e for name in {"w1","w3","w2"}.
     fmts[name] = (fmt, bits, group).  tokens: subset whose outputs are wanted
     (default: all).  Routing is computed for every token.
+    forced_ids: int [T, k] -- learned routing only: use these experts instead
+    of the top-k selection (weights as in route_forced); "gap" is then the
+    free routing's gap, so near-tie tokens can still be recognised.
     """
     T, d, E, k, f = dims["T"], dims["d"], dims["E"], dims["k"], dims["f"]
     xs = np.asarray(x, np.float64)
     res: Dict[str, np.ndarray] = {}
     if dims["routing"] == "hash":
+        if forced_ids is not None:
+            raise ValueError("forced routing applies to learned routing only")
         ids, w = route_hash(xs, router_w, token_ids, tid2eid)
         gap = np.full(T, np.inf)
     else:
         ids, w, gap, L = route_learned(xs, router_w, router_b, k)
         res["logits"] = L
+        # the selection keys, so a caller can check that another selection
+        # of a near-tie token is also a valid top-k
+        res["keys"] = sqrtsoftplus(L) + (0.0 if router_b is None else np.asarray(router_b, np.float64)[None, :])
+        if forced_ids is not None:
+            res["free_ids"] = ids
+            ids, w, _ = route_forced(xs, router_w, forced_ids)
     res["ids"], res["w"], res["gap"] = ids, w, gap
     offs, rows, inv = permute(ids, E)
     res["expert_offsets"], res["sorted_rows"], res["inv"] = offs, rows, inv

@@ -377,7 +377,85 @@ def pin_round_bf16():
     assert oracle.round_bf16(np.array([1 + 3 * 2 ** -8]))[0] == 1 + 2 ** -6
 
 
+# ---------------------------------------------------------------- parity harness
+def pin_parity_stats():
+    """The output tolerance statistics on hand-computed vectors.
+
+    ref = [3, -4, 0, 1], out = [3.5, -4, 0.25, 1]: |err| = [0.5, 0, 0.25, 0],
+    max|err| = 0.5, rms(ref) = sqrt(26/4), sum|err| / sum|ref| = 0.75 / 8.
+    A second case has a zero in ref where out is not zero (an elementwise
+    relative error would be infinite there) and out's rms differing from ref's.
+    """
+    st = oracle.parity_stats(np.array([3.5, -4.0, 0.25, 1.0]), np.array([3.0, -4.0, 0.0, 1.0]))
+    assert st["max_err"] == 0.5
+    assert abs(st["rms_ref"] - math.sqrt(6.5)) < 1e-15
+    assert abs(st["max_err_over_rms"] - 0.5 / math.sqrt(6.5)) < 1e-15
+    assert abs(st["mean_rel_err"] - 0.09375) < 1e-15
+    st = oracle.parity_stats(np.array([[0.0, 2.0], [10.0, 1.0]]), np.array([[1.0, 0.0], [2.0, 1.0]]))
+    # |err| = [1, 2, 8, 0]; rms(ref) = sqrt(6/4); sum|ref| = 4
+    assert st["max_err"] == 8.0
+    assert abs(st["max_err_over_rms"] - 8.0 / math.sqrt(1.5)) < 1e-14
+    assert abs(st["mean_rel_err"] - 11.0 / 4.0) < 1e-15
+    # identical arrays: zero error; the statistics are symmetric in nothing else
+    z = oracle.parity_stats(np.ones(5), np.ones(5))
+    assert z["max_err"] == 0.0 and z["mean_rel_err"] == 0.0 and z["rms_ref"] == 1.0
+
+
+def pin_forward_token_subset():
+    """forward(tokens=S) gives, for each token of S, the row the all-tokens
+    run gives (same routing, same slot outputs, same combine), up to fp64
+    rounding order (BLAS blocks a matrix product differently per batch)."""
+    from synthetic import CONFIGS
+    for name, over, subset in (("tiny", {}, [3, 0, 2]),
+                               ("tiny", dict(shared=("affine", 8, 64), f_shared=64, T=9, seed=41), [8, 1, 1, 4]),
+                               ("tiny", dict(routing="hash", vocab=61, T=7, seed=42), [6, 2])):
+        cfg = dict(CONFIGS[name])
+        cfg.update(over)
+        inp = make_custom(cfg)
+        full = oracle_run(inp)
+        part = oracle_run(inp, tokens=subset)
+        assert list(part["tokens"]) == list(subset)
+        for a, t in enumerate(subset):
+            scale = np.abs(full["out"]).max()
+            assert np.allclose(part["out"][a], full["out"][t], rtol=1e-12, atol=1e-13 * scale), (over, t)
+            assert np.allclose(part["y_slots"][a], full["y_slots"][t], rtol=1e-12, atol=1e-13 * scale), (over, t)
+        assert np.array_equal(part["ids"], full["ids"]) and np.array_equal(part["w"], full["w"])
+
+
+def pin_forced_routing():
+    """Forced routing: with the oracle's own ids it reproduces the free run;
+    with other ids the output is the dense mixture gated by those ids with
+    weights = renormalised sqrtsoftplus of their fp64 logits (scipy softplus),
+    whatever the selection bias; slot order permutes weights and slot outputs
+    only."""
+    from scipy.special import softplus
+    from synthetic import CONFIGS
+    cfg = dict(CONFIGS["tiny"])
+    cfg.update(T=6, seed=43, bias_std=0.3)
+    inp = make_custom(cfg)
+    free = oracle_run(inp)
+    same = oracle_run(inp, forced_ids=free["ids"])
+    assert np.array_equal(same["out"], free["out"]) and np.array_equal(same["w"], free["w"])
+    rng = np.random.default_rng(44)
+    T, E, k = cfg["T"], cfg["E"], cfg["k"]
+    forced = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+    res = oracle_run(inp, forced_ids=forced)
+    assert np.array_equal(res["ids"], forced) and np.array_equal(res["free_ids"], free["ids"])
+    assert np.array_equal(res["gap"], free["gap"])
+    L = inp.x.double().numpy() @ inp.router_w.double().numpy().T
+    s = np.sqrt(softplus(L))
+    sel = np.take_along_axis(s, forced, 1)
+    assert np.allclose(res["w"], sel / sel.sum(1, keepdims=True), rtol=1e-12)
+    dense = _dense_reference(inp, {"ids": forced, "w": sel / sel.sum(1, keepdims=True)})
+    assert np.abs(res["out"] - dense).max() / np.abs(dense).max() < 1e-12
+    swapped = forced[:, ::-1].copy()
+    res2 = oracle_run(inp, forced_ids=swapped)
+    assert np.allclose(res2["w"], res["w"][:, ::-1], rtol=1e-15)
+    assert np.allclose(res2["out"], res["out"], rtol=1e-13, atol=1e-15)
+
+
 ALL_PINS = [pin_e2m1_table, pin_e8m0, pin_unpack_golden, pin_unpack_bigint, pin_affine_dequant,
             pin_mxfp4_dequant, pin_sqrtsoftplus, pin_topk_bruteforce, pin_route_learned,
             pin_route_hash, pin_permutation, pin_dense_equivalence, pin_single_expert_swiglu,
-            pin_round_bf16, pin_e4m3_table, pin_mxfp8_dequant, pin_block128_scales]
+            pin_round_bf16, pin_e4m3_table, pin_mxfp8_dequant, pin_block128_scales, pin_parity_stats,
+            pin_forward_token_subset, pin_forced_routing]

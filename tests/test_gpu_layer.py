@@ -11,7 +11,7 @@ import torch
 
 import bit_quantized_moe_route_b200 as moe
 from synthetic import make_custom
-from tests.gpu_utils import TIE_EPS, bf16_to_np, check_output
+from tests.gpu_utils import check_layer
 from tests.helpers import oracle_run
 
 pytestmark = pytest.mark.gpu
@@ -25,17 +25,15 @@ def test_layer_object_matches_oracle_over_batch_sizes(cuda_device):
     inp = make_custom(CFG, cuda_device)
     c = inp.cfg
     res = oracle_run(inp)
-    ties = set(np.nonzero(res["gap"] < TIE_EPS)[0].tolist())
     layer = moe.MoELayer(d_model=c["d"], d_ff=c["f"], n_experts=c["E"], top_k=c["k"], max_tokens=c["T"],
                          w1=inp.w1, w3=inp.w3, w2=inp.w2, router_w=inp.router_w, router_b=inp.router_b,
                          shared=inp.shared, device=cuda_device)
     for T in (2, 37, c["T"]):
         ids = torch.empty(T, c["k"], dtype=torch.int32, device=cuda_device)
-        out = layer(inp.x[:T], topk_ids=ids)
+        w = torch.empty(T, c["k"], dtype=torch.float32, device=cuda_device)
+        out = layer(inp.x[:T], topk_ids=ids, topk_w=w)
         torch.cuda.synchronize()
-        keep = [t for t in range(T) if t not in ties]
-        assert np.array_equal(ids.cpu().numpy().astype(np.int64)[keep], res["ids"][:T][keep]), f"T={T}: expert ids"
-        check_output(bf16_to_np(out)[keep], res["out"][:T][keep], f"layer T={T}")
+        check_layer(inp, res, out, ids, w, f"layer T={T}", tokens=np.arange(T))
         assert layer.device_error() == 0
 
 

@@ -7,7 +7,7 @@ import torch
 
 import bit_quantized_moe_route_b200 as moe
 from synthetic import CONFIGS, make_custom, make_inputs
-from tests.gpu_utils import bf16_to_np, check_output, check_routing, dims_for, run_forward
+from tests.gpu_utils import bf16_to_np, check_layer, check_output, check_routing, dims_for, run_forward
 from tests.helpers import oracle_run
 
 pytestmark = pytest.mark.gpu
@@ -63,9 +63,7 @@ def test_forward_matches_oracle(device, name):
     inp = make_custom(VARIANTS[name], device)
     res = oracle_run(inp)
     out, ids, w, ws = run_forward(inp)
-    ties = check_routing(res, ids, w, hash_mode=inp.cfg["routing"] == "hash")
-    keep = np.setdiff1d(np.arange(inp.cfg["T"]), ties)
-    check_output(bf16_to_np(out)[keep], res["out"][keep], name)
+    check_layer(inp, res, out, ids, w, name)
     assert moe.read_device_error(ws) == 0
 
 

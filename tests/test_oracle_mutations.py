@@ -71,6 +71,41 @@ def _round_trunc(a):
     return np.ldexp(np.trunc(m * 256) / 256, e)
 
 
+def _stats_rms_of_out(out, ref):
+    st = _ORIG_STATS(out, ref)
+    out = np.asarray(out, np.float64)
+    rms = float(np.sqrt(np.mean(out * out)))
+    st["rms_ref"] = rms
+    st["max_err_over_rms"] = st["max_err"] / rms if rms > 0 else 0.0
+    return st
+
+
+def _stats_mean_err(out, ref):
+    st = _ORIG_STATS(out, ref)
+    err = np.abs(np.asarray(out, np.float64) - np.asarray(ref, np.float64))
+    st["mean_rel_err"] = float(err.mean() / np.abs(np.asarray(ref, np.float64)).sum())
+    return st
+
+
+def _stats_elementwise_rel(out, ref):
+    st = _ORIG_STATS(out, ref)
+    out, ref = np.asarray(out, np.float64), np.asarray(ref, np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        st["mean_rel_err"] = float(np.mean(np.abs(out - ref) / np.abs(ref)))
+    return st
+
+
+def _forced_biased_weights(x, w_router, forced_ids):
+    # weights from the biased keys would need the bias; a plausible slip is
+    # to take the weights without renormalising them
+    ids = np.asarray(forced_ids, np.int64)
+    s = om.sqrtsoftplus(om.router_logits(x, w_router))
+    return ids, np.take_along_axis(s, ids, axis=1), None
+
+
+_ORIG_STATS = om.parity_stats
+
+
 MUTATIONS = [
     ("E2M1_VALUES", _bad_e2m1(), [pins.pin_e2m1_table, pins.pin_mxfp4_dequant]),
     ("e8m0_value", lambda e: np.ldexp(1.0, np.asarray(e, np.int64) - 128), [pins.pin_e8m0, pins.pin_mxfp4_dequant]),
@@ -84,6 +119,10 @@ MUTATIONS = [
     ("round_bf16", _round_trunc, [pins.pin_round_bf16]),
     ("E4M3_VALUES", _bad_e4m3(), [pins.pin_e4m3_table, pins.pin_mxfp8_dequant]),
     ("block128_scales_to_group32", _block_scales_wrong_group, [pins.pin_block128_scales]),
+    ("parity_stats", _stats_rms_of_out, [pins.pin_parity_stats]),
+    ("parity_stats", _stats_mean_err, [pins.pin_parity_stats]),
+    ("parity_stats", _stats_elementwise_rel, [pins.pin_parity_stats]),
+    ("route_forced", _forced_biased_weights, [pins.pin_forced_routing]),
 ]
 
 

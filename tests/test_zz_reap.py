@@ -77,7 +77,7 @@ GPU_CASES = {
 @pytest.mark.parametrize("name", list(GPU_CASES))
 def test_pruned_expert_counts_match_oracle(cuda_device, name, path):
     import bit_quantized_moe_route_b200 as moe
-    from tests.gpu_utils import bf16_to_np, check_output, check_routing, run_forward
+    from tests.gpu_utils import check_layer, run_forward
     from tests.helpers import oracle_run
     moe.load_library()
     prev = moe.set_ffn_path(moe.FFN_GEMV if path == "gemv" else moe.FFN_TENSOR_CORE)
@@ -87,8 +87,6 @@ def test_pruned_expert_counts_match_oracle(cuda_device, name, path):
         out, ids, w, ws = run_forward(inp)
     finally:
         moe.set_ffn_path(prev)
-    ties = check_routing(res, ids, w)
-    keep = np.setdiff1d(np.arange(inp.cfg["T"]), ties)
-    check_output(bf16_to_np(out)[keep], res["out"][keep], f"{name}/{path}")
+    check_layer(inp, res, out, ids, w, f"{name}/{path}")
     assert moe.read_device_error(ws) == 0
     assert int(torch.as_tensor(ids).max()) < inp.cfg["E"]
