@@ -1,13 +1,17 @@
 """Benchmark of the routed low-bit MoE layer on B200.
 
-python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME|all] [--impl ours|reference]
 
 One step = one full layer forward (routing, permutation, grouped SwiGLU
 expert FFN over packed weights, combine) over one batch of synthetic input
 resident in HBM.  The default workload is the decode layer (T=1 token,
 d_model=4096, 256 routed experts, top-8, d_ff=2048, affine 4-bit group-64
-experts plus an 8-bit shared expert).  L2 is flushed (a 512 MiB write)
-between timed steps, outside the timed events.
+experts plus an 8-bit shared expert).  L2 is flushed between timed steps,
+outside the timed events, by READING a 512 MiB buffer (a read leaves no
+dirty lines whose write-back would compete with the timed weight stream).
+The reported step time is the median over the timed steps (min, mean and
+p90 beside it).  --config all prints one line per layer configuration
+(tiny, hash, mixed, prefill, then the decode line last).
 
 With N > 1 (launched by torchrun) every rank runs an independent replica of
 the layer on its own GPU ("replicas only": the layer has no exchange step on
@@ -43,7 +47,7 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", default="decode")
+    ap.add_argument("--config", default="decode", help="workload name, or 'all' (one line each, decode last)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ffn-path", default="auto", choices=["auto", "gemv", "tc"],
@@ -69,23 +73,26 @@ NOMINAL_F16_TFLOPS = 2250.0    # B200 dense fp16/bf16 tensor rate
 
 
 def roofline_entry(dom, dom_ms, work, kflops, tensor_path, peak, traffic):
-    """The binding roofline of the dominant kernel `dom` (mean launch time
+    """The binding roofline of the dominant kernel `dom` (median launch time
     `dom_ms`): tensor FLOPs or HBM bytes, whichever it is closer to (small
     batches on the tensor-core path stream weights far below the machine
     balance point).  `peak` = (hbm GB/s, bf16 burst TFLOP/s, bf16 sustained
-    TFLOP/s, "measured"|"fallback")."""
+    TFLOP/s, "measured"|"fallback").  The tensor denominator is the burst
+    rate: the kernel runs for about a millisecond inside a few-millisecond
+    step, not in a seconds-long loop; the sustained fraction is reported
+    beside it."""
     hbm, bf16, bf16_sus, peak_kind = peak
     sec = dom_ms * 1e-3
     tflops_dom = kflops.get(dom, 0.0) / sec / 1e12 if tensor_path else 0.0
     gbs_dom = work.get(dom, 0) / sec / 1e9
-    if tensor_path and dom in kflops and tflops_dom / bf16_sus >= gbs_dom / hbm:
+    if tensor_path and dom in kflops and tflops_dom / bf16 >= gbs_dom / hbm:
         # fp16 x fp16 -> fp32 tcgen05 MMAs: the nominal fp16 and bf16 dense rates are equal,
-        # so the measured bf16 cuBLAS rate is the denominator (sustained: the kernel runs
-        # inside a long back-to-back step loop under the power cap)
-        return {"bound": "tensor", "kernel": dom, "achieved": tflops_dom, "peak": bf16_sus, "unit": "TFLOP/s",
-                "frac": tflops_dom / bf16_sus, "traffic": traffic,
-                "peak_kind": f"{peak_kind} bf16_tflops_sustained (cuBLAS; fp16 nominal = bf16 nominal)",
-                "frac_of_burst_peak": tflops_dom / bf16, "frac_of_nominal": tflops_dom / NOMINAL_F16_TFLOPS,
+        # so the measured bf16 cuBLAS rate is the denominator
+        return {"bound": "tensor", "kernel": dom, "achieved": tflops_dom, "peak": bf16, "unit": "TFLOP/s",
+                "frac": tflops_dom / bf16, "traffic": traffic,
+                "peak_kind": f"{peak_kind} bf16_tflops burst (cuBLAS; fp16 nominal = bf16 nominal)",
+                "frac_of_sustained_peak": tflops_dom / bf16_sus, "sustained_peak": bf16_sus,
+                "frac_of_nominal": tflops_dom / NOMINAL_F16_TFLOPS,
                 "nominal_peak": NOMINAL_F16_TFLOPS, "algorithmic_flops_per_launch": kflops[dom],
                 "algorithmic_bytes_per_launch": work.get(dom, 0), "hbm_frac": gbs_dom / hbm}
     out = {"bound": "hbm", "kernel": dom, "achieved": gbs_dom, "peak": hbm, "unit": "GB/s",
@@ -93,7 +100,7 @@ def roofline_entry(dom, dom_ms, work, kflops, tensor_path, peak, traffic):
            "frac_of_nominal": gbs_dom / NOMINAL_HBM_GBS, "nominal_peak": NOMINAL_HBM_GBS,
            "algorithmic_bytes_per_launch": work.get(dom, 0)}
     if tensor_path and dom in kflops:
-        out["tensor_frac"] = tflops_dom / bf16_sus
+        out["tensor_frac"] = tflops_dom / bf16
     return out
 
 
@@ -120,8 +127,14 @@ def workload_desc(cfg):
 
 
 # ---------------------------------------------------------------- algorithmic bytes / flops
-def kernel_work(inp, ids):
-    """Algorithmic bytes (and flops) of each kernel of one forward."""
+def kernel_work(inp, ids, tensor_path=False):
+    """Algorithmic bytes of each kernel label the library can report for one
+    forward (and the flops).  The expert-FFN entries depend on the path: the
+    weight-streaming GEMV runs the shared expert inside the routed launches
+    and keeps h in fp32; the tensor-core path runs it as its own launches
+    (the *_shared labels) and keeps token rows and h in fp16.
+
+    Returns (work, flops, distinct routed experts, weight bytes, kflops)."""
     import numpy as np
     c = inp.cfg
     T, d, E, k, f = c["T"], c["d"], c["E"], c["k"], c["f"]
@@ -131,33 +144,54 @@ def kernel_work(inp, ids):
     b13 = inp.w1.packed_bytes_per_expert() + inp.w3.packed_bytes_per_expert()
     b2 = inp.w2.packed_bytes_per_expert()
     sh13 = sh2 = 0
-    P = T * k
+    Tk = T * k
+    Ts = T if inp.shared is not None else 0
     if inp.shared is not None:
         sh13 = inp.shared[0].packed_bytes_per_expert() + inp.shared[1].packed_bytes_per_expert()
         sh2 = inp.shared[2].packed_bytes_per_expert()
-        P += T
     fs = c.get("f_shared", 0) if inp.shared is not None else 0
     work = {}
+    perm = Tk * 4 * 3 + (E + 1) * 4               # ids in, sorted rows + inverse out, offsets
     if c["routing"] == "hash":
         rows = len(np.unique(ids))
-        work["route_hash"] = T * d * 2 + T * 4 + T * k * 4 + rows * d * 4 + T * k * 8
+        work["route_hash"] = T * d * 2 + T * 4 + Tk * 4 + rows * d * 4 + Tk * 8
+        work["route_hash_permute"] = work["route_hash"] + perm
     else:
         work["router_logits"] = E * d * 4 + T * d * 2 + T * E * 4
-        work["topk"] = T * E * 4 + E * 4 + T * k * 8
-    work["permute"] = T * k * 4 * 3 + (E + 1) * 4
-    work["ffn_w13_swiglu"] = n_act * b13 + sh13 + T * d * 2 + P * max(f, fs) * 4
-    work["ffn_w2"] = n_act * b2 + sh2 + P * max(f, fs) * 4 + P * d * 4
-    work["combine"] = P * d * 4 + T * d * 2 + T * k * 8
-    # tensor-core path: fp16 copy of x, tile plan, and fp16 H (the shared
-    # expert runs as its own launches there)
-    work["gather_f16"] = T * d * 2 + P * d * 2 + T * k * 4
-    work["tile_plan"] = (E + 1) * 4 + ((T * k + 127) // 128 + E) * 16
-    work["ffn_w13_swiglu_shared"] = sh13 + T * d * 2 + T * fs * 2
-    work["ffn_w2_shared"] = sh2 + T * fs * 2 + T * d * 4
+        work["topk"] = T * E * 4 + E * 4 + Tk * 8
+        work["route_topk_permute"] = E * d * 4 + T * d * 2 + E * 4 + Tk * 8 + perm
+    n_chunks = (Tk + 1023) // 1024                 # multi-CTA permutation: per-chunk expert counts
+    work["permute_count"] = Tk * 4 + n_chunks * E * 4
+    work["permute_scan"] = 2 * n_chunks * E * 4 + (E + 1) * 4
+    work["permute"] = perm
+    if tensor_path:
+        work["gather_f16"] = T * d * 2 + (Tk + Ts) * d * 2 + Tk * 4
+        work["tile_plan"] = (E + 1) * 4 + ((Tk + 127) // 128 + E) * 16
+        work["ffn_w13_swiglu"] = n_act * b13 + Tk * d * 2 + Tk * f * 2
+        work["ffn_w2"] = n_act * b2 + Tk * f * 2 + Tk * d * 4
+        work["ffn_w13_swiglu_shared"] = sh13 + Ts * d * 2 + Ts * fs * 2
+        work["ffn_w2_shared"] = sh2 + Ts * fs * 2 + Ts * d * 4
+    else:
+        P = Tk + Ts
+        work["ffn_w13_swiglu"] = n_act * b13 + sh13 + T * d * 2 + P * max(f, fs) * 4
+        work["ffn_w2"] = n_act * b2 + sh2 + P * max(f, fs) * 4 + P * d * 4
+    work["combine"] = (Tk + Ts) * d * 4 + T * d * 2 + Tk * 8
     flops = 2.0 * T * k * 3 * d * f + (2.0 * T * 3 * d * fs if fs else 0.0)
     kflops = {"ffn_w13_swiglu": 2.0 * T * k * 2 * d * f, "ffn_w2": 2.0 * T * k * d * f,
               "ffn_w13_swiglu_shared": 2.0 * T * 2 * d * fs, "ffn_w2_shared": 2.0 * T * d * fs}
     return work, flops, n_act, (n_act * (b13 + b2) + sh13 + sh2), kflops
+
+
+def layer_bytes(work, labels):
+    """Algorithmic bytes of one forward: the kernels that actually ran."""
+    return sum(work.get(lab, 0) for lab in labels)
+
+
+def step_stats(ms):
+    """Median (the reported step), min, mean and p90 of the timed steps."""
+    srt = sorted(ms)
+    return {"median": statistics.median(srt), "min": srt[0], "mean": statistics.mean(srt),
+            "p90": srt[min(len(srt) - 1, int(0.9 * len(srt)))]}
 
 
 # ---------------------------------------------------------------- clocks
@@ -294,9 +328,15 @@ def reference_arm(args):
     import torch
     from synthetic import make_inputs
     dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
-    inp = make_inputs(args.config, dev, **overrides(args))
+    names = CONFIG_ORDER if args.config == "all" else [args.config]
+    for name in names:
+        inp = make_inputs(name, dev, **overrides(args))
+        reference_line(args, inp, 150.0 / len(names))
+
+
+def reference_line(args, inp, budget_total):
+    """One reference-arm line: the oracle on a bounded sample of inp's workload."""
     c = inp.cfg
-    budget_total = 150.0
     step_budget = max(0.5, budget_total / max(1, args.steps + args.warmup))
     times, pairs = [], 0
     desc = ""
@@ -324,25 +364,18 @@ def reference_arm(args):
 
 
 # ---------------------------------------------------------------- our arm
-def ours_arm(args):
-    import numpy as np
+CONFIG_ORDER = ["tiny", "hash", "mixed", "prefill", "decode"]   # --config all: decode (the headline) last
+
+
+def run_config(name, args, dev, world, rank):
+    """Time one layer configuration; returns its JSON line (dict)."""
+    import numpy as np  # noqa: F401
     import torch
-    import torch.distributed as dist
 
     import bit_quantized_moe_route_b200 as moe
     from synthetic import make_inputs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dev = torch.device(f"cuda:{local}")
-    torch.cuda.set_device(dev)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    moe.load_library()
-    moe.set_ffn_path({"auto": moe.FFN_AUTO, "gemv": moe.FFN_GEMV, "tc": moe.FFN_TENSOR_CORE}[args.ffn_path])
-    inp = make_inputs(args.config, dev, **overrides(args))
+    inp = make_inputs(name, dev, **overrides(args))
     c = inp.cfg
     T, d, k = c["T"], c["d"], c["k"]
     dims = moe.make_dims(T, d, c["f"], c["E"], k, c["routing"] == "hash",
@@ -352,31 +385,36 @@ def ours_arm(args):
     out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
     wts = torch.empty(T, k, dtype=torch.float32, device=dev)
-    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    # L2 flush by a read of 512 MiB (> 4x L2) into one small result
+    flush = torch.ones(128 * 1024 * 1024, dtype=torch.int32, device=dev)
+    flush_sum = torch.empty((), dtype=torch.int64, device=dev)
     stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        torch.sum(flush, dtype=torch.int64, out=flush_sum)
 
     def fwd():
         moe.forward(dims, inp.x, inp.token_ids, inp.router_w, inp.router_b, inp.tid2eid, inp.w1, inp.w3, inp.w2,
                     inp.shared, out, ws, topk_ids_out=ids, topk_w_out=wts)
 
     for i in range(max(3, args.warmup)):
-        flush.fill_(i & 0xFF)
+        flush_l2()
         fwd()
     torch.cuda.synchronize()
-    work, flops, n_act, weight_bytes, kflops = kernel_work(inp, ids.cpu().numpy())
 
     # ---- timed region: K forwards, L2 flushed between them (outside the events)
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
     props = torch.cuda.get_device_properties(dev)
-    sampler = ClockSampler("GPU-" + str(props.uuid) if getattr(props, "uuid", None) else str(local))
+    sampler = ClockSampler("GPU-" + str(props.uuid) if getattr(props, "uuid", None) else str(dev.index))
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.2)
     for s in range(args.steps):
-        flush.fill_(s & 0xFF)
+        flush_l2()
         step_ev[s][0].record(stream)
         fwd()
         step_ev[s][1].record(stream)
@@ -384,8 +422,8 @@ def ours_arm(args):
     clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    ms_per_step = max_over_ranks(sum(step_ms) / args.steps, dev)
+    st = step_stats([a.elapsed_time(b) for a, b in step_ev])
+    ms_per_step = max_over_ranks(st["median"], dev)
 
     # ---- per-kernel durations: a second timed pass with CUDA events recorded
     # by the library between its kernels on the same stream (the events add
@@ -395,7 +433,7 @@ def ours_arm(args):
     keep = []
     torch.cuda.synchronize()
     for s in range(k_steps):
-        flush.fill_(s & 0xFF)
+        flush_l2()
         keep.append(moe.set_timing_events(evs[s]))
         fwd()
     torch.cuda.synchronize()
@@ -404,7 +442,7 @@ def ours_arm(args):
     for s in range(k_steps):
         for i, lab in enumerate(labels):
             per_kernel.setdefault(lab, []).append(evs[s][i].elapsed_time(evs[s][i + 1]))
-    kern_ms = {lab: statistics.mean(v) for lab, v in per_kernel.items()}
+    kern_ms = {lab: statistics.median(v) for lab, v in per_kernel.items()}
 
     # ---- end-to-end through the C ABI with host buffers (pinned), copies inside
     x_h = inp.x.cpu().pin_memory()
@@ -415,20 +453,22 @@ def ours_arm(args):
         moe.forward_host(dims, x_h, tok_h, *layer_args, out_h, ws)
     torch.cuda.synchronize()
     e2e_steps = max(10, min(args.steps, 200))
-    e2e_ms = 0.0
+    e2e = []
     for s in range(e2e_steps):
-        flush.fill_(s & 0xFF)
+        flush_l2()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         moe.forward_host(dims, x_h, tok_h, *layer_args, out_h, ws)
         b.record(stream)
         b.synchronize()
-        e2e_ms += a.elapsed_time(b)
-    e2e_ms = max_over_ranks(e2e_ms / e2e_steps, dev)
+        e2e.append(a.elapsed_time(b))
+    e2e_ms = max_over_ranks(statistics.median(e2e), dev)
     h2d = T * d * 2 + (T * 4 if tok_h is not None else 0)
     d2h = T * d * 2
     err = moe.read_device_error(ws)
 
+    tensor_path = "tile_plan" in labels
+    work, flops, n_act, weight_bytes, kflops = kernel_work(inp, ids.cpu().numpy(), tensor_path)
     hbm, bf16, bf16_sus, peak_kind = peaks()
     dom = max(kern_ms, key=kern_ms.get)
     dom_ms = kern_ms[dom]
@@ -440,28 +480,23 @@ def ours_arm(args):
         ent = tj.get(c["name"], {}).get(dom)
         if ent and ent.get("src_hash") == src_hash(ent.get("files")):
             traffic = ent.get("dram_bytes_per_launch")
-    tensor_path = "tile_plan" in labels
-    if tensor_path:  # H is fp16 on the tensor-core path
-        fs_ = c.get("f_shared", 0) if inp.shared is not None else 0
-        P_ = T * k + (T if inp.shared is not None else 0)
-        for lab in ("ffn_w13_swiglu", "ffn_w2"):
-            work[lab] -= P_ * max(c["f"], fs_) * 2
     roofline = roofline_entry(dom, dom_ms, work, kflops, tensor_path, (hbm, bf16, bf16_sus, peak_kind), traffic)
-    layer_bytes = sum(work.values())
+    lbytes = layer_bytes(work, labels)
     value = whole_job_rate(T, world, ms_per_step)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16" if tensor_path else "f32", "data": "synthetic",
         "config": dict(workload_desc(c), ffn_path=args.ffn_path,
-                       l2="flushed by a 512 MiB write between timed steps (outside the events)",
+                       l2="flushed by reading a 512 MiB buffer between timed steps (outside the events)",
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "step_ms": st,
         "roofline": roofline,
-        "layer": {"bytes_per_step": layer_bytes, "weight_bytes": weight_bytes, "distinct_routed_experts": n_act,
-                  "GBps_whole_step": layer_bytes / (ms_per_step * 1e-3) / 1e9,
-                  "frac_whole_step": layer_bytes / (ms_per_step * 1e-3) / 1e9 / hbm,
+        "layer": {"bytes_per_step": lbytes, "weight_bytes": weight_bytes, "distinct_routed_experts": n_act,
+                  "GBps_whole_step": lbytes / (ms_per_step * 1e-3) / 1e9,
+                  "frac_whole_step": lbytes / (ms_per_step * 1e-3) / 1e9 / hbm,
                   "flops_per_step": flops, "TFLOPs_whole_step": flops / (ms_per_step * 1e-3) / 1e12,
-                  "kernel_ms": kern_ms},
+                  "kernel_ms_median": kern_ms, "kernels": labels},
         "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": len(labels) * args.steps,
@@ -470,11 +505,36 @@ def ours_arm(args):
         "device_error": err,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_tok, desc, done, blas = oracle_sample_time(inp, args.cpu_budget)
+        budget = args.cpu_budget if name == "decode" or args.config != "all" else min(args.cpu_budget, 10.0)
+        per_tok, desc, done, blas = oracle_sample_time(inp, budget)
         line["cpu_baseline"] = {"value": 1.0 / per_tok, "unit": "tokens/s", "cores": blas, "kind": "oracle",
                                 "sample": desc, "cores_available": len(os.sched_getaffinity(0))}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    del inp, flush, ws
+    torch.cuda.empty_cache()
+    return line
+
+
+def ours_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    import bit_quantized_moe_route_b200 as moe
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    moe.load_library()
+    moe.set_ffn_path({"auto": moe.FFN_AUTO, "gemv": moe.FFN_GEMV, "tc": moe.FFN_TENSOR_CORE}[args.ffn_path])
+    names = CONFIG_ORDER if args.config == "all" else [args.config]
+    for name in names:
+        line = run_config(name, args, dev, world, rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
 

@@ -24,6 +24,7 @@ from ._lib import (  # noqa: F401
     permute,
     qmat,
     read_device_error,
+    read_noalloc_error,
     route,
     set_ffn_path,
     set_timing_events,

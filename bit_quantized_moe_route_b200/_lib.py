@@ -59,6 +59,7 @@ _SIGS = {
                                         ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP,
                                         _VP, ctypes.c_size_t, _VP]),
     "moe_read_device_error": (ctypes.c_int, [_VP, ctypes.POINTER(ctypes.c_int32), _VP]),
+    "moe_read_noalloc_error": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int32), _VP]),
     "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "moe_last_error_detail": (ctypes.c_char_p, []),
     "moe_set_timing_events": (ctypes.c_int, [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]),
@@ -206,12 +207,20 @@ def read_device_error(ws, stream=None) -> int:
     return code.value
 
 
+def read_noalloc_error(stream=None) -> int:
+    """Device error word of expert_ffn_noalloc's static scratch (read and cleared)."""
+    code = ctypes.c_int32(0)
+    _check(load_library().moe_read_noalloc_error(ctypes.byref(code), _stream(stream)), "moe_read_noalloc_error")
+    return code.value
+
+
 FFN_AUTO, FFN_GEMV, FFN_TENSOR_CORE = 0, 1, 2
 
 
 def set_ffn_path(path: int) -> int:
     """Select the expert-FFN implementation (FFN_AUTO / FFN_GEMV /
-    FFN_TENSOR_CORE) for this process; returns the previous setting."""
+    FFN_TENSOR_CORE) for the calling thread's calls; returns its previous
+    setting."""
     prev = load_library().moe_set_ffn_path(int(path))
     if prev < 0:
         raise ValueError(f"unknown FFN path {path}")

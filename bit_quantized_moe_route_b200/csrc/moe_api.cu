@@ -447,7 +447,9 @@ const TcLaunchFn kTcLaunch[2][5] = {
 const TcAttrFn kTcAttrs[10] = {attrs_tc_s1_A2, attrs_tc_s1_A3, attrs_tc_s1_A4, attrs_tc_s1_A8, attrs_tc_s1_MX4,
                                attrs_tc_s2_A2, attrs_tc_s2_A3, attrs_tc_s2_A4, attrs_tc_s2_A8, attrs_tc_s2_MX4};
 
-std::atomic<int> g_ffn_path{MOE_FFN_AUTO};
+// Expert-FFN implementation choice of the calling thread (moe_set_ffn_path):
+// one thread's setting never changes another thread's calls.
+thread_local int g_ffn_path = MOE_FFN_AUTO;
 
 // The tensor-core kernel tiles 128 output rows x 64 inputs.
 bool tc_shape_ok(const QMatDev& A) { return A.n_out % kTcM == 0 && A.n_in % kTcK == 0; }
@@ -458,7 +460,7 @@ bool tc_shape_ok(const QMatDev& A) { return A.n_out % kTcM == 0 && A.n_in % kTcK
 // keeps pace with HBM) or when forced, if the workspace has its regions and
 // every matrix has a supported shape.
 bool use_tc(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w2, const QMatDev* sh, const WsLayout& L) {
-  const int mode = g_ffn_path.load(std::memory_order_relaxed);
+  const int mode = g_ffn_path;
   if (mode == MOE_FFN_GEMV || !L.tc) return false;
   if (!tc_shape_ok(w1) || !tc_shape_ok(w2) || (sh && (!tc_shape_ok(sh[0]) || !tc_shape_ok(sh[2])))) return false;
   if (mode == MOE_FFN_TENSOR_CORE) return true;
@@ -534,7 +536,8 @@ moe_status_t um_weight_maps(UmParams& p, int m, const QMatDev& Q, int E, int row
 
 moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offsets, const int* sorted,
                            const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh,
-                           float* y, int ld_y, void* ws, const WsLayout& L, cudaStream_t s, const DevInfo& di) {
+                           float* y, int ld_y, void* ws, const WsLayout& L, cudaStream_t s, const DevInfo& di,
+                           const int* valid) {
   const int Tk = d.T * d.top_k;
   const int P = Tk + (sh ? d.T : 0);
   int* err = &ws_at<WsHeader>(ws, L.hdr)->err;
@@ -546,11 +549,11 @@ moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offset
     const size_t n8 = (size_t)P * d.d_model / 8;
     const int grid = (int)std::min<size_t>((n8 + 255) / 256, (size_t)di.sms * 8);
     tc_gather_f16_kernel<<<std::max(grid, 1), 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(x), sorted,
-                                                           d.top_k, Tk, d.T, d.d_model, sh ? 1 : 0, xs, err);
+                                                           d.top_k, Tk, d.T, d.d_model, sh ? 1 : 0, xs, err, valid);
     MOE_CHECK_LAUNCH("tc_gather_f16_kernel");
     hook_mark(s, "gather_f16");
     tc_plan_kernel<<<1, 1024, 0, s>>>(offsets, d.n_experts, kTcN, ws_at<int4>(ws, L.tiles), n_tiles, kUmN,
-                                      ws_at<int4>(ws, L.tiles2), n_tiles + 1);
+                                      ws_at<int4>(ws, L.tiles2), n_tiles + 1, valid);
     MOE_CHECK_LAUNCH("tc_plan_kernel");
     hook_mark(s, "tile_plan");
   }
@@ -628,13 +631,17 @@ moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offset
 }
 
 // Stage 1 + stage 2 of the expert FFN (routed pairs, optional shared expert).
+// `valid`: the flag the permutation check wrote for a caller-supplied
+// permutation (NULL for the library's own).
 moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, const int* sorted,
                         const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh,
-                        float* y, int ld_y, void* ws, const WsLayout& L, cudaStream_t s) {
+                        float* y, int ld_y, void* ws, const WsLayout& L, cudaStream_t s,
+                        const int* valid = nullptr) {
   DevInfo* di = nullptr;
   moe_status_t st = dev_info(&di);
   if (st != MOE_OK) return st;
-  if (use_tc(d, w1, w2, sh, L)) return launch_ffn_tc(d, x, offsets, sorted, w1, w3, w2, sh, y, ld_y, ws, L, s, *di);
+  if (use_tc(d, w1, w2, sh, L))
+    return launch_ffn_tc(d, x, offsets, sorted, w1, w3, w2, sh, y, ld_y, ws, L, s, *di, valid);
   const int Tk = d.T * d.top_k;
   const int max_active = std::min(d.n_experts, Tk);
   float* h = ws_at<float>(ws, L.h);
@@ -825,7 +832,9 @@ const char* moe_last_error_detail(void) { return g_detail; }
 
 int32_t moe_set_ffn_path(int32_t path) {
   if (path != MOE_FFN_AUTO && path != MOE_FFN_GEMV && path != MOE_FFN_TENSOR_CORE) return -1;
-  return g_ffn_path.exchange(path);
+  const int prev = g_ffn_path;
+  g_ffn_path = path;
+  return prev;
 }
 
 moe_status_t moe_set_timing_events(void* const* events, int32_t n_events) {
@@ -903,11 +912,14 @@ moe_status_t moe_expert_ffn(const moe_dims_t* dims, const void* x, const int32_t
   DevInfo* di;
   if ((st = dev_info(&di)) != MOE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  active_from_offsets_kernel<<<1, kPermThreads, 0, s>>>(expert_offsets, d.n_experts, ws_at<int>(ws, L.active));
+  WsHeader* hdr = ws_at<WsHeader>(ws, L.hdr);
+  active_from_offsets_kernel<<<1, kPermThreads, 0, s>>>(expert_offsets, d.n_experts, d.T * d.top_k, sorted_rows,
+                                                        ws_at<int>(ws, L.active), &hdr->err, &hdr->counters[2]);
   MOE_CHECK_LAUNCH("active_from_offsets_kernel");
   moe_dims_t dn = d;
   dn.d_ff_shared = 0;
-  return launch_ffn(dn, x, expert_offsets, sorted_rows, q1, q3, q2, nullptr, y, d.d_model, ws, L, s);
+  return launch_ffn(dn, x, expert_offsets, sorted_rows, q1, q3, q2, nullptr, y, d.d_model, ws, L, s,
+                    &hdr->counters[2]);
 }
 
 moe_status_t moe_combine(const moe_dims_t* dims, const float* y, const int32_t* inv, const float* topk_w,
@@ -1076,6 +1088,12 @@ moe_status_t static_scratch_addr(void** out) {
       cudaGetLastError();
       return cuda_fail(e, "cudaGetSymbolAddress(static scratch)");
     }
+    // the error word starts at zero once; afterwards only the reader clears it
+    e = cudaMemset(p, 0, sizeof(WsHeader));
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return cuda_fail(e, "clear static scratch header");
+    }
     g_static_addr[dev] = p;
   }
   *out = g_static_addr[dev];
@@ -1119,13 +1137,31 @@ extern "C" moe_status_t moe_expert_ffn_noalloc(const moe_dims_t* dims, const voi
   void* scratch = nullptr;
   if ((st = static_scratch_addr(&scratch)) != MOE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the error word starts at zero on every call; the active list and h are
-  // fully rewritten before they are read
-  cudaError_t e = cudaMemsetAsync(scratch, 0, sizeof(WsHeader), s);
-  if (e != cudaSuccess) return cuda_fail(e, "clear static scratch header");
-  active_from_offsets_kernel<<<1, kPermThreads, 0, s>>>(expert_offsets, d.n_experts, ws_at<int>(scratch, Ls.active));
+  // the active list and h are fully rewritten before they are read; the
+  // error word keeps the first device error since the last
+  // moe_read_noalloc_error on this device
+  WsHeader* hdr = ws_at<WsHeader>(scratch, Ls.hdr);
+  active_from_offsets_kernel<<<1, kPermThreads, 0, s>>>(expert_offsets, d.n_experts, d.T * d.top_k, sorted_rows,
+                                                        ws_at<int>(scratch, Ls.active), &hdr->err, nullptr);
   MOE_CHECK_LAUNCH("active_from_offsets_kernel");
   moe_dims_t dn = d;
   dn.d_ff_shared = 0;
   return launch_ffn(dn, x, expert_offsets, sorted_rows, q1, q3, q2, nullptr, y, d.d_model, scratch, Ls, s);
+}
+
+extern "C" moe_status_t moe_read_noalloc_error(int32_t* code_out, void* stream) {
+  g_detail[0] = 0;
+  if (!code_out) return fail(MOE_ERR_INVALID_ARG, "code_out is NULL");
+  void* scratch = nullptr;
+  moe_status_t st = static_scratch_addr(&scratch);
+  if (st != MOE_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int v = 0;
+  e = cudaMemcpy(&v, scratch, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  e = cudaMemset(scratch, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  *code_out = v;
+  return MOE_OK;
 }

@@ -271,9 +271,34 @@ permute_scatter_kernel(const int* __restrict__ ids, int N, int E, const int* __r
 
 // Active-expert list from caller-provided offsets (single CTA).
 __global__ void __launch_bounds__(kPermThreads)
-active_from_offsets_kernel(const int* __restrict__ offsets, int E, int* __restrict__ active) {
+active_from_offsets_kernel(const int* __restrict__ offsets, int E, int Tk, const int* __restrict__ sorted_rows,
+                           int* __restrict__ active, int* __restrict__ err, int* __restrict__ valid) {
+  // A caller-supplied permutation is checked before any expert FFN kernel
+  // reads through it: offsets[0] = 0, offsets[E] = Tk, non-decreasing, and
+  // every sorted row a flat pair index in [0, Tk).  A violation records
+  // MOE_ERR_DEVICE_INPUT and leaves no active expert (and *valid = 0), so
+  // nothing downstream touches memory through the bad lists.
   __shared__ int warp_tot[32];
   __shared__ int total;
+  __shared__ int bad;
+  if (threadIdx.x == 0) bad = (offsets[0] != 0 || offsets[E] != Tk) ? 1 : 0;
+  __syncthreads();
+  int mine = 0;
+  for (int e = threadIdx.x; e < E; e += kPermThreads) {
+    const int o0 = offsets[e], o1 = offsets[e + 1];
+    mine |= (o0 < 0 || o1 < o0 || o1 > Tk) ? 1 : 0;
+  }
+  for (int p = threadIdx.x; p < Tk; p += kPermThreads) mine |= ((unsigned)sorted_rows[p] >= (unsigned)Tk) ? 1 : 0;
+  if (mine) bad = 1;
+  __syncthreads();
+  if (bad) {
+    if (threadIdx.x == 0) {
+      active[0] = 0;
+      if (valid) *valid = 0;
+      set_error(err, kErrDeviceInput);
+    }
+    return;
+  }
   int acarry = 0;
   for (int e0 = 0; e0 < E; e0 += kPermThreads) {
     const int e = e0 + threadIdx.x;
@@ -283,7 +308,10 @@ active_from_offsets_kernel(const int* __restrict__ offsets, int E, int* __restri
     acarry += total;
     __syncthreads();
   }
-  if (threadIdx.x == 0) active[0] = acarry;
+  if (threadIdx.x == 0) {
+    active[0] = acarry;
+    if (valid) *valid = 1;
+  }
 }
 
 }  // namespace moe

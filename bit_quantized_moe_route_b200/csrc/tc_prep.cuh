@@ -16,7 +16,8 @@ namespace moe {
 // flagged (fp16 overflow) and stored as inf.
 __global__ void tc_gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const int* __restrict__ sorted_rows,
                                      int k, int Tk, int T, int d, int shared, __half* __restrict__ xs,
-                                     int* __restrict__ err) {
+                                     int* __restrict__ err, const int* __restrict__ valid) {
+  if (valid && !*valid) return;  // a caller permutation that failed its check: no expert runs
   const int c8 = d / 8;
   const size_t rows = (size_t)Tk + (shared ? T : 0);
   const size_t n8 = rows * c8;
@@ -43,14 +44,16 @@ __global__ void tc_gather_f16_kernel(const __nv_bfloat16* __restrict__ x, const 
 // Token tiles from the per-expert position ranges, for two tile sizes at
 // once: expert e with n_e sorted positions gets ceil(n_e / size) tiles
 // {e, first position, tokens, 0}, in expert order.  One block of 1024
-// threads; E <= 1024.
+// threads; E <= 1024.  With `valid` given and zero (a caller permutation
+// that failed its check) the plans are empty.
 __global__ void tc_plan_kernel(const int* __restrict__ offsets, int E, int size_a, int4* __restrict__ tiles_a,
                                int* __restrict__ n_a, int size_b, int4* __restrict__ tiles_b,
-                               int* __restrict__ n_b) {
+                               int* __restrict__ n_b, const int* __restrict__ valid) {
   __shared__ int warp_tot[2][32];
   const int e = threadIdx.x, lane = e & 31, warp = e >> 5;
-  const int beg = e < E ? offsets[e] : 0;
-  const int n = e < E ? offsets[e + 1] - beg : 0;
+  const bool ok = !valid || *valid;
+  const int beg = e < E && ok ? offsets[e] : 0;
+  const int n = e < E && ok ? offsets[e + 1] - beg : 0;
   const int c[2] = {(n + size_a - 1) / size_a, (n + size_b - 1) / size_b};
   int incl[2] = {c[0], c[1]};  // inclusive scans of the tile counts across the block
 #pragma unroll

@@ -177,6 +177,12 @@ moe_status_t moe_permute(const moe_dims_t* dims, const int32_t* topk_ids, int32_
  *   y[p] = W2[e] . (silu(W1[e] . x[t]) * (W3[e] . x[t])),  silu(a) = a/(1+e^-a)
  * with fp32 accumulation.  w1 and w3 must share one format.
  *   x : bf16 [T, d_model];  w1, w3 : [E, d_ff, d_model];  w2 : [E, d_model, d_ff]
+ *   expert_offsets : int32 [n_experts+1], sorted_rows : int32 [T*k] as
+ *            moe_permute writes them.  They are checked on the device before
+ *            use: offsets[0] = 0, offsets[n_experts] = T*k, non-decreasing,
+ *            every sorted row in [0, T*k).  A violation records
+ *            MOE_ERR_DEVICE_INPUT in the error word and no expert runs (y is
+ *            left unwritten); nothing is read or written out of bounds.
  *   y : fp32 [T*k, d_model] (out) in sorted order.
  * Two implementations (moe_set_ffn_path): a weight-streaming GEMV that
  * dequantises in registers and keeps x and h in fp32, for small batches; and
@@ -208,11 +214,23 @@ moe_status_t moe_expert_ffn(const moe_dims_t* dims, const void* x, const int32_t
  * on a device shares the same array and leaves its contents behind: calls
  * that overlap on the GPU (different streams without ordering, or several
  * host threads) race and corrupt each other's results.  The library itself
- * allocates nothing on this path.
+ * allocates nothing on this path.  Device-side errors (a permutation that
+ * fails its check, a bounded wait that gave up) are kept in the array's
+ * error word, the first one since the last read; moe_read_noalloc_error
+ * reports and clears it.
  */
 moe_status_t moe_expert_ffn_noalloc(const moe_dims_t* dims, const void* x, const int32_t* expert_offsets,
                                     const int32_t* sorted_rows, const moe_qmat_t* w1, const moe_qmat_t* w3,
                                     const moe_qmat_t* w2, float* y, void* stream);
+
+/*
+ * The device error word of moe_expert_ffn_noalloc's static scratch on the
+ * current device (the counterpart of moe_read_device_error for that entry
+ * point; no counterpart on the pages).  Synchronises `stream`, stores
+ * MOE_OK, MOE_ERR_DEVICE_INPUT or MOE_ERR_TIMEOUT in *code_out and clears
+ * the word.  Allocates nothing.
+ */
+moe_status_t moe_read_noalloc_error(int32_t* code_out, void* stream);
 
 /*
  * Step 4 -- weighted combine:
@@ -275,9 +293,10 @@ int32_t moe_timing_count(void);
 const char* moe_timing_label(int32_t i);
 
 /*
- * Expert-FFN implementation used by moe_expert_ffn / moe_forward /
- * moe_forward_host (process-wide setting; not for the allocation-free entry
- * point, which always streams).  AUTO (default) takes the tensor-core path
+ * Expert-FFN implementation used by the calling thread's moe_expert_ffn /
+ * moe_forward / moe_forward_host calls (a per-thread setting: other
+ * threads' calls are not affected; not for the allocation-free entry point,
+ * which always streams).  AUTO (default) takes the tensor-core path
  * from T >= 4 tokens when the shapes allow it (d_ff, d_model multiples of
  * 128), and the weight-streaming GEMV below that.
  * Returns the previous setting, or -1 (setting unchanged) for an unknown

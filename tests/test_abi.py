@@ -111,3 +111,21 @@ def test_plain_c_caller(lib, tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stderr
     assert r.stdout.startswith("ok ")
+
+
+def test_ffn_path_setting_is_per_thread(lib):
+    """moe_set_ffn_path changes only the calling thread's setting."""
+    import threading
+    from bit_quantized_moe_route_b200 import _lib
+    main_prev = _lib.set_ffn_path(_lib.FFN_TENSOR_CORE)
+    seen = {}
+
+    def other():
+        seen["initial"] = _lib.set_ffn_path(_lib.FFN_GEMV)   # returns this thread's previous value
+        seen["after"] = _lib.set_ffn_path(_lib.FFN_GEMV)
+
+    th = threading.Thread(target=other)
+    th.start()
+    th.join()
+    assert seen == {"initial": _lib.FFN_AUTO, "after": _lib.FFN_GEMV}
+    assert _lib.set_ffn_path(main_prev) == _lib.FFN_TENSOR_CORE    # the other thread did not change it

@@ -113,10 +113,10 @@ def test_roofline_prefill_is_tensor_bound():
     flops = 2.0 * 4096 * 8 * 2 * 4096 * 2048
     r = bench.roofline_entry("ffn_w13_swiglu", 1.40, {"ffn_w13_swiglu": 3.0e9}, {"ffn_w13_swiglu": flops}, True,
                              PEAK, None)
-    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == 1376.7
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["peak"] == 1624.7
     assert r["achieved"] == pytest.approx(flops / 1.40e-3 / 1e12)
-    assert r["frac"] == pytest.approx(r["achieved"] / 1376.7)
-    assert r["frac_of_burst_peak"] == pytest.approx(r["achieved"] / 1624.7)
+    assert r["frac"] == pytest.approx(r["achieved"] / 1624.7)
+    assert r["frac_of_sustained_peak"] == pytest.approx(r["achieved"] / 1376.7)
     assert r["frac_of_nominal"] == pytest.approx(r["achieved"] / 2250.0)
 
 
@@ -126,7 +126,7 @@ def test_roofline_small_batch_tensor_path_stays_hbm_bound():
     r = bench.roofline_entry("ffn_w13_swiglu", 0.758, {"ffn_w13_swiglu": 1.49e9}, {"ffn_w13_swiglu": flops}, True,
                              PEAK, None)
     assert r["bound"] == "hbm"
-    assert r["tensor_frac"] == pytest.approx(flops / 0.758e-3 / 1e12 / 1376.7)
+    assert r["tensor_frac"] == pytest.approx(flops / 0.758e-3 / 1e12 / 1624.7)
     assert r["tensor_frac"] < r["frac"]
 
 
@@ -146,3 +146,55 @@ def test_every_workload_accounts_and_describes(name):
     assert ("route_hash" in work) == (c["routing"] == "hash")
     desc = bench.workload_desc(c)
     assert desc["workload"] == name and desc["T"] == c["T"] and desc["n_experts"] == c["E"]
+
+
+def test_decode_layer_bytes_count_only_kernels_that_ran():
+    """Decode on the GEMV path: the four launches read the routed experts,
+    the shared expert once, the fp32 router, x, h and y -- about 144.2 MB
+    with 8 distinct experts -- and nothing of the tensor-core path."""
+    d, f, k, E = 4096, 2048, 8, 256
+    inp = layer(1, d, E, k, f, ("affine", 4, 64), ("affine", 4, 64), shared=("affine", 8, 64), f_shared=2048)
+    ids = np.array([[3, 17, 40, 41, 99, 120, 200, 255]])
+    work, flops, n_act, weight_bytes, kflops = bench.kernel_work(inp, ids)
+    labels = ["route_topk_permute", "ffn_w13_swiglu", "ffn_w2", "combine"]
+    total = bench.layer_bytes(work, labels)
+    assert weight_bytes == 8 * 14_155_776 + 26_738_688
+    P = k + 1
+    acts = (E * d * 4 + d * 2 + E * 4 + k * 8 + k * 12 + (E + 1) * 4     # routing + permutation
+            + d * 2 + P * f * 4                                          # x in, h out
+            + P * f * 4 + P * d * 4                                      # h in, y out
+            + P * d * 4 + d * 2 + k * 8)                                 # combine
+    assert total == weight_bytes + acts
+    assert abs(total / 1e6 - 144.2) < 0.5
+    assert "ffn_w13_swiglu_shared" not in work and "gather_f16" not in work
+
+
+def test_tensor_core_path_counts_the_shared_expert_once():
+    d, f, k, E, T = 1024, 512, 4, 16, 64
+    inp = layer(T, d, E, k, f, ("affine", 4, 64), ("affine", 4, 64), shared=("affine", 8, 64), f_shared=512)
+    ids = (np.arange(T * k) % E).reshape(T, k)
+    work, flops, n_act, weight_bytes, kflops = bench.kernel_work(inp, ids, tensor_path=True)
+    sh = sum(m.packed_bytes_per_expert() for m in inp.shared)
+    routed = E * (inp.w1.packed_bytes_per_expert() * 2 + inp.w2.packed_bytes_per_expert())
+    labels = ["router_logits", "topk", "permute", "gather_f16", "tile_plan", "ffn_w13_swiglu",
+              "ffn_w13_swiglu_shared", "ffn_w2", "ffn_w2_shared", "combine"]
+    weights_counted = (work["ffn_w13_swiglu"] - T * k * d * 2 - T * k * f * 2) + \
+        (work["ffn_w2"] - T * k * f * 2 - T * k * d * 4) + \
+        (work["ffn_w13_swiglu_shared"] - T * d * 2 - T * 512 * 2) + (work["ffn_w2_shared"] - T * 512 * 2 - T * d * 4)
+    assert weights_counted == routed + sh == weight_bytes
+    assert bench.layer_bytes(work, labels) > weight_bytes
+
+
+def test_step_stats_median_is_the_reported_step():
+    st = bench.step_stats([0.1, 0.5, 0.11, 0.12, 0.1])
+    assert st["median"] == 0.11 and st["min"] == 0.1 and st["p90"] == 0.5
+    assert st["mean"] == pytest.approx(0.186)
+
+
+def test_roofline_tensor_bound_uses_the_burst_peak():
+    flops = 2.0 * 4096 * 8 * 2 * 4096 * 2048
+    r = bench.roofline_entry("ffn_w13_swiglu", 1.444, {"ffn_w13_swiglu": 3.0e9}, {"ffn_w13_swiglu": flops}, True,
+                             PEAK, None)
+    assert r["peak"] == 1624.7
+    assert r["frac"] == pytest.approx(flops / 1.444e-3 / 1e12 / 1624.7)
+    assert r["frac"] < 0.5 < r["frac_of_sustained_peak"]

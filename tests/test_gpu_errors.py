@@ -106,3 +106,44 @@ def test_misaligned_and_unsupported(cuda_device):
                          inp.router_b.data_ptr(), None, ctypes.byref(q1), ctypes.byref(qm), ctypes.byref(q2), None,
                          out.data_ptr(), None, None, ws.data_ptr(), ws.numel(), None)
     assert st == 2 and b"share" in lib.moe_last_error_detail()
+
+
+BAD_PERMUTATIONS = {
+    "offsets_start_nonzero": lambda o, r: o.__setitem__(0, 1),
+    "offsets_decrease": lambda o, r: (o.__setitem__(3, int(o[5]) + 1)),
+    "offsets_end_past_pairs": lambda o, r: o.__setitem__(-1, int(o[-1]) + 64),
+    "row_past_pairs": lambda o, r: r.__setitem__(5, len(r) + 1000),
+    "row_negative": lambda o, r: r.__setitem__(0, -7),
+}
+
+
+@pytest.mark.parametrize("path", ["gemv", "tc"])
+@pytest.mark.parametrize("bad", list(BAD_PERMUTATIONS))
+def test_bad_permutation_in_expert_ffn(cuda_device, bad, path):
+    """A caller permutation that fails its device-side check records
+    MOE_ERR_DEVICE_INPUT, runs no expert (y keeps its contents) and touches
+    nothing out of bounds; a correct call afterwards is clean."""
+    inp = make_custom(dict(CONFIGS["tiny"], T=12, seed=303), cuda_device)
+    c = inp.cfg
+    res = oracle_run(inp)
+    dims = dims_for(inp)
+    ws = moe.alloc_workspace(dims, cuda_device)
+    n = c["T"] * c["k"]
+    offs = res["expert_offsets"].astype(np.int32).copy()
+    rows = res["sorted_rows"].astype(np.int32).copy()
+    BAD_PERMUTATIONS[bad](offs, rows)
+    prev = moe.set_ffn_path(moe.FFN_GEMV if path == "gemv" else moe.FFN_TENSOR_CORE)
+    try:
+        y = torch.full((n, c["d"]), 7.0, dtype=torch.float32, device=cuda_device)
+        moe.expert_ffn(dims, inp.x, torch.from_numpy(offs).to(cuda_device), torch.from_numpy(rows).to(cuda_device),
+                       inp.w1, inp.w3, inp.w2, y, ws)
+        assert moe.read_device_error(ws) == 6
+        assert torch.all(y == 7.0)
+        good_offs = torch.from_numpy(res["expert_offsets"].astype(np.int32)).to(cuda_device)
+        good_rows = torch.from_numpy(res["sorted_rows"].astype(np.int32)).to(cuda_device)
+        moe.expert_ffn(dims, inp.x, good_offs, good_rows, inp.w1, inp.w3, inp.w2, y, ws)
+        assert moe.read_device_error(ws) == 0
+    finally:
+        moe.set_ffn_path(prev)
+    y_ref = res["y_slots"].reshape(n, c["d"])[res["sorted_rows"]]
+    check_output(y.cpu().double().numpy(), y_ref, f"{bad}/{path} follow-up")

@@ -72,3 +72,27 @@ def test_noalloc_rejects_oversized_problem(cuda_device):
     with pytest.raises(moe.MoEError) as ei:
         moe.expert_ffn_noalloc(dims, inp.x, offs, rows, inp.w1, inp.w3, inp.w2, y)
     assert ei.value.status == 2 and "scratch" in str(ei.value)
+
+
+def test_noalloc_error_word_is_readable(cuda_device):
+    """The static scratch's error word: clean after a correct call, set by a
+    permutation that fails its check (no expert runs then), cleared by the
+    read."""
+    inp = make_custom(CASES["tiny"], cuda_device)
+    c = inp.cfg
+    res, offs, rows = _routing(inp, cuda_device)
+    dims = dims_for(inp)
+    n = c["T"] * c["k"]
+    y = torch.empty(n, c["d"], dtype=torch.float32, device=cuda_device)
+    moe.expert_ffn_noalloc(dims, inp.x, offs, rows, inp.w1, inp.w3, inp.w2, y)
+    assert moe.read_noalloc_error() == 0
+    bad_rows = rows.clone()
+    bad_rows[1] = n + 5
+    y_bad = torch.full((n, c["d"]), 3.0, dtype=torch.float32, device=cuda_device)
+    moe.expert_ffn_noalloc(dims, inp.x, offs, bad_rows, inp.w1, inp.w3, inp.w2, y_bad)
+    assert moe.read_noalloc_error() == 6
+    assert torch.all(y_bad == 3.0)
+    assert moe.read_noalloc_error() == 0
+    moe.expert_ffn_noalloc(dims, inp.x, offs, rows, inp.w1, inp.w3, inp.w2, y_bad)
+    assert moe.read_noalloc_error() == 0
+    assert torch.equal(y_bad, y)
