@@ -35,6 +35,14 @@ and section:
 [CARD-MLX4-SRC]  model card "DeepSeek-V4-Flash-MLX-4bit", the note after
           "What this port implements": the source checkpoint stores most
           matmuls as FP8 e4m3 with e8m0 128x128 block scales.
+[PR1192-SK]  the same pull request's review note "Sinkhorn normalization":
+          the reference path is a softmax followed by a loop of sum-and-divide
+          steps (about forty launches per call), which a fused kernel does in
+          one register-resident pass.
+[CARD-4BIT-MHC]  model card "mlx-community / DeepSeek-V4-Flash-4bit",
+          Architecture ("mHC": hc_mult = 4 parallel copies of the hidden
+          state recombined through a doubly-stochastic, Sinkhorn-normalised
+          mixing matrix) and Performance (the fused Sinkhorn kernel).
 [CARD-MIXED]  model card "DeepSeek-V4-Flash-0731-MLX-Serve-mixed-2-3-8bit",
           precision table (w1/w3 affine 2-bit g128, w2 affine 3-bit g128,
           shared experts 8-bit g64) and conversion notes (fp4 e2m1 with e8m0
@@ -63,7 +71,7 @@ __all__ = [
     "dequant_mxfp8", "block128_scales_to_group32",
     "dequant", "router_logits", "sqrtsoftplus", "topk_select", "renormalize",
     "route_learned", "route_hash", "route_forced", "permute", "silu", "swiglu_ffn", "combine",
-    "round_bf16", "forward", "parity_stats",
+    "round_bf16", "forward", "parity_stats", "hc_sinkhorn", "hc_mix",
 ]
 
 # --------------------------------------------------------------------------
@@ -383,3 +391,30 @@ def parity_stats(out: np.ndarray, ref: np.ndarray) -> Dict[str, float]:
         "max_err_over_rms": float(err.max() / rms) if err.size and rms > 0 else 0.0,
         "mean_rel_err": float(err.sum() / np.abs(ref).sum()) if err.size and np.abs(ref).sum() > 0 else 0.0,
     }
+
+
+# --------------------------------------------------------------------------
+# mHC residual mixing  [PR1192-SK; CARD-4BIT-MHC]
+# --------------------------------------------------------------------------
+# Readings where the pages are silent: the mixing logits are per token,
+# [T, n, n] with n = hc_mult; the softmax runs along each row (the last
+# axis); one iteration is a column normalisation followed by a row
+# normalisation (so rows sum to one on exit); eps is added to every divisor
+# (0 by default); the n -> n mix is out[t, i] = sum_j P[t, i, j] * h[t, j].
+def hc_sinkhorn(logits, iters: int, eps: float = 0.0) -> np.ndarray:
+    """Sinkhorn-normalised mixing matrices P [T, n, n] in fp64: a row-wise
+    softmax of the logits, then `iters` rounds of dividing every column by
+    its sum and then every row by its sum."""
+    L = np.asarray(logits, np.float64)
+    P = np.exp(L - L.max(axis=-1, keepdims=True))
+    P = P / P.sum(axis=-1, keepdims=True)
+    for _ in range(iters):
+        P = P / (P.sum(axis=-2, keepdims=True) + eps)
+        P = P / (P.sum(axis=-1, keepdims=True) + eps)
+    return P
+
+
+def hc_mix(P, h) -> np.ndarray:
+    """out[t, i, :] = sum_j P[t, i, j] * h[t, j, :] for the n parallel copies
+    h [T, n, d] of the residual stream."""
+    return np.einsum("tij,tjd->tid", np.asarray(P, np.float64), np.asarray(h, np.float64))

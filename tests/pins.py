@@ -454,8 +454,80 @@ def pin_forced_routing():
     assert np.allclose(res2["out"], res["out"], rtol=1e-13, atol=1e-15)
 
 
+# ---------------------------------------------------------------- mHC Sinkhorn mixing
+def pin_hc_sinkhorn_softmax():
+    """Zero iterations: the row-wise softmax (scipy); rows sum to one after
+    any number of iterations, columns approach one as they grow."""
+    from scipy.special import softmax
+    rng = np.random.default_rng(51)
+    L = rng.normal(scale=2.0, size=(6, 4, 4))
+    assert np.allclose(oracle.hc_sinkhorn(L, 0), softmax(L, axis=-1), rtol=1e-14, atol=1e-16)
+    errs = []
+    for it in (1, 3, 10, 40, 300):
+        P = oracle.hc_sinkhorn(L, it)
+        assert np.abs(P.sum(-1) - 1).max() < 1e-14
+        errs.append(np.abs(P.sum(-2) - 1).max())
+    assert errs[-1] < 1e-9 and errs == sorted(errs, reverse=True)
+
+
+def pin_hc_sinkhorn_limits():
+    """The Sinkhorn limit of a positive matrix A is the unique doubly
+    stochastic D1 A D2.  For 2x2 it has the closed form [[p, 1-p], [1-p, p]],
+    p = sqrt(ad) / (sqrt(ad) + sqrt(bc)); for 4x4 it is checked against an
+    independent solve of u_i sum_j A_ij v_j = 1 = v_j sum_i A_ij u_i
+    (scipy root finding on log u, log v).  The limit is invariant under
+    positive diagonal scalings, i.e. adding r_i + c_j to the logits."""
+    from scipy.optimize import root
+    rng = np.random.default_rng(52)
+    for _ in range(5):
+        L = rng.normal(size=(1, 2, 2))
+        A = np.exp(L[0])
+        a, b, c, d = A[0, 0], A[0, 1], A[1, 0], A[1, 1]
+        pp = math.sqrt(a * d) / (math.sqrt(a * d) + math.sqrt(b * c))
+        want = np.array([[pp, 1 - pp], [1 - pp, pp]])
+        assert np.abs(oracle.hc_sinkhorn(L, 200)[0] - want).max() < 1e-12
+    for _ in range(3):
+        L = rng.normal(size=(1, 4, 4))
+        A = np.exp(L[0])
+
+        def eqs(z):
+            u, v = np.exp(z[:4]), np.exp(z[4:])
+            return np.concatenate([u * (A @ v) - 1, v * (A.T @ u) - 1])
+
+        sol = root(eqs, np.zeros(8), tol=1e-14)
+        u, v = np.exp(sol.x[:4]), np.exp(sol.x[4:])
+        want = u[:, None] * A * v[None, :]
+        assert np.abs(oracle.hc_sinkhorn(L, 500)[0] - want).max() < 1e-10
+        shifted = L + rng.normal(size=(1, 4, 1)) + rng.normal(size=(1, 1, 4))
+        assert np.abs(oracle.hc_sinkhorn(shifted, 500)[0] - want).max() < 1e-10
+
+
+def pin_hc_sinkhorn_fixed_point():
+    """A doubly stochastic matrix (a mixture of permutation matrices) given
+    as logits log(P) comes back unchanged after any number of iterations."""
+    rng = np.random.default_rng(53)
+    perms = [np.eye(4)[rng.permutation(4)] for _ in range(5)]
+    wts = rng.dirichlet(np.ones(5))
+    P0 = sum(w * m for w, m in zip(wts, perms)) * 0.9 + 0.1 / 4   # strictly positive, doubly stochastic
+    for it in (0, 1, 20):
+        assert np.abs(oracle.hc_sinkhorn(np.log(P0)[None], it)[0] - P0).max() < 1e-14
+
+
+def pin_hc_mix():
+    """The n -> n mix against torch.bmm in fp64; a permutation matrix moves
+    the copies."""
+    rng = np.random.default_rng(54)
+    P = rng.random(size=(3, 4, 4))
+    h = rng.normal(size=(3, 4, 16))
+    want = torch.bmm(torch.from_numpy(P), torch.from_numpy(h)).numpy()
+    assert np.allclose(oracle.hc_mix(P, h), want, rtol=1e-14, atol=1e-14)
+    perm = np.eye(4)[[2, 0, 3, 1]][None]
+    assert np.array_equal(oracle.hc_mix(perm, h[:1])[0], h[0][[2, 0, 3, 1]])
+
+
 ALL_PINS = [pin_e2m1_table, pin_e8m0, pin_unpack_golden, pin_unpack_bigint, pin_affine_dequant,
             pin_mxfp4_dequant, pin_sqrtsoftplus, pin_topk_bruteforce, pin_route_learned,
             pin_route_hash, pin_permutation, pin_dense_equivalence, pin_single_expert_swiglu,
             pin_round_bf16, pin_e4m3_table, pin_mxfp8_dequant, pin_block128_scales, pin_parity_stats,
-            pin_forward_token_subset, pin_forced_routing]
+            pin_forward_token_subset, pin_forced_routing, pin_hc_sinkhorn_softmax, pin_hc_sinkhorn_limits,
+            pin_hc_sinkhorn_fixed_point, pin_hc_mix]

@@ -103,6 +103,39 @@ def _forced_biased_weights(x, w_router, forced_ids):
     return ids, np.take_along_axis(s, ids, axis=1), None
 
 
+def _sk_rows_first(logits, iters, eps=0.0):
+    L = np.asarray(logits, np.float64)
+    P = np.exp(L - L.max(-1, keepdims=True))
+    P = P / P.sum(-1, keepdims=True)
+    for _ in range(iters):
+        P = P / (P.sum(-1, keepdims=True) + eps)
+        P = P / (P.sum(-2, keepdims=True) + eps)
+    return P
+
+
+def _sk_column_softmax(logits, iters, eps=0.0):
+    L = np.asarray(logits, np.float64)
+    P = np.exp(L - L.max(-2, keepdims=True))
+    P = P / P.sum(-2, keepdims=True)
+    for _ in range(iters):
+        P = P / (P.sum(-2, keepdims=True) + eps)
+        P = P / (P.sum(-1, keepdims=True) + eps)
+    return P
+
+
+def _sk_no_exp(logits, iters, eps=0.0):
+    P = np.abs(np.asarray(logits, np.float64))
+    P = P / P.sum(-1, keepdims=True)
+    for _ in range(iters):
+        P = P / (P.sum(-2, keepdims=True) + eps)
+        P = P / (P.sum(-1, keepdims=True) + eps)
+    return P
+
+
+def _mix_transposed(P, h):
+    return np.einsum("tji,tjd->tid", np.asarray(P, np.float64), np.asarray(h, np.float64))
+
+
 _ORIG_STATS = om.parity_stats
 
 
@@ -123,6 +156,10 @@ MUTATIONS = [
     ("parity_stats", _stats_mean_err, [pins.pin_parity_stats]),
     ("parity_stats", _stats_elementwise_rel, [pins.pin_parity_stats]),
     ("route_forced", _forced_biased_weights, [pins.pin_forced_routing]),
+    ("hc_sinkhorn", _sk_rows_first, [pins.pin_hc_sinkhorn_softmax]),
+    ("hc_sinkhorn", _sk_column_softmax, [pins.pin_hc_sinkhorn_softmax]),
+    ("hc_sinkhorn", _sk_no_exp, [pins.pin_hc_sinkhorn_limits]),
+    ("hc_mix", _mix_transposed, [pins.pin_hc_mix]),
 ]
 
 
