@@ -262,10 +262,10 @@ def oracle_sample_time(inp, budget_s: float, max_pairs=None, start_pair: int = 0
     x = inp.x.float().cpu().numpy()
     t0 = time.perf_counter()
     if c["routing"] == "hash":
-        ids, w = oracle.route_hash(x, inp.router_w.cpu().numpy(), inp.token_ids.cpu().numpy(),
+        ids, w = oracle.route_hash(x, inp.router_w.float().cpu().numpy(), inp.token_ids.cpu().numpy(),
                                    inp.tid2eid.cpu().numpy())
     else:
-        ids, w, _, _ = oracle.route_learned(x, inp.router_w.cpu().numpy(), inp.router_b.cpu().numpy(), k)
+        ids, w, _, _ = oracle.route_learned(x, inp.router_w.float().cpu().numpy(), inp.router_b.cpu().numpy(), k)
     oracle.permute(ids, c["E"])
     t_route = time.perf_counter() - t0
     ppt = k + (1 if inp.shared is not None else 0)
@@ -380,7 +380,7 @@ def run_config(name, args, dev, world, rank):
     T, d, k = c["T"], c["d"], c["k"]
     dims = moe.make_dims(T, d, c["f"], c["E"], k, c["routing"] == "hash",
                          c.get("vocab", 0) if c["routing"] == "hash" else 0,
-                         c.get("f_shared", 0) if inp.shared is not None else 0)
+                         c.get("f_shared", 0) if inp.shared is not None else 0, router_dtype=inp.router_w.dtype)
     ws = moe.alloc_workspace(dims, dev)
     out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
@@ -514,6 +514,101 @@ def run_config(name, args, dev, world, rank):
     return line
 
 
+def run_hc_config(name, args, dev, world, rank):
+    """Time the fused mHC Sinkhorn mixing kernel on its own (one launch per
+    step); HBM-bound: the n residual copies are read once and written once."""
+    import torch
+
+    import bit_quantized_moe_route_b200 as moe
+    from synthetic import HC_CONFIGS, make_hc_inputs
+
+    cfg = dict(HC_CONFIGS[name], name=name)
+    cfg.update(overrides(args))
+    inp = make_hc_inputs(cfg, dev)
+    T, n, d = cfg["T"], cfg["n"], cfg["d"]
+    out = torch.empty_like(inp.h)
+    flush = torch.ones(128 * 1024 * 1024, dtype=torch.int32, device=dev)
+    flush_sum = torch.empty((), dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.hc_sinkhorn_mix(inp.logits, inp.h, out, cfg["iters"], cfg["eps"])
+
+    for _ in range(max(3, args.warmup)):
+        torch.sum(flush, dtype=torch.int64, out=flush_sum)
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid) if getattr(props, "uuid", None) else str(dev.index))
+    sampler.start()
+    time.sleep(0.2)
+    for s in range(args.steps):
+        torch.sum(flush, dtype=torch.int64, out=flush_sum)
+        evs[s][0].record(stream)
+        step()
+        evs[s][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    st = step_stats([a.elapsed_time(b) for a, b in evs])
+    ms = max_over_ranks(st["median"], dev)
+    # e2e: host logits and copies in, mixed copies back
+    L_h = inp.logits.cpu().pin_memory()
+    h_h = inp.h.cpu().pin_memory()
+    o_h = torch.empty_like(h_h).pin_memory()
+    L_d, h_d = torch.empty_like(inp.logits), torch.empty_like(inp.h)
+    e2e = []
+    for s in range(max(10, min(args.steps, 50))):
+        torch.sum(flush, dtype=torch.int64, out=flush_sum)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        L_d.copy_(L_h, non_blocking=True)
+        h_d.copy_(h_h, non_blocking=True)
+        moe.hc_sinkhorn_mix(L_d, h_d, out, cfg["iters"], cfg["eps"])
+        o_h.copy_(out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e.append(a.elapsed_time(b))
+    e2e_ms = max_over_ranks(statistics.median(e2e), dev)
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    nbytes = T * n * d * 2 * 2 + T * n * n * 4
+    roof = {"bound": "hbm", "kernel": "hc_sinkhorn_mix", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm,
+            "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "traffic": None,
+            "peak_kind": f"{peak_kind} hbm_gbs (copy)", "algorithmic_bytes_per_launch": nbytes,
+            "frac_of_nominal": nbytes / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS}
+    line = {"metric": "mHC Sinkhorn-mixed tokens/s at 1 B200; achieved HBM GB/s vs peak",
+            "value": whole_job_rate(T, world, ms), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": name, "T": T, "hc_mult": n, "d": d, "iters": cfg["iters"], "eps": cfg["eps"],
+                       "l2": "flushed by reading a 512 MiB buffer between timed steps (outside the events)"},
+            "step_ms": st, "roofline": roof,
+            "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * n * d * 2 + T * n * n * 4, "d2h_bytes_per_step": T * n * d * 2,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps, "clocks": clocks}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import numpy as np
+        import oracle
+        sample = min(T, 256)
+        L = inp.logits[:sample].cpu().double().numpy()
+        h = inp.h[:sample].cpu().double().numpy()
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            oracle.hc_mix(oracle.hc_sinkhorn(L, cfg["iters"], cfg["eps"]), h)
+            reps += 1
+            if time.perf_counter() - t0 > min(args.cpu_budget, 10.0):
+                break
+        per_tok = (time.perf_counter() - t0) / (reps * sample)
+        line["cpu_baseline"] = {"value": 1.0 / per_tok, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{reps} x {sample} tokens of the same workload (numpy fp64)",
+                                "cores_available": len(os.sched_getaffinity(0))}
+    del inp, flush
+    torch.cuda.empty_cache()
+    return line
+
+
 def ours_arm(args):
     import torch
     import torch.distributed as dist
@@ -532,7 +627,7 @@ def ours_arm(args):
     moe.set_ffn_path({"auto": moe.FFN_AUTO, "gemv": moe.FFN_GEMV, "tc": moe.FFN_TENSOR_CORE}[args.ffn_path])
     names = CONFIG_ORDER if args.config == "all" else [args.config]
     for name in names:
-        line = run_config(name, args, dev, world, rank)
+        line = (run_hc_config if name.startswith("mhc") else run_config)(name, args, dev, world, rank)
         if rank == 0:
             print(json.dumps(line), flush=True)
     if world > 1:

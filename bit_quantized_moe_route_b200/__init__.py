@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     expert_ffn_noalloc,
     forward,
     forward_host,
+    hc_sinkhorn_mix,
     load_library,
     make_dims,
     permute,

@@ -31,7 +31,7 @@ class MoEError(RuntimeError):
 class Dims(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32),
                 ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("hash_mode", ctypes.c_int32),
-                ("vocab", ctypes.c_int32), ("d_ff_shared", ctypes.c_int32)]
+                ("vocab", ctypes.c_int32), ("d_ff_shared", ctypes.c_int32), ("router_dtype", ctypes.c_int32)]
 
 
 class QMatC(ctypes.Structure):
@@ -66,6 +66,8 @@ _SIGS = {
     "moe_timing_count": (ctypes.c_int32, []),
     "moe_timing_label": (ctypes.c_char_p, [ctypes.c_int32]),
     "moe_set_ffn_path": (ctypes.c_int32, [ctypes.c_int32]),
+    "moe_hc_sinkhorn_mix": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_float, _VP, _VP, _VP, _VP, _VP]),
 }
 
 
@@ -109,8 +111,10 @@ def _stream(stream=None) -> int:
 
 
 def make_dims(T: int, d_model: int, d_ff: int, n_experts: int, top_k: int, hash_mode: bool = False,
-              vocab: int = 0, d_ff_shared: int = 0) -> Dims:
-    return Dims(T, d_model, d_ff, n_experts, top_k, int(bool(hash_mode)), vocab, d_ff_shared)
+              vocab: int = 0, d_ff_shared: int = 0, router_dtype=None) -> Dims:
+    """router_dtype: None/torch.float32 (fp32 router weights) or torch.bfloat16."""
+    rd = 1 if router_dtype in (torch.bfloat16, "bf16", 1) else 0
+    return Dims(T, d_model, d_ff, n_experts, top_k, int(bool(hash_mode)), vocab, d_ff_shared, rd)
 
 
 def qmat(m) -> QMatC:
@@ -205,6 +209,15 @@ def read_device_error(ws, stream=None) -> int:
     _check(load_library().moe_read_device_error(_ptr(ws), ctypes.byref(code), _stream(stream)),
            "moe_read_device_error")
     return code.value
+
+
+def hc_sinkhorn_mix(logits, h, out, iters: int, eps: float = 0.0, P_out=None, stream=None):
+    """moe_hc_sinkhorn_mix: logits fp32 [T, n, n], h/out bf16 [T, n, d]."""
+    T, n, d = h.shape
+    if tuple(logits.shape) != (T, n, n) or tuple(out.shape) != (T, n, d):
+        raise ValueError("shapes: logits [T, n, n], h and out [T, n, d]")
+    _check(load_library().moe_hc_sinkhorn_mix(T, n, d, int(iters), float(eps), _ptr(logits), _ptr(h), _ptr(P_out),
+                                              _ptr(out), _stream(stream)), "moe_hc_sinkhorn_mix")
 
 
 def read_noalloc_error(stream=None) -> int:

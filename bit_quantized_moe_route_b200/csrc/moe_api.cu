@@ -18,6 +18,7 @@
 #include "route.cuh"
 #include "tc_prep.cuh"
 #include "ffn_umma.cuh"
+#include "hc_mix.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -155,6 +156,8 @@ moe_status_t check_dims(const moe_dims_t* d) {
   if (d->d_ff_shared < 0 || (d->d_ff_shared > 0 && !width_ok(d->d_ff_shared)))
     return fail(MOE_ERR_UNSUPPORTED, "d_ff_shared=%d not supported", d->d_ff_shared);
   if (d->hash_mode && d->vocab < 1) return fail(MOE_ERR_INVALID_ARG, "hash mode needs vocab >= 1");
+  if (d->router_dtype != 0 && d->router_dtype != 1)
+    return fail(MOE_ERR_UNSUPPORTED, "router_dtype=%d not in {0 (fp32), 1 (bf16)}", d->router_dtype);
   return MOE_OK;
 }
 
@@ -216,6 +219,16 @@ extern const StreamAttrFn kStreamAttrs[10];
 extern const TcAttrFn kTcAttrs[10];
 extern const UmAttrFn kUmAttrs[10];
 
+template <typename WT>
+void route_attrs() {
+  cudaFuncSetAttribute(router_logits_small_kernel<8, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 8 * 8192 * 2);
+  cudaFuncSetAttribute(route_small_fused_kernel<1, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+  cudaFuncSetAttribute(route_small_fused_kernel<8, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+  cudaFuncSetAttribute(route_small_fused_kernel<32, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+  cudaFuncSetAttribute(route_hash_fused_kernel<8, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+  cudaFuncSetAttribute(route_hash_fused_kernel<32, WT>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+}
+
 struct DevInfo {
   int sms = 0;
   int ffn1_blocks = 0, ffn2_blocks = 0;
@@ -235,13 +248,8 @@ moe_status_t dev_info(DevInfo** out) {
       cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev);
       cudaFuncSetAttribute(permute_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 34 * 1024 * 4);
       cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024 * 4);
-      cudaFuncSetAttribute(router_logits_small_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           8 * 8192 * 2);
-      cudaFuncSetAttribute(route_small_fused_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(route_small_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(route_small_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(route_hash_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      cudaFuncSetAttribute(route_hash_fused_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      route_attrs<float>();
+      route_attrs<__nv_bfloat16>();
       for (StreamAttrFn f : kStreamAttrs) f();
       for (TcAttrFn f : kTcAttrs) f();
       for (UmAttrFn f : kUmAttrs) f();
@@ -270,7 +278,8 @@ moe_status_t dev_info(DevInfo** out) {
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // ---------------------------------------------------------------- launches
-moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, const float* rb,
+template <typename WT>
+moe_status_t launch_route_t(const moe_dims_t& d, const void* x, const WT* rw, const float* rb,
                           const int* tok, const int* table, int* ids, float* wts, void* ws,
                           const WsLayout& L, cudaStream_t s) {
   int* err = &ws_at<WsHeader>(ws, L.hdr)->err;
@@ -278,10 +287,10 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
   if (d.hash_mode) {
     const int blocks = ceil_div(d.T * 32, 256);
     if (d.top_k <= 8)
-      route_hash_kernel<8><<<blocks, 256, 0, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts, d.top_k,
+      route_hash_kernel<8, WT><<<blocks, 256, 0, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts, d.top_k,
                                                   d.vocab, ids, wts, err);
     else
-      route_hash_kernel<32><<<blocks, 256, 0, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts, d.top_k,
+      route_hash_kernel<32, WT><<<blocks, 256, 0, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts, d.top_k,
                                                    d.vocab, ids, wts, err);
     MOE_CHECK_LAUNCH("route_hash_kernel");
     hook_mark(s, "route_hash");
@@ -291,7 +300,7 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
   int split = 1;  // K halves of the logits GEMM (partials summed by the top-k)
   if (d.T <= 64) {
     dim3 grid(ceil_div(d.n_experts, kLogitWarps), ceil_div(d.T, 8));
-    router_logits_small_kernel<8><<<grid, kLogitWarps * 32, 8 * d.d_model * 2, s>>>(xb, rw, logits, d.T,
+    router_logits_small_kernel<8, WT><<<grid, kLogitWarps * 32, 8 * d.d_model * 2, s>>>(xb, rw, logits, d.T,
                                                                                       d.d_model, d.n_experts);
     MOE_CHECK_LAUNCH("router_logits_small_kernel");
     hook_mark(s, "router_logits");
@@ -299,7 +308,7 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
     // two K halves (more CTAs than SMs) when there is enough work
     split = d.T >= 256 && d.d_model % (2 * kLBK) == 0 ? 2 : 1;
     dim3 grid(ceil_div(d.n_experts, kLBN), ceil_div(d.T, kLBM), split);
-    router_logits_tiled_kernel<<<grid, 256, 0, s>>>(xb, rw, logits, d.T, d.d_model, d.n_experts);
+    router_logits_tiled_kernel<WT><<<grid, 256, 0, s>>>(xb, rw, logits, d.T, d.d_model, d.n_experts);
     MOE_CHECK_LAUNCH("router_logits_tiled_kernel");
     hook_mark(s, "router_logits");
   }
@@ -316,12 +325,20 @@ moe_status_t launch_route(const moe_dims_t& d, const void* x, const float* rw, c
   return MOE_OK;
 }
 
+moe_status_t launch_route(const moe_dims_t& d, const void* x, const void* rw, const float* rb, const int* tok,
+                          const int* table, int* ids, float* wts, void* ws, const WsLayout& L, cudaStream_t s) {
+  if (d.router_dtype == 1)
+    return launch_route_t(d, x, static_cast<const __nv_bfloat16*>(rw), rb, tok, table, ids, wts, ws, L, s);
+  return launch_route_t(d, x, static_cast<const float*>(rw), rb, tok, table, ids, wts, ws, L, s);
+}
+
 // Routing and permutation in one launch for small batches.
 bool fused_route_ok(const moe_dims_t& d) {
   return d.T <= kFusedMaxT && d.d_model <= 4096 && d.d_model % 64 == 0 && d.top_k <= 32;
 }
 
-moe_status_t launch_route_fused(const moe_dims_t& d, const void* x, const float* rw, const float* rb, const int* tok,
+template <typename WT>
+moe_status_t launch_route_fused_t(const moe_dims_t& d, const void* x, const WT* rw, const float* rb, const int* tok,
                                 const int* table, int* ids, float* wts, int* offsets, int* sorted, int* inv, void* ws,
                                 const WsLayout& L, cudaStream_t s) {
   WsHeader* hdr = ws_at<WsHeader>(ws, L.hdr);
@@ -332,11 +349,11 @@ moe_status_t launch_route_fused(const moe_dims_t& d, const void* x, const float*
   if (d.hash_mode) {
     const int blocks = d.T;  // one block (8 warps) per token
     if (d.top_k <= 8)
-      route_hash_fused_kernel<8><<<blocks, 256, perm_smem, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts,
+      route_hash_fused_kernel<8, WT><<<blocks, 256, perm_smem, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts,
                                                                d.top_k, d.vocab, ids, wts, offsets, sorted, inv,
                                                                active, &hdr->counters[1], &hdr->err);
     else
-      route_hash_fused_kernel<32><<<blocks, 256, perm_smem, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts,
+      route_hash_fused_kernel<32, WT><<<blocks, 256, perm_smem, s>>>(xb, rw, tok, table, d.T, d.d_model, d.n_experts,
                                                                 d.top_k, d.vocab, ids, wts, offsets, sorted, inv,
                                                                 active, &hdr->counters[1], &hdr->err);
     MOE_CHECK_LAUNCH("route_hash_fused_kernel");
@@ -347,20 +364,30 @@ moe_status_t launch_route_fused(const moe_dims_t& d, const void* x, const float*
   const size_t smem = std::max((size_t)kFusedTB * d.d_model * 2, perm_smem);
   const int blocks = ceil_div(d.n_experts, 2);
   if (d.n_experts <= 32)
-    route_small_fused_kernel<1><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
+    route_small_fused_kernel<1, WT><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
                                                           ids, wts, offsets, sorted, inv, active, &hdr->counters[0],
                                                           &hdr->err);
   else if (d.n_experts <= 256)
-    route_small_fused_kernel<8><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
+    route_small_fused_kernel<8, WT><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
                                                           ids, wts, offsets, sorted, inv, active, &hdr->counters[0],
                                                           &hdr->err);
   else
-    route_small_fused_kernel<32><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
+    route_small_fused_kernel<32, WT><<<blocks, 256, smem, s>>>(xb, rw, rb, d.T, d.d_model, d.n_experts, d.top_k, logits,
                                                            ids, wts, offsets, sorted, inv, active, &hdr->counters[0],
                                                            &hdr->err);
   MOE_CHECK_LAUNCH("route_small_fused_kernel");
   hook_mark(s, "route_topk_permute");
   return MOE_OK;
+}
+
+moe_status_t launch_route_fused(const moe_dims_t& d, const void* x, const void* rw, const float* rb, const int* tok,
+                                const int* table, int* ids, float* wts, int* offsets, int* sorted, int* inv, void* ws,
+                                const WsLayout& L, cudaStream_t s) {
+  if (d.router_dtype == 1)
+    return launch_route_fused_t(d, x, static_cast<const __nv_bfloat16*>(rw), rb, tok, table, ids, wts, offsets,
+                                sorted, inv, ws, L, s);
+  return launch_route_fused_t(d, x, static_cast<const float*>(rw), rb, tok, table, ids, wts, offsets, sorted, inv,
+                              ws, L, s);
 }
 
 moe_status_t launch_permute(const moe_dims_t& d, const int* ids, int* offsets, int* sorted, int* inv,
@@ -784,7 +811,7 @@ moe_status_t check_ws(const moe_dims_t& d, void* ws, size_t ws_bytes, WsLayout* 
   return check_dev_ptr(ws, "workspace");
 }
 
-moe_status_t check_route_args(const moe_dims_t& d, const void* x, const float* rw, const int* tok,
+moe_status_t check_route_args(const moe_dims_t& d, const void* x, const void* rw, const int* tok,
                               const int* table) {
   moe_status_t st = check_dev_ptr(x, "x");
   if (st != MOE_OK) return st;
@@ -800,7 +827,7 @@ moe_status_t check_route_args(const moe_dims_t& d, const void* x, const float* r
   return MOE_OK;
 }
 
-moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t* token_ids, const float* router_w,
+moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t* token_ids, const void* router_w,
                               const float* router_b, const int32_t* tid2eid, const QMatDev& q1, const QMatDev& q3,
                               const QMatDev& q2, const QMatDev* qs, void* out, int32_t* topk_ids_out,
                               float* topk_w_out, void* ws, const WsLayout& L, cudaStream_t s);
@@ -853,7 +880,7 @@ const char* moe_timing_label(int32_t i) {
   return g_hook_labels[i];
 }
 
-moe_status_t moe_route(const moe_dims_t* dims, const void* x, const float* router_w, const float* router_b,
+moe_status_t moe_route(const moe_dims_t* dims, const void* x, const void* router_w, const float* router_b,
                        const int32_t* token_ids, const int32_t* tid2eid, int32_t* topk_ids, float* topk_w,
                        void* ws, size_t ws_bytes, void* stream) {
   g_detail[0] = 0;
@@ -937,7 +964,7 @@ moe_status_t moe_combine(const moe_dims_t* dims, const float* y, const int32_t* 
   return launch_combine(*dims, y, inv, topk_w, y_shared, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* token_ids, const float* router_w,
+moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* token_ids, const void* router_w,
                          const float* router_b, const int32_t* tid2eid, const moe_qmat_t* w1,
                          const moe_qmat_t* w3, const moe_qmat_t* w2, const moe_qmat_t* shared, void* out,
                          int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
@@ -976,7 +1003,7 @@ moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* t
 }  // extern "C"
 
 namespace {
-moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t* token_ids, const float* router_w,
+moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t* token_ids, const void* router_w,
                               const float* router_b, const int32_t* tid2eid, const QMatDev& q1, const QMatDev& q3,
                               const QMatDev& q2, const QMatDev* qs, void* out, int32_t* topk_ids_out,
                               float* topk_w_out, void* ws, const WsLayout& L, cudaStream_t s) {
@@ -1007,7 +1034,7 @@ moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t*
 extern "C" {
 
 moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const int32_t* token_ids_host,
-                              const float* router_w, const float* router_b, const int32_t* tid2eid,
+                              const void* router_w, const float* router_b, const int32_t* tid2eid,
                               const moe_qmat_t* w1, const moe_qmat_t* w3, const moe_qmat_t* w2,
                               const moe_qmat_t* shared, void* out_host, void* ws, size_t ws_bytes, void* stream) {
   g_detail[0] = 0;
@@ -1163,5 +1190,39 @@ extern "C" moe_status_t moe_read_noalloc_error(int32_t* code_out, void* stream) 
   e = cudaMemset(scratch, 0, sizeof(int));
   if (e != cudaSuccess) return cuda_fail(e, "clear error word");
   *code_out = v;
+  return MOE_OK;
+}
+
+extern "C" moe_status_t moe_hc_sinkhorn_mix(int32_t T, int32_t n, int32_t d, int32_t iters, float eps,
+                                            const float* logits, const void* h, float* P_out, void* out,
+                                            void* stream) {
+  g_detail[0] = 0;
+  if (T < 1) return fail(MOE_ERR_INVALID_ARG, "T=%d must be >= 1", T);
+  if (n < 1 || n > kHcMaxN) return fail(MOE_ERR_UNSUPPORTED, "n=%d outside [1, %d]", n, kHcMaxN);
+  if (d < 8 || d % 8) return fail(MOE_ERR_INVALID_ARG, "d=%d must be a positive multiple of 8", d);
+  if (iters < 0 || iters > 10000) return fail(MOE_ERR_INVALID_ARG, "iters=%d outside [0, 10000]", iters);
+  if (!(eps >= 0.f) || eps > 1.f) return fail(MOE_ERR_INVALID_ARG, "eps must be in [0, 1]");
+  moe_status_t st;
+  if ((st = check_dev_ptr(logits, "logits")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(h, "h")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(out, "out")) != MOE_OK) return st;
+  if (P_out && (st = check_dev_ptr(P_out, "P_out")) != MOE_OK) return st;
+  if (!aligned16(h) || !aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "h and out must be 16-byte aligned");
+  DevInfo* di;
+  if ((st = dev_info(&di)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int grid = std::min(T, di->sms * 8);
+  const __nv_bfloat16* hb = reinterpret_cast<const __nv_bfloat16*>(h);
+  __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(out);
+  switch (n) {
+#define MOE_HC_CASE(N)                                                                                  \
+  case N:                                                                                               \
+    hc_sinkhorn_mix_kernel<N><<<grid, kHcThreads, 0, s>>>(logits, hb, P_out, ob, T, n, d, iters, eps); \
+    break;
+    MOE_HC_CASE(1) MOE_HC_CASE(2) MOE_HC_CASE(3) MOE_HC_CASE(4)
+    MOE_HC_CASE(5) MOE_HC_CASE(6) MOE_HC_CASE(7) MOE_HC_CASE(8)
+#undef MOE_HC_CASE
+  }
+  MOE_CHECK_LAUNCH("hc_sinkhorn_mix_kernel");
   return MOE_OK;
 }

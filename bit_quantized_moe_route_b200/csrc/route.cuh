@@ -26,9 +26,20 @@ namespace moe {
 // ---------------------------------------------------------------------------
 constexpr int kLogitWarps = 4;
 
-template <int NTB>
+// Router weight rows are fp32 or bf16 (the checkpoints store the gate in
+// bf16 [model card "DeepSeek-V4-Flash-0731-MLX-Serve-mixed-2-3-8bit",
+// precision table]); either way the logits are fp32 dot products [mlx-lm PR
+// "Add DeepSeek-v4 (Flash/Pro)", table row "MoE gate dtype"].  ldw4 returns
+// elements 4*i4 .. 4*i4+3 of a row as floats (bf16 widens exactly).
+MOE_DEV float4 ldw4(const float* __restrict__ W, size_t i4) { return __ldg(reinterpret_cast<const float4*>(W) + i4); }
+MOE_DEV float4 ldw4(const __nv_bfloat16* __restrict__ W, size_t i4) {
+  const uint2 v = __ldg(reinterpret_cast<const uint2*>(W) + i4);
+  return make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
+}
+
+template <int NTB, typename WT>
 __global__ void __launch_bounds__(kLogitWarps * 32)
-router_logits_small_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+router_logits_small_kernel(const __nv_bfloat16* __restrict__ x, const WT* __restrict__ W,
                            float* __restrict__ L, int T, int d, int E) {
   extern __shared__ __align__(16) uint32_t xs_raw[];
   const int t0 = blockIdx.y * NTB;
@@ -47,11 +58,11 @@ router_logits_small_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
   float acc[NTB];
 #pragma unroll
   for (int t = 0; t < NTB; ++t) acc[t] = 0.f;
-  const float4* wr = reinterpret_cast<const float4*>(W + (size_t)e * d);
+  const WT* wr = W + (size_t)e * d;
   const int n4 = d >> 2;
 #pragma unroll 4
   for (int i = lane; i < n4; i += 32) {
-    const float4 w = __ldg(wr + i);
+    const float4 w = ldw4(wr, i);
 #pragma unroll
     for (int t = 0; t < NTB; ++t) {
       if (t < nt) {
@@ -78,8 +89,9 @@ router_logits_small_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
 // ---------------------------------------------------------------------------
 constexpr int kLBM = 128, kLBN = 64, kLBK = 16;
 
+template <typename WT>
 __global__ void __launch_bounds__(256)
-router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const WT* __restrict__ W,
                            float* __restrict__ L, int T, int d, int E) {
   __shared__ __align__(16) float xs[kLBK][kLBM + 4];
   __shared__ __align__(16) float wsm[kLBK][kLBN + 4];
@@ -103,8 +115,7 @@ router_logits_tiled_kernel(const __nv_bfloat16* __restrict__ x, const float* __r
     const int gm = m0 + xr;
     xreg = (gm < T) ? *reinterpret_cast<const uint4*>(x + (size_t)gm * d + k0 + xc) : make_uint4(0, 0, 0, 0);
     const int gn = n0 + wr;
-    wreg = (gn < E) ? __ldg(reinterpret_cast<const float4*>(W + (size_t)gn * d + k0 + wc))
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    wreg = (gn < E) ? ldw4(W + (size_t)gn * d + k0 + wc, 0) : make_float4(0.f, 0.f, 0.f, 0.f);
   };
   load(kbeg);
   for (int k0 = kbeg; k0 < kend; k0 += kLBK) {
@@ -234,8 +245,8 @@ topk_kernel(const float* __restrict__ L, const float* __restrict__ bias, int T, 
 // Hash routing: one warp per token.  Out-of-range ids are reported through
 // the error word and routed to expert 0 with weight 0.
 // ---------------------------------------------------------------------------
-template <int KMAX>
-MOE_DEV void route_hash_warp(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+template <int KMAX, typename WT>
+MOE_DEV void route_hash_warp(const __nv_bfloat16* __restrict__ x, const WT* __restrict__ W,
                              const int* __restrict__ token_ids, const int* __restrict__ table, int T, int d, int E,
                              int k, int vocab, int* __restrict__ ids, float* __restrict__ wts, int* err) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -273,7 +284,7 @@ MOE_DEV void route_hash_warp(const __nv_bfloat16* __restrict__ x, const float* _
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
         if (j < k) {
-          const float4 w = __ldg(reinterpret_cast<const float4*>(W + (size_t)eid[j] * d) + i);
+          const float4 w = ldw4(W + (size_t)eid[j] * d, i);
           acc[j] = fmaf(w.x, x0, fmaf(w.y, x1, fmaf(w.z, x2, fmaf(w.w, x3, acc[j]))));
         }
       }
@@ -301,12 +312,12 @@ MOE_DEV void route_hash_warp(const __nv_bfloat16* __restrict__ x, const float* _
   }
 }
 
-template <int KMAX>
+template <int KMAX, typename WT>
 __global__ void __launch_bounds__(256)
-route_hash_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+route_hash_kernel(const __nv_bfloat16* __restrict__ x, const WT* __restrict__ W,
                   const int* __restrict__ token_ids, const int* __restrict__ table, int T, int d, int E,
                   int k, int vocab, int* __restrict__ ids, float* __restrict__ wts, int* err) {
-  route_hash_warp<KMAX>(x, W, token_ids, table, T, d, E, k, vocab, ids, wts, err);
+  route_hash_warp<KMAX, WT>(x, W, token_ids, table, T, d, E, k, vocab, ids, wts, err);
 }
 
 // ---------------------------------------------------------------------------
@@ -407,9 +418,9 @@ __device__ void permute_ranks_block(const int* __restrict__ ids, int N, int E, i
 constexpr int kFusedTB = 8;            // tokens per pass over the staged x rows
 constexpr int kFusedMaxT = 32;
 
-template <int MAXPER>
+template <int MAXPER, typename WT>
 __global__ void __launch_bounds__(256)
-route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const WT* __restrict__ W,
                          const float* __restrict__ bias, int T, int d, int E, int k, float* __restrict__ L,
                          int* __restrict__ ids, float* __restrict__ wts, int* __restrict__ offsets,
                          int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
@@ -428,11 +439,11 @@ route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __res
   float4 wv[8];
   const bool live = e < E;
   {
-    const float4* wr = reinterpret_cast<const float4*>(W + (size_t)min(e, E - 1) * d) + quarter * q4;
+    const WT* wr = W + (size_t)min(e, E - 1) * d + (size_t)quarter * q4 * 4;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int i = lane + 32 * u;
-      wv[u] = (live && i < q4) ? __ldg(wr + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      wv[u] = (live && i < q4) ? ldw4(wr, i) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   for (int t0 = 0; t0 < T; t0 += kFusedTB) {
@@ -508,8 +519,8 @@ route_small_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __res
 // the token's table row, every warp dots x[t] with the k router rows over its
 // slice of d (partials in `part`), warp 0 finishes the weights.  Same rules as
 // route_hash_warp (bad ids: expert 0, weight 0, error word).
-template <int KMAX>
-MOE_DEV void route_hash_block(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+template <int KMAX, typename WT>
+MOE_DEV void route_hash_block(const __nv_bfloat16* __restrict__ x, const WT* __restrict__ W,
                               const int* __restrict__ token_ids, const int* __restrict__ table, int d, int E, int k,
                               int vocab, int* __restrict__ ids, float* __restrict__ wts, int* err,
                               float (*part)[KMAX], int* s_eid, int* s_good) {
@@ -539,16 +550,16 @@ MOE_DEV void route_hash_block(const __nv_bfloat16* __restrict__ x, const float* 
     const int n4 = d >> 2;
     const int lo = n4 * warp / nw, hi = n4 * (warp + 1) / nw;
     const uint2* xr = reinterpret_cast<const uint2*>(x + (size_t)t * d);
-    const float4* wr[KMAX];
+    const WT* wr[KMAX];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) wr[j] = reinterpret_cast<const float4*>(W + (size_t)(j < k ? s_eid[j] : 0) * d);
+    for (int j = 0; j < KMAX; ++j) wr[j] = W + (size_t)(j < k ? s_eid[j] : 0) * d;
     for (int i = lo + lane; i < hi; i += 32) {
       const uint2 xv = xr[i];
       const float x0 = bf16lo(xv.x), x1 = bf16hi(xv.x), x2 = bf16lo(xv.y), x3 = bf16hi(xv.y);
 #pragma unroll
       for (int j = 0; j < KMAX; ++j) {
         if (j < k) {
-          const float4 w = __ldg(wr[j] + i);
+          const float4 w = ldw4(wr[j], i);
           acc[j] = fmaf(w.x, x0, fmaf(w.y, x1, fmaf(w.z, x2, fmaf(w.w, x3, acc[j]))));
         }
       }
@@ -582,9 +593,9 @@ MOE_DEV void route_hash_block(const __nv_bfloat16* __restrict__ x, const float* 
 
 // Hash routing plus permutation, one launch: one block per token, the last
 // block groups the pairs by expert.
-template <int KMAX>
+template <int KMAX, typename WT>
 __global__ void __launch_bounds__(256)
-route_hash_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __restrict__ W,
+route_hash_fused_kernel(const __nv_bfloat16* __restrict__ x, const WT* __restrict__ W,
                         const int* __restrict__ token_ids, const int* __restrict__ table, int T, int d, int E,
                         int k, int vocab, int* __restrict__ ids, float* __restrict__ wts, int* __restrict__ offsets,
                         int* __restrict__ sorted_rows, int* __restrict__ inv, int* __restrict__ active,
@@ -596,7 +607,7 @@ route_hash_fused_kernel(const __nv_bfloat16* __restrict__ x, const float* __rest
   __shared__ float part[8][KMAX];
   __shared__ int s_eid[KMAX], s_good[KMAX];
   pdl_trigger();  // the expert FFN may start its launch (it waits for this grid before reading)
-  route_hash_block<KMAX>(x, W, token_ids, table, d, E, k, vocab, ids, wts, err, part, s_eid, s_good);
+  route_hash_block<KMAX, WT>(x, W, token_ids, table, d, E, k, vocab, ids, wts, err, part, s_eid, s_good);
   __threadfence();  // publish this token's ids/weights before the arrival below
   __syncthreads();
   if (threadIdx.x == 0) {

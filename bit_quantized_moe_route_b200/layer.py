@@ -13,7 +13,7 @@ class MoELayer:
 
     w1/w3/w2 (and the optional shared triple) are objects with attributes
     fmt, bits, group, q, scales, biases whose tensors live on the device;
-    router_w is fp32 [E, d]; router_b fp32 [E] or None; tid2eid int32
+    router_w is fp32 or bf16 [E, d]; router_b fp32 [E] or None; tid2eid int32
     [vocab, k] selects hash routing.
     """
 
@@ -34,7 +34,8 @@ class MoELayer:
 
     def dims(self, T: int) -> _lib.Dims:
         return _lib.make_dims(T, self.d_model, self.d_ff, self.n_experts, self.top_k, self.hash_mode,
-                              self.vocab, self.d_ff_shared)
+                              self.vocab, self.d_ff_shared,
+                              router_dtype=None if self.router_w is None else self.router_w.dtype)
 
     def __call__(self, x: torch.Tensor, token_ids: Optional[torch.Tensor] = None,
                  out: Optional[torch.Tensor] = None, topk_ids: Optional[torch.Tensor] = None,

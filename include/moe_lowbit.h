@@ -117,6 +117,10 @@ typedef struct {
  * n_experts is the layer's own routed expert count: a REAP-pruned layer
  * [CARD-MLX4 "REAP-pruned builds"] passes the number of experts it kept and
  * the survivors' router rows and packs, so routing renormalises over them.
+ * router_dtype selects the router weight's storage type: fp32 (0) or bf16
+ * (1), the gate's storage in the released checkpoints [CARD-MIXED precision
+ * table]; either way each logit is an fp32 dot product of x with the widened
+ * row [PR1192 "MoE gate dtype"].
  * Limits: 1 <= T, 32 <= d_model, d_ff, d_ff_shared <= 8192 and multiples of
  * 32 and of every group size used; 1 <= top_k <= min(n_experts, 32);
  * n_experts <= 1024.
@@ -130,6 +134,7 @@ typedef struct {
   int32_t hash_mode;
   int32_t vocab;
   int32_t d_ff_shared;
+  int32_t router_dtype; /* router_w storage: 0 = fp32, 1 = bf16 (logits are fp32 either way) */
 } moe_dims_t;
 
 /* Bytes of scratch the calls below need for these dims (0 if dims invalid). */
@@ -148,13 +153,14 @@ size_t moe_workspace_size(const moe_dims_t* dims);
  *     w = renormalised s of those experts' fp32 logits, or 1/k when
  *     router_w is NULL.
  *   x        : bf16 [T, d_model]
- *   router_w : fp32 [n_experts, d_model]   (NULL only in hash mode)
+ *   router_w : fp32 or bf16 (dims->router_dtype) [n_experts, d_model]
+ *              (NULL only in hash mode)
  *   router_b : fp32 [n_experts] or NULL    (learned mode only)
  *   token_ids: int32 [T]                   (hash mode only)
  *   tid2eid  : int32 [vocab, top_k]        (hash mode only)
  *   topk_ids : int32 [T, top_k] (out);  topk_w : fp32 [T, top_k] (out)
  */
-moe_status_t moe_route(const moe_dims_t* dims, const void* x, const float* router_w,
+moe_status_t moe_route(const moe_dims_t* dims, const void* x, const void* router_w,
                        const float* router_b, const int32_t* token_ids, const int32_t* tid2eid,
                        int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, void* stream);
 
@@ -254,7 +260,7 @@ moe_status_t moe_combine(const moe_dims_t* dims, const float* y, const int32_t* 
  * GEMV path.  Results agree within the stated output tolerance.
  */
 moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* token_ids,
-                         const float* router_w, const float* router_b, const int32_t* tid2eid,
+                         const void* router_w, const float* router_b, const int32_t* tid2eid,
                          const moe_qmat_t* w1, const moe_qmat_t* w3, const moe_qmat_t* w2,
                          const moe_qmat_t* shared, void* out, int32_t* topk_ids_out,
                          float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
@@ -268,10 +274,28 @@ moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* t
  * reading out_host.
  */
 moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const int32_t* token_ids_host,
-                              const float* router_w, const float* router_b, const int32_t* tid2eid,
+                              const void* router_w, const float* router_b, const int32_t* tid2eid,
                               const moe_qmat_t* w1, const moe_qmat_t* w3, const moe_qmat_t* w2,
                               const moe_qmat_t* shared, void* out_host, void* ws, size_t ws_bytes,
                               void* stream);
+
+/*
+ * mHC residual mixing, fused (the block next to the MoE layer in each
+ * DeepSeek-V4 layer) [CARD-4BIT Architecture "mHC": hc_mult parallel copies
+ * of the hidden state recombined by a doubly-stochastic, Sinkhorn-normalised
+ * mixing matrix; PR1192 review note "Sinkhorn normalization": softmax then
+ * sum-and-divide iterations, fused into one pass].  Per token t:
+ *   P = row-wise softmax of logits[t];
+ *   iters times: every column of P divided by (its sum + eps), then every
+ *                row divided by (its sum + eps);
+ *   out[t, i, :] = bf16_rne( sum_j P[i, j] * h[t, j, :] )   (fp32 sums)
+ *   logits : fp32 [T, n, n];  h : bf16 [T, n, d];  out : bf16 [T, n, d]
+ *            (must not alias h);  P_out : fp32 [T, n, n] or NULL.
+ * Limits: 1 <= n <= 8, d a positive multiple of 8, 0 <= iters <= 10000,
+ * 0 <= eps <= 1; h and out 16-byte aligned.  One launch, no workspace.
+ */
+moe_status_t moe_hc_sinkhorn_mix(int32_t T, int32_t n, int32_t d, int32_t iters, float eps,
+                                 const float* logits, const void* h, float* P_out, void* out, void* stream);
 
 /*
  * Synchronises `stream`, reads the workspace error word into *code_out

@@ -8,6 +8,9 @@ consume what it produces.
 """
 from .moe_inputs import (  # noqa: F401
     CONFIGS,
+    HC_CONFIGS,
+    HcInputs,
+    make_hc_inputs,
     QMat,
     MoEInputs,
     make_inputs,

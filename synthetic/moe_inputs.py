@@ -217,6 +217,8 @@ def make_custom(cfg: dict, device="cpu") -> MoEInputs:
     gen.manual_seed(int(cfg["seed"]))
     x = torch.randn(T, d, generator=gen, device=device).to(torch.bfloat16)
     router_w = torch.randn(E, d, generator=gen, device=device) * cfg.get("router_std", 0.02)
+    if cfg.get("router_dtype", "fp32") == "bf16":
+        router_w = router_w.to(torch.bfloat16)   # the gate stored in bf16 (RNE of the fp32 draw)
     bias_std = cfg.get("bias_std", 0.0)
     router_b = None
     if cfg["routing"] == "learned":
@@ -250,3 +252,33 @@ def make_inputs(name: str, device="cpu", **overrides) -> MoEInputs:
     cfg["name"] = name
     cfg.update(overrides)
     return make_custom(cfg, device)
+
+
+# --------------------------------------------------------------------------
+# mHC residual mixing inputs (the block beside the MoE layer)
+# --------------------------------------------------------------------------
+HC_CONFIGS: Dict[str, dict] = {
+    # the residual stream of a prefill batch: 4096 tokens, hc_mult = 4 copies
+    # of a 4096-wide hidden state, 20 Sinkhorn iterations
+    "mhc": dict(T=4096, n=4, d=4096, iters=20, eps=0.0, logit_std=1.0, seed=5),
+    # one decode token
+    "mhc_decode": dict(T=1, n=4, d=4096, iters=20, eps=0.0, logit_std=1.0, seed=6),
+}
+
+
+@dataclasses.dataclass
+class HcInputs:
+    cfg: dict
+    logits: torch.Tensor   # fp32 [T, n, n]
+    h: torch.Tensor        # bf16 [T, n, d]
+
+
+def make_hc_inputs(cfg: dict, device="cpu") -> HcInputs:
+    """Mixing logits ~ N(0, logit_std) and residual copies ~ N(0, 1) (bf16),
+    drawn in that order from one generator seeded with cfg["seed"]."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(cfg["seed"]))
+    T, n, d = cfg["T"], cfg["n"], cfg["d"]
+    logits = torch.randn(T, n, n, generator=gen, device=device) * cfg.get("logit_std", 1.0)
+    h = torch.randn(T, n, d, generator=gen, device=device).to(torch.bfloat16)
+    return HcInputs(dict(cfg), logits.contiguous(), h.contiguous())

@@ -18,9 +18,9 @@ static int failures = 0;
   } while (0)
 
 int main(void) {
-  moe_dims_t decode = {1, 4096, 2048, 256, 8, 0, 0, 2048};
-  moe_dims_t prefill = {4096, 4096, 2048, 256, 8, 0, 0, 0};
-  moe_dims_t no_k = {4, 256, 128, 8, 0, 0, 0, 0};
+  moe_dims_t decode = {1, 4096, 2048, 256, 8, 0, 0, 2048, 0};
+  moe_dims_t prefill = {4096, 4096, 2048, 256, 8, 0, 0, 0, 0};
+  moe_dims_t no_k = {4, 256, 128, 8, 0, 0, 0, 0, 0};
   size_t n_decode = moe_workspace_size(&decode);
   size_t n_prefill = moe_workspace_size(&prefill);
   static char ws_buf[512];

@@ -24,7 +24,8 @@ def dims_for(inp, T=None):
     c = inp.cfg
     return moe.make_dims(T or c["T"], c["d"], c["f"], c["E"], c["k"], c["routing"] == "hash",
                          c.get("vocab", 0) if c["routing"] == "hash" else 0,
-                         c["f_shared"] if inp.shared is not None else 0)
+                         c["f_shared"] if inp.shared is not None else 0,
+                         router_dtype=None if inp.router_w is None else inp.router_w.dtype)
 
 
 def run_forward(inp, ws=None):

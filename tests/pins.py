@@ -525,9 +525,26 @@ def pin_hc_mix():
     assert np.array_equal(oracle.hc_mix(perm, h[:1])[0], h[0][[2, 0, 3, 1]])
 
 
+def pin_bf16_router_is_its_values():
+    """A bf16-stored router gate routes exactly like an fp32 gate holding the
+    same (widened) values: the logits are fp32-or-wider dot products of the
+    stored values, so the oracle's routing depends on the values only --
+    checked against torch's bf16 -> fp64 widening and F.linear."""
+    from synthetic import CONFIGS
+    cfg = dict(CONFIGS["tiny"], T=9, seed=45, router_dtype="bf16")
+    inp = make_custom(cfg)
+    assert inp.router_w.dtype == torch.bfloat16
+    wide = inp.router_w.double()
+    res = oracle_run(inp)
+    want = F.linear(inp.x.double(), wide).numpy()
+    assert np.allclose(res["logits"], want, rtol=1e-13, atol=1e-13)
+    ids, w, _, _ = oracle.route_learned(inp.x.double().numpy(), wide.numpy(), inp.router_b.double().numpy(), cfg["k"])
+    assert np.array_equal(ids, res["ids"]) and np.array_equal(w, res["w"])
+
+
 ALL_PINS = [pin_e2m1_table, pin_e8m0, pin_unpack_golden, pin_unpack_bigint, pin_affine_dequant,
             pin_mxfp4_dequant, pin_sqrtsoftplus, pin_topk_bruteforce, pin_route_learned,
             pin_route_hash, pin_permutation, pin_dense_equivalence, pin_single_expert_swiglu,
             pin_round_bf16, pin_e4m3_table, pin_mxfp8_dequant, pin_block128_scales, pin_parity_stats,
             pin_forward_token_subset, pin_forced_routing, pin_hc_sinkhorn_softmax, pin_hc_sinkhorn_limits,
-            pin_hc_sinkhorn_fixed_point, pin_hc_mix]
+            pin_hc_sinkhorn_fixed_point, pin_hc_mix, pin_bf16_router_is_its_values]

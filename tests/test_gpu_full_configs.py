@@ -29,6 +29,8 @@ pytestmark = pytest.mark.gpu
 
 OUTPUT_TOKENS = {"tiny": None, "decode": None, "mixed": None, "hash": list(range(0, 32, 2)),
                  "prefill": [0, 1234, 2047, 4095]}
+# the same layers with the router gate stored in bf16 (the released checkpoints' dtype)
+BF16_ROUTER = {"decode": None, "prefill": [7, 4000]}
 
 
 @pytest.fixture(scope="module")
@@ -49,12 +51,12 @@ def _routing_weights(inp, res, ids):
     if inp.cfg["routing"] == "hash":
         return res["w"]
     x = inp.x.float().cpu().numpy()
-    return oracle.route_forced(x, inp.router_w.cpu().numpy(), ids)[1]
+    return oracle.route_forced(x, inp.router_w.float().cpu().numpy(), ids)[1]
 
 
-@pytest.mark.parametrize("name", list(OUTPUT_TOKENS))
-def test_full_config(cuda_device, pool, name):
-    inp = make_inputs(name, cuda_device)
+@pytest.mark.parametrize("name,router", [(n, "fp32") for n in OUTPUT_TOKENS] + [(n, "bf16") for n in BF16_ROUTER])
+def test_full_config(cuda_device, pool, name, router):
+    inp = make_inputs(name, cuda_device, router_dtype=router)
     try:
         c = inp.cfg
         T, k, E = c["T"], c["k"], c["E"]
@@ -74,11 +76,12 @@ def test_full_config(cuda_device, pool, name):
         assert np.array_equal(offs.cpu().numpy(), o_off)
         assert np.array_equal(rows.cpu().numpy(), o_rows)
         assert np.array_equal(inv.cpu().numpy(), o_inv)
-        tok = np.arange(T) if OUTPUT_TOKENS[name] is None else np.asarray(OUTPUT_TOKENS[name])
+        sample = (OUTPUT_TOKENS if router == "fp32" else BF16_ROUTER)[name]
+        tok = np.arange(T) if sample is None else np.asarray(sample)
         ref = oracle_outputs(inp, tok, ids_np, _routing_weights(inp, res, ids_np), pool)
         stats = check_output(bf16_to_np(out)[tok], ref, name)
         assert moe.read_device_error(ws) == 0
-        print(f"\n{name}: tokens checked={len(tok)} near-ties={len(ties)} stats={stats}")
+        print(f"\n{name} ({router} router): tokens checked={len(tok)} near-ties={len(ties)} stats={stats}")
     finally:
         _free(inp)
 

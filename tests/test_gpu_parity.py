@@ -45,6 +45,9 @@ VARIANTS = {
     "stream_a4g32": dict(SMALL, d=1024, f=1024, T=3, w13=("affine", 4, 32), w2=("affine", 4, 32), seed=127),
     "stream_a2g64_a3g64": dict(SMALL, d=1024, f=1024, T=7, w13=("affine", 2, 64), w2=("affine", 3, 64), seed=128),
     "stream_many_per_expert": dict(SMALL, d=1024, f=1024, T=40, E=4, k=2, seed=129),
+    "bf16_router": dict(SMALL, router_dtype="bf16", seed=130),
+    "bf16_router_T1_d4096": dict(SMALL, T=1, d=4096, f=1024, E=64, k=8, router_dtype="bf16", seed=131),
+    "bf16_router_hash": dict(SMALL, routing="hash", vocab=300, T=11, router_dtype="bf16", seed=132),
 }
 
 

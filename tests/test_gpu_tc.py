@@ -46,6 +46,7 @@ TC_VARIANTS = {
     "tma_shared8": dict(BASE, T=200, d=1024, f=512, shared=("affine", 8, 64), f_shared=512, seed=235),
     "tma_big_experts": dict(BASE, T=600, E=4, d=512, f=512, seed=236),  # ~300 tokens per expert: 192 + rest
     "tma_a3g128": dict(BASE, T=200, d=1024, f=1024, w13=("affine", 3, 128), w2=("affine", 3, 128), seed=237),
+    "tma_bf16_router": dict(BASE, T=300, d=1024, f=1024, router_dtype="bf16", seed=238),
 }
 
 
