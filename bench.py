@@ -391,7 +391,7 @@ def run_config(name, args, dev, world, rank):
     stream = torch.cuda.current_stream()
 
     def flush_l2():
-        torch.sum(flush, dtype=torch.int64, out=flush_sum)
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
 
     def fwd():
         moe.forward(dims, inp.x, inp.token_ids, inp.router_w, inp.router_b, inp.tid2eid, inp.w1, inp.w3, inp.w2,
@@ -535,7 +535,7 @@ def run_hc_config(name, args, dev, world, rank):
         moe.hc_sinkhorn_mix(inp.logits, inp.h, out, cfg["iters"], cfg["eps"])
 
     for _ in range(max(3, args.warmup)):
-        torch.sum(flush, dtype=torch.int64, out=flush_sum)
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
         step()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -544,7 +544,7 @@ def run_hc_config(name, args, dev, world, rank):
     sampler.start()
     time.sleep(0.2)
     for s in range(args.steps):
-        torch.sum(flush, dtype=torch.int64, out=flush_sum)
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
         evs[s][0].record(stream)
         step()
         evs[s][1].record(stream)
@@ -559,7 +559,7 @@ def run_hc_config(name, args, dev, world, rank):
     L_d, h_d = torch.empty_like(inp.logits), torch.empty_like(inp.h)
     e2e = []
     for s in range(max(10, min(args.steps, 50))):
-        torch.sum(flush, dtype=torch.int64, out=flush_sum)
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         L_d.copy_(L_h, non_blocking=True)
