@@ -176,6 +176,11 @@ def kernel_work(inp, ids, tensor_path=False):
         work["ffn_w13_swiglu"] = n_act * b13 + sh13 + T * d * 2 + P * max(f, fs) * 4
         work["ffn_w2"] = n_act * b2 + sh2 + P * max(f, fs) * 4 + P * d * 4
     work["combine"] = (Tk + Ts) * d * 4 + T * d * 2 + Tk * 8
+    # the fused small-batch launch: every weight byte once, the router's
+    # rows (all of them, or the table's experts in hash mode), x in, out back
+    rw_bytes = inp.router_w.element_size() if getattr(inp, "router_w", None) is not None else 4
+    router = (len(np.unique(ids)) if c["routing"] == "hash" else E) * d * rw_bytes
+    work["decode_fused"] = n_act * (b13 + b2) + sh13 + sh2 + router + 2 * T * d * 2
     flops = 2.0 * T * k * 3 * d * f + (2.0 * T * 3 * d * fs if fs else 0.0)
     kflops = {"ffn_w13_swiglu": 2.0 * T * k * 2 * d * f, "ffn_w2": 2.0 * T * k * d * f,
               "ffn_w13_swiglu_shared": 2.0 * T * 2 * d * fs, "ffn_w2_shared": 2.0 * T * d * fs}

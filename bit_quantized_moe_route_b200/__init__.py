@@ -5,6 +5,7 @@ C ABI in ``include/moe_lowbit.h``); this package is its thin Python binding.
 """
 from ._lib import (  # noqa: F401
     FFN_AUTO,
+    FFN_DECODE_FUSED,
     FFN_GEMV,
     FFN_TENSOR_CORE,
     FMT_AFFINE,

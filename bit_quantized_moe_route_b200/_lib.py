@@ -227,13 +227,13 @@ def read_noalloc_error(stream=None) -> int:
     return code.value
 
 
-FFN_AUTO, FFN_GEMV, FFN_TENSOR_CORE = 0, 1, 2
+FFN_AUTO, FFN_GEMV, FFN_TENSOR_CORE, FFN_DECODE_FUSED = 0, 1, 2, 3
 
 
 def set_ffn_path(path: int) -> int:
     """Select the expert-FFN implementation (FFN_AUTO / FFN_GEMV /
-    FFN_TENSOR_CORE) for the calling thread's calls; returns its previous
-    setting."""
+    FFN_TENSOR_CORE / FFN_DECODE_FUSED) for the calling thread's calls;
+    returns its previous setting."""
     prev = load_library().moe_set_ffn_path(int(path))
     if prev < 0:
         raise ValueError(f"unknown FFN path {path}")

@@ -19,6 +19,7 @@
 #include "tc_prep.cuh"
 #include "ffn_umma.cuh"
 #include "hc_mix.cuh"
+#include "ffn_decode.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -94,6 +95,7 @@ struct WsLayout {
   size_t hdr, logits, ids, wts, offsets, sorted, inv, active, h, y, xstage, tokstage, outstage;
   size_t x16, tiles, tiles2, ntiles;  // tensor-core FFN: fp16 token rows by position, token-tile plans
   size_t pchunks;                     // multi-CTA permutation: per-chunk expert counts / bases
+  size_t dxp, dxsx, dhp, dhsx, dcnth, dcnty, dsync;  // fused decode: planes, block steps, counters
   bool tc = false;            // the regions above exist
   size_t total;
 };
@@ -129,6 +131,19 @@ WsLayout layout_of(const moe_dims_t& d) {
   L.tiles2 = take(((T * k + kUmN - 1) / kUmN + E) * sizeof(int4));
   L.ntiles = take(2 * sizeof(int));
   L.pchunks = take(((T * k + kPermThreads - 1) / kPermThreads) * E * sizeof(int));
+  {
+    // fused small-batch layer (T <= 32): activation planes of x (two layouts)
+    // and of h, their per-64-input steps and sums, dependency counters
+    const bool dec = T <= (size_t)kDecMaxT;
+    const size_t fm = (size_t)f_max_of(d);
+    L.dxp = take(dec ? 2 * T * D * 4 : 0);
+    L.dxsx = take(dec ? T * (D / 64 + 1) * 16 : 0);
+    L.dhp = take(dec ? P * fm * 4 : 0);
+    L.dhsx = take(dec ? P * (fm / 64 + 1) * 16 : 0);
+    L.dcnth = take(dec ? (kDecMaxPairs + 8) * sizeof(int) : 0);
+    L.dcnty = take(dec ? (D / 64 + 1) * sizeof(int) : 0);
+    L.dsync = take(dec ? 4 * sizeof(int) : 0);
+  }
   L.tc = true;
   L.total = o;
   return L;
@@ -232,6 +247,7 @@ void route_attrs() {
 struct DevInfo {
   int sms = 0;
   int ffn1_blocks = 0, ffn2_blocks = 0;
+  int dec_blocks = 0;  // fused decode: co-resident CTAs (one per SM)
 };
 DevInfo g_dev[64];
 std::atomic<int> g_dev_ready[64];
@@ -258,6 +274,10 @@ moe_status_t dev_info(DevInfo** out) {
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, ffn_gemv_kernel<2, 8>, kFfnThreads, 0);
       di.ffn1_blocks = std::max(1, b1);
       di.ffn2_blocks = std::max(1, b2);
+      cudaFuncSetAttribute(ffn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmem);
+      int bd = 0;
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bd, ffn_decode_kernel, kDecThreads, kDecSmem);
+      di.dec_blocks = std::min(bd, 1) * di.sms;
       cudaError_t le = cudaGetLastError();
       if (le != cudaSuccess) {
         g_dev_ready[dev].store(0);
@@ -780,6 +800,117 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------- fused small-batch layer
+// Stage geometry of a packed matrix in the fused kernel: inputs per stage
+// (256 code bytes per row; 3-bit: 192), TMA box width.
+bool dec_mat(const QMatDev& Q, DecMat* m) {
+  m->scales = Q.scales;
+  m->biases = Q.biases;
+  m->fmt = Q.fmt;
+  m->group = Q.group;
+  m->n_out = Q.n_out;
+  m->n_in = Q.n_in;
+  m->gpr = Q.gpr;
+  switch (Q.fmt) {
+    case F_A2: m->ks = 1024; break;
+    case F_A8: m->ks = 256; break;
+    default: m->ks = 512; break;
+  }
+  m->stage_row = Q.fmt == F_A3 ? 192 : 256;
+  m->box = Q.fmt == F_A3 ? 96 : 128;
+  if (Q.n_in % m->ks || Q.n_out % kDecRows || Q.group > m->ks) return false;
+  if (Q.fmt == F_A2 && Q.group == 32) return false;  // a 2-bit k-block mixes two 32-input groups
+  const int esz = Q.fmt == F_MX4 ? 1 : 2;
+  const int sbytes = m->ks / Q.group * esz;
+  if (sbytes > 32 || sbytes < 4) return false;
+  if ((Q.gpr * esz) % std::min(16, sbytes)) return false;  // cp.async source alignment
+  if ((Q.wpr * 4) % 16) return false;                         // TMA row stride
+  return true;
+}
+
+bool dec_eligible(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh) {
+  if (d.T > kDecMaxT || d.T * d.top_k > kDecMaxPairs || d.n_experts > 1024) return false;
+  // d_model a multiple of 128: the logit pass gives each lane 8 consecutive inputs of a 1/16 slice
+  if (d.d_model % 128 || d.d_ff % 64 || (sh && d.d_ff_shared % 64)) return false;
+  DecMat m;
+  if (!dec_mat(w1, &m) || !dec_mat(w3, &m) || !dec_mat(w2, &m)) return false;
+  if (sh && (!dec_mat(sh[0], &m) || !dec_mat(sh[1], &m) || !dec_mat(sh[2], &m))) return false;
+  return true;
+}
+
+bool use_dec(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh) {
+  const int mode = g_ffn_path;
+  if (mode == MOE_FFN_GEMV || mode == MOE_FFN_TENSOR_CORE) return false;
+  return dec_eligible(d, w1, w3, w2, sh);
+}
+
+moe_status_t dec_code_map(CUtensorMap* map, const QMatDev& Q, int E, const DecMat& m) {
+  return tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.q, (uint64_t)Q.wpr * 4, (uint64_t)E * Q.n_out,
+                 (uint64_t)Q.wpr * 4, m.box, kDecRows, Q.fmt != F_A3);
+}
+
+moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32_t* token_ids, const void* router_w,
+                                 const float* router_b, const int32_t* tid2eid, const QMatDev& q1, const QMatDev& q3,
+                                 const QMatDev& q2, const QMatDev* qs, void* out, int32_t* ids_out, float* w_out,
+                                 void* ws, const WsLayout& L, cudaStream_t s, const DevInfo& di) {
+  DecParams p{};
+  const QMatDev* mats[6] = {&q1, &q3, &q2, qs ? &qs[0] : &q1, qs ? &qs[1] : &q3, qs ? &qs[2] : &q2};
+  for (int i = 0; i < 6; ++i) {
+    dec_mat(*mats[i], &p.m[i]);
+    moe_status_t st = dec_code_map(&p.map[i], *mats[i], (i < 3 || !qs) ? d.n_experts : 1, p.m[i]);
+    if (st != MOE_OK) return st;
+  }
+  p.x = reinterpret_cast<const __nv_bfloat16*>(x);
+  p.router_w = router_w;
+  p.router_b = router_b;
+  p.token_ids = token_ids;
+  p.tid2eid = tid2eid;
+  p.router_bf16 = d.router_dtype == 1;
+  p.T = d.T;
+  p.d = d.d_model;
+  p.f = d.d_ff;
+  p.fs = qs ? d.d_ff_shared : 0;
+  p.E = d.n_experts;
+  p.k = d.top_k;
+  p.hash = d.hash_mode;
+  p.vocab = d.vocab;
+  p.has_shared = qs != nullptr;
+  p.logits = ws_at<float>(ws, L.logits);
+  p.hids = ws_at<int>(ws, L.ids);
+  p.hw = ws_at<float>(ws, L.wts);
+  p.xplanes = ws_at<uint8_t>(ws, L.dxp);
+  p.xsx = ws_at<float4>(ws, L.dxsx);
+  p.hplanes = ws_at<uint8_t>(ws, L.dhp);
+  p.hsx = ws_at<float4>(ws, L.dhsx);
+  p.y = ws_at<float>(ws, L.y);
+  p.cnt_h = ws_at<int>(ws, L.dcnth);
+  p.cnt_y = ws_at<int>(ws, L.dcnty);
+  p.sync = ws_at<int>(ws, L.dsync);
+  p.err = &ws_at<WsHeader>(ws, L.hdr)->err;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.ids_out = ids_out;
+  p.w_out = w_out;
+  p.G = di.dec_blocks;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the kernel's CTAs wait on one another
+  attr[0].val.cooperative = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.G);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = kDecSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le = cudaLaunchKernelEx(&cfg, ffn_decode_kernel, p);
+  if (le != cudaSuccess) {
+    cudaGetLastError();
+    return cuda_fail(le, "ffn_decode_kernel");
+  }
+  MOE_CHECK_LAUNCH("ffn_decode_kernel");
+  hook_mark(s, "decode_fused");
+  return MOE_OK;
+}
+
 moe_status_t launch_combine(const moe_dims_t& d, const float* y, const int* inv, const float* w,
                             const float* y_shared, void* out, cudaStream_t s) {
   cudaLaunchAttribute attr[1];
@@ -858,7 +989,8 @@ const char* moe_status_string(moe_status_t s) {
 const char* moe_last_error_detail(void) { return g_detail; }
 
 int32_t moe_set_ffn_path(int32_t path) {
-  if (path != MOE_FFN_AUTO && path != MOE_FFN_GEMV && path != MOE_FFN_TENSOR_CORE) return -1;
+  if (path != MOE_FFN_AUTO && path != MOE_FFN_GEMV && path != MOE_FFN_TENSOR_CORE && path != MOE_FFN_DECODE_FUSED)
+    return -1;
   const int prev = g_ffn_path;
   g_ffn_path = path;
   return prev;
@@ -1009,6 +1141,16 @@ moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t*
                               float* topk_w_out, void* ws, const WsLayout& L, cudaStream_t s) {
   moe_status_t st;
   hook_begin(s);
+  {
+    DevInfo* di = nullptr;
+    if ((st = dev_info(&di)) != MOE_OK) return st;
+    const QMatDev* sh = d.d_ff_shared > 0 ? qs : nullptr;
+    if (di->dec_blocks > 0 && use_dec(d, q1, q3, q2, sh))
+      return launch_decode_fused(d, x, token_ids, router_w, router_b, tid2eid, q1, q3, q2, sh, out, topk_ids_out,
+                                 topk_w_out, ws, L, s, *di);
+    if (g_ffn_path == MOE_FFN_DECODE_FUSED)
+      return fail(MOE_ERR_UNSUPPORTED, "the fused decode path does not take these shapes or formats");
+  }
   int* ids = topk_ids_out ? topk_ids_out : ws_at<int>(ws, L.ids);
   float* wts = topk_w_out ? topk_w_out : ws_at<float>(ws, L.wts);
   int* offsets = ws_at<int>(ws, L.offsets);

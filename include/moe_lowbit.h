@@ -320,13 +320,26 @@ const char* moe_timing_label(int32_t i);
  * Expert-FFN implementation used by the calling thread's moe_expert_ffn /
  * moe_forward / moe_forward_host calls (a per-thread setting: other
  * threads' calls are not affected; not for the allocation-free entry point,
- * which always streams).  AUTO (default) takes the tensor-core path
- * from T >= 4 tokens when the shapes allow it (d_ff, d_model multiples of
- * 128), and the weight-streaming GEMV below that.
+ * which always streams).  For moe_forward / moe_forward_host, AUTO (default)
+ * runs the whole layer as ONE fused launch for small batches when the shapes
+ * allow it (T <= 32, T*top_k <= 256, d_model and d_ff multiples of 64 and of
+ * the formats' stage widths -- 1024 inputs for 2-bit, 512 for 3/4-bit and
+ * mxfp4, 256 for 8-bit -- and not 2-bit with 32-input groups): routing,
+ * both FFN stages on the integer tensor-core MMA, and the combine (whose k
+ * slots are summed in ascending j, then the shared expert, one bf16
+ * rounding).  Otherwise AUTO takes the tcgen05 grouped GEMM from T >= 4
+ * (d_ff, d_model multiples of 128) and the weight-streaming GEMV below.
+ * DECODE_FUSED forces the fused launch (MOE_ERR_UNSUPPORTED when the shapes
+ * do not allow it); GEMV and TENSOR_CORE force the step-by-step kernels.
  * Returns the previous setting, or -1 (setting unchanged) for an unknown
  * value.
  */
-typedef enum { MOE_FFN_AUTO = 0, MOE_FFN_GEMV = 1, MOE_FFN_TENSOR_CORE = 2 } moe_ffn_path_t;
+typedef enum {
+  MOE_FFN_AUTO = 0,
+  MOE_FFN_GEMV = 1,
+  MOE_FFN_TENSOR_CORE = 2,
+  MOE_FFN_DECODE_FUSED = 3
+} moe_ffn_path_t;
 int32_t moe_set_ffn_path(int32_t path);
 
 /* Static description of a status code. */
