@@ -66,6 +66,7 @@ _SIGS = {
     "moe_timing_count": (ctypes.c_int32, []),
     "moe_timing_label": (ctypes.c_char_p, [ctypes.c_int32]),
     "moe_set_ffn_path": (ctypes.c_int32, [ctypes.c_int32]),
+    "moe_test_stall_fused_wait": (ctypes.c_int32, [ctypes.c_int32]),
     "moe_hc_sinkhorn_mix": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                            ctypes.c_float, _VP, _VP, _VP, _VP, _VP]),
 }

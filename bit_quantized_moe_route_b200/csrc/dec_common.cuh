@@ -93,6 +93,11 @@ MOE_DEV uint32_t lds8u(uint32_t a) {
   asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
+MOE_DEV float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
 MOE_DEV float2 lds_f2(uint32_t a) {
   float2 v;
   asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
@@ -163,13 +168,14 @@ MOE_DEV void red_release_add(int* p, int v) {
 
 constexpr long long kDecWaitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
 
-// Spin (bounded) until *p >= target; false on timeout or abort.
-MOE_DEV bool dec_wait_count(const int* p, int target, const volatile int* abort_flag) {
+// Spin (bounded by `limit` cycles) until *p >= target; false on timeout or abort.
+MOE_DEV bool dec_wait_count(const int* p, int target, const volatile int* abort_flag,
+                            long long limit = kDecWaitCycles) {
   if (ld_acquire(p) >= target) return true;
   const long long t0 = clock64();
   while (ld_acquire(p) < target) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kDecWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
     __nanosleep(64);
   }
   return true;

@@ -25,13 +25,17 @@
 // Units are dealt round-robin over the CTAs in the order [S1 shared, S1
 // routed, S2 by group], so every CTA does the same amount of streaming.
 //
-// Inside a CTA one producer warp streams each unit's weights in stages of 64
-// rows x 256 code bytes per matrix (TMA, 128-byte swizzle; 3-bit: two
-// unswizzled 96-byte boxes), scales and biases (cp.async) and the activation
-// planes (bulk copies) into a 3-slot ring; 16 consumer warps, one per
-// (16-row tile, quarter of the stage's inputs), unpack codes to bytes, run
-// m16n8k32 integer MMAs against the planes (exact int32 sums per 64-input
-// block) and fold each block into fp32 with the weight scale and bias.
+// Inside a CTA one producer warp streams each unit's weights into a 3-slot
+// ring, one stage = 512 code bytes of each of 32 rows of W1 and of W3 (S1;
+// a unit's 64 rows are two halves) or of 64 rows of W2 (S2), as 128-byte
+// wide TMA boxes with the 128-byte swizzle (3-bit: 96-byte unswizzled
+// boxes), plus the rows' scales and biases (TMA) and the activation planes
+// of the group's tokens (bulk copies).  Per-row runs of 512 bytes keep the
+// weight stream near the copy rate (narrower runs cost DRAM and TMA
+// efficiency).  16 consumer warps, one per (16-row tile, slice of the
+// stage's inputs), unpack codes to bytes, run m16n8k32 integer MMAs against
+// the planes (exact int32 sums per 64-input block) and fold each block into
+// fp32 with the weight scale and bias.
 // Every wait is bounded: on timeout the kernel records MOE_ERR_TIMEOUT, keeps
 // every warp's barrier sequence, lets in-flight copies land and returns.
 #pragma once
@@ -44,20 +48,20 @@ namespace moe {
 constexpr int kDecConsumerWarps = 16;
 constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
 constexpr int kDecStages = 3;
-constexpr int kDecRows = 64;        // weight rows per unit
-constexpr int kDecMaxTok = 8;       // tokens per group (MMA N)
+constexpr int kDecRows = 64;        // weight rows per unit (S1: two halves of 32)
+constexpr int kDecMaxTok = 4;       // tokens per group (B columns 0..3 of the MMA)
 constexpr int kDecMaxT = 32;
 constexpr int kDecMaxPairs = 256;   // T * top_k
-constexpr int kDecCodeMat = 16384;  // code bytes per matrix and stage (64 rows x 256 B)
-constexpr int kDecScaleMat = 4096;  // scales (2 KB) + biases (2 KB) per matrix and stage
-constexpr int kDecPlaneStride = 2112;  // per token and stage: <= 2048 plane bytes + bank padding
-constexpr int kDecSlotCodes = 0;
-constexpr int kDecSlotScales = 2 * kDecCodeMat;
-constexpr int kDecSlotPlanes = kDecSlotScales + 2 * kDecScaleMat;
+constexpr int kDecStageRow = 512;   // code bytes per row and stage (3-bit: 384)
+constexpr int kDecScaleRow = 64;    // scale (or bias) bytes per row and stage, at most
+constexpr int kDecPlaneStride = 4160;  // per token and stage: <= 4096 plane bytes + bank padding
+constexpr int kDecSxStride = 512;      // per token and stage: <= 32 blocks x (step, sum lo, sum hi, sum)
+constexpr int kDecSlotCodes = 0;       // 32 KB: S1 32 rows x 512 B x 2 matrices, S2 64 rows x 512 B
+constexpr int kDecSlotScales = 32768;  // 8 KB: scales and biases
+constexpr int kDecSlotPlanes = kDecSlotScales + 8192;
 constexpr int kDecSlotSx = kDecSlotPlanes + kDecMaxTok * kDecPlaneStride;
-constexpr int kDecSxStride = 256;     // per token and stage: <= 16 blocks x (step, sum lo, sum hi, sum)
 constexpr int kDecSlotBytes = ((kDecSlotSx + kDecMaxTok * kDecSxStride) + 1023) / 1024 * 1024;
-constexpr int kDecRedBytes = 16 * 2 * 16 * 8 * 4;  // 16 warps x 2 matrices x 16 rows x 8 tokens
+constexpr int kDecRedBytes = 16 * 2 * 16 * 8 * 4;  // 16 warps x 2 matrices x 16 rows x 8 columns
 constexpr int kDecHBytes = kDecMaxTok * kDecRows * 4;
 constexpr int kDecOffLen = 1028;   // offsets / active list entries (E + 1 <= 1025, padded to 16 bytes)
 constexpr int kDecRouteBytes = 6 * kDecMaxPairs * 4 + 2 * kDecOffLen * 4 + (kDecMaxPairs + 8) * 16;
@@ -70,19 +74,19 @@ static_assert((kDecRedBytes + kDecHBytes) % 16 == 0 && (6 * kDecMaxPairs * 4 + 2
 
 // One packed matrix as the fused kernel reads it.
 struct DecMat {
-  const void* scales;
-  const void* biases;
   int fmt, group, n_out, n_in;
-  int gpr;        // scale groups per row
+  int rows;       // rows per stage: 32 (W1, W3) or 64 (W2)
+  int box;        // TMA box width in bytes (128 swizzled, or 96 unswizzled for 3-bit); 4 boxes per stage
   int ks;         // inputs per stage
-  int stage_row;  // code bytes per row per stage (256, or 192 for 3-bit)
-  int box;        // TMA box width in bytes (128, or 96 unswizzled for 3-bit)
+  int sbytes;     // scale (and bias) bytes per row and stage
 };
 
 enum DecMatIdx { DM_W1 = 0, DM_W3 = 1, DM_W2 = 2, DM_S1 = 3, DM_S3 = 4, DM_S2 = 5 };
 
 struct DecParams {
-  CUtensorMap map[6];  // codes of w1, w3, w2, shared w1, w3, w2
+  CUtensorMap map[6];   // codes of w1, w3, w2, shared w1, w3, w2
+  CUtensorMap smap[6];  // their scales
+  CUtensorMap bmap[6];  // their biases (affine)
   DecMat m[6];
   const __nv_bfloat16* x;
   const void* router_w;
@@ -108,6 +112,7 @@ struct DecParams {
   __nv_bfloat16* out;  // [T][d]
   int* ids_out;        // [T][k] or NULL
   float* w_out;        // [T][k] or NULL
+  int stall_test;      // testing the timeout path: the first W2 dependency waits on a count nothing reaches
 };
 
 // ------------------------------------------------------------ grid barrier
@@ -190,118 +195,114 @@ MOE_DEV float4 dec_make_block(float v0, float v1, int perm, bool with_neg, uint8
 }
 
 // ------------------------------------------------------------ A operands
-// Code bytes of (row tile rt, k-block) of matrix slot `mat` in a stage slot,
-// as the four A-fragment registers (unsigned bytes).  For mxfp4 `an` gets the
-// magnitudes of the negative codes (positive ones in `a`).
-template <int FMT>
-struct DecA;
+// Stage layout of one matrix's codes: 4 TMA boxes side by side along the row
+// (box b = bytes [b*box, (b+1)*box) of each of `rows` rows), each box `rows`
+// lines of `box` bytes; 128-byte boxes are swizzled (16-byte chunk c of line
+// r sits at chunk c ^ (r & 7)), so the 8 rows an ldmatrix phase reads hit
+// distinct banks.
+struct DecTile {
+  uint32_t codes;  // shared address of the matrix's first box
+  int rows;        // lines per box
+  int rt;          // 16-row tile
+  int byte0;       // first code byte (in the stage row) of this warp's slice
+};
 
-// 128-byte swizzled box: 16-byte chunk c of row r sits at chunk c ^ (r & 7)
 MOE_DEV uint32_t swz(uint32_t box, int row, int chunk) {
   return box + (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
+// ldmatrix x4 of two 16-byte chunks (bytes `byte`, `byte`+16 of the stage row)
+// of the tile's rows: d[0] = (row g, chunk 0), d[1] = (g+8, chunk 0),
+// d[2] = (g, chunk 1), d[3] = (g+8, chunk 1)
+MOE_DEV void dec_ldsm2(const DecTile& tl, int byte, uint32_t (&d)[4]) {
+  const int lane = threadIdx.x & 31, mtx = lane >> 3;
+  const int row = tl.rt * 16 + (mtx & 1) * 8 + (lane & 7);
+  const int b = byte + (mtx >> 1) * 16;
+  ldsm_x4(swz(tl.codes + (b >> 7) * tl.rows * 128, row, (b & 127) >> 4), d[0], d[1], d[2], d[3]);
+}
 
-template <>
-struct DecA<F_A8> {  // 32 bytes per k-block and row: chunks 2kb, 2kb+1
-  static constexpr int KB_PER_WARP = 2;
-  MOE_DEV static void load(uint32_t codes, int rt, int kq, int kbw, uint32_t (&a)[4], uint32_t (&)[4]) {
-    const int lane = threadIdx.x & 31, mtx = lane >> 3;
-    const int row = rt * 16 + (mtx & 1) * 8 + (lane & 7);
-    const int chunk = (kq & 1) * 4 + 2 * kbw + (mtx >> 1);
-    ldsm_x4(swz(codes + (kq >> 1) * 8192, row, chunk), a[0], a[1], a[2], a[3]);
-  }
+// ldmatrix x2 of one 16-byte chunk of the tile's rows: d[0] = row g, d[1] = row g+8
+MOE_DEV void dec_ldsm1(const DecTile& tl, int byte, uint32_t (&d)[4]) {
+  const int lane = threadIdx.x & 31;
+  const int row = tl.rt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(d[0]), "=r"(d[1])
+               : "r"(swz(tl.codes + (byte >> 7) * tl.rows * 128, row, (byte & 127) >> 4)));
+}
+
+// per format: bits per code, and how a k-block's codes become A registers
+template <int FMT>
+struct DecA {
+  static constexpr int bits = FMT == F_A2 ? 2 : FMT == F_A3 ? 3 : FMT == F_A8 ? 8 : 4;
 };
 
-template <>
-struct DecA<F_A4> {  // 16 bytes per k-block and row (one chunk)
-  static constexpr int KB_PER_WARP = 4;
-  MOE_DEV static void load2(uint32_t codes, int rt, int kq, int kbw, uint32_t (&w)[4]) {
-    const int lane = threadIdx.x & 31, mtx = lane >> 3;
-    const int row = rt * 16 + (mtx & 1) * 8 + (lane & 7);
-    const int chunk = (kq & 1) * 4 + kbw + (mtx >> 1);  // k-blocks kbw, kbw+1
-    ldsm_x4(swz(codes + (kq >> 1) * 8192, row, chunk), w[0], w[1], w[2], w[3]);
-  }
-  MOE_DEV static void unpack(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
-    a[0] = wg & 0x0F0F0F0Fu;
-    a[1] = wg8 & 0x0F0F0F0Fu;
-    a[2] = (wg >> 4) & 0x0F0F0F0Fu;
-    a[3] = (wg8 >> 4) & 0x0F0F0F0Fu;
-  }
-};
-
-template <>
-struct DecA<F_MX4> {
-  static constexpr int KB_PER_WARP = 4;
-  // 2 * |e2m1| of codes 0..7 (sign bit clear): 0, 1, 2, 3, 4, 6, 8, 12; a
-  // selector nibble with its top bit set (a negative code) yields 0
-  MOE_DEV static uint32_t mag4(uint32_t sel) {
-    uint32_t r;  // prmt default mode: a selector nibble's top bit replicates the chosen byte's sign bit
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(0x03020100u), "r"(0x0C080604u), "r"(sel));
-    return r;
-  }
-  MOE_DEV static void unpack(uint32_t wg, uint32_t wg8, uint32_t (&a)[4], uint32_t (&an)[4]) {
-    const uint32_t fg = wg ^ 0x88888888u, fg8 = wg8 ^ 0x88888888u;
-    a[0] = mag4(wg);
-    a[2] = mag4(wg >> 16);
-    a[1] = mag4(wg8);
-    a[3] = mag4(wg8 >> 16);
-    an[0] = mag4(fg);
-    an[2] = mag4(fg >> 16);
-    an[1] = mag4(fg8);
-    an[3] = mag4(fg8 >> 16);
-  }
-};
-
-template <>
-struct DecA<F_A2> {  // one chunk = 64 codes = two k-blocks
-  static constexpr int KB_PER_WARP = 8;
-  MOE_DEV static void unpack(uint32_t wg, uint32_t wg8, int kb2, uint32_t (&a)[4]) {
-    const int s0 = 4 * kb2, s1 = 4 * kb2 + 2;
-    a[0] = (wg >> s0) & 0x03030303u;
-    a[1] = (wg8 >> s0) & 0x03030303u;
-    a[2] = (wg >> s1) & 0x03030303u;
-    a[3] = (wg8 >> s1) & 0x03030303u;
-  }
-};
-
-template <>
-struct DecA<F_A3> {  // 12 bytes per k-block and row, two 96-byte unswizzled boxes of 64 rows
-  static constexpr int KB_PER_WARP = 4;
-  // four 3-bit codes (12 bits) -> bytes 0..3
-  MOE_DEV static uint32_t spread4(uint32_t t) {
-    const uint32_t ev = ((t & 0x1C7u) * 0x401u) & 0x00070007u;
-    const uint32_t od = ((t & 0xE38u) * 0x8020u) & 0x07000700u;
-    return ev | od;
-  }
-  MOE_DEV static uint32_t codes8(uint32_t codes, int row, int kq, int kbw, int t) {
-    const uint32_t base = codes + (kq >> 1) * (64 * 96) + row * 96 + (kq & 1) * 48 + kbw * 12;
-    const int byte = 3 * t;  // codes 8t..8t+7 = bits 24t..24t+23
-    const uint32_t w0 = lds32u(base + (byte & ~3)), w1 = lds32u(base + (byte & ~3) + 4);
-    return __funnelshift_r(w0, w1, 8 * (byte & 3)) & 0xFFFFFFu;
-  }
-  MOE_DEV static void load(uint32_t codes, int rt, int kq, int kbw, uint32_t (&a)[4], uint32_t (&)[4]) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    const uint32_t vg = codes8(codes, rt * 16 + g, kq, kbw, t), vg8 = codes8(codes, rt * 16 + 8 + g, kq, kbw, t);
-    a[0] = spread4(vg & 0xFFFu);
-    a[2] = spread4(vg >> 12);
-    a[1] = spread4(vg8 & 0xFFFu);
-    a[3] = spread4(vg8 >> 12);
-  }
-};
+MOE_DEV void unpack_a4(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
+  a[0] = wg & 0x0F0F0F0Fu;
+  a[1] = wg8 & 0x0F0F0F0Fu;
+  a[2] = (wg >> 4) & 0x0F0F0F0Fu;
+  a[3] = (wg8 >> 4) & 0x0F0F0F0Fu;
+}
+// 2 * |e2m1| of codes 0..7 (sign bit clear): 0, 1, 2, 3, 4, 6, 8, 12; a
+// selector nibble with its top bit set (a negative code) yields 0
+MOE_DEV uint32_t mag4(uint32_t sel) {
+  uint32_t r;  // prmt default mode: a selector nibble's top bit replicates the chosen byte's sign bit
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(0x03020100u), "r"(0x0C080604u), "r"(sel));
+  return r;
+}
+MOE_DEV void unpack_mx4(uint32_t wg, uint32_t wg8, uint32_t (&a)[4], uint32_t (&an)[4]) {
+  const uint32_t fg = wg ^ 0x88888888u, fg8 = wg8 ^ 0x88888888u;
+  a[0] = mag4(wg);
+  a[2] = mag4(wg >> 16);
+  a[1] = mag4(wg8);
+  a[3] = mag4(wg8 >> 16);
+  an[0] = mag4(fg);
+  an[2] = mag4(fg >> 16);
+  an[1] = mag4(fg8);
+  an[3] = mag4(fg8 >> 16);
+}
+MOE_DEV void unpack_a2(uint32_t wg, uint32_t wg8, int kb2, uint32_t (&a)[4]) {
+  const int s0 = 4 * kb2, s1 = 4 * kb2 + 2;
+  a[0] = (wg >> s0) & 0x03030303u;
+  a[1] = (wg8 >> s0) & 0x03030303u;
+  a[2] = (wg >> s1) & 0x03030303u;
+  a[3] = (wg8 >> s1) & 0x03030303u;
+}
+// four 3-bit codes (12 bits) -> bytes 0..3
+MOE_DEV uint32_t spread3x4(uint32_t t) {
+  const uint32_t ev = ((t & 0x1C7u) * 0x401u) & 0x00070007u;
+  const uint32_t od = ((t & 0xE38u) * 0x8020u) & 0x07000700u;
+  return ev | od;
+}
+// codes 8t..8t+7 of k-block (12 bytes) starting at stage byte `byte` of `row`
+// (unswizzled 96-byte boxes)
+MOE_DEV uint32_t codes3x8(const DecTile& tl, int row, int byte, int t) {
+  const int box = byte / 96, off = byte - box * 96;
+  const uint32_t base = tl.codes + box * tl.rows * 96 + row * 96 + off;
+  const int bt = 3 * t;
+  const uint32_t w0 = lds32u(base + (bt & ~3)), w1 = lds32u(base + (bt & ~3) + 4);
+  return __funnelshift_r(w0, w1, 8 * (bt & 3)) & 0xFFFFFFu;
+}
+MOE_DEV void load_a3(const DecTile& tl, int byte, uint32_t (&a)[4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const uint32_t vg = codes3x8(tl, tl.rt * 16 + g, byte, t), vg8 = codes3x8(tl, tl.rt * 16 + 8 + g, byte, t);
+  a[0] = spread3x4(vg & 0xFFFu);
+  a[2] = spread3x4(vg >> 12);
+  a[1] = spread3x4(vg8 & 0xFFFu);
+  a[3] = spread3x4(vg8 >> 12);
+}
 
 // ------------------------------------------------------------ one stage
-// Consumer warp (rt, kq) over its quarter of one stage: integer MMAs per
+// Consumer warp (rt, kq) over its slice of one stage: integer MMAs per
 // k-block, folded into acc[m][4] once per 64-input block (or per 32-input
 // group).  ntok tokens occupy B columns 0..ntok-1.
 struct DecStageCtx {
   uint32_t slot;        // shared address of the stage slot
   int rt, kq, ntok;
-  const DecMat* mat[2];
+  int group, ks, rows;  // of the unit's matrices
 };
 
 template <int FMT>
-MOE_DEV void dec_scale_bias(const DecStageCtx& c, int m, int grp, int row, float& s, float& b) {
-  const uint32_t sc = c.slot + kDecSlotScales + m * kDecScaleMat + row * 32;
+MOE_DEV void dec_scale_bias(const DecStageCtx& c, int m, int grp, int row, int sbytes, float& s, float& b) {
+  const uint32_t sc = c.slot + kDecSlotScales + m * 4096 + row * sbytes;
   if constexpr (FMT == F_MX4) {
     const uint32_t e = lds8u(sc + grp);
     // 2^(e-127) / 2 (the A operand holds 2*e2m1)
@@ -309,113 +310,95 @@ MOE_DEV void dec_scale_bias(const DecStageCtx& c, int m, int grp, int row, float
     b = 0.f;
   } else {
     s = bf16_bits_to_float(lds16u(sc + 2 * grp));
-    b = bf16_bits_to_float(lds16u(sc + 2048 + 2 * grp));
+    b = bf16_bits_to_float(lds16u(sc + c.rows * kDecScaleRow + 2 * grp));
   }
 }
 
+// acc[0..3] += s_r * step_c * P_rc + b_r * sum_c for the C-fragment layout
+// (rows g, g+8; columns 2t, 2t+1) of one group; `si` selects the sum over
+// the group's inputs in the (step, sum lo, sum hi, sum) record of the block
+template <int FMT>
+MOE_DEV void dec_fold(const DecStageCtx& c, int m, int grp, int sbytes, int bs, int si, const int (&ch)[4],
+                      const int (&cl)[4], float (&acc)[4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int r0 = c.rt * 16 + g, r1 = r0 + 8;
+  const int c0 = 2 * t, c1 = c0 + 1;
+  const uint32_t sx = c.slot + kDecSlotSx + bs * 16;
+  const float st0 = c0 < c.ntok ? lds_f32(sx + c0 * kDecSxStride) : 0.f;
+  const float st1 = c1 < c.ntok ? lds_f32(sx + c1 * kDecSxStride) : 0.f;
+  const float sm0 = c0 < c.ntok ? lds_f32(sx + c0 * kDecSxStride + 4 * si) : 0.f;
+  const float sm1 = c1 < c.ntok ? lds_f32(sx + c1 * kDecSxStride + 4 * si) : 0.f;
+  float s0, b0, s1, b1;
+  dec_scale_bias<FMT>(c, m, grp, r0, sbytes, s0, b0);
+  dec_scale_bias<FMT>(c, m, grp, r1, sbytes, s1, b1);
+  acc[0] = fmaf(s0 * st0, (float)(ch[0] * 256 + cl[0]), fmaf(b0, sm0, acc[0]));
+  acc[1] = fmaf(s0 * st1, (float)(ch[1] * 256 + cl[1]), fmaf(b0, sm1, acc[1]));
+  acc[2] = fmaf(s1 * st0, (float)(ch[2] * 256 + cl[2]), fmaf(b1, sm0, acc[2]));
+  acc[3] = fmaf(s1 * st1, (float)(ch[3] * 256 + cl[3]), fmaf(b1, sm1, acc[3]));
+}
+
+// M = 2: S1 (W1, W3; 2 tiles x 8 slices of 64 code bytes); M = 1: S2 (W2; 4
+// tiles x 4 slices of 128 code bytes).  3-bit: slices of 48 / 96 bytes.
 template <int FMT, int M>
 MOE_DEV void dec_stage(const DecStageCtx& c, float (&acc)[2][4]) {
-  constexpr int KBW = DecA<FMT>::KB_PER_WARP;  // k-blocks of this warp in the stage
+  constexpr int BITS = DecA<FMT>::bits;
+  constexpr int WB = (FMT == F_A3 ? 48 : 64) * (M == 2 ? 1 : 2);  // code bytes of this warp per row
+  constexpr int KBW = WB * 8 / BITS / 32;                         // k-blocks of this warp
+  constexpr int KBB = 32 * BITS / 8;                              // code bytes per k-block and row
   constexpr bool MX = FMT == F_MX4;
-  constexpr int REC = MX ? 32 : 16;            // plane record bytes per (k-block, thread)
+  constexpr int REC = MX ? 32 : 16;  // plane record bytes per (k-block, thread)
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const bool live = g < c.ntok;
-  const int pstride = c.mat[0]->ks * plane_bytes_per_input(FMT) + (MX ? 16 : 64);
-  const uint32_t planes = c.slot + kDecSlotPlanes + (uint32_t)(live ? g : 0) * pstride;
-  const uint32_t sxb = c.slot + kDecSlotSx;
-  const int group = c.mat[0]->group;
-  const int kb0 = c.kq * KBW;                  // first k-block (within the stage) of this warp
-  const int r0 = c.rt * 16 + g, r1 = r0 + 8;
+  const int pstride = c.ks * plane_bytes_per_input(FMT) + (MX ? 16 : 64);
+  const uint32_t planes = c.slot + kDecSlotPlanes + (uint32_t)(live ? g : 0) * pstride + t * REC;
+  const int group = c.group;
+  const bool g32 = group == 32;  // 32-input groups: each k-block has its own scale
+  const int sbytes = c.ks / group * (MX ? 1 : 2);
+  const int kb0 = c.kq * KBW;    // first k-block (within the stage) of this warp
+  const int byte0 = c.kq * WB;   // first code byte (within the stage row) of this warp
 #pragma unroll
-  for (int blk = 0; blk < KBW / 2; ++blk) {    // 64-input blocks
-    const int kbs = kb0 + 2 * blk;             // stage k-block of the block's first half
-    const int bs = kbs >> 1;                   // stage block index
-    // activations of the two k-blocks
-    uint4 B[2], Bn[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      B[h] = live ? lds128u(planes + (kbs + h) * 4 * REC + t * REC) : make_uint4(0, 0, 0, 0);
-      if constexpr (MX) Bn[h] = live ? lds128u(planes + (kbs + h) * 4 * REC + t * REC + 16) : make_uint4(0, 0, 0, 0);
-    }
-    // (step, sums) of the block for this lane's two columns
-    const int c0 = 2 * t, c1 = 2 * t + 1;
-    const float4 x0 = c0 < c.ntok ? lds_f4(sxb + c0 * kDecSxStride + bs * 16) : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4 x1 = c1 < c.ntok ? lds_f4(sxb + c1 * kDecSxStride + bs * 16) : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int blk = 0; blk < KBW / 2; ++blk) {  // 64-input blocks
+    const int kbs = kb0 + 2 * blk;           // stage k-block of the block's first half
+    const int bs = kbs >> 1;                 // stage block index
+    const int byte = byte0 + 2 * blk * KBB;  // the block's first code byte
 #pragma unroll
     for (int m = 0; m < M; ++m) {
-      const uint32_t codes = c.slot + kDecSlotCodes + m * kDecCodeMat;
-      int ch[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}}, cl[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-      if constexpr (FMT == F_A4 || FMT == F_MX4) {
-        uint32_t w[4];
-        DecA<F_A4>::load2(codes, c.rt, c.kq, 2 * blk, w);
+      DecTile tl;
+      tl.codes = c.slot + kDecSlotCodes + m * 16384;
+      tl.rows = c.rows;
+      tl.rt = c.rt;
+      int ch[4] = {0, 0, 0, 0}, cl[4] = {0, 0, 0, 0};
+      uint32_t w[4];
+      if constexpr (FMT == F_A4 || FMT == F_MX4) dec_ldsm2(tl, byte, w);  // both k-blocks
+      if constexpr (FMT == F_A2) dec_ldsm1(tl, byte, w);                  // the block is one chunk
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t a[4], an[4];
-          if constexpr (FMT == F_A4) {
-            DecA<F_A4>::unpack(w[2 * h], w[2 * h + 1], a);
-          } else {
-            DecA<F_MX4>::unpack(w[2 * h], w[2 * h + 1], a, an);
-          }
-          const int hh = group == 32 ? h : 0;  // 32-input groups: keep the halves apart
-          mma_u8s8(ch[hh], a, B[h].x, B[h].y);
-          mma_u8u8(cl[hh], a, B[h].z, B[h].w);
-          if constexpr (MX) {
-            mma_u8s8(ch[hh], an, Bn[h].x, Bn[h].y);
-            mma_u8u8(cl[hh], an, Bn[h].z, Bn[h].w);
-          }
+      for (int h = 0; h < 2; ++h) {
+        const uint4 B = live ? lds128u(planes + (kbs + h) * 4 * REC) : make_uint4(0, 0, 0, 0);
+        uint32_t a[4];
+        if constexpr (FMT == F_A4) {
+          unpack_a4(w[2 * h], w[2 * h + 1], a);
+        } else if constexpr (FMT == F_MX4) {
+          uint32_t an[4];
+          unpack_mx4(w[2 * h], w[2 * h + 1], a, an);
+          const uint4 Bn = live ? lds128u(planes + (kbs + h) * 4 * REC + 16) : make_uint4(0, 0, 0, 0);
+          mma_u8s8(ch, an, Bn.x, Bn.y);
+          mma_u8u8(cl, an, Bn.z, Bn.w);
+        } else if constexpr (FMT == F_A8) {
+          dec_ldsm2(tl, byte + h * 32, a);  // one k-block = two chunks
+        } else if constexpr (FMT == F_A2) {
+          unpack_a2(w[0], w[1], h, a);
+        } else {
+          load_a3(tl, byte + h * KBB, a);
         }
-      } else if constexpr (FMT == F_A2) {
-        uint32_t wg, wg8;
-        {
-          // one chunk (64 codes) per block: rows g / g+8 of chunk (kq&1)*4 + blk
-          const int mtx = (lane >> 3) & 1;
-          const int row = c.rt * 16 + mtx * 8 + (lane & 7);
-          const int chunk = (c.kq & 1) * 4 + blk;
-          uint32_t d0, d1, d2, d3;
-          ldsm_x4(swz(codes + (c.kq >> 1) * 8192, row, chunk), d0, d1, d2, d3);
-          wg = d0;
-          wg8 = d1;
-          (void)d2;
-          (void)d3;
-        }
+        mma_u8s8(ch, a, B.x, B.y);
+        mma_u8u8(cl, a, B.z, B.w);
+        if (g32) {  // fold each 32-input group on its own
+          dec_fold<FMT>(c, m, kbs + h, sbytes, bs, 1 + h, ch, cl, acc[m]);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t a[4];
-          DecA<F_A2>::unpack(wg, wg8, h, a);
-          mma_u8s8(ch[0], a, B[h].x, B[h].y);
-          mma_u8u8(cl[0], a, B[h].z, B[h].w);
-        }
-      } else {  // F_A8, F_A3: one A load per k-block
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t a[4], an[4];
-          DecA<FMT>::load(codes, c.rt, c.kq, 2 * blk + h, a, an);
-          const int hh = group == 32 ? h : 0;
-          mma_u8s8(ch[hh], a, B[h].x, B[h].y);
-          mma_u8u8(cl[hh], a, B[h].z, B[h].w);
+          for (int q = 0; q < 4; ++q) ch[q] = cl[q] = 0;
         }
       }
-      // fold into fp32: acc += s * step * (256*hi + lo) + b * sum
-      const int nh = group == 32 ? 2 : 1;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (hh < nh) {
-          const int grp = group == 32 ? (kbs + hh) : (bs * 64) / group;
-          float s0, b0, s1, b1;
-          dec_scale_bias<FMT>(c, m, grp, r0, s0, b0);
-          dec_scale_bias<FMT>(c, m, grp, r1, s1, b1);
-          const float p00 = (float)(ch[hh][0] * 256 + cl[hh][0]), p01 = (float)(ch[hh][1] * 256 + cl[hh][1]);
-          const float p10 = (float)(ch[hh][2] * 256 + cl[hh][2]), p11 = (float)(ch[hh][3] * 256 + cl[hh][3]);
-          // bias term: the group's bias times the sum of the inputs it covers
-          const float xs0 = x0.x, xs1 = x1.x;
-          const float xm0 = group == 32 ? (hh ? x0.z : x0.y) : x0.w;
-          const float xm1 = group == 32 ? (hh ? x1.z : x1.y) : x1.w;
-          acc[m][0] = fmaf(s0 * xs0, p00, fmaf(b0, xm0, acc[m][0]));
-          acc[m][1] = fmaf(s0 * xs1, p01, fmaf(b0, xm1, acc[m][1]));
-          acc[m][2] = fmaf(s1 * xs0, p10, fmaf(b1, xm0, acc[m][2]));
-          acc[m][3] = fmaf(s1 * xs1, p11, fmaf(b1, xm1, acc[m][3]));
-        }
-      }
+      if (!g32) dec_fold<FMT>(c, m, (bs * 64) / group, sbytes, bs, 3, ch, cl, acc[m]);
     }
   }
 }
@@ -464,7 +447,8 @@ struct DecUnit {
   int mi;     // first matrix index (DecMatIdx)
   int M;      // matrices (2: W1 and W3; 1: W2)
   int row0;   // first weight row in the stacked matrix
-  int nchunks;
+  int nchunks;  // stages along the inputs
+  int nhalf;    // S1: the 64 rows come as two stages of 32 rows (per input chunk); S2: 1
 };
 
 MOE_DEV DecUnit dec_unit(const DecParams& p, const int4* groups, int nsg, int nrg, int i) {
@@ -497,6 +481,7 @@ MOE_DEV DecUnit dec_unit(const DecParams& p, const int4* groups, int nsg, int nr
     U.row0 = (sh ? 0 : groups[U.grp].x * p.d) + kDecRows * U.u;
   }
   U.nchunks = p.m[U.mi].n_in / p.m[U.mi].ks;
+  U.nhalf = U.stage == 1 ? 2 : 1;
   return U;
 }
 
@@ -536,7 +521,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
 
   if (tid == 0) {
     for (int s = 0; s < kDecStages; ++s) {
-      dec_bar_init(full0 + 8 * s, 33);
+      dec_bar_init(full0 + 8 * s, 1);  // the producer's expect_tx arrive; the copies complete the transactions
       dec_bar_init(empty0 + 8 * s, kDecConsumerWarps);
     }
     misc[0] = 0;
@@ -567,43 +552,45 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     if (!p.hash) {
       // router logits of experts blockIdx.x, +G, ... for every token (warps 0..15 split d)
       for (int e = blockIdx.x; e < E; e += p.G) {
-        float acc[kDecMaxT];
-#pragma unroll
-        for (int t = 0; t < kDecMaxT; ++t) acc[t] = 0.f;
         if (warp < kDecConsumerWarps) {
           const int span = d / kDecConsumerWarps;
-          for (int i = warp * span + lane * 8; i < (warp + 1) * span; i += 256) {
-            float wv[8];
-            if (p.router_bf16) {
-              const uint4 r = __ldg(reinterpret_cast<const uint4*>(
-                  reinterpret_cast<const __nv_bfloat16*>(p.router_w) + (size_t)e * d + i));
-              wv[0] = bf16lo(r.x); wv[1] = bf16hi(r.x); wv[2] = bf16lo(r.y); wv[3] = bf16hi(r.y);
-              wv[4] = bf16lo(r.z); wv[5] = bf16hi(r.z); wv[6] = bf16lo(r.w); wv[7] = bf16hi(r.w);
-            } else {
-              const float4* rr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.router_w) +
-                                                                 (size_t)e * d + i);
-              const float4 a = __ldg(rr), bq = __ldg(rr + 1);
-              wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
-              wv[4] = bq.x; wv[5] = bq.y; wv[6] = bq.z; wv[7] = bq.w;
-            }
+          for (int t0 = 0; t0 < T; t0 += 8) {  // tokens in groups of 8 (registers)
+            float acc[8];
 #pragma unroll
-            for (int t = 0; t < kDecMaxT; ++t) {
-              if (t < T) {
-                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)t * d + i));
-                float a = acc[t];
-                a = fmaf(wv[0], bf16lo(xv.x), a); a = fmaf(wv[1], bf16hi(xv.x), a);
-                a = fmaf(wv[2], bf16lo(xv.y), a); a = fmaf(wv[3], bf16hi(xv.y), a);
-                a = fmaf(wv[4], bf16lo(xv.z), a); a = fmaf(wv[5], bf16hi(xv.z), a);
-                a = fmaf(wv[6], bf16lo(xv.w), a); a = fmaf(wv[7], bf16hi(xv.w), a);
-                acc[t] = a;
+            for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+            for (int i = warp * span + lane * 8; i < (warp + 1) * span; i += 256) {
+              float wv[8];
+              if (p.router_bf16) {
+                const uint4 r = __ldg(reinterpret_cast<const uint4*>(
+                    reinterpret_cast<const __nv_bfloat16*>(p.router_w) + (size_t)e * d + i));
+                wv[0] = bf16lo(r.x); wv[1] = bf16hi(r.x); wv[2] = bf16lo(r.y); wv[3] = bf16hi(r.y);
+                wv[4] = bf16lo(r.z); wv[5] = bf16hi(r.z); wv[6] = bf16lo(r.w); wv[7] = bf16hi(r.w);
+              } else {
+                const float4* rr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.router_w) +
+                                                                   (size_t)e * d + i);
+                const float4 a = __ldg(rr), bq = __ldg(rr + 1);
+                wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
+                wv[4] = bq.x; wv[5] = bq.y; wv[6] = bq.z; wv[7] = bq.w;
+              }
+#pragma unroll
+              for (int t = 0; t < 8; ++t) {
+                if (t0 + t < T) {
+                  const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)(t0 + t) * d + i));
+                  float a = acc[t];
+                  a = fmaf(wv[0], bf16lo(xv.x), a); a = fmaf(wv[1], bf16hi(xv.x), a);
+                  a = fmaf(wv[2], bf16lo(xv.y), a); a = fmaf(wv[3], bf16hi(xv.y), a);
+                  a = fmaf(wv[4], bf16lo(xv.z), a); a = fmaf(wv[5], bf16hi(xv.z), a);
+                  a = fmaf(wv[6], bf16lo(xv.w), a); a = fmaf(wv[7], bf16hi(xv.w), a);
+                  acc[t] = a;
+                }
               }
             }
-          }
 #pragma unroll
-          for (int t = 0; t < kDecMaxT; ++t) {
-            if (t < T) {
-              const float v = warp_sum(acc[t]);
-              if (lane == 0) red[warp * kDecMaxT + t] = v;
+            for (int t = 0; t < 8; ++t) {
+              if (t0 + t < T) {
+                const float v = warp_sum(acc[t]);
+                if (lane == 0) red[warp * kDecMaxT + t0 + t] = v;
+              }
             }
           }
         }
@@ -636,42 +623,44 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
       }
       __syncthreads();
       if (p.router_w != nullptr && warp < kDecConsumerWarps) {
-        float acc[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) acc[j] = 0.f;
         const int span = d / kDecConsumerWarps;
-        for (int i = warp * span + lane * 8; i < (warp + 1) * span; i += 256) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)t * d + i));
-          const float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
-                               bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
+        for (int j0 = 0; j0 < k; j0 += 8) {  // the table's experts in groups of 8 (registers)
+          float acc[8];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (j < k) {
-              const size_t off = (size_t)s_e[j] * d + i;
-              float wv[8];
-              if (p.router_bf16) {
-                const uint4 r = __ldg(reinterpret_cast<const uint4*>(
-                    reinterpret_cast<const __nv_bfloat16*>(p.router_w) + off));
-                wv[0] = bf16lo(r.x); wv[1] = bf16hi(r.x); wv[2] = bf16lo(r.y); wv[3] = bf16hi(r.y);
-                wv[4] = bf16lo(r.z); wv[5] = bf16hi(r.z); wv[6] = bf16lo(r.w); wv[7] = bf16hi(r.w);
-              } else {
-                const float4* rr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.router_w) + off);
-                const float4 a = __ldg(rr), bq = __ldg(rr + 1);
-                wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
-                wv[4] = bq.x; wv[5] = bq.y; wv[6] = bq.z; wv[7] = bq.w;
+          for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+          for (int i = warp * span + lane * 8; i < (warp + 1) * span; i += 256) {
+            const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)t * d + i));
+            const float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
+                                 bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              if (j0 + j < k) {
+                const size_t off = (size_t)s_e[j0 + j] * d + i;
+                float wv[8];
+                if (p.router_bf16) {
+                  const uint4 r = __ldg(reinterpret_cast<const uint4*>(
+                      reinterpret_cast<const __nv_bfloat16*>(p.router_w) + off));
+                  wv[0] = bf16lo(r.x); wv[1] = bf16hi(r.x); wv[2] = bf16lo(r.y); wv[3] = bf16hi(r.y);
+                  wv[4] = bf16lo(r.z); wv[5] = bf16hi(r.z); wv[6] = bf16lo(r.w); wv[7] = bf16hi(r.w);
+                } else {
+                  const float4* rr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.router_w) + off);
+                  const float4 a = __ldg(rr), bq = __ldg(rr + 1);
+                  wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
+                  wv[4] = bq.x; wv[5] = bq.y; wv[6] = bq.z; wv[7] = bq.w;
+                }
+                float a = acc[j];
+#pragma unroll
+                for (int q = 0; q < 8; ++q) a = fmaf(wv[q], xf[q], a);
+                acc[j] = a;
               }
-              float a = acc[j];
-#pragma unroll
-              for (int q = 0; q < 8; ++q) a = fmaf(wv[q], xf[q], a);
-              acc[j] = a;
             }
           }
-        }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (j < k) {
-            const float v = warp_sum(acc[j]);
-            if (lane == 0) red[warp * 32 + j] = v;
+          for (int j = 0; j < 8; ++j) {
+            if (j0 + j < k) {
+              const float v = warp_sum(acc[j]);
+              if (lane == 0) red[warp * 32 + j0 + j] = v;
+            }
           }
         }
       }
@@ -749,81 +738,76 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
       const DecUnit U = dec_unit(p, R.groups, nsg, nrg, ui);
       const int4 grp = R.groups[U.grp];
       const DecMat& m0 = p.m[U.mi];
-      const int esz = m0.fmt == F_MX4 ? 1 : 2;
-      const int gps = m0.ks / m0.group;      // scale groups per stage and row
-      const int sbytes = gps * esz;          // scale bytes per stage and row
+      const bool mx = m0.fmt == F_MX4;
       const int pb = plane_bytes_per_input(m0.fmt);
-      const int pstride = m0.ks * pb + (m0.fmt == F_MX4 ? 16 : 64);
-      const int nbox = m0.stage_row / m0.box;
-      const uint32_t tx = (uint32_t)(U.M * nbox * kDecRows * m0.box + grp.z * (m0.ks * pb + (m0.ks / 64) * 16));
+      const int pstride = m0.ks * pb + (mx ? 16 : 64);
+      const uint32_t box_bytes = (uint32_t)(m0.rows * m0.box);
+      const uint32_t sc_bytes = (uint32_t)(m0.rows * m0.sbytes);
+      const uint32_t tx = (uint32_t)U.M * (4 * box_bytes + sc_bytes * (mx ? 1 : 2)) +
+                          (uint32_t)grp.z * (m0.ks * pb + (m0.ks / 64) * 16);
       bool dep_ok = U.stage == 1;
-      for (int kc = 0; kc < U.nchunks; ++kc, ++n) {
+      for (int st = 0; st < U.nhalf * U.nchunks; ++st, ++n) {
+        const int half = st / U.nchunks, kc = st % U.nchunks;
+        const int row0 = U.row0 + half * m0.rows;
         const int s = n % kDecStages;
         const uint32_t slot = su32(ring + (size_t)s * kDecSlotBytes);
         const uint32_t full = full0 + 8 * s, empty = empty0 + 8 * s;
-        if (lane == 0 && n >= kDecStages && !dec_wait_bar(empty, ((n / kDecStages) - 1) & 1, abort_flag)) {
-          set_error(p.err, kErrTimeout);
-          *abort_flag = 1;
+        if (lane == 0) {
+          if (n >= kDecStages && !dec_wait_bar(empty, ((n / kDecStages) - 1) & 1, abort_flag)) {
+            set_error(p.err, kErrTimeout);
+            *abort_flag = 1;
+          }
+          if (!*abort_flag) {
+            dec_expect_tx(full, tx);
+            for (int mm = 0; mm < U.M; ++mm) {
+              const int mi = U.mi + mm;
+              const uint32_t cbase = slot + kDecSlotCodes + mm * 16384;
+              for (int b = 0; b < 4; ++b)
+                dec_tma_2d(cbase + b * box_bytes, &p.map[mi], kc * 4 * m0.box + b * m0.box, row0, full);
+              const uint32_t sbase = slot + kDecSlotScales + mm * 4096;
+              const int sx = kc * (m0.ks / m0.group);  // first scale entry of the stage
+              dec_tma_2d(sbase, &p.smap[mi], sx, row0, full);
+              if (!mx) dec_tma_2d(sbase + m0.rows * kDecScaleRow, &p.bmap[mi], sx, row0, full);
+            }
+            if (!dep_ok) {
+              // W2 stages read the group's h planes: wait for all its S1 units.
+              // (On a timeout the plane copies below are still issued -- they
+              // stay in bounds -- so the stage's transaction count completes.)
+              const int target = p.stall_test ? 0x3fffffff : (grp.x < 0 ? p.fs / kDecRows : p.f / kDecRows);
+              if (!dec_wait_count(p.cnt_h + U.grp, target, abort_flag, p.stall_test ? 2000000LL : kDecWaitCycles)) {
+                set_error(p.err, kErrTimeout);
+                *abort_flag = 1;
+              }
+              fence_proxy_async_global();
+              dep_ok = true;
+            }
+            for (int i = 0; i < grp.z; ++i) {
+              const uint8_t* src;
+              const float4* ssrc;
+              if (U.stage == 1) {
+                const int tok = dec_token(p, R, grp, i);
+                const int layout = grp.x < 0 ? 1 : 0;
+                src = p.xplanes + ((size_t)layout * T + tok) * d * 4;
+                ssrc = p.xsx + (size_t)tok * (d / 64);
+              } else {
+                const int sl = dec_slot(p, R, grp, i);
+                src = p.hplanes + (size_t)sl * fmax * 4;
+                ssrc = p.hsx + (size_t)sl * (fmax / 64);
+              }
+              dec_bulk(slot + kDecSlotPlanes + i * pstride, src + (size_t)kc * m0.ks * pb, m0.ks * pb, full);
+              dec_bulk(slot + kDecSlotSx + i * kDecSxStride, ssrc + (size_t)kc * (m0.ks / 64), (m0.ks / 64) * 16,
+                       full);
+            }
+          }
         }
         __syncwarp();
         if (*abort_flag) {
           ok = false;
           break;
         }
-        if (lane == 0) {
-          dec_expect_tx(full, tx);
-          for (int mm = 0; mm < U.M; ++mm)
-            for (int b = 0; b < nbox; ++b)
-              dec_tma_2d(slot + kDecSlotCodes + mm * kDecCodeMat + b * (kDecRows * m0.box), &p.map[U.mi + mm],
-                         kc * m0.stage_row + b * m0.box, U.row0, full);
-        }
-        // scales and biases: lanes take rows lane and lane + 32
-        for (int mm = 0; mm < U.M; ++mm) {
-          const DecMat& mt = p.m[U.mi + mm];
-          for (int rr = lane; rr < kDecRows; rr += 32) {
-            const size_t src = ((size_t)(U.row0 + rr) * mt.gpr + (size_t)kc * gps) * esz;
-            const uint32_t dst = slot + kDecSlotScales + mm * kDecScaleMat + rr * 32;
-            for (int o = 0; o < sbytes; o += 16) {
-              const int nbytes = min(16, sbytes - o);
-              dec_cp_async(dst + o, reinterpret_cast<const uint8_t*>(mt.scales) + src + o, nbytes);
-              if (mt.fmt != F_MX4)
-                dec_cp_async(dst + 2048 + o, reinterpret_cast<const uint8_t*>(mt.biases) + src + o, nbytes);
-            }
-          }
-        }
-        if (lane == 0) {
-          if (!dep_ok) {
-            // W2 stages read the group's h planes: wait for all its S1 units
-            const int target = grp.x < 0 ? p.fs / kDecRows : p.f / kDecRows;
-            if (!dec_wait_count(p.cnt_h + U.grp, target, abort_flag)) {
-              set_error(p.err, kErrTimeout);
-              *abort_flag = 1;
-            }
-            fence_proxy_async_global();
-            dep_ok = true;
-          }
-          for (int i = 0; i < grp.z; ++i) {
-            const uint8_t* src;
-            const float4* ssrc;
-            if (U.stage == 1) {
-              const int tok = dec_token(p, R, grp, i);
-              const int layout = grp.x < 0 ? 1 : 0;
-              src = p.xplanes + ((size_t)layout * T + tok) * d * 4;
-              ssrc = p.xsx + (size_t)tok * (d / 64);
-            } else {
-              const int sl = dec_slot(p, R, grp, i);
-              src = p.hplanes + (size_t)sl * fmax * 4;
-              ssrc = p.hsx + (size_t)sl * (fmax / 64);
-            }
-            dec_bulk(slot + kDecSlotPlanes + i * pstride, src + (size_t)kc * m0.ks * pb, m0.ks * pb, full);
-            dec_bulk(slot + kDecSlotSx + i * kDecSxStride, ssrc + (size_t)kc * (m0.ks / 64), (m0.ks / 64) * 16, full);
-          }
-        }
-        dec_cp_async_arrive(full);
       }
     }
     // drain: every issued copy must land before the block exits
-    asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0) {
       for (int q = max(0, n - kDecStages); q < n; ++q) {
         const uint32_t full = full0 + 8 * (q % kDecStages);
@@ -834,65 +818,70 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     }
   } else {
     // ============================================================ consumers
-    const int rt = warp & 3, kq = warp >> 2;
     const int g = lane >> 2, t4 = lane & 3;
     int n = 0;
     for (int ui = blockIdx.x; ui < n_units; ui += p.G) {
       const DecUnit U = dec_unit(p, R.groups, nsg, nrg, ui);
       const int4 grp = R.groups[U.grp];
+      const DecMat& m0 = p.m[U.mi];
       DecStageCtx c;
-      c.rt = rt;
-      c.kq = kq;
+      // S1: 2 row tiles x 8 input slices; S2: 4 row tiles x 4 input slices
+      c.rt = U.M == 2 ? (warp & 1) : (warp & 3);
+      c.kq = U.M == 2 ? (warp >> 1) : (warp >> 2);
       c.ntok = grp.z;
-      c.mat[0] = &p.m[U.mi];
-      c.mat[1] = &p.m[U.mi + (U.M > 1 ? 1 : 0)];
-      const int fmt = p.m[U.mi].fmt;
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      for (int kc = 0; kc < U.nchunks; ++kc, ++n) {
-        const int s = n % kDecStages;
-        const uint32_t full = full0 + 8 * s;
-        bool have = !*abort_flag;
-        if (have && !dec_wait_bar(full, (n / kDecStages) & 1, abort_flag)) {
-          set_error(p.err, kErrTimeout);
-          *abort_flag = 1;
-          have = false;
+      c.group = m0.group;
+      c.ks = m0.ks;
+      c.rows = m0.rows;
+      const int fmt = m0.fmt;
+      for (int half = 0; half < U.nhalf; ++half) {
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        for (int kc = 0; kc < U.nchunks; ++kc, ++n) {
+          const int s = n % kDecStages;
+          const uint32_t full = full0 + 8 * s;
+          bool have = !*abort_flag;
+          if (have && !dec_wait_bar(full, (n / kDecStages) & 1, abort_flag)) {
+            set_error(p.err, kErrTimeout);
+            *abort_flag = 1;
+            have = false;
+          }
+          have = __all_sync(0xffffffffu, have);  // the MMAs below need every lane
+          if (have) {
+            c.slot = su32(ring + (size_t)s * kDecSlotBytes);
+            dec_stage_any(fmt, U.M, c, acc);
+          }
+          __syncwarp();
+          if (lane == 0 && have) dec_arrive(empty0 + 8 * s);
         }
-        have = __all_sync(0xffffffffu, have);  // the MMAs below need every lane
-        if (have) {
-          c.slot = su32(ring + (size_t)s * kDecSlotBytes);
-          dec_stage_any(fmt, U.M, c, acc);
-        }
-        __syncwarp();
-        if (lane == 0 && have) dec_arrive(empty0 + 8 * s);
-      }
-      // ---- unit end: sum the four input quarters of every (row, token)
+        // ---- sum the input slices of every (row, token) of this half
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        if (m < U.M) {
-          float* dst = red + ((warp * 2 + m) * 16) * 8;
-          dst[g * 8 + 2 * t4] = acc[m][0];
-          dst[g * 8 + 2 * t4 + 1] = acc[m][1];
-          dst[(g + 8) * 8 + 2 * t4] = acc[m][2];
-          dst[(g + 8) * 8 + 2 * t4 + 1] = acc[m][3];
-        }
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
-      {
-        const int row = tid >> 3, tok = tid & 7;  // tid < 512: 64 rows x 8 tokens
-        const int rtt = row >> 4, rl = row & 15;
-        if (tok < grp.z) {
-          float v[2] = {0.f, 0.f};
-          for (int q = 0; q < 4; ++q)
-            for (int m = 0; m < U.M; ++m) v[m] += red[(((q * 4 + rtt) * 2 + m) * 16 + rl) * 8 + tok];
-          if (U.stage == 1) {
-            hbuf[tok * kDecRows + row] = v[0] / (1.f + expf(-v[0])) * v[1];  // silu(g) * u
-          } else {
-            const int sl = dec_slot(p, R, grp, tok);
-            p.y[(size_t)sl * d + kDecRows * U.u + row] = v[0];
+        for (int m = 0; m < 2; ++m) {
+          if (m < U.M) {
+            float* dst = red + ((warp * 2 + m) * 16) * 8;
+            dst[g * 8 + 2 * t4] = acc[m][0];
+            dst[g * 8 + 2 * t4 + 1] = acc[m][1];
+            dst[(g + 8) * 8 + 2 * t4] = acc[m][2];
+            dst[(g + 8) * 8 + 2 * t4 + 1] = acc[m][3];
           }
         }
+        asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
+        {
+          const int nrt = U.M == 2 ? 2 : 4, nkq = kDecConsumerWarps / nrt;
+          const int row = tid >> 3, tok = tid & 7;  // S1: rows 0..31 (tid < 256); S2: rows 0..63
+          if (row < nrt * 16 && tok < grp.z) {
+            const int rtt = row >> 4, rl = row & 15;
+            float v[2] = {0.f, 0.f};
+            for (int q = 0; q < nkq; ++q)
+              for (int m = 0; m < U.M; ++m) v[m] += red[(((q * nrt + rtt) * 2 + m) * 16 + rl) * 8 + tok];
+            if (U.stage == 1) {
+              hbuf[tok * kDecRows + half * 32 + row] = v[0] / (1.f + expf(-v[0])) * v[1];  // silu(g) * u
+            } else {
+              const int sl = dec_slot(p, R, grp, tok);
+              p.y[(size_t)sl * d + kDecRows * U.u + row] = v[0];
+            }
+          }
+        }
+        asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
       }
-      asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
       if (U.stage == 1) {
         // h of each token over these 64 rows -> one 64-input block of W2's planes
         if (warp < grp.z) {
@@ -923,10 +912,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
           // every slot of this 64-column block is final: out = sum_j w y (+ shared), one rounding
           for (int i = tid; i < T * kDecRows; i += kDecConsumerWarps * 32) {
             const int t = i / kDecRows, col = kDecRows * U.u + (i % kDecRows);
-            float s = 0.f;
-            for (int j = 0; j < k; ++j) s = fmaf(R.w[t * k + j], __ldcg(p.y + (size_t)(t * k + j) * d + col), s);
-            if (p.has_shared) s += __ldcg(p.y + (size_t)(Tk + t) * d + col);
-            p.out[(size_t)t * d + col] = __float2bfloat16_rn(s);
+            float sacc = 0.f;
+            for (int j = 0; j < k; ++j) sacc = fmaf(R.w[t * k + j], __ldcg(p.y + (size_t)(t * k + j) * d + col), sacc);
+            if (p.has_shared) sacc += __ldcg(p.y + (size_t)(Tk + t) * d + col);
+            p.out[(size_t)t * d + col] = __float2bfloat16_rn(sacc);
           }
           asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
           if (tid == 0) p.cnt_y[U.u] = 0;

@@ -494,6 +494,10 @@ const TcLaunchFn kTcLaunch[2][5] = {
 const TcAttrFn kTcAttrs[10] = {attrs_tc_s1_A2, attrs_tc_s1_A3, attrs_tc_s1_A4, attrs_tc_s1_A8, attrs_tc_s1_MX4,
                                attrs_tc_s2_A2, attrs_tc_s2_A3, attrs_tc_s2_A4, attrs_tc_s2_A8, attrs_tc_s2_MX4};
 
+// Test hook of the calling thread (moe_test_stall_fused_wait): the next fused
+// launches wait on a dependency count that nothing completes.
+thread_local int g_stall_test = 0;
+
 // Expert-FFN implementation choice of the calling thread (moe_set_ffn_path):
 // one thread's setting never changes another thread's calls.
 thread_local int g_ffn_path = MOE_FFN_AUTO;
@@ -801,30 +805,24 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
 }
 
 // ---------------------------------------------------------------- fused small-batch layer
-// Stage geometry of a packed matrix in the fused kernel: inputs per stage
-// (256 code bytes per row; 3-bit: 192), TMA box width.
-bool dec_mat(const QMatDev& Q, DecMat* m) {
-  m->scales = Q.scales;
-  m->biases = Q.biases;
+// Stage geometry of a packed matrix in the fused kernel: 512 code bytes per
+// row and stage (3-bit: 384) as four 128-byte swizzled (3-bit: 96-byte
+// unswizzled) TMA boxes; W1/W3 stages carry 32 rows, W2 stages 64.
+bool dec_mat(const QMatDev& Q, bool w2, DecMat* m) {
   m->fmt = Q.fmt;
   m->group = Q.group;
   m->n_out = Q.n_out;
   m->n_in = Q.n_in;
-  m->gpr = Q.gpr;
-  switch (Q.fmt) {
-    case F_A2: m->ks = 1024; break;
-    case F_A8: m->ks = 256; break;
-    default: m->ks = 512; break;
-  }
-  m->stage_row = Q.fmt == F_A3 ? 192 : 256;
+  m->rows = w2 ? 64 : 32;
   m->box = Q.fmt == F_A3 ? 96 : 128;
-  if (Q.n_in % m->ks || Q.n_out % kDecRows || Q.group > m->ks) return false;
-  if (Q.fmt == F_A2 && Q.group == 32) return false;  // a 2-bit k-block mixes two 32-input groups
+  const int bits = Q.fmt == F_A2 ? 2 : Q.fmt == F_A3 ? 3 : Q.fmt == F_A8 ? 8 : 4;
+  m->ks = 4 * m->box * 8 / bits;
   const int esz = Q.fmt == F_MX4 ? 1 : 2;
-  const int sbytes = m->ks / Q.group * esz;
-  if (sbytes > 32 || sbytes < 4) return false;
-  if ((Q.gpr * esz) % std::min(16, sbytes)) return false;  // cp.async source alignment
-  if ((Q.wpr * 4) % 16) return false;                         // TMA row stride
+  m->sbytes = m->ks / Q.group * esz;
+  if (Q.n_in % m->ks || Q.n_out % 64) return false;
+  if (Q.fmt == F_A2 && Q.group == 32) return false;  // a 2-bit k-block mixes two 32-input groups
+  if (m->sbytes != 16 && m->sbytes != 32 && m->sbytes != 64) return false;  // TMA box of scales
+  if ((Q.gpr * esz) % 16 || (Q.wpr * 4) % 16) return false;                 // TMA row strides
   return true;
 }
 
@@ -833,8 +831,8 @@ bool dec_eligible(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, con
   // d_model a multiple of 128: the logit pass gives each lane 8 consecutive inputs of a 1/16 slice
   if (d.d_model % 128 || d.d_ff % 64 || (sh && d.d_ff_shared % 64)) return false;
   DecMat m;
-  if (!dec_mat(w1, &m) || !dec_mat(w3, &m) || !dec_mat(w2, &m)) return false;
-  if (sh && (!dec_mat(sh[0], &m) || !dec_mat(sh[1], &m) || !dec_mat(sh[2], &m))) return false;
+  if (!dec_mat(w1, false, &m) || !dec_mat(w3, false, &m) || !dec_mat(w2, true, &m)) return false;
+  if (sh && (!dec_mat(sh[0], false, &m) || !dec_mat(sh[1], false, &m) || !dec_mat(sh[2], true, &m))) return false;
   return true;
 }
 
@@ -844,9 +842,19 @@ bool use_dec(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, const QM
   return dec_eligible(d, w1, w3, w2, sh);
 }
 
-moe_status_t dec_code_map(CUtensorMap* map, const QMatDev& Q, int E, const DecMat& m) {
-  return tmap_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.q, (uint64_t)Q.wpr * 4, (uint64_t)E * Q.n_out,
-                 (uint64_t)Q.wpr * 4, m.box, kDecRows, Q.fmt != F_A3);
+moe_status_t dec_maps(DecParams& p, int i, const QMatDev& Q, int E) {
+  const DecMat& m = p.m[i];
+  const uint64_t rows = (uint64_t)E * Q.n_out;
+  moe_status_t st = tmap_2d(&p.map[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.q, (uint64_t)Q.wpr * 4, rows,
+                            (uint64_t)Q.wpr * 4, m.box, m.rows, Q.fmt != F_A3);
+  if (st != MOE_OK) return st;
+  if (Q.fmt == F_MX4)
+    return tmap_2d(&p.smap[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.scales, Q.gpr, rows, Q.gpr, m.sbytes, m.rows, false);
+  st = tmap_2d(&p.smap[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q.scales, Q.gpr, rows, (uint64_t)Q.gpr * 2, m.sbytes / 2,
+               m.rows, false);
+  if (st != MOE_OK) return st;
+  return tmap_2d(&p.bmap[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q.biases, Q.gpr, rows, (uint64_t)Q.gpr * 2,
+                 m.sbytes / 2, m.rows, false);
 }
 
 moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32_t* token_ids, const void* router_w,
@@ -856,8 +864,8 @@ moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32
   DecParams p{};
   const QMatDev* mats[6] = {&q1, &q3, &q2, qs ? &qs[0] : &q1, qs ? &qs[1] : &q3, qs ? &qs[2] : &q2};
   for (int i = 0; i < 6; ++i) {
-    dec_mat(*mats[i], &p.m[i]);
-    moe_status_t st = dec_code_map(&p.map[i], *mats[i], (i < 3 || !qs) ? d.n_experts : 1, p.m[i]);
+    dec_mat(*mats[i], i % 3 == 2, &p.m[i]);
+    moe_status_t st = dec_maps(p, i, *mats[i], (i < 3 || !qs) ? d.n_experts : 1);
     if (st != MOE_OK) return st;
   }
   p.x = reinterpret_cast<const __nv_bfloat16*>(x);
@@ -890,6 +898,7 @@ moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.ids_out = ids_out;
   p.w_out = w_out;
+  p.stall_test = g_stall_test;
   p.G = di.dec_blocks;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the kernel's CTAs wait on one another
@@ -1367,4 +1376,10 @@ extern "C" moe_status_t moe_hc_sinkhorn_mix(int32_t T, int32_t n, int32_t d, int
   }
   MOE_CHECK_LAUNCH("hc_sinkhorn_mix_kernel");
   return MOE_OK;
+}
+
+extern "C" int32_t moe_test_stall_fused_wait(int32_t enable) {
+  const int prev = g_stall_test;
+  g_stall_test = enable ? 1 : 0;
+  return prev;
 }

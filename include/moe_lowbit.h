@@ -342,6 +342,18 @@ typedef enum {
 } moe_ffn_path_t;
 int32_t moe_set_ffn_path(int32_t path);
 
+/*
+ * Testing aid for the bounded device-side waits (no counterpart on the
+ * pages).  While enabled on the calling thread, the fused small-batch launch
+ * makes its W2 stages wait on a dependency count that nothing completes,
+ * with a ~1 ms limit instead of ~2 s: the launch then records
+ * MOE_ERR_TIMEOUT in the workspace error word, lets its in-flight copies
+ * land, resets its counters and returns; the output is not valid.  A later
+ * call with the hook disabled runs normally on the same workspace.  Returns
+ * the previous setting.  Not for production use.
+ */
+int32_t moe_test_stall_fused_wait(int32_t enable);
+
 /* Static description of a status code. */
 const char* moe_status_string(moe_status_t status);
 

@@ -1,9 +1,10 @@
 """The fused small-batch layer (one launch: routing, both FFN stages on the
 integer tensor-core MMA, combine) against the oracle, with the path forced,
 over every packed format and group size it takes, hash routing, experts
-with more than 8 tokens (several token groups), the shared expert, bf16
+with more than 4 tokens (several token groups), the shared expert, bf16
 router weights and a pruned expert count; plus run-to-run determinism, the
-AUTO choice and the error word on bad hash data."""
+AUTO choice, the bounded-wait timeout and the error word on bad hash
+data."""
 import numpy as np
 import pytest
 import torch
@@ -25,19 +26,20 @@ VARIANTS = {
     "a4g128_T8": dict(B, T=8, w13=("affine", 4, 128), w2=("affine", 4, 128), seed=804),
     "a8g64_T3": dict(B, T=3, w13=("affine", 8, 64), w2=("affine", 8, 64), seed=805),
     "a8g32_T2": dict(B, T=2, w13=("affine", 8, 32), w2=("affine", 8, 32), seed=806),
-    "a8g128_T2": dict(B, T=2, w13=("affine", 8, 128), w2=("affine", 8, 128), seed=807),
-    "a2g128_a3g128_T8": dict(B, T=8, w13=("affine", 2, 128), w2=("affine", 3, 128), seed=808),
-    "a2g64_T4": dict(B, T=4, w13=("affine", 2, 64), w2=("affine", 2, 64), seed=809),
+    "a8_shared_g128_T2": dict(B, T=2, shared=("affine", 8, 64), f_shared=512, seed=807),
+    "a2g128_a3g128_T8": dict(B, T=8, d=2048, w13=("affine", 2, 128), w2=("affine", 3, 128), seed=808),
+    "a2g64_T4": dict(B, T=4, d=2048, f=2048, w13=("affine", 2, 64), w2=("affine", 2, 64), seed=809),
     "a3g64_T6": dict(B, T=6, w13=("affine", 3, 64), w2=("affine", 3, 64), seed=810),
     "mxfp4_hash_T32": dict(B, T=32, E=32, k=8, routing="hash", vocab=500, w13=("mxfp4", 4, 32),
                            w2=("mxfp4", 4, 32), seed=811),
     "mxfp4_learned_T9": dict(B, T=9, w13=("mxfp4", 4, 32), w2=("mxfp4", 4, 32), seed=812),
     "groups_over_8_tokens": dict(B, T=32, E=4, k=2, seed=813),
     "shared_narrower_T12": dict(B, T=12, shared=("affine", 8, 64), f_shared=512, seed=814),
+    "tokens_4_per_group_T24": dict(B, T=24, E=8, k=2, seed=820),
     "shared_a4_T9": dict(B, T=9, shared=("affine", 4, 64), f_shared=1024, seed=815),
     "bf16_router_T7": dict(B, T=7, router_dtype="bf16", seed=816),
     "E161_k8_T20": dict(B, T=20, E=161, k=8, seed=817),
-    "d2048_f512_T32": dict(B, T=32, d=2048, f=512, E=64, k=8, seed=818),
+    "d2048_f1024_T32": dict(B, T=32, d=2048, f=1024, E=64, k=8, seed=818),
     "hash_shared_T16": dict(B, T=16, E=32, k=8, routing="hash", vocab=300, shared=("affine", 8, 64),
                             f_shared=1024, seed=819),
 }
@@ -104,3 +106,21 @@ def test_fused_bad_hash_data_sets_error_word(fused):
     from tests.gpu_utils import bf16_to_np, check_output
     check_output(bf16_to_np(out)[keep], good["out"][keep], "bad hash token")
     assert torch.all(out[3] == 0)
+
+
+def test_bounded_wait_times_out_and_recovers(fused):
+    """A wait that nothing completes (the test hook) gives up within its short
+    limit: the call reports MOE_ERR_TIMEOUT through the error word, the
+    context stays usable and the next call on the same workspace is right."""
+    inp = make_custom(VARIANTS["a4g64_shared8_T1"], fused)
+    lib = moe.load_library()
+    prev = lib.moe_test_stall_fused_wait(1)
+    try:
+        _, _, _, ws = run_forward(inp)
+        assert moe.read_device_error(ws) == 5
+    finally:
+        lib.moe_test_stall_fused_wait(prev)
+    out, ids, w, _ = run_forward(inp, ws=ws)
+    res = oracle_run(inp)
+    check_layer(inp, res, out, ids, w, "after a timed-out call")
+    assert moe.read_device_error(ws) == 0
