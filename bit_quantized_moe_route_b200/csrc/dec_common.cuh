@@ -1,23 +1,23 @@
 // Building blocks of the fused decode kernel (ffn_decode.cuh): legacy
 // tensor-core integer MMA and ldmatrix wrappers, the fixed-point activation
-// planes, TMA / bulk-copy / cp.async issue helpers and a bounded grid-wide
-// barrier.
+// planes, TMA / bulk-copy issue helpers and bounded waits.
 //
 // Activation planes.  The expert contraction runs on the int8 tensor-core
-// path (mma.sync m16n8k32): weights are the A operand as unsigned code bytes
-// (or e2m1 magnitudes), activations the B operand.  An activation row (x for
-// W1/W3, the SwiGLU hidden row h for W2) is cut into blocks of 64 inputs;
-// each block is held as a 16-bit fixed-point vector xq = rint(v * 2^(141-E))
-// (E: largest fp32 exponent field in the block, so |xq| < 2^15) split into a
-// signed high byte plane and an unsigned low byte plane, together with the
-// block's step xs = 2^(E-141) and its dequantised sum xsum = xs * sum(xq).
-// For every 32-input k-block and quad thread t the planes are stored as the
-// 16 bytes {hi b0, hi b1, lo b0, lo b1} that thread t passes as its B
-// fragment (b0: k-slots 4t..4t+3, b1: k-slots 16+4t..16+4t+3); which inputs
-// sit in those k-slots depends on how the weight format's codes reach the A
-// fragment (the "permutation" of the consuming format, see plane_input).
-// mxfp4 weights add the planes of -v (32 bytes per k-block and thread):
-// positive and negative e2m1 codes become two unsigned A operands.
+// path (mma.sync m16n8k32, unsigned A x signed B): weights are the A operand
+// as unsigned code bytes (or e2m1 magnitudes), activations the B operand.
+// An activation row (x for W1/W3, the SwiGLU hidden row h for W2) is cut
+// into blocks of 64 inputs; each block is held as a fixed-point vector
+// xq = rint(v * 2^(140-E)) (E: largest fp32 exponent field in the block, so
+// |xq| <= 2^14) split as xq = 256 * hi + lo with lo the sign-extended low
+// byte (both planes signed bytes, |hi| <= 64), together with the block's
+// step xs = 2^(E-140) and its dequantised sums xs * sum(xq).  For every
+// 32-input k-block and quad thread t the planes are stored as the 16 bytes
+// {hi b0, hi b1, lo b0, lo b1}, b0 holding k-slots 4t..4t+3 and b1 k-slots
+// 16+4t..16+4t+3; which inputs sit in those k-slots depends on how the
+// weight format's codes reach the A fragment (the "permutation" of the
+// consuming format, see plane_input).  The MMA takes token j's hi plane as
+// B column 2j and its lo plane as column 2j+1, so one MMA gives a thread
+// both halves of its (row, token) sum: 256 * C[., 2j] + C[., 2j+1].
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -39,7 +39,7 @@ enum PlanePerm : int {
 MOE_DEV int perm_of(int fmt) {
   return fmt == F_A8 ? PERM_NATURAL : fmt == F_A4 ? PERM_EVENODD : fmt == F_A2 ? PERM_2BIT : PERM_HALVES;
 }
-__host__ __device__ inline int plane_bytes_per_input(int fmt) { return fmt == F_MX4 ? 4 : 2; }
+__host__ __device__ inline int plane_bytes_per_input(int) { return 2; }
 
 // Input index (within a 64-input block) of byte j of half h of quad thread
 // t's B fragment, for k-block kb2 (0 or 1) of the block.
@@ -60,12 +60,6 @@ MOE_DEV void mma_u8s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-MOE_DEV void mma_u8u8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 // four 8x(16 bytes) matrices; lane i gives the row address of matrix i/8,
 // row i%8; lane (g, t) receives bytes 4t..4t+3 of row g of each matrix
 MOE_DEV void ldsm_x4(uint32_t addr, uint32_t& d0, uint32_t& d1, uint32_t& d2, uint32_t& d3) {
@@ -76,6 +70,11 @@ MOE_DEV void ldsm_x4(uint32_t addr, uint32_t& d0, uint32_t& d1, uint32_t& d2, ui
 MOE_DEV uint4 lds128u(uint32_t a) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+MOE_DEV uint2 lds64u(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
   return v;
 }
 MOE_DEV uint32_t lds32u(uint32_t a) {
@@ -118,6 +117,13 @@ MOE_DEV void dec_tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+MOE_DEV void dec_tma_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
 MOE_DEV void dec_bulk(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
@@ -135,25 +141,11 @@ MOE_DEV void dec_bar_init(uint32_t bar, uint32_t n) {
 MOE_DEV bool dec_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(20000)
+      : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
-}
-// cp.async of 4/8/16 bytes (global -> shared), tracked by the issuing thread
-MOE_DEV void dec_cp_async(uint32_t dst, const void* src, int bytes) {
-  if (bytes == 16)
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-  else if (bytes == 8)
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
-  else
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-// the thread's cp.asyncs so far arrive on `bar` when complete (counted in
-// the barrier's expected arrivals)
-MOE_DEV void dec_cp_async_arrive(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 MOE_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
@@ -194,10 +186,10 @@ MOE_DEV bool dec_wait_bar(uint32_t bar, uint32_t parity, const volatile int* abo
 
 // ------------------------------------------------------------ fixed point
 // Step of a block whose largest magnitude has fp32 exponent field emax:
-// values map to |xq| < 2^15.  Returns (scale_up, step); zero for tiny blocks.
+// values map to |xq| <= 2^14.  Returns (scale_up, step); zero for tiny blocks.
 MOE_DEV float2 fix_scales(uint32_t emax) {
   if (emax >= 14 && emax < 255)
-    return make_float2(__uint_as_float((268u - emax) << 23), __uint_as_float((emax - 14u) << 23));
+    return make_float2(__uint_as_float((267u - emax) << 23), __uint_as_float((emax - 13u) << 23));
   return make_float2(0.f, 0.f);
 }
 

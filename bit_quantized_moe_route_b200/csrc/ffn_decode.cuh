@@ -12,9 +12,10 @@
 //       table row and weights of one token (hash), and the fixed-point planes
 //       of a slice of the activation blocks (dec_common.cuh);
 //       grid barrier (bounded);
-//   P1  every CTA, redundantly: top-k of every token, the stable grouping of
-//       the (token, slot) pairs by expert, and "groups" of <= 8 tokens of one
-//       expert (the shared expert's tokens form their own groups);
+//   P1  every CTA, redundantly: top-k of every token (one warp per token),
+//       per-expert counts, offsets and "groups" of <= ntmax (<= 4) tokens of one expert
+//       (one warp scan; the shared expert's tokens form their own groups),
+//       the stable (token, slot) order within each expert (warp match);
 //   S1  units (group, 64 rows of d_ff): h = silu(W1 x) * (W3 x) for the
 //       group's tokens, written as the planes W2 reads; a per-group counter
 //       counts finished units;
@@ -23,19 +24,25 @@
 //       of an output row block sums the k slots of every token in ascending
 //       j, adds the shared expert and writes bf16 (one rounding).
 // Units are dealt round-robin over the CTAs in the order [S1 shared, S1
-// routed, S2 by group], so every CTA does the same amount of streaming.
+// routed, S2 by group].
 //
-// Inside a CTA one producer warp streams each unit's weights into a 3-slot
-// ring, one stage = 512 code bytes of each of 32 rows of W1 and of W3 (S1;
-// a unit's 64 rows are two halves) or of 64 rows of W2 (S2), as 128-byte
-// wide TMA boxes with the 128-byte swizzle (3-bit: 96-byte unswizzled
-// boxes), plus the rows' scales and biases (TMA) and the activation planes
-// of the group's tokens (bulk copies).  Per-row runs of 512 bytes keep the
-// weight stream near the copy rate (narrower runs cost DRAM and TMA
-// efficiency).  16 consumer warps, one per (16-row tile, slice of the
-// stage's inputs), unpack codes to bytes, run m16n8k32 integer MMAs against
-// the planes (exact int32 sums per 64-input block) and fold each block into
-// fp32 with the weight scale and bias.
+// Weight stream.  One producer warp fills a ring of 32 KB stages; a stage is
+// a set of WHOLE row segments: 16 rows of W1 and the same 16 rows of W3 (S1)
+// or 32 rows of W2 (S2), each row contributing up to 1024 contiguous code
+// bytes (768 for 3-bit).  Each matrix's segment arrives as ONE 3-D TMA box
+// over a chunk-major view of the packed rows (dims: 128-byte line, row,
+// line index within the row), so the box lands as [line][row][128 B] with the
+// 128-byte swizzle keyed on the row: the 8 rows an ldmatrix phase reads sit in
+// distinct banks, and DRAM sees 16 or 32 runs of 1 KB per box.  The scales
+// and biases of those rows come as 2-D boxes.  The activation planes of the
+// unit's tokens for the stage's inputs go to one of two plane buffers (bulk
+// copies), loaded once per input chunk and shared by the chunk's 4 (S1) or 2
+// (S2) row sets.  Eight consumer warps = 2 row tiles x 4 input slices: a S1
+// tile is 8 rows of W1 stacked on the same 8 rows of W3 (so one thread holds
+// both halves of its SwiGLU pair), a S2 tile 16 rows of W2.  They unpack
+// codes to bytes, run m16n8k32 integer MMAs against the planes (exact int32
+// sums per 64-input block) and fold each block into fp32 with the weight
+// scale and bias; the slices are summed in a fixed order at the unit's end.
 // Every wait is bounded: on timeout the kernel records MOE_ERR_TIMEOUT, keeps
 // every warp's barrier sequence, lets in-flight copies land and returns.
 #pragma once
@@ -46,45 +53,64 @@
 namespace moe {
 
 constexpr int kDecConsumerWarps = 16;
-constexpr int kDecThreads = (kDecConsumerWarps + 1) * 32;
-constexpr int kDecStages = 3;
-constexpr int kDecRows = 64;        // weight rows per unit (S1: two halves of 32)
-constexpr int kDecMaxTok = 4;       // tokens per group (B columns 0..3 of the MMA)
+constexpr int kDecNkq = kDecConsumerWarps / 2;      // input slices (2 row tiles x 8 slices)
+constexpr int kDecProducerWarp = kDecConsumerWarps;
+constexpr int kDecServiceWarp = kDecConsumerWarps + 1;
+constexpr int kDecWarps = kDecConsumerWarps + 2;
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kDecConsumerThreads = kDecConsumerWarps * 32;
+constexpr int kDecMaxSlots = 6;
+constexpr int kDecSlotCap = 4;     // ring slots used (more 32 KB stages in flight lower the copy rate)
+constexpr int kDecRows = 64;       // output rows per unit
+constexpr int kDecR1 = 16;         // rows of W1 (and of W3) per stage
+constexpr int kDecR2 = 32;         // rows of W2 per stage
+constexpr int kDecMaxTok = 4;      // tokens per group (B columns 0..7 of the MMA: hi and lo plane of each)
 constexpr int kDecMaxT = 32;
-constexpr int kDecMaxPairs = 256;   // T * top_k
-constexpr int kDecStageRow = 512;   // code bytes per row and stage (3-bit: 384)
-constexpr int kDecScaleRow = 64;    // scale (or bias) bytes per row and stage, at most
-constexpr int kDecPlaneStride = 4160;  // per token and stage: <= 4096 plane bytes + bank padding
-constexpr int kDecSxStride = 512;      // per token and stage: <= 32 blocks x (step, sum lo, sum hi, sum)
-constexpr int kDecSlotCodes = 0;       // 32 KB: S1 32 rows x 512 B x 2 matrices, S2 64 rows x 512 B
-constexpr int kDecSlotScales = 32768;  // 8 KB: scales and biases
-constexpr int kDecSlotPlanes = kDecSlotScales + 8192;
-constexpr int kDecSlotSx = kDecSlotPlanes + kDecMaxTok * kDecPlaneStride;
-constexpr int kDecSlotBytes = ((kDecSlotSx + kDecMaxTok * kDecSxStride) + 1023) / 1024 * 1024;
-constexpr int kDecRedBytes = 16 * 2 * 16 * 8 * 4;  // 16 warps x 2 matrices x 16 rows x 8 columns
-constexpr int kDecHBytes = kDecMaxTok * kDecRows * 4;
-constexpr int kDecOffLen = 1028;   // offsets / active list entries (E + 1 <= 1025, padded to 16 bytes)
-constexpr int kDecRouteBytes = 6 * kDecMaxPairs * 4 + 2 * kDecOffLen * 4 + (kDecMaxPairs + 8) * 16;
-constexpr int kDecMiscBytes = 256;
-constexpr size_t kDecSmem = 1024 + (size_t)kDecStages * kDecSlotBytes + kDecRedBytes + kDecHBytes + kDecRouteBytes +
-                            kDecMiscBytes;
-static_assert(kDecSmem <= 227 * 1024, "fused decode kernel exceeds the per-block shared memory limit");
-static_assert((kDecRedBytes + kDecHBytes) % 16 == 0 && (6 * kDecMaxPairs * 4 + 2 * kDecOffLen * 4) % 16 == 0,
-              "the group records (int4) must stay 16-byte aligned");
+constexpr int kDecMaxPairs = 256;  // T * top_k
+constexpr int kDecMaxE = 1024;
+constexpr int kDecCodeBytes = 32768;  // code bytes of a stage, at most
+constexpr int kDecMaxSeg = 1024;      // code bytes per row and stage, at most
+constexpr int kDecRedFloats = kDecNkq * 4 * 16 * 8;
+constexpr int kDecOffLen = kDecMaxE + 4;
+constexpr int kDecMaxGroups = kDecMaxPairs + 8;
+// fixed shared region (after the ring and the two plane buffers), byte offsets
+constexpr int kDecFxRed = 0;
+constexpr int kDecFxH = kDecFxRed + kDecRedFloats * 4;           // 2 buffers x 4 tokens x 64 h values
+constexpr int kDecFxZero = kDecFxH + 2 * kDecMaxTok * kDecRows * 4;  // 256 zero bytes (dead B columns)
+constexpr int kDecFxScr = kDecFxZero + 256;                      // the service warp's scratch (64 ints)
+constexpr int kDecFxIds = kDecFxScr + 256;
+constexpr int kDecFxW = kDecFxIds + kDecMaxPairs * 4;
+constexpr int kDecFxSorted = kDecFxW + kDecMaxPairs * 4;
+constexpr int kDecFxInv = kDecFxSorted + kDecMaxPairs * 4;
+constexpr int kDecFxOff = kDecFxInv + kDecMaxPairs * 4;
+constexpr int kDecFxCur = kDecFxOff + kDecOffLen * 4;
+constexpr int kDecFxGroups = kDecFxCur + kDecOffLen * 4;
+constexpr int kDecFxBars = kDecFxGroups + kDecMaxGroups * 16;
+constexpr int kDecFxMisc = kDecFxBars + (2 * kDecMaxSlots + 8) * 8;
+constexpr int kDecFixedBytes = kDecFxMisc + 64;
+constexpr int kDecSmemMax = 227 * 1024;
+static_assert(kDecFxGroups % 16 == 0 && kDecFxBars % 8 == 0, "group records and barriers must stay aligned");
 
-// One packed matrix as the fused kernel reads it.
+// One packed matrix as the fused kernel streams it.
 struct DecMat {
   int fmt, group, n_out, n_in;
-  int rows;       // rows per stage: 32 (W1, W3) or 64 (W2)
-  int box;        // TMA box width in bytes (128 swizzled, or 96 unswizzled for 3-bit); 4 boxes per stage
-  int ks;         // inputs per stage
-  int sbytes;     // scale (and bias) bytes per row and stage
+  int R;       // rows per stage and box: 16 (W1, W3) or 32 (W2)
+  int lb;      // bytes per line of the box: 128 (swizzled) or 96 (3-bit, unswizzled)
+  int seg;     // code bytes per row and stage (a multiple of lb)
+  int nch;     // stages along a row (row bytes / seg)
+  int K;       // inputs per stage
+  int nbw;     // 64-input blocks per consumer warp and stage (K / 256)
+  int gshift;  // log2(group / 64) for groups of 64 or 128; -1 for 32
+  int sK;      // scale entries per row and stage
+  int spitch;  // bytes per row of a scale box: the stage's scales padded to an odd multiple of 16
+  int ptok;    // plane bytes per token in a plane buffer (n_in * 2, bank-padded)
+  int sxtok;   // block-record bytes per token in a plane buffer (n_in / 64 * 16, bank-padded)
 };
 
 enum DecMatIdx { DM_W1 = 0, DM_W3 = 1, DM_W2 = 2, DM_S1 = 3, DM_S3 = 4, DM_S2 = 5 };
 
 struct DecParams {
-  CUtensorMap map[6];   // codes of w1, w3, w2, shared w1, w3, w2
+  CUtensorMap map[6];   // codes of w1, w3, w2, shared w1, w3, w2 (3-D, chunk-major)
   CUtensorMap smap[6];  // their scales
   CUtensorMap bmap[6];  // their biases (affine)
   DecMat m[6];
@@ -95,17 +121,22 @@ struct DecParams {
   const int* tid2eid;
   int router_bf16;
   int T, d, f, fs, E, k, hash, vocab, has_shared;
-  int G;               // grid size
+  int G;           // grid size
+  int nslot;       // ring slots
+  int slot_bytes;  // 32 KB of codes + scales and biases (multiple of 1024)
+  int pbuf;        // bytes per plane buffer (multiple of 128): one unit's activation rows
+  int sx_off;      // offset of the per-block records within a plane buffer
+  int ntmax;       // tokens per group (<= 4): the plane buffers hold this many rows
   // workspace
   float* logits;       // [T][E]
   int* hids;           // [T][k] (hash)
   float* hw;           // [T][k] (hash)
-  uint8_t* xplanes;    // [2][T][d*4]: planes for the routed (0) and shared (1) W1/W3 formats
+  uint8_t* xplanes;    // [2][T][d*4]: planes (d*2 bytes used) for the routed (0) and shared (1) W1/W3 formats
   float4* xsx;         // [T][d/64]: (step, sum of inputs 0..31, sum of 32..63, sum)
   uint8_t* hplanes;    // [P][fmax*4]
   float4* hsx;         // [P][fmax/64]
   float* y;            // [P][d]
-  int* cnt_h;          // [kDecMaxPairs + 8]
+  int* cnt_h;          // [kDecMaxGroups]
   int* cnt_y;          // [d/64]
   int* sync;           // [0] barrier count, [1] barrier generation, [2] exit count
   int* err;
@@ -135,7 +166,6 @@ MOE_DEV void dec_grid_barrier(int* sync, int nblocks, int* err, volatile int* ab
           *abort_flag = 1;
           break;
         }
-        __nanosleep(32);
       }
     }
     __threadfence();
@@ -147,11 +177,9 @@ MOE_DEV void dec_grid_barrier(int* sync, int nblocks, int* err, volatile int* ab
 // The planes of one 64-input block of one activation row (64 values, two
 // per lane, already in registers; lane l holds inputs 2l, 2l+1): warp-wide.
 // `q_scratch`: 64 ints of this warp's shared scratch.  Writes the records of
-// `perm` (and the negated records for mxfp4) at `dst` (2 k-blocks x 4
-// threads) and returns (step, dequantised sum of inputs 0..31, of 32..63, of
-// all 64) to every lane.
-MOE_DEV float4 dec_make_block(float v0, float v1, int perm, bool with_neg, uint8_t* dst, int* q_scratch,
-                              int* err) {
+// `perm` at `dst` (2 k-blocks x 4 threads x 16 bytes) and returns (step,
+// dequantised sum of inputs 0..31, of 32..63, of all 64) to every lane.
+MOE_DEV float4 dec_make_block(float v0, float v1, int perm, uint8_t* dst, int* q_scratch, int* err) {
   const int lane = threadIdx.x & 31;
   uint32_t e = max((__float_as_uint(v0) >> 23) & 0xFFu, (__float_as_uint(v1) >> 23) & 0xFFu);
 #pragma unroll
@@ -168,68 +196,27 @@ MOE_DEV float4 dec_make_block(float v0, float v1, int perm, bool with_neg, uint8
   __syncwarp();
   if (lane < 8) {
     const int kb2 = lane >> 2, t = lane & 3;
-    uint32_t rec[2][4];  // [sign][hi b0, hi b1, lo b0, lo b1]
+    uint32_t hw[2], lw[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      uint32_t hp = 0, lp = 0, hn = 0, ln = 0;
+      uint32_t hp = 0, lp = 0;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int q = q_scratch[plane_input(perm, kb2, t, h, j)];
-        hp |= (uint32_t)((q >> 8) & 0xFF) << (8 * j);
-        lp |= (uint32_t)(q & 0xFF) << (8 * j);
-        hn |= (uint32_t)(((-q) >> 8) & 0xFF) << (8 * j);
-        ln |= (uint32_t)((-q) & 0xFF) << (8 * j);
+        const int lo = (int)(signed char)(q & 0xFF);  // q = 256 * hi + lo, lo in [-128, 127]
+        hp |= (uint32_t)(((q - lo) >> 8) & 0xFF) << (8 * j);
+        lp |= (uint32_t)(lo & 0xFF) << (8 * j);
       }
-      rec[0][h] = hp;
-      rec[0][2 + h] = lp;
-      rec[1][h] = hn;
-      rec[1][2 + h] = ln;
+      hw[h] = hp;
+      lw[h] = lp;
     }
-    const int rb = with_neg ? 32 : 16;
-    uint4* d0 = reinterpret_cast<uint4*>(dst + kb2 * 4 * rb + t * rb);
-    d0[0] = make_uint4(rec[0][0], rec[0][1], rec[0][2], rec[0][3]);
-    if (with_neg) d0[1] = make_uint4(rec[1][0], rec[1][1], rec[1][2], rec[1][3]);
+    *reinterpret_cast<uint4*>(dst + kb2 * 64 + t * 16) = make_uint4(hw[0], hw[1], lw[0], lw[1]);
   }
   __syncwarp();
   return make_float4(sc.y, sc.y * (float)s_lo, sc.y * (float)s_hi, sc.y * (float)(s_lo + s_hi));
 }
 
 // ------------------------------------------------------------ A operands
-// Stage layout of one matrix's codes: 4 TMA boxes side by side along the row
-// (box b = bytes [b*box, (b+1)*box) of each of `rows` rows), each box `rows`
-// lines of `box` bytes; 128-byte boxes are swizzled (16-byte chunk c of line
-// r sits at chunk c ^ (r & 7)), so the 8 rows an ldmatrix phase reads hit
-// distinct banks.
-struct DecTile {
-  uint32_t codes;  // shared address of the matrix's first box
-  int rows;        // lines per box
-  int rt;          // 16-row tile
-  int byte0;       // first code byte (in the stage row) of this warp's slice
-};
-
-MOE_DEV uint32_t swz(uint32_t box, int row, int chunk) {
-  return box + (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
-// ldmatrix x4 of two 16-byte chunks (bytes `byte`, `byte`+16 of the stage row)
-// of the tile's rows: d[0] = (row g, chunk 0), d[1] = (g+8, chunk 0),
-// d[2] = (g, chunk 1), d[3] = (g+8, chunk 1)
-MOE_DEV void dec_ldsm2(const DecTile& tl, int byte, uint32_t (&d)[4]) {
-  const int lane = threadIdx.x & 31, mtx = lane >> 3;
-  const int row = tl.rt * 16 + (mtx & 1) * 8 + (lane & 7);
-  const int b = byte + (mtx >> 1) * 16;
-  ldsm_x4(swz(tl.codes + (b >> 7) * tl.rows * 128, row, (b & 127) >> 4), d[0], d[1], d[2], d[3]);
-}
-
-// ldmatrix x2 of one 16-byte chunk of the tile's rows: d[0] = row g, d[1] = row g+8
-MOE_DEV void dec_ldsm1(const DecTile& tl, int byte, uint32_t (&d)[4]) {
-  const int lane = threadIdx.x & 31;
-  const int row = tl.rt * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-               : "=r"(d[0]), "=r"(d[1])
-               : "r"(swz(tl.codes + (byte >> 7) * tl.rows * 128, row, (byte & 127) >> 4)));
-}
-
-// per format: bits per code, and how a k-block's codes become A registers
 template <int FMT>
 struct DecA {
   static constexpr int bits = FMT == F_A2 ? 2 : FMT == F_A3 ? 3 : FMT == F_A8 ? 8 : 4;
@@ -272,183 +259,178 @@ MOE_DEV uint32_t spread3x4(uint32_t t) {
   const uint32_t od = ((t & 0xE38u) * 0x8020u) & 0x07000700u;
   return ev | od;
 }
-// codes 8t..8t+7 of k-block (12 bytes) starting at stage byte `byte` of `row`
-// (unswizzled 96-byte boxes)
-MOE_DEV uint32_t codes3x8(const DecTile& tl, int row, int byte, int t) {
-  const int box = byte / 96, off = byte - box * 96;
-  const uint32_t base = tl.codes + box * tl.rows * 96 + row * 96 + off;
+// codes 8t..8t+7 of the 12-byte k-block at byte `off` of the 96-byte line
+// starting at `line` (unswizzled)
+MOE_DEV uint32_t codes3x8(uint32_t line, int off, int t) {
+  const uint32_t base = line + off;
   const int bt = 3 * t;
   const uint32_t w0 = lds32u(base + (bt & ~3)), w1 = lds32u(base + (bt & ~3) + 4);
   return __funnelshift_r(w0, w1, 8 * (bt & 3)) & 0xFFFFFFu;
 }
-MOE_DEV void load_a3(const DecTile& tl, int byte, uint32_t (&a)[4]) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const uint32_t vg = codes3x8(tl, tl.rt * 16 + g, byte, t), vg8 = codes3x8(tl, tl.rt * 16 + 8 + g, byte, t);
-  a[0] = spread3x4(vg & 0xFFFu);
-  a[2] = spread3x4(vg >> 12);
-  a[1] = spread3x4(vg8 & 0xFFFu);
-  a[3] = spread3x4(vg8 >> 12);
-}
 
 // ------------------------------------------------------------ one stage
-// Consumer warp (rt, kq) over its slice of one stage: integer MMAs per
-// k-block, folded into acc[m][4] once per 64-input block (or per 32-input
-// group).  ntok tokens occupy B columns 0..ntok-1.
-struct DecStageCtx {
-  uint32_t slot;        // shared address of the stage slot
-  int rt, kq, ntok;
-  int group, ks, rows;  // of the unit's matrices
+// What a consumer warp needs to address its tile in any stage of a unit.
+// Shared addresses are relative to the stage slot.  A rows 0..7 of the tile
+// live in code box `a0` at box rows r0..r0+7, A rows 8..15 in box `a8` at
+// rows r8..r8+7; their scales in scale boxes `s0` / `s8` (biases `brow`
+// bytes further).
+struct DecWarp {
+  uint32_t a0, a8, s0, s8;
+  int r0, r8;
+  int R;       // rows per box
+  int nbw;     // 64-input blocks of this warp per stage
+  int kq;      // input slice
+  int gshift;  // log2(group / 64), -1 for 32-input groups
+  int spitch, brow;
+  int ptok, sxtok;
 };
 
+// acc[0] (A row g) and acc[1] (A row g+8) of token t += s_r * st * P + b_r * sm
+// over one scale group: P = 256 * C[., 2t] + C[., 2t+1] is the exact
+// integer sum of codes x fixed-point inputs, st the inputs' step, sm their
+// dequantised sum; `gi`: the group's scale entry in the stage.
 template <int FMT>
-MOE_DEV void dec_scale_bias(const DecStageCtx& c, int m, int grp, int row, int sbytes, float& s, float& b) {
-  const uint32_t sc = c.slot + kDecSlotScales + m * 4096 + row * sbytes;
+MOE_DEV void dec_fold(const DecWarp& q, uint32_t slot, float st, float sm, int gi, const int (&c)[4],
+                      float (&acc)[2]) {
+  const int g = (threadIdx.x & 31) >> 2;
+  const uint32_t sc0 = slot + q.s0 + (q.r0 + g) * q.spitch, sc8 = slot + q.s8 + (q.r8 + g) * q.spitch;
+  float s0, b0, s8, b8;
   if constexpr (FMT == F_MX4) {
-    const uint32_t e = lds8u(sc + grp);
     // 2^(e-127) / 2 (the A operand holds 2*e2m1)
-    s = __uint_as_float(e > 1 ? ((e - 1) << 23) : (e ? 0x00400000u : 0x00200000u));
-    b = 0.f;
+    const uint32_t e0 = lds8u(sc0 + gi), e8 = lds8u(sc8 + gi);
+    s0 = __uint_as_float(e0 > 1 ? ((e0 - 1) << 23) : (e0 ? 0x00400000u : 0x00200000u));
+    s8 = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));
+    b0 = b8 = 0.f;
   } else {
-    s = bf16_bits_to_float(lds16u(sc + 2 * grp));
-    b = bf16_bits_to_float(lds16u(sc + c.rows * kDecScaleRow + 2 * grp));
+    s0 = bf16_bits_to_float(lds16u(sc0 + 2 * gi));
+    b0 = bf16_bits_to_float(lds16u(sc0 + q.brow + 2 * gi));
+    s8 = bf16_bits_to_float(lds16u(sc8 + 2 * gi));
+    b8 = bf16_bits_to_float(lds16u(sc8 + q.brow + 2 * gi));
   }
+  acc[0] = fmaf(s0 * st, (float)(c[0] * 256 + c[1]), fmaf(b0, sm, acc[0]));
+  acc[1] = fmaf(s8 * st, (float)(c[2] * 256 + c[3]), fmaf(b8, sm, acc[1]));
 }
 
-// acc[0..3] += s_r * step_c * P_rc + b_r * sum_c for the C-fragment layout
-// (rows g, g+8; columns 2t, 2t+1) of one group; `si` selects the sum over
-// the group's inputs in the (step, sum lo, sum hi, sum) record of the block
+// Column pairs a fold unit of a group of ntok tokens occupies: 1, 2 or 4.
+MOE_DEV int dec_ntp(int ntok) { return ntok == 1 ? 1 : ntok == 2 ? 2 : 4; }
+
+// The warp's input slice of one stage.  The MMA has 4 column pairs (hi and
+// lo plane of a token each); a group of ntok tokens needs ntp of them, so the
+// slice's fold units (64-input blocks, or k-blocks for 32-input groups) are
+// taken R = 4 / ntp at a time: unit r of a round writes its products into
+// column pairs r*ntp .. r*ntp+ntp-1 (the lanes supplying the other columns
+// read the zero block), the round's units accumulate in one C fragment
+// without mixing, and each lane folds the unit whose column pair it holds.
+// One fold then serves R units; the lanes holding the same token are summed
+// once per row set (dec_reduce_lanes).  `plb`: the stage's inputs in the plane
+// buffer (token j at j * ptok), `sxb`: their block records (token j at
+// j * sxtok), `zb`: 256 zero bytes.
 template <int FMT>
-MOE_DEV void dec_fold(const DecStageCtx& c, int m, int grp, int sbytes, int bs, int si, const int (&ch)[4],
-                      const int (&cl)[4], float (&acc)[4]) {
+MOE_DEV void dec_stage(const DecWarp& q, uint32_t slot, uint32_t plb, uint32_t sxb, uint32_t zb, int ntok,
+                       float (&acc)[2]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const int r0 = c.rt * 16 + g, r1 = r0 + 8;
-  const int c0 = 2 * t, c1 = c0 + 1;
-  const uint32_t sx = c.slot + kDecSlotSx + bs * 16;
-  const float st0 = c0 < c.ntok ? lds_f32(sx + c0 * kDecSxStride) : 0.f;
-  const float st1 = c1 < c.ntok ? lds_f32(sx + c1 * kDecSxStride) : 0.f;
-  const float sm0 = c0 < c.ntok ? lds_f32(sx + c0 * kDecSxStride + 4 * si) : 0.f;
-  const float sm1 = c1 < c.ntok ? lds_f32(sx + c1 * kDecSxStride + 4 * si) : 0.f;
-  float s0, b0, s1, b1;
-  dec_scale_bias<FMT>(c, m, grp, r0, sbytes, s0, b0);
-  dec_scale_bias<FMT>(c, m, grp, r1, sbytes, s1, b1);
-  acc[0] = fmaf(s0 * st0, (float)(ch[0] * 256 + cl[0]), fmaf(b0, sm0, acc[0]));
-  acc[1] = fmaf(s0 * st1, (float)(ch[1] * 256 + cl[1]), fmaf(b0, sm1, acc[1]));
-  acc[2] = fmaf(s1 * st0, (float)(ch[2] * 256 + cl[2]), fmaf(b1, sm0, acc[2]));
-  acc[3] = fmaf(s1 * st1, (float)(ch[3] * 256 + cl[3]), fmaf(b1, sm1, acc[3]));
-}
-
-// M = 2: S1 (W1, W3; 2 tiles x 8 slices of 64 code bytes); M = 1: S2 (W2; 4
-// tiles x 4 slices of 128 code bytes).  3-bit: slices of 48 / 96 bytes.
-template <int FMT, int M>
-MOE_DEV void dec_stage(const DecStageCtx& c, float (&acc)[2][4]) {
-  constexpr int BITS = DecA<FMT>::bits;
-  constexpr int WB = (FMT == F_A3 ? 48 : 64) * (M == 2 ? 1 : 2);  // code bytes of this warp per row
-  constexpr int KBW = WB * 8 / BITS / 32;                         // k-blocks of this warp
-  constexpr int KBB = 32 * BITS / 8;                              // code bytes per k-block and row
-  constexpr bool MX = FMT == F_MX4;
-  constexpr int REC = MX ? 32 : 16;  // plane record bytes per (k-block, thread)
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const bool live = g < c.ntok;
-  const int pstride = c.ks * plane_bytes_per_input(FMT) + (MX ? 16 : 64);
-  const uint32_t planes = c.slot + kDecSlotPlanes + (uint32_t)(live ? g : 0) * pstride + t * REC;
-  const int group = c.group;
-  const bool g32 = group == 32;  // 32-input groups: each k-block has its own scale
-  const int sbytes = c.ks / group * (MX ? 1 : 2);
-  const int kb0 = c.kq * KBW;    // first k-block (within the stage) of this warp
-  const int byte0 = c.kq * WB;   // first code byte (within the stage row) of this warp
-#pragma unroll
-  for (int blk = 0; blk < KBW / 2; ++blk) {  // 64-input blocks
-    const int kbs = kb0 + 2 * blk;           // stage k-block of the block's first half
-    const int bs = kbs >> 1;                 // stage block index
-    const int byte = byte0 + 2 * blk * KBB;  // the block's first code byte
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-      DecTile tl;
-      tl.codes = c.slot + kDecSlotCodes + m * 16384;
-      tl.rows = c.rows;
-      tl.rt = c.rt;
-      int ch[4] = {0, 0, 0, 0}, cl[4] = {0, 0, 0, 0};
-      uint32_t w[4];
-      if constexpr (FMT == F_A4 || FMT == F_MX4) dec_ldsm2(tl, byte, w);  // both k-blocks
-      if constexpr (FMT == F_A2) dec_ldsm1(tl, byte, w);                  // the block is one chunk
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint4 B = live ? lds128u(planes + (kbs + h) * 4 * REC) : make_uint4(0, 0, 0, 0);
-        uint32_t a[4];
-        if constexpr (FMT == F_A4) {
-          unpack_a4(w[2 * h], w[2 * h + 1], a);
-        } else if constexpr (FMT == F_MX4) {
-          uint32_t an[4];
-          unpack_mx4(w[2 * h], w[2 * h + 1], a, an);
-          const uint4 Bn = live ? lds128u(planes + (kbs + h) * 4 * REC + 16) : make_uint4(0, 0, 0, 0);
-          mma_u8s8(ch, an, Bn.x, Bn.y);
-          mma_u8u8(cl, an, Bn.z, Bn.w);
-        } else if constexpr (FMT == F_A8) {
-          dec_ldsm2(tl, byte + h * 32, a);  // one k-block = two chunks
-        } else if constexpr (FMT == F_A2) {
-          unpack_a2(w[0], w[1], h, a);
-        } else {
-          load_a3(tl, byte + h * KBB, a);
-        }
-        mma_u8s8(ch, a, B.x, B.y);
-        mma_u8u8(cl, a, B.z, B.w);
-        if (g32) {  // fold each 32-input group on its own
-          dec_fold<FMT>(c, m, kbs + h, sbytes, bs, 1 + h, ch, cl, acc[m]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) ch[q] = cl[q] = 0;
+  const bool g32 = q.gshift < 0;
+  const int GU = g32 ? 1 : 2;  // k-blocks per fold unit
+  const int ntp = dec_ntp(ntok);
+  const int R = min(4 / ntp, 2 * q.nbw / GU);  // fold units per round
+  // B side: this lane supplies column g = plane (g & 1) of column pair g >> 1 = rB * ntp + jB
+  const int cpB = g >> 1, rB = cpB / ntp, jB = cpB - rB * ntp;
+  const bool liveB = jB < ntok && rB < R;
+  const uint32_t bbase = liveB ? plb + jB * q.ptok + t * 16 + (g & 1) * 8 : zb;
+  const uint32_t bstride = liveB ? 128 : 0;
+  // C side: this lane holds column pair t = rC * ntp + jC
+  const int rC = t / ntp, jC = t - rC * ntp;
+  const bool liveC = jC < ntok && rC < R;
+  const uint32_t sxbase = liveC ? sxb + jC * q.sxtok : zb;
+  const uint32_t sxstride = liveC ? 16 : 0;
+  // this lane's ldmatrix row: matrix (lane >> 3) = (A rows 0..7 | 8..15) x (chunk 0 | 1)
+  const int mtx = lane >> 3;
+  const uint32_t lbox = slot + ((mtx & 1) ? q.a8 : q.a0);
+  const int lrow = ((mtx & 1) ? q.r8 : q.r0) + (lane & 7);
+  const int csel = mtx >> 1;
+  const int ku0 = q.kq * 2 * q.nbw;  // the slice's first k-block in the stage
+  const int nk = 2 * q.nbw, rk = R * GU;
+  for (int k0 = 0; k0 < nk; k0 += rk) {
+    int c[4] = {0, 0, 0, 0}, cn[4] = {0, 0, 0, 0};
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll 2
+    for (int kk = 0; kk < rk; ++kk) {
+      const int u = ku0 + k0 + kk;  // stage k-block
+      const int r = kk / GU;        // the fold unit's column-pair group in this round
+      uint32_t a[4];
+      if constexpr (FMT == F_A4 || FMT == F_MX4) {  // a k-block is one 16-byte chunk: rows g and g+8
+        const int by = u * 16, ln = by >> 7;
+        asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                     : "=r"(w[0]), "=r"(w[1])
+                     : "r"(lbox + (uint32_t)((ln * q.R + lrow) * 128 + ((((by & 127) >> 4) ^ (lrow & 7)) << 4))));
+      } else if constexpr (FMT == F_A8) {  // a k-block is two chunks
+        const int by = u * 32, ln = by >> 7;
+        ldsm_x4(lbox + (uint32_t)((ln * q.R + lrow) * 128 + (((((by & 127) >> 4) + csel) ^ (lrow & 7)) << 4)), a[0],
+                a[1], a[2], a[3]);
+      } else if constexpr (FMT == F_A2) {  // a 64-input block is one chunk holding both k-blocks
+        if ((u & 1) == 0) {
+          const int by = (u >> 1) * 16, ln = by >> 7;
+          asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+                       : "=r"(w[0]), "=r"(w[1])
+                       : "r"(lbox + (uint32_t)((ln * q.R + lrow) * 128 + ((((by & 127) >> 4) ^ (lrow & 7)) << 4))));
         }
       }
-      if (!g32) dec_fold<FMT>(c, m, (bs * 64) / group, sbytes, bs, 3, ch, cl, acc[m]);
+      const uint32_t baddr = r == rB ? bbase + (u >> 1) * bstride + (u & 1) * 64 : zb + (u & 1) * 64;
+      const uint2 B = lds64u(baddr);
+      if constexpr (FMT == F_A4) {
+        unpack_a4(w[0], w[1], a);
+      } else if constexpr (FMT == F_MX4) {
+        uint32_t an[4];
+        unpack_mx4(w[0], w[1], a, an);
+        mma_u8s8(cn, an, B.x, B.y);
+      } else if constexpr (FMT == F_A2) {
+        unpack_a2(w[0], w[1], u & 1, a);
+      } else if constexpr (FMT == F_A3) {  // 12-byte k-blocks in 96-byte unswizzled lines
+        const int by = u * 12, ln = by / 96, off = by - ln * 96;
+        const uint32_t v0 = codes3x8(slot + q.a0 + (uint32_t)((ln * q.R + q.r0 + g) * 96), off, t);
+        const uint32_t v8 = codes3x8(slot + q.a8 + (uint32_t)((ln * q.R + q.r8 + g) * 96), off, t);
+        a[0] = spread3x4(v0 & 0xFFFu);
+        a[2] = spread3x4(v0 >> 12);
+        a[1] = spread3x4(v8 & 0xFFFu);
+        a[3] = spread3x4(v8 >> 12);
+      }
+      mma_u8s8(c, a, B.x, B.y);
     }
+    // fold this lane's unit of the round (dead lanes fold a valid unit against the zero record)
+    const int f = (ku0 + k0) / GU + (liveC ? rC : 0);
+    const int bf = (f * GU) >> 1;  // its 64-input block
+    const float4 rec = lds_f4(sxbase + bf * sxstride);
+    const float sm = g32 ? (((f & 1) != 0) ? rec.z : rec.y) : rec.w;
+    int d4[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d4[i] = c[i] - cn[i];
+    dec_fold<FMT>(q, slot, rec.x, sm, g32 ? f : (bf >> q.gshift), d4, acc);
   }
 }
 
-}  // namespace moe
-
-namespace moe {
-
-MOE_DEV void dec_stage_any(int fmt, int M, const DecStageCtx& c, float (&acc)[2][4]) {
-  if (M == 2) {
-    switch (fmt) {
-      case F_A2: dec_stage<F_A2, 2>(c, acc); break;
-      case F_A3: dec_stage<F_A3, 2>(c, acc); break;
-      case F_A4: dec_stage<F_A4, 2>(c, acc); break;
-      case F_A8: dec_stage<F_A8, 2>(c, acc); break;
-      default: dec_stage<F_MX4, 2>(c, acc); break;
+// Sum the lanes that folded the same token's rows (dec_stage): afterwards
+// lane t < ntok of each quad holds token t's totals.
+MOE_DEV void dec_reduce_lanes(int ntok, float (&acc)[2]) {
+  const int ntp = dec_ntp(ntok);
+  if (ntp == 1) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 1);
+      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
     }
-  } else {
-    switch (fmt) {
-      case F_A2: dec_stage<F_A2, 1>(c, acc); break;
-      case F_A3: dec_stage<F_A3, 1>(c, acc); break;
-      case F_A4: dec_stage<F_A4, 1>(c, acc); break;
-      case F_A8: dec_stage<F_A8, 1>(c, acc); break;
-      default: dec_stage<F_MX4, 1>(c, acc); break;
-    }
+  } else if (ntp == 2) {
+#pragma unroll
+    for (int i = 0; i < 2; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
   }
 }
 
 // Routing results and work groups, shared by every CTA (built in P1).
-struct DecRoute {
-  int* ids;     // [T*k]
-  float* w;     // [T*k]
-  int* sorted;  // [T*k] flat pair indices grouped by expert
-  int* inv;
-  int* ev;
-  int* first;
-  int* off;     // [E+1]
-  int* active;  // [1 + E]
-  int4* groups; // {expert or -1 (shared), start (sorted position / first token), tokens, 0}
-};
-
 struct DecUnit {
   int stage;  // 1 or 2
   int grp;
   int u;      // 64-row block of the unit's output rows
   int mi;     // first matrix index (DecMatIdx)
-  int M;      // matrices (2: W1 and W3; 1: W2)
   int row0;   // first weight row in the stacked matrix
-  int nchunks;  // stages along the inputs
-  int nhalf;    // S1: the 64 rows come as two stages of 32 rows (per input chunk); S2: 1
 };
 
 MOE_DEV DecUnit dec_unit(const DecParams& p, const int4* groups, int nsg, int nrg, int i) {
@@ -457,7 +439,6 @@ MOE_DEV DecUnit dec_unit(const DecParams& p, const int4* groups, int nsg, int nr
   const int U1s = nsg * ufs, U1 = U1s + nrg * uf;
   if (i < U1) {
     U.stage = 1;
-    U.M = 2;
     if (i < U1s) {
       U.grp = i / ufs;
       U.u = i % ufs;
@@ -473,67 +454,202 @@ MOE_DEV DecUnit dec_unit(const DecParams& p, const int4* groups, int nsg, int nr
   } else {
     const int j = i - U1;
     U.stage = 2;
-    U.M = 1;
     U.grp = j / ud;
     U.u = j % ud;
     const bool sh = groups[U.grp].x < 0;
     U.mi = sh ? DM_S2 : DM_W2;
     U.row0 = (sh ? 0 : groups[U.grp].x * p.d) + kDecRows * U.u;
   }
-  U.nchunks = p.m[U.mi].n_in / p.m[U.mi].ks;
-  U.nhalf = U.stage == 1 ? 2 : 1;
   return U;
 }
 
 // Slot (flat index into the P = T*k + T activation rows) of token i of a group.
-MOE_DEV int dec_slot(const DecParams& p, const DecRoute& R, int4 g, int i) {
-  return g.x < 0 ? p.T * p.k + g.y + i : R.sorted[g.y + i];
+MOE_DEV int dec_slot(const DecParams& p, const int* sorted, int4 g, int i) {
+  return g.x < 0 ? p.T * p.k + g.y + i : sorted[g.y + i];
 }
-MOE_DEV int dec_token(const DecParams& p, const DecRoute& R, int4 g, int i) {
-  return g.x < 0 ? g.y + i : R.sorted[g.y + i] / p.k;
+MOE_DEV int dec_token(const DecParams& p, const int* sorted, int4 g, int i) {
+  return g.x < 0 ? g.y + i : sorted[g.y + i] / p.k;
+}
+
+// Bounded mbarrier wait of a consumer warp; false once the kernel aborts.
+MOE_DEV bool dec_consumer_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
+  bool have = !*abort_flag;
+  if (have && !dec_wait_bar(bar, parity, abort_flag)) {
+    set_error(err, kErrTimeout);
+    *abort_flag = 1;
+    have = false;
+  }
+  return __all_sync(0xffffffffu, have);  // the MMAs need every lane
+}
+
+// Consumer side of one unit's stages, row set by row set (FMT: the unit's
+// weight format; S1: W1/W3 in 4 row sets of 16, else W2 in 2 row sets of 32,
+// each over nch stages along the inputs).  Each row set's slice partials go
+// to `red`: S1 [(kq*4 + rs)*16 + row][token][W1 | W3], S2 [(kq*2 + rs)*32 +
+// row][token].
+template <int FMT, bool S1>
+MOE_DEV void dec_consume(const DecWarp& q, int nch, int K, int ntok, uint32_t ring, int slot_bytes, int nslot,
+                         uint32_t pl, uint32_t sx0, uint32_t zb, uint32_t full0, uint32_t empty0, int& n,
+                         bool have_pl, volatile int* abort_flag, int* err, float* red, int tt) {
+  constexpr int NRS = S1 ? 4 : 2;
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  for (int rs = 0; rs < NRS; ++rs) {
+    float acc[2] = {0.f, 0.f};
+    for (int chn = 0; chn < nch; ++chn, ++n) {
+      const int s = n % nslot;
+      const bool have = dec_consumer_wait(full0 + 8 * s, (n / nslot) & 1, abort_flag, err) && have_pl;
+      if (have) dec_stage<FMT>(q, ring + s * slot_bytes, pl + chn * K * 2, sx0 + chn * (K / 64) * 16, zb, ntok, acc);
+      __syncwarp();
+      if (lane == 0 && have) dec_arrive(empty0 + 8 * s);
+    }
+    dec_reduce_lanes(ntok, acc);
+    if constexpr (S1) {
+      *reinterpret_cast<float2*>(red + ((q.kq * 4 + rs) * 16 + tt * 8 + g) * 8 + 2 * t) = make_float2(acc[0], acc[1]);
+    } else {
+      red[((q.kq * 2 + rs) * 32 + tt * 16 + g) * 4 + t] = acc[0];
+      red[((q.kq * 2 + rs) * 32 + tt * 16 + g + 8) * 4 + t] = acc[1];
+    }
+  }
+}
+
+template <bool S1>
+MOE_DEV void dec_consume_any(int fmt, const DecWarp& q, int nch, int K, int ntok, uint32_t ring, int slot_bytes,
+                             int nslot, uint32_t pl, uint32_t sx0, uint32_t zb, uint32_t full0, uint32_t empty0,
+                             int& n, bool have_pl, volatile int* abort_flag, int* err, float* red, int tt) {
+#define MOE_DEC_CONSUME(F)                                                                                         \
+  dec_consume<F, S1>(q, nch, K, ntok, ring, slot_bytes, nslot, pl, sx0, zb, full0, empty0, n, have_pl, abort_flag, \
+                     err, red, tt)
+  switch (fmt) {
+    case F_A2: MOE_DEC_CONSUME(F_A2); break;
+    case F_A3: MOE_DEC_CONSUME(F_A3); break;
+    case F_A4: MOE_DEC_CONSUME(F_A4); break;
+    case F_A8: MOE_DEC_CONSUME(F_A8); break;
+    default: MOE_DEC_CONSUME(F_MX4); break;
+  }
+#undef MOE_DEC_CONSUME
+}
+
+// fp32 order as an unsigned order (larger float -> larger key); NaN is
+// mapped to -inf's key, like the router kernels' NaN handling
+MOE_DEV uint32_t dec_key(float v) {
+  if (v != v) v = -INFINITY;
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Top-k of one token's router logits (one warp): scores sqrtsoftplus(L),
+// keys score + bias, the k largest keys (ties: the smaller expert), weights
+// the selected scores renormalised to sum 1 (same rule as topk_token in
+// route.cuh).  Every load is issued before the first use; each round is a
+// warp max of the lanes' best keys (redux.sync) and a min of the expert
+// index among the lanes holding it.
+template <int MAXPER>
+MOE_DEV void dec_topk(const float* __restrict__ L, const float* __restrict__ bias, int E, int k, int* ids, float* w) {
+  const int lane = threadIdx.x & 31;
+  float lv[MAXPER], bv[MAXPER];
+#pragma unroll
+  for (int i = 0; i < MAXPER; ++i) {
+    const int e = i * 32 + lane;
+    lv[i] = e < E ? __ldcg(L + e) : 0.f;
+    bv[i] = (bias != nullptr && e < E) ? __ldg(bias + e) : 0.f;
+  }
+  uint32_t key[MAXPER];  // 0: no expert (past E) or already taken; any real key is larger
+  float sc[MAXPER];
+#pragma unroll
+  for (int i = 0; i < MAXPER; ++i) {
+    sc[i] = sqrt_softplus(lv[i]);
+    key[i] = i * 32 + lane < E ? dec_key(sc[i] + bv[i]) : 0u;
+  }
+  float ssum = 0.f, my_s = 0.f;
+  int my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    uint32_t bk = 0;
+    int bslot = 0;
+#pragma unroll
+    for (int i = 0; i < MAXPER; ++i)
+      if (key[i] > bk) {  // strict: the lowest slot among equal keys
+        bk = key[i];
+        bslot = i;
+      }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const int e = bslot * 32 + lane;
+    const int emin = __reduce_min_sync(0xffffffffu, bk == m ? e : 0x7fffffff);
+    const int owner = emin & 31, oslot = emin >> 5;
+    float s_sel = 0.f;
+    if (lane == owner) {
+#pragma unroll
+      for (int i = 0; i < MAXPER; ++i)
+        if (i == oslot) {
+          s_sel = sc[i];
+          key[i] = 0u;
+        }
+    }
+    s_sel = __shfl_sync(0xffffffffu, s_sel, owner);
+    ssum += s_sel;
+    if (lane == j) {
+      my_s = s_sel;
+      my_id = emin;
+    }
+  }
+  if (lane < k) {
+    ids[lane] = my_id;
+    w[lane] = ssum > 0.f ? my_s / ssum : 1.f / (float)k;
+  }
 }
 
 __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid_constant__ DecParams p) {
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = base;
-  float* red = reinterpret_cast<float*>(ring + (size_t)kDecStages * kDecSlotBytes);
-  float* hbuf = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(red) + kDecRedBytes);
-  int* rbase = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(hbuf) + kDecHBytes);
-  DecRoute R;
-  R.ids = rbase;
-  R.w = reinterpret_cast<float*>(rbase + kDecMaxPairs);
-  R.sorted = rbase + 2 * kDecMaxPairs;
-  R.inv = rbase + 3 * kDecMaxPairs;
-  R.ev = rbase + 4 * kDecMaxPairs;
-  R.first = rbase + 5 * kDecMaxPairs;
-  R.off = rbase + 6 * kDecMaxPairs;
-  R.active = R.off + kDecOffLen;
-  R.groups = reinterpret_cast<int4*>(R.active + kDecOffLen);  // 16-byte aligned
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(R.groups) + (kDecMaxPairs + 8) * 16);
-  volatile int* misc = reinterpret_cast<volatile int*>(bars + 2 * kDecStages);
-  volatile int* abort_flag = misc;  // [0] abort, [1] groups shared, [2] groups routed, [3] last flag
-  const uint32_t full0 = su32(bars), empty0 = su32(bars + kDecStages);
+  const uint32_t ring = su32(base);
+  const uint32_t planes0 = ring + (uint32_t)(p.nslot * p.slot_bytes);
+  uint8_t* fx = base + (size_t)p.nslot * p.slot_bytes + 2 * (size_t)p.pbuf;
+  float* red = reinterpret_cast<float*>(fx + kDecFxRed);
+  float* hbuf = reinterpret_cast<float*>(fx + kDecFxH);  // [2][4][64]
+  const uint32_t zb = su32(fx + kDecFxZero);
+  int* r_ids = reinterpret_cast<int*>(fx + kDecFxIds);
+  float* r_w = reinterpret_cast<float*>(fx + kDecFxW);
+  int* r_sorted = reinterpret_cast<int*>(fx + kDecFxSorted);
+  int* r_inv = reinterpret_cast<int*>(fx + kDecFxInv);
+  int* r_off = reinterpret_cast<int*>(fx + kDecFxOff);
+  int* r_cur = reinterpret_cast<int*>(fx + kDecFxCur);
+  int4* r_groups = reinterpret_cast<int4*>(fx + kDecFxGroups);
+  const uint32_t full0 = su32(fx + kDecFxBars), empty0 = full0 + 8 * kDecMaxSlots;
+  const uint32_t pfull0 = empty0 + 8 * kDecMaxSlots, pempty0 = pfull0 + 16;
+  const uint32_t efull0 = pempty0 + 16, eempty0 = efull0 + 16;  // unit epilogues: consumers -> service warp
+  volatile int* misc = reinterpret_cast<volatile int*>(fx + kDecFxMisc);
+  volatile int* abort_flag = misc;  // [0] abort, [1] groups shared, [2] groups routed
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = p.T, k = p.k, E = p.E, d = p.d;
   const int Tk = T * k;
 
   if (tid == 0) {
-    for (int s = 0; s < kDecStages; ++s) {
+    for (int s = 0; s < p.nslot; ++s) {
       dec_bar_init(full0 + 8 * s, 1);  // the producer's expect_tx arrive; the copies complete the transactions
       dec_bar_init(empty0 + 8 * s, kDecConsumerWarps);
+    }
+    for (int b = 0; b < 2; ++b) {
+      dec_bar_init(pfull0 + 8 * b, 1);
+      dec_bar_init(pempty0 + 8 * b, kDecConsumerWarps);
+      dec_bar_init(efull0 + 8 * b, kDecConsumerWarps);
+      dec_bar_init(eempty0 + 8 * b, 1);
     }
     misc[0] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  if (warp == kDecProducerWarp && lane < 18) {
+    const CUtensorMap* mp = lane < 6 ? &p.map[lane] : lane < 12 ? &p.smap[lane - 6] : &p.bmap[lane - 12];
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mp)) : "memory");
+  }
+  for (int e = tid; e < E; e += kDecThreads) r_off[e] = 0;  // per-expert counts (P1)
+  if (tid < 64) reinterpret_cast<int*>(fx + kDecFxZero)[tid] = 0;
   __syncthreads();
 
   // ------------------------------------------------------------ P0
   {
     // activation planes: (token, 64-input block) tasks over every warp of the grid
     const int nb = d / 64;
-    const int gw = blockIdx.x * (kDecConsumerWarps + 1) + warp, W = p.G * (kDecConsumerWarps + 1);
+    const int gw = blockIdx.x * kDecWarps + warp, W = p.G * kDecWarps;
     int* scratch = reinterpret_cast<int*>(red) + warp * 64;
     const int f0 = p.m[DM_W1].fmt, f1 = p.m[DM_S1].fmt;
     for (int it = gw; it < T * nb; it += W) {
@@ -541,16 +657,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
       const uint32_t xv = __ldg(reinterpret_cast<const uint32_t*>(p.x + (size_t)t * d + 64 * b) + lane);
       const float v0 = bf16lo(xv), v1 = bf16hi(xv);
       uint8_t* d0 = p.xplanes + (size_t)t * d * 4 + (size_t)b * 64 * plane_bytes_per_input(f0);
-      const float4 sx = dec_make_block(v0, v1, perm_of(f0), f0 == F_MX4, d0, scratch, p.err);
+      const float4 sx = dec_make_block(v0, v1, perm_of(f0), d0, scratch, p.err);
       if (p.has_shared) {
         uint8_t* d1 = p.xplanes + ((size_t)T + t) * d * 4 + (size_t)b * 64 * plane_bytes_per_input(f1);
-        dec_make_block(v0, v1, perm_of(f1), f1 == F_MX4, d1, scratch, p.err);
+        dec_make_block(v0, v1, perm_of(f1), d1, scratch, p.err);
       }
       if (lane == 0) p.xsx[(size_t)t * nb + b] = sx;
     }
     __syncthreads();
     if (!p.hash) {
-      // router logits of experts blockIdx.x, +G, ... for every token (warps 0..15 split d)
+      // router logits of experts blockIdx.x, +G, ... for every token (the consumer warps split d)
       for (int e = blockIdx.x; e < E; e += p.G) {
         if (warp < kDecConsumerWarps) {
           const int span = d / kDecConsumerWarps;
@@ -689,40 +805,98 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
 
   // ------------------------------------------------------------ P1
   if (!p.hash) {
-    for (int t = warp; t < T; t += kDecConsumerWarps + 1) {
+    for (int t = warp; t < T; t += kDecWarps) {
       if (E <= 32)
-        topk_token<1>(p.logits + (size_t)t * E, p.router_b, E, k, R.ids + t * k, R.w + t * k);
+        dec_topk<1>(p.logits + (size_t)t * E, p.router_b, E, k, r_ids + t * k, r_w + t * k);
       else if (E <= 256)
-        topk_token<8>(p.logits + (size_t)t * E, p.router_b, E, k, R.ids + t * k, R.w + t * k);
+        dec_topk<8>(p.logits + (size_t)t * E, p.router_b, E, k, r_ids + t * k, r_w + t * k);
       else
-        topk_token<32>(p.logits + (size_t)t * E, p.router_b, E, k, R.ids + t * k, R.w + t * k);
+        dec_topk<32>(p.logits + (size_t)t * E, p.router_b, E, k, r_ids + t * k, r_w + t * k);
     }
   } else {
     for (int i = tid; i < Tk; i += kDecThreads) {
-      R.ids[i] = __ldcg(p.hids + i);
-      R.w[i] = __ldcg(p.hw + i);
+      r_ids[i] = __ldcg(p.hids + i);
+      r_w[i] = __ldcg(p.hw + i);
     }
   }
   __syncthreads();
-  permute_ranks_block(R.ids, Tk, E, R.off, R.sorted, R.inv, R.active, p.err, R.ev, R.first);
-  __syncthreads();
-  if (tid == 0) {
-    int ng = 0;
-    if (p.has_shared)
-      for (int t0 = 0; t0 < T; t0 += kDecMaxTok) R.groups[ng++] = make_int4(-1, t0, min(kDecMaxTok, T - t0), 0);
-    const int nsg = ng;
-    for (int a = 0; a < R.active[0]; ++a) {
-      const int e = R.active[1 + a];
-      const int cnt = R.off[e + 1] - R.off[e];
-      for (int s0 = 0; s0 < cnt; s0 += kDecMaxTok) R.groups[ng++] = make_int4(e, R.off[e] + s0, min(kDecMaxTok, cnt - s0), 0);
+  // per-expert counts (out-of-range ids are reported and counted as expert 0)
+  {
+    bool bad = false;
+    for (int i = tid; i < Tk; i += kDecThreads) {
+      int e = r_ids[i];
+      if (e < 0 || e >= E) {
+        bad = true;
+        e = 0;
+      }
+      atomicAdd(r_off + e, 1);
     }
-    misc[1] = nsg;
-    misc[2] = ng - nsg;
+    if (bad) set_error(p.err, kErrDeviceInput);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // offsets (exclusive scan), cursors and groups: lane l owns experts
+    // [l*per, (l+1)*per); groups in ascending expert order after the shared ones
+    const int gsz = p.ntmax;
+    const int nsg = p.has_shared ? (T + gsz - 1) / gsz : 0;
+    const int per = (E + 31) / 32;
+    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+    int s = 0, ng = 0;
+    for (int e = e0; e < e1; ++e) {
+      const int c = r_off[e];
+      s += c;
+      ng += (c + gsz - 1) / gsz;
+    }
+    int sx = s, gx = ng;  // inclusive warp scans
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int a = __shfl_up_sync(0xffffffffu, sx, o), b = __shfl_up_sync(0xffffffffu, gx, o);
+      if (lane >= o) {
+        sx += a;
+        gx += b;
+      }
+    }
+    int run = sx - s, gi = nsg + gx - ng;
+    for (int e = e0; e < e1; ++e) {
+      const int c = r_off[e];
+      r_off[e] = run;
+      r_cur[e] = run;
+      for (int q0 = 0; q0 < c; q0 += gsz) r_groups[gi++] = make_int4(e, run + q0, min(gsz, c - q0), 0);
+      run += c;
+    }
+    if (lane == 31) {
+      r_off[E] = run;
+      misc[1] = nsg;
+      misc[2] = gx;
+    }
+    if (lane < nsg) r_groups[lane] = make_int4(-1, lane * gsz, min(gsz, T - lane * gsz), 0);
+    __syncwarp();
+    // stable order within each expert: pairs in ascending flat index
+    const unsigned lt = (1u << lane) - 1u;
+    for (int c0 = 0; c0 < Tk; c0 += 32) {
+      const int i = c0 + lane;
+      int e = -1;
+      if (i < Tk) {
+        e = r_ids[i];
+        if (e < 0 || e >= E) e = 0;
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      int base = 0;
+      if (i < Tk) {
+        base = r_cur[e];
+        const int pos = base + __popc(peers & lt);
+        r_sorted[pos] = i;
+        r_inv[i] = pos;
+      }
+      __syncwarp();
+      if (i < Tk && (peers >> lane) == 1u) r_cur[e] = base + __popc(peers);  // highest lane of its expert
+      __syncwarp();
+    }
   }
   if (blockIdx.x == 0) {
     for (int i = tid; i < Tk; i += kDecThreads) {
-      if (p.ids_out) p.ids_out[i] = R.ids[i];
-      if (p.w_out) p.w_out[i] = R.w[i];
+      if (p.ids_out) p.ids_out[i] = r_ids[i];
+      if (p.w_out) p.w_out[i] = r_w[i];
     }
   }
   __syncthreads();
@@ -730,197 +904,224 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
   const int n_units = nsg * (p.fs / kDecRows) + nrg * (p.f / kDecRows) + (nsg + nrg) * (d / kDecRows);
   const int fmax = max(p.f, p.fs);
 
-  if (warp == kDecConsumerWarps) {
+  if (warp == kDecProducerWarp) {
     // ============================================================ producer
-    int n = 0;  // stages issued
-    bool ok = true;
-    for (int ui = blockIdx.x; ui < n_units && ok; ui += p.G) {
-      const DecUnit U = dec_unit(p, R.groups, nsg, nrg, ui);
-      const int4 grp = R.groups[U.grp];
-      const DecMat& m0 = p.m[U.mi];
-      const bool mx = m0.fmt == F_MX4;
-      const int pb = plane_bytes_per_input(m0.fmt);
-      const int pstride = m0.ks * pb + (mx ? 16 : 64);
-      const uint32_t box_bytes = (uint32_t)(m0.rows * m0.box);
-      const uint32_t sc_bytes = (uint32_t)(m0.rows * m0.sbytes);
-      const uint32_t tx = (uint32_t)U.M * (4 * box_bytes + sc_bytes * (mx ? 1 : 2)) +
-                          (uint32_t)grp.z * (m0.ks * pb + (m0.ks / 64) * 16);
-      bool dep_ok = U.stage == 1;
-      for (int st = 0; st < U.nhalf * U.nchunks; ++st, ++n) {
-        const int half = st / U.nchunks, kc = st % U.nchunks;
-        const int row0 = U.row0 + half * m0.rows;
-        const int s = n % kDecStages;
-        const uint32_t slot = su32(ring + (size_t)s * kDecSlotBytes);
-        const uint32_t full = full0 + 8 * s, empty = empty0 + 8 * s;
-        if (lane == 0) {
-          if (n >= kDecStages && !dec_wait_bar(empty, ((n / kDecStages) - 1) & 1, abort_flag)) {
-            set_error(p.err, kErrTimeout);
-            *abort_flag = 1;
-          }
-          if (!*abort_flag) {
-            dec_expect_tx(full, tx);
-            for (int mm = 0; mm < U.M; ++mm) {
-              const int mi = U.mi + mm;
-              const uint32_t cbase = slot + kDecSlotCodes + mm * 16384;
-              for (int b = 0; b < 4; ++b)
-                dec_tma_2d(cbase + b * box_bytes, &p.map[mi], kc * 4 * m0.box + b * m0.box, row0, full);
-              const uint32_t sbase = slot + kDecSlotScales + mm * 4096;
-              const int sx = kc * (m0.ks / m0.group);  // first scale entry of the stage
-              dec_tma_2d(sbase, &p.smap[mi], sx, row0, full);
-              if (!mx) dec_tma_2d(sbase + m0.rows * kDecScaleRow, &p.bmap[mi], sx, row0, full);
-            }
-            if (!dep_ok) {
-              // W2 stages read the group's h planes: wait for all its S1 units.
-              // (On a timeout the plane copies below are still issued -- they
-              // stay in bounds -- so the stage's transaction count completes.)
-              const int target = p.stall_test ? 0x3fffffff : (grp.x < 0 ? p.fs / kDecRows : p.f / kDecRows);
-              if (!dec_wait_count(p.cnt_h + U.grp, target, abort_flag, p.stall_test ? 2000000LL : kDecWaitCycles)) {
-                set_error(p.err, kErrTimeout);
-                *abort_flag = 1;
-              }
-              fence_proxy_async_global();
-              dep_ok = true;
-            }
-            for (int i = 0; i < grp.z; ++i) {
-              const uint8_t* src;
-              const float4* ssrc;
-              if (U.stage == 1) {
-                const int tok = dec_token(p, R, grp, i);
-                const int layout = grp.x < 0 ? 1 : 0;
-                src = p.xplanes + ((size_t)layout * T + tok) * d * 4;
-                ssrc = p.xsx + (size_t)tok * (d / 64);
-              } else {
-                const int sl = dec_slot(p, R, grp, i);
-                src = p.hplanes + (size_t)sl * fmax * 4;
-                ssrc = p.hsx + (size_t)sl * (fmax / 64);
-              }
-              dec_bulk(slot + kDecSlotPlanes + i * pstride, src + (size_t)kc * m0.ks * pb, m0.ks * pb, full);
-              dec_bulk(slot + kDecSlotSx + i * kDecSxStride, ssrc + (size_t)kc * (m0.ks / 64), (m0.ks / 64) * 16,
-                       full);
-            }
-          }
-        }
-        __syncwarp();
-        if (*abort_flag) {
-          ok = false;
-          break;
-        }
-      }
-    }
-    // drain: every issued copy must land before the block exits
+    int n = 0, np = 0;  // stages and plane buffers issued
     if (lane == 0) {
-      for (int q = max(0, n - kDecStages); q < n; ++q) {
-        const uint32_t full = full0 + 8 * (q % kDecStages);
-        const long long t0 = clock64();
-        while (!dec_try_wait(full, (q / kDecStages) & 1) && clock64() - t0 < kDecWaitCycles) {
-        }
-      }
-    }
-  } else {
-    // ============================================================ consumers
-    const int g = lane >> 2, t4 = lane & 3;
-    int n = 0;
-    for (int ui = blockIdx.x; ui < n_units; ui += p.G) {
-      const DecUnit U = dec_unit(p, R.groups, nsg, nrg, ui);
-      const int4 grp = R.groups[U.grp];
-      const DecMat& m0 = p.m[U.mi];
-      DecStageCtx c;
-      // S1: 2 row tiles x 8 input slices; S2: 4 row tiles x 4 input slices
-      c.rt = U.M == 2 ? (warp & 1) : (warp & 3);
-      c.kq = U.M == 2 ? (warp >> 1) : (warp >> 2);
-      c.ntok = grp.z;
-      c.group = m0.group;
-      c.ks = m0.ks;
-      c.rows = m0.rows;
-      const int fmt = m0.fmt;
-      for (int half = 0; half < U.nhalf; ++half) {
-        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-        for (int kc = 0; kc < U.nchunks; ++kc, ++n) {
-          const int s = n % kDecStages;
-          const uint32_t full = full0 + 8 * s;
-          bool have = !*abort_flag;
-          if (have && !dec_wait_bar(full, (n / kDecStages) & 1, abort_flag)) {
+      for (int ui = blockIdx.x; ui < n_units && !*abort_flag; ui += p.G) {
+        const DecUnit U = dec_unit(p, r_groups, nsg, nrg, ui);
+        const int4 grp = r_groups[U.grp];
+        const DecMat& m0 = p.m[U.mi];
+        const bool s1 = U.stage == 1;
+        const bool mx = m0.fmt == F_MX4;
+        const int nsb = mx ? 1 : 2;
+        const uint32_t box_bytes = (uint32_t)(m0.R * m0.seg);
+        const uint32_t sc_bytes = (uint32_t)(m0.R * m0.spitch);
+        const uint32_t tx = (s1 ? 2u : 1u) * (box_bytes + sc_bytes * nsb);
+        if (!s1) {
+          // W2 stages read the group's h planes: wait for all its S1 units
+          const int target = p.stall_test ? 0x3fffffff : (grp.x < 0 ? p.fs / kDecRows : p.f / kDecRows);
+          if (!dec_wait_count(p.cnt_h + U.grp, target, abort_flag, p.stall_test ? 2000000LL : kDecWaitCycles)) {
             set_error(p.err, kErrTimeout);
             *abort_flag = 1;
-            have = false;
+            break;
           }
-          have = __all_sync(0xffffffffu, have);  // the MMAs below need every lane
-          if (have) {
-            c.slot = su32(ring + (size_t)s * kDecSlotBytes);
-            dec_stage_any(fmt, U.M, c, acc);
-          }
-          __syncwarp();
-          if (lane == 0 && have) dec_arrive(empty0 + 8 * s);
+          fence_proxy_async_global();
         }
-        // ---- sum the input slices of every (row, token) of this half
-#pragma unroll
-        for (int m = 0; m < 2; ++m) {
-          if (m < U.M) {
-            float* dst = red + ((warp * 2 + m) * 16) * 8;
-            dst[g * 8 + 2 * t4] = acc[m][0];
-            dst[g * 8 + 2 * t4 + 1] = acc[m][1];
-            dst[(g + 8) * 8 + 2 * t4] = acc[m][2];
-            dst[(g + 8) * 8 + 2 * t4 + 1] = acc[m][3];
-          }
-        }
-        asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
         {
-          const int nrt = U.M == 2 ? 2 : 4, nkq = kDecConsumerWarps / nrt;
-          const int row = tid >> 3, tok = tid & 7;  // S1: rows 0..31 (tid < 256); S2: rows 0..63
-          if (row < nrt * 16 && tok < grp.z) {
-            const int rtt = row >> 4, rl = row & 15;
-            float v[2] = {0.f, 0.f};
-            for (int q = 0; q < nkq; ++q)
-              for (int m = 0; m < U.M; ++m) v[m] += red[(((q * nrt + rtt) * 2 + m) * 16 + rl) * 8 + tok];
-            if (U.stage == 1) {
-              hbuf[tok * kDecRows + half * 32 + row] = v[0] / (1.f + expf(-v[0])) * v[1];  // silu(g) * u
+          // the unit's activation rows (planes and block records) for every token of the group
+          const int pb = np & 1;
+          if (np >= 2 && !dec_wait_bar(pempty0 + 8 * pb, ((np >> 1) - 1) & 1, abort_flag)) {
+            set_error(p.err, kErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          const uint32_t pl = planes0 + pb * p.pbuf;
+          const int nin = m0.n_in;
+          dec_expect_tx(pfull0 + 8 * pb, (uint32_t)grp.z * (uint32_t)(nin * 2 + (nin / 64) * 16));
+          for (int i = 0; i < grp.z; ++i) {
+            const uint8_t* src;
+            const float4* ssrc;
+            if (s1) {
+              const int tok = dec_token(p, r_sorted, grp, i);
+              src = p.xplanes + ((size_t)(grp.x < 0 ? 1 : 0) * T + tok) * d * 4;
+              ssrc = p.xsx + (size_t)tok * (d / 64);
             } else {
-              const int sl = dec_slot(p, R, grp, tok);
-              p.y[(size_t)sl * d + kDecRows * U.u + row] = v[0];
+              const int sl = dec_slot(p, r_sorted, grp, i);
+              src = p.hplanes + (size_t)sl * fmax * 4;
+              ssrc = p.hsx + (size_t)sl * (fmax / 64);
+            }
+            dec_bulk(pl + i * m0.ptok, src, nin * 2, pfull0 + 8 * pb);
+            dec_bulk(pl + p.sx_off + i * m0.sxtok, ssrc, (nin / 64) * 16, pfull0 + 8 * pb);
+          }
+          ++np;
+        }
+        const int nrs = s1 ? kDecRows / kDecR1 : kDecRows / kDecR2;
+        for (int rs = 0; rs < nrs && !*abort_flag; ++rs) {
+          for (int chn = 0; chn < m0.nch; ++chn, ++n) {
+            const int s = n % p.nslot;
+            if (n >= p.nslot && !dec_wait_bar(empty0 + 8 * s, ((n / p.nslot) - 1) & 1, abort_flag)) {
+              set_error(p.err, kErrTimeout);
+              *abort_flag = 1;
+              break;
+            }
+            const uint32_t slot = ring + s * p.slot_bytes, full = full0 + 8 * s;
+            const int row = U.row0 + rs * m0.R;
+            const int cx = chn * (m0.seg / m0.lb);
+            const int sxe = chn * m0.sK;
+            dec_expect_tx(full, tx);
+            for (int mm = 0; mm < (s1 ? 2 : 1); ++mm) {
+              const int mi = U.mi + mm;
+              dec_tma_3d(slot + mm * box_bytes, &p.map[mi], 0, row, cx, full);
+              const uint32_t sb = slot + kDecCodeBytes + mm * nsb * sc_bytes;
+              dec_tma_2d(sb, &p.smap[mi], sxe, row, full);
+              if (!mx) dec_tma_2d(sb + sc_bytes, &p.bmap[mi], sxe, row, full);
             }
           }
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
       }
-      if (U.stage == 1) {
-        // h of each token over these 64 rows -> one 64-input block of W2's planes
-        if (warp < grp.z) {
-          const int sl = dec_slot(p, R, grp, warp);
-          const int f2 = grp.x < 0 ? p.m[DM_S2].fmt : p.m[DM_W2].fmt;
-          const int pb = plane_bytes_per_input(f2);
-          uint8_t* dst = p.hplanes + (size_t)sl * fmax * 4 + (size_t)U.u * 64 * pb;
-          const float4 sx = dec_make_block(hbuf[warp * kDecRows + 2 * lane], hbuf[warp * kDecRows + 2 * lane + 1],
-                                           perm_of(f2), f2 == F_MX4, dst, reinterpret_cast<int*>(red) + warp * 64,
-                                           p.err);
+      // drain: every issued copy must land before the block exits
+      for (int q = max(0, n - p.nslot); q < n; ++q) {
+        const long long t0 = clock64();
+        while (!dec_try_wait(full0 + 8 * (q % p.nslot), (q / p.nslot) & 1) && clock64() - t0 < kDecWaitCycles) {
+        }
+      }
+      for (int q = max(0, np - 2); q < np; ++q) {
+        const long long t0 = clock64();
+        while (!dec_try_wait(pfull0 + 8 * (q & 1), (q >> 1) & 1) && clock64() - t0 < kDecWaitCycles) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kDecServiceWarp) {
+    // ============================================================ service
+    // Unit epilogues that wait on global memory, off the consumers' path:
+    // S1: the h block of every token -> W2's planes, then the group's count;
+    // S2: the output block's count, and the combine by its last arriver.
+    int* scr = reinterpret_cast<int*>(fx + kDecFxScr);
+    int ne = 0;
+    for (int ui = blockIdx.x; ui < n_units; ui += p.G, ++ne) {
+      const DecUnit U = dec_unit(p, r_groups, nsg, nrg, ui);
+      const int4 grp = r_groups[U.grp];
+      const int eb = ne & 1;
+      bool ok = !*abort_flag;
+      if (ok && !dec_wait_bar(efull0 + 8 * eb, (ne >> 1) & 1, abort_flag)) {
+        if (lane == 0) set_error(p.err, kErrTimeout);
+        *abort_flag = 1;
+        ok = false;
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok && U.stage == 1) {
+        const float* hb = hbuf + eb * kDecMaxTok * kDecRows;
+        const int f2 = grp.x < 0 ? p.m[DM_S2].fmt : p.m[DM_W2].fmt;
+        for (int i = 0; i < grp.z; ++i) {
+          const int sl = dec_slot(p, r_sorted, grp, i);
+          uint8_t* dst = p.hplanes + (size_t)sl * fmax * 4 + (size_t)U.u * 64 * plane_bytes_per_input(f2);
+          const float4 sx = dec_make_block(hb[i * kDecRows + 2 * lane], hb[i * kDecRows + 2 * lane + 1], perm_of(f2),
+                                           dst, scr, p.err);
           if (lane == 0) p.hsx[(size_t)sl * (fmax / 64) + U.u] = sx;
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
-        if (tid == 0) {
+        __syncwarp();
+        if (lane == 0) {
           __threadfence();
           red_release_add(p.cnt_h + U.grp, 1);
         }
-      } else {
-        if (tid == 0) {
+      } else if (ok) {
+        int last = 0;
+        if (lane == 0) {
           __threadfence();
-          const int done = atomicAdd(p.cnt_y + U.u, 1) + 1;
-          const int last = done == nsg + nrg;
+          last = atomicAdd(p.cnt_y + U.u, 1) + 1 == nsg + nrg;
           if (last) __threadfence();
-          misc[3] = last;
         }
-        asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
-        if (misc[3]) {
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
           // every slot of this 64-column block is final: out = sum_j w y (+ shared), one rounding
-          for (int i = tid; i < T * kDecRows; i += kDecConsumerWarps * 32) {
+          for (int i = lane; i < T * kDecRows; i += 32) {
             const int t = i / kDecRows, col = kDecRows * U.u + (i % kDecRows);
             float sacc = 0.f;
-            for (int j = 0; j < k; ++j) sacc = fmaf(R.w[t * k + j], __ldcg(p.y + (size_t)(t * k + j) * d + col), sacc);
+            for (int j = 0; j < k; ++j) sacc = fmaf(r_w[t * k + j], __ldcg(p.y + (size_t)(t * k + j) * d + col), sacc);
             if (p.has_shared) sacc += __ldcg(p.y + (size_t)(Tk + t) * d + col);
             p.out[(size_t)t * d + col] = __float2bfloat16_rn(sacc);
           }
-          asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerWarps * 32) : "memory");
-          if (tid == 0) p.cnt_y[U.u] = 0;
+          __syncwarp();
+          if (lane == 0) p.cnt_y[U.u] = 0;
         }
       }
+      __syncwarp();
+      if (lane == 0) dec_arrive(eempty0 + 8 * eb);
+    }
+  } else {
+    // ============================================================ consumers
+    const int tt = warp & 1, kq = warp >> 1;  // row tile, input slice
+    int n = 0, np = 0, ne = 0;
+    for (int ui = blockIdx.x; ui < n_units; ui += p.G, ++ne) {
+      const DecUnit U = dec_unit(p, r_groups, nsg, nrg, ui);
+      const int4 grp = r_groups[U.grp];
+      const DecMat& m0 = p.m[U.mi];
+      const bool s1 = U.stage == 1;
+      DecWarp q;
+      const int nsb = m0.fmt == F_MX4 ? 1 : 2;
+      q.R = m0.R;
+      q.nbw = m0.nbw;
+      q.kq = kq;
+      q.gshift = m0.gshift;
+      q.spitch = m0.spitch;
+      q.brow = m0.R * m0.spitch;
+      q.ptok = m0.ptok;
+      q.sxtok = m0.sxtok;
+      if (s1) {  // A rows 0..7: W1 rows tt*8.., rows 8..15: the same rows of W3
+        q.a0 = 0;
+        q.a8 = m0.R * m0.seg;
+        q.r0 = q.r8 = tt * 8;
+        q.s0 = kDecCodeBytes;
+        q.s8 = kDecCodeBytes + nsb * m0.R * m0.spitch;
+      } else {  // A rows 0..15: W2 rows tt*16..
+        q.a0 = q.a8 = 0;
+        q.r0 = tt * 16;
+        q.r8 = tt * 16 + 8;
+        q.s0 = q.s8 = kDecCodeBytes;
+      }
+      const int pb = np & 1;
+      const bool have_pl = dec_consumer_wait(pfull0 + 8 * pb, (np >> 1) & 1, abort_flag, p.err);
+      const uint32_t pl = planes0 + pb * p.pbuf;
+      if (s1)
+        dec_consume_any<true>(m0.fmt, q, m0.nch, m0.K, grp.z, ring, p.slot_bytes, p.nslot, pl, pl + p.sx_off, zb,
+                              full0, empty0, n, have_pl, abort_flag, p.err, red, tt);
+      else
+        dec_consume_any<false>(m0.fmt, q, m0.nch, m0.K, grp.z, ring, p.slot_bytes, p.nslot, pl, pl + p.sx_off, zb,
+                               full0, empty0, n, have_pl, abort_flag, p.err, red, tt);
+      __syncwarp();
+      if (lane == 0 && have_pl) dec_arrive(pempty0 + 8 * pb);
+      ++np;
+      // this unit's epilogue buffer must be free (the service warp is done with unit ne - 2)
+      const int eb = ne & 1;
+      bool have_e = true;
+      if (ne >= 2) have_e = dec_consumer_wait(eempty0 + 8 * eb, ((ne >> 1) - 1) & 1, abort_flag, p.err);
+      asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerThreads) : "memory");  // every slice partial is in red
+      if (tid < kDecMaxTok * kDecRows) {
+        const int r = tid >> 2, tok = tid & 3;  // the unit's output row, token
+        if (tok < grp.z) {
+          if (s1) {
+            const int rs = r >> 4, row = r & 15;
+            float v1 = 0.f, v3 = 0.f;
+#pragma unroll
+            for (int sl = 0; sl < kDecNkq; ++sl) {  // input slices in a fixed order
+              const float2 pr = *reinterpret_cast<const float2*>(red + ((sl * 4 + rs) * 16 + row) * 8 + tok * 2);
+              v1 += pr.x;
+              v3 += pr.y;
+            }
+            if (have_e) hbuf[(eb * kDecMaxTok + tok) * kDecRows + r] = v1 / (1.f + expf(-v1)) * v3;  // silu(g) * u
+          } else {
+            const int rs = r >> 5, row = r & 31;
+            float v = 0.f;
+#pragma unroll
+            for (int sl = 0; sl < kDecNkq; ++sl) v += red[((sl * 2 + rs) * 32 + row) * 4 + tok];  // fixed order
+            p.y[(size_t)dec_slot(p, r_sorted, grp, tok) * d + kDecRows * U.u + r] = v;
+          }
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerThreads) : "memory");  // red is free, the h block complete
+      if (lane == 0) dec_arrive(efull0 + 8 * eb);
     }
   }
   // ------------------------------------------------------------ exit

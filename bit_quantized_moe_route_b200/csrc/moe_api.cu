@@ -274,9 +274,9 @@ moe_status_t dev_info(DevInfo** out) {
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, ffn_gemv_kernel<2, 8>, kFfnThreads, 0);
       di.ffn1_blocks = std::max(1, b1);
       di.ffn2_blocks = std::max(1, b2);
-      cudaFuncSetAttribute(ffn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmem);
+      cudaFuncSetAttribute(ffn_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmemMax);
       int bd = 0;
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bd, ffn_decode_kernel, kDecThreads, kDecSmem);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bd, ffn_decode_kernel, kDecThreads, kDecSmemMax);
       di.dec_blocks = std::min(bd, 1) * di.sms;
       cudaError_t le = cudaGetLastError();
       if (le != cudaSuccess) {
@@ -805,35 +805,87 @@ moe_status_t launch_ffn(const moe_dims_t& d, const void* x, const int* offsets, 
 }
 
 // ---------------------------------------------------------------- fused small-batch layer
-// Stage geometry of a packed matrix in the fused kernel: 512 code bytes per
-// row and stage (3-bit: 384) as four 128-byte swizzled (3-bit: 96-byte
-// unswizzled) TMA boxes; W1/W3 stages carry 32 rows, W2 stages 64.
+// Stage geometry of a packed matrix in the fused kernel: up to 1024 code
+// bytes of every row per stage (3-bit: 768), as one chunk-major 3-D TMA box
+// of 16 (W1, W3) or 32 (W2) rows; 8 consumer slices of whole 64-input blocks.
 bool dec_mat(const QMatDev& Q, bool w2, DecMat* m) {
   m->fmt = Q.fmt;
   m->group = Q.group;
   m->n_out = Q.n_out;
   m->n_in = Q.n_in;
-  m->rows = w2 ? 64 : 32;
-  m->box = Q.fmt == F_A3 ? 96 : 128;
   const int bits = Q.fmt == F_A2 ? 2 : Q.fmt == F_A3 ? 3 : Q.fmt == F_A8 ? 8 : 4;
-  m->ks = 4 * m->box * 8 / bits;
-  const int esz = Q.fmt == F_MX4 ? 1 : 2;
-  m->sbytes = m->ks / Q.group * esz;
-  if (Q.n_in % m->ks || Q.n_out % 64) return false;
+  const int row_bytes = Q.wpr * 4;
+  m->R = w2 ? kDecR2 : kDecR1;
+  m->lb = Q.fmt == F_A3 ? 96 : 128;
+  m->seg = std::min(row_bytes, Q.fmt == F_A3 ? 768 : kDecMaxSeg);
+  if (row_bytes <= 0 || m->seg % m->lb || row_bytes % m->seg) return false;
+  if (row_bytes * 8 != Q.n_in * bits) return false;  // rows packed without padding
+  m->nch = row_bytes / m->seg;
+  m->K = m->seg * 8 / bits;
+  if (m->K % (64 * kDecNkq)) return false;  // input slices of whole 64-input blocks
+  m->nbw = m->K / (64 * kDecNkq);
+  if (m->nbw & (m->nbw - 1)) return false;  // rounds of 1, 2 or 4 fold units tile the slice
+  if (Q.group != 32 && Q.group != 64 && Q.group != 128) return false;
   if (Q.fmt == F_A2 && Q.group == 32) return false;  // a 2-bit k-block mixes two 32-input groups
-  if (m->sbytes != 16 && m->sbytes != 32 && m->sbytes != 64) return false;  // TMA box of scales
-  if ((Q.gpr * esz) % 16 || (Q.wpr * 4) % 16) return false;                 // TMA row strides
+  if (m->K % Q.group) return false;
+  m->gshift = Q.group == 32 ? -1 : Q.group == 64 ? 0 : 1;
+  m->sK = m->K / Q.group;
+  const int esz = Q.fmt == F_MX4 ? 1 : 2;
+  const int sbytes = m->sK * esz;
+  if (sbytes % 16) return false;          // TMA box of scales
+  if ((Q.gpr * esz) % 16) return false;   // TMA row stride of scales
+  // scale rows land at an odd multiple of 16 bytes apart: the 8 rows a fold reads hit distinct banks
+  m->spitch = (sbytes / 16) % 2 ? sbytes : sbytes + 16;
+  if (m->spitch / esz > 256) return false;
+  if (Q.n_out % kDecRows) return false;
+  m->ptok = Q.n_in * 2 + 64;        // = 64 mod 128: token j and j+1 of a B load use different banks
+  m->sxtok = Q.n_in / 64 * 16 + 16;  // = 16 mod 128: the four tokens of a record load use different banks
+  return true;
+}
+
+// Shared-memory plan of one launch: ring slots, plane buffers.  False when
+// the shapes do not fit the fused kernel.
+bool dec_plan(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh,
+              DecParams* p, size_t* smem) {
+  if (d.T < 1 || d.T > kDecMaxT || d.T * d.top_k > kDecMaxPairs || d.n_experts > kDecMaxE) return false;
+  // d_model a multiple of 128: the logit pass gives each lane 8 consecutive inputs of a 1/8 slice
+  if (d.d_model % 128 || d.d_ff % kDecRows || (sh && d.d_ff_shared % kDecRows)) return false;
+  const QMatDev* mats[6] = {&w1, &w3, &w2, sh ? &sh[0] : &w1, sh ? &sh[1] : &w3, sh ? &sh[2] : &w2};
+  DecMat m[6];
+  for (int i = 0; i < 6; ++i)
+    if (!dec_mat(*mats[i], i % 3 == 2, &m[i])) return false;
+  for (int b = 0; b < 6; b += 3)  // W1 and W3 of an expert stream side by side
+    if (m[b].fmt != m[b + 1].fmt || m[b].group != m[b + 1].group || m[b].seg != m[b + 1].seg ||
+        m[b].n_in != m[b + 1].n_in || m[b].n_out != m[b + 1].n_out)
+      return false;
+  const int ntmax = std::min(kDecMaxTok, d.hash_mode ? d.T * d.top_k : d.T);
+  int pst = 0, sxs = 0, sc = 0;
+  for (int i = 0; i < 6; ++i) {
+    pst = std::max(pst, m[i].ptok);
+    sxs = std::max(sxs, m[i].sxtok);
+    const int nsb = m[i].fmt == F_MX4 ? 1 : 2;
+    sc = std::max(sc, (i % 3 == 2 ? 1 : 2) * nsb * m[i].R * m[i].spitch);
+  }
+  const int sx_off = ntmax * pst;
+  const int pbuf = (sx_off + ntmax * sxs + 127) / 128 * 128;
+  const int slot_bytes = kDecCodeBytes + (sc + 1023) / 1024 * 1024;
+  const long avail = (long)kDecSmemMax - 1024 - kDecFixedBytes - 2L * pbuf;
+  const int nslot = (int)std::min<long>(kDecSlotCap, avail / slot_bytes);
+  if (nslot < 2) return false;
+  if (p) {
+    for (int i = 0; i < 6; ++i) p->m[i] = m[i];
+    p->nslot = nslot;
+    p->slot_bytes = slot_bytes;
+    p->pbuf = pbuf;
+    p->sx_off = sx_off;
+    p->ntmax = ntmax;
+  }
+  if (smem) *smem = 1024 + (size_t)nslot * slot_bytes + 2 * (size_t)pbuf + kDecFixedBytes;
   return true;
 }
 
 bool dec_eligible(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh) {
-  if (d.T > kDecMaxT || d.T * d.top_k > kDecMaxPairs || d.n_experts > 1024) return false;
-  // d_model a multiple of 128: the logit pass gives each lane 8 consecutive inputs of a 1/16 slice
-  if (d.d_model % 128 || d.d_ff % 64 || (sh && d.d_ff_shared % 64)) return false;
-  DecMat m;
-  if (!dec_mat(w1, false, &m) || !dec_mat(w3, false, &m) || !dec_mat(w2, true, &m)) return false;
-  if (sh && (!dec_mat(sh[0], false, &m) || !dec_mat(sh[1], false, &m) || !dec_mat(sh[2], true, &m))) return false;
-  return true;
+  return dec_plan(d, w1, w3, w2, sh, nullptr, nullptr);
 }
 
 bool use_dec(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh) {
@@ -842,19 +894,37 @@ bool use_dec(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, const QM
   return dec_eligible(d, w1, w3, w2, sh);
 }
 
+// Codes as a chunk-major 3-D view: (line of lb bytes, row, line index within
+// the row), so a box of R rows x C lines lands as [line][row][lb].
+moe_status_t tmap_rows_3d(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t row_bytes, uint32_t lb,
+                          uint32_t R, uint32_t C) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[3] = {lb, rows, row_bytes / lb};
+  const cuuint64_t strides[2] = {row_bytes, lb};
+  const cuuint32_t box[3] = {lb, R, C};
+  const cuuint32_t es[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, es,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, lb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled (3-D rows) failed (%d)", (int)r);
+  return MOE_OK;
+}
+
 moe_status_t dec_maps(DecParams& p, int i, const QMatDev& Q, int E) {
   const DecMat& m = p.m[i];
   const uint64_t rows = (uint64_t)E * Q.n_out;
-  moe_status_t st = tmap_2d(&p.map[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.q, (uint64_t)Q.wpr * 4, rows,
-                            (uint64_t)Q.wpr * 4, m.box, m.rows, Q.fmt != F_A3);
+  moe_status_t st = tmap_rows_3d(&p.map[i], Q.q, rows, (uint64_t)Q.wpr * 4, m.lb, m.R, m.seg / m.lb);
   if (st != MOE_OK) return st;
+  // scale boxes are spitch bytes wide: the stage's scales plus padding (the
+  // next stage's scales, or zero fill past the row end)
   if (Q.fmt == F_MX4)
-    return tmap_2d(&p.smap[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.scales, Q.gpr, rows, Q.gpr, m.sbytes, m.rows, false);
-  st = tmap_2d(&p.smap[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q.scales, Q.gpr, rows, (uint64_t)Q.gpr * 2, m.sbytes / 2,
-               m.rows, false);
+    return tmap_2d(&p.smap[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, Q.scales, Q.gpr, rows, Q.gpr, m.spitch, m.R, false);
+  st = tmap_2d(&p.smap[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q.scales, Q.gpr, rows, (uint64_t)Q.gpr * 2,
+               m.spitch / 2, m.R, false);
   if (st != MOE_OK) return st;
   return tmap_2d(&p.bmap[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q.biases, Q.gpr, rows, (uint64_t)Q.gpr * 2,
-                 m.sbytes / 2, m.rows, false);
+                 m.spitch / 2, m.R, false);
 }
 
 moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32_t* token_ids, const void* router_w,
@@ -862,9 +932,10 @@ moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32
                                  const QMatDev& q2, const QMatDev* qs, void* out, int32_t* ids_out, float* w_out,
                                  void* ws, const WsLayout& L, cudaStream_t s, const DevInfo& di) {
   DecParams p{};
+  size_t smem = 0;
+  if (!dec_plan(d, q1, q3, q2, qs, &p, &smem)) return fail(MOE_ERR_UNSUPPORTED, "shapes outside the fused kernel");
   const QMatDev* mats[6] = {&q1, &q3, &q2, qs ? &qs[0] : &q1, qs ? &qs[1] : &q3, qs ? &qs[2] : &q2};
   for (int i = 0; i < 6; ++i) {
-    dec_mat(*mats[i], i % 3 == 2, &p.m[i]);
     moe_status_t st = dec_maps(p, i, *mats[i], (i < 3 || !qs) ? d.n_experts : 1);
     if (st != MOE_OK) return st;
   }
@@ -906,7 +977,7 @@ moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.G);
   cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = kDecSmem;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
