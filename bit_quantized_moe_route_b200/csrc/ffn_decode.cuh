@@ -76,8 +76,7 @@ constexpr int kDecMaxGroups = kDecMaxPairs + 8;
 // fixed shared region (after the ring and the two plane buffers), byte offsets
 constexpr int kDecFxRed = 0;
 constexpr int kDecFxH = kDecFxRed + kDecRedFloats * 4;           // 2 buffers x 4 tokens x 64 h values
-constexpr int kDecFxZero = kDecFxH + 2 * kDecMaxTok * kDecRows * 4;  // 256 zero bytes (dead B columns)
-constexpr int kDecFxScr = kDecFxZero + 256;                      // the service warp's scratch (64 ints)
+constexpr int kDecFxScr = kDecFxH + 2 * kDecMaxTok * kDecRows * 4;  // the service warp's scratch (64 ints)
 constexpr int kDecFxIds = kDecFxScr + 256;
 constexpr int kDecFxW = kDecFxIds + kDecMaxPairs * 4;
 constexpr int kDecFxSorted = kDecFxW + kDecMaxPairs * 4;
@@ -99,8 +98,7 @@ struct DecMat {
   int seg;     // code bytes per row and stage (a multiple of lb)
   int nch;     // stages along a row (row bytes / seg)
   int K;       // inputs per stage
-  int nbw;     // 64-input blocks per consumer warp and stage (K / 256)
-  int gshift;  // log2(group / 64) for groups of 64 or 128; -1 for 32
+  int nbw;     // 64-input blocks per consumer warp and stage (K / 512)
   int sK;      // scale entries per row and stage
   int spitch;  // bytes per row of a scale box: the stage's scales padded to an odd multiple of 16
   int ptok;    // plane bytes per token in a plane buffer (n_in * 2, bank-padded)
@@ -269,159 +267,180 @@ MOE_DEV uint32_t codes3x8(uint32_t line, int off, int t) {
 }
 
 // ------------------------------------------------------------ one stage
-// What a consumer warp needs to address its tile in any stage of a unit.
-// Shared addresses are relative to the stage slot.  A rows 0..7 of the tile
+// What a consumer warp needs to address its tile in any stage of a unit
+// (shared addresses relative to the stage slot).  A rows 0..7 of the tile
 // live in code box `a0` at box rows r0..r0+7, A rows 8..15 in box `a8` at
-// rows r8..r8+7; their scales in scale boxes `s0` / `s8` (biases `brow`
+// rows r8..r8+7; their scales in scale boxes `s0` / `s8` (biases R * spitch
 // bytes further).
 struct DecWarp {
   uint32_t a0, a8, s0, s8;
   int r0, r8;
-  int R;       // rows per box
-  int nbw;     // 64-input blocks of this warp per stage
-  int kq;      // input slice
-  int gshift;  // log2(group / 64), -1 for 32-input groups
-  int spitch, brow;
+  int R;   // rows per box
+  int kq;  // input slice
+  int spitch;
   int ptok, sxtok;
 };
+
+// Per-lane constants of a consumer warp for every stage of one unit.  All
+// per-block offsets inside a stage are then compile-time immediates.
+struct DecLane {
+  uint32_t la;    // slot-relative ldmatrix row address of this lane (its A row, the slice's 128-byte line)
+  uint32_t ly;    // XOR applied to the 16-byte chunk offset (the 128-byte swizzle and the chunk pair)
+  uint32_t l3a, l3b;  // 3-bit: slot-relative address of this thread's codes of A rows g and g+8
+  uint32_t sh3;   // 3-bit: bit offset of those codes in the loaded pair of words
+  uint32_t b;     // plane-buffer-relative B address (token row, quad thread, plane)
+  uint32_t sx;    // record-relative address (token, the slice's first block)
+  uint32_t s0, s8, brow;  // slot-relative scale addresses of A rows g / g+8 (the slice's first group), bias offset
+};
+
+
+// Lanes whose B column or C column pair belongs to a token past the group
+// read another token's data: those columns are never read back.
+template <int FMT, int G, int NBW>
+MOE_DEV DecLane dec_lane(const DecWarp& q, int ntok) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int mtx = lane >> 3, lr = lane & 7, csel = mtx >> 1;
+  const uint32_t box = (mtx & 1) ? q.a8 : q.a0;
+  const int row = ((mtx & 1) ? q.r8 : q.r0) + lr;
+  const int bs0 = q.kq * NBW;  // the slice's first block in the stage
+  DecLane L;
+  int line = 0, mk = 0;
+  if constexpr (FMT == F_A4 || FMT == F_MX4) {  // 32 bytes per block: 4 blocks per line, 2 chunks each
+    line = bs0 >> 2;
+    mk = bs0 & 3;
+    L.ly = (uint32_t)(((2 * mk) ^ csel ^ lr) << 4);
+  } else if constexpr (FMT == F_A8) {  // 64 bytes per block: 2 blocks (4 k-blocks of 2 chunks) per line
+    line = (2 * bs0) >> 2;
+    mk = (2 * bs0) & 3;
+    L.ly = (uint32_t)(((2 * mk) ^ csel ^ lr) << 4);
+  } else if constexpr (FMT == F_A2) {  // 16 bytes per block: 8 blocks per line
+    line = bs0 >> 3;
+    mk = bs0 & 7;
+    L.ly = (uint32_t)((mk ^ lr) << 4);
+  } else {
+    L.ly = 0;
+  }
+  L.la = box + (uint32_t)((line * q.R + row) * 128);
+  if constexpr (FMT == F_A3) {  // 24 bytes per block in 96-byte lines
+    const int by = bs0 * 24, ln = by / 96, off = by - ln * 96 + ((3 * t) & ~3);
+    L.l3a = q.a0 + (uint32_t)((ln * q.R + q.r0 + g) * 96 + off);
+    L.l3b = q.a8 + (uint32_t)((ln * q.R + q.r8 + g) * 96 + off);
+    L.sh3 = 8 * ((3 * t) & 3);
+  } else {
+    L.l3a = L.l3b = L.sh3 = 0;
+  }
+  const int jb = min(g >> 1, ntok - 1), jc = min(t, ntok - 1);
+  L.b = (uint32_t)(jb * q.ptok + bs0 * 128 + t * 16 + (g & 1) * 8);
+  L.sx = (uint32_t)(jc * q.sxtok + bs0 * 16);
+  const int esz = FMT == F_MX4 ? 1 : 2;
+  const int gbase = G == 32 ? 2 * bs0 : (bs0 * 64) / G;
+  L.s0 = q.s0 + (uint32_t)((q.r0 + g) * q.spitch + esz * gbase);
+  L.s8 = q.s8 + (uint32_t)((q.r8 + g) * q.spitch + esz * gbase);
+  L.brow = (uint32_t)(q.R * q.spitch);
+  return L;
+}
 
 // acc[0] (A row g) and acc[1] (A row g+8) of token t += s_r * st * P + b_r * sm
 // over one scale group: P = 256 * C[., 2t] + C[., 2t+1] is the exact
 // integer sum of codes x fixed-point inputs, st the inputs' step, sm their
-// dequantised sum; `gi`: the group's scale entry in the stage.
-template <int FMT>
-MOE_DEV void dec_fold(const DecWarp& q, uint32_t slot, float st, float sm, int gi, const int (&c)[4],
+// dequantised sum; GI: the group's scale entry relative to the slice.
+template <int FMT, int GI>
+MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, float st, float sm, const int (&c)[4],
                       float (&acc)[2]) {
-  const int g = (threadIdx.x & 31) >> 2;
-  const uint32_t sc0 = slot + q.s0 + (q.r0 + g) * q.spitch, sc8 = slot + q.s8 + (q.r8 + g) * q.spitch;
-  float s0, b0, s8, b8;
+  float sc0, b0, sc8, b8;
   if constexpr (FMT == F_MX4) {
     // 2^(e-127) / 2 (the A operand holds 2*e2m1)
-    const uint32_t e0 = lds8u(sc0 + gi), e8 = lds8u(sc8 + gi);
-    s0 = __uint_as_float(e0 > 1 ? ((e0 - 1) << 23) : (e0 ? 0x00400000u : 0x00200000u));
-    s8 = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));
+    const uint32_t e0 = lds8u(s0 + GI), e8 = lds8u(s8 + GI);
+    sc0 = __uint_as_float(e0 > 1 ? ((e0 - 1) << 23) : (e0 ? 0x00400000u : 0x00200000u));
+    sc8 = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));
     b0 = b8 = 0.f;
   } else {
-    s0 = bf16_bits_to_float(lds16u(sc0 + 2 * gi));
-    b0 = bf16_bits_to_float(lds16u(sc0 + q.brow + 2 * gi));
-    s8 = bf16_bits_to_float(lds16u(sc8 + 2 * gi));
-    b8 = bf16_bits_to_float(lds16u(sc8 + q.brow + 2 * gi));
+    sc0 = bf16_bits_to_float(lds16u(s0 + 2 * GI));
+    b0 = bf16_bits_to_float(lds16u(s0 + brow + 2 * GI));
+    sc8 = bf16_bits_to_float(lds16u(s8 + 2 * GI));
+    b8 = bf16_bits_to_float(lds16u(s8 + brow + 2 * GI));
   }
-  acc[0] = fmaf(s0 * st, (float)(c[0] * 256 + c[1]), fmaf(b0, sm, acc[0]));
-  acc[1] = fmaf(s8 * st, (float)(c[2] * 256 + c[3]), fmaf(b8, sm, acc[1]));
+  acc[0] = fmaf(sc0 * st, (float)(c[0] * 256 + c[1]), fmaf(b0, sm, acc[0]));
+  acc[1] = fmaf(sc8 * st, (float)(c[2] * 256 + c[3]), fmaf(b8, sm, acc[1]));
 }
 
-// Column pairs a fold unit of a group of ntok tokens occupies: 1, 2 or 4.
-MOE_DEV int dec_ntp(int ntok) { return ntok == 1 ? 1 : ntok == 2 ? 2 : 4; }
+// k-block H of block B of the warp's slice: A fragment, one MMA (two for
+// mxfp4: positive and negative magnitudes), with B from the plane buffer.
+template <int FMT, int B, int H>
+MOE_DEV void dec_kblock(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, const uint32_t (&w)[4], int (&c)[4],
+                        int (&cn)[4]) {
+  const uint2 bv = lds64u(bp + B * 128 + H * 64);
+  uint32_t a[4];
+  if constexpr (FMT == F_A4) {
+    unpack_a4(w[2 * H], w[2 * H + 1], a);
+  } else if constexpr (FMT == F_MX4) {
+    uint32_t an[4];
+    unpack_mx4(w[2 * H], w[2 * H + 1], a, an);
+    mma_u8s8(cn, an, bv.x, bv.y);
+  } else if constexpr (FMT == F_A8) {  // a k-block is two chunks of the line
+    ldsm_x4(la + ((uint32_t)((4 * B + 2 * H) << 4) ^ L.ly), a[0], a[1], a[2], a[3]);
+  } else if constexpr (FMT == F_A2) {
+    unpack_a2(w[0], w[1], H, a);
+  } else {  // 3-bit: 12-byte k-blocks, this thread's 8 codes of rows g and g+8
+    const uint32_t pa = sl + L.l3a + (2 * B + H) * 12, pb = sl + L.l3b + (2 * B + H) * 12;
+    const uint32_t v0 = __funnelshift_r(lds32u(pa), lds32u(pa + 4), L.sh3) & 0xFFFFFFu;
+    const uint32_t v8 = __funnelshift_r(lds32u(pb), lds32u(pb + 4), L.sh3) & 0xFFFFFFu;
+    a[0] = spread3x4(v0 & 0xFFFu);
+    a[2] = spread3x4(v0 >> 12);
+    a[1] = spread3x4(v8 & 0xFFFu);
+    a[3] = spread3x4(v8 >> 12);
+  }
+  mma_u8s8(c, a, bv.x, bv.y);
+}
 
-// The warp's input slice of one stage.  The MMA has 4 column pairs (hi and
-// lo plane of a token each); a group of ntok tokens needs ntp of them, so the
-// slice's fold units (64-input blocks, or k-blocks for 32-input groups) are
-// taken R = 4 / ntp at a time: unit r of a round writes its products into
-// column pairs r*ntp .. r*ntp+ntp-1 (the lanes supplying the other columns
-// read the zero block), the round's units accumulate in one C fragment
-// without mixing, and each lane folds the unit whose column pair it holds.
-// One fold then serves R units; the lanes holding the same token are summed
-// once per row set (dec_reduce_lanes).  `plb`: the stage's inputs in the plane
-// buffer (token j at j * ptok), `sxb`: their block records (token j at
-// j * sxtok), `zb`: 256 zero bytes.
-template <int FMT>
-MOE_DEV void dec_stage(const DecWarp& q, uint32_t slot, uint32_t plb, uint32_t sxb, uint32_t zb, int ntok,
-                       float (&acc)[2]) {
-  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  const bool g32 = q.gshift < 0;
-  const int GU = g32 ? 1 : 2;  // k-blocks per fold unit
-  const int ntp = dec_ntp(ntok);
-  const int R = min(4 / ntp, 2 * q.nbw / GU);  // fold units per round
-  // B side: this lane supplies column g = plane (g & 1) of column pair g >> 1 = rB * ntp + jB
-  const int cpB = g >> 1, rB = cpB / ntp, jB = cpB - rB * ntp;
-  const bool liveB = jB < ntok && rB < R;
-  const uint32_t bbase = liveB ? plb + jB * q.ptok + t * 16 + (g & 1) * 8 : zb;
-  const uint32_t bstride = liveB ? 128 : 0;
-  // C side: this lane holds column pair t = rC * ntp + jC
-  const int rC = t / ntp, jC = t - rC * ntp;
-  const bool liveC = jC < ntok && rC < R;
-  const uint32_t sxbase = liveC ? sxb + jC * q.sxtok : zb;
-  const uint32_t sxstride = liveC ? 16 : 0;
-  // this lane's ldmatrix row: matrix (lane >> 3) = (A rows 0..7 | 8..15) x (chunk 0 | 1)
-  const int mtx = lane >> 3;
-  const uint32_t lbox = slot + ((mtx & 1) ? q.a8 : q.a0);
-  const int lrow = ((mtx & 1) ? q.r8 : q.r0) + (lane & 7);
-  const int csel = mtx >> 1;
-  const int ku0 = q.kq * 2 * q.nbw;  // the slice's first k-block in the stage
-  const int nk = 2 * q.nbw, rk = R * GU;
-  for (int k0 = 0; k0 < nk; k0 += rk) {
-    int c[4] = {0, 0, 0, 0}, cn[4] = {0, 0, 0, 0};
-    uint32_t w[2] = {0u, 0u};
-#pragma unroll 2
-    for (int kk = 0; kk < rk; ++kk) {
-      const int u = ku0 + k0 + kk;  // stage k-block
-      const int r = kk / GU;        // the fold unit's column-pair group in this round
-      uint32_t a[4];
-      if constexpr (FMT == F_A4 || FMT == F_MX4) {  // a k-block is one 16-byte chunk: rows g and g+8
-        const int by = u * 16, ln = by >> 7;
-        asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-                     : "=r"(w[0]), "=r"(w[1])
-                     : "r"(lbox + (uint32_t)((ln * q.R + lrow) * 128 + ((((by & 127) >> 4) ^ (lrow & 7)) << 4))));
-      } else if constexpr (FMT == F_A8) {  // a k-block is two chunks
-        const int by = u * 32, ln = by >> 7;
-        ldsm_x4(lbox + (uint32_t)((ln * q.R + lrow) * 128 + (((((by & 127) >> 4) + csel) ^ (lrow & 7)) << 4)), a[0],
-                a[1], a[2], a[3]);
-      } else if constexpr (FMT == F_A2) {  // a 64-input block is one chunk holding both k-blocks
-        if ((u & 1) == 0) {
-          const int by = (u >> 1) * 16, ln = by >> 7;
-          asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
-                       : "=r"(w[0]), "=r"(w[1])
-                       : "r"(lbox + (uint32_t)((ln * q.R + lrow) * 128 + ((((by & 127) >> 4) ^ (lrow & 7)) << 4))));
-        }
-      }
-      const uint32_t baddr = r == rB ? bbase + (u >> 1) * bstride + (u & 1) * 64 : zb + (u & 1) * 64;
-      const uint2 B = lds64u(baddr);
-      if constexpr (FMT == F_A4) {
-        unpack_a4(w[0], w[1], a);
-      } else if constexpr (FMT == F_MX4) {
-        uint32_t an[4];
-        unpack_mx4(w[0], w[1], a, an);
-        mma_u8s8(cn, an, B.x, B.y);
-      } else if constexpr (FMT == F_A2) {
-        unpack_a2(w[0], w[1], u & 1, a);
-      } else if constexpr (FMT == F_A3) {  // 12-byte k-blocks in 96-byte unswizzled lines
-        const int by = u * 12, ln = by / 96, off = by - ln * 96;
-        const uint32_t v0 = codes3x8(slot + q.a0 + (uint32_t)((ln * q.R + q.r0 + g) * 96), off, t);
-        const uint32_t v8 = codes3x8(slot + q.a8 + (uint32_t)((ln * q.R + q.r8 + g) * 96), off, t);
-        a[0] = spread3x4(v0 & 0xFFFu);
-        a[2] = spread3x4(v0 >> 12);
-        a[1] = spread3x4(v8 & 0xFFFu);
-        a[3] = spread3x4(v8 >> 12);
-      }
-      mma_u8s8(c, a, B.x, B.y);
-    }
-    // fold this lane's unit of the round (dead lanes fold a valid unit against the zero record)
-    const int f = (ku0 + k0) / GU + (liveC ? rC : 0);
-    const int bf = (f * GU) >> 1;  // its 64-input block
-    const float4 rec = lds_f4(sxbase + bf * sxstride);
-    const float sm = g32 ? (((f & 1) != 0) ? rec.z : rec.y) : rec.w;
-    int d4[4];
+// One 64-input block B of the warp's slice: its k-blocks, folded per scale
+// group (G = 32: per k-block).
+template <int FMT, int G, int B>
+MOE_DEV void dec_block(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, uint32_t xp, uint32_t s0,
+                       uint32_t s8, float (&acc)[2]) {
+  const float4 rec = lds_f4(xp + B * 16);
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  if constexpr (FMT == F_A4 || FMT == F_MX4)  // both k-blocks: two 16-byte chunks of the line
+    ldsm_x4(la + ((uint32_t)(B << 5) ^ L.ly), w[0], w[1], w[2], w[3]);
+  if constexpr (FMT == F_A2) {  // the block is one chunk; lanes 0..15 address rows 0..15
+    const uint32_t ad = la + ((uint32_t)(B << 4) ^ L.ly);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(ad));
+  }
+  int c[4] = {0, 0, 0, 0}, cn[4] = {0, 0, 0, 0};
+  dec_kblock<FMT, B, 0>(L, la, sl, bp, w, c, cn);
+  if constexpr (G == 32) {
+    int d[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) d4[i] = c[i] - cn[i];
-    dec_fold<FMT>(q, slot, rec.x, sm, g32 ? f : (bf >> q.gshift), d4, acc);
+    for (int i = 0; i < 4; ++i) {
+      d[i] = c[i] - cn[i];
+      c[i] = cn[i] = 0;
+    }
+    dec_fold<FMT, 2 * B>(s0, s8, L.brow, rec.x, rec.y, d, acc);
+  }
+  dec_kblock<FMT, B, 1>(L, la, sl, bp, w, c, cn);
+  int d[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = c[i] - cn[i];
+  if constexpr (G == 32)
+    dec_fold<FMT, 2 * B + 1>(s0, s8, L.brow, rec.x, rec.z, d, acc);
+  else
+    dec_fold<FMT, (B * 64) / G>(s0, s8, L.brow, rec.x, rec.w, d, acc);
+}
+
+template <int FMT, int G, int NBW, int B = 0>
+MOE_DEV void dec_blocks(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, uint32_t xp, uint32_t s0,
+                        uint32_t s8, float (&acc)[2]) {
+  if constexpr (B < NBW) {
+    dec_block<FMT, G, B>(L, la, sl, bp, xp, s0, s8, acc);
+    dec_blocks<FMT, G, NBW, B + 1>(L, la, sl, bp, xp, s0, s8, acc);
   }
 }
 
-// Sum the lanes that folded the same token's rows (dec_stage): afterwards
-// lane t < ntok of each quad holds token t's totals.
-MOE_DEV void dec_reduce_lanes(int ntok, float (&acc)[2]) {
-  const int ntp = dec_ntp(ntok);
-  if (ntp == 1) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 1);
-      acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
-    }
-  } else if (ntp == 2) {
-#pragma unroll
-    for (int i = 0; i < 2; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 2);
-  }
+// The warp's input slice of one stage (slot `sl`; `pl`: the stage's inputs
+// in the plane buffer, `sxb`: their block records).
+template <int FMT, int G, int NBW>
+MOE_DEV void dec_stage(const DecLane& L, uint32_t sl, uint32_t pl, uint32_t sxb, float (&acc)[2]) {
+  dec_blocks<FMT, G, NBW>(L, sl + L.la, sl, pl + L.b, sxb + L.sx, sl + L.s0, sl + L.s8, acc);
 }
 
 // Routing results and work groups, shared by every CTA (built in P1).
@@ -482,28 +501,27 @@ MOE_DEV bool dec_consumer_wait(uint32_t bar, uint32_t parity, volatile int* abor
   return __all_sync(0xffffffffu, have);  // the MMAs need every lane
 }
 
-// Consumer side of one unit's stages, row set by row set (FMT: the unit's
-// weight format; S1: W1/W3 in 4 row sets of 16, else W2 in 2 row sets of 32,
-// each over nch stages along the inputs).  Each row set's slice partials go
-// to `red`: S1 [(kq*4 + rs)*16 + row][token][W1 | W3], S2 [(kq*2 + rs)*32 +
-// row][token].
-template <int FMT, bool S1>
-MOE_DEV void dec_consume(const DecWarp& q, int nch, int K, int ntok, uint32_t ring, int slot_bytes, int nslot,
-                         uint32_t pl, uint32_t sx0, uint32_t zb, uint32_t full0, uint32_t empty0, int& n,
-                         bool have_pl, volatile int* abort_flag, int* err, float* red, int tt) {
-  constexpr int NRS = S1 ? 4 : 2;
+// Consumer side of one unit's stages, row set by row set (S1: W1/W3 in 4
+// row sets of 16, else W2 in 2 row sets of 32, each over nch stages along
+// the inputs).  Each row set's slice partials go to `red`: S1 [(kq*4 + rs)*16
+// + row][token][W1 | W3], S2 [(kq*2 + rs)*32 + row][token].
+template <int FMT, int G, int NBW>
+MOE_DEV void dec_consume(const DecWarp& q, bool s1, int nch, int K, int ntok, uint32_t ring, int slot_bytes,
+                         int nslot, uint32_t pl, uint32_t sx0, uint32_t full0, uint32_t empty0, int& n, bool have_pl,
+                         volatile int* abort_flag, int* err, float* red, int tt) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-  for (int rs = 0; rs < NRS; ++rs) {
+  const DecLane L = dec_lane<FMT, G, NBW>(q, ntok);
+  const int nrs = s1 ? kDecRows / kDecR1 : kDecRows / kDecR2;
+  for (int rs = 0; rs < nrs; ++rs) {
     float acc[2] = {0.f, 0.f};
     for (int chn = 0; chn < nch; ++chn, ++n) {
       const int s = n % nslot;
       const bool have = dec_consumer_wait(full0 + 8 * s, (n / nslot) & 1, abort_flag, err) && have_pl;
-      if (have) dec_stage<FMT>(q, ring + s * slot_bytes, pl + chn * K * 2, sx0 + chn * (K / 64) * 16, zb, ntok, acc);
+      if (have) dec_stage<FMT, G, NBW>(L, ring + s * slot_bytes, pl + chn * K * 2, sx0 + chn * (K / 64) * 16, acc);
       __syncwarp();
       if (lane == 0 && have) dec_arrive(empty0 + 8 * s);
     }
-    dec_reduce_lanes(ntok, acc);
-    if constexpr (S1) {
+    if (s1) {
       *reinterpret_cast<float2*>(red + ((q.kq * 4 + rs) * 16 + tt * 8 + g) * 8 + 2 * t) = make_float2(acc[0], acc[1]);
     } else {
       red[((q.kq * 2 + rs) * 32 + tt * 16 + g) * 4 + t] = acc[0];
@@ -512,21 +530,56 @@ MOE_DEV void dec_consume(const DecWarp& q, int nch, int K, int ntok, uint32_t ri
   }
 }
 
-template <bool S1>
-MOE_DEV void dec_consume_any(int fmt, const DecWarp& q, int nch, int K, int ntok, uint32_t ring, int slot_bytes,
-                             int nslot, uint32_t pl, uint32_t sx0, uint32_t zb, uint32_t full0, uint32_t empty0,
-                             int& n, bool have_pl, volatile int* abort_flag, int* err, float* red, int tt) {
-#define MOE_DEC_CONSUME(F)                                                                                         \
-  dec_consume<F, S1>(q, nch, K, ntok, ring, slot_bytes, nslot, pl, sx0, zb, full0, empty0, n, have_pl, abort_flag, \
-                     err, red, tt)
+// (format, scale group, blocks per slice) combinations the fused kernel
+// instantiates; the host admits only these (dec_supported).
+__host__ __device__ inline bool dec_supported(int fmt, int group, int nbw) {
   switch (fmt) {
-    case F_A2: MOE_DEC_CONSUME(F_A2); break;
-    case F_A3: MOE_DEC_CONSUME(F_A3); break;
-    case F_A4: MOE_DEC_CONSUME(F_A4); break;
-    case F_A8: MOE_DEC_CONSUME(F_A8); break;
-    default: MOE_DEC_CONSUME(F_MX4); break;
+    case F_A4:
+    case F_A3: return (group == 32 || group == 64 || group == 128) && (nbw == 2 || nbw == 4);
+    case F_A8: return (group == 32 || group == 64 || (group == 128 && nbw == 2)) && (nbw == 1 || nbw == 2);
+    case F_A2: return (group == 64 || group == 128) && (nbw == 4 || nbw == 8);
+    default: return group == 32 && (nbw == 2 || nbw == 4);
   }
-#undef MOE_DEC_CONSUME
+}
+
+MOE_DEV void dec_consume_any(int fmt, int group, int nbw, const DecWarp& q, bool s1, int nch, int K, int ntok,
+                             uint32_t ring, int slot_bytes, int nslot, uint32_t pl, uint32_t sx0, uint32_t full0,
+                             uint32_t empty0, int& n, bool have_pl, volatile int* abort_flag, int* err, float* red,
+                             int tt) {
+#define MOE_DC(F, GG, NB)                                                                                        \
+  dec_consume<F, GG, NB>(q, s1, nch, K, ntok, ring, slot_bytes, nslot, pl, sx0, full0, empty0, n, have_pl, abort_flag, \
+                         err, red, tt)
+#define MOE_DC_G(F, NB)                  \
+  do {                                   \
+    if (group == 32) MOE_DC(F, 32, NB);  \
+    else if (group == 64) MOE_DC(F, 64, NB); \
+    else MOE_DC(F, 128, NB);             \
+  } while (0)
+  switch (fmt) {
+    case F_A4:
+      if (nbw == 4) MOE_DC_G(F_A4, 4); else MOE_DC_G(F_A4, 2);
+      break;
+    case F_A3:
+      if (nbw == 4) MOE_DC_G(F_A3, 4); else MOE_DC_G(F_A3, 2);
+      break;
+    case F_A8:
+      if (nbw == 2) MOE_DC_G(F_A8, 2);
+      else if (group == 32) MOE_DC(F_A8, 32, 1);
+      else MOE_DC(F_A8, 64, 1);
+      break;
+    case F_A2:
+      if (nbw == 8) {
+        if (group == 64) MOE_DC(F_A2, 64, 8); else MOE_DC(F_A2, 128, 8);
+      } else {
+        if (group == 64) MOE_DC(F_A2, 64, 4); else MOE_DC(F_A2, 128, 4);
+      }
+      break;
+    default:
+      if (nbw == 4) MOE_DC(F_MX4, 32, 4); else MOE_DC(F_MX4, 32, 2);
+      break;
+  }
+#undef MOE_DC_G
+#undef MOE_DC
 }
 
 // fp32 order as an unsigned order (larger float -> larger key); NaN is
@@ -605,7 +658,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
   uint8_t* fx = base + (size_t)p.nslot * p.slot_bytes + 2 * (size_t)p.pbuf;
   float* red = reinterpret_cast<float*>(fx + kDecFxRed);
   float* hbuf = reinterpret_cast<float*>(fx + kDecFxH);  // [2][4][64]
-  const uint32_t zb = su32(fx + kDecFxZero);
   int* r_ids = reinterpret_cast<int*>(fx + kDecFxIds);
   float* r_w = reinterpret_cast<float*>(fx + kDecFxW);
   int* r_sorted = reinterpret_cast<int*>(fx + kDecFxSorted);
@@ -642,7 +694,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mp)) : "memory");
   }
   for (int e = tid; e < E; e += kDecThreads) r_off[e] = 0;  // per-expert counts (P1)
-  if (tid < 64) reinterpret_cast<int*>(fx + kDecFxZero)[tid] = 0;
   __syncthreads();
 
   // ------------------------------------------------------------ P0
@@ -1062,11 +1113,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
       DecWarp q;
       const int nsb = m0.fmt == F_MX4 ? 1 : 2;
       q.R = m0.R;
-      q.nbw = m0.nbw;
       q.kq = kq;
-      q.gshift = m0.gshift;
       q.spitch = m0.spitch;
-      q.brow = m0.R * m0.spitch;
       q.ptok = m0.ptok;
       q.sxtok = m0.sxtok;
       if (s1) {  // A rows 0..7: W1 rows tt*8.., rows 8..15: the same rows of W3
@@ -1084,12 +1132,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
       const int pb = np & 1;
       const bool have_pl = dec_consumer_wait(pfull0 + 8 * pb, (np >> 1) & 1, abort_flag, p.err);
       const uint32_t pl = planes0 + pb * p.pbuf;
-      if (s1)
-        dec_consume_any<true>(m0.fmt, q, m0.nch, m0.K, grp.z, ring, p.slot_bytes, p.nslot, pl, pl + p.sx_off, zb,
-                              full0, empty0, n, have_pl, abort_flag, p.err, red, tt);
-      else
-        dec_consume_any<false>(m0.fmt, q, m0.nch, m0.K, grp.z, ring, p.slot_bytes, p.nslot, pl, pl + p.sx_off, zb,
-                               full0, empty0, n, have_pl, abort_flag, p.err, red, tt);
+      dec_consume_any(m0.fmt, m0.group, m0.nbw, q, s1, m0.nch, m0.K, grp.z, ring, p.slot_bytes, p.nslot, pl,
+                      pl + p.sx_off, full0, empty0, n, have_pl, abort_flag, p.err, red, tt);
       __syncwarp();
       if (lane == 0 && have_pl) dec_arrive(pempty0 + 8 * pb);
       ++np;

@@ -824,11 +824,8 @@ bool dec_mat(const QMatDev& Q, bool w2, DecMat* m) {
   m->K = m->seg * 8 / bits;
   if (m->K % (64 * kDecNkq)) return false;  // input slices of whole 64-input blocks
   m->nbw = m->K / (64 * kDecNkq);
-  if (m->nbw & (m->nbw - 1)) return false;  // rounds of 1, 2 or 4 fold units tile the slice
-  if (Q.group != 32 && Q.group != 64 && Q.group != 128) return false;
-  if (Q.fmt == F_A2 && Q.group == 32) return false;  // a 2-bit k-block mixes two 32-input groups
+  if (!dec_supported(Q.fmt, Q.group, m->nbw)) return false;  // the instantiated (format, group, slice) shapes
   if (m->K % Q.group) return false;
-  m->gshift = Q.group == 32 ? -1 : Q.group == 64 ? 0 : 1;
   m->sK = m->K / Q.group;
   const int esz = Q.fmt == F_MX4 ? 1 : 2;
   const int sbytes = m->sK * esz;
