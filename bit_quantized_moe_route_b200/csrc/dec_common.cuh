@@ -173,15 +173,33 @@ MOE_DEV bool dec_wait_count(const int* p, int target, const volatile int* abort_
   return true;
 }
 
-// Mbarrier phase wait (bounded); false on timeout or abort.
-MOE_DEV bool dec_wait_bar(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
+// try_wait that may suspend the thread until the phase completes (for warps
+// with nothing else to do: a spinning warp takes issue slots from the math)
+MOE_DEV bool dec_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(1000000)
+      : "memory");
+  return ok != 0;
+}
+
+// Mbarrier phase wait (bounded); false on timeout or abort.  A waiting warp
+// backs off with nanosleep between polls (a spinning warp takes issue slots
+// from the warps still computing) and checks the abort flag and the clock
+// every 8 polls.
+MOE_DEV bool dec_wait_bar(uint32_t bar, uint32_t parity, const volatile int* abort_flag, bool sleep = false) {
   if (dec_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!dec_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > kDecWaitCycles) return false;
+  for (uint32_t it = 1;; ++it) {
+    if (sleep ? dec_try_wait_sleep(bar, parity) : dec_try_wait(bar, parity)) return true;
+    __nanosleep(32);
+    if ((it & 7) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > kDecWaitCycles) return false;
+    }
   }
-  return true;
 }
 
 // ------------------------------------------------------------ fixed point

@@ -19,12 +19,15 @@
 //   S1  units (group, 64 rows of d_ff): h = silu(W1 x) * (W3 x) for the
 //       group's tokens, written as the planes W2 reads; a per-group counter
 //       counts finished units;
-//   S2  units (group, 64 rows of d_model): y = W2 h, started once the
-//       group's S1 units are all counted; the CTA that finishes the last unit
-//       of an output row block sums the k slots of every token in ascending
-//       j, adds the shared expert and writes bf16 (one rounding).
-// Units are dealt round-robin over the CTAs in the order [S1 shared, S1
-// routed, S2 by group].
+//   S2  units (group, 128 rows of d_model): y = W2 h, whose weight stages
+//       are issued at once and whose h planes follow once the group's S1
+//       units are all counted;
+//   C   grid barrier, then every CTA sums the k slots of a slice of the
+//       output in ascending j, adds the shared expert and writes bf16 (one
+//       rounding).
+// Units are claimed dynamically in the order [S1 shared, S1 routed, S2 by
+// group]: a CTA's first unit is its index, the next comes from a launch-wide
+// counter, claimed one unit ahead.
 //
 // Weight stream.  One producer warp fills a ring of 32 KB stages; a stage is
 // a set of WHOLE row segments: 16 rows of W1 and the same 16 rows of W3 (S1)
@@ -52,8 +55,8 @@
 
 namespace moe {
 
-constexpr int kDecConsumerWarps = 16;
-constexpr int kDecNkq = kDecConsumerWarps / 2;      // input slices (2 row tiles x 8 slices)
+constexpr int kDecConsumerWarps = 8;
+constexpr int kDecNkq = kDecConsumerWarps;          // input slices: one per consumer warp (both row tiles)
 constexpr int kDecProducerWarp = kDecConsumerWarps;
 constexpr int kDecServiceWarp = kDecConsumerWarps + 1;
 constexpr int kDecWarps = kDecConsumerWarps + 2;
@@ -61,7 +64,8 @@ constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kDecConsumerThreads = kDecConsumerWarps * 32;
 constexpr int kDecMaxSlots = 6;
 constexpr int kDecSlotCap = 4;     // ring slots used (more 32 KB stages in flight lower the copy rate)
-constexpr int kDecRows = 64;       // output rows per unit
+constexpr int kDecRows = 64;       // hidden rows per S1 unit (one 64-input block of W2's planes)
+constexpr int kDecRows2 = 128;     // output rows per S2 unit
 constexpr int kDecR1 = 16;         // rows of W1 (and of W3) per stage
 constexpr int kDecR2 = 32;         // rows of W2 per stage
 constexpr int kDecMaxTok = 4;      // tokens per group (B columns 0..7 of the MMA: hi and lo plane of each)
@@ -77,7 +81,8 @@ constexpr int kDecMaxGroups = kDecMaxPairs + 8;
 constexpr int kDecFxRed = 0;
 constexpr int kDecFxH = kDecFxRed + kDecRedFloats * 4;           // 2 buffers x 4 tokens x 64 h values
 constexpr int kDecFxScr = kDecFxH + 2 * kDecMaxTok * kDecRows * 4;  // the service warp's scratch (64 ints)
-constexpr int kDecFxIds = kDecFxScr + 256;
+constexpr int kDecFxLut = kDecFxScr + 256;                      // e8m0 byte -> 2^(e-128) (fp32)
+constexpr int kDecFxIds = kDecFxLut + 1024;
 constexpr int kDecFxW = kDecFxIds + kDecMaxPairs * 4;
 constexpr int kDecFxSorted = kDecFxW + kDecMaxPairs * 4;
 constexpr int kDecFxInv = kDecFxSorted + kDecMaxPairs * 4;
@@ -135,8 +140,7 @@ struct DecParams {
   float4* hsx;         // [P][fmax/64]
   float* y;            // [P][d]
   int* cnt_h;          // [kDecMaxGroups]
-  int* cnt_y;          // [d/64]
-  int* sync;           // [0] barrier count, [1] barrier generation, [2] exit count
+  int* sync;           // [0] barrier count, [1] barrier generation, [2] units claimed past the first G
   int* err;
   __nv_bfloat16* out;  // [T][d]
   int* ids_out;        // [T][k] or NULL
@@ -244,12 +248,12 @@ MOE_DEV void unpack_mx4(uint32_t wg, uint32_t wg8, uint32_t (&a)[4], uint32_t (&
   an[1] = mag4(fg8);
   an[3] = mag4(fg8 >> 16);
 }
-MOE_DEV void unpack_a2(uint32_t wg, uint32_t wg8, int kb2, uint32_t (&a)[4]) {
-  const int s0 = 4 * kb2, s1 = 4 * kb2 + 2;
-  a[0] = (wg >> s0) & 0x03030303u;
-  a[1] = (wg8 >> s0) & 0x03030303u;
-  a[2] = (wg >> s1) & 0x03030303u;
-  a[3] = (wg8 >> s1) & 0x03030303u;
+template <int KB2>
+MOE_DEV void unpack_a2(uint32_t wg, uint32_t wg8, uint32_t (&a)[4]) {
+  a[0] = (wg >> (4 * KB2)) & 0x03030303u;
+  a[1] = (wg8 >> (4 * KB2)) & 0x03030303u;
+  a[2] = (wg >> (4 * KB2 + 2)) & 0x03030303u;
+  a[3] = (wg8 >> (4 * KB2 + 2)) & 0x03030303u;
 }
 // four 3-bit codes (12 bits) -> bytes 0..3
 MOE_DEV uint32_t spread3x4(uint32_t t) {
@@ -273,8 +277,10 @@ MOE_DEV uint32_t codes3x8(uint32_t line, int off, int t) {
 // rows r8..r8+7; their scales in scale boxes `s0` / `s8` (biases R * spitch
 // bytes further).
 struct DecWarp {
+  uint32_t lut;  // shared address of the e8m0 table
   uint32_t a0, a8, s0, s8;
-  int r0, r8;
+  int r0, r8;    // tile 0; tile 1 is `tstep` rows further in every box
+  int tstep;
   int R;   // rows per box
   int kq;  // input slice
   int spitch;
@@ -291,6 +297,8 @@ struct DecLane {
   uint32_t b;     // plane-buffer-relative B address (token row, quad thread, plane)
   uint32_t sx;    // record-relative address (token, the slice's first block)
   uint32_t s0, s8, brow;  // slot-relative scale addresses of A rows g / g+8 (the slice's first group), bias offset
+  uint32_t lut;           // shared address of the e8m0 table
+  uint32_t ta, ts;        // tile 1: code byte offset (tstep rows), scale byte offset
 };
 
 
@@ -337,6 +345,9 @@ MOE_DEV DecLane dec_lane(const DecWarp& q, int ntok) {
   L.s0 = q.s0 + (uint32_t)((q.r0 + g) * q.spitch + esz * gbase);
   L.s8 = q.s8 + (uint32_t)((q.r8 + g) * q.spitch + esz * gbase);
   L.brow = (uint32_t)(q.R * q.spitch);
+  L.lut = q.lut;
+  L.ta = (uint32_t)(q.tstep * (FMT == F_A3 ? 96 : 128));
+  L.ts = (uint32_t)(q.tstep * q.spitch);
   return L;
 }
 
@@ -345,7 +356,7 @@ MOE_DEV DecLane dec_lane(const DecWarp& q, int ntok) {
 // integer sum of codes x fixed-point inputs, st the inputs' step, sm their
 // dequantised sum; GI: the group's scale entry relative to the slice.
 template <int FMT, int GI>
-MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, float st, float sm, const int (&c)[4],
+MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, uint32_t lut, float st, float sm, const int (&c)[4],
                       float (&acc)[2]) {
   float sc0, b0, sc8, b8;
   if constexpr (FMT == F_MX4) {
@@ -353,6 +364,7 @@ MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, float st, float s
     const uint32_t e0 = lds8u(s0 + GI), e8 = lds8u(s8 + GI);
     sc0 = __uint_as_float(e0 > 1 ? ((e0 - 1) << 23) : (e0 ? 0x00400000u : 0x00200000u));
     sc8 = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));
+    (void)lut;
     b0 = b8 = 0.f;
   } else {
     sc0 = bf16_bits_to_float(lds16u(s0 + 2 * GI));
@@ -364,12 +376,11 @@ MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, float st, float s
   acc[1] = fmaf(sc8 * st, (float)(c[2] * 256 + c[3]), fmaf(b8, sm, acc[1]));
 }
 
-// k-block H of block B of the warp's slice: A fragment, one MMA (two for
-// mxfp4: positive and negative magnitudes), with B from the plane buffer.
+// k-block H of block B of the warp's slice for one tile: A fragment, one MMA
+// (two for mxfp4: positive and negative magnitudes) with the shared B.
 template <int FMT, int B, int H>
-MOE_DEV void dec_kblock(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, const uint32_t (&w)[4], int (&c)[4],
-                        int (&cn)[4]) {
-  const uint2 bv = lds64u(bp + B * 128 + H * 64);
+MOE_DEV void dec_kblock(const DecLane& L, uint32_t la, uint32_t sl, uint32_t t3, const uint2 bv,
+                        const uint32_t (&w)[4], int (&c)[4], int (&cn)[4]) {
   uint32_t a[4];
   if constexpr (FMT == F_A4) {
     unpack_a4(w[2 * H], w[2 * H + 1], a);
@@ -380,9 +391,9 @@ MOE_DEV void dec_kblock(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp,
   } else if constexpr (FMT == F_A8) {  // a k-block is two chunks of the line
     ldsm_x4(la + ((uint32_t)((4 * B + 2 * H) << 4) ^ L.ly), a[0], a[1], a[2], a[3]);
   } else if constexpr (FMT == F_A2) {
-    unpack_a2(w[0], w[1], H, a);
+    unpack_a2<H>(w[0], w[1], a);
   } else {  // 3-bit: 12-byte k-blocks, this thread's 8 codes of rows g and g+8
-    const uint32_t pa = sl + L.l3a + (2 * B + H) * 12, pb = sl + L.l3b + (2 * B + H) * 12;
+    const uint32_t pa = sl + L.l3a + t3 + (2 * B + H) * 12, pb = sl + L.l3b + t3 + (2 * B + H) * 12;
     const uint32_t v0 = __funnelshift_r(lds32u(pa), lds32u(pa + 4), L.sh3) & 0xFFFFFFu;
     const uint32_t v8 = __funnelshift_r(lds32u(pb), lds32u(pb + 4), L.sh3) & 0xFFFFFFu;
     a[0] = spread3x4(v0 & 0xFFFu);
@@ -393,53 +404,81 @@ MOE_DEV void dec_kblock(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp,
   mma_u8s8(c, a, bv.x, bv.y);
 }
 
-// One 64-input block B of the warp's slice: its k-blocks, folded per scale
-// group (G = 32: per k-block).
-template <int FMT, int G, int B>
-MOE_DEV void dec_block(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, uint32_t xp, uint32_t s0,
-                       uint32_t s8, float (&acc)[2]) {
-  const float4 rec = lds_f4(xp + B * 16);
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
+// A fragments of block B (both k-blocks) for the tile whose ldmatrix row is `la`
+template <int FMT, int B>
+MOE_DEV void dec_loadA(const DecLane& L, uint32_t la, uint32_t (&w)[4]) {
   if constexpr (FMT == F_A4 || FMT == F_MX4)  // both k-blocks: two 16-byte chunks of the line
     ldsm_x4(la + ((uint32_t)(B << 5) ^ L.ly), w[0], w[1], w[2], w[3]);
   if constexpr (FMT == F_A2) {  // the block is one chunk; lanes 0..15 address rows 0..15
     const uint32_t ad = la + ((uint32_t)(B << 4) ^ L.ly);
     asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(ad));
   }
-  int c[4] = {0, 0, 0, 0}, cn[4] = {0, 0, 0, 0};
-  dec_kblock<FMT, B, 0>(L, la, sl, bp, w, c, cn);
+}
+
+// One 64-input block B of the warp's slice for both row tiles (acc[0..1]:
+// tile 0, acc[2..3]: tile 1), folded per scale group (G = 32: per k-block).
+template <int FMT, int G, int B>
+MOE_DEV void dec_block(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, uint32_t xp, uint32_t s0,
+                       uint32_t s8, float (&acc)[4]) {
+  const float4 rec = lds_f4(xp + B * 16);
+  uint32_t w0[4] = {0u, 0u, 0u, 0u}, w1[4] = {0u, 0u, 0u, 0u};
+  dec_loadA<FMT, B>(L, la, w0);
+  dec_loadA<FMT, B>(L, la + L.ta, w1);
+  int c0[4] = {0, 0, 0, 0}, cn0[4] = {0, 0, 0, 0}, c1[4] = {0, 0, 0, 0}, cn1[4] = {0, 0, 0, 0};
+  float a0[2] = {acc[0], acc[1]}, a1[2] = {acc[2], acc[3]};
+  {
+    const uint2 bv = lds64u(bp + B * 128);
+    dec_kblock<FMT, B, 0>(L, la, sl, 0u, bv, w0, c0, cn0);
+    dec_kblock<FMT, B, 0>(L, la + L.ta, sl, L.ta, bv, w1, c1, cn1);
+  }
   if constexpr (G == 32) {
-    int d[4];
+    int d0[4], d1[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      d[i] = c[i] - cn[i];
-      c[i] = cn[i] = 0;
+      d0[i] = c0[i] - cn0[i];
+      d1[i] = c1[i] - cn1[i];
+      c0[i] = cn0[i] = c1[i] = cn1[i] = 0;
     }
-    dec_fold<FMT, 2 * B>(s0, s8, L.brow, rec.x, rec.y, d, acc);
+    dec_fold<FMT, 2 * B>(s0, s8, L.brow, L.lut, rec.x, rec.y, d0, a0);
+    dec_fold<FMT, 2 * B>(s0 + L.ts, s8 + L.ts, L.brow, L.lut, rec.x, rec.y, d1, a1);
   }
-  dec_kblock<FMT, B, 1>(L, la, sl, bp, w, c, cn);
-  int d[4];
+  {
+    const uint2 bv = lds64u(bp + B * 128 + 64);
+    dec_kblock<FMT, B, 1>(L, la, sl, 0u, bv, w0, c0, cn0);
+    dec_kblock<FMT, B, 1>(L, la + L.ta, sl, L.ta, bv, w1, c1, cn1);
+  }
+  int d0[4], d1[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) d[i] = c[i] - cn[i];
-  if constexpr (G == 32)
-    dec_fold<FMT, 2 * B + 1>(s0, s8, L.brow, rec.x, rec.z, d, acc);
-  else
-    dec_fold<FMT, (B * 64) / G>(s0, s8, L.brow, rec.x, rec.w, d, acc);
+  for (int i = 0; i < 4; ++i) {
+    d0[i] = c0[i] - cn0[i];
+    d1[i] = c1[i] - cn1[i];
+  }
+  if constexpr (G == 32) {
+    dec_fold<FMT, 2 * B + 1>(s0, s8, L.brow, L.lut, rec.x, rec.z, d0, a0);
+    dec_fold<FMT, 2 * B + 1>(s0 + L.ts, s8 + L.ts, L.brow, L.lut, rec.x, rec.z, d1, a1);
+  } else {
+    dec_fold<FMT, (B * 64) / G>(s0, s8, L.brow, L.lut, rec.x, rec.w, d0, a0);
+    dec_fold<FMT, (B * 64) / G>(s0 + L.ts, s8 + L.ts, L.brow, L.lut, rec.x, rec.w, d1, a1);
+  }
+  acc[0] = a0[0];
+  acc[1] = a0[1];
+  acc[2] = a1[0];
+  acc[3] = a1[1];
 }
 
 template <int FMT, int G, int NBW, int B = 0>
 MOE_DEV void dec_blocks(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, uint32_t xp, uint32_t s0,
-                        uint32_t s8, float (&acc)[2]) {
+                        uint32_t s8, float (&acc)[4]) {
   if constexpr (B < NBW) {
     dec_block<FMT, G, B>(L, la, sl, bp, xp, s0, s8, acc);
     dec_blocks<FMT, G, NBW, B + 1>(L, la, sl, bp, xp, s0, s8, acc);
   }
 }
 
-// The warp's input slice of one stage (slot `sl`; `pl`: the stage's inputs
-// in the plane buffer, `sxb`: their block records).
+// The warp's input slice of one stage for both row tiles (slot `sl`; `pl`:
+// the stage's inputs in the plane buffer, `sxb`: their block records).
 template <int FMT, int G, int NBW>
-MOE_DEV void dec_stage(const DecLane& L, uint32_t sl, uint32_t pl, uint32_t sxb, float (&acc)[2]) {
+MOE_DEV void dec_stage(const DecLane& L, uint32_t sl, uint32_t pl, uint32_t sxb, float (&acc)[4]) {
   dec_blocks<FMT, G, NBW>(L, sl + L.la, sl, pl + L.b, sxb + L.sx, sl + L.s0, sl + L.s8, acc);
 }
 
@@ -454,7 +493,7 @@ struct DecUnit {
 
 MOE_DEV DecUnit dec_unit(const DecParams& p, const int4* groups, int nsg, int nrg, int i) {
   DecUnit U;
-  const int ufs = p.fs / kDecRows, uf = p.f / kDecRows, ud = p.d / kDecRows;
+  const int ufs = p.fs / kDecRows, uf = p.f / kDecRows, ud = p.d / kDecRows2;
   const int U1s = nsg * ufs, U1 = U1s + nrg * uf;
   if (i < U1) {
     U.stage = 1;
@@ -477,7 +516,7 @@ MOE_DEV DecUnit dec_unit(const DecParams& p, const int4* groups, int nsg, int nr
     U.u = j % ud;
     const bool sh = groups[U.grp].x < 0;
     U.mi = sh ? DM_S2 : DM_W2;
-    U.row0 = (sh ? 0 : groups[U.grp].x * p.d) + kDecRows * U.u;
+    U.row0 = (sh ? 0 : groups[U.grp].x * p.d) + kDecRows2 * U.u;
   }
   return U;
 }
@@ -490,10 +529,23 @@ MOE_DEV int dec_token(const DecParams& p, const int* sorted, int4 g, int i) {
   return g.x < 0 ? g.y + i : sorted[g.y + i] / p.k;
 }
 
+// Position in the stage ring: stage count, slot, and the parity of the
+// slot's current use (advanced without division).
+struct DecRing {
+  int n, s, ph;
+  MOE_DEV void next(int nslot) {
+    ++n;
+    if (++s == nslot) {
+      s = 0;
+      ph ^= 1;
+    }
+  }
+};
+
 // Bounded mbarrier wait of a consumer warp; false once the kernel aborts.
 MOE_DEV bool dec_consumer_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* err) {
   bool have = !*abort_flag;
-  if (have && !dec_wait_bar(bar, parity, abort_flag)) {
+  if (have && !dec_wait_bar(bar, parity, abort_flag, true)) {
     set_error(err, kErrTimeout);
     *abort_flag = 1;
     have = false;
@@ -502,30 +554,34 @@ MOE_DEV bool dec_consumer_wait(uint32_t bar, uint32_t parity, volatile int* abor
 }
 
 // Consumer side of one unit's stages, row set by row set (S1: W1/W3 in 4
-// row sets of 16, else W2 in 2 row sets of 32, each over nch stages along
+// row sets of 16, else W2 in 4 row sets of 32, each over nch stages along
 // the inputs).  Each row set's slice partials go to `red`: S1 [(kq*4 + rs)*16
-// + row][token][W1 | W3], S2 [(kq*2 + rs)*32 + row][token].
+// + row][token][W1 | W3], S2 [(kq*4 + rs)*32 + row][token].
 template <int FMT, int G, int NBW>
 MOE_DEV void dec_consume(const DecWarp& q, bool s1, int nch, int K, int ntok, uint32_t ring, int slot_bytes,
-                         int nslot, uint32_t pl, uint32_t sx0, uint32_t full0, uint32_t empty0, int& n, bool have_pl,
-                         volatile int* abort_flag, int* err, float* red, int tt) {
+                         int nslot, uint32_t pl, uint32_t sx0, uint32_t full0, uint32_t empty0, DecRing& rg,
+                         bool have_pl, volatile int* abort_flag, int* err, float* red) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
   const DecLane L = dec_lane<FMT, G, NBW>(q, ntok);
-  const int nrs = s1 ? kDecRows / kDecR1 : kDecRows / kDecR2;
+  const int nrs = s1 ? kDecRows / kDecR1 : kDecRows2 / kDecR2;  // 4 row sets either way
   for (int rs = 0; rs < nrs; ++rs) {
-    float acc[2] = {0.f, 0.f};
-    for (int chn = 0; chn < nch; ++chn, ++n) {
-      const int s = n % nslot;
-      const bool have = dec_consumer_wait(full0 + 8 * s, (n / nslot) & 1, abort_flag, err) && have_pl;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int chn = 0; chn < nch; ++chn, rg.next(nslot)) {
+      const int s = rg.s;
+      const bool have = dec_consumer_wait(full0 + 8 * s, rg.ph, abort_flag, err) && have_pl;
       if (have) dec_stage<FMT, G, NBW>(L, ring + s * slot_bytes, pl + chn * K * 2, sx0 + chn * (K / 64) * 16, acc);
       __syncwarp();
       if (lane == 0 && have) dec_arrive(empty0 + 8 * s);
     }
-    if (s1) {
-      *reinterpret_cast<float2*>(red + ((q.kq * 4 + rs) * 16 + tt * 8 + g) * 8 + 2 * t) = make_float2(acc[0], acc[1]);
-    } else {
-      red[((q.kq * 2 + rs) * 32 + tt * 16 + g) * 4 + t] = acc[0];
-      red[((q.kq * 2 + rs) * 32 + tt * 16 + g + 8) * 4 + t] = acc[1];
+    if (s1) {  // tile tt: W1 rows tt*8 + g (acc[2tt]) and the same W3 rows (acc[2tt+1])
+      *reinterpret_cast<float2*>(red + ((q.kq * 4 + rs) * 16 + g) * 8 + 2 * t) = make_float2(acc[0], acc[1]);
+      *reinterpret_cast<float2*>(red + ((q.kq * 4 + rs) * 16 + 8 + g) * 8 + 2 * t) = make_float2(acc[2], acc[3]);
+    } else {  // tile tt: rows tt*16 + g and + 8
+      float* rr = red + ((q.kq * 4 + rs) * 32 + g) * 4 + t;
+      rr[0] = acc[0];
+      rr[8 * 4] = acc[1];
+      rr[16 * 4] = acc[2];
+      rr[24 * 4] = acc[3];
     }
   }
 }
@@ -544,11 +600,11 @@ __host__ __device__ inline bool dec_supported(int fmt, int group, int nbw) {
 
 MOE_DEV void dec_consume_any(int fmt, int group, int nbw, const DecWarp& q, bool s1, int nch, int K, int ntok,
                              uint32_t ring, int slot_bytes, int nslot, uint32_t pl, uint32_t sx0, uint32_t full0,
-                             uint32_t empty0, int& n, bool have_pl, volatile int* abort_flag, int* err, float* red,
-                             int tt) {
+                             uint32_t empty0, DecRing& rg, bool have_pl, volatile int* abort_flag, int* err,
+                             float* red) {
 #define MOE_DC(F, GG, NB)                                                                                        \
-  dec_consume<F, GG, NB>(q, s1, nch, K, ntok, ring, slot_bytes, nslot, pl, sx0, full0, empty0, n, have_pl, abort_flag, \
-                         err, red, tt)
+  dec_consume<F, GG, NB>(q, s1, nch, K, ntok, ring, slot_bytes, nslot, pl, sx0, full0, empty0, rg, have_pl, abort_flag, \
+                         err, red)
 #define MOE_DC_G(F, NB)                  \
   do {                                   \
     if (group == 32) MOE_DC(F, 32, NB);  \
@@ -669,7 +725,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
   const uint32_t pfull0 = empty0 + 8 * kDecMaxSlots, pempty0 = pfull0 + 16;
   const uint32_t efull0 = pempty0 + 16, eempty0 = efull0 + 16;  // unit epilogues: consumers -> service warp
   volatile int* misc = reinterpret_cast<volatile int*>(fx + kDecFxMisc);
-  volatile int* abort_flag = misc;  // [0] abort, [1] groups shared, [2] groups routed
+  // misc: [0] abort, [1] groups shared, [2] groups routed, [4] the consumers' unit,
+  // [8..11] unit of each plane-buffer use (producer -> consumers, -1: no more),
+  // [12..13] unit of each epilogue buffer (consumers -> service warp, -1: no more)
+  volatile int* abort_flag = misc;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int T = p.T, k = p.k, E = p.E, d = p.d;
@@ -694,6 +753,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mp)) : "memory");
   }
   for (int e = tid; e < E; e += kDecThreads) r_off[e] = 0;  // per-expert counts (P1)
+  if (tid < 256) {  // e8m0 byte -> 2^(e-128): exact for every byte (subnormal for 0 and 1)
+    const uint32_t e = tid;
+    reinterpret_cast<float*>(fx + kDecFxLut)[tid] =
+        __uint_as_float(e > 1 ? ((e - 1) << 23) : (e ? 0x00400000u : 0x00200000u));
+  }
   __syncthreads();
 
   // ------------------------------------------------------------ P0
@@ -952,14 +1016,32 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
   }
   __syncthreads();
   const int nsg = misc[1], nrg = misc[2];
-  const int n_units = nsg * (p.fs / kDecRows) + nrg * (p.f / kDecRows) + (nsg + nrg) * (d / kDecRows);
+  const int n_units = nsg * (p.fs / kDecRows) + nrg * (p.f / kDecRows) + (nsg + nrg) * (d / kDecRows2);
   const int fmax = max(p.f, p.fs);
 
   if (warp == kDecProducerWarp) {
     // ============================================================ producer
-    int n = 0, np = 0;  // stages and plane buffers issued
+    DecRing rg{0, 0, 0};  // stages issued
+    int np = 0;           // plane buffers issued
     if (lane == 0) {
-      for (int ui = blockIdx.x; ui < n_units && !*abort_flag; ui += p.G) {
+      // units are claimed dynamically: the CTA's first is blockIdx.x, every
+      // later one comes from the launch-wide counter, claimed one unit ahead
+      int ui = blockIdx.x;
+      while (!*abort_flag) {
+        if (ui >= n_units) {
+          // no more units: hand the consumers a -1 through the next plane buffer
+          const int pb = np & 1;
+          if (np >= 2 && !dec_wait_bar(pempty0 + 8 * pb, ((np >> 1) - 1) & 1, abort_flag, true)) {
+            set_error(p.err, kErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          misc[8 + (np & 3)] = -1;
+          dec_arrive(pfull0 + 8 * pb);
+          ++np;
+          break;
+        }
+        const int ui_next = p.G + atomicAdd(p.sync + 2, 1);
         const DecUnit U = dec_unit(p, r_groups, nsg, nrg, ui);
         const int4 grp = r_groups[U.grp];
         const DecMat& m0 = p.m[U.mi];
@@ -969,8 +1051,39 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
         const uint32_t box_bytes = (uint32_t)(m0.R * m0.seg);
         const uint32_t sc_bytes = (uint32_t)(m0.R * m0.spitch);
         const uint32_t tx = (s1 ? 2u : 1u) * (box_bytes + sc_bytes * nsb);
+        const int nrs = s1 ? kDecRows / kDecR1 : kDecRows2 / kDecR2;
+        const int nst = nrs * m0.nch;  // stages of the unit, row set by row set
+        // one stage: codes of the row set's rows (and their W3 twins) and scales
+        auto issue_stage = [&](int st) -> bool {
+          const int rs = st / m0.nch, chn = st - rs * m0.nch;
+          const int s = rg.s;
+          if (rg.n >= p.nslot && !dec_wait_bar(empty0 + 8 * s, rg.ph ^ 1, abort_flag, true)) {
+            set_error(p.err, kErrTimeout);
+            *abort_flag = 1;
+            return false;
+          }
+          const uint32_t slot = ring + s * p.slot_bytes, full = full0 + 8 * s;
+          const int row = U.row0 + rs * m0.R;
+          const int cx = chn * (m0.seg / m0.lb);
+          const int sxe = chn * m0.sK;
+          dec_expect_tx(full, tx);
+          for (int mm = 0; mm < (s1 ? 2 : 1); ++mm) {
+            const int mi = U.mi + mm;
+            dec_tma_3d(slot + mm * box_bytes, &p.map[mi], 0, row, cx, full);
+            const uint32_t sb = slot + kDecCodeBytes + mm * nsb * sc_bytes;
+            dec_tma_2d(sb, &p.smap[mi], sxe, row, full);
+            if (!mx) dec_tma_2d(sb + sc_bytes, &p.bmap[mi], sxe, row, full);
+          }
+          rg.next(p.nslot);
+          return true;
+        };
+        int st = 0;
         if (!s1) {
-          // W2 stages read the group's h planes: wait for all its S1 units
+          // W2 weights do not depend on h: fill the ring with the unit's first
+          // stages, then wait until the group's S1 units are all counted
+          for (; st < nst && st < p.nslot; ++st)
+            if (!issue_stage(st)) break;
+          if (*abort_flag) break;
           const int target = p.stall_test ? 0x3fffffff : (grp.x < 0 ? p.fs / kDecRows : p.f / kDecRows);
           if (!dec_wait_count(p.cnt_h + U.grp, target, abort_flag, p.stall_test ? 2000000LL : kDecWaitCycles)) {
             set_error(p.err, kErrTimeout);
@@ -982,13 +1095,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
         {
           // the unit's activation rows (planes and block records) for every token of the group
           const int pb = np & 1;
-          if (np >= 2 && !dec_wait_bar(pempty0 + 8 * pb, ((np >> 1) - 1) & 1, abort_flag)) {
+          if (np >= 2 && !dec_wait_bar(pempty0 + 8 * pb, ((np >> 1) - 1) & 1, abort_flag, true)) {
             set_error(p.err, kErrTimeout);
             *abort_flag = 1;
             break;
           }
           const uint32_t pl = planes0 + pb * p.pbuf;
           const int nin = m0.n_in;
+          misc[8 + (np & 3)] = ui;
           dec_expect_tx(pfull0 + 8 * pb, (uint32_t)grp.z * (uint32_t)(nin * 2 + (nin / 64) * 16));
           for (int i = 0; i < grp.z; ++i) {
             const uint8_t* src;
@@ -1007,32 +1121,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
           }
           ++np;
         }
-        const int nrs = s1 ? kDecRows / kDecR1 : kDecRows / kDecR2;
-        for (int rs = 0; rs < nrs && !*abort_flag; ++rs) {
-          for (int chn = 0; chn < m0.nch; ++chn, ++n) {
-            const int s = n % p.nslot;
-            if (n >= p.nslot && !dec_wait_bar(empty0 + 8 * s, ((n / p.nslot) - 1) & 1, abort_flag)) {
-              set_error(p.err, kErrTimeout);
-              *abort_flag = 1;
-              break;
-            }
-            const uint32_t slot = ring + s * p.slot_bytes, full = full0 + 8 * s;
-            const int row = U.row0 + rs * m0.R;
-            const int cx = chn * (m0.seg / m0.lb);
-            const int sxe = chn * m0.sK;
-            dec_expect_tx(full, tx);
-            for (int mm = 0; mm < (s1 ? 2 : 1); ++mm) {
-              const int mi = U.mi + mm;
-              dec_tma_3d(slot + mm * box_bytes, &p.map[mi], 0, row, cx, full);
-              const uint32_t sb = slot + kDecCodeBytes + mm * nsb * sc_bytes;
-              dec_tma_2d(sb, &p.smap[mi], sxe, row, full);
-              if (!mx) dec_tma_2d(sb + sc_bytes, &p.bmap[mi], sxe, row, full);
-            }
-          }
-        }
+        for (; st < nst; ++st)
+          if (!issue_stage(st)) break;
+        ui = ui_next;
       }
       // drain: every issued copy must land before the block exits
-      for (int q = max(0, n - p.nslot); q < n; ++q) {
+      for (int q = max(0, rg.n - p.nslot); q < rg.n; ++q) {
         const long long t0 = clock64();
         while (!dec_try_wait(full0 + 8 * (q % p.nslot), (q / p.nslot) & 1) && clock64() - t0 < kDecWaitCycles) {
         }
@@ -1047,22 +1141,22 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
   } else if (warp == kDecServiceWarp) {
     // ============================================================ service
     // Unit epilogues that wait on global memory, off the consumers' path:
-    // S1: the h block of every token -> W2's planes, then the group's count;
-    // S2: the output block's count, and the combine by its last arriver.
+    // S1: the h block of every token -> W2's planes, then the group's count.
     int* scr = reinterpret_cast<int*>(fx + kDecFxScr);
-    int ne = 0;
-    for (int ui = blockIdx.x; ui < n_units; ui += p.G, ++ne) {
-      const DecUnit U = dec_unit(p, r_groups, nsg, nrg, ui);
-      const int4 grp = r_groups[U.grp];
+    for (int ne = 0;; ++ne) {
       const int eb = ne & 1;
       bool ok = !*abort_flag;
-      if (ok && !dec_wait_bar(efull0 + 8 * eb, (ne >> 1) & 1, abort_flag)) {
+      if (ok && !dec_wait_bar(efull0 + 8 * eb, (ne >> 1) & 1, abort_flag, true)) {
         if (lane == 0) set_error(p.err, kErrTimeout);
         *abort_flag = 1;
         ok = false;
       }
-      ok = __all_sync(0xffffffffu, ok);
-      if (ok && U.stage == 1) {
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int ui = misc[12 + eb];
+      if (ui < 0) break;
+      const DecUnit U = dec_unit(p, r_groups, nsg, nrg, ui);
+      const int4 grp = r_groups[U.grp];
+      if (U.stage == 1) {
         const float* hb = hbuf + eb * kDecMaxTok * kDecRows;
         const int f2 = grp.x < 0 ? p.m[DM_S2].fmt : p.m[DM_W2].fmt;
         for (int i = 0; i < grp.z; ++i) {
@@ -1077,73 +1171,66 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
           __threadfence();
           red_release_add(p.cnt_h + U.grp, 1);
         }
-      } else if (ok) {
-        int last = 0;
-        if (lane == 0) {
-          __threadfence();
-          last = atomicAdd(p.cnt_y + U.u, 1) + 1 == nsg + nrg;
-          if (last) __threadfence();
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          // every slot of this 64-column block is final: out = sum_j w y (+ shared), one rounding
-          for (int i = lane; i < T * kDecRows; i += 32) {
-            const int t = i / kDecRows, col = kDecRows * U.u + (i % kDecRows);
-            float sacc = 0.f;
-            for (int j = 0; j < k; ++j) sacc = fmaf(r_w[t * k + j], __ldcg(p.y + (size_t)(t * k + j) * d + col), sacc);
-            if (p.has_shared) sacc += __ldcg(p.y + (size_t)(Tk + t) * d + col);
-            p.out[(size_t)t * d + col] = __float2bfloat16_rn(sacc);
-          }
-          __syncwarp();
-          if (lane == 0) p.cnt_y[U.u] = 0;
-        }
       }
       __syncwarp();
       if (lane == 0) dec_arrive(eempty0 + 8 * eb);
     }
   } else {
     // ============================================================ consumers
-    const int tt = warp & 1, kq = warp >> 1;  // row tile, input slice
-    int n = 0, np = 0, ne = 0;
-    for (int ui = blockIdx.x; ui < n_units; ui += p.G, ++ne) {
+    const int kq = warp;  // input slice (both row tiles)
+    DecRing rg{0, 0, 0};
+    int np = 0;
+    for (int ne = 0;; ++ne) {
+      // the unit comes with its plane buffer; warp 0's view decides for every warp
+      const int pb = np & 1;
+      const bool have_pl = dec_consumer_wait(pfull0 + 8 * pb, (np >> 1) & 1, abort_flag, p.err);
+      if (tid == 0) misc[4] = have_pl ? misc[8 + (np & 3)] : -1;
+      asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerThreads) : "memory");
+      const int ui = misc[4];
+      const int eb = ne & 1;
+      bool have_e = true;
+      if (ne >= 2) have_e = dec_consumer_wait(eempty0 + 8 * eb, ((ne >> 1) - 1) & 1, abort_flag, p.err);
+      if (ui < 0) {  // no more units: tell the service warp
+        if (tid == 0) misc[12 + eb] = -1;
+        __syncwarp();
+        if (lane == 0) dec_arrive(efull0 + 8 * eb);
+        break;
+      }
       const DecUnit U = dec_unit(p, r_groups, nsg, nrg, ui);
       const int4 grp = r_groups[U.grp];
       const DecMat& m0 = p.m[U.mi];
       const bool s1 = U.stage == 1;
       DecWarp q;
       const int nsb = m0.fmt == F_MX4 ? 1 : 2;
+      q.lut = su32(fx + kDecFxLut);
       q.R = m0.R;
       q.kq = kq;
       q.spitch = m0.spitch;
       q.ptok = m0.ptok;
       q.sxtok = m0.sxtok;
-      if (s1) {  // A rows 0..7: W1 rows tt*8.., rows 8..15: the same rows of W3
+      if (s1) {  // tile t: A rows 0..7 = W1 rows t*8.., rows 8..15 = the same rows of W3
         q.a0 = 0;
         q.a8 = m0.R * m0.seg;
-        q.r0 = q.r8 = tt * 8;
+        q.r0 = q.r8 = 0;
+        q.tstep = 8;
         q.s0 = kDecCodeBytes;
         q.s8 = kDecCodeBytes + nsb * m0.R * m0.spitch;
-      } else {  // A rows 0..15: W2 rows tt*16..
+      } else {  // tile t: A rows 0..15 = W2 rows t*16..
         q.a0 = q.a8 = 0;
-        q.r0 = tt * 16;
-        q.r8 = tt * 16 + 8;
+        q.r0 = 0;
+        q.r8 = 8;
+        q.tstep = 16;
         q.s0 = q.s8 = kDecCodeBytes;
       }
-      const int pb = np & 1;
-      const bool have_pl = dec_consumer_wait(pfull0 + 8 * pb, (np >> 1) & 1, abort_flag, p.err);
       const uint32_t pl = planes0 + pb * p.pbuf;
       dec_consume_any(m0.fmt, m0.group, m0.nbw, q, s1, m0.nch, m0.K, grp.z, ring, p.slot_bytes, p.nslot, pl,
-                      pl + p.sx_off, full0, empty0, n, have_pl, abort_flag, p.err, red, tt);
+                      pl + p.sx_off, full0, empty0, rg, have_pl, abort_flag, p.err, red);
       __syncwarp();
       if (lane == 0 && have_pl) dec_arrive(pempty0 + 8 * pb);
       ++np;
-      // this unit's epilogue buffer must be free (the service warp is done with unit ne - 2)
-      const int eb = ne & 1;
-      bool have_e = true;
-      if (ne >= 2) have_e = dec_consumer_wait(eempty0 + 8 * eb, ((ne >> 1) - 1) & 1, abort_flag, p.err);
       asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerThreads) : "memory");  // every slice partial is in red
-      if (tid < kDecMaxTok * kDecRows) {
-        const int r = tid >> 2, tok = tid & 3;  // the unit's output row, token
+      for (int i = tid; i < kDecMaxTok * (s1 ? kDecRows : kDecRows2); i += kDecConsumerThreads) {
+        const int r = i >> 2, tok = i & 3;  // the unit's output row, token
         if (tok < grp.z) {
           if (s1) {
             const int rs = r >> 4, row = r & 15;
@@ -1159,25 +1246,61 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
             const int rs = r >> 5, row = r & 31;
             float v = 0.f;
 #pragma unroll
-            for (int sl = 0; sl < kDecNkq; ++sl) v += red[((sl * 2 + rs) * 32 + row) * 4 + tok];  // fixed order
-            p.y[(size_t)dec_slot(p, r_sorted, grp, tok) * d + kDecRows * U.u + r] = v;
+            for (int sl = 0; sl < kDecNkq; ++sl) v += red[((sl * 4 + rs) * 32 + row) * 4 + tok];  // fixed order
+            p.y[(size_t)dec_slot(p, r_sorted, grp, tok) * d + kDecRows2 * U.u + r] = v;
           }
         }
       }
+      if (tid == 0) misc[12 + eb] = ui;
       asm volatile("bar.sync 1, %0;" ::"r"(kDecConsumerThreads) : "memory");  // red is free, the h block complete
       if (lane == 0) dec_arrive(efull0 + 8 * eb);
     }
   }
-  // ------------------------------------------------------------ exit
+  // ------------------------------------------------------------ combine
+  // Every y slot is final once the whole grid is here: out = sum_j w y (+ the
+  // shared expert), ascending j, one rounding; a thread per 4 columns of a
+  // token, its k slot loads issued together.
   __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(p.sync + 2, 1) == p.G - 1) {
-      for (int i = 0; i < nsg + nrg; ++i) p.cnt_h[i] = 0;
-      for (int i = 0; i < d / kDecRows; ++i) p.cnt_y[i] = 0;
-      p.sync[2] = 0;
-      __threadfence();
+  dec_grid_barrier(p.sync, p.G, p.err, abort_flag);
+  {
+    const int nc4 = d / 4;
+    for (int i = blockIdx.x * kDecThreads + tid; i < T * nc4; i += p.G * kDecThreads) {
+      const int t = i / nc4, c4 = (i - t * nc4) * 4;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int j0 = 0; j0 < k; j0 += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          if (j0 + jj < k) v[jj] = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)(t * k + j0 + jj) * d + c4));
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          if (j0 + jj < k) {
+            const float wj = r_w[t * k + j0 + jj];
+            a.x = fmaf(wj, v[jj].x, a.x);
+            a.y = fmaf(wj, v[jj].y, a.y);
+            a.z = fmaf(wj, v[jj].z, a.z);
+            a.w = fmaf(wj, v[jj].w, a.w);
+          }
+        }
+      }
+      if (p.has_shared) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)(Tk + t) * d + c4));
+        a.x += v.x;
+        a.y += v.y;
+        a.z += v.z;
+        a.w += v.w;
+      }
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
+      uint2 o;
+      o.x = *reinterpret_cast<const uint32_t*>(&lo);
+      o.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(p.out + (size_t)t * d + c4) = o;
     }
+  }
+  // every unit is done: the dependency counters start the next launch at zero
+  if (blockIdx.x == 0) {
+    for (int i = tid; i < nsg + nrg; i += kDecThreads) p.cnt_h[i] = 0;
+    if (tid == 0) p.sync[2] = 0;  // the unit counter
   }
 }
 

@@ -95,7 +95,7 @@ struct WsLayout {
   size_t hdr, logits, ids, wts, offsets, sorted, inv, active, h, y, xstage, tokstage, outstage;
   size_t x16, tiles, tiles2, ntiles;  // tensor-core FFN: fp16 token rows by position, token-tile plans
   size_t pchunks;                     // multi-CTA permutation: per-chunk expert counts / bases
-  size_t dxp, dxsx, dhp, dhsx, dcnth, dcnty, dsync;  // fused decode: planes, block steps, counters
+  size_t dxp, dxsx, dhp, dhsx, dcnth, dsync;  // fused decode: planes, block steps, counters
   bool tc = false;            // the regions above exist
   size_t total;
 };
@@ -141,7 +141,6 @@ WsLayout layout_of(const moe_dims_t& d) {
     L.dhp = take(dec ? P * fm * 4 : 0);
     L.dhsx = take(dec ? P * (fm / 64 + 1) * 16 : 0);
     L.dcnth = take(dec ? (kDecMaxPairs + 8) * sizeof(int) : 0);
-    L.dcnty = take(dec ? (D / 64 + 1) * sizeof(int) : 0);
     L.dsync = take(dec ? 4 * sizeof(int) : 0);
   }
   L.tc = true;
@@ -960,7 +959,6 @@ moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32
   p.hsx = ws_at<float4>(ws, L.dhsx);
   p.y = ws_at<float>(ws, L.y);
   p.cnt_h = ws_at<int>(ws, L.dcnth);
-  p.cnt_y = ws_at<int>(ws, L.dcnty);
   p.sync = ws_at<int>(ws, L.dsync);
   p.err = &ws_at<WsHeader>(ws, L.hdr)->err;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
