@@ -20,6 +20,7 @@ from ._lib import (  # noqa: F401
     expert_ffn_noalloc,
     forward,
     forward_host,
+    forward_partial,
     hc_sinkhorn_mix,
     load_library,
     make_dims,
@@ -34,4 +35,4 @@ from ._lib import (  # noqa: F401
     timing_labels,
     workspace_size,
 )
-from .layer import MoELayer  # noqa: F401
+from .layer import MoELayer, expert_range  # noqa: F401

@@ -55,6 +55,10 @@ _SIGS = {
     "moe_forward": (ctypes.c_int, [ctypes.POINTER(Dims), _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(QMatC),
                                    ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP, _VP,
                                    _VP, _VP, ctypes.c_size_t, _VP]),
+    "moe_forward_partial": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _VP,
+                                           _VP, _VP, _VP, _VP, ctypes.POINTER(QMatC), ctypes.POINTER(QMatC),
+                                           ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP, _VP, _VP, _VP,
+                                           ctypes.c_size_t, _VP]),
     "moe_forward_host": (ctypes.c_int, [ctypes.POINTER(Dims), _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(QMatC),
                                         ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP,
                                         _VP, ctypes.c_size_t, _VP]),
@@ -189,6 +193,21 @@ def forward(dims, x, token_ids, router_w, router_b, tid2eid, w1, w3, w2, shared,
         ctypes.byref(dims), _ptr(x), _ptr(token_ids), _ptr(router_w), _ptr(router_b), _ptr(tid2eid),
         ctypes.byref(q1), ctypes.byref(q3), ctypes.byref(q2), sh, _ptr(out), _ptr(topk_ids_out),
         _ptr(topk_w_out), _ptr(ws), ws.numel(), _stream(stream)), "moe_forward")
+
+
+def forward_partial(dims, expert_begin, expert_end, include_shared, x, token_ids, router_w, router_b, tid2eid,
+                    w1, w3, w2, shared, out_partial, ws, topk_ids_out=None, topk_w_out=None, stream=None):
+    """moe_forward_partial: the fp32 partial output [T, d_model] of experts
+    expert_begin <= e < expert_end (plus the shared expert when include_shared)."""
+    if out_partial.dtype != torch.float32:
+        raise ValueError("out_partial must be float32")
+    q1, q3, q2 = qmat(w1), qmat(w3), qmat(w2)
+    sh = _shared_arr(shared)
+    _check(load_library().moe_forward_partial(
+        ctypes.byref(dims), int(expert_begin), int(expert_end), 1 if include_shared else 0, _ptr(x), _ptr(token_ids),
+        _ptr(router_w), _ptr(router_b), _ptr(tid2eid), ctypes.byref(q1), ctypes.byref(q3), ctypes.byref(q2), sh,
+        _ptr(out_partial), _ptr(topk_ids_out), _ptr(topk_w_out), _ptr(ws), ws.numel(), _stream(stream)),
+        "moe_forward_partial")
 
 
 def forward_host(dims, x_host: torch.Tensor, token_ids_host, router_w, router_b, tid2eid, w1, w3, w2, shared,

@@ -146,6 +146,11 @@ struct DecParams {
   int* ids_out;        // [T][k] or NULL
   float* w_out;        // [T][k] or NULL
   int stall_test;      // testing the timeout path: the first W2 dependency waits on a count nothing reaches
+  // expert parallelism: only experts e_begin <= e < e_end run and enter the
+  // combine, the shared expert only when with_shared; out_f32 (when not
+  // NULL) receives the fp32 partial instead of the bf16 output
+  int e_begin, e_end, with_shared;
+  float* out_f32;
 };
 
 // ------------------------------------------------------------ grid barrier
@@ -953,14 +958,14 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     // offsets (exclusive scan), cursors and groups: lane l owns experts
     // [l*per, (l+1)*per); groups in ascending expert order after the shared ones
     const int gsz = p.ntmax;
-    const int nsg = p.has_shared ? (T + gsz - 1) / gsz : 0;
+    const int nsg = p.has_shared && p.with_shared ? (T + gsz - 1) / gsz : 0;
     const int per = (E + 31) / 32;
     const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
     int s = 0, ng = 0;
     for (int e = e0; e < e1; ++e) {
       const int c = r_off[e];
       s += c;
-      ng += (c + gsz - 1) / gsz;
+      if (e >= p.e_begin && e < p.e_end) ng += (c + gsz - 1) / gsz;
     }
     int sx = s, gx = ng;  // inclusive warp scans
 #pragma unroll
@@ -976,7 +981,8 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
       const int c = r_off[e];
       r_off[e] = run;
       r_cur[e] = run;
-      for (int q0 = 0; q0 < c; q0 += gsz) r_groups[gi++] = make_int4(e, run + q0, min(gsz, c - q0), 0);
+      if (e >= p.e_begin && e < p.e_end)
+        for (int q0 = 0; q0 < c; q0 += gsz) r_groups[gi++] = make_int4(e, run + q0, min(gsz, c - q0), 0);
       run += c;
     }
     if (lane == 31) {
@@ -1269,12 +1275,20 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
       float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int j0 = 0; j0 < k; j0 += 4) {
         float4 v[4];
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          if (j0 + jj < k) v[jj] = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)(t * k + j0 + jj) * d + c4));
+        bool own[4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
+          own[jj] = false;
           if (j0 + jj < k) {
+            int e = r_ids[t * k + j0 + jj];
+            if (e < 0 || e >= E) e = 0;  // as counted in P1
+            own[jj] = e >= p.e_begin && e < p.e_end;
+            if (own[jj]) v[jj] = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)(t * k + j0 + jj) * d + c4));
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          if (own[jj]) {
             const float wj = r_w[t * k + j0 + jj];
             a.x = fmaf(wj, v[jj].x, a.x);
             a.y = fmaf(wj, v[jj].y, a.y);
@@ -1283,12 +1297,16 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
           }
         }
       }
-      if (p.has_shared) {
+      if (p.has_shared && p.with_shared) {
         const float4 v = __ldcg(reinterpret_cast<const float4*>(p.y + (size_t)(Tk + t) * d + c4));
         a.x += v.x;
         a.y += v.y;
         a.z += v.z;
         a.w += v.w;
+      }
+      if (p.out_f32 != nullptr) {
+        *reinterpret_cast<float4*>(p.out_f32 + (size_t)t * d + c4) = a;
+        continue;
       }
       const __nv_bfloat162 lo = __floats2bfloat162_rn(a.x, a.y), hi = __floats2bfloat162_rn(a.z, a.w);
       uint2 o;

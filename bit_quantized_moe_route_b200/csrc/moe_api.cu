@@ -923,10 +923,17 @@ moe_status_t dec_maps(DecParams& p, int i, const QMatDev& Q, int E) {
                  m.spitch / 2, m.R, false);
 }
 
+// An expert slice of the layer (expert parallelism): experts [e_begin,
+// e_end), the shared expert when with_shared, fp32 partial to out_f32.
+struct DecPart {
+  int e_begin, e_end, with_shared;
+  float* out_f32;
+};
+
 moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32_t* token_ids, const void* router_w,
                                  const float* router_b, const int32_t* tid2eid, const QMatDev& q1, const QMatDev& q3,
                                  const QMatDev& q2, const QMatDev* qs, void* out, int32_t* ids_out, float* w_out,
-                                 void* ws, const WsLayout& L, cudaStream_t s, const DevInfo& di) {
+                                 void* ws, const WsLayout& L, cudaStream_t s, const DevInfo& di, const DecPart& part) {
   DecParams p{};
   size_t smem = 0;
   if (!dec_plan(d, q1, q3, q2, qs, &p, &smem)) return fail(MOE_ERR_UNSUPPORTED, "shapes outside the fused kernel");
@@ -965,6 +972,10 @@ moe_status_t launch_decode_fused(const moe_dims_t& d, const void* x, const int32
   p.ids_out = ids_out;
   p.w_out = w_out;
   p.stall_test = g_stall_test;
+  p.e_begin = part.e_begin;
+  p.e_end = part.e_end;
+  p.with_shared = part.with_shared;
+  p.out_f32 = part.out_f32;
   p.G = di.dec_blocks;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;  // every CTA resident: the kernel's CTAs wait on one another
@@ -1207,6 +1218,47 @@ moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* t
   return st;
 }
 
+moe_status_t moe_forward_partial(const moe_dims_t* dims, int32_t expert_begin, int32_t expert_end,
+                                 int32_t include_shared, const void* x, const int32_t* token_ids,
+                                 const void* router_w, const float* router_b, const int32_t* tid2eid,
+                                 const moe_qmat_t* w1, const moe_qmat_t* w3, const moe_qmat_t* w2,
+                                 const moe_qmat_t* shared, float* out_partial, int32_t* topk_ids_out,
+                                 float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  g_detail[0] = 0;
+  moe_status_t st = check_dims(dims);
+  if (st != MOE_OK) return st;
+  const moe_dims_t& d = *dims;
+  if (expert_begin < 0 || expert_begin > expert_end || expert_end > d.n_experts)
+    return fail(MOE_ERR_INVALID_ARG, "expert range [%d, %d) outside [0, %d]", expert_begin, expert_end, d.n_experts);
+  if (include_shared != 0 && include_shared != 1) return fail(MOE_ERR_INVALID_ARG, "include_shared must be 0 or 1");
+  WsLayout L;
+  if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
+  if ((st = check_route_args(d, x, router_w, token_ids, tid2eid)) != MOE_OK) return st;
+  if ((st = check_dev_ptr(out_partial, "out_partial")) != MOE_OK) return st;
+  if (!aligned16(out_partial)) return fail(MOE_ERR_INVALID_ARG, "out_partial must be 16-byte aligned");
+  QMatDev q1, q3, q2, qs[3];
+  if ((st = check_qmat(w1, d.d_model, "w1", &q1, d.d_ff)) != MOE_OK) return st;
+  if ((st = check_qmat(w3, d.d_model, "w3", &q3, d.d_ff)) != MOE_OK) return st;
+  if ((st = check_qmat(w2, d.d_ff, "w2", &q2, d.d_model)) != MOE_OK) return st;
+  if (d.d_ff_shared > 0) {
+    if (!shared) return fail(MOE_ERR_INVALID_ARG, "d_ff_shared > 0 but shared is NULL");
+    if ((st = check_qmat(&shared[0], d.d_model, "shared w1", &qs[0], d.d_ff_shared)) != MOE_OK) return st;
+    if ((st = check_qmat(&shared[1], d.d_model, "shared w3", &qs[1], d.d_ff_shared)) != MOE_OK) return st;
+    if ((st = check_qmat(&shared[2], d.d_ff_shared, "shared w2", &qs[2], d.d_model)) != MOE_OK) return st;
+  }
+  DevInfo* di;
+  if ((st = dev_info(&di)) != MOE_OK) return st;
+  const QMatDev* sh = d.d_ff_shared > 0 ? qs : nullptr;
+  if (di->dec_blocks <= 0 || !dec_eligible(d, q1, q3, q2, sh))
+    return fail(MOE_ERR_UNSUPPORTED, "expert slices run on the fused single-launch path only (T <= %d)", kDecMaxT);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  hook_begin(s);
+  st = launch_decode_fused(d, x, token_ids, router_w, router_b, tid2eid, q1, q3, q2, sh, nullptr, topk_ids_out,
+                           topk_w_out, ws, L, s, *di, DecPart{expert_begin, expert_end, include_shared, out_partial});
+  hook_end();
+  return st;
+}
+
 }  // extern "C"
 
 namespace {
@@ -1222,7 +1274,7 @@ moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t*
     const QMatDev* sh = d.d_ff_shared > 0 ? qs : nullptr;
     if (di->dec_blocks > 0 && use_dec(d, q1, q3, q2, sh))
       return launch_decode_fused(d, x, token_ids, router_w, router_b, tid2eid, q1, q3, q2, sh, out, topk_ids_out,
-                                 topk_w_out, ws, L, s, *di);
+                                 topk_w_out, ws, L, s, *di, DecPart{0, (int)d.n_experts, 1, nullptr});
     if (g_ffn_path == MOE_FFN_DECODE_FUSED)
       return fail(MOE_ERR_UNSUPPORTED, "the fused decode path does not take these shapes or formats");
   }

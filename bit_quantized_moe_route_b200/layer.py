@@ -8,6 +8,16 @@ import torch
 from . import _lib
 
 
+def expert_range(rank: int, world: int, n_experts: int) -> tuple:
+    """Contiguous expert slice [begin, end) owned by `rank` of `world` in the
+    expert-parallel split (routing replicated, each rank runs its experts and
+    the partial outputs are all-reduced; the shared expert goes to rank 0).
+    Slices differ in size by at most one expert."""
+    if not 0 <= rank < world:
+        raise ValueError(f"rank {rank} outside [0, {world})")
+    return rank * n_experts // world, (rank + 1) * n_experts // world
+
+
 class MoELayer:
     """Holds the packed experts, router and workspace of one routed-MoE layer.
 

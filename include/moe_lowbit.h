@@ -266,6 +266,29 @@ moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* t
                          float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * One expert slice of the layer, for expert parallelism (no counterpart on
+ * the pages; the layer's combine is a sum over (token, slot) terms, so it
+ * splits by expert): routing runs over all n_experts as in moe_forward, but
+ * only experts expert_begin <= e < expert_end run, only their slots enter
+ * the combine, and the shared expert is added when include_shared is 1.
+ *   out_partial : fp32 [T, d_model], 16-byte aligned:
+ *     out_partial[t] = sum_{j<k, e(t,j) in range} topk_w[t,j] * y[t,j]
+ *                      (+ y_shared[t]), ascending j, fp32, no rounding to bf16
+ * Ranks owning a partition of [0, n_experts), the shared expert on exactly
+ * one of them, add (all-reduce) their partials to the layer's output before
+ * its bf16 rounding.  Runs on the fused single-launch path: T <= 32 and the
+ * shapes that path admits; otherwise MOE_ERR_UNSUPPORTED.  A range outside
+ * [0, n_experts] or include_shared not 0/1: MOE_ERR_INVALID_ARG.  Other
+ * arguments as in moe_forward.
+ */
+moe_status_t moe_forward_partial(const moe_dims_t* dims, int32_t expert_begin, int32_t expert_end,
+                                 int32_t include_shared, const void* x, const int32_t* token_ids,
+                                 const void* router_w, const float* router_b, const int32_t* tid2eid,
+                                 const moe_qmat_t* w1, const moe_qmat_t* w3, const moe_qmat_t* w2,
+                                 const moe_qmat_t* shared, float* out_partial, int32_t* topk_ids_out,
+                                 float* topk_w_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * moe_forward with HOST activations: x_host (bf16 [T, d_model]) and, in hash
  * mode, token_ids_host (int32 [T]) are copied to the workspace, the layer
  * runs, and the bf16 result is copied back to out_host.  Weights, router and

@@ -314,7 +314,9 @@ def forward(dims: Dict, x: np.ndarray, *, router_w=None, router_b=None, token_id
             tid2eid=None, fetch: ExpertFetch, fmts: Dict[str, Tuple[str, int, int]],
             shared_fetch: Optional[ExpertFetch] = None, shared_fmts=None,
             tokens: Optional[Sequence[int]] = None,
-            forced_ids: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+            forced_ids: Optional[np.ndarray] = None,
+            expert_range: Optional[Tuple[int, int]] = None,
+            include_shared: bool = True) -> Dict[str, np.ndarray]:
     """Run the layer for all tokens' routing and the requested tokens' outputs.
 
     dims: T, d, E, k, f, f_shared, routing ("learned"|"hash").
@@ -324,6 +326,12 @@ def forward(dims: Dict, x: np.ndarray, *, router_w=None, router_b=None, token_id
     forced_ids: int [T, k] -- learned routing only: use these experts instead
     of the top-k selection (weights as in route_forced); "gap" is then the
     free routing's gap, so near-tie tokens can still be recognised.
+    expert_range: (begin, end) -- expert parallelism: routing over all E
+    experts as usual, but only experts begin <= e < end are run and only their
+    slots enter the combine; the shared expert is added when include_shared.
+    The layer's output is the sum of such partials over a partition of
+    [0, E) with the shared expert in exactly one of them, because the combine
+    is a sum over (token, slot) terms.
     """
     T, d, E, k, f = dims["T"], dims["d"], dims["E"], dims["k"], dims["f"]
     xs = np.asarray(x, np.float64)
@@ -348,10 +356,15 @@ def forward(dims: Dict, x: np.ndarray, *, router_w=None, router_b=None, token_id
 
     tok = np.arange(T) if tokens is None else np.asarray(tokens, np.int64)
     y = np.zeros((len(tok), k, d))
+    eb, ee = (0, E) if expert_range is None else (int(expert_range[0]), int(expert_range[1]))
+    if not 0 <= eb <= ee <= E:
+        raise ValueError(f"expert_range {expert_range} outside [0, {E}]")
+    owned = (ids >= eb) & (ids < ee)
     need: Dict[int, list] = {}
     for a, t in enumerate(tok):
         for j in range(k):
-            need.setdefault(int(ids[t, j]), []).append((a, j))
+            if owned[t, j]:
+                need.setdefault(int(ids[t, j]), []).append((a, j))
     dims_of = {"w1": (f, d), "w3": (f, d), "w2": (d, f)}
     for e in sorted(need):
         W = {}
@@ -363,7 +376,7 @@ def forward(dims: Dict, x: np.ndarray, *, router_w=None, router_b=None, token_id
         for r, (a, j) in enumerate(need[e]):
             y[a, j] = ye[r]
     y_sh = None
-    if shared_fetch is not None:
+    if shared_fetch is not None and include_shared:
         fs = dims["f_shared"]
         dsh = {"w1": (fs, d), "w3": (fs, d), "w2": (d, fs)}
         Ws = {}
@@ -374,7 +387,7 @@ def forward(dims: Dict, x: np.ndarray, *, router_w=None, router_b=None, token_id
         res["y_shared"] = y_sh
     res["tokens"] = tok
     res["y_slots"] = y
-    res["out"] = combine(y, w[tok], y_sh)
+    res["out"] = combine(y, np.where(owned, w, 0.0)[tok], y_sh)
     res["out_bf16"] = round_bf16(res["out"])
     return res
 

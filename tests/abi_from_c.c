@@ -35,6 +35,11 @@ int main(void) {
   EXPECT(st == MOE_ERR_INVALID_ARG);
   EXPECT(strlen(moe_last_error_detail()) > 0);
 
+  /* an expert slice past n_experts */
+  st = moe_forward_partial(&decode, 0, decode.n_experts + 1, 1, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
+                           NULL, NULL, NULL, NULL, ws, 256, NULL);
+  EXPECT(st == MOE_ERR_INVALID_ARG);
+
   st = moe_permute(&no_k, NULL, NULL, NULL, NULL, ws, 256, NULL);
   EXPECT(st == MOE_ERR_INVALID_ARG);
 

@@ -13,11 +13,12 @@ def dims_of(inp):
                 routing=c["routing"])
 
 
-def oracle_run(inp, tokens=None, forced_ids=None):
+def oracle_run(inp, tokens=None, forced_ids=None, expert_range=None, include_shared=True):
     """Run the fp64 oracle on MoEInputs (tensors may live on any device).
 
     forced_ids: optional int [T, k] experts to use instead of the oracle's own
-    top-k (the oracle's forced-routing mode)."""
+    top-k (the oracle's forced-routing mode).  expert_range / include_shared:
+    the partial output of the experts begin <= e < end (expert parallelism)."""
     fmts = {n: (m.fmt, m.bits, m.group) for n, m in
             (("w1", inp.w1), ("w3", inp.w3), ("w2", inp.w2))}
     mats = {"w1": inp.w1, "w3": inp.w3, "w2": inp.w2}
@@ -41,7 +42,8 @@ def oracle_run(inp, tokens=None, forced_ids=None):
         token_ids=None if inp.token_ids is None else inp.token_ids.cpu().numpy(),
         tid2eid=None if inp.tid2eid is None else inp.tid2eid.cpu().numpy(),
         fetch=fetch, fmts=fmts, shared_fetch=shared_fetch, shared_fmts=shared_fmts,
-        tokens=tokens, forced_ids=None if forced_ids is None else np.asarray(forced_ids, np.int64))
+        tokens=tokens, forced_ids=None if forced_ids is None else np.asarray(forced_ids, np.int64),
+        expert_range=expert_range, include_shared=include_shared)
 
 
 def bigint_words(codes, bits):

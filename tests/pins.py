@@ -542,9 +542,40 @@ def pin_bf16_router_is_its_values():
     assert np.array_equal(ids, res["ids"]) and np.array_equal(w, res["w"])
 
 
+def pin_expert_partition():
+    """Expert parallelism: the partial of an expert range is the dense
+    mixture gated by the routing weights of the owned experts only (library
+    fp64 linear/silu on every expert), the shared expert added once; partials
+    over a partition of [0, E) (shared in one part) add up to the full layer,
+    and an empty range gives zero (or the shared expert alone)."""
+    from synthetic import CONFIGS
+    cfg = dict(CONFIGS["tiny"])
+    cfg.update(T=5, seed=51, shared=("affine", 8, 64), f_shared=128)
+    inp = make_custom(cfg)
+    full = oracle_run(inp)
+    E = cfg["E"]
+    cuts = [(0, 3), (3, 5), (5, E)]  # (3, 5) owns no (token, slot) pair of this draw: its partial is 0
+    parts = [oracle_run(inp, expert_range=r, include_shared=(i == 0)) for i, r in enumerate(cuts)]
+    total = sum(p["out"] for p in parts)
+    assert np.abs(total - full["out"]).max() / np.abs(full["out"]).max() < 1e-13
+    for i, (r, p) in enumerate(zip(cuts, parts)):
+        assert np.array_equal(p["ids"], full["ids"]) and np.array_equal(p["w"], full["w"])
+        owned = (full["ids"] >= r[0]) & (full["ids"] < r[1])
+        gated = {"ids": full["ids"], "w": np.where(owned, full["w"], 0.0)}
+        dense = _dense_reference(inp, gated)
+        if i > 0:  # the dense reference always adds the shared expert: take it out for the other parts
+            dense = dense - oracle_run(inp, expert_range=(0, 0))["out"]
+        assert np.abs(p["out"] - dense).max() / np.abs(full["out"]).max() < 1e-12
+    assert not parts[1]["out"].any()
+    none = oracle_run(inp, expert_range=(0, 0), include_shared=False)
+    assert not none["out"].any()
+    shared_only = oracle_run(inp, expert_range=(2, 2))
+    assert np.allclose(shared_only["out"], full["y_shared"], rtol=0, atol=0)
+
+
 ALL_PINS = [pin_e2m1_table, pin_e8m0, pin_unpack_golden, pin_unpack_bigint, pin_affine_dequant,
             pin_mxfp4_dequant, pin_sqrtsoftplus, pin_topk_bruteforce, pin_route_learned,
             pin_route_hash, pin_permutation, pin_dense_equivalence, pin_single_expert_swiglu,
             pin_round_bf16, pin_e4m3_table, pin_mxfp8_dequant, pin_block128_scales, pin_parity_stats,
             pin_forward_token_subset, pin_forced_routing, pin_hc_sinkhorn_softmax, pin_hc_sinkhorn_limits,
-            pin_hc_sinkhorn_fixed_point, pin_hc_mix, pin_bf16_router_is_its_values]
+            pin_hc_sinkhorn_fixed_point, pin_hc_mix, pin_bf16_router_is_its_values, pin_expert_partition]

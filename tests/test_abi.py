@@ -73,6 +73,11 @@ def test_host_validation_without_gpu(lib):
     # NULL workspace
     st = lib.moe_route(ctypes.byref(d), None, None, None, None, None, None, None, None, 0, None)
     assert st == 1 and b"workspace" in lib.moe_last_error_detail()
+    # expert slice outside [0, n_experts], include_shared not 0/1
+    assert lib.moe_forward_partial(ctypes.byref(d), 3, 9, 1, *([None] * 13), 0, None) == 1
+    assert b"expert range" in lib.moe_last_error_detail()
+    assert lib.moe_forward_partial(ctypes.byref(d), 0, 8, 2, *([None] * 13), 0, None) == 1
+    assert b"include_shared" in lib.moe_last_error_detail()
     # bad dims
     bad = _lib.make_dims(4, 256, 128, 8, 0)
     assert lib.moe_permute(ctypes.byref(bad), None, None, None, None, None, 0, None) == 1
