@@ -335,8 +335,50 @@ def reference_arm(args):
     dev = torch.device("cuda:0") if torch.cuda.is_available() else torch.device("cpu")
     names = CONFIG_ORDER if args.config == "all" else [args.config]
     for name in names:
+        if name.startswith("mhc") or name.startswith("mxfp8"):
+            reference_kernel_line(args, name, dev, 150.0 / len(names))
+            continue
         inp = make_inputs(name, dev, **overrides(args))
         reference_line(args, inp, 150.0 / len(names))
+
+
+def reference_kernel_line(args, name, dev, budget_total):
+    """Reference-arm line of a single-kernel workload (mHC mixing, mxfp8
+    rows): the oracle on a bounded sample, in the metric of our line."""
+    if name.startswith("mhc"):
+        from synthetic import HC_CONFIGS, make_hc_inputs
+        cfg = dict(HC_CONFIGS[name], name=name)
+        cfg.update(overrides(args))
+        inp = make_hc_inputs(cfg, dev)
+        metric = "mHC Sinkhorn-mixed tokens/s at 1 B200; achieved HBM GB/s vs peak"
+        config = {"workload": name, "T": cfg["T"], "hc_mult": cfg["n"], "d": cfg["d"], "iters": cfg["iters"],
+                  "eps": cfg["eps"]}
+        rate = lambda b: hc_oracle_rate(inp, b)  # noqa: E731
+    else:
+        from synthetic import FP8_CONFIGS, make_fp8_inputs
+        cfg = dict(FP8_CONFIGS[name], name=name)
+        cfg.update(overrides(args))
+        inp = make_fp8_inputs(cfg, dev)
+        metric = "mxfp8 weight elements/s dequantised to bf16 at 1 B200; achieved HBM GB/s vs peak"
+        config = {"workload": name, "rows": cfg["rows"], "n_in": cfg["n_in"]}
+        rate = lambda b: fp8_oracle_rate(inp, b)  # noqa: E731
+    step_budget = max(0.5, budget_total / max(1, args.steps + args.warmup))
+    vals, t0 = [], time.perf_counter()
+    for s in range(args.warmup + args.steps):
+        cb = rate(step_budget)
+        if s >= args.warmup:
+            vals.append(cb["value"])
+        if time.perf_counter() - t0 > budget_total:
+            break
+    value = statistics.mean(vals) if vals else cb["value"]
+    unit = cb["unit"]
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus,
+            "steps": len(vals), "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+            "cpu_baseline": dict(cb, value=value,
+                                 sample=f"per step: {cb['sample']}; steps capped at {budget_total:.0f}s of CPU work"),
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
 
 
 def reference_line(args, inp, budget_total):
@@ -593,25 +635,130 @@ def run_hc_config(name, args, dev, world, rank):
                     "ms_per_step": e2e_ms},
             "gpu_launches": args.steps, "clocks": clocks}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import numpy as np
-        import oracle
-        sample = min(T, 256)
-        L = inp.logits[:sample].cpu().double().numpy()
-        h = inp.h[:sample].cpu().double().numpy()
-        t0 = time.perf_counter()
-        reps = 0
-        while True:
-            oracle.hc_mix(oracle.hc_sinkhorn(L, cfg["iters"], cfg["eps"]), h)
-            reps += 1
-            if time.perf_counter() - t0 > min(args.cpu_budget, 10.0):
-                break
-        per_tok = (time.perf_counter() - t0) / (reps * sample)
-        line["cpu_baseline"] = {"value": 1.0 / per_tok, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                                "sample": f"{reps} x {sample} tokens of the same workload (numpy fp64)",
-                                "cores_available": len(os.sched_getaffinity(0))}
+        line["cpu_baseline"] = hc_oracle_rate(inp, min(args.cpu_budget, 10.0))
     del inp, flush
     torch.cuda.empty_cache()
     return line
+
+
+def run_fp8_config(name, args, dev, world, rank):
+    """Time the mxfp8 -> bf16 row dequantisation on its own (one launch per
+    step); HBM-bound: 1 + 1/32 bytes read and 2 written per element."""
+    import torch
+
+    import bit_quantized_moe_route_b200 as moe
+    from synthetic import FP8_CONFIGS, make_fp8_inputs
+
+    cfg = dict(FP8_CONFIGS[name], name=name)
+    cfg.update(overrides(args))
+    inp = make_fp8_inputs(cfg, dev)
+    rows, n_in = cfg["rows"], cfg["n_in"]
+    out = torch.empty(rows, n_in, dtype=torch.bfloat16, device=dev)
+    flush = torch.ones(128 * 1024 * 1024, dtype=torch.int32, device=dev)
+    flush_sum = torch.empty((), dtype=torch.int64, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        moe.dequant_mxfp8(inp.codes, inp.scales, out)
+
+    for _ in range(max(3, args.warmup)):
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler("GPU-" + str(props.uuid) if getattr(props, "uuid", None) else str(dev.index))
+    sampler.start()
+    time.sleep(0.2)
+    for s in range(args.steps):
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
+        evs[s][0].record(stream)
+        step()
+        evs[s][1].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    st = step_stats([a.elapsed_time(b) for a, b in evs])
+    ms = max_over_ranks(st["median"], dev)
+    # e2e: host codes and scales in, bf16 rows back
+    c_h, s_h = inp.codes.cpu().pin_memory(), inp.scales.cpu().pin_memory()
+    o_h = torch.empty(rows, n_in, dtype=torch.bfloat16).pin_memory()
+    c_d, s_d = torch.empty_like(inp.codes), torch.empty_like(inp.scales)
+    e2e = []
+    for s in range(max(10, min(args.steps, 30))):
+        torch.sum(flush, dim=0, dtype=torch.int64, out=flush_sum)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        c_d.copy_(c_h, non_blocking=True)
+        s_d.copy_(s_h, non_blocking=True)
+        moe.dequant_mxfp8(c_d, s_d, out)
+        o_h.copy_(out, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e.append(a.elapsed_time(b))
+    e2e_ms = max_over_ranks(statistics.median(e2e), dev)
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    n = rows * n_in
+    nbytes = n + n // 32 + 2 * n
+    roof = {"bound": "hbm", "kernel": "dequant_mxfp8", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": hbm,
+            "unit": "GB/s", "frac": nbytes / (ms * 1e-3) / 1e9 / hbm, "traffic": None,
+            "peak_kind": f"{peak_kind} hbm_gbs (copy)", "algorithmic_bytes_per_launch": nbytes,
+            "frac_of_nominal": nbytes / (ms * 1e-3) / 1e9 / NOMINAL_HBM_GBS}
+    line = {"metric": "mxfp8 weight elements/s dequantised to bf16 at 1 B200; achieved HBM GB/s vs peak",
+            "value": world * n / (ms * 1e-3), "unit": "elements/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "e4m3->bf16", "data": "synthetic",
+            "config": {"workload": name, "rows": rows, "n_in": n_in, "e8m0_range": [cfg["e_lo"], cfg["e_hi"]],
+                       "l2": "flushed by reading a 512 MiB buffer between timed steps (outside the events)"},
+            "step_ms": st, "roofline": roof,
+            "e2e": {"value": world * n / (e2e_ms * 1e-3), "unit": "elements/s",
+                    "h2d_bytes_per_step": n + n // 32, "d2h_bytes_per_step": 2 * n, "ms_per_step": e2e_ms},
+            "gpu_launches": args.steps, "clocks": clocks}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = fp8_oracle_rate(inp, min(args.cpu_budget, 10.0))
+    del inp, flush, out
+    torch.cuda.empty_cache()
+    return line
+
+
+def fp8_oracle_rate(inp, budget):
+    """The oracle's mxfp8 decode on a bounded sample of rows (elements/s)."""
+    import numpy as np
+    import oracle
+    sample = min(inp.cfg["rows"], 64)
+    codes = np.ascontiguousarray(inp.codes[:sample].cpu().numpy())
+    words = codes.view(np.uint32)
+    scales = inp.scales[:sample].cpu().numpy()
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.dequant_mxfp8(words, scales, inp.cfg["n_in"])
+        reps += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    rate = reps * sample * inp.cfg["n_in"] / (time.perf_counter() - t0)
+    return {"value": rate, "unit": "elements/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} x {sample} rows of the same workload (numpy fp64)",
+            "cores_available": len(os.sched_getaffinity(0))}
+
+
+def hc_oracle_rate(inp, budget):
+    """The oracle's Sinkhorn mixing on a bounded sample of tokens (tokens/s)."""
+    import oracle
+    cfg = inp.cfg
+    sample = min(cfg["T"], 256)
+    L = inp.logits[:sample].cpu().double().numpy()
+    h = inp.h[:sample].cpu().double().numpy()
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.hc_mix(oracle.hc_sinkhorn(L, cfg["iters"], cfg["eps"]), h)
+        reps += 1
+        if time.perf_counter() - t0 > budget:
+            break
+    per_tok = (time.perf_counter() - t0) / (reps * sample)
+    return {"value": 1.0 / per_tok, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} x {sample} tokens of the same workload (numpy fp64)",
+            "cores_available": len(os.sched_getaffinity(0))}
 
 
 def ours_arm(args):
@@ -632,7 +779,8 @@ def ours_arm(args):
     moe.set_ffn_path({"auto": moe.FFN_AUTO, "gemv": moe.FFN_GEMV, "tc": moe.FFN_TENSOR_CORE}[args.ffn_path])
     names = CONFIG_ORDER if args.config == "all" else [args.config]
     for name in names:
-        line = (run_hc_config if name.startswith("mhc") else run_config)(name, args, dev, world, rank)
+        run = run_hc_config if name.startswith("mhc") else run_fp8_config if name.startswith("mxfp8") else run_config
+        line = run(name, args, dev, world, rank)
         if rank == 0:
             print(json.dumps(line), flush=True)
     if world > 1:

@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     QMatC,
     alloc_workspace,
     combine,
+    dequant_mxfp8,
     expert_ffn,
     expert_ffn_noalloc,
     forward,

@@ -59,6 +59,7 @@ _SIGS = {
                                            _VP, _VP, _VP, _VP, ctypes.POINTER(QMatC), ctypes.POINTER(QMatC),
                                            ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP, _VP, _VP, _VP,
                                            ctypes.c_size_t, _VP]),
+    "moe_dequant_mxfp8": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, ctypes.c_int32, _VP, _VP]),
     "moe_forward_host": (ctypes.c_int, [ctypes.POINTER(Dims), _VP, _VP, _VP, _VP, _VP, ctypes.POINTER(QMatC),
                                         ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), ctypes.POINTER(QMatC), _VP,
                                         _VP, ctypes.c_size_t, _VP]),
@@ -208,6 +209,17 @@ def forward_partial(dims, expert_begin, expert_end, include_shared, x, token_ids
         _ptr(router_w), _ptr(router_b), _ptr(tid2eid), ctypes.byref(q1), ctypes.byref(q3), ctypes.byref(q2), sh,
         _ptr(out_partial), _ptr(topk_ids_out), _ptr(topk_w_out), _ptr(ws), ws.numel(), _stream(stream)),
         "moe_forward_partial")
+
+
+def dequant_mxfp8(codes: torch.Tensor, scales: torch.Tensor, out: torch.Tensor, stream=None):
+    """moe_dequant_mxfp8: codes uint8 [rows, n_in], scales uint8 [rows, n_in/32], out bf16 [rows, n_in]."""
+    if codes.dtype != torch.uint8 or scales.dtype != torch.uint8 or out.dtype != torch.bfloat16:
+        raise ValueError("codes and scales must be uint8, out bfloat16")
+    rows, n_in = codes.shape
+    if tuple(scales.shape) != (rows, n_in // 32) or tuple(out.shape) != (rows, n_in):
+        raise ValueError("shape mismatch")
+    _check(load_library().moe_dequant_mxfp8(_ptr(codes), _ptr(scales), rows, n_in, _ptr(out), _stream(stream)),
+           "moe_dequant_mxfp8")
 
 
 def forward_host(dims, x_host: torch.Tensor, token_ids_host, router_w, router_b, tid2eid, w1, w3, w2, shared,

@@ -18,6 +18,7 @@
 #include "route.cuh"
 #include "tc_prep.cuh"
 #include "ffn_umma.cuh"
+#include "dequant_fp8.cuh"
 #include "hc_mix.cuh"
 #include "ffn_decode.cuh"
 
@@ -1500,4 +1501,28 @@ extern "C" int32_t moe_test_stall_fused_wait(int32_t enable) {
   const int prev = g_stall_test;
   g_stall_test = enable ? 1 : 0;
   return prev;
+}
+
+extern "C" moe_status_t moe_dequant_mxfp8(const void* codes, const uint8_t* scales, int64_t rows, int32_t n_in,
+                                          void* out, void* stream) {
+  g_detail[0] = 0;
+  if (rows < 0) return fail(MOE_ERR_INVALID_ARG, "rows=%lld must be >= 0", (long long)rows);
+  if (n_in < 32 || n_in % 32) return fail(MOE_ERR_INVALID_ARG, "n_in=%d must be a positive multiple of 32", n_in);
+  if (rows == 0) return MOE_OK;
+  moe_status_t st;
+  if ((st = check_dev_ptr(codes, "codes")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(scales, "scales")) != MOE_OK) return st;
+  if ((st = check_dev_ptr(out, "out")) != MOE_OK) return st;
+  if (!aligned16(codes) || !aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "codes and out must be 16-byte aligned");
+  DevInfo* di;
+  if ((st = dev_info(&di)) != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long work = rows * (long long)(n_in / 8);
+  const int grid = (int)std::max<long long>(
+      1, std::min<long long>((work + (long long)kFp8Threads * kFp8Unroll - 1) / ((long long)kFp8Threads * kFp8Unroll),
+                             (long long)di->sms * 8));
+  dequant_mxfp8_kernel<<<grid, kFp8Threads, 0, s>>>(reinterpret_cast<const uint8_t*>(codes), scales,
+                                                    reinterpret_cast<__nv_bfloat16*>(out), (long long)rows, n_in);
+  MOE_CHECK_LAUNCH("dequant_mxfp8_kernel");
+  return MOE_OK;
 }

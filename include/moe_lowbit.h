@@ -303,6 +303,24 @@ moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const 
                               void* stream);
 
 /*
+ * mxfp8 weight rows to bf16 [PR1192 FP8 re-quantisation thread: fp8 e4m3
+ * weight bytes, one e8m0 scale byte per 32 consecutive elements of a row]:
+ *   out[r, i] = bf16( e4m3(codes[r, i]) * 2^(scales[r, i/32] - 127) )
+ *   codes : bytes [rows, n_in] (byte i of a row is element i), 16-byte aligned
+ *   scales: bytes [rows, n_in/32];  out : bf16 [rows, n_in], 16-byte aligned
+ * Exact (each value has 4 significant bits times a power of two) while the
+ * product lies within bf16's range: every normal e4m3 code for any scale
+ * byte from 1 to 254 whose result is finite, subnormal codes for scale
+ * bytes >= 5.  Scale byte 255 (the format's NaN) gives +-inf.  n_in a
+ * positive multiple of 32, rows >= 0 (0: nothing to do); otherwise
+ * MOE_ERR_INVALID_ARG.  One launch, no workspace; the 128x128 block scales of
+ * FP8 checkpoints map to these per-32-group bytes on the host (each row's
+ * group g takes block (row / 128, g / 4)).
+ */
+moe_status_t moe_dequant_mxfp8(const void* codes, const uint8_t* scales, int64_t rows, int32_t n_in, void* out,
+                               void* stream);
+
+/*
  * mHC residual mixing, fused (the block next to the MoE layer in each
  * DeepSeek-V4 layer) [CARD-4BIT Architecture "mHC": hc_mult parallel copies
  * of the hidden state recombined by a doubly-stochastic, Sinkhorn-normalised

@@ -8,6 +8,9 @@ consume what it produces.
 """
 from .moe_inputs import (  # noqa: F401
     CONFIGS,
+    FP8_CONFIGS,
+    Fp8Inputs,
+    make_fp8_inputs,
     HC_CONFIGS,
     HcInputs,
     make_hc_inputs,

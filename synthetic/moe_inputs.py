@@ -282,3 +282,35 @@ def make_hc_inputs(cfg: dict, device="cpu") -> HcInputs:
     logits = torch.randn(T, n, n, generator=gen, device=device) * cfg.get("logit_std", 1.0)
     h = torch.randn(T, n, d, generator=gen, device=device).to(torch.bfloat16)
     return HcInputs(dict(cfg), logits.contiguous(), h.contiguous())
+
+
+# --------------------------------------------------------------------------
+# mxfp8 weight rows (e4m3 bytes with e8m0 group-32 scales)
+# --------------------------------------------------------------------------
+FP8_CONFIGS: Dict[str, dict] = {
+    # a 16384 x 4096 weight matrix (64 Mi elements: 64 MiB of codes, 128 MiB
+    # of bf16 out, more than L2) with e8m0 exponents uniform in [117, 123]
+    # like the mxfp4 experts
+    "mxfp8": dict(rows=16384, n_in=4096, e_lo=117, e_hi=123, seed=7),
+}
+
+
+@dataclasses.dataclass
+class Fp8Inputs:
+    cfg: dict
+    codes: torch.Tensor    # uint8 [rows, n_in]
+    scales: torch.Tensor   # uint8 [rows, n_in / 32]
+
+
+def make_fp8_inputs(cfg: dict, device="cpu") -> Fp8Inputs:
+    """e4m3 bytes uniform over the finite codes (the two NaN bytes 0x7F and
+    0xFF become 0x38 = 1.0) and e8m0 bytes uniform in [e_lo, e_hi], drawn in
+    that order from one generator seeded with cfg["seed"]."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(cfg["seed"]))
+    rows, n_in = cfg["rows"], cfg["n_in"]
+    codes = torch.randint(0, 256, (rows, n_in), generator=gen, device=device, dtype=torch.int32)
+    codes = torch.where((codes & 0x7F) == 0x7F, torch.full_like(codes, 0x38), codes).to(torch.uint8)
+    scales = torch.randint(cfg["e_lo"], cfg["e_hi"] + 1, (rows, n_in // 32), generator=gen, device=device,
+                           dtype=torch.int32).to(torch.uint8)
+    return Fp8Inputs(dict(cfg), codes.contiguous(), scales.contiguous())

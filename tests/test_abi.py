@@ -78,6 +78,10 @@ def test_host_validation_without_gpu(lib):
     assert b"expert range" in lib.moe_last_error_detail()
     assert lib.moe_forward_partial(ctypes.byref(d), 0, 8, 2, *([None] * 13), 0, None) == 1
     assert b"include_shared" in lib.moe_last_error_detail()
+    # mxfp8 rows: n_in not a multiple of 32, negative rows
+    assert lib.moe_dequant_mxfp8(None, None, 4, 48, None, None) == 1
+    assert lib.moe_dequant_mxfp8(None, None, -1, 64, None, None) == 1
+    assert lib.moe_dequant_mxfp8(None, None, 0, 64, None, None) == 0
     # bad dims
     bad = _lib.make_dims(4, 256, 128, 8, 0)
     assert lib.moe_permute(ctypes.byref(bad), None, None, None, None, None, 0, None) == 1
