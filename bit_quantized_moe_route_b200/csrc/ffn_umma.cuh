@@ -19,15 +19,17 @@
 //     blocks per 128-input stage, with the 128-byte swizzle the tensor core
 //     reads directly, in boxes of 16 / 64 / 128 / 192 rows as the tile needs
 //     (3-stage ring);
-//   * 8 dequant warps in two groups (even / odd stages) turn each 128-input
-//     stage of codes into fp16 weights and write them straight into tensor
-//     memory (tcgen05.st): the weights are the MMA's A operand in TMEM (two
-//     stage slots of 64 columns, one per group), so the shared memory only
-//     carries the token tiles and the packed codes;
+//   * kUmGroups groups of 4 dequant warps (stage g goes to group g mod
+//     kUmGroups) turn each 128-input stage of codes into fp16 weights and
+//     write them straight into tensor memory (tcgen05.st): the weights are
+//     the MMA's A operand in TMEM, in a ring of kUmNA stage slots of 64
+//     columns, so a group dequantises ahead while the MMAs of earlier stages
+//     run, and the shared memory only carries the token tiles and the packed
+//     codes;
 //   * the packed-code and token-tile TMA loads are issued by two separate
 //     threads, so neither ring waits on the other;
 //   * one thread issues 8 tcgen05.mma per stage (A from TMEM, B from shared
-//     memory, fp32 accumulators in TMEM, double-buffered: 2 x 192 columns);
+//     memory, fp32 accumulators in TMEM: kUmNAcc buffers of 192 columns);
 //     stages are 128 inputs deep because every barrier wait, fence and
 //     commit on the issuing thread delays the next MMA;
 //   * 4 epilogue warps read the accumulators (tcgen05.ld) and write H
@@ -50,18 +52,34 @@ namespace moe {
 constexpr int kUmN = 192;        // tokens per tile (MMA N <= 192, multiple of 16)
 constexpr int kUmK = 128;        // inputs per MMA stage (8 MMAs of K = 16)
 constexpr int kUmKB = 64;        // inputs per 128-byte swizzle atom of a token row
-constexpr int kUmThreads = 16 * 32;
-constexpr int kUmMmaWarp = 8;
-constexpr int kUmRawWarp = 9;    // TMA issuer of packed codes / scales / biases
-constexpr int kUmBWarp = 10;     // TMA issuer of token tiles
-constexpr int kUmEpiWarp0 = 12;  // warps 12-15: warp % 4 = TMEM lane quarter
+#ifndef MOE_UM_GROUPS
+#define MOE_UM_GROUPS 2
+#endif
+#ifndef MOE_UM_NA
+#define MOE_UM_NA 2
+#endif
+#ifndef MOE_UM_NACC
+#define MOE_UM_NACC 2
+#endif
+constexpr int kUmGroups = MOE_UM_GROUPS;        // dequant groups of 4 warps
+constexpr int kUmNA = MOE_UM_NA;                // A stage slots in TMEM
+constexpr int kUmNAcc = MOE_UM_NACC;            // accumulator buffers in TMEM
+constexpr int kUmDqWarps = 4 * kUmGroups;
+constexpr int kUmMmaWarp = kUmDqWarps;
+constexpr int kUmRawWarp = kUmDqWarps + 1;      // TMA issuer of packed codes / scales / biases
+constexpr int kUmBWarp = kUmDqWarps + 2;        // TMA issuer of token tiles
+constexpr int kUmEpiWarp0 = kUmDqWarps + 4;     // 4 epilogue warps: warp % 4 = TMEM lane quarter
+constexpr int kUmThreads = (kUmEpiWarp0 + 4) * 32;
 constexpr int kUmBStages = 3;
 constexpr int kUmBBlock = kUmN * 128;       // one 64-input column block of a token tile
 constexpr int kUmBTile = 2 * kUmBBlock;     // 192 rows x 128 inputs fp16 = 48 KB
 constexpr uint32_t kUmASlotCols = kUmK / 2; // 64 TMEM columns per A stage slot
-constexpr uint32_t kUmAccCol0 = 2 * kUmASlotCols;  // accumulators at 128 and 320
+constexpr uint32_t kUmAccCol0 = kUmNA * kUmASlotCols;  // A slots first, then the accumulators
 constexpr uint32_t kUmAccCols = kUmN;
 constexpr uint32_t kUmTmemCols = 512;
+static_assert(kUmEpiWarp0 % 4 == 0, "epilogue warps must cover the four TMEM lane quarters in order");
+static_assert(kUmAccCol0 + kUmNAcc * kUmAccCols <= kUmTmemCols, "TMEM columns");
+static_assert(kUmNA >= kUmGroups, "every dequant group needs a stage slot");
 
 struct alignas(64) UmParams {
   CUtensorMap b_map[4];  // B rows: fp16 [rows, n_in], boxes {64, 16 / 64 / 128 / 192 rows}, 128B swizzle
@@ -103,7 +121,10 @@ struct UmCfg {
   static constexpr int GBOX = mx ? 16 : 8;              // groups per 16-byte scale box
   static constexpr int ESZ = mx ? 1 : 2;                // scale element bytes
   static constexpr int NRS = 3;                         // raw slots
-  static constexpr int RAW_USERS = QS == 1 ? 4 : 8;     // dequant warps reading one raw slot
+  // dequant warps reading one raw slot: its QS consecutive stages belong to
+  // min(QS, groups) groups (the host admits only whole raw slots per row
+  // when the groups do not all read every slot)
+  static constexpr int RAW_USERS = 4 * (QS < kUmGroups ? QS : kUmGroups);
   static constexpr size_t smem = 1024 + NRS * (size_t)slot_bytes + (size_t)kUmBStages * kUmBTile + 256;
   static_assert(slot_bytes % 1024 == 0, "raw slots keep the 1024-byte alignment of the swizzled boxes");
   static_assert(smem <= 227 * 1024, "TMA/TMEM FFN exceeds the per-block shared memory limit");
@@ -208,14 +229,16 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
   auto raw_empty = [&](int s) { return bar + 8u * (NRS + s); };             // [NRS] dequant warps
   auto b_full = [&](int s) { return bar + 8u * (2 * NRS + s); };            // [NB] TMA bytes
   auto b_empty = [&](int s) { return bar + 8u * (2 * NRS + NB + s); };      // [NB] MMA commit
-  auto a_full = [&](int s) { return bar + 8u * (2 * NRS + 2 * NB + s); };   // [2] 4 dequant warps
-  auto a_empty = [&](int s) { return bar + 8u * (2 * NRS + 2 * NB + 2 + s); };    // [2] MMA commit
-  auto acc_full = [&](int s) { return bar + 8u * (2 * NRS + 2 * NB + 4 + s); };   // [2] MMA commit
-  auto acc_empty = [&](int s) { return bar + 8u * (2 * NRS + 2 * NB + 6 + s); };  // [2] 4 epilogue warps
-  const uint32_t drain = bar + 8u * (2 * NRS + 2 * NB + 8);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_gen + 8 * (2 * NRS + 2 * NB + 9));
+  constexpr int NA = kUmNA, NAC = kUmNAcc, NG = kUmGroups;
+  constexpr int BA = 2 * NRS + 2 * NB;  // first A / accumulator barrier
+  auto a_full = [&](int s) { return bar + 8u * (BA + s); };                         // [NA] 4 dequant warps
+  auto a_empty = [&](int s) { return bar + 8u * (BA + NA + s); };                   // [NA] MMA commit
+  auto acc_full = [&](int s) { return bar + 8u * (BA + 2 * NA + s); };              // [NAC] MMA commit
+  auto acc_empty = [&](int s) { return bar + 8u * (BA + 2 * NA + NAC + s); };       // [NAC] 4 epilogue warps
+  const uint32_t drain = bar + 8u * (BA + 2 * NA + 2 * NAC);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_gen + 8 * (BA + 2 * NA + 2 * NAC + 1));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  static_assert(8 * (2 * NRS + 2 * NB + 9) + 8 <= 256, "barrier block");
+  static_assert(8 * (BA + 2 * NA + 2 * NAC + 1) + 8 <= 256, "barrier block");
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_mt = p.n_out / (STAGE == 1 ? 64 : 128);
@@ -236,9 +259,11 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
       tc_bar_init(b_full(s), 1);
       tc_bar_init(b_empty(s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NA; ++s) {
       tc_bar_init(a_full(s), 4);
       tc_bar_init(a_empty(s), 1);
+    }
+    for (int s = 0; s < NAC; ++s) {
       tc_bar_init(acc_full(s), 1);
       tc_bar_init(acc_empty(s), 4);
     }
@@ -257,19 +282,20 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 8) {
-    // ================= dequant warps: group G takes the stages g = G mod 2
-    // into A slot G; warp quarter q owns TMEM lanes 32q..32q+31 (= A rows)
+  if (warp < kUmDqWarps) {
+    // ================= dequant warps: group G takes the stages g = G mod NG
+    // into A slot g mod NA; warp quarter q owns TMEM lanes 32q..32q+31 (= A rows)
     const int G = warp >> 2, q = warp & 3;
     const int m = STAGE == 1 ? (lane >> 4) : 0;                        // matrix of this lane's row
     const int rr = STAGE == 1 ? 16 * q + (lane & 15) : 32 * q + lane;  // row within that matrix's box
     UmCursor cur;
     cur.init(p, n_items, n_mt);
-    if (G == 1 && total > 1) cur.advance(p, n_items, n_mt, n_kt);
+    for (int i = 0; i < G && i < total; ++i) cur.advance(p, n_items, n_mt, n_kt);
     int held = -1;  // raw slot sequence number whose data this group is reading
     bool bad = false;
-    const uint32_t tcol = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)G * kUmASlotCols;
-    for (int g = G; g < total; g += 2) {
+    for (int g = G; g < total; g += NG) {
+      const int as = g % NA;
+      const uint32_t tcol = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)as * kUmASlotCols;
       const int kt = cur.sub, qs = kt % QS, ri = kt / QS;
       const int seq = cur.k * n_rng + ri;
       const int rs = seq % NRS;
@@ -278,7 +304,7 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
         ok = tc_bar_wait(raw_full(rs), (uint32_t)(seq / NRS) & 1u, abort_flag);
         held = seq;
       }
-      if (ok && g >= 2) ok = tc_bar_wait(a_empty(G), (uint32_t)((g >> 1) - 1) & 1u, abort_flag);
+      if (ok && g >= NA) ok = tc_bar_wait(a_empty(as), (uint32_t)(g / NA - 1) & 1u, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.st below is warp-collective
       const uint32_t slot = slot0 + (uint32_t)(rs * C::slot_bytes);
       const uint32_t prow = slot + (uint32_t)(m * C::PBOX + rr * C::BOXB);
@@ -332,10 +358,9 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) tc_bar_arrive(a_full(G));
-      cur.advance(p, n_items, n_mt, n_kt);
-      if (g + 1 < total) cur.advance(p, n_items, n_mt, n_kt);
-      const int next_seq = g + 2 < total ? cur.k * n_rng + cur.sub / QS : -1;
+      if (lane == 0) tc_bar_arrive(a_full(as));
+      for (int i = 0; i < NG && g + i < total; ++i) cur.advance(p, n_items, n_mt, n_kt);
+      const int next_seq = g + NG < total ? cur.k * n_rng + cur.sub / QS : -1;
       if (next_seq != seq && lane == 0) tc_bar_arrive(raw_empty(rs));  // this group's last use of the slot
     }
     if (bad) set_error(p.err, kErrDeviceInput);
@@ -404,14 +429,14 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
       int g = 0;
       for (int it = 0; it < my_items && !*abort_flag; ++it) {
         const uint32_t idesc = umma_idesc_f16((cur.tile.z + 15) & ~15);
-        const int ab = it & 1;
-        if (it >= 2 && !tc_bar_wait(acc_empty(ab), (uint32_t)((it >> 1) - 1) & 1u, abort_flag)) break;
+        const int ab = it % NAC;
+        if (it >= NAC && !tc_bar_wait(acc_empty(ab), (uint32_t)(it / NAC - 1) & 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + kUmAccCol0 + (uint32_t)ab * kUmAccCols;
         bool ok = true;
         for (int kt = 0; kt < n_kt; ++kt, ++g) {
-          const int as = g & 1, bs = g % NB;
-          if (!tc_bar_wait(a_full(as), (uint32_t)(g >> 1) & 1u, abort_flag) ||
+          const int as = g % NA, bs = g % NB;
+          if (!tc_bar_wait(a_full(as), (uint32_t)(g / NA) & 1u, abort_flag) ||
               !tc_bar_wait(b_full(bs), (uint32_t)(g / NB) & 1u, abort_flag)) {
             ok = false;
             break;
@@ -445,8 +470,8 @@ __global__ void __launch_bounds__(kUmThreads, 1) ffn_umma_kernel(const __grid_co
     cur.init(p, n_items, n_mt);
     bool bad = false;
     for (int it = 0; it < my_items; ++it) {
-      const int ab = it & 1;
-      const bool ok = tc_bar_wait(acc_full(ab), (uint32_t)(it >> 1) & 1u, abort_flag);
+      const int ab = it % NAC;
+      const bool ok = tc_bar_wait(acc_full(ab), (uint32_t)(it / NAC) & 1u, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld is warp-collective
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(32 * q) << 16) + kUmAccCol0 + (uint32_t)ab * kUmAccCols;

@@ -560,9 +560,12 @@ moe_status_t tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, ui
 // Shapes the TMA/TMEM kernel takes: any packed format, rows of a multiple of
 // 16 bytes, scale rows of a multiple of 16 bytes (the TMA stride rule), 64
 // (stage 1) or 128 (stage 2) output rows per tile, an even number of
-// 128-input stages (the two dequant groups split them).
+// 128-input stages.
 bool um_ok(const QMatDev& Q, int stage) {
   if (Q.n_in % (2 * kUmK) || Q.n_out % (stage == 1 ? 64 : 128)) return false;
+  // more dequant groups than two: every raw slot of a row must be whole
+  // (2-bit slots hold 512 inputs), so that the groups reading it are fixed
+  if (kUmGroups > 2 && Q.n_in % (Q.fmt == F_A2 ? 512 : 256)) return false;
   if ((Q.wpr * 4) % 16) return false;
   if (Q.group != 32 && Q.group != 64 && Q.group != 128) return false;
   return Q.fmt == F_MX4 ? Q.gpr % 16 == 0 : (Q.gpr * 2) % 16 == 0;
