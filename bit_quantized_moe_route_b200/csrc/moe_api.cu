@@ -248,6 +248,7 @@ struct DevInfo {
   int sms = 0;
   int ffn1_blocks = 0, ffn2_blocks = 0;
   int dec_blocks = 0;  // fused decode: co-resident CTAs (one per SM)
+  int um_pairs[10] = {};  // TMA/TMEM FFN: resident CTA pairs per (stage, format) kernel
 };
 DevInfo g_dev[64];
 std::atomic<int> g_dev_ready[64];
@@ -268,7 +269,7 @@ moe_status_t dev_info(DevInfo** out) {
       route_attrs<__nv_bfloat16>();
       for (StreamAttrFn f : kStreamAttrs) f();
       for (TcAttrFn f : kTcAttrs) f();
-      for (UmAttrFn f : kUmAttrs) f();
+      for (int i = 0; i < 10; ++i) di.um_pairs[i] = kUmAttrs[i]();
       int b1 = 0, b2 = 0;
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b1, ffn_gemv_kernel<1, 4>, kFfnThreads, 0);
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b2, ffn_gemv_kernel<2, 8>, kFfnThreads, 0);
@@ -558,11 +559,11 @@ moe_status_t tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, ui
 }
 
 // Shapes the TMA/TMEM kernel takes: any packed format, rows of a multiple of
-// 16 bytes, scale rows of a multiple of 16 bytes (the TMA stride rule), 64
-// (stage 1) or 128 (stage 2) output rows per tile, an even number of
+// 16 bytes, scale rows of a multiple of 16 bytes (the TMA stride rule), 128
+// features (stage 1) or 256 output rows (stage 2) per pair item, an even number of
 // 128-input stages.
 bool um_ok(const QMatDev& Q, int stage) {
-  if (Q.n_in % (2 * kUmK) || Q.n_out % (stage == 1 ? 64 : 128)) return false;
+  if (Q.n_in % (2 * kUmK) || Q.n_out % (stage == 1 ? kUmRowsS1 : kUmRowsS2)) return false;
   // more dequant groups than two: every raw slot of a row must be whole
   // (2-bit slots hold 512 inputs), so that the groups reading it are fixed
   if (kUmGroups > 2 && Q.n_in % (Q.fmt == F_A2 ? 512 : 256)) return false;
@@ -617,11 +618,12 @@ moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offset
   auto run = [&](int stage, const QMatDev& a0, const QMatDev& a1, bool shared, const char* label) -> moe_status_t {
     const int pos_base = shared ? Tk : 0;
     const int E = shared ? 1 : d.n_experts;
-    if (um_ok(a0, stage) && um_ok(a1, stage)) {
+    const int um_pairs = di.um_pairs[(stage - 1) * 5 + a0.fmt];
+    if (um_pairs > 0 && um_ok(a0, stage) && um_ok(a1, stage)) {
       UmParams q{};
       moe_status_t st = MOE_OK;
-      for (int h = 0; h < 4 && st == MOE_OK; ++h) {  // token boxes of 16, 64, 128, 192 rows
-        const uint32_t box_rows = h == 0 ? 16u : 64u * h;
+      for (int h = 0; h < 4 && st == MOE_OK; ++h) {  // half-tile token boxes of 16, 32, 64, 96 rows
+        const uint32_t box_rows = h == 0 ? 16u : h == 1 ? 32u : h == 2 ? 64u : 96u;
         if (stage == 1)
           st = tmap_2d(&q.b_map[h], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs, d.d_model, (uint64_t)P,
                        (uint64_t)d.d_model * 2, kUmKB, box_rows, true);
@@ -648,9 +650,9 @@ moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offset
       q.n_tiles = n_tiles + 1;
       q.pos_base = pos_base;
       q.err = err;
-      const int rows_per_item = stage == 1 ? 64 : 128;
-      const int grid = shared ? std::min(di.sms, (d.T + kUmN - 1) / kUmN * (a0.n_out / rows_per_item)) : di.sms;
-      if (!kUmLaunch[stage - 1][a0.fmt](q, grid, s)) return fail(MOE_ERR_UNSUPPORTED, "no TMA/TMEM kernel");
+      const int rows_per_item = stage == 1 ? kUmRowsS1 : kUmRowsS2;
+      const int pairs = shared ? std::min(um_pairs, (d.T + kUmN - 1) / kUmN * (a0.n_out / rows_per_item)) : um_pairs;
+      if (!kUmLaunch[stage - 1][a0.fmt](q, pairs, s)) return fail(MOE_ERR_UNSUPPORTED, "no TMA/TMEM kernel");
     } else {
       TcParams q{};
       q.x16 = xs;
