@@ -81,8 +81,7 @@ constexpr int kDecMaxGroups = kDecMaxPairs + 8;
 constexpr int kDecFxRed = 0;
 constexpr int kDecFxH = kDecFxRed + kDecRedFloats * 4;           // 2 buffers x 4 tokens x 64 h values
 constexpr int kDecFxScr = kDecFxH + 2 * kDecMaxTok * kDecRows * 4;  // the service warp's scratch (64 ints)
-constexpr int kDecFxLut = kDecFxScr + 256;                      // e8m0 byte -> 2^(e-128) (fp32)
-constexpr int kDecFxIds = kDecFxLut + 1024;
+constexpr int kDecFxIds = kDecFxScr + 256;
 constexpr int kDecFxW = kDecFxIds + kDecMaxPairs * 4;
 constexpr int kDecFxSorted = kDecFxW + kDecMaxPairs * 4;
 constexpr int kDecFxInv = kDecFxSorted + kDecMaxPairs * 4;
@@ -282,7 +281,6 @@ MOE_DEV uint32_t codes3x8(uint32_t line, int off, int t) {
 // rows r8..r8+7; their scales in scale boxes `s0` / `s8` (biases R * spitch
 // bytes further).
 struct DecWarp {
-  uint32_t lut;  // shared address of the e8m0 table
   uint32_t a0, a8, s0, s8;
   int r0, r8;    // tile 0; tile 1 is `tstep` rows further in every box
   int tstep;
@@ -302,7 +300,6 @@ struct DecLane {
   uint32_t b;     // plane-buffer-relative B address (token row, quad thread, plane)
   uint32_t sx;    // record-relative address (token, the slice's first block)
   uint32_t s0, s8, brow;  // slot-relative scale addresses of A rows g / g+8 (the slice's first group), bias offset
-  uint32_t lut;           // shared address of the e8m0 table
   uint32_t ta, ts;        // tile 1: code byte offset (tstep rows), scale byte offset
 };
 
@@ -350,7 +347,6 @@ MOE_DEV DecLane dec_lane(const DecWarp& q, int ntok) {
   L.s0 = q.s0 + (uint32_t)((q.r0 + g) * q.spitch + esz * gbase);
   L.s8 = q.s8 + (uint32_t)((q.r8 + g) * q.spitch + esz * gbase);
   L.brow = (uint32_t)(q.R * q.spitch);
-  L.lut = q.lut;
   L.ta = (uint32_t)(q.tstep * (FMT == F_A3 ? 96 : 128));
   L.ts = (uint32_t)(q.tstep * q.spitch);
   return L;
@@ -361,7 +357,7 @@ MOE_DEV DecLane dec_lane(const DecWarp& q, int ntok) {
 // integer sum of codes x fixed-point inputs, st the inputs' step, sm their
 // dequantised sum; GI: the group's scale entry relative to the slice.
 template <int FMT, int GI>
-MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, uint32_t lut, float st, float sm, const int (&c)[4],
+MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, float st, float sm, const int (&c)[4],
                       float (&acc)[2]) {
   float sc0, b0, sc8, b8;
   if constexpr (FMT == F_MX4) {
@@ -369,7 +365,6 @@ MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, uint32_t lut, flo
     const uint32_t e0 = lds8u(s0 + GI), e8 = lds8u(s8 + GI);
     sc0 = __uint_as_float(e0 > 1 ? ((e0 - 1) << 23) : (e0 ? 0x00400000u : 0x00200000u));
     sc8 = __uint_as_float(e8 > 1 ? ((e8 - 1) << 23) : (e8 ? 0x00400000u : 0x00200000u));
-    (void)lut;
     b0 = b8 = 0.f;
   } else {
     sc0 = bf16_bits_to_float(lds16u(s0 + 2 * GI));
@@ -444,8 +439,8 @@ MOE_DEV void dec_block(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, 
       d1[i] = c1[i] - cn1[i];
       c0[i] = cn0[i] = c1[i] = cn1[i] = 0;
     }
-    dec_fold<FMT, 2 * B>(s0, s8, L.brow, L.lut, rec.x, rec.y, d0, a0);
-    dec_fold<FMT, 2 * B>(s0 + L.ts, s8 + L.ts, L.brow, L.lut, rec.x, rec.y, d1, a1);
+    dec_fold<FMT, 2 * B>(s0, s8, L.brow, rec.x, rec.y, d0, a0);
+    dec_fold<FMT, 2 * B>(s0 + L.ts, s8 + L.ts, L.brow, rec.x, rec.y, d1, a1);
   }
   {
     const uint2 bv = lds64u(bp + B * 128 + 64);
@@ -459,11 +454,11 @@ MOE_DEV void dec_block(const DecLane& L, uint32_t la, uint32_t sl, uint32_t bp, 
     d1[i] = c1[i] - cn1[i];
   }
   if constexpr (G == 32) {
-    dec_fold<FMT, 2 * B + 1>(s0, s8, L.brow, L.lut, rec.x, rec.z, d0, a0);
-    dec_fold<FMT, 2 * B + 1>(s0 + L.ts, s8 + L.ts, L.brow, L.lut, rec.x, rec.z, d1, a1);
+    dec_fold<FMT, 2 * B + 1>(s0, s8, L.brow, rec.x, rec.z, d0, a0);
+    dec_fold<FMT, 2 * B + 1>(s0 + L.ts, s8 + L.ts, L.brow, rec.x, rec.z, d1, a1);
   } else {
-    dec_fold<FMT, (B * 64) / G>(s0, s8, L.brow, L.lut, rec.x, rec.w, d0, a0);
-    dec_fold<FMT, (B * 64) / G>(s0 + L.ts, s8 + L.ts, L.brow, L.lut, rec.x, rec.w, d1, a1);
+    dec_fold<FMT, (B * 64) / G>(s0, s8, L.brow, rec.x, rec.w, d0, a0);
+    dec_fold<FMT, (B * 64) / G>(s0 + L.ts, s8 + L.ts, L.brow, rec.x, rec.w, d1, a1);
   }
   acc[0] = a0[0];
   acc[1] = a0[1];
@@ -758,11 +753,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mp)) : "memory");
   }
   for (int e = tid; e < E; e += kDecThreads) r_off[e] = 0;  // per-expert counts (P1)
-  if (tid < 256) {  // e8m0 byte -> 2^(e-128): exact for every byte (subnormal for 0 and 1)
-    const uint32_t e = tid;
-    reinterpret_cast<float*>(fx + kDecFxLut)[tid] =
-        __uint_as_float(e > 1 ? ((e - 1) << 23) : (e ? 0x00400000u : 0x00200000u));
-  }
   __syncthreads();
 
   // ------------------------------------------------------------ P0
@@ -1208,7 +1198,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
       const bool s1 = U.stage == 1;
       DecWarp q;
       const int nsb = m0.fmt == F_MX4 ? 1 : 2;
-      q.lut = su32(fx + kDecFxLut);
       q.R = m0.R;
       q.kq = kq;
       q.spitch = m0.spitch;
