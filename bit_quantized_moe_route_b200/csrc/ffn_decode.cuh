@@ -153,20 +153,24 @@ struct DecParams {
 };
 
 // ------------------------------------------------------------ grid barrier
-// Generation barrier over the whole (co-resident) grid; bounded wait.
+// Generation barrier over the whole (co-resident) grid; bounded wait.  The
+// arrive is one acquire-release atomic (its release covers the CTA's writes,
+// ordered before it by bar.sync); the last arriver resets the count and
+// publishes the next generation with a release, which the others acquire.
 MOE_DEV void dec_grid_barrier(int* sync, int nblocks, int* err, volatile int* abort_flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    volatile int* gen = sync + 1;
-    const int my_gen = *gen;
-    __threadfence();
-    if (atomicAdd(sync, 1) == nblocks - 1) {
-      sync[0] = 0;
-      __threadfence();
-      atomicAdd(sync + 1, 1);
+    int* gen = sync + 1;
+    int my_gen;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(my_gen) : "l"(gen) : "memory");
+    int t;
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(t) : "l"(sync) : "memory");
+    if (t == nblocks - 1) {
+      asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(sync), "r"(0) : "memory");
+      red_release_add(gen, 1);
     } else {
       const long long t0 = clock64();
-      while (*gen == my_gen) {
+      while (ld_acquire(gen) == my_gen) {
         if (clock64() - t0 > kDecWaitCycles) {
           set_error(err, kErrTimeout);
           *abort_flag = 1;
@@ -174,7 +178,6 @@ MOE_DEV void dec_grid_barrier(int* sync, int nblocks, int* err, volatile int* ab
         }
       }
     }
-    __threadfence();
   }
   __syncthreads();
 }
