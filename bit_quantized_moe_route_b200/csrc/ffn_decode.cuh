@@ -948,40 +948,42 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
   }
   __syncthreads();
   if (warp == 0) {
-    // offsets (exclusive scan), cursors and groups: lane l owns experts
-    // [l*per, (l+1)*per); groups in ascending expert order after the shared ones
+    // offsets (exclusive scan), cursors and groups, in rounds of 32 experts
+    // (lane l takes expert 32r + l: conflict-free shared accesses) with the
+    // running totals carried between rounds; groups in ascending expert
+    // order after the shared ones
     const int gsz = p.ntmax;
     const int nsg = p.has_shared && p.with_shared ? (T + gsz - 1) / gsz : 0;
-    const int per = (E + 31) / 32;
-    const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-    int s = 0, ng = 0;
-    for (int e = e0; e < e1; ++e) {
-      const int c = r_off[e];
-      s += c;
-      if (e >= p.e_begin && e < p.e_end) ng += (c + gsz - 1) / gsz;
-    }
-    int sx = s, gx = ng;  // inclusive warp scans
+    int run = 0, gbase = nsg;  // pairs and groups before this round
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = e < E ? r_off[e] : 0;
+      const bool own = e < E && e >= p.e_begin && e < p.e_end;
+      // ceil(c / gsz) for gsz in 1..4 without a runtime division
+      const int ng = !own ? 0 : gsz == 1 ? c : gsz == 2 ? (c + 1) >> 1 : gsz == 3 ? (c + 2) / 3 : (c + 3) >> 2;
+      int sc = c, sg = ng;  // inclusive warp scans
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int a = __shfl_up_sync(0xffffffffu, sx, o), b = __shfl_up_sync(0xffffffffu, gx, o);
-      if (lane >= o) {
-        sx += a;
-        gx += b;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int a = __shfl_up_sync(0xffffffffu, sc, o), b = __shfl_up_sync(0xffffffffu, sg, o);
+        if (lane >= o) {
+          sc += a;
+          sg += b;
+        }
       }
+      const int off = run + sc - c;
+      if (e < E) {
+        r_off[e] = off;
+        r_cur[e] = off;
+      }
+      if (own)
+        for (int q0 = 0, gi = gbase + sg - ng; q0 < c; q0 += gsz) r_groups[gi++] = make_int4(e, off + q0, min(gsz, c - q0), 0);
+      run += __shfl_sync(0xffffffffu, sc, 31);
+      gbase += __shfl_sync(0xffffffffu, sg, 31);
     }
-    int run = sx - s, gi = nsg + gx - ng;
-    for (int e = e0; e < e1; ++e) {
-      const int c = r_off[e];
-      r_off[e] = run;
-      r_cur[e] = run;
-      if (e >= p.e_begin && e < p.e_end)
-        for (int q0 = 0; q0 < c; q0 += gsz) r_groups[gi++] = make_int4(e, run + q0, min(gsz, c - q0), 0);
-      run += c;
-    }
-    if (lane == 31) {
+    if (lane == 0) {
       r_off[E] = run;
       misc[1] = nsg;
-      misc[2] = gx;
+      misc[2] = gbase - nsg;
     }
     if (lane < nsg) r_groups[lane] = make_int4(-1, lane * gsz, min(gsz, T - lane * gsz), 0);
     __syncwarp();
