@@ -182,6 +182,49 @@ MOE_DEV void dec_grid_barrier(int* sync, int nblocks, int* err, volatile int* ab
   __syncthreads();
 }
 
+// 8 router weights of expert e at inputs i..i+7 as floats (fp32 or bf16 rows)
+MOE_DEV void dec_router8(const DecParams& p, int e, int i, float (&w)[8]) {
+  if (p.router_bf16) {
+    const uint4 r =
+        __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.router_w) + (size_t)e * p.d + i));
+    w[0] = bf16lo(r.x); w[1] = bf16hi(r.x); w[2] = bf16lo(r.y); w[3] = bf16hi(r.y);
+    w[4] = bf16lo(r.z); w[5] = bf16hi(r.z); w[6] = bf16lo(r.w); w[7] = bf16hi(r.w);
+  } else {
+    const float4* rr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.router_w) + (size_t)e * p.d + i);
+    const float4 a = __ldg(rr), b = __ldg(rr + 1);
+    w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
+}
+
+// Sums each of 16 per-lane values over the warp with 16 shuffles: halves of
+// the values are exchanged with lane ^ 16, ^ 8, ^ 4, ^ 2, then ^ 1.  Value
+// 8*b4 + 4*b3 + 2*b2 + b1 (b: bits of the lane id) ends in the lane pair
+// (2m, 2m+1) holding those bits; the order of additions is fixed.
+MOE_DEV float dec_transpose_sum16(const float (&a)[16]) {
+  const int lane = threadIdx.x & 31;
+  float b[8], c[4], d2[2];
+  const bool h4 = lane & 16, h3 = lane & 8, h2 = lane & 4, h1 = lane & 2;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float send = h4 ? a[j] : a[8 + j], keep = h4 ? a[8 + j] : a[j];
+    b[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float send = h3 ? b[j] : b[4 + j], keep = h3 ? b[4 + j] : b[j];
+    c[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float send = h2 ? c[j] : c[2 + j], keep = h2 ? c[2 + j] : c[j];
+    d2[j] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+  }
+  const float send = h1 ? d2[0] : d2[1], keep = h1 ? d2[1] : d2[0];
+  const float e = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+  return e + __shfl_xor_sync(0xffffffffu, e, 1);
+}
+
 // ------------------------------------------------------------ P0: planes
 // The planes of one 64-input block of one activation row (64 values, two
 // per lane, already in registers; lane l holds inputs 2l, 2l+1): warp-wide.
@@ -779,57 +822,62 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     }
     __syncthreads();
     if (!p.hash) {
-      // router logits of experts blockIdx.x, +G, ... for every token (the consumer warps split d)
-      for (int e = blockIdx.x; e < E; e += p.G) {
-        if (warp < kDecConsumerWarps) {
-          const int span = d / kDecConsumerWarps;
-          for (int t0 = 0; t0 < T; t0 += 8) {  // tokens in groups of 8 (registers)
-            float acc[8];
+      // router logits of experts blockIdx.x, +G, ... for every token: passes
+      // of (2 experts, 8 tokens); every warp takes 256-input chunks, loads the
+      // chunk's x once for both experts, and reduces its 16 (expert, token)
+      // partials with one transposed butterfly; the chunks' partials are then
+      // summed in a fixed order (d is a multiple of 256 here)
+      const int ne = (int)blockIdx.x < E ? (E - 1 - (int)blockIdx.x) / p.G + 1 : 0;
+      const int nch = d / 256;
+      float* part = red;  // [chunk][2 experts][8 tokens]
+      for (int eb = 0; eb < ne; eb += 2) {
+        const int ea = blockIdx.x + eb * p.G, ebx = ea + p.G;
+        const bool two = eb + 1 < ne;
+        for (int t0 = 0; t0 < T; t0 += 8) {
+          for (int c = warp; c < nch; c += kDecWarps) {
+            const int i = c * 256 + lane * 8;
+            float wa[8], wb[8];
+            dec_router8(p, ea, i, wa);
+            if (two) dec_router8(p, ebx, i, wb);
+            else
 #pragma unroll
-            for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-            for (int i = warp * span + lane * 8; i < (warp + 1) * span; i += 256) {
-              float wv[8];
-              if (p.router_bf16) {
-                const uint4 r = __ldg(reinterpret_cast<const uint4*>(
-                    reinterpret_cast<const __nv_bfloat16*>(p.router_w) + (size_t)e * d + i));
-                wv[0] = bf16lo(r.x); wv[1] = bf16hi(r.x); wv[2] = bf16lo(r.y); wv[3] = bf16hi(r.y);
-                wv[4] = bf16lo(r.z); wv[5] = bf16hi(r.z); wv[6] = bf16lo(r.w); wv[7] = bf16hi(r.w);
-              } else {
-                const float4* rr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.router_w) +
-                                                                   (size_t)e * d + i);
-                const float4 a = __ldg(rr), bq = __ldg(rr + 1);
-                wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
-                wv[4] = bq.x; wv[5] = bq.y; wv[6] = bq.z; wv[7] = bq.w;
-              }
-#pragma unroll
-              for (int t = 0; t < 8; ++t) {
-                if (t0 + t < T) {
-                  const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)(t0 + t) * d + i));
-                  float a = acc[t];
-                  a = fmaf(wv[0], bf16lo(xv.x), a); a = fmaf(wv[1], bf16hi(xv.x), a);
-                  a = fmaf(wv[2], bf16lo(xv.y), a); a = fmaf(wv[3], bf16hi(xv.y), a);
-                  a = fmaf(wv[4], bf16lo(xv.z), a); a = fmaf(wv[5], bf16hi(xv.z), a);
-                  a = fmaf(wv[6], bf16lo(xv.w), a); a = fmaf(wv[7], bf16hi(xv.w), a);
-                  acc[t] = a;
-                }
-              }
-            }
+              for (int q = 0; q < 8; ++q) wb[q] = 0.f;
+            float acc[16];  // [expert][token]
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
+              float a0 = 0.f, a1 = 0.f;
               if (t0 + t < T) {
-                const float v = warp_sum(acc[t]);
-                if (lane == 0) red[warp * kDecMaxT + t0 + t] = v;
+                const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)(t0 + t) * d + i));
+                const float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
+                                     bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                  a0 = fmaf(wa[q], xf[q], a0);
+                  a1 = fmaf(wb[q], xf[q], a1);
+                }
               }
+              acc[t] = a0;
+              acc[8 + t] = a1;
+            }
+            // value v = 8 * expert + token ends in lanes 2v' and 2v'+1, where
+            // v' = 8*bit4 + 4*bit3 + 2*bit2 + bit1 of the lane
+            const float tot = dec_transpose_sum16(acc);
+            if ((lane & 1) == 0) {
+              const int v = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
+              part[c * 16 + v] = tot;
             }
           }
+          __syncthreads();
+          if (tid < 16) {
+            const int x = tid >> 3, t = tid & 7;
+            if (t0 + t < T && (x == 0 || two)) {
+              float sum = 0.f;
+              for (int c = 0; c < nch; ++c) sum += part[c * 16 + tid];  // fixed order
+              p.logits[(size_t)(t0 + t) * E + (x ? ebx : ea)] = sum;
+            }
+          }
+          __syncthreads();
         }
-        __syncthreads();
-        if (tid < T) {
-          float s = 0.f;
-          for (int w = 0; w < kDecConsumerWarps; ++w) s += red[w * kDecMaxT + tid];  // fixed order
-          p.logits[(size_t)tid * E + e] = s;
-        }
-        __syncthreads();
       }
     } else if ((int)blockIdx.x < T) {
       // hash routing of token blockIdx.x: table row, logits of its experts, weights
