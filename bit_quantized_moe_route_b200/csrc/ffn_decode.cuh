@@ -71,6 +71,7 @@ constexpr int kDecR2 = 32;         // rows of W2 per stage
 constexpr int kDecMaxTok = 4;      // tokens per group (B columns 0..7 of the MMA: hi and lo plane of each)
 constexpr int kDecMaxT = 32;
 constexpr int kDecMaxPairs = 256;  // T * top_k
+static_assert(kDecMaxPairs <= kDecThreads, "hash weights take one (token, slot) pair per thread");
 constexpr int kDecMaxE = 1024;
 constexpr int kDecCodeBytes = 32768;  // code bytes of a stage, at most
 constexpr int kDecMaxSeg = 1024;      // code bytes per row and stage, at most
@@ -879,86 +880,57 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
           __syncthreads();
         }
       }
-    } else if ((int)blockIdx.x < T) {
-      // hash routing of token blockIdx.x: table row, logits of its experts, weights
-      const int t = blockIdx.x;
+    } else {
+      // hash routing: the (token, slot) pairs blockIdx.x, +G, ...: the table
+      // entry and the fp32 logit of that expert (every warp takes 256-input
+      // chunks, summed in a fixed order); P1 turns logits into weights.  An
+      // out-of-range token id or table entry stores expert 0 with logit -inf
+      // (weight 0) and is reported.
       int* s_e = reinterpret_cast<int*>(hbuf);
-      int* s_ok = s_e + 32;
-      if (warp == 0) {
-        const int tok = p.token_ids[t];
-        const bool tok_ok = tok >= 0 && tok < p.vocab;
-        int e = 0;
-        bool good = false;
-        if (lane < k && tok_ok) {
-          e = p.tid2eid[(size_t)tok * k + lane];
-          good = e >= 0 && e < E;
-          if (!good) e = 0;
+      const int nch = d / 256;
+      for (int q = blockIdx.x; q < Tk; q += p.G) {
+        const int t = q / k, j = q - t * k;
+        if (tid == 0) {
+          const int tok = p.token_ids[t];
+          int e = 0, good = 0;
+          if (tok >= 0 && tok < p.vocab) {
+            e = p.tid2eid[(size_t)tok * k + j];
+            good = e >= 0 && e < E;
+            if (!good) e = 0;
+          }
+          if (!good) set_error(p.err, kErrDeviceInput);
+          s_e[0] = e;
+          s_e[1] = good;
         }
-        if (__any_sync(0xffffffffu, !tok_ok || (lane < k && !good)) && lane == 0) set_error(p.err, kErrDeviceInput);
-        s_e[lane] = e;
-        s_ok[lane] = good ? 1 : 0;
-      }
-      __syncthreads();
-      if (p.router_w != nullptr && warp < kDecConsumerWarps) {
-        const int span = d / kDecConsumerWarps;
-        for (int j0 = 0; j0 < k; j0 += 8) {  // the table's experts in groups of 8 (registers)
-          float acc[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-          for (int i = warp * span + lane * 8; i < (warp + 1) * span; i += 256) {
+        __syncthreads();
+        const int e = s_e[0], good = s_e[1];
+        if (good && p.router_w != nullptr) {
+          for (int c = warp; c < nch; c += kDecWarps) {
+            const int i = c * 256 + lane * 8;
+            float w[8];
+            dec_router8(p, e, i, w);
             const uint4 xv = __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)t * d + i));
             const float xf[8] = {bf16lo(xv.x), bf16hi(xv.x), bf16lo(xv.y), bf16hi(xv.y),
                                  bf16lo(xv.z), bf16hi(xv.z), bf16lo(xv.w), bf16hi(xv.w)};
+            float a = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (j0 + j < k) {
-                const size_t off = (size_t)s_e[j0 + j] * d + i;
-                float wv[8];
-                if (p.router_bf16) {
-                  const uint4 r = __ldg(reinterpret_cast<const uint4*>(
-                      reinterpret_cast<const __nv_bfloat16*>(p.router_w) + off));
-                  wv[0] = bf16lo(r.x); wv[1] = bf16hi(r.x); wv[2] = bf16lo(r.y); wv[3] = bf16hi(r.y);
-                  wv[4] = bf16lo(r.z); wv[5] = bf16hi(r.z); wv[6] = bf16lo(r.w); wv[7] = bf16hi(r.w);
-                } else {
-                  const float4* rr = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.router_w) + off);
-                  const float4 a = __ldg(rr), bq = __ldg(rr + 1);
-                  wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w;
-                  wv[4] = bq.x; wv[5] = bq.y; wv[6] = bq.z; wv[7] = bq.w;
-                }
-                float a = acc[j];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) a = fmaf(wv[q], xf[q], a);
-                acc[j] = a;
-              }
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (j0 + j < k) {
-              const float v = warp_sum(acc[j]);
-              if (lane == 0) red[warp * 32 + j0 + j] = v;
-            }
+            for (int u = 0; u < 8; ++u) a = fmaf(w[u], xf[u], a);
+            a = warp_sum(a);
+            if (lane == 0) red[c] = a;
           }
         }
-      }
-      __syncthreads();
-      if (warp == 0) {
-        float sj = 0.f;
-        const bool gj = lane < k && s_ok[lane];
-        if (gj) {
-          if (p.router_w != nullptr) {
-            float l = 0.f;
-            for (int w = 0; w < kDecConsumerWarps; ++w) l += red[w * 32 + lane];
-            sj = sqrt_softplus(l);
-          } else {
-            sj = 1.f;
+        __syncthreads();
+        if (tid == 0) {
+          float l = -INFINITY;
+          if (good) {
+            l = 0.f;
+            if (p.router_w != nullptr)
+              for (int c = 0; c < nch; ++c) l += red[c];  // fixed order
           }
+          p.hids[q] = e;
+          p.hw[q] = l;
         }
-        const float ssum = warp_sum(sj);
-        if (lane < k) {
-          p.hids[t * k + lane] = s_e[lane];
-          p.hw[t * k + lane] = gj && ssum > 0.f ? sj / ssum : 0.f;
-        }
+        __syncthreads();
       }
     }
   }
@@ -975,10 +947,25 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
         dec_topk<32>(p.logits + (size_t)t * E, p.router_b, E, k, r_ids + t * k, r_w + t * k);
     }
   } else {
-    for (int i = tid; i < Tk; i += kDecThreads) {
-      r_ids[i] = __ldcg(p.hids + i);
-      r_w[i] = __ldcg(p.hw + i);
+    // weights from the P0 logits: renormalised sqrtsoftplus over the token's
+    // slots (uniform over its valid slots without a router; -inf marks an
+    // invalid entry, weight 0); Tk <= 256 < threads: one pair per thread
+    float sj = 0.f;
+    if (tid < Tk) {
+      r_ids[tid] = __ldcg(p.hids + tid);
+      const float l = __ldcg(p.hw + tid);
+      sj = l == -INFINITY ? 0.f : (p.router_w != nullptr ? sqrt_softplus(l) : 1.f);
+      r_w[tid] = sj;
     }
+    __syncthreads();
+    if (tid < Tk) {
+      const int t0 = tid - tid % k;
+      float ssum = 0.f;
+      for (int jj = 0; jj < k; ++jj) ssum += r_w[t0 + jj];  // ascending slot
+      sj = ssum > 0.f ? sj / ssum : 0.f;
+    }
+    __syncthreads();
+    if (tid < Tk) r_w[tid] = sj;
   }
   __syncthreads();
   // per-expert counts (out-of-range ids are reported and counted as expert 0)
