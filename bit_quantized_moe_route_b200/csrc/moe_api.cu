@@ -850,8 +850,8 @@ bool dec_mat(const QMatDev& Q, bool w2, DecMat* m) {
 bool dec_plan(const moe_dims_t& d, const QMatDev& w1, const QMatDev& w3, const QMatDev& w2, const QMatDev* sh,
               DecParams* p, size_t* smem) {
   if (d.T < 1 || d.T > kDecMaxT || d.T * d.top_k > kDecMaxPairs || d.n_experts > kDecMaxE) return false;
-  // d_model a multiple of 128: the logit pass gives each lane 8 consecutive inputs of a 1/8 slice
-  if (d.d_model % 128 || d.d_ff % kDecRows || (sh && d.d_ff_shared % kDecRows)) return false;
+  // d_model a multiple of 256: the routing passes take 256-input chunks (8 inputs per lane)
+  if (d.d_model % 256 || d.d_ff % kDecRows || (sh && d.d_ff_shared % kDecRows)) return false;
   const QMatDev* mats[6] = {&w1, &w3, &w2, sh ? &sh[0] : &w1, sh ? &sh[1] : &w3, sh ? &sh[2] : &w2};
   DecMat m[6];
   for (int i = 0; i < 6; ++i)

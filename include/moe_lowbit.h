@@ -363,9 +363,10 @@ const char* moe_timing_label(int32_t i);
  * threads' calls are not affected; not for the allocation-free entry point,
  * which always streams).  For moe_forward / moe_forward_host, AUTO (default)
  * runs the whole layer as ONE fused launch for small batches when the shapes
- * allow it (T <= 32, T*top_k <= 256, d_model and d_ff multiples of 64 and of
- * the formats' stage widths -- 1024 inputs for 2-bit, 512 for 3/4-bit and
- * mxfp4, 256 for 8-bit -- and not 2-bit with 32-input groups): routing,
+ * allow it (T <= 32, T*top_k <= 256, d_model a multiple of 256, d_model and
+ * d_ff multiples of 64 and of the formats' stage widths -- 1024 inputs for
+ * 2-bit, 512 for 3/4-bit and mxfp4, 256 for 8-bit -- and not 2-bit with
+ * 32-input groups): routing,
  * both FFN stages on the integer tensor-core MMA, and the combine (whose k
  * slots are summed in ascending j, then the shared expert, one bf16
  * rounding).  Otherwise AUTO takes the tcgen05 grouped GEMM from T >= 4
