@@ -1188,18 +1188,21 @@ moe_status_t moe_combine(const moe_dims_t* dims, const float* y, const int32_t* 
   return launch_combine(*dims, y, inv, topk_w, y_shared, out, reinterpret_cast<cudaStream_t>(stream));
 }
 
-moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* token_ids, const void* router_w,
-                         const float* router_b, const int32_t* tid2eid, const moe_qmat_t* w1,
-                         const moe_qmat_t* w3, const moe_qmat_t* w2, const moe_qmat_t* shared, void* out,
-                         int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
-  g_detail[0] = 0;
+namespace {
+// The whole layer; `out_mapped`: `out` is the device address of page-locked
+// host memory (moe_forward_host's direct output), not device memory.
+moe_status_t forward_impl(const moe_dims_t* dims, const void* x, const int32_t* token_ids, const void* router_w,
+                          const float* router_b, const int32_t* tid2eid, const moe_qmat_t* w1,
+                          const moe_qmat_t* w3, const moe_qmat_t* w2, const moe_qmat_t* shared, void* out,
+                          bool out_mapped, int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                          void* stream) {
   moe_status_t st = check_dims(dims);
   if (st != MOE_OK) return st;
   const moe_dims_t& d = *dims;
   WsLayout L;
   if ((st = check_ws(d, ws, ws_bytes, &L)) != MOE_OK) return st;
   if ((st = check_route_args(d, x, router_w, token_ids, tid2eid)) != MOE_OK) return st;
-  if ((st = check_dev_ptr(out, "out")) != MOE_OK) return st;
+  if (!out_mapped && (st = check_dev_ptr(out, "out")) != MOE_OK) return st;
   if (!aligned16(out)) return fail(MOE_ERR_INVALID_ARG, "out must be 16-byte aligned");
   QMatDev q1, q3, q2, qs[3];
   if ((st = check_qmat(w1, d.d_model, "w1", &q1, d.d_ff)) != MOE_OK) return st;
@@ -1222,6 +1225,16 @@ moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* t
                         ws, L, s);
   hook_end();
   return st;
+}
+}  // namespace
+
+moe_status_t moe_forward(const moe_dims_t* dims, const void* x, const int32_t* token_ids, const void* router_w,
+                         const float* router_b, const int32_t* tid2eid, const moe_qmat_t* w1,
+                         const moe_qmat_t* w3, const moe_qmat_t* w2, const moe_qmat_t* shared, void* out,
+                         int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  g_detail[0] = 0;
+  return forward_impl(dims, x, token_ids, router_w, router_b, tid2eid, w1, w3, w2, shared, out, false, topk_ids_out,
+                      topk_w_out, ws, ws_bytes, stream);
 }
 
 moe_status_t moe_forward_partial(const moe_dims_t* dims, int32_t expert_begin, int32_t expert_end,
@@ -1308,6 +1321,9 @@ moe_status_t forward_launches(const moe_dims_t& d, const void* x, const int32_t*
 
 extern "C" {
 
+// Outputs up to this size go straight into mapped host memory (moe_forward_host).
+constexpr size_t kHostDirectOutMax = 1u << 20;
+
 moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const int32_t* token_ids_host,
                               const void* router_w, const float* router_b, const int32_t* tid2eid,
                               const moe_qmat_t* w1, const moe_qmat_t* w3, const moe_qmat_t* w2,
@@ -1331,11 +1347,27 @@ moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const 
     e = cudaMemcpyAsync(td, token_ids_host, (size_t)d.T * sizeof(int), cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return cuda_fail(e, "copy token ids to device");
   }
-  st = moe_forward(dims, xd, d.hash_mode ? td : nullptr, router_w, router_b, tid2eid, w1, w3, w2, shared, od,
-                   nullptr, nullptr, ws, ws_bytes, stream);
+  // A small output into page-locked, device-mapped host memory is written
+  // there by the layer's last kernel (no separate device-to-host copy);
+  // otherwise it goes through the workspace and one copy.
+  bool direct = false;
+  if (xbytes <= kHostDirectOutMax) {
+    cudaPointerAttributes pa{};
+    if (cudaPointerGetAttributes(&pa, out_host) == cudaSuccess && pa.type == cudaMemoryTypeHost &&
+        pa.devicePointer != nullptr && aligned16(pa.devicePointer)) {
+      od = pa.devicePointer;
+      direct = true;
+    } else {
+      cudaGetLastError();  // pageable memory: not an error
+    }
+  }
+  st = forward_impl(dims, xd, d.hash_mode ? td : nullptr, router_w, router_b, tid2eid, w1, w3, w2, shared, od, direct,
+                    nullptr, nullptr, ws, ws_bytes, stream);
   if (st != MOE_OK) return st;
-  e = cudaMemcpyAsync(out_host, od, xbytes, cudaMemcpyDeviceToHost, s);
-  if (e != cudaSuccess) return cuda_fail(e, "copy out to host");
+  if (!direct) {
+    e = cudaMemcpyAsync(out_host, od, xbytes, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy out to host");
+  }
   return MOE_OK;
 }
 

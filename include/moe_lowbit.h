@@ -291,10 +291,13 @@ moe_status_t moe_forward_partial(const moe_dims_t* dims, int32_t expert_begin, i
 /*
  * moe_forward with HOST activations: x_host (bf16 [T, d_model]) and, in hash
  * mode, token_ids_host (int32 [T]) are copied to the workspace, the layer
- * runs, and the bf16 result is copied back to out_host.  Weights, router and
- * table stay device pointers.  Copies are cudaMemcpyAsync on `stream`; use
- * pinned host memory for asynchrony and synchronise the stream before
- * reading out_host.
+ * runs, and the bf16 result reaches out_host: written there directly by the
+ * layer's last kernel when out_host is page-locked host memory mapped into
+ * the device's address space (cudaHostAlloc, or a pinned torch tensor) and
+ * the output is at most 1 MiB, else copied back from the workspace.
+ * Weights, router and table stay device pointers.  Copies are
+ * cudaMemcpyAsync on `stream`; use pinned host memory for asynchrony and
+ * synchronise the stream before reading out_host.
  */
 moe_status_t moe_forward_host(const moe_dims_t* dims, const void* x_host, const int32_t* token_ids_host,
                               const void* router_w, const float* router_b, const int32_t* tid2eid,

@@ -159,14 +159,33 @@ def test_large_permutation_bit_exact(device):
     assert np.array_equal(inv.cpu().numpy(), o_inv)
 
 
-def test_forward_host_matches_device_path(device):
-    inp = make_inputs("tiny", device)
-    out, _, _, ws = run_forward(inp)
-    dims = dims_for(inp)
-    x_h = inp.x.cpu().pin_memory()
-    out_h = torch.empty(inp.cfg["T"], inp.cfg["d"], dtype=torch.bfloat16).pin_memory()
-    moe.forward_host(dims, x_h, None, inp.router_w, inp.router_b, None, inp.w1, inp.w3, inp.w2, None, out_h, ws)
-    torch.cuda.synchronize()
+FUSED_HOST = dict(T=1, d=1024, E=16, k=4, f=1024, routing="learned", vocab=0, w13=("affine", 4, 64),
+                  w2=("affine", 4, 64), shared=("affine", 8, 64), f_shared=1024, weight_std=0.02, router_std=0.05,
+                  bias_std=0.01, seed=830)
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+@pytest.mark.parametrize("layer", ["tiny", "fused"])
+def test_forward_host_matches_device_path(device, layer, pinned):
+    """Host buffers in and out: pinned (mapped) output is written directly by
+    the layer's last kernel, pageable output is copied back; both equal the
+    device-pointer call bit for bit."""
+    inp = make_inputs("tiny", device) if layer == "tiny" else make_custom(FUSED_HOST, device)
+    prev = moe.set_ffn_path(moe.FFN_DECODE_FUSED) if layer == "fused" else None  # this thread only
+    try:
+        out, _, _, ws = run_forward(inp)
+        dims = dims_for(inp)
+        x_h = inp.x.cpu().pin_memory()
+        out_h = torch.full((inp.cfg["T"], inp.cfg["d"]), float("nan"), dtype=torch.bfloat16)
+        if pinned:
+            out_h = out_h.pin_memory()
+        moe.forward_host(dims, x_h, None, inp.router_w, inp.router_b, None, inp.w1, inp.w3, inp.w2, inp.shared, out_h,
+                         ws)
+        torch.cuda.synchronize()
+    finally:
+        if prev is not None:
+            moe.set_ffn_path(prev)
+    assert moe.read_device_error(ws) == 0
     assert torch.equal(out_h, out.cpu())
 
 
