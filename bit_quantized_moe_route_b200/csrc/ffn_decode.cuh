@@ -419,8 +419,16 @@ MOE_DEV void dec_fold(uint32_t s0, uint32_t s8, uint32_t brow, float st, float s
     sc8 = bf16_bits_to_float(lds16u(s8 + 2 * GI));
     b8 = bf16_bits_to_float(lds16u(s8 + brow + 2 * GI));
   }
-  acc[0] = fmaf(sc0 * st, (float)(c[0] * 256 + c[1]), fmaf(b0, sm, acc[0]));
-  acc[1] = fmaf(sc8 * st, (float)(c[2] * 256 + c[3]), fmaf(b8, sm, acc[1]));
+  if constexpr (FMT == F_MX4) {  // no bias term
+    (void)b0;
+    (void)b8;
+    (void)sm;
+    acc[0] = fmaf(sc0 * st, (float)(c[0] * 256 + c[1]), acc[0]);
+    acc[1] = fmaf(sc8 * st, (float)(c[2] * 256 + c[3]), acc[1]);
+  } else {
+    acc[0] = fmaf(sc0 * st, (float)(c[0] * 256 + c[1]), fmaf(b0, sm, acc[0]));
+    acc[1] = fmaf(sc8 * st, (float)(c[2] * 256 + c[3]), fmaf(b8, sm, acc[1]));
+  }
 }
 
 // k-block H of block B of the warp's slice for one tile: A fragment, one MMA
