@@ -14,7 +14,8 @@
 //       grid barrier (bounded);
 //   P1  every CTA, redundantly: top-k of every token (one warp per token),
 //       per-expert counts, offsets and "groups" of <= ntmax (<= 4) tokens of one expert
-//       (one warp scan; the shared expert's tokens form their own groups),
+//       (warp scans over 32-expert chunks, one chunk per warp; the shared
+//       expert's tokens form their own groups),
 //       the stable (token, slot) order within each expert (warp match);
 //   S1  units (group, 64 rows of d_ff): h = silu(W1 x) * (W3 x) for the
 //       group's tokens, written as the planes W2 reads; a per-group counter
@@ -27,7 +28,7 @@
 //       rounding).
 // Units are claimed dynamically in the order [S1 shared, S1 routed, S2 by
 // group]: a CTA's first unit is its index, the next comes from a launch-wide
-// counter, claimed one unit ahead.
+// counter, claimed once the current unit's weight stages are all issued.
 //
 // Weight stream.  One producer warp fills a ring of 32 KB stages; a stage is
 // a set of WHOLE row segments: 16 rows of W1 and the same 16 rows of W3 (S1)
@@ -807,6 +808,11 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     const CUtensorMap* mp = lane < 6 ? &p.map[lane] : lane < 12 ? &p.smap[lane - 6] : &p.bmap[lane - 12];
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(mp)) : "memory");
   }
+  if (warp == kDecServiceWarp && !p.hash && p.router_b != nullptr && lane * 32 < E) {
+    // every CTA's top-k reads the selection bias right after the grid
+    // barrier: bring its lines into L2 now, off that path
+    asm volatile("prefetch.global.L2 [%0];" ::"l"((uint64_t)__cvta_generic_to_global(p.router_b + lane * 32)) : "memory");
+  }
   for (int e = tid; e < E; e += kDecThreads) r_off[e] = 0;  // per-expert counts (P1)
   __syncthreads();
 
@@ -990,21 +996,27 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     if (bad) set_error(p.err, kErrDeviceInput);
   }
   __syncthreads();
-  if (warp == 0) {
-    // offsets (exclusive scan), cursors and groups, in rounds of 32 experts
-    // (lane l takes expert 32r + l: conflict-free shared accesses) with the
-    // running totals carried between rounds; groups in ascending expert
-    // order after the shared ones
+  {
+    // offsets (exclusive scan of the counts), cursors and groups, one chunk of
+    // 32 experts per warp at a time (lane l takes expert 32c + l:
+    // conflict-free shared accesses): the first pass scans within each chunk
+    // and records the chunk's totals, the second adds the totals of the
+    // chunks before it.  Groups in ascending expert order after the shared
+    // ones.
     const int gsz = p.ntmax;
     const int nsg = p.has_shared && p.with_shared ? (T + gsz - 1) / gsz : 0;
-    int run = 0, gbase = nsg;  // pairs and groups before this round
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      const int c = e < E ? r_off[e] : 0;
-      const bool own = e < E && e >= p.e_begin && e < p.e_end;
-      // ceil(c / gsz) for gsz in 1..4 without a runtime division
-      const int ng = !own ? 0 : gsz == 1 ? c : gsz == 2 ? (c + 1) >> 1 : gsz == 3 ? (c + 2) / 3 : (c + 3) >> 2;
-      int sc = c, sg = ng;  // inclusive warp scans
+    const int nchk = (E + 31) >> 5;  // <= 32
+    int* tot = reinterpret_cast<int*>(red);  // [chunk]: pairs, groups (red is free until the units)
+    // groups of expert e's n pairs: ceil(n / gsz) for gsz in 1..4 without a
+    // runtime division; none for an expert outside [e_begin, e_end)
+    auto ngroups = [&](int e, int n) {
+      if (e >= E || e < p.e_begin || e >= p.e_end) return 0;
+      return gsz == 1 ? n : gsz == 2 ? (n + 1) >> 1 : gsz == 3 ? (n + 2) / 3 : (n + 3) >> 2;
+    };
+    for (int c = warp; c < nchk; c += kDecWarps) {
+      const int e = 32 * c + lane;
+      const int n = e < E ? r_off[e] : 0, ng = ngroups(e, n);
+      int sc = n, sg = ng;  // inclusive warp scans
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int a = __shfl_up_sync(0xffffffffu, sc, o), b = __shfl_up_sync(0xffffffffu, sg, o);
@@ -1013,23 +1025,39 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
           sg += b;
         }
       }
-      const int off = run + sc - c;
+      if (e < E) r_cur[e] = (sc - n) | ((sg - ng) << 16);  // exclusive within the chunk (each < 2^16)
+      if (lane == 31) {
+        tot[2 * c] = sc;
+        tot[2 * c + 1] = sg;
+      }
+    }
+    __syncthreads();
+    for (int c = warp; c < nchk; c += kDecWarps) {
+      const int pc = __reduce_add_sync(0xffffffffu, lane < c ? tot[2 * lane] : 0);
+      const int pg = __reduce_add_sync(0xffffffffu, lane < c ? tot[2 * lane + 1] : 0);
+      const int e = 32 * c + lane;
       if (e < E) {
+        const int n = r_off[e], w = r_cur[e];
+        const int off = pc + (w & 0xffff);
         r_off[e] = off;
         r_cur[e] = off;
+        if (ngroups(e, n) > 0)
+          for (int q0 = 0, gi = nsg + pg + (w >> 16); q0 < n; q0 += gsz) r_groups[gi++] = make_int4(e, off + q0, min(gsz, n - q0), 0);
       }
-      if (own)
-        for (int q0 = 0, gi = gbase + sg - ng; q0 < c; q0 += gsz) r_groups[gi++] = make_int4(e, off + q0, min(gsz, c - q0), 0);
-      run += __shfl_sync(0xffffffffu, sc, 31);
-      gbase += __shfl_sync(0xffffffffu, sg, 31);
     }
-    if (lane == 0) {
-      r_off[E] = run;
-      misc[1] = nsg;
-      misc[2] = gbase - nsg;
+    if (warp == 0) {
+      const int run = __reduce_add_sync(0xffffffffu, lane < nchk ? tot[2 * lane] : 0);
+      const int ngr = __reduce_add_sync(0xffffffffu, lane < nchk ? tot[2 * lane + 1] : 0);
+      if (lane == 0) {
+        r_off[E] = run;
+        misc[1] = nsg;
+        misc[2] = ngr;
+      }
+      if (lane < nsg) r_groups[lane] = make_int4(-1, lane * gsz, min(gsz, T - lane * gsz), 0);
     }
-    if (lane < nsg) r_groups[lane] = make_int4(-1, lane * gsz, min(gsz, T - lane * gsz), 0);
-    __syncwarp();
+    __syncthreads();
+  }
+  if (warp == 0) {
     // stable order within each expert: pairs in ascending flat index
     const unsigned lt = (1u << lane) - 1u;
     for (int c0 = 0; c0 < Tk; c0 += 32) {
@@ -1069,7 +1097,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     int np = 0;           // plane buffers issued
     if (lane == 0) {
       // units are claimed dynamically: the CTA's first is blockIdx.x, every
-      // later one comes from the launch-wide counter, claimed one unit ahead
+      // later one comes from the launch-wide counter
       int ui = blockIdx.x;
       while (!*abort_flag) {
         if (ui >= n_units) {
@@ -1085,7 +1113,6 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
           ++np;
           break;
         }
-        const int ui_next = p.G + atomicAdd(p.sync + 2, 1);
         const DecUnit U = dec_unit(p, r_groups, nsg, nrg, ui);
         const int4 grp = r_groups[U.grp];
         const DecMat& m0 = p.m[U.mi];
@@ -1167,7 +1194,9 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
         }
         for (; st < nst; ++st)
           if (!issue_stage(st)) break;
-        ui = ui_next;
+        // the next unit is claimed only now: a unit claimed while this one
+        // still streams could wait behind it while another CTA idles
+        ui = p.G + atomicAdd(p.sync + 2, 1);
       }
       // drain: every issued copy must land before the block exits
       for (int q = max(0, rg.n - p.nslot); q < rg.n; ++q) {
