@@ -818,9 +818,10 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
 
   // ------------------------------------------------------------ P0
   {
-    // activation planes: (token, 64-input block) tasks over every warp of the grid
+    // activation planes: (token, 64-input block) tasks over every warp of the
+    // grid, from the last CTA down: the first CTAs take the most router rows
     const int nb = d / 64;
-    const int gw = blockIdx.x * kDecWarps + warp, W = p.G * kDecWarps;
+    const int gw = (p.G - 1 - (int)blockIdx.x) * kDecWarps + warp, W = p.G * kDecWarps;
     int* scratch = reinterpret_cast<int*>(red) + warp * 64;
     const int f0 = p.m[DM_W1].fmt, f1 = p.m[DM_S1].fmt;
     for (int it = gw; it < T * nb; it += W) {
@@ -849,14 +850,23 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
         const int ea = blockIdx.x + eb * p.G, ebx = ea + p.G;
         const bool two = eb + 1 < ne;
         for (int t0 = 0; t0 < T; t0 += 8) {
-          for (int c = warp; c < nch; c += kDecWarps) {
+          // the router weights of the warp's next chunk are requested before
+          // this chunk's sums, so a warp's chunks wait on DRAM together
+          auto load = [&](int c, float(&a)[8], float(&b)[8]) {
             const int i = c * 256 + lane * 8;
-            float wa[8], wb[8];
-            dec_router8(p, ea, i, wa);
-            if (two) dec_router8(p, ebx, i, wb);
+            dec_router8(p, ea, i, a);
+            if (two) dec_router8(p, ebx, i, b);
             else
 #pragma unroll
-              for (int q = 0; q < 8; ++q) wb[q] = 0.f;
+              for (int q = 0; q < 8; ++q) b[q] = 0.f;
+          };
+          float wa[8], wb[8];
+          if (warp < nch) load(warp, wa, wb);
+          for (int c = warp; c < nch; c += kDecWarps) {
+            const int i = c * 256 + lane * 8;
+            const bool more = c + kDecWarps < nch;
+            float na[8], nb[8];
+            if (more) load(c + kDecWarps, na, nb);
             float acc[16];  // [expert][token]
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
@@ -881,6 +891,12 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
               const int v = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 + ((lane >> 1) & 1);
               part[c * 16 + v] = tot;
             }
+            if (more)
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                wa[q] = na[q];
+                wb[q] = nb[q];
+              }
           }
           __syncthreads();
           if (tid < 16) {
