@@ -96,6 +96,12 @@ class QMat:
             self, q=self.q.to(device), scales=self.scales.to(device),
             biases=None if self.biases is None else self.biases.to(device))
 
+    def clone(self) -> "QMat":
+        """The same packs in fresh buffers (equal values, other addresses)."""
+        return dataclasses.replace(
+            self, q=self.q.clone(), scales=self.scales.clone(),
+            biases=None if self.biases is None else self.biases.clone())
+
     def expert_numpy(self, e: int):
         """Host copies of expert ``e``'s packs: (uint32 words, scales, biases).
 
@@ -136,6 +142,17 @@ class MoEInputs:
             token_ids=mv(self.token_ids), tid2eid=mv(self.tid2eid),
             w1=self.w1.to(device), w3=self.w3.to(device), w2=self.w2.to(device),
             shared=None if self.shared is None else tuple(m.to(device) for m in self.shared))
+
+    def clone(self) -> "MoEInputs":
+        """The same layer in fresh buffers on the same device: equal values
+        (so equal routing and work), other addresses (so no cache line of one
+        copy serves a read of another)."""
+        cp = lambda t: None if t is None else t.clone()  # noqa: E731
+        return dataclasses.replace(
+            self, x=cp(self.x), router_w=cp(self.router_w), router_b=cp(self.router_b),
+            token_ids=cp(self.token_ids), tid2eid=cp(self.tid2eid),
+            w1=self.w1.clone(), w3=self.w3.clone(), w2=self.w2.clone(),
+            shared=None if self.shared is None else tuple(m.clone() for m in self.shared))
 
 
 # --------------------------------------------------------------------------
