@@ -6,15 +6,16 @@ One step = one full layer forward (routing, permutation, grouped SwiGLU
 expert FFN over packed weights, combine) over one batch of synthetic input
 resident in HBM.  The default workload is the decode layer (T=1 token,
 d_model=4096, 256 routed experts, top-8, d_ff=2048, affine 4-bit group-64
-experts plus an 8-bit shared expert).  The layer's inputs are larger than
-L2 across steps: --layers copies of the layer (equal values, distinct
-buffers, several GB in all) are cycled, so each step reads weights last
-touched --layers - 1 steps earlier, behind hundreds of MB of other weight
-traffic, as the layers of a model do; the kernels' code stays resident as it
-does when every layer runs it.  The same steps are also timed on ONE copy
-with L2 flushed before each step by READING a 512 MiB buffer (outside the
-events; a read leaves no dirty lines), code evicted too, and reported as
-"l2_flushed" in the same line.  The reported step time is the median over
+experts plus an 8-bit shared expert).  Inputs larger than L2 between
+steps: where a step reads under 8x L2 of weights (decode, mixed), 4 copies
+of the layer (equal values, distinct buffers, GBs in all) are cycled, so a
+step reads weights last touched 3 steps earlier, behind hundreds of MB of
+other copies' traffic, as the layers of a model do, and the same kernel ran
+just before it; the same steps are also timed on ONE copy with L2 flushed
+before each step by READING a 512 MiB buffer (outside the events; a read
+leaves no dirty lines) and reported as "l2_flushed" in the same line.
+Workloads that read many times L2 per step (hash, prefill) take one copy
+flushed before each step (--layers overrides).  The reported step time is the median over
 the timed steps (min, mean and p90 beside it).  --config all prints one line
 per layer configuration (tiny, hash, mixed, prefill, then the decode line
 last).
@@ -59,8 +60,9 @@ def parse():
     ap.add_argument("--ffn-path", default="auto", choices=["auto", "gemv", "tc"],
                     help="expert-FFN implementation: library default, weight-streaming GEMV, tensor-core GEMM")
     ap.add_argument("--cpu-budget", type=float, default=25.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--layers", type=int, default=4,
-                    help="copies of the layer cycled between timed steps (1: one copy, L2 flushed before each step)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="copies of the layer cycled between timed steps (1: one copy, L2 flushed before each step; "
+                         "0: 4 copies when a step reads under 8x L2 of weights, else 1)")
     ap.add_argument("--override", action="append", default=[],
                     help="key=value change to the workload (profiling small cases), e.g. E=16")
     return ap.parse_args()
@@ -448,8 +450,16 @@ def run_config(name, args, dev, world, rank):
     out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
     ids = torch.empty(T, k, dtype=torch.int32, device=dev)
     wts = torch.empty(T, k, dtype=torch.float32, device=dev)
-    # copies of the layer in distinct buffers, cycled between timed steps
-    n_layers = max(1, args.layers)
+    # copies of the layer in distinct buffers, cycled between timed steps,
+    # where a step reads few enough weight bytes that L2 could otherwise carry
+    # some from one step to the next; a step reading many times L2 takes one
+    # copy with L2 flushed before each step
+    moe.forward(dims, inp.x, inp.token_ids, inp.router_w, inp.router_b, inp.tid2eid, inp.w1, inp.w3, inp.w2,
+                inp.shared, out, ws, topk_ids_out=ids, topk_w_out=wts)
+    torch.cuda.synchronize()
+    step_weight_bytes = kernel_work(inp, ids.cpu().numpy(), False)[3]
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_layers = args.layers if args.layers > 0 else (4 if step_weight_bytes < 8 * l2_bytes else 1)
     layers = [inp] + [inp.clone() for _ in range(n_layers - 1)]
     # L2 flush by a read of 512 MiB (> 4x L2) into one small result
     flush = torch.ones(128 * 1024 * 1024, dtype=torch.int32, device=dev)
@@ -496,19 +506,6 @@ def run_config(name, args, dev, world, rank):
         dist.barrier()
     st = step_stats([a.elapsed_time(b) for a, b in step_ev])
     ms_per_step = max_over_ranks(st["median"], dev)
-    # the same steps on one copy with L2 (code included) flushed before each
-    flushed = None
-    if n_layers > 1:
-        for s in range(args.steps):
-            flush_l2()
-            step_ev[s][0].record(stream)
-            fwd(0)
-            step_ev[s][1].record(stream)
-        torch.cuda.synchronize()
-        stf = step_stats([a.elapsed_time(b) for a, b in step_ev])
-        ms_flushed = max_over_ranks(stf["median"], dev)
-        flushed = {"value": whole_job_rate(T, world, ms_flushed), "ms_per_step": ms_flushed, "step_ms": stf}
-
     # ---- per-kernel durations: a second timed pass with CUDA events recorded
     # by the library between its kernels on the same stream (the events add
     # small gaps between kernels, so the step time above is taken without them)
@@ -527,6 +524,21 @@ def run_config(name, args, dev, world, rank):
         for i, lab in enumerate(labels):
             per_kernel.setdefault(lab, []).append(evs[s][i].elapsed_time(evs[s][i + 1]))
     kern_ms = {lab: statistics.median(v) for lab, v in per_kernel.items()}
+
+    # the same steps on one copy with L2 (code included) flushed before each
+    # (after the per-kernel pass, so that pass follows the same load as the
+    # timed steps)
+    flushed = None
+    if n_layers > 1:
+        for s in range(args.steps):
+            flush_l2()
+            step_ev[s][0].record(stream)
+            fwd(0)
+            step_ev[s][1].record(stream)
+        torch.cuda.synchronize()
+        stf = step_stats([a.elapsed_time(b) for a, b in step_ev])
+        ms_flushed = max_over_ranks(stf["median"], dev)
+        flushed = {"value": whole_job_rate(T, world, ms_flushed), "ms_per_step": ms_flushed, "step_ms": stf}
 
     # ---- end-to-end through the C ABI with host buffers (pinned), copies inside
     x_h = inp.x.cpu().pin_memory()
