@@ -587,8 +587,8 @@ def run_config(name, args, dev, world, rank):
         copy_gb = sum(t.numel() * t.element_size() for t in layer_tensors(inp)) / 1e9
         l2_desc = (f"inputs larger than L2: {n_layers} copies of the layer ({copy_gb:.2f} GB each, distinct buffers) "
                    f"cycled, no flush; a step's weights were last read {n_layers - 1} steps earlier, behind "
-                   f"{(n_layers - 1) * lbytes / 1e6:.0f} MB of other copies' traffic; kernel code stays L2-resident "
-                   "as in a multi-layer model (one copy with L2 flushed before each step: l2_flushed)")
+                   f"{(n_layers - 1) * lbytes / 1e6:.0f} MB of other copies' traffic, and the same kernels ran "
+                   "just before, as in a multi-layer model (one copy with L2 flushed before each step: l2_flushed)")
     else:
         l2_desc = "flushed by reading a 512 MiB buffer between timed steps (outside the events)"
     line = {
