@@ -15,10 +15,10 @@ just before it; the same steps are also timed on ONE copy with L2 flushed
 before each step by READING a 512 MiB buffer (outside the events; a read
 leaves no dirty lines) and reported as "l2_flushed" in the same line.
 Workloads that read many times L2 per step (hash, prefill) take one copy
-flushed before each step (--layers overrides).  The reported step time is the median over
-the timed steps (min, mean and p90 beside it).  --config all prints one line
-per layer configuration (tiny, hash, mixed, prefill, then the decode line
-last).
+flushed before each step (--layers overrides).  The reported step time is
+the median over the timed steps (min, mean and p90 beside it).  --config all
+prints one line per layer configuration (tiny, hash, mixed, prefill, then
+the decode line last).
 
 With N > 1 (launched by torchrun) every rank runs an independent replica of
 the layer on its own GPU ("replicas only": the layer has no exchange step on
