@@ -80,7 +80,6 @@ static_assert(kUmEpiWarp0 % 4 == 0, "epilogue warps must cover the four TMEM lan
 static_assert(kUmAccCol0 + kUmNAcc * kUmAccCols <= kUmTmemCols, "TMEM columns");
 static_assert(kUmNA >= kUmGroups, "every dequant group needs a stage slot");
 static_assert(kUmN % 32 == 0 && kUmBBlock % 1024 == 0, "pair MMA N and swizzle atoms");
-static_assert(kUmBHalf > 64 && kUmBHalf <= 256, "the largest token box holds a half tile");
 
 struct alignas(64) UmParams {
   CUtensorMap b_map[4];  // B rows: fp16 [rows, n_in], boxes {64, 16 / 64 / 128 / 192 rows}, 128B swizzle
@@ -283,9 +282,9 @@ struct UmCursor {
 
 // MMA width of a tile (tokens rounded up to 32: N/2 rows per CTA, 16-row multiples)
 MOE_DEV int um_np(int tokens) { return tokens <= 32 ? 32 : (tokens + 31) & ~31; }
-// token box of a CTA's half: 0..3 = 16, 32, 64, kUmBHalf rows
+// token box of a CTA's half: 0..3 = 16, 32, 64, 96 rows
 MOE_DEV int um_box(int half) { return half <= 16 ? 0 : half <= 32 ? 1 : half <= 64 ? 2 : 3; }
-MOE_DEV int um_box_rows(int h) { return h == 0 ? 16 : h == 1 ? 32 : h == 2 ? 64 : kUmBHalf; }
+MOE_DEV int um_box_rows(int h) { return h == 0 ? 16 : h == 1 ? 32 : h == 2 ? 64 : 96; }
 
 // ------------------------------------------------------------ the kernel
 // Launched in clusters of two CTAs (gridDim.x even).

@@ -622,8 +622,8 @@ moe_status_t launch_ffn_tc(const moe_dims_t& d, const void* x, const int* offset
     if (um_pairs > 0 && um_ok(a0, stage) && um_ok(a1, stage)) {
       UmParams q{};
       moe_status_t st = MOE_OK;
-      for (int h = 0; h < 4 && st == MOE_OK; ++h) {  // half-tile token boxes of 16, 32, 64, kUmBHalf rows
-        const uint32_t box_rows = h == 0 ? 16u : h == 1 ? 32u : h == 2 ? 64u : (uint32_t)kUmBHalf;
+      for (int h = 0; h < 4 && st == MOE_OK; ++h) {  // half-tile token boxes of 16, 32, 64, 96 rows
+        const uint32_t box_rows = h == 0 ? 16u : h == 1 ? 32u : h == 2 ? 64u : 96u;
         if (stage == 1)
           st = tmap_2d(&q.b_map[h], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, xs, d.d_model, (uint64_t)P,
                        (uint64_t)d.d_model * 2, kUmKB, box_rows, true);
