@@ -17,6 +17,8 @@
 //       (warp scans over 32-expert chunks, one chunk per warp; the shared
 //       expert's tokens form their own groups),
 //       the stable (token, slot) order within each expert (warp match);
+//       for one token (learned routing) the top-k warp orders its k experts
+//       itself, with no counting pass;
 //   S1  units (group, 64 rows of d_ff): h = silu(W1 x) * (W3 x) for the
 //       group's tokens, written as the planes W2 reads; a per-group counter
 //       counts finished units;
@@ -997,103 +999,136 @@ __global__ void __launch_bounds__(kDecThreads, 1) ffn_decode_kernel(const __grid
     __syncthreads();
     if (tid < Tk) r_w[tid] = sj;
   }
-  __syncthreads();
-  // per-expert counts (out-of-range ids are reported and counted as expert 0)
-  {
-    bool bad = false;
-    for (int i = tid; i < Tk; i += kDecThreads) {
-      int e = r_ids[i];
-      if (e < 0 || e >= E) {
-        bad = true;
-        e = 0;
-      }
-      atomicAdd(r_off + e, 1);
-    }
-    if (bad) set_error(p.err, kErrDeviceInput);
-  }
-  __syncthreads();
-  {
-    // offsets (exclusive scan of the counts), cursors and groups, one chunk of
-    // 32 experts per warp at a time (lane l takes expert 32c + l:
-    // conflict-free shared accesses): the first pass scans within each chunk
-    // and records the chunk's totals, the second adds the totals of the
-    // chunks before it.  Groups in ascending expert order after the shared
-    // ones.
-    const int gsz = p.ntmax;
-    const int nsg = p.has_shared && p.with_shared ? (T + gsz - 1) / gsz : 0;
-    const int nchk = (E + 31) >> 5;  // <= 32
-    int* tot = reinterpret_cast<int*>(red);  // [chunk]: pairs, groups (red is free until the units)
-    // groups of expert e's n pairs: ceil(n / gsz) for gsz in 1..4 without a
-    // runtime division; none for an expert outside [e_begin, e_end)
-    auto ngroups = [&](int e, int n) {
-      if (e >= E || e < p.e_begin || e >= p.e_end) return 0;
-      return gsz == 1 ? n : gsz == 2 ? (n + 1) >> 1 : gsz == 3 ? (n + 2) / 3 : (n + 3) >> 2;
-    };
-    for (int c = warp; c < nchk; c += kDecWarps) {
-      const int e = 32 * c + lane;
-      const int n = e < E ? r_off[e] : 0, ng = ngroups(e, n);
-      int sc = n, sg = ng;  // inclusive warp scans
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int a = __shfl_up_sync(0xffffffffu, sc, o), b = __shfl_up_sync(0xffffffffu, sg, o);
-        if (lane >= o) {
-          sc += a;
-          sg += b;
+  if (!p.hash && T == 1) {
+    // one token: its k experts (distinct, in range: the top-k chose them)
+    // are one pair and one group each, so warp 0, which chose them, orders
+    // them itself: pair j's position is the number of its experts with a
+    // smaller id, and its group follows the shared group and the owned
+    // experts with smaller ids (what the counting path below yields)
+    if (warp == 0) {
+      __syncwarp();
+      const int e = lane < k ? r_ids[lane] : 0x7fffffff;
+      const bool own = lane < k && e >= p.e_begin && e < p.e_end;
+      int pos = 0, gpre = 0;
+      for (int i = 0; i < k; ++i) {
+        const int ei = __shfl_sync(0xffffffffu, e, i);
+        if (ei < e) {
+          ++pos;
+          gpre += ei >= p.e_begin && ei < p.e_end;
         }
       }
-      if (e < E) r_cur[e] = (sc - n) | ((sg - ng) << 16);  // exclusive within the chunk (each < 2^16)
-      if (lane == 31) {
-        tot[2 * c] = sc;
-        tot[2 * c + 1] = sg;
+      const int nsg = p.has_shared && p.with_shared ? 1 : 0;
+      if (lane < k) {
+        r_sorted[pos] = lane;
+        r_inv[lane] = pos;
+      }
+      if (own) r_groups[nsg + gpre] = make_int4(e, pos, 1, 0);
+      const int nown = __popc(__ballot_sync(0xffffffffu, own));
+      if (lane == 0) {
+        misc[1] = nsg;
+        misc[2] = nown;
+        if (nsg) r_groups[0] = make_int4(-1, 0, 1, 0);
       }
     }
+  } else {
     __syncthreads();
-    for (int c = warp; c < nchk; c += kDecWarps) {
-      const int pc = __reduce_add_sync(0xffffffffu, lane < c ? tot[2 * lane] : 0);
-      const int pg = __reduce_add_sync(0xffffffffu, lane < c ? tot[2 * lane + 1] : 0);
-      const int e = 32 * c + lane;
-      if (e < E) {
-        const int n = r_off[e], w = r_cur[e];
-        const int off = pc + (w & 0xffff);
-        r_off[e] = off;
-        r_cur[e] = off;
-        if (ngroups(e, n) > 0)
-          for (int q0 = 0, gi = nsg + pg + (w >> 16); q0 < n; q0 += gsz) r_groups[gi++] = make_int4(e, off + q0, min(gsz, n - q0), 0);
+    // per-expert counts (out-of-range ids are reported and counted as expert 0)
+    {
+      bool bad = false;
+      for (int i = tid; i < Tk; i += kDecThreads) {
+        int e = r_ids[i];
+        if (e < 0 || e >= E) {
+          bad = true;
+          e = 0;
+        }
+        atomicAdd(r_off + e, 1);
       }
+      if (bad) set_error(p.err, kErrDeviceInput);
+    }
+    __syncthreads();
+    {
+      // offsets (exclusive scan of the counts), cursors and groups, one chunk of
+      // 32 experts per warp at a time (lane l takes expert 32c + l:
+      // conflict-free shared accesses): the first pass scans within each chunk
+      // and records the chunk's totals, the second adds the totals of the
+      // chunks before it.  Groups in ascending expert order after the shared
+      // ones.
+      const int gsz = p.ntmax;
+      const int nsg = p.has_shared && p.with_shared ? (T + gsz - 1) / gsz : 0;
+      const int nchk = (E + 31) >> 5;  // <= 32
+      int* tot = reinterpret_cast<int*>(red);  // [chunk]: pairs, groups (red is free until the units)
+      // groups of expert e's n pairs: ceil(n / gsz) for gsz in 1..4 without a
+      // runtime division; none for an expert outside [e_begin, e_end)
+      auto ngroups = [&](int e, int n) {
+        if (e >= E || e < p.e_begin || e >= p.e_end) return 0;
+        return gsz == 1 ? n : gsz == 2 ? (n + 1) >> 1 : gsz == 3 ? (n + 2) / 3 : (n + 3) >> 2;
+      };
+      for (int c = warp; c < nchk; c += kDecWarps) {
+        const int e = 32 * c + lane;
+        const int n = e < E ? r_off[e] : 0, ng = ngroups(e, n);
+        int sc = n, sg = ng;  // inclusive warp scans
+  #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int a = __shfl_up_sync(0xffffffffu, sc, o), b = __shfl_up_sync(0xffffffffu, sg, o);
+          if (lane >= o) {
+            sc += a;
+            sg += b;
+          }
+        }
+        if (e < E) r_cur[e] = (sc - n) | ((sg - ng) << 16);  // exclusive within the chunk (each < 2^16)
+        if (lane == 31) {
+          tot[2 * c] = sc;
+          tot[2 * c + 1] = sg;
+        }
+      }
+      __syncthreads();
+      for (int c = warp; c < nchk; c += kDecWarps) {
+        const int pc = __reduce_add_sync(0xffffffffu, lane < c ? tot[2 * lane] : 0);
+        const int pg = __reduce_add_sync(0xffffffffu, lane < c ? tot[2 * lane + 1] : 0);
+        const int e = 32 * c + lane;
+        if (e < E) {
+          const int n = r_off[e], w = r_cur[e];
+          const int off = pc + (w & 0xffff);
+          r_off[e] = off;
+          r_cur[e] = off;
+          if (ngroups(e, n) > 0)
+            for (int q0 = 0, gi = nsg + pg + (w >> 16); q0 < n; q0 += gsz) r_groups[gi++] = make_int4(e, off + q0, min(gsz, n - q0), 0);
+        }
+      }
+      if (warp == 0) {
+        const int run = __reduce_add_sync(0xffffffffu, lane < nchk ? tot[2 * lane] : 0);
+        const int ngr = __reduce_add_sync(0xffffffffu, lane < nchk ? tot[2 * lane + 1] : 0);
+        if (lane == 0) {
+          r_off[E] = run;
+          misc[1] = nsg;
+          misc[2] = ngr;
+        }
+        if (lane < nsg) r_groups[lane] = make_int4(-1, lane * gsz, min(gsz, T - lane * gsz), 0);
+      }
+      __syncthreads();
     }
     if (warp == 0) {
-      const int run = __reduce_add_sync(0xffffffffu, lane < nchk ? tot[2 * lane] : 0);
-      const int ngr = __reduce_add_sync(0xffffffffu, lane < nchk ? tot[2 * lane + 1] : 0);
-      if (lane == 0) {
-        r_off[E] = run;
-        misc[1] = nsg;
-        misc[2] = ngr;
+      // stable order within each expert: pairs in ascending flat index
+      const unsigned lt = (1u << lane) - 1u;
+      for (int c0 = 0; c0 < Tk; c0 += 32) {
+        const int i = c0 + lane;
+        int e = -1;
+        if (i < Tk) {
+          e = r_ids[i];
+          if (e < 0 || e >= E) e = 0;
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        int base = 0;
+        if (i < Tk) {
+          base = r_cur[e];
+          const int pos = base + __popc(peers & lt);
+          r_sorted[pos] = i;
+          r_inv[i] = pos;
+        }
+        __syncwarp();
+        if (i < Tk && (peers >> lane) == 1u) r_cur[e] = base + __popc(peers);  // highest lane of its expert
+        __syncwarp();
       }
-      if (lane < nsg) r_groups[lane] = make_int4(-1, lane * gsz, min(gsz, T - lane * gsz), 0);
-    }
-    __syncthreads();
-  }
-  if (warp == 0) {
-    // stable order within each expert: pairs in ascending flat index
-    const unsigned lt = (1u << lane) - 1u;
-    for (int c0 = 0; c0 < Tk; c0 += 32) {
-      const int i = c0 + lane;
-      int e = -1;
-      if (i < Tk) {
-        e = r_ids[i];
-        if (e < 0 || e >= E) e = 0;
-      }
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      int base = 0;
-      if (i < Tk) {
-        base = r_cur[e];
-        const int pos = base + __popc(peers & lt);
-        r_sorted[pos] = i;
-        r_inv[i] = pos;
-      }
-      __syncwarp();
-      if (i < Tk && (peers >> lane) == 1u) r_cur[e] = base + __popc(peers);  // highest lane of its expert
-      __syncwarp();
     }
   }
   if (blockIdx.x == 0) {
