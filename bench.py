@@ -197,6 +197,14 @@ def kernel_work(inp, ids, tensor_path=False):
     return work, flops, n_act, (n_act * (b13 + b2) + sh13 + sh2), kflops
 
 
+def layer_copies(requested, step_weight_bytes, l2_bytes):
+    """Copies of the layer cycled between timed steps: the requested number,
+    or (0) four when a step reads under 8x L2 of weights, else one (flushed)."""
+    if requested > 0:
+        return requested
+    return 4 if step_weight_bytes < 8 * l2_bytes else 1
+
+
 def layer_tensors(inp):
     """Every device tensor of one layer's inputs (for its size)."""
     ts = [inp.x, inp.router_w, inp.router_b, inp.token_ids, inp.tid2eid]
@@ -459,7 +467,7 @@ def run_config(name, args, dev, world, rank):
     torch.cuda.synchronize()
     step_weight_bytes = kernel_work(inp, ids.cpu().numpy(), False)[3]
     l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
-    n_layers = args.layers if args.layers > 0 else (4 if step_weight_bytes < 8 * l2_bytes else 1)
+    n_layers = layer_copies(args.layers, step_weight_bytes, l2_bytes)
     layers = [inp] + [inp.clone() for _ in range(n_layers - 1)]
     # L2 flush by a read of 512 MiB (> 4x L2) into one small result
     flush = torch.ones(128 * 1024 * 1024, dtype=torch.int32, device=dev)

@@ -198,3 +198,23 @@ def test_roofline_tensor_bound_uses_the_burst_peak():
     assert r["peak"] == 1624.7
     assert r["frac"] == pytest.approx(flops / 1.444e-3 / 1e12 / 1624.7)
     assert r["frac"] < 0.5 < r["frac_of_sustained_peak"]
+
+
+def test_layer_copies_cycle_only_small_steps():
+    l2 = 126 * 1024 * 1024
+    # decode reads ~140 MB of weights per step: copies are cycled
+    assert bench.layer_copies(0, 140_000_000, l2) == 4
+    # a prefill step reads GBs: one copy, flushed between steps
+    assert bench.layer_copies(0, 3_600_000_000, l2) == 1
+    assert bench.layer_copies(0, 8 * l2, l2) == 1
+    # an explicit request wins either way
+    assert bench.layer_copies(1, 140_000_000, l2) == 1
+    assert bench.layer_copies(6, 3_600_000_000, l2) == 6
+
+
+def test_layer_copies_share_values_not_buffers():
+    from synthetic import make_inputs
+    inp = make_inputs("tiny", "cpu")
+    cp = inp.clone()
+    for a, b in zip(bench.layer_tensors(inp), bench.layer_tensors(cp)):
+        assert torch.equal(a, b) and a.data_ptr() != b.data_ptr()
